@@ -1,0 +1,121 @@
+"""Seeded synthetic inputs for the quantised linear layer.
+
+This module only draws random tensors with the shapes and distributions of the
+workloads below; it holds none of the method's arithmetic. Both the test suite's
+CPU oracle and the CUDA path take their inputs from here.
+
+Conventions:
+* ``N(0, s)`` names the standard deviation s.
+* Every tensor has its own stream, seeded ``seed * 1000 + index`` in the order
+  W, outlier positions/signs, X, A, B, dY.
+* Values are drawn in fp32 and rounded to bf16 (nearest-even); the bf16 bit
+  patterns are what both sides consume.
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+import torch
+
+W_IDX, OUTLIER_IDX, X_IDX, A_IDX, B_IDX, DY_IDX = range(6)
+
+
+def _rng(seed: int, idx: int) -> np.random.Generator:
+    return np.random.default_rng(seed * 1000 + idx)
+
+
+def to_bf16(x: np.ndarray) -> torch.Tensor:
+    """fp32 numpy -> bf16 torch CPU tensor (round to nearest even)."""
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16)
+
+
+def normal_bf16(shape, std: float, seed: int, idx: int) -> torch.Tensor:
+    x = _rng(seed, idx).standard_normal(size=shape, dtype=np.float32) * np.float32(std)
+    return to_bf16(x)
+
+
+def weight_with_outliers(N: int, K: int, std: float, frac: float, mult: float,
+                         seed: int) -> torch.Tensor:
+    """W ~ N(0, std) with round(frac * N * K) positions, drawn without replacement,
+    set to +-mult*std (random sign)."""
+    w = _rng(seed, W_IDX).standard_normal(size=(N, K), dtype=np.float32) * np.float32(std)
+    n_out = int(round(frac * N * K))
+    if n_out:
+        g = _rng(seed, OUTLIER_IDX)
+        pos = g.choice(N * K, size=n_out, replace=False)
+        sign = np.where(g.integers(0, 2, size=n_out) == 1, 1.0, -1.0).astype(np.float32)
+        w.reshape(-1)[pos] = sign * np.float32(mult * std)
+    return to_bf16(w)
+
+
+@dataclasses.dataclass(frozen=True)
+class LinearCase:
+    """One quantised linear: weight [N, K], tokens M, rank r, alpha, format."""
+    name: str
+    N: int
+    K: int
+    M: int
+    r: int
+    alpha: float
+    fmt: str = "nf4_dq"          # "nf4_dq" or "int8"
+    w_std: float = 0.02
+    outlier_frac: float = 0.0
+    outlier_mult: float = 20.0
+    a_std: float | None = None   # None -> 1/K
+    b_std: float = 0.01
+    backward: bool = True
+    seed: int = 0
+
+    @property
+    def s(self) -> float:
+        return self.alpha / self.r
+
+
+def make_inputs(case: LinearCase) -> dict:
+    """All bf16 CPU tensors of one case: W, X, A, B and (if backward) dY."""
+    seed = case.seed
+    W = weight_with_outliers(case.N, case.K, case.w_std, case.outlier_frac,
+                             case.outlier_mult, seed)
+    X = normal_bf16((case.M, case.K), 1.0, seed, X_IDX)
+    a_std = case.a_std if case.a_std is not None else 1.0 / case.K
+    A = normal_bf16((case.r, case.K), a_std, seed, A_IDX)
+    B = normal_bf16((case.N, case.r), case.b_std, seed, B_IDX)
+    out = {"W": W, "X": X, "A": A, "B": B}
+    if case.backward:
+        out["dY"] = normal_bf16((case.M, case.N), 1.0, seed, DY_IDX)
+    return out
+
+
+def device_normal_bf16(shape, std: float, seed: int, idx: int,
+                       device="cuda") -> torch.Tensor:
+    """Large tensors drawn on the device with torch's Philox generator (for the
+    multi-layer stacks, whose bf16 sources are too big to draw on the host)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed * 1000 + idx)
+    x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    return (x * std).to(torch.bfloat16)
+
+
+# The five workloads: a single small linear, a decode-shaped 7B linear, a
+# fine-tune-shaped MLP up-projection, a 32-layer 7B-shaped stack and 80 layers of
+# 65B-shaped linears with a per-layer (format, rank) mix.
+CFG1 = LinearCase("single-256", N=256, K=256, M=64, r=8, alpha=16.0, a_std=1.0 / 256)
+CFG2 = [LinearCase(f"decode-7b-M{m}", N=4096, K=4096, M=m, r=16, alpha=32.0,
+                   outlier_frac=0.001, outlier_mult=20.0, backward=False)
+        for m in (1, 4, 16)]
+CFG3 = LinearCase("upproj-11008x4096-M8192", N=11008, K=4096, M=8192, r=64, alpha=16.0)
+
+STACK_7B = [("q", 4096, 4096), ("k", 4096, 4096), ("v", 4096, 4096), ("o", 4096, 4096),
+            ("gate", 11008, 4096), ("up", 11008, 4096), ("down", 4096, 11008)]
+STACK_65B = [("q", 8192, 8192), ("k", 8192, 8192), ("v", 8192, 8192), ("o", 8192, 8192),
+             ("gate", 22016, 8192), ("up", 22016, 8192), ("down", 8192, 22016)]
+
+
+def layer_mix_65b(n_layers: int = 80, seed: int = 0):
+    """Per decoder layer: (format, rank) drawn uniformly from {nf4_dq, int8} x
+    {8, 16, 32, 64} by a seed-0 generator, shared by the layer's 7 linears."""
+    g = np.random.default_rng(seed * 1000 + 900)
+    fmts = g.integers(0, 2, size=n_layers)
+    ranks = g.integers(0, 4, size=n_layers)
+    return [("nf4_dq" if f == 0 else "int8", (8, 16, 32, 64)[r]) for f, r in zip(fmts, ranks)]

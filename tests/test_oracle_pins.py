@@ -1,0 +1,382 @@
+"""Pins for the CPU oracle: each test fixes part of it against something other than
+itself (a closed form, an independent high-precision evaluation, exact rational
+brute force, finite differences, or a figure printed on the QLoRA page)."""
+import json
+import math
+import os
+from fractions import Fraction
+
+import mpmath
+import numpy as np
+import pytest
+import torch
+
+import oracle.qlora_oracle as o
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def bf16_f32(x):
+    return torch.tensor(np.asarray(x, np.float32)).to(torch.bfloat16).float().numpy()
+
+
+# ---------------------------------------------------------------- P1 codebook
+
+def _mp_rn32(x: mpmath.mpf):
+    """Round an mpmath real to the nearest fp32 directly (no fp64 step); also
+    return the distance from the nearest rounding boundary in ulps."""
+    if x == 0:
+        return np.float32(0), 0.5
+    e = int(mpmath.floor(mpmath.log(abs(x), 2)))
+    scaled = abs(x) * mpmath.mpf(2) ** (23 - e)
+    n = int(mpmath.nint(scaled))
+    margin = 0.5 - abs(float(scaled - mpmath.floor(scaled)) - 0.5)
+    val = math.copysign(n * 2.0 ** (e - 23), float(x))
+    return np.float32(val), margin
+
+
+def test_codebook_matches_50_digit_evaluation():
+    mpmath.mp.dps = 50
+    q = o.nf4_codebook()
+    scale = mpmath.sqrt(2) * mpmath.erfinv(2 * mpmath.mpf(31) / 32 - 1)
+    for i in range(16):
+        p = (mpmath.mpf(i) + mpmath.mpf(1) / 2) / 16
+        exact = mpmath.sqrt(2) * mpmath.erfinv(2 * p - 1) / scale
+        ref, margin = _mp_rn32(exact)
+        assert ref.view(np.uint32) == q[i].view(np.uint32), (i, ref, q[i])
+        # far from a rounding boundary, so RN32 of the fp64 quantile is unambiguous
+        assert margin > 0.02 or i in (0, 15)
+
+
+def test_codebook_shape_symmetry_endpoints():
+    q = o.nf4_codebook()
+    assert q.dtype == np.float32 and q.size == 16
+    assert q[0] == -1.0 and q[15] == 1.0
+    assert np.all(np.diff(q) > 0)
+    assert np.array_equal(q[::-1], -q)           # exact antisymmetry
+    assert not np.any(q == 0)                    # the centred grid has no zero point
+
+
+def test_codebook_equal_mass():
+    """Phi(q_i * Q(31/32)) = (i + 1/2)/16: every point is the centre of an equal-mass
+    bin of N(0, 1) (checked with math.erfc, independent of the quantile routine)."""
+    q = o.nf4_codebook().astype(np.float64)
+    c = o.normal_quantile(31 / 32)
+    for i in range(16):
+        z = q[i] * c
+        phi = 0.5 * math.erfc(-z / math.sqrt(2))
+        assert abs(phi - (i + 0.5) / 16) < 2e-7, i
+
+
+def test_page_grid_size():
+    g = json.load(open(os.path.join(GOLDEN, "qlora_page_figures.json")))
+    assert o.nf4_codebook().size == g["grid_points"]["value"] == 2 ** g["grid_bits"]["value"]
+    assert o.BLOCK == g["block_size"]["value"]
+
+
+# ---------------------------------------------------------------- P2 midpoints
+
+def test_midpoints():
+    q = o.nf4_codebook().astype(np.float64)
+    m = o.nf4_midpoints()
+    assert m.size == 15 and m[7] == 0.0
+    assert np.all(np.diff(m) > 0)
+    assert np.all((q[:-1] < m) & (m < q[1:]))
+    assert np.array_equal(2.0 * m - q[:-1], q[1:])     # exact midpoints
+    assert np.array_equal(m[::-1], -m)
+
+
+def test_midpoints_have_many_significant_bits():
+    """a * m_j is never a bf16 value for a bf16 a (so no exact ties except at 0):
+    the odd part of every nonzero m_j has more than 8 bits."""
+    for j, v in enumerate(o.nf4_midpoints()):
+        if v == 0:
+            continue
+        num = Fraction(float(v)).numerator
+        while num % 2 == 0:
+            num //= 2
+        assert abs(num).bit_length() > 8, j
+
+
+# ---------------------------------------------------------------- P3 encoder brute force
+
+def _brute_code(x: float, a: float, qf):
+    if a == 0:
+        return 8
+    r = Fraction(x) / Fraction(a)
+    d = [abs(r - qi) for qi in qf]
+    best = min(d)
+    return max(i for i in range(16) if d[i] == best)     # ties go to the upper point
+
+
+def _all_bf16_upto(a: float):
+    bits = np.arange(0, 0x7F80, dtype=np.uint32)          # +0 .. largest finite
+    vals = (bits << 16).view(np.float32)
+    vals = vals[vals <= a]
+    return np.concatenate([vals, -vals])
+
+
+@pytest.mark.parametrize("a_bits", [0x3F80, 0x3CE0, 0x7F7F, 0x0080, 0x0003, 0x4123])
+def test_encoder_matches_exact_rational_nearest(a_bits):
+    """Every bf16 x with |x| <= a (or a 3000-sample of them), including +-0 and
+    subnormals, against the exact-rational nearest grid point with ties upward."""
+    a = float(np.array([a_bits << 16], np.uint32).view(np.float32)[0])
+    xs = _all_bf16_upto(a)
+    rng = np.random.default_rng(a_bits)
+    if xs.size > 3000:
+        keep = rng.choice(xs.size, 3000, replace=False)
+        xs = np.concatenate([xs[keep], np.float32([0.0, -0.0, a, -a])])
+    qf = [Fraction(float(v)) for v in o.nf4_codebook()]
+    nb = (xs.size + 63) // 64
+    codes = o.nf4_encode(xs, np.full(nb, a, np.float32))
+    for x, c in zip(xs.tolist(), codes.tolist()):
+        assert c == _brute_code(x, a, qf), (x, a, c)
+
+
+def test_encoder_zero_block_and_signed_zero():
+    codes = o.nf4_encode(np.float32([0.0, -0.0] * 32), np.float32([0.0]))
+    assert np.all(codes == 8)
+    codes = o.nf4_encode(np.float32([0.0, -0.0, 1.0, -1.0] + [0.5] * 60), np.float32([1.0]))
+    assert codes[:4].tolist() == [8, 8, 15, 0]
+
+
+def test_block_absmax_partial_last_block():
+    w = bf16_f32(np.random.default_rng(1).standard_normal(64 * 3 + 5))
+    a = o.block_absmax(w)
+    assert a.size == 4
+    for b in range(4):
+        assert a[b] == np.max(np.abs(w[b * 64:(b + 1) * 64]))
+
+
+# ---------------------------------------------------------------- P4 exact codebook dequant
+
+@pytest.mark.parametrize("e", [-20, -3, 0, 7, 100])
+def test_codebook_points_roundtrip_exactly(e):
+    """A block built from RNbf(q_c * 2^e) with one entry 2^e (so a = 2^e) encodes
+    back to c and, without double quantisation, dequantises to itself bit-exactly."""
+    rng = np.random.default_rng(e + 50)
+    c = rng.integers(0, 16, size=64).astype(np.uint8)
+    c[5] = 15
+    q = o.nf4_codebook()
+    w = bf16_f32(q[c] * np.float32(2.0 ** e))
+    packed, a = o.nf4_quantize(w)
+    assert a[0] == np.float32(2.0 ** e)
+    assert np.array_equal(o.unpack_nibbles(packed, 64), c)
+    wd = o.nf4_dequant(packed, a, 64)
+    assert np.array_equal(wd.view(np.uint32), w.view(np.uint32))
+
+
+def test_pack_order():
+    c = np.arange(16, dtype=np.uint8)
+    p = o.pack_nibbles(c)
+    assert p[0] == 0x10 and p[1] == 0x32 and p[7] == 0xFE
+    assert np.array_equal(o.unpack_nibbles(o.pack_nibbles(c[:5]), 5), c[:5])
+    assert o.pack_nibbles(c[:5])[2] == 0x04                   # odd count: high nibble 0
+
+
+# ---------------------------------------------------------------- P5 idempotence
+
+def test_requantise_idempotent_without_dq():
+    w = bf16_f32(np.random.default_rng(7).standard_normal(64 * 512) * 0.02)
+    packed, a = o.nf4_quantize(w)
+    wd = o.nf4_dequant(packed, a, w.size)
+    packed2, a2 = o.nf4_quantize(wd)
+    assert np.array_equal(packed2, packed)
+    assert np.array_equal(a2, a)
+    wd2 = o.nf4_dequant(packed2, a2, w.size)
+    assert np.array_equal(wd2.view(np.uint32), wd.view(np.uint32))
+
+
+def test_requantise_codes_stable_with_dq():
+    w = bf16_f32(np.random.default_rng(8).standard_normal(64 * 1024) * 0.02)
+    r = o.quantize_weight(w, "nf4_dq")
+    r2 = o.quantize_weight(r["wdeq"], "nf4_dq")
+    assert np.array_equal(r2["codes"], r["codes"])
+    # the re-derived constants differ by at most half a DQ step, so W'' differs from
+    # W' by at most that (|q| <= 1) plus one bf16 rounding on each side
+    g = (np.arange(w.size) // 64) // 256
+    d = np.abs(r2["wdeq"].astype(np.float64) - r["wdeq"])
+    bound = r2["group_scale"][g] * 0.5 + np.abs(r["wdeq"]) * 2.0 ** -7 + 1e-30
+    assert np.all(d <= bound)
+
+
+# ---------------------------------------------------------------- P6 accounting
+
+def test_bits_per_param_accounting():
+    g = json.load(open(os.path.join(GOLDEN, "qlora_page_figures.json")))
+    for n in (16384, 4096 * 4096, 11008 * 4096):
+        sb = o.storage_bytes("nf4_dq", n)
+        assert sb["codes"] * 2 == n                         # ~N/2 bytes of NF4 weights
+        per_group = (sb["codes"] + sb["qabsmax"] + sb["group_scale"]) * 8 / n
+        assert per_group == 4.126953125                     # 4 + 8/64 + 32/(64*256)
+        total = sum(sb.values()) * 8 / n
+        assert total == 4.126953125 + 32 / n                # plus one fp32 mean
+        const_bits = per_group - 4
+        assert abs(const_bits - g["const_bits_after_dq"]["value"]) <= g["const_bits_after_dq"]["tol"]
+        # the page's 0.37 saving holds against 32-bit constants (32/64 - 0.127)
+        assert abs((32 / 64 - const_bits) - g["saving_bits"]["value"]) <= g["saving_bits"]["tol"]
+        assert 16 / g["block_size"]["value"] == g["const_bits_16bit"]["value"]
+        assert sb["codes"] / n == g["nf4_weight_bytes_per_param"]["value"]
+        sb8 = o.storage_bytes("int8", n)
+        assert sum(sb8.values()) * 8 / n == 8.5
+    # 65B parameters in fp16: the page's ~130 GB
+    assert abs(65e9 * 2 / 1e9 - g["fp16_65b_full_gb"]["value"]) <= g["fp16_65b_full_gb"]["tol"]
+
+
+# ---------------------------------------------------------------- P7 double quantisation
+
+def test_dq_worked_example():
+    """absmax [1, 3]: mu = 2, d = [-1, 1], s = RN32(1/127), codes -127/+127, and the
+    reconstruction is exact (worked by hand: RN32(127 * RN32(1/127)) = 1)."""
+    qa, sc, mu = o.dq_encode(np.float32([1.0, 3.0]))
+    assert mu == 2.0
+    assert sc.tolist() == [float(np.float32(1.0) / np.float32(127))]
+    assert qa.tolist() == [-127, 127]
+    assert o.dq_decode(qa, sc, mu).tolist() == [1.0, 3.0]
+
+
+def test_dq_constant_tensor_is_exact():
+    a = np.full(1000, 0.046875, np.float32)
+    qa, sc, mu = o.dq_encode(a)
+    assert mu == np.float32(0.046875) and np.all(sc == 0) and np.all(qa == 0)
+    assert np.array_equal(o.dq_decode(qa, sc, mu), a)
+
+
+def test_dq_roundtrip_bound_and_mean():
+    w = bf16_f32(np.random.default_rng(3).standard_normal(64 * 256 * 9 + 64 * 17) * 0.02)
+    a = o.block_absmax(w)
+    qa, sc, mu = o.dq_encode(a)
+    assert sc.size == (a.size + 255) // 256
+    # exact mean, by rational arithmetic
+    exact = sum(Fraction(float(v)) for v in a) / a.size
+    assert mu == np.float32(float(exact))
+    ar = o.dq_decode(qa, sc, mu)
+    g = np.arange(a.size) // 256
+    ulp = np.spacing(np.maximum(np.abs(a), abs(mu)).astype(np.float32))
+    assert np.all(np.abs(ar.astype(np.float64) - a) <= sc[g] * 0.5 + 4 * ulp)
+    assert np.all(np.abs(qa.astype(int)) <= 127) and np.max(np.abs(qa.astype(int))) == 127
+
+
+def test_rint_half_even_in_dq():
+    # d/s = 2.5 exactly -> 2 ; 3.5 -> 4 (round half to even)
+    a = np.float32([0.0, 2.5, 3.5, -127.0 + 0.0]) + np.float32(127.0)
+    qa, sc, mu = o.dq_encode(a)
+    d = a - mu
+    t = d / sc[0]
+    assert np.array_equal(qa, np.clip(np.rint(t), -127, 127).astype(np.int8))
+
+
+# ---------------------------------------------------------------- int8 format
+
+def test_int8_format():
+    w = bf16_f32(np.random.default_rng(4).standard_normal(64 * 300) * 0.02)
+    c, a = o.int8_quantize(w)
+    assert c.dtype == np.int8 and np.max(np.abs(c.astype(int))) == 127
+    sc = a / np.float32(127)
+    wd = o.int8_dequant(c, a)
+    b = np.arange(w.size) // 64
+    assert np.all(np.abs(wd - w) <= sc[b] * 0.5 * (1 + 2 ** -7) + np.abs(w) * 2 ** -8)
+    # the element equal to the absmax maps to +-127 and back to itself
+    i = np.argmax(np.abs(w[:64]))
+    assert abs(int(c[i])) == 127
+    # a zero block stays zero
+    c0, a0 = o.int8_quantize(np.zeros(64, np.float32))
+    assert np.all(c0 == 0) and o.int8_dequant(c0, a0).tolist() == [0.0] * 64
+
+
+# ---------------------------------------------------------------- bf16 rounding
+
+def test_rn_bf16_matches_torch():
+    rng = np.random.default_rng(5)
+    x = np.concatenate([
+        rng.standard_normal(20000).astype(np.float32) * 10.0 ** rng.integers(-40, 38, 20000),
+        np.float32([0.0, -0.0, np.inf, -np.inf, 3.4028235e38, 1e-45, -1e-45]),
+        (np.arange(0, 1 << 16, dtype=np.uint32) << 16 | 0x8000).view(np.float32)[:0x7F80],
+    ]).astype(np.float32)
+    x = x[np.isfinite(x) | np.isinf(x)]
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(o.f32_to_bf16_bits(x), ref)
+    assert np.isnan(o.rn_bf16(np.float32([np.nan]))[0])
+
+
+# ---------------------------------------------------------------- P8-P11 linear layer
+
+def _naive_fwd(X, W, A, B, s):
+    M, K = X.shape
+    N, r = B.shape
+    Y = np.zeros((M, N))
+    T = np.zeros((M, r))
+    for m in range(M):
+        for j in range(r):
+            T[m, j] = sum(X[m, k] * A[j, k] for k in range(K))
+        for n in range(N):
+            Y[m, n] = sum(X[m, k] * W[n, k] for k in range(K)) \
+                + s * sum(T[m, j] * B[n, j] for j in range(r))
+    return Y, T
+
+
+def _tiny(seed=11, M=3, N=5, K=64, r=2):
+    g = np.random.default_rng(seed)
+    return (g.standard_normal((M, K)), g.standard_normal((N, K)),
+            g.standard_normal((r, K)), g.standard_normal((N, r)), g.standard_normal((M, N)))
+
+
+def test_forward_against_naive_loops():
+    X, W, A, B, _ = _tiny()
+    Y, T = o.linear_fwd(X, W, A, B, alpha=6.0, r=2)
+    Yn, Tn = _naive_fwd(X, W, A, B, 3.0)
+    assert np.allclose(Y, Yn, rtol=1e-12, atol=1e-12)
+    assert np.allclose(T, Tn, rtol=1e-12, atol=1e-12)
+
+
+def test_backward_against_finite_differences():
+    """L = sum(Y * G); Y is linear in X, in A (B fixed) and in B (A fixed), so
+    central differences are exact up to rounding."""
+    X, W, A, B, G = _tiny()
+    alpha, r = 6.0, 2
+    dX, dA, dB = o.linear_bwd(X, G, W, A, B, alpha, r)
+
+    def L(X_, A_, B_):
+        return float(np.sum(o.linear_fwd(X_, W, A_, B_, alpha, r)[0] * G))
+
+    h = 1e-3
+    for (arr, grad, which) in ((X, dX, 0), (A, dA, 1), (B, dB, 2)):
+        fd = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            p = arr.copy(); p[idx] += h
+            m = arr.copy(); m[idx] -= h
+            args_p = [X, A, B]; args_p[which] = p
+            args_m = [X, A, B]; args_m[which] = m
+            fd[idx] = (L(*args_p) - L(*args_m)) / (2 * h)
+        assert np.allclose(grad, fd, rtol=1e-7, atol=1e-7), which
+
+
+def test_special_cases_B0_A0_W0():
+    X, W, A, B, G = _tiny(seed=12)
+    base = X @ W.T
+    Y, _ = o.linear_fwd(X, W, A, np.zeros_like(B), 4.0, 2)
+    assert np.array_equal(Y, base)
+    dX, dA, dB = o.linear_bwd(X, G, W, A, np.zeros_like(B), 4.0, 2)
+    assert np.all(dA == 0)
+    Y, T = o.linear_fwd(X, W, np.zeros_like(A), B, 4.0, 2)
+    assert np.array_equal(Y, base) and np.all(T == 0)
+    dX, dA, dB = o.linear_bwd(X, G, W, np.zeros_like(A), B, 4.0, 2)
+    assert np.all(dB == 0)
+    # W = 0: every block has absmax 0, codes are 8 and W' = +0, so Y is the branch alone
+    r = o.quantize_weight(np.zeros(5 * 64, np.float32), "nf4_dq")
+    assert np.all(o.unpack_nibbles(r["codes"], 320) == 8)
+    assert np.all(r["wdeq"].view(np.uint32) == 0)
+    Y, T = o.linear_fwd(X, r["wdeq"].reshape(5, 64), A, B, 4.0, 2)
+    assert np.allclose(Y, 2.0 * T @ B.T, rtol=0, atol=1e-12)
+
+
+def test_forward_backward_against_torch_autograd():
+    X, W, A, B, G = _tiny(seed=13, M=7, N=9, K=128, r=4)
+    tX, tA, tB = (torch.tensor(v, requires_grad=True) for v in (X, A, B))
+    Y = tX @ torch.tensor(W).T + 0.5 * (tX @ tA.T) @ tB.T
+    (Y * torch.tensor(G)).sum().backward()
+    Yo, _ = o.linear_fwd(X, W, A, B, 2.0, 4)
+    dX, dA, dB = o.linear_bwd(X, G, W, A, B, 2.0, 4)
+    assert np.allclose(Yo, Y.detach().numpy(), rtol=1e-12, atol=1e-12)
+    for a, b in ((dX, tX.grad), (dA, tA.grad), (dB, tB.grad)):
+        assert np.allclose(a, b.numpy(), rtol=1e-12, atol=1e-12)
