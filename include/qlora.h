@@ -1,0 +1,162 @@
+/*
+ * qlora.h — C ABI of the B200 (sm_100a) QLoRA-style quantised linear library.
+ *
+ * The library implements one layer: a frozen weight W [N, K] stored 4-bit (NF4 with
+ * double-quantised constants) or 8-bit (blockwise int8), and an unmerged low-rank
+ * adapter A [r, K], B [N, r], computing
+ *
+ *     Y  = X W'^T + s (X A^T) B^T,             s = alpha / r
+ *     dX = dY W' + s (dY B) A,  dA = s (dY B)^T X,  dB = s dY^T (X A^T)
+ *
+ * where W' is the dequantised weight. The formats follow the QLoRA explainer page
+ * (aizip.shop/methodologies/qlora): section "1. 4-bit NormalFloat (NF4)" for the grid
+ * and section "2. Double Quantization" for blocks of 64 and re-quantised constants;
+ * its "memory decomposition" section for the frozen 4-bit base with bf16 adapters.
+ * The per-layer choice of bit-width and rank is the allocation C = {(q_l, r_l)} of the
+ * AutoQRA page (gist.science/ko/paper/2602.22268), section 3.1.
+ *
+ * Conventions, for every entry point:
+ *  - Pointers named "device" are CUDA device pointers owned by the caller. The library
+ *    never allocates or frees caller-visible memory; scratch comes from the caller's
+ *    workspace (size from ql_workspace_bytes).
+ *  - bf16 tensors are passed as uint16_t bit patterns, row-major, densely packed.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream). All work is
+ *    asynchronous on it; outputs are valid once the stream reaches that point.
+ *  - Arguments are checked before anything is launched; a bad argument returns an
+ *    error status and launches nothing. No exception crosses the ABI.
+ *  - Data-dependent faults found on the device (non-finite inputs, a bounded wait that
+ *    gave up) set a sticky device flag instead of trapping; ql_get_device_status
+ *    reads and clears it.
+ *  - Device pointers must be 16-byte aligned unless stated otherwise.
+ */
+#ifndef QLORA_B200_H
+#define QLORA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t ql_bf16;   /* bf16 bit pattern */
+
+typedef enum {
+  QL_OK = 0,
+  QL_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, negative size, bad enum */
+  QL_ERR_UNSUPPORTED = 2,   /* well-formed but outside what the kernels handle */
+  QL_ERR_WORKSPACE = 3,     /* workspace smaller than ql_workspace_bytes() */
+  QL_ERR_NONFINITE = 4,     /* device flag: an input held inf or NaN */
+  QL_ERR_TIMEOUT = 5,       /* device flag: a bounded wait inside a kernel gave up */
+  QL_ERR_CUDA = 6           /* a CUDA runtime call failed */
+} ql_status;
+
+typedef enum {
+  QL_FMT_NF4_DQ = 0,        /* 4-bit NF4 codes + double-quantised absmax */
+  QL_FMT_INT8_B64 = 1       /* int8 codes + fp32 absmax per block of 64 */
+} ql_format;
+
+/* A quantised weight W [N, K] (row-major flattening, blocks of 64 consecutive
+ * elements, groups of 256 consecutive blocks). All pointers are device pointers.
+ *   NF4_DQ : codes   uint8 [ceil(N*K/2)]   element 2j in the low nibble of byte j
+ *            qabsmax int8  [N*K/64]        double-quantised block absmax
+ *            group_scale fp32 [ceil(N*K/64/256)]
+ *            mean    fp32  [1]             per-tensor mean of the block absmax
+ *            absmax  unused (may be NULL)
+ *   INT8_B64: codes  int8  [N*K]
+ *            absmax  fp32  [N*K/64]
+ *            qabsmax, group_scale, mean unused (may be NULL)                       */
+typedef struct {
+  int32_t fmt;              /* ql_format */
+  int32_t reserved;
+  int64_t N, K;
+  void*   codes;
+  float*  absmax;
+  int8_t* qabsmax;
+  float*  group_scale;
+  float*  mean;
+} ql_weight;
+
+/* NF4 blockwise quantisation (QLoRA page, "1. 4-bit NormalFloat (NF4)").
+ * W: device bf16 [n]. For every block b of 64 consecutive elements (the last block
+ * may be partial): absmax[b] = max |W_j| (fp32, exact), and each element's code is the
+ * index of the grid point q_i = Q_N((i+1/2)/16)/Q_N(31/32) nearest to W_j/absmax[b]
+ * (exact decision, ties to the upper point; an all-zero block gives code 8).
+ * codes: device uint8 [ceil(n/2)], absmax: device fp32 [ceil(n/64)].
+ * W needs 2-byte alignment; codes and absmax 4-byte. n = 0 is a no-op.
+ * Non-finite elements set QL_ERR_NONFINITE on the device flag. */
+ql_status nf4_quantize(const ql_bf16* W, int64_t n, uint8_t* codes, float* absmax,
+                       void* stream);
+
+/* Double quantisation of the block constants (QLoRA page, "2. Double Quantization").
+ * absmax: device fp32 [nblocks], finite and >= 0. mean[0] = fp32(S / nblocks), S the
+ * exact sum of absmax rounded once to fp64. Per group g of 256 blocks:
+ * d = fp32(a - mean), group_scale[g] = fp32(max|d| / 127),
+ * qabsmax[b] = clamp(rint_half_even(fp32(d / group_scale[g])), -127, 127)
+ * (0 when group_scale[g] == 0).
+ * ws: device workspace of at least ql_workspace_bytes(QL_OP_DQ, 0, 0, 0, 0) bytes.
+ * nblocks must be in [1, 2^24]. */
+ql_status dq_quantize(const float* absmax, int64_t nblocks, int8_t* qabsmax,
+                      float* group_scale, float* mean, void* ws, size_t ws_bytes,
+                      void* stream);
+
+/* Blockwise int8 (the 8-bit choice of the per-layer bit-width, AutoQRA page 3.1):
+ * absmax[b] as in nf4_quantize; sc = fp32(absmax[b]/127);
+ * codes[j] = clamp(rint_half_even(fp32(W_j / sc)), -127, 127) (0 when sc == 0).
+ * W: device bf16 [n]; codes: device int8 [n]; absmax: device fp32 [ceil(n/64)]. */
+ql_status int8_quantize(const ql_bf16* W, int64_t n, int8_t* codes, float* absmax,
+                        void* stream);
+
+/* Dequantise a whole weight into bf16 W' [N, K] (device). NF4_DQ:
+ * a' = fp32(fp32(qabsmax*group_scale) + mean), W'_j = bf16(fp32(q[code_j] * a'));
+ * INT8_B64: W'_j = bf16(fp32(code_j * fp32(absmax/127))). Used for checks; the
+ * linear kernels dequantise on the fly and never materialise W'. */
+ql_status ql_dequantize(const ql_weight* w, ql_bf16* Wout, void* stream);
+
+/* Forward of the quantised linear with an unmerged adapter (QLoRA page, "memory
+ * decomposition": frozen 4-bit base + bf16 adapters).
+ *   X [M, K] bf16, A [r, K] bf16, B [N, r] bf16 (device), s = alpha / r.
+ *   T = X A^T (fp32 accumulate); P = bf16(s T);
+ *   Y [M, N] bf16 = bf16(X W'^T + P B^T), fp32 accumulation.
+ *   T_save [M, r] bf16 = bf16(T) if non-NULL (needed by qlora_linear_bwd).
+ * K % 64 == 0, 1 <= r <= 256, M >= 1. ws: ql_workspace_bytes(QL_OP_FWD, M, N, K, r). */
+ql_status qlora_linear_fwd(const ql_weight* w, const ql_bf16* X, int64_t M,
+                           const ql_bf16* A, const ql_bf16* B, int32_t r, float alpha,
+                           ql_bf16* Y, ql_bf16* T_save, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/* Backward with the base frozen: U = dY B (fp32), Q = bf16(s U),
+ *   dX [M, K] bf16 = bf16(dY W' + Q A)          (fp32 accumulation)
+ *   dA [r, K] fp32 = s U^T X,   dB [N, r] fp32 = s dY^T T_saved
+ * X, dY [M, N], T_saved [M, r] from the forward; dA, dB are overwritten.
+ * Same shape limits as the forward. ws: ql_workspace_bytes(QL_OP_BWD, M, N, K, r). */
+ql_status qlora_linear_bwd(const ql_weight* w, const ql_bf16* X, const ql_bf16* dY,
+                           int64_t M, const ql_bf16* A, const ql_bf16* B,
+                           const ql_bf16* T_saved, int32_t r, float alpha,
+                           ql_bf16* dX, float* dA, float* dB, void* ws,
+                           size_t ws_bytes, void* stream);
+
+enum { QL_OP_DQ = 0, QL_OP_FWD = 1, QL_OP_BWD = 2 };
+
+/* Workspace bytes that op (QL_OP_*) needs for these sizes (0 if none). */
+size_t ql_workspace_bytes(int32_t op, int64_t M, int64_t N, int64_t K, int32_t r);
+
+/* Synchronise `stream`, then return and clear the sticky device flag of the current
+ * device (QL_OK, QL_ERR_NONFINITE or QL_ERR_TIMEOUT). */
+ql_status ql_get_device_status(void* stream);
+
+/* Upper bound, in nanoseconds, on every wait inside the GEMM kernels (0 restores the
+ * default of 2 s). A wait that exceeds it makes the kernel give up cleanly and report
+ * QL_ERR_TIMEOUT through ql_get_device_status. Process-wide; meant for diagnostics. */
+void ql_set_wait_timeout_ns(uint64_t ns);
+
+/* Static description of a status code. */
+const char* ql_status_string(ql_status s);
+
+/* The 16 NF4 grid points as the library computes them (host memory, fp32[16]). */
+void ql_nf4_codebook(float* out16);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QLORA_B200_H */

@@ -1,0 +1,250 @@
+"""ctypes binding of libqlora_b200.so: the C entry points under the same names, with
+torch tensors marshalled to device pointers. No computation happens here; every step
+of the path runs in the library's CUDA kernels. The library must be built
+(``python -m quantized_base_rank_b200.build``); loading fails loudly otherwise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libqlora_b200.so")
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "qlora.h")
+
+QL_OK, QL_ERR_INVALID_ARG, QL_ERR_UNSUPPORTED, QL_ERR_WORKSPACE, QL_ERR_NONFINITE, \
+    QL_ERR_TIMEOUT, QL_ERR_CUDA = range(7)
+QL_FMT_NF4_DQ, QL_FMT_INT8_B64 = 0, 1
+QL_OP_DQ, QL_OP_FWD, QL_OP_BWD = 0, 1, 2
+FORMATS = {"nf4_dq": QL_FMT_NF4_DQ, "int8": QL_FMT_INT8_B64}
+
+
+class QLError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class QLWeight(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("codes", ctypes.c_void_p), ("absmax", ctypes.c_void_p),
+                ("qabsmax", ctypes.c_void_p), ("group_scale", ctypes.c_void_p),
+                ("mean", ctypes.c_void_p)]
+
+
+_lib = None
+_lock = threading.Lock()
+P, I64, I32, F32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+_SIGS = {
+    "nf4_quantize": ([P, I64, P, P, P], I32),
+    "int8_quantize": ([P, I64, P, P, P], I32),
+    "dq_quantize": ([P, I64, P, P, P, P, SZ, P], I32),
+    "ql_dequantize": ([ctypes.POINTER(QLWeight), P, P], I32),
+    "qlora_linear_fwd": ([ctypes.POINTER(QLWeight), P, I64, P, P, I32, F32, P, P, P, SZ, P], I32),
+    "qlora_linear_bwd": ([ctypes.POINTER(QLWeight), P, P, I64, P, P, P, I32, F32, P, P, P, P, SZ, P], I32),
+    "ql_workspace_bytes": ([I32, I64, I64, I64, I32], SZ),
+    "ql_get_device_status": ([P], I32),
+    "ql_status_string": ([I32], ctypes.c_char_p),
+    "ql_nf4_codebook": ([ctypes.POINTER(ctypes.c_float)], None),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load the shared library (once). Raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                                   "`python -m quantized_base_rank_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            for name, (args, res) in _SIGS.items():
+                f = getattr(L, name)
+                f.argtypes = args
+                f.restype = res
+            _lib = L
+    return _lib
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/qlora.h declares."""
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s+([A-Za-z_][A-Za-z0-9_]*)\s*\(",
+                      src, flags=re.M)
+
+
+def status_string(s: int) -> str:
+    return lib().ql_status_string(int(s)).decode()
+
+
+def _check(status: int, where: str):
+    if status != QL_OK:
+        raise QLError(status, where)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device: torch.device | None = None) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _need(t: torch.Tensor, dtype: torch.dtype, name: str):
+    if not isinstance(t, torch.Tensor) or t.dtype != dtype or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+
+
+# ---- workspace: caller-owned device memory, allocated by torch, reused ----------------
+_ws = {}
+
+
+def workspace(nbytes: int, device: torch.device) -> torch.Tensor:
+    key = (device.index, torch.cuda.current_stream(device).cuda_stream)
+    buf = _ws.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        _ws[key] = buf
+    return buf
+
+
+def workspace_bytes(op: int, M: int, N: int, K: int, r: int) -> int:
+    return int(lib().ql_workspace_bytes(op, M, N, K, r))
+
+
+# ---- entry points ---------------------------------------------------------------------
+
+def nf4_quantize(W: torch.Tensor, codes: torch.Tensor | None = None,
+                 absmax: torch.Tensor | None = None):
+    _need(W, torch.bfloat16, "W")
+    n = W.numel()
+    if codes is None:
+        codes = torch.empty((n + 1) // 2, dtype=torch.uint8, device=W.device)
+    if absmax is None:
+        absmax = torch.empty((n + 63) // 64, dtype=torch.float32, device=W.device)
+    _check(lib().nf4_quantize(_ptr(W), n, _ptr(codes), _ptr(absmax), _stream(W.device)),
+           "nf4_quantize")
+    return codes, absmax
+
+
+def int8_quantize(W: torch.Tensor, codes: torch.Tensor | None = None,
+                  absmax: torch.Tensor | None = None):
+    _need(W, torch.bfloat16, "W")
+    n = W.numel()
+    if codes is None:
+        codes = torch.empty(n, dtype=torch.int8, device=W.device)
+    if absmax is None:
+        absmax = torch.empty((n + 63) // 64, dtype=torch.float32, device=W.device)
+    _check(lib().int8_quantize(_ptr(W), n, _ptr(codes), _ptr(absmax), _stream(W.device)),
+           "int8_quantize")
+    return codes, absmax
+
+
+def dq_quantize(absmax: torch.Tensor, qabsmax=None, group_scale=None, mean=None):
+    _need(absmax, torch.float32, "absmax")
+    nb = absmax.numel()
+    dev = absmax.device
+    if qabsmax is None:
+        qabsmax = torch.empty(nb, dtype=torch.int8, device=dev)
+    if group_scale is None:
+        group_scale = torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev)
+    if mean is None:
+        mean = torch.empty(1, dtype=torch.float32, device=dev)
+    nws = workspace_bytes(QL_OP_DQ, 0, 0, 0, 0)
+    ws = workspace(nws, dev)
+    _check(lib().dq_quantize(_ptr(absmax), nb, _ptr(qabsmax), _ptr(group_scale), _ptr(mean),
+                             _ptr(ws), ws.numel(), _stream(dev)), "dq_quantize")
+    return qabsmax, group_scale, mean
+
+
+class QuantWeight:
+    """A quantised weight W [N, K] held in device tensors, plus its ABI descriptor."""
+
+    def __init__(self, fmt: str, N: int, K: int, codes, absmax=None, qabsmax=None,
+                 group_scale=None, mean=None):
+        self.fmt, self.N, self.K = fmt, N, K
+        self.codes, self.absmax = codes, absmax
+        self.qabsmax, self.group_scale, self.mean = qabsmax, group_scale, mean
+        self.desc = QLWeight(FORMATS[fmt], 0, N, K, _ptr(codes), _ptr(absmax), _ptr(qabsmax),
+                             _ptr(group_scale), _ptr(mean))
+
+    @property
+    def device(self):
+        return self.codes.device
+
+    def nbytes(self) -> int:
+        ts = [self.codes, self.qabsmax, self.group_scale, self.mean] if self.fmt == "nf4_dq" \
+            else [self.codes, self.absmax]
+        return sum(t.numel() * t.element_size() for t in ts)
+
+
+def quantize_weight(W: torch.Tensor, fmt: str = "nf4_dq", keep_absmax: bool = False) -> QuantWeight:
+    """Quantise a bf16 [N, K] weight: NF4 + double quantisation, or blockwise int8."""
+    N, K = W.shape
+    if fmt == "nf4_dq":
+        codes, absmax = nf4_quantize(W)
+        qa, gs, mu = dq_quantize(absmax)
+        return QuantWeight(fmt, N, K, codes, absmax if keep_absmax else None, qa, gs, mu)
+    if fmt == "int8":
+        codes, absmax = int8_quantize(W)
+        return QuantWeight(fmt, N, K, codes, absmax)
+    raise ValueError(fmt)
+
+
+def dequantize(qw: QuantWeight) -> torch.Tensor:
+    out = torch.empty((qw.N, qw.K), dtype=torch.bfloat16, device=qw.device)
+    _check(lib().ql_dequantize(ctypes.byref(qw.desc), _ptr(out), _stream(qw.device)),
+           "ql_dequantize")
+    return out
+
+
+def linear_fwd(qw: QuantWeight, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
+               alpha: float, save_T: bool = True, Y: torch.Tensor | None = None):
+    """Y = X W'^T + (alpha/r) (X A^T) B^T. Returns (Y, T) with T = bf16(X A^T) or None."""
+    for t, nm in ((X, "X"), (A, "A"), (B, "B")):
+        _need(t, torch.bfloat16, nm)
+    M, K = X.shape
+    r = A.shape[0]
+    dev = X.device
+    if Y is None:
+        Y = torch.empty((M, qw.N), dtype=torch.bfloat16, device=dev)
+    T = torch.empty((M, r), dtype=torch.bfloat16, device=dev) if save_T else None
+    ws = workspace(workspace_bytes(QL_OP_FWD, M, qw.N, K, r), dev)
+    _check(lib().qlora_linear_fwd(ctypes.byref(qw.desc), _ptr(X), M, _ptr(A), _ptr(B), r,
+                                  float(alpha), _ptr(Y), _ptr(T), _ptr(ws), ws.numel(),
+                                  _stream(dev)), "qlora_linear_fwd")
+    return Y, T
+
+
+def linear_bwd(qw: QuantWeight, X, dY, A, B, T, alpha: float):
+    """Returns (dX bf16 [M,K], dA fp32 [r,K], dB fp32 [N,r])."""
+    for t, nm in ((X, "X"), (dY, "dY"), (A, "A"), (B, "B"), (T, "T")):
+        _need(t, torch.bfloat16, nm)
+    M, K = X.shape
+    r = A.shape[0]
+    dev = X.device
+    dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    dA = torch.empty((r, K), dtype=torch.float32, device=dev)
+    dB = torch.empty((qw.N, r), dtype=torch.float32, device=dev)
+    ws = workspace(workspace_bytes(QL_OP_BWD, M, qw.N, K, r), dev)
+    _check(lib().qlora_linear_bwd(ctypes.byref(qw.desc), _ptr(X), _ptr(dY), M, _ptr(A), _ptr(B),
+                                  _ptr(T), r, float(alpha), _ptr(dX), _ptr(dA), _ptr(dB),
+                                  _ptr(ws), ws.numel(), _stream(dev)), "qlora_linear_bwd")
+    return dX, dA, dB
+
+
+def device_status(device: torch.device | None = None) -> int:
+    """Synchronise and return (and clear) the library's sticky device flag."""
+    return int(lib().ql_get_device_status(_stream(device)))
+
+
+def nf4_codebook() -> list[float]:
+    buf = (ctypes.c_float * 16)()
+    lib().ql_nf4_codebook(buf)
+    return list(buf)

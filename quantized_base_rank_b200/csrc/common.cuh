@@ -1,0 +1,65 @@
+// Shared device/host helpers of the B200 quantised-linear library (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "qlora.h"
+
+namespace qlb {
+
+constexpr int kBlock = 64;        // elements per quantisation block
+constexpr int kGroup = 256;       // blocks per double-quantisation group
+constexpr int kFlagNonfinite = 1;
+constexpr int kFlagTimeout = 2;
+
+// NF4 grid and its exact decision points, computed once on the host by this
+// library (codebook.cu) and passed to kernels by value.
+struct Nf4Tables {
+  float q[16];          // grid points q_0 < ... < q_15, fp32
+  double mid_pos[7];    // positive midpoints (q_j + q_{j+1})/2, j = 8..14, exact in fp64
+};
+
+const Nf4Tables& nf4_tables();          // host, computed on first use
+int* device_flag_ptr();                 // device address of the sticky flag (current device)
+int num_sms();                          // SM count of the current device
+
+__host__ __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
+__host__ __device__ __forceinline__ int64_t imax64(int64_t a, int64_t b) { return a > b ? a : b; }
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned(const void* p, uintptr_t a) {
+  return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+#define QL_CHECK_LAUNCH()                                         \
+  do {                                                            \
+    if (cudaGetLastError() != cudaSuccess) return QL_ERR_CUDA;    \
+  } while (0)
+
+// ---- device helpers -------------------------------------------------------------
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t b16) {
+  return __uint_as_float(b16 << 16);
+}
+
+// fp32 -> bf16 bits, round to nearest even (the hardware conversion).
+__device__ __forceinline__ uint32_t float_to_bf16_bits(float f) {
+  uint16_t r;
+  asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(f));
+  return r;
+}
+
+// two fp32 -> packed bf16x2 (lo in bits 0..15), round to nearest even.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ void raise_flag(int* flag, int bits) {
+  if (flag) atomicOr(flag, bits);
+}
+
+}  // namespace qlb

@@ -1,0 +1,111 @@
+// Host-side runtime pieces: the NF4 tables, the sticky device flag, status strings.
+#include <math.h>
+
+#include <mutex>
+
+#include "common.cuh"
+
+namespace qlb {
+
+// Standard normal CDF through the complementary error function.
+static double norm_cdf(double z) { return 0.5 * erfc(-z / 1.4142135623730950488); }
+
+// Q_N(p): the standard normal quantile, by bisection on the CDF until the bracket is
+// two adjacent doubles (erfc is accurate to about one ulp, which puts the quantile
+// within a few ulps of the true value for the probabilities used here).
+static double norm_quantile(double p) {
+  double lo = -12.0, hi = 12.0;
+  for (int it = 0; it < 400; ++it) {
+    double mid = 0.5 * (lo + hi);
+    if (mid <= lo || mid >= hi) break;
+    if (norm_cdf(mid) < p) lo = mid; else hi = mid;
+  }
+  return 0.5 * (lo + hi);
+}
+
+// The NF4 grid of the QLoRA page ("1. 4-bit NormalFloat (NF4)"): quantiles of N(0,1)
+// at the centres (i + 1/2)/16 of 16 equal-probability bins, normalised so the largest
+// magnitude is 1, each rounded once to fp32.
+static Nf4Tables build_tables() {
+  Nf4Tables t;
+  const double zmax = norm_quantile(31.0 / 32.0);
+  for (int i = 0; i < 16; ++i) t.q[i] = (float)(norm_quantile((i + 0.5) / 16.0) / zmax);
+  // exact midpoints of adjacent fp32 points (sum and halving are exact in fp64)
+  for (int k = 0; k < 7; ++k) t.mid_pos[k] = ((double)t.q[8 + k] + (double)t.q[9 + k]) * 0.5;
+  return t;
+}
+
+const Nf4Tables& nf4_tables() {
+  static const Nf4Tables t = build_tables();
+  return t;
+}
+
+__device__ int g_ql_flag;
+
+int* device_flag_ptr() {
+  static std::mutex mu;
+  static int* ptrs[128] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_ql_flag) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
+int num_sms() {
+  static std::mutex mu;
+  static int cache[128] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 148;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev]) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = v > 0 ? v : 148;
+  }
+  return cache[dev];
+}
+
+}  // namespace qlb
+
+extern "C" {
+
+ql_status ql_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(qlb::as_stream(stream)) != cudaSuccess) return QL_ERR_CUDA;
+  int* p = qlb::device_flag_ptr();
+  if (!p) return QL_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return QL_ERR_CUDA;
+  if (v) {
+    int z = 0;
+    if (cudaMemcpy(p, &z, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return QL_ERR_CUDA;
+  }
+  if (v & qlb::kFlagTimeout) return QL_ERR_TIMEOUT;
+  if (v & qlb::kFlagNonfinite) return QL_ERR_NONFINITE;
+  return QL_OK;
+}
+
+const char* ql_status_string(ql_status s) {
+  switch (s) {
+    case QL_OK: return "ok";
+    case QL_ERR_INVALID_ARG: return "invalid argument";
+    case QL_ERR_UNSUPPORTED: return "unsupported shape or format";
+    case QL_ERR_WORKSPACE: return "workspace too small";
+    case QL_ERR_NONFINITE: return "non-finite input";
+    case QL_ERR_TIMEOUT: return "bounded device wait timed out";
+    case QL_ERR_CUDA: return "CUDA runtime error";
+  }
+  return "unknown status";
+}
+
+void ql_nf4_codebook(float* out16) {
+  if (!out16) return;
+  const qlb::Nf4Tables& t = qlb::nf4_tables();
+  for (int i = 0; i < 16; ++i) out16[i] = t.q[i];
+}
+
+}  // extern "C"

@@ -1,0 +1,62 @@
+"""CPU checks of the C-ABI library: it builds, loads, exports every declared symbol,
+and its host-only entry points behave (no kernel is launched here)."""
+import ctypes
+import os
+
+import numpy as np
+import pytest
+
+import oracle.qlora_oracle as o
+from quantized_base_rank_b200 import binding as B
+from quantized_base_rank_b200 import build as build_mod
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(B.LIB_PATH):
+        build_mod.build()
+    return B.lib()
+
+
+def test_header_declares_the_boundary():
+    names = set(B.header_functions())
+    for required in ("nf4_quantize", "dq_quantize", "int8_quantize", "ql_dequantize",
+                     "qlora_linear_fwd", "qlora_linear_bwd", "ql_workspace_bytes",
+                     "ql_get_device_status", "ql_status_string", "ql_nf4_codebook"):
+        assert required in names, required
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in B.header_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert B.status_string(s)
+    assert B.status_string(0) == "ok"
+
+
+def test_library_codebook_equals_oracle(lib):
+    """The library computes its grid independently (bisection on erfc, in C); it must
+    land on the same fp32 points as the oracle."""
+    q = np.float32(B.nf4_codebook())
+    assert np.array_equal(q.view(np.uint32), o.nf4_codebook().view(np.uint32))
+
+
+def test_argument_validation_without_a_device(lib):
+    # rejected before any CUDA call
+    assert lib.nf4_quantize(None, 64, None, None, None) == B.QL_ERR_INVALID_ARG
+    assert lib.nf4_quantize(None, -1, None, None, None) == B.QL_ERR_INVALID_ARG
+    assert lib.nf4_quantize(None, 0, None, None, None) == B.QL_OK
+    assert lib.int8_quantize(None, 64, None, None, None) == B.QL_ERR_INVALID_ARG
+    assert lib.dq_quantize(None, 4, None, None, None, None, 0, None) == B.QL_ERR_INVALID_ARG
+    assert lib.ql_dequantize(None, None, None) == B.QL_ERR_INVALID_ARG
+    w = B.QLWeight(0, 0, 64, 64, 16, 0, 16, 16, 16)
+    # misaligned or null pointers, bad shapes: all rejected synchronously
+    assert lib.qlora_linear_fwd(ctypes.byref(w), None, 1, None, None, 8, 16.0, None, None,
+                                None, 0, None) == B.QL_ERR_INVALID_ARG
+
+
+def test_workspace_query(lib):
+    assert B.workspace_bytes(B.QL_OP_DQ, 0, 0, 0, 0) >= 128

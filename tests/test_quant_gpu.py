@@ -1,0 +1,121 @@
+"""GPU vs oracle, bit-exact: NF4 codes, absmax, double-quantised constants, int8
+codes and dequantised weights, on the workloads' weights and on edge cases."""
+import numpy as np
+import pytest
+import torch
+
+import oracle.qlora_oracle as o
+from quantized_base_rank_b200 import binding as B
+from quantized_base_rank_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _u32(x):
+    return np.asarray(x, np.float32).view(np.uint32)
+
+
+def _weights():
+    yield "cfg1-256x256", synth.make_inputs(synth.CFG1)["W"]
+    yield "cfg2-4096x4096-outliers", synth.weight_with_outliers(4096, 4096, 0.02, 0.001, 20.0, 0)
+    yield "ragged-odd", synth.normal_bf16((64 * 1000 + 37,), 0.02, 5, 0)
+    rng = np.random.default_rng(9)
+    special = np.zeros(64 * 64, np.float32)
+    special[64:128] = 0.0                                            # zero block
+    special[128:192] = -0.0
+    special[192:256] = rng.standard_normal(64) * 1e-39               # subnormal block
+    special[256:320] = rng.standard_normal(64) * 3e38 / 4            # huge block
+    special[320:384] = np.float32([1.0, -1.0] * 32)                  # +-absmax only
+    vals = (np.arange(0, 0x7F80, 7, dtype=np.uint32) << 16).view(np.float32)
+    special[384:384 + 2048] = np.resize(vals, 2048) * np.resize([1, -1], 2048)
+    special[2432:] = rng.standard_normal(special.size - 2432) * 0.05
+    yield "special-values", synth.to_bf16(special)
+
+
+WEIGHTS = list(_weights())
+
+
+@pytest.mark.parametrize("name,W", WEIGHTS, ids=[w[0] for w in WEIGHTS])
+def test_nf4_dq_bitexact(name, W):
+    w = W.float().numpy().ravel()
+    n = w.size
+    codes, absmax = B.nf4_quantize(W.cuda().contiguous().view(-1))
+    qa, gs, mu = B.dq_quantize(absmax)
+    ref_codes, ref_a = o.nf4_quantize(w)
+    ref_qa, ref_gs, ref_mu = o.dq_encode(ref_a)
+    assert np.array_equal(codes.cpu().numpy(), ref_codes)
+    assert np.array_equal(_u32(absmax.cpu().numpy()), _u32(ref_a))
+    assert np.array_equal(qa.cpu().numpy(), ref_qa)
+    assert np.array_equal(_u32(gs.cpu().numpy()), _u32(ref_gs))
+    assert _u32(mu.cpu().numpy())[0] == _u32(np.float32(ref_mu))
+    if n % 64 == 0:
+        Wr = W.reshape(-1, 64)
+        qw = B.QuantWeight("nf4_dq", Wr.shape[0], 64, codes, None, qa, gs, mu)
+        wd = B.dequantize(qw).float().cpu().numpy().ravel()
+        ref_wd = o.nf4_dequant(ref_codes, o.dq_decode(ref_qa, ref_gs, ref_mu), n)
+        assert np.array_equal(_u32(wd), _u32(ref_wd))
+    assert B.device_status() == B.QL_OK
+
+
+@pytest.mark.parametrize("name,W", WEIGHTS, ids=[w[0] for w in WEIGHTS])
+def test_int8_bitexact(name, W):
+    w = W.float().numpy().ravel()
+    codes, absmax = B.int8_quantize(W.cuda().contiguous().view(-1))
+    ref_c, ref_a = o.int8_quantize(w)
+    assert np.array_equal(codes.cpu().numpy(), ref_c)
+    assert np.array_equal(_u32(absmax.cpu().numpy()), _u32(ref_a))
+    if w.size % 64 == 0:
+        qw = B.QuantWeight("int8", w.size // 64, 64, codes, absmax)
+        wd = B.dequantize(qw).float().cpu().numpy().ravel()
+        assert np.array_equal(_u32(wd), _u32(o.int8_dequant(ref_c, ref_a)))
+    assert B.device_status() == B.QL_OK
+
+
+def test_unaligned_input_takes_scalar_path():
+    W = synth.normal_bf16((64 * 300 + 3,), 0.02, 6, 0).cuda()
+    Wu = W[1:]                                   # 2-byte aligned, not 16
+    codes, absmax = B.nf4_quantize(Wu)
+    ref_codes, ref_a = o.nf4_quantize(Wu.float().cpu().numpy())
+    assert np.array_equal(codes.cpu().numpy(), ref_codes)
+    assert np.array_equal(_u32(absmax.cpu().numpy()), _u32(ref_a))
+
+
+def test_dq_exact_mean_on_wide_exponent_range():
+    """Arbitrary fp32 constants spanning ~240 binades: the mean comes from the exact
+    sum, so GPU and oracle (math.fsum) agree bit for bit."""
+    rng = np.random.default_rng(21)
+    a = (rng.random(300_000) * 2.0 ** rng.integers(-148, 100, 300_000)).astype(np.float32)
+    a[:5] = np.float32([0.0, 1e-45, 3.0e38, 1.0, 2.0 ** -126])
+    qa, gs, mu = B.dq_quantize(torch.from_numpy(a).cuda())
+    rqa, rgs, rmu = o.dq_encode(a)
+    assert _u32(mu.cpu().numpy())[0] == _u32(np.float32(rmu))
+    assert np.array_equal(_u32(gs.cpu().numpy()), _u32(rgs))
+    assert np.array_equal(qa.cpu().numpy(), rqa)
+
+
+def test_nonfinite_input_sets_device_flag():
+    assert B.device_status() == B.QL_OK
+    W = synth.normal_bf16((64 * 8,), 0.02, 7, 0)
+    W[100] = float("nan")
+    B.nf4_quantize(W.cuda())
+    assert B.device_status() == B.QL_ERR_NONFINITE
+    assert B.device_status() == B.QL_OK            # cleared on read
+    W[100] = float("inf")
+    B.int8_quantize(W.cuda())
+    assert B.device_status() == B.QL_ERR_NONFINITE
+
+
+@pytest.mark.parametrize("N,K", [(8192, 8192), (22016, 8192)])
+def test_full_size_65b_shapes(N, K):
+    W = synth.normal_bf16((N, K), 0.02, 3, N % 7).cuda()
+    codes, absmax = B.nf4_quantize(W.view(-1))
+    qa, gs, mu = B.dq_quantize(absmax)
+    w = W.float().cpu().numpy().ravel()
+    ref_codes, ref_a = o.nf4_quantize(w)
+    ref_qa, ref_gs, ref_mu = o.dq_encode(ref_a)
+    assert np.array_equal(codes.cpu().numpy(), ref_codes)
+    assert np.array_equal(qa.cpu().numpy(), ref_qa)
+    assert _u32(mu.cpu().numpy())[0] == _u32(np.float32(ref_mu))
+    c8, a8 = B.int8_quantize(W.view(-1))
+    rc8, ra8 = o.int8_quantize(w)
+    assert np.array_equal(c8.cpu().numpy(), rc8)
