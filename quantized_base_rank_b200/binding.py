@@ -51,6 +51,7 @@ _SIGS = {
     "ql_get_device_status": ([P], I32),
     "ql_status_string": ([I32], ctypes.c_char_p),
     "ql_nf4_codebook": ([ctypes.POINTER(ctypes.c_float)], None),
+    "ql_set_wait_timeout_ns": ([ctypes.c_uint64], None),
 }
 
 

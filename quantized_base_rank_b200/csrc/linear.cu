@@ -1,0 +1,306 @@
+// The quantised linear layer with an unmerged LoRA branch: forward, input-backward and
+// adapter gradients, built from instances of the tcgen05 GEMM in gemm.cuh.
+//
+// QLoRA page (aizip.shop/methodologies/qlora), "memory decomposition": the frozen base
+// is stored 4-bit and the adapters stay bf16 and unmerged. AutoQRA page
+// (gist.science/ko/paper/2602.22268) section 3.1: each layer picks its bit-width
+// (NF4+DQ or int8 here) and its rank r.
+//
+// Forward  (3 launches): pad B -> Bp;  [T | P] = X A^T  (P = bf16(s T));
+//                        Y = X W'^T + P Bp^T  (W' decoded in the producer warps, P Bp^T
+//                        as extra contraction chunks of the same accumulator)
+// Backward (5 launches): prep (B^T, A^T padded, T padded); Q = bf16(s dY B);
+//                        dB = s dY^T T;  dA = Q^T X;  dX = dY W' + Q A.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "common.cuh"
+#include "gemm.cuh"
+
+namespace qlb {
+
+static std::atomic<uint64_t> g_wait_timeout_ns{2000000000ull};
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// bf16 matrix [outer, inner] with row stride `ld` elements; box {64, box_outer} with
+// the 128-byte swizzle (one 128-byte smem row per box row).
+static bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld,
+                     uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {64, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, int NP, bool A_MN, BSrc BS, bool B_MN, int EPI>
+static ql_status launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& ae,
+                             const CUtensorMap& be, const GemmArgs& args, cudaStream_t st) {
+  auto kern = qgemm_kernel<BN, NP, A_MN, BS, B_MN, EPI>;
+  const size_t smem = GemmCfg<BN>::kSmem;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return QL_ERR_CUDA;
+  const int64_t tiles = ((args.R + 127) / 128) * ((args.Cn + BN - 1) / BN);
+  const int grid = (int)imin64(tiles, num_sms());
+  if (grid <= 0) return QL_OK;
+  kern<<<grid, (6 + NP) * 32, smem, st>>>(a, b, ae, be, args);
+  QL_CHECK_LAUNCH();
+  return QL_OK;
+}
+
+// ---- small layout kernels (adapter-sized tensors only) ----------------------------
+
+// dst[i, j] = j < r ? src[i, j] : 0, dst [rows, rp]
+__global__ void pad_cols_kernel(const uint16_t* __restrict__ src, int64_t rows, int r, int rp,
+                                uint16_t* __restrict__ dst) {
+  const int64_t total = rows * rp;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = i / rp;
+    const int j = (int)(i % rp);
+    dst[i] = j < r ? src[row * r + j] : (uint16_t)0;
+  }
+}
+
+// dst[c, j] = j < r ? src[j, c] : 0, src [r, cols], dst [cols, rp]
+__global__ void transpose_pad_kernel(const uint16_t* __restrict__ src, int r, int64_t cols, int rp,
+                                     uint16_t* __restrict__ dst) {
+  const int64_t total = cols * rp;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t c = i / rp;
+    const int j = (int)(i % rp);
+    dst[i] = j < r ? src[(int64_t)j * cols + c] : (uint16_t)0;
+  }
+}
+
+// dst[j, n] = src[n, j], src [rows, r], dst [r, rows]
+__global__ void transpose_kernel(const uint16_t* __restrict__ src, int64_t rows, int r,
+                                 uint16_t* __restrict__ dst) {
+  const int64_t total = rows * r;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int j = (int)(i / rows);
+    const int64_t n = i % rows;
+    dst[i] = src[n * r + j];
+  }
+}
+
+static int small_grid(int64_t n) { return (int)imax64(1, imin64((n + 255) / 256, (int64_t)num_sms() * 8)); }
+
+static int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+struct WsLayout {
+  int64_t off[4];
+  int64_t total;
+};
+
+static WsLayout ws_layout(int op, int64_t M, int64_t N, int64_t K, int r) {
+  WsLayout L{};
+  const int64_t rp = round_up(r, 64);
+  int64_t sz[4] = {0, 0, 0, 0};
+  if (op == QL_OP_FWD) {
+    sz[0] = M * rp * 2;        // P
+    sz[1] = N * rp * 2;        // B padded
+  } else if (op == QL_OP_BWD) {
+    sz[0] = M * rp * 2;        // Q
+    sz[1] = (int64_t)r * N * 2;  // B^T
+    sz[2] = K * rp * 2;        // A^T padded
+    sz[3] = M * rp * 2;        // T padded
+  } else if (op == QL_OP_DQ) {
+    sz[0] = 256;
+  }
+  int64_t o = 0;
+  for (int i = 0; i < 4; ++i) {
+    L.off[i] = o;
+    o += round_up(sz[i], 256);
+  }
+  L.total = o;
+  return L;
+}
+
+static GemmArgs base_args(const ql_weight* w) {
+  GemmArgs a{};
+  const Nf4Tables& t = nf4_tables();
+  for (int i = 0; i < 16; ++i) a.q[i] = t.q[i];
+  if (w) {
+    a.codes = static_cast<const uint8_t*>(w->codes);
+    a.qabsmax = w->qabsmax;
+    a.gscale = w->group_scale;
+    a.mean = w->mean;
+    a.absmax = w->absmax;
+    a.Nw = w->N;
+    a.Kw = w->K;
+  }
+  a.timeout_ns = g_wait_timeout_ns.load();
+  a.flag = device_flag_ptr();
+  return a;
+}
+
+static ql_status check_weight(const ql_weight* w) {
+  if (!w || w->N < 1 || w->K < 64 || !w->codes || !aligned(w->codes, 16)) return QL_ERR_INVALID_ARG;
+  if (w->K % 64 != 0 || w->N % 8 != 0) return QL_ERR_UNSUPPORTED;
+  if (w->fmt == QL_FMT_NF4_DQ) {
+    if (!w->qabsmax || !w->group_scale || !w->mean) return QL_ERR_INVALID_ARG;
+  } else if (w->fmt == QL_FMT_INT8_B64) {
+    if (!w->absmax || !aligned(w->absmax, 4)) return QL_ERR_INVALID_ARG;
+  } else {
+    return QL_ERR_INVALID_ARG;
+  }
+  return QL_OK;
+}
+
+}  // namespace qlb
+
+using namespace qlb;
+
+extern "C" {
+
+size_t ql_workspace_bytes(int32_t op, int64_t M, int64_t N, int64_t K, int32_t r) {
+  if (op == QL_OP_DQ) return 256;
+  if ((op != QL_OP_FWD && op != QL_OP_BWD) || M < 0 || N < 0 || K < 0 || r < 1 || r > 256) return 0;
+  return (size_t)ws_layout(op, M, N, K, r).total;
+}
+
+void ql_set_wait_timeout_ns(uint64_t ns) {
+  g_wait_timeout_ns.store(ns ? ns : 2000000000ull);
+}
+
+ql_status qlora_linear_fwd(const ql_weight* w, const ql_bf16* X, int64_t M, const ql_bf16* A,
+                           const ql_bf16* B, int32_t r, float alpha, ql_bf16* Y, ql_bf16* T_save,
+                           void* ws, size_t ws_bytes, void* stream) {
+  ql_status st0 = check_weight(w);
+  if (st0 != QL_OK) return st0;
+  if (!X || !A || !B || !Y || !ws || M < 1 || r < 1) return QL_ERR_INVALID_ARG;
+  if (r > 256 || M > (int64_t(1) << 31)) return QL_ERR_UNSUPPORTED;
+  if (!aligned(X, 16) || !aligned(A, 16) || !aligned(B, 2) || !aligned(Y, 16) || !aligned(ws, 256) ||
+      (T_save && !aligned(T_save, 2)))
+    return QL_ERR_INVALID_ARG;
+  const int64_t N = w->N, K = w->K;
+  const WsLayout L = ws_layout(QL_OP_FWD, M, N, K, r);
+  if ((int64_t)ws_bytes < L.total) return QL_ERR_WORKSPACE;
+  const int rp = (int)round_up(r, 64);
+  const float s = alpha / (float)r;
+  cudaStream_t st = as_stream(stream);
+  uint16_t* P = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + L.off[0]);
+  uint16_t* Bp = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + L.off[1]);
+
+  pad_cols_kernel<<<small_grid(N * rp), 256, 0, st>>>(B, N, r, rp, Bp);
+  QL_CHECK_LAUNCH();
+
+  CUtensorMap mX, mA, mP, mBp, none;
+  memset(&none, 0, sizeof(none));
+  if (!make_map(&mX, X, K, M, K, 128) || !make_map(&mA, A, K, r, K, rp) ||
+      !make_map(&mP, P, rp, M, rp, 128) || !make_map(&mBp, Bp, rp, N, rp, 256))
+    return QL_ERR_CUDA;
+
+  // [T | P] = X A^T
+  GemmArgs t = base_args(nullptr);
+  t.R = M; t.Cn = rp; t.Kc = K; t.n_ext = 0; t.r = r;
+  t.out = T_save; t.ld_out = r; t.out2 = P; t.ld_out2 = rp; t.scale = s;
+  ql_status e;
+  if (rp == 64) e = launch_gemm<64, 0, false, BSrc::TMA, false, EPI_LORA_T>(mX, mA, none, none, t, st);
+  else if (rp == 128) e = launch_gemm<128, 0, false, BSrc::TMA, false, EPI_LORA_T>(mX, mA, none, none, t, st);
+  else e = launch_gemm<256, 0, false, BSrc::TMA, false, EPI_LORA_T>(mX, mA, none, none, t, st);
+  if (e != QL_OK) return e;
+
+  // Y = X W'^T + P Bp^T
+  GemmArgs y = base_args(w);
+  y.R = M; y.Cn = N; y.Kc = K; y.n_ext = rp / 64; y.r = r;
+  y.out = Y; y.ld_out = N; y.scale = 1.0f;
+  if (w->fmt == QL_FMT_NF4_DQ)
+    return launch_gemm<256, 8, false, BSrc::NF4, false, EPI_BF16>(mX, none, mP, mBp, y, st);
+  return launch_gemm<256, 8, false, BSrc::INT8, false, EPI_BF16>(mX, none, mP, mBp, y, st);
+}
+
+ql_status qlora_linear_bwd(const ql_weight* w, const ql_bf16* X, const ql_bf16* dY, int64_t M,
+                           const ql_bf16* A, const ql_bf16* B, const ql_bf16* T_saved, int32_t r,
+                           float alpha, ql_bf16* dX, float* dA, float* dB, void* ws, size_t ws_bytes,
+                           void* stream) {
+  ql_status st0 = check_weight(w);
+  if (st0 != QL_OK) return st0;
+  if (!X || !dY || !A || !B || !T_saved || !dX || !dA || !dB || !ws || M < 1 || r < 1)
+    return QL_ERR_INVALID_ARG;
+  if (r > 256 || M > (int64_t(1) << 31)) return QL_ERR_UNSUPPORTED;
+  if (!aligned(X, 16) || !aligned(dY, 16) || !aligned(A, 2) || !aligned(B, 2) || !aligned(T_saved, 2) ||
+      !aligned(dX, 16) || !aligned(dA, 4) || !aligned(dB, 4) || !aligned(ws, 256))
+    return QL_ERR_INVALID_ARG;
+  const int64_t N = w->N, K = w->K;
+  const WsLayout L = ws_layout(QL_OP_BWD, M, N, K, r);
+  if ((int64_t)ws_bytes < L.total) return QL_ERR_WORKSPACE;
+  const int rp = (int)round_up(r, 64);
+  const float s = alpha / (float)r;
+  cudaStream_t st = as_stream(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  uint16_t* Q = reinterpret_cast<uint16_t*>(wsb + L.off[0]);
+  uint16_t* Bt = reinterpret_cast<uint16_t*>(wsb + L.off[1]);
+  uint16_t* At = reinterpret_cast<uint16_t*>(wsb + L.off[2]);
+  uint16_t* Tp = reinterpret_cast<uint16_t*>(wsb + L.off[3]);
+
+  transpose_kernel<<<small_grid(N * r), 256, 0, st>>>(B, N, r, Bt);
+  QL_CHECK_LAUNCH();
+  transpose_pad_kernel<<<small_grid(K * rp), 256, 0, st>>>(A, r, K, rp, At);
+  QL_CHECK_LAUNCH();
+  pad_cols_kernel<<<small_grid(M * rp), 256, 0, st>>>(T_saved, M, r, rp, Tp);
+  QL_CHECK_LAUNCH();
+
+  CUtensorMap mdY_k, mBt, mQ_k, mAt, mdY_mn, mTp_mn, mX_mn, mQ_mn, none;
+  memset(&none, 0, sizeof(none));
+  if (!make_map(&mdY_k, dY, N, M, N, 128) || !make_map(&mBt, Bt, N, r, N, rp) ||
+      !make_map(&mQ_k, Q, rp, M, rp, 128) || !make_map(&mAt, At, rp, K, rp, 256) ||
+      !make_map(&mdY_mn, dY, N, M, N, 64) || !make_map(&mTp_mn, Tp, rp, M, rp, 64) ||
+      !make_map(&mX_mn, X, K, M, K, 64) || !make_map(&mQ_mn, Q, rp, M, rp, 64))
+    return QL_ERR_CUDA;
+  ql_status e;
+
+  // Q = bf16(s dY B)
+  GemmArgs u = base_args(nullptr);
+  u.R = M; u.Cn = rp; u.Kc = N; u.r = r; u.out = Q; u.ld_out = rp; u.scale = s;
+  if (rp == 64) e = launch_gemm<64, 0, false, BSrc::TMA, false, EPI_LORA_Q>(mdY_k, mBt, none, none, u, st);
+  else if (rp == 128) e = launch_gemm<128, 0, false, BSrc::TMA, false, EPI_LORA_Q>(mdY_k, mBt, none, none, u, st);
+  else e = launch_gemm<256, 0, false, BSrc::TMA, false, EPI_LORA_Q>(mdY_k, mBt, none, none, u, st);
+  if (e != QL_OK) return e;
+
+  // dB = s dY^T T     (rows n, columns j, contraction over tokens)
+  GemmArgs b = base_args(nullptr);
+  b.R = N; b.Cn = rp; b.Kc = M; b.r = r; b.out = dB; b.ld_out = r; b.scale = s;
+  if (rp == 64) e = launch_gemm<64, 0, true, BSrc::TMA, true, EPI_DB>(mdY_mn, mTp_mn, none, none, b, st);
+  else if (rp == 128) e = launch_gemm<128, 0, true, BSrc::TMA, true, EPI_DB>(mdY_mn, mTp_mn, none, none, b, st);
+  else e = launch_gemm<256, 0, true, BSrc::TMA, true, EPI_DB>(mdY_mn, mTp_mn, none, none, b, st);
+  if (e != QL_OK) return e;
+
+  // dA = Q^T X        (computed as dA^T: rows k, columns j)
+  GemmArgs a = base_args(nullptr);
+  a.R = K; a.Cn = rp; a.Kc = M; a.r = r; a.out = dA; a.ld_out = K; a.scale = 1.0f;
+  if (rp == 64) e = launch_gemm<64, 0, true, BSrc::TMA, true, EPI_DA>(mX_mn, mQ_mn, none, none, a, st);
+  else if (rp == 128) e = launch_gemm<128, 0, true, BSrc::TMA, true, EPI_DA>(mX_mn, mQ_mn, none, none, a, st);
+  else e = launch_gemm<256, 0, true, BSrc::TMA, true, EPI_DA>(mX_mn, mQ_mn, none, none, a, st);
+  if (e != QL_OK) return e;
+
+  // dX = dY W' + Q A^T-padded
+  GemmArgs x = base_args(w);
+  x.R = M; x.Cn = K; x.Kc = N; x.n_ext = rp / 64; x.r = r; x.out = dX; x.ld_out = K; x.scale = 1.0f;
+  if (w->fmt == QL_FMT_NF4_DQ)
+    return launch_gemm<256, 8, false, BSrc::NF4, true, EPI_BF16>(mdY_k, none, mQ_k, mAt, x, st);
+  return launch_gemm<256, 8, false, BSrc::INT8, true, EPI_BF16>(mdY_k, none, mQ_k, mAt, x, st);
+}
+
+}  // extern "C"
