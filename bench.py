@@ -1,0 +1,394 @@
+#!/usr/bin/env python
+"""Benchmark of the QLoRA-style quantised linear on B200.
+
+One step = the whole hot path on one batch: NF4 quantisation + double quantisation of
+the frozen bf16 weight, the fused forward Y = X W'^T + s (X A^T) B^T, and the backward
+(dX, dA, dB). Workload: the fine-tune-shaped MLP up-projection (W 11008x4096 ~N(0,0.02),
+X 8192x4096 ~N(0,1), LoRA r=64, alpha=16, dY ~N(0,1)), seeded synthetic data.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs its own batch (weak scaling) and the adapter
+gradients dA, dB are summed across ranks with NCCL, the data-parallel exchange step.
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused NF4+LoRA linear TFLOP/s & HBM GB/s (% of roofline); quantize GB/s"
+NF4_DQ_BYTES_PER_PARAM = 2.0 + 0.5 + 1.0 / 64 + 4.0 / 16384   # bf16 read + codes + consts
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def linear_flops(M, N, K, r):
+    fwd = 2 * M * N * K + 2 * M * K * r + 2 * M * N * r
+    bwd = (2 * M * N * K + 2 * M * N * r + 2 * M * r * K) + 2 * M * r * K + 2 * M * N * r
+    return fwd, bwd
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples taken while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            target = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:
+            target = str(device_index)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", target], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------------------
+# CPU oracle leg (reported baseline / reference arm)
+# --------------------------------------------------------------------------------------
+
+def oracle_step(inp_np, case, m_rows: int, n_rows: int):
+    """One bounded sample of the step on the host: quantise n_rows rows of W (NF4 + DQ),
+    then forward + backward in fp64 for m_rows tokens over the full weight."""
+    import oracle.qlora_oracle as o
+    w = inp_np["W"]
+    t0 = time.perf_counter()
+    o.quantize_weight(w[:n_rows], "nf4_dq")
+    wd = inp_np["Wd"]
+    X = inp_np["X"][:m_rows]
+    dY = inp_np["dY"][:m_rows]
+    o.linear_fwd(X, wd, inp_np["A"], inp_np["B"], case.alpha, case.r)
+    o.linear_bwd(X, dY, wd, inp_np["A"], inp_np["B"], case.alpha, case.r)
+    dt = time.perf_counter() - t0
+    f, b = linear_flops(m_rows, case.N, case.K, case.r)
+    return dt, f + b
+
+
+def oracle_inputs(case):
+    import oracle.qlora_oracle as o
+    from quantized_base_rank_b200 import synth
+    inp = synth.make_inputs(case)
+    f = lambda t: t.float().numpy()
+    w = f(inp["W"])
+    wd = o.quantize_weight(w, "nf4_dq")["wdeq"].reshape(case.N, case.K).astype(np.float64)
+    return {"W": w, "Wd": wd, "X": f(inp["X"]).astype(np.float64), "A": f(inp["A"]).astype(np.float64),
+            "B": f(inp["B"]).astype(np.float64), "dY": f(inp["dY"]).astype(np.float64)}
+
+
+def blas_threads() -> int:
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        return max(i.get("num_threads", 1) for i in info) if info else os.cpu_count()
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return "unknown"
+
+
+def run_reference(args, case, world, rank):
+    if rank != 0:
+        return
+    inp = oracle_inputs(case)
+    # per step: 256 weight rows quantised, 32 tokens through fwd + bwd over the full weight
+    m_rows, n_rows = 32, 256
+    for _ in range(args.warmup):
+        oracle_step(inp, case, m_rows, n_rows)
+    tot_t, tot_f = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, fl = oracle_step(inp, case, m_rows, n_rows)
+        tot_t += dt
+        tot_f += fl
+    value = tot_f / tot_t / 1e12
+    sample = (f"each step: NF4+DQ quantise of {n_rows} of {case.N} weight rows, fp64 forward + "
+              f"backward for {m_rows} of {case.M} tokens over the full {case.N}x{case.K} weight")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": case.name, "M": case.M, "N": case.N, "K": case.K, "r": case.r,
+                       "alpha": case.alpha, "format": "nf4_dq"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(),
+                             "kind": "oracle", "sample": sample, "cpu": cpu_model()},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------------------
+# GPU leg
+# --------------------------------------------------------------------------------------
+
+def run_ours(args, case, world, rank, local_rank):
+    from quantized_base_rank_b200 import binding as B
+    from quantized_base_rank_b200 import synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+    peaks = load_peaks()
+    seed_case = synth.LinearCase(**{**case.__dict__, "seed": case.seed + rank})
+    inp = synth.make_inputs(seed_case)
+    M, N, K, r = case.M, case.N, case.K, case.r
+    W = inp["W"].to(dev)
+    X, A, Bm, dY = (inp[k].to(dev) for k in ("X", "A", "B", "dY"))
+    n = N * K
+    codes = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+    absmax = torch.empty(n // 64, dtype=torch.float32, device=dev)
+    qa = torch.empty(n // 64, dtype=torch.int8, device=dev)
+    gs = torch.empty((n // 64 + 255) // 256, dtype=torch.float32, device=dev)
+    mu = torch.empty(1, dtype=torch.float32, device=dev)
+    qw = B.QuantWeight("nf4_dq", N, K, codes, None, qa, gs, mu)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    T = torch.empty((M, r), dtype=torch.bfloat16, device=dev)
+    dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    dA = torch.empty((r, K), dtype=torch.float32, device=dev)
+    dB = torch.empty((N, r), dtype=torch.float32, device=dev)
+
+    def step():
+        B.nf4_quantize(W, codes, absmax)
+        B.dq_quantize(absmax, qa, gs, mu)
+        B.linear_fwd(qw, X, A, Bm, case.alpha, Y=Y, T=T)
+        B.linear_bwd(qw, X, dY, A, Bm, T, case.alpha, dX=dX, dA=dA, dB=dB)
+        if dist is not None:
+            dist.all_reduce(dA)
+            dist.all_reduce(dB)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def timed(fn, steps):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(steps):
+            fn()
+        e.record()
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        ms = s.elapsed_time(e) / steps
+        if dist is not None:
+            t = torch.tensor([ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    # ---- device-resident timed region ----
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    for g in B.PROFILE_GROUPS:
+        B.profile_read(g)                     # drop anything recorded so far
+    clocks = ClockSampler(dev.index) if rank == 0 else None
+    B.profile_enable(True)
+    c0 = B.launch_count()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ev_s, ev_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev_s.record()
+    for _ in range(args.steps):
+        step()
+    ev_e.record()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    B.profile_enable(False)
+    launches = B.launch_count() - c0
+    clk = clocks.stop() if clocks else None
+    ms = ev_s.elapsed_time(ev_e) / args.steps
+    if dist is not None:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    prof = {g: B.profile_read(g) for g in B.PROFILE_GROUPS}
+    assert B.device_status() == B.QL_OK
+
+    fwd_f, bwd_f = linear_flops(M, N, K, r)
+    value = world * (fwd_f + bwd_f) / (ms * 1e-3) / 1e12
+
+    def avg(g):
+        t, c = prof[g]
+        return t / c if c else float("nan")
+
+    fwd_ms = sum(avg(g) for g in ("fwd_prep", "fwd_xa", "fwd_main"))
+    bwd_ms = sum(avg(g) for g in ("bwd_prep", "bwd_dyb", "bwd_db", "bwd_da", "bwd_dx"))
+    q_ms = avg("nf4") + avg("dq")
+    main_flops = 2 * M * N * (K + r)                # algorithmic work of the fused forward GEMM
+    main_ms = avg("fwd_main")
+    achieved = main_flops / (main_ms * 1e-3) / 1e12
+    dx_ms = avg("bwd_dx")
+    dx_flops = 2 * M * N * K + 2 * M * r * K
+
+    # ---- end-to-end through the public API with host buffers ----
+    pin = lambda t: t.pin_memory()
+    hW, hX, hA, hB, hdY = (pin(inp[k]) for k in ("W", "X", "A", "B", "dY"))
+    hdA = torch.empty_like(dA, device="cpu").pin_memory()
+    hdB = torch.empty_like(dB, device="cpu").pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hW, hX, hA, hB, hdY))
+    d2h = hdA.numel() * 4 + hdB.numel() * 4
+
+    def e2e_step():
+        W.copy_(hW, non_blocking=True)
+        X.copy_(hX, non_blocking=True)
+        A.copy_(hA, non_blocking=True)
+        Bm.copy_(hB, non_blocking=True)
+        dY.copy_(hdY, non_blocking=True)
+        step()
+        hdA.copy_(dA, non_blocking=True)
+        hdB.copy_(dB, non_blocking=True)
+
+    e2e_steps = max(3, args.steps // 10)
+    e2e_ms = timed(e2e_step, e2e_steps)
+    e2e_value = world * (fwd_f + bwd_f) / (e2e_ms * 1e-3) / 1e12
+
+    # ---- CPU oracle baseline (rank 0, one GPU only) ----
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        o_inp = oracle_inputs(case)
+        m_rows, n_rows = 1024, case.N
+        dt, fl = oracle_step(o_inp, case, m_rows, n_rows)
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": (f"one step with the full {N}x{K} weight quantised (NF4+DQ) and fp64 "
+                          f"forward + backward for {m_rows} of {M} tokens; {dt:.1f} s"),
+               "cpu": cpu_model()}
+
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": case.name, "M": M, "N": N, "K": K, "r": r, "alpha": case.alpha,
+                   "format": "nf4_dq", "step": "quantise(NF4+DQ) + fwd + bwd(dX,dA,dB)",
+                   "l2": "inputs larger than L2 (X 64 MB, W 90 MB, dY 180 MB > 126 MB)",
+                   "parallelism": f"dp{world}" if world > 1 else "single"},
+        "roofline": {"kernel": "fused forward GEMM (NF4 decode + X W'^T + P B^T)", "bound": "tensor",
+                     "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                     "peak_source": f"{peaks['source']} bf16 burst",
+                     "frac_of_sustained": (achieved / peaks["bf16_tflops_sustained"]
+                                           if peaks["bf16_tflops_sustained"] else None)},
+        "components": {
+            "quantize_nf4_dq": {"ms": q_ms, "GB/s": n * NF4_DQ_BYTES_PER_PARAM / (q_ms * 1e-3) / 1e9,
+                                "frac_hbm": n * NF4_DQ_BYTES_PER_PARAM / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+            "forward": {"ms": fwd_ms, "TFLOP/s": fwd_f / (fwd_ms * 1e-3) / 1e12},
+            "backward": {"ms": bwd_ms, "TFLOP/s": bwd_f / (bwd_ms * 1e-3) / 1e12},
+            "fwd_main_gemm": {"ms": main_ms, "TFLOP/s": achieved},
+            "bwd_dx_gemm": {"ms": dx_ms, "TFLOP/s": dx_flops / (dx_ms * 1e-3) / 1e12},
+            "per_group_ms": {g: avg(g) for g in B.PROFILE_GROUPS if prof[g][1]},
+        },
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": launches,
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    from quantized_base_rank_b200 import synth
+    case = synth.CFG3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, case, world, rank)
+        return
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, case, world, rank, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

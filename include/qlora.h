@@ -150,6 +150,18 @@ ql_status ql_get_device_status(void* stream);
  * QL_ERR_TIMEOUT through ql_get_device_status. Process-wide; meant for diagnostics. */
 void ql_set_wait_timeout_ns(uint64_t ns);
 
+/* Measurement hooks. When enabled, every kernel group launched by the entry points is
+ * bracketed by two CUDA events on its launch stream; ql_profile_read synchronises on
+ * them and returns (then forgets) the summed milliseconds and the number of launches of
+ * one group. Groups: 0 nf4 encode, 1 double quantisation, 2 int8 encode, 3 dequantise,
+ * 4 forward layout prep, 5 forward X A^T, 6 forward main GEMM, 7 backward layout prep,
+ * 8 backward dY B, 9 dB, 10 dA, 11 dX, 12 small-M forward. ql_launch_count is the
+ * running number of kernels the library has launched in this process. Returns 0, or -1
+ * for an unknown group. */
+void ql_profile_enable(int on);
+int ql_profile_read(int kind, double* total_ms, int64_t* count);
+uint64_t ql_launch_count(void);
+
 /* Static description of a status code. */
 const char* ql_status_string(ql_status s);
 

@@ -52,7 +52,14 @@ _SIGS = {
     "ql_status_string": ([I32], ctypes.c_char_p),
     "ql_nf4_codebook": ([ctypes.POINTER(ctypes.c_float)], None),
     "ql_set_wait_timeout_ns": ([ctypes.c_uint64], None),
+    "ql_profile_enable": ([ctypes.c_int], None),
+    "ql_profile_read": ([ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)], ctypes.c_int),
+    "ql_launch_count": ([], ctypes.c_uint64),
 }
+
+# kernel groups of ql_profile_read
+PROFILE_GROUPS = ["nf4", "dq", "int8", "dequant", "fwd_prep", "fwd_xa", "fwd_main", "bwd_prep",
+                  "bwd_dyb", "bwd_db", "bwd_da", "bwd_dx", "fwd_small"]
 
 
 def lib() -> ctypes.CDLL:
@@ -206,7 +213,8 @@ def dequantize(qw: QuantWeight) -> torch.Tensor:
 
 
 def linear_fwd(qw: QuantWeight, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
-               alpha: float, save_T: bool = True, Y: torch.Tensor | None = None):
+               alpha: float, save_T: bool = True, Y: torch.Tensor | None = None,
+               T: torch.Tensor | None = None):
     """Y = X W'^T + (alpha/r) (X A^T) B^T. Returns (Y, T) with T = bf16(X A^T) or None."""
     for t, nm in ((X, "X"), (A, "A"), (B, "B")):
         _need(t, torch.bfloat16, nm)
@@ -215,7 +223,8 @@ def linear_fwd(qw: QuantWeight, X: torch.Tensor, A: torch.Tensor, B: torch.Tenso
     dev = X.device
     if Y is None:
         Y = torch.empty((M, qw.N), dtype=torch.bfloat16, device=dev)
-    T = torch.empty((M, r), dtype=torch.bfloat16, device=dev) if save_T else None
+    if T is None and save_T:
+        T = torch.empty((M, r), dtype=torch.bfloat16, device=dev)
     ws = workspace(workspace_bytes(QL_OP_FWD, M, qw.N, K, r), dev)
     _check(lib().qlora_linear_fwd(ctypes.byref(qw.desc), _ptr(X), M, _ptr(A), _ptr(B), r,
                                   float(alpha), _ptr(Y), _ptr(T), _ptr(ws), ws.numel(),
@@ -223,16 +232,19 @@ def linear_fwd(qw: QuantWeight, X: torch.Tensor, A: torch.Tensor, B: torch.Tenso
     return Y, T
 
 
-def linear_bwd(qw: QuantWeight, X, dY, A, B, T, alpha: float):
+def linear_bwd(qw: QuantWeight, X, dY, A, B, T, alpha: float, dX=None, dA=None, dB=None):
     """Returns (dX bf16 [M,K], dA fp32 [r,K], dB fp32 [N,r])."""
     for t, nm in ((X, "X"), (dY, "dY"), (A, "A"), (B, "B"), (T, "T")):
         _need(t, torch.bfloat16, nm)
     M, K = X.shape
     r = A.shape[0]
     dev = X.device
-    dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
-    dA = torch.empty((r, K), dtype=torch.float32, device=dev)
-    dB = torch.empty((qw.N, r), dtype=torch.float32, device=dev)
+    if dX is None:
+        dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    if dA is None:
+        dA = torch.empty((r, K), dtype=torch.float32, device=dev)
+    if dB is None:
+        dB = torch.empty((qw.N, r), dtype=torch.float32, device=dev)
     ws = workspace(workspace_bytes(QL_OP_BWD, M, qw.N, K, r), dev)
     _check(lib().qlora_linear_bwd(ctypes.byref(qw.desc), _ptr(X), _ptr(dY), M, _ptr(A), _ptr(B),
                                   _ptr(T), r, float(alpha), _ptr(dX), _ptr(dA), _ptr(dB),
@@ -243,6 +255,22 @@ def linear_bwd(qw: QuantWeight, X, dY, A, B, T, alpha: float):
 def device_status(device: torch.device | None = None) -> int:
     """Synchronise and return (and clear) the library's sticky device flag."""
     return int(lib().ql_get_device_status(_stream(device)))
+
+
+def profile_enable(on: bool = True):
+    lib().ql_profile_enable(1 if on else 0)
+
+
+def profile_read(group: str):
+    """(total milliseconds, launches) of one kernel group since the last read."""
+    ms = ctypes.c_double(0.0)
+    cnt = ctypes.c_int64(0)
+    lib().ql_profile_read(PROFILE_GROUPS.index(group), ctypes.byref(ms), ctypes.byref(cnt))
+    return ms.value, cnt.value
+
+
+def launch_count() -> int:
+    return int(lib().ql_launch_count())
 
 
 def nf4_codebook() -> list[float]:

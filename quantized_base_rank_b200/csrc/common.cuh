@@ -27,6 +27,26 @@ int num_sms();                          // SM count of the current device
 __host__ __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
 __host__ __device__ __forceinline__ int64_t imax64(int64_t a, int64_t b) { return a > b ? a : b; }
 
+// Kernel groups that can be timed with CUDA events (ql_profile_enable / ql_profile_read).
+enum ProfKind : int {
+  PK_NF4 = 0, PK_DQ = 1, PK_INT8 = 2, PK_DEQ = 3, PK_FWD_PREP = 4, PK_FWD_T = 5, PK_FWD_MAIN = 6,
+  PK_BWD_PREP = 7, PK_BWD_U = 8, PK_BWD_DB = 9, PK_BWD_DA = 10, PK_BWD_DX = 11, PK_FWD_SMALL = 12,
+  PK_COUNT = 13
+};
+
+// Counts the kernels a scope launches and, when profiling is on, brackets them with a
+// pair of CUDA events recorded on the launch stream.
+class ProfScope {
+ public:
+  ProfScope(int kind, cudaStream_t st, int nlaunch);
+  ~ProfScope();
+ private:
+  int kind_;
+  cudaStream_t st_;
+  bool on_;
+  cudaEvent_t a_;
+};
+
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
 inline bool aligned(const void* p, uintptr_t a) {

@@ -203,8 +203,11 @@ ql_status qlora_linear_fwd(const ql_weight* w, const ql_bf16* X, int64_t M, cons
   uint16_t* P = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + L.off[0]);
   uint16_t* Bp = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + L.off[1]);
 
-  pad_cols_kernel<<<small_grid(N * rp), 256, 0, st>>>(B, N, r, rp, Bp);
-  QL_CHECK_LAUNCH();
+  {
+    ProfScope prof(PK_FWD_PREP, st, 1);
+    pad_cols_kernel<<<small_grid(N * rp), 256, 0, st>>>(B, N, r, rp, Bp);
+    QL_CHECK_LAUNCH();
+  }
 
   CUtensorMap mX, mA, mP, mBp, none;
   memset(&none, 0, sizeof(none));
@@ -217,15 +220,19 @@ ql_status qlora_linear_fwd(const ql_weight* w, const ql_bf16* X, int64_t M, cons
   t.R = M; t.Cn = rp; t.Kc = K; t.n_ext = 0; t.r = r;
   t.out = T_save; t.ld_out = r; t.out2 = P; t.ld_out2 = rp; t.scale = s;
   ql_status e;
+  {
+  ProfScope prof(PK_FWD_T, st, 1);
   if (rp == 64) e = launch_gemm<64, 0, false, BSrc::TMA, false, EPI_LORA_T>(mX, mA, none, none, t, st);
   else if (rp == 128) e = launch_gemm<128, 0, false, BSrc::TMA, false, EPI_LORA_T>(mX, mA, none, none, t, st);
   else e = launch_gemm<256, 0, false, BSrc::TMA, false, EPI_LORA_T>(mX, mA, none, none, t, st);
+  }
   if (e != QL_OK) return e;
 
   // Y = X W'^T + P Bp^T
   GemmArgs y = base_args(w);
   y.R = M; y.Cn = N; y.Kc = K; y.n_ext = rp / 64; y.r = r;
   y.out = Y; y.ld_out = N; y.scale = 1.0f;
+  ProfScope prof(PK_FWD_MAIN, st, 1);
   if (w->fmt == QL_FMT_NF4_DQ)
     return launch_gemm<256, 8, false, BSrc::NF4, false, EPI_BF16>(mX, none, mP, mBp, y, st);
   return launch_gemm<256, 8, false, BSrc::INT8, false, EPI_BF16>(mX, none, mP, mBp, y, st);
@@ -255,12 +262,15 @@ ql_status qlora_linear_bwd(const ql_weight* w, const ql_bf16* X, const ql_bf16* 
   uint16_t* At = reinterpret_cast<uint16_t*>(wsb + L.off[2]);
   uint16_t* Tp = reinterpret_cast<uint16_t*>(wsb + L.off[3]);
 
-  transpose_kernel<<<small_grid(N * r), 256, 0, st>>>(B, N, r, Bt);
-  QL_CHECK_LAUNCH();
-  transpose_pad_kernel<<<small_grid(K * rp), 256, 0, st>>>(A, r, K, rp, At);
-  QL_CHECK_LAUNCH();
-  pad_cols_kernel<<<small_grid(M * rp), 256, 0, st>>>(T_saved, M, r, rp, Tp);
-  QL_CHECK_LAUNCH();
+  {
+    ProfScope prof(PK_BWD_PREP, st, 3);
+    transpose_kernel<<<small_grid(N * r), 256, 0, st>>>(B, N, r, Bt);
+    QL_CHECK_LAUNCH();
+    transpose_pad_kernel<<<small_grid(K * rp), 256, 0, st>>>(A, r, K, rp, At);
+    QL_CHECK_LAUNCH();
+    pad_cols_kernel<<<small_grid(M * rp), 256, 0, st>>>(T_saved, M, r, rp, Tp);
+    QL_CHECK_LAUNCH();
+  }
 
   CUtensorMap mdY_k, mBt, mQ_k, mAt, mdY_mn, mTp_mn, mX_mn, mQ_mn, none;
   memset(&none, 0, sizeof(none));
@@ -274,30 +284,40 @@ ql_status qlora_linear_bwd(const ql_weight* w, const ql_bf16* X, const ql_bf16* 
   // Q = bf16(s dY B)
   GemmArgs u = base_args(nullptr);
   u.R = M; u.Cn = rp; u.Kc = N; u.r = r; u.out = Q; u.ld_out = rp; u.scale = s;
+  {
+  ProfScope prof(PK_BWD_U, st, 1);
   if (rp == 64) e = launch_gemm<64, 0, false, BSrc::TMA, false, EPI_LORA_Q>(mdY_k, mBt, none, none, u, st);
   else if (rp == 128) e = launch_gemm<128, 0, false, BSrc::TMA, false, EPI_LORA_Q>(mdY_k, mBt, none, none, u, st);
   else e = launch_gemm<256, 0, false, BSrc::TMA, false, EPI_LORA_Q>(mdY_k, mBt, none, none, u, st);
+  }
   if (e != QL_OK) return e;
 
   // dB = s dY^T T     (rows n, columns j, contraction over tokens)
   GemmArgs b = base_args(nullptr);
   b.R = N; b.Cn = rp; b.Kc = M; b.r = r; b.out = dB; b.ld_out = r; b.scale = s;
+  {
+  ProfScope prof(PK_BWD_DB, st, 1);
   if (rp == 64) e = launch_gemm<64, 0, true, BSrc::TMA, true, EPI_DB>(mdY_mn, mTp_mn, none, none, b, st);
   else if (rp == 128) e = launch_gemm<128, 0, true, BSrc::TMA, true, EPI_DB>(mdY_mn, mTp_mn, none, none, b, st);
   else e = launch_gemm<256, 0, true, BSrc::TMA, true, EPI_DB>(mdY_mn, mTp_mn, none, none, b, st);
+  }
   if (e != QL_OK) return e;
 
   // dA = Q^T X        (computed as dA^T: rows k, columns j)
   GemmArgs a = base_args(nullptr);
   a.R = K; a.Cn = rp; a.Kc = M; a.r = r; a.out = dA; a.ld_out = K; a.scale = 1.0f;
+  {
+  ProfScope prof(PK_BWD_DA, st, 1);
   if (rp == 64) e = launch_gemm<64, 0, true, BSrc::TMA, true, EPI_DA>(mX_mn, mQ_mn, none, none, a, st);
   else if (rp == 128) e = launch_gemm<128, 0, true, BSrc::TMA, true, EPI_DA>(mX_mn, mQ_mn, none, none, a, st);
   else e = launch_gemm<256, 0, true, BSrc::TMA, true, EPI_DA>(mX_mn, mQ_mn, none, none, a, st);
+  }
   if (e != QL_OK) return e;
 
   // dX = dY W' + Q A^T-padded
   GemmArgs x = base_args(w);
   x.R = M; x.Cn = K; x.Kc = N; x.n_ext = rp / 64; x.r = r; x.out = dX; x.ld_out = K; x.scale = 1.0f;
+  ProfScope prof(PK_BWD_DX, st, 1);
   if (w->fmt == QL_FMT_NF4_DQ)
     return launch_gemm<256, 8, false, BSrc::NF4, true, EPI_BF16>(mdY_k, none, mQ_k, mAt, x, st);
   return launch_gemm<256, 8, false, BSrc::INT8, true, EPI_BF16>(mdY_k, none, mQ_k, mAt, x, st);

@@ -338,6 +338,7 @@ ql_status nf4_quantize(const ql_bf16* W, int64_t n, uint8_t* codes, float* absma
   if (!aligned(W, 2) || !aligned(codes, 4) || !aligned(absmax, 4)) return QL_ERR_INVALID_ARG;
   const int vec = aligned(W, 16) && aligned(codes, 16);
   const int64_t nb = (n + kBlock - 1) / kBlock;
+  ProfScope prof(PK_NF4, as_stream(stream), 1);
   nf4_quantize_kernel<<<grid_for(nb, 256), 256, 0, as_stream(stream)>>>(
       W, n, codes, absmax, nf4_tables(), vec, device_flag_ptr());
   QL_CHECK_LAUNCH();
@@ -351,6 +352,7 @@ ql_status int8_quantize(const ql_bf16* W, int64_t n, int8_t* codes, float* absma
   if (!aligned(W, 2) || !aligned(absmax, 4)) return QL_ERR_INVALID_ARG;
   const int vec = aligned(W, 16) && aligned(codes, 16);
   const int64_t nb = (n + kBlock - 1) / kBlock;
+  ProfScope prof(PK_INT8, as_stream(stream), 1);
   int8_quantize_kernel<<<grid_for(nb, 256), 256, 0, as_stream(stream)>>>(
       W, n, codes, absmax, vec, device_flag_ptr());
   QL_CHECK_LAUNCH();
@@ -366,6 +368,7 @@ ql_status dq_quantize(const float* absmax, int64_t nblocks, int8_t* qabsmax, flo
   if (ws_bytes < ql_workspace_bytes(QL_OP_DQ, 0, 0, 0, 0)) return QL_ERR_WORKSPACE;
   cudaStream_t st = as_stream(stream);
   unsigned long long* bins = static_cast<unsigned long long*>(ws);
+  ProfScope prof(PK_DQ, st, 3);
   if (cudaMemsetAsync(bins, 0, kSumBins * sizeof(unsigned long long), st) != cudaSuccess)
     return QL_ERR_CUDA;
   dq_sum_kernel<<<grid_for(nblocks, 256), 256, 0, st>>>(absmax, nblocks, bins, device_flag_ptr());
@@ -383,6 +386,7 @@ ql_status ql_dequantize(const ql_weight* w, ql_bf16* Wout, void* stream) {
   const int64_t n = w->N * w->K;
   const int64_t nb = (n + kBlock - 1) / kBlock;
   cudaStream_t st = as_stream(stream);
+  ProfScope prof(PK_DEQ, st, 1);
   if (w->fmt == QL_FMT_NF4_DQ) {
     if (!w->qabsmax || !w->group_scale || !w->mean) return QL_ERR_INVALID_ARG;
     dequant_nf4_kernel<<<grid_for(nb, 256), 256, 0, st>>>(

@@ -1,7 +1,9 @@
 // Host-side runtime pieces: the NF4 tables, the sticky device flag, status strings.
 #include <math.h>
 
+#include <atomic>
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 
@@ -70,9 +72,75 @@ int num_sms() {
   return cache[dev];
 }
 
+// ---- profiling events and launch counting -------------------------------------------
+
+static std::atomic<int> g_prof_on{0};
+static std::atomic<uint64_t> g_launches{0};
+static std::mutex g_prof_mu;
+static std::vector<std::pair<cudaEvent_t, cudaEvent_t>> g_prof[PK_COUNT];
+static std::vector<cudaEvent_t> g_ev_pool;
+
+static cudaEvent_t take_event() {
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  if (!g_ev_pool.empty()) {
+    cudaEvent_t e = g_ev_pool.back();
+    g_ev_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+ProfScope::ProfScope(int kind, cudaStream_t st, int nlaunch)
+    : kind_(kind), st_(st), on_(g_prof_on.load() != 0), a_(nullptr) {
+  g_launches += (uint64_t)nlaunch;
+  if (on_) {
+    a_ = take_event();
+    cudaEventRecord(a_, st_);
+  }
+}
+
+ProfScope::~ProfScope() {
+  if (!on_) return;
+  cudaEvent_t b = take_event();
+  cudaEventRecord(b, st_);
+  std::lock_guard<std::mutex> lock(g_prof_mu);
+  g_prof[kind_].push_back({a_, b});
+}
+
 }  // namespace qlb
 
 extern "C" {
+
+void ql_profile_enable(int on) { qlb::g_prof_on.store(on ? 1 : 0); }
+
+uint64_t ql_launch_count(void) { return qlb::g_launches.load(); }
+
+int ql_profile_read(int kind, double* total_ms, int64_t* count) {
+  if (kind < 0 || kind >= qlb::PK_COUNT) return -1;
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> v;
+  {
+    std::lock_guard<std::mutex> lock(qlb::g_prof_mu);
+    v.swap(qlb::g_prof[kind]);
+  }
+  double tot = 0.0;
+  for (auto& p : v) {
+    float ms = 0.0f;
+    if (cudaEventSynchronize(p.second) == cudaSuccess && cudaEventElapsedTime(&ms, p.first, p.second) == cudaSuccess)
+      tot += ms;
+  }
+  {
+    std::lock_guard<std::mutex> lock(qlb::g_prof_mu);
+    for (auto& p : v) {
+      qlb::g_ev_pool.push_back(p.first);
+      qlb::g_ev_pool.push_back(p.second);
+    }
+  }
+  if (total_ms) *total_ms = tot;
+  if (count) *count = (int64_t)v.size();
+  return 0;
+}
 
 ql_status ql_get_device_status(void* stream) {
   if (cudaStreamSynchronize(qlb::as_stream(stream)) != cudaSuccess) return QL_ERR_CUDA;
