@@ -1,20 +1,26 @@
-// Persistent warp-specialised tcgen05 GEMM with an on-the-fly NF4 / int8 decoding
-// producer for the weight operand and a K-extension for the unmerged LoRA term.
+// Persistent warp-specialised tcgen05 GEMMs for the quantised linear layer.
 //
 //   C[R, Cn] = sum_k Aop[R, k] * Bop[Cn, k]  (+ sum_e Aext[R, e] * Bext[Cn, e])
 //
-// Tiles: 128 rows x BN columns, contraction in chunks of 64 (one 128-byte swizzled
-// smem row per operand row). Roles (warp index):
-//   0..3  epilogue: TMEM -> registers -> global (one TMEM lane quarter each)
-//   4     TMA producer for Aop (and Bop when it is plain bf16), and the extension
-//   5     MMA issuer (one elected thread), also owns the TMEM allocation
-//   6..   NP decode warps: weight codes -> bf16 rows written straight into the
-//         swizzled UMMA layout of the stage's B tile (QLoRA page, "1. NF4" and
-//         "2. Double Quantization": w' = q[code] * a', a' rebuilt from the 8-bit constant)
-// Accumulators are double-buffered in TMEM so the epilogue of one tile overlaps the
-// main loop of the next. Every wait is bounded; a wait that gives up raises the CTA's
-// abort word, every role then leaves its loop, and the kernel reports QL_ERR_TIMEOUT
-// through the device flag after freeing its TMEM.
+// Tiles are 128 rows x BN columns; the contraction runs in chunks of 64 (one 128-byte
+// swizzled smem row per operand row). Accumulators are double-buffered in TMEM so the
+// epilogue of one tile overlaps the main loop of the next.
+//
+// qgemm_tma_kernel — both operands by TMA (the adapter-sized GEMMs). Warps:
+//   0..3 epilogue, 4 TMA, 5 MMA issuer (also owns TMEM).
+// qgemm_dec_kernel — the weight operand is decoded from its quantised form (QLoRA page,
+// "1. NF4" and "2. Double Quantization": w' = q[code] * a'). Warps:
+//   0..3 epilogue, 4 TMA for the activation tiles (and the adapter extension's left
+//   factor), 5 MMA issuer, 6 TMA for the weight codes + rebuilt block scales,
+//   7..14 decode: codes in smem -> bf16 rows written straight into the 128-byte-swizzled
+//   UMMA layout of the weight tile (they also issue the TMA of the extension's right
+//   factor, so each ring keeps a single producer). Nothing in the decode warps reads
+//   global memory, so they never wait on it.
+// The unmerged LoRA term enters as extra contraction chunks of the same accumulator.
+//
+// Every wait is bounded; a wait that gives up raises the CTA's abort word, every role then
+// leaves its loop, copies and MMAs in flight are drained (bounded), TMEM is freed, and the
+// kernel reports QL_ERR_TIMEOUT through the device flag.
 #pragma once
 
 #include "common.cuh"
@@ -22,21 +28,14 @@
 
 namespace qlb {
 
-enum class BSrc : int { TMA = 0, NF4 = 1, INT8 = 2 };
+enum class BSrc : int { NF4 = 1, INT8 = 2 };
 enum Epi : int { EPI_BF16 = 0, EPI_LORA_T = 1, EPI_LORA_Q = 2, EPI_DA = 3, EPI_DB = 4 };
 
 struct GemmArgs {
   int64_t R, Cn, Kc;     // rows, columns, main contraction length
   int32_t n_ext;         // number of 64-wide extension chunks
   int32_t r;             // adapter rank (epilogue masks)
-  // weight operand (decode modes): W [Nw, Kw]
-  const uint8_t* codes;
-  const int8_t* qabsmax;
-  const float* gscale;
-  const float* mean;
-  const float* absmax;
-  int64_t Nw, Kw;
-  float q[16];
+  float q[16];           // NF4 grid
   // epilogue
   void* out;  int64_t ld_out;
   void* out2; int64_t ld_out2;
@@ -45,104 +44,74 @@ struct GemmArgs {
   int* flag;
 };
 
-template <int BN>
-struct GemmCfg {
-  static constexpr int kABytes = 128 * 64 * 2;
-  static constexpr int kBBytes = BN * 128;
-  static constexpr int kStages = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
-  static constexpr int kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;
-  static constexpr size_t kSmem = (size_t)kStages * (kABytes + kBBytes) + 2048;
-};
-
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t r;
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
   return r;
 }
 
-// 16-entry bf16 table lookup of 4 nibbles (bits 0..15 of sel16), giving two packed
-// bf16x2 words (elements 0,1 and 2,3). L/H hold the low/high bytes of entries
-// 0..15 (entry c in byte c%4 of word c/4).
-__device__ __forceinline__ void lut4(uint32_t sel16, const uint32_t (&L)[4],
-                                     const uint32_t (&H)[4], uint32_t& w01, uint32_t& w23) {
-  const uint32_t s7 = sel16 & 0x7777u;
-  const uint32_t mask = prmt(sel16 << 4, sel16, 0xD9C8u);   // 0xFF where the code is >= 8
-  const uint32_t lo = (prmt(L[2], L[3], s7) & mask) | (prmt(L[0], L[1], s7) & ~mask);
-  const uint32_t hi = (prmt(H[2], H[3], s7) & mask) | (prmt(H[0], H[1], s7) & ~mask);
-  w01 = prmt(lo, hi, 0x5140u);
-  w23 = prmt(lo, hi, 0x7362u);
+// ---------------------------------------------------------------------------------
+// NF4 decode. For a block with rebuilt scale a', the eight non-negative-index entries
+// M[i] = bf16(fp32(q_{8+i} * a')) are formed with 8 multiplies; since the grid is
+// symmetric (q_{7-i} = -q_{8+i} exactly) and rounding is symmetric, code c decodes to
+// M[c-8] for c >= 8 and to -M[7-c] for c < 8. L/H hold the low/high bytes of M[0..7].
+// ---------------------------------------------------------------------------------
+__device__ __forceinline__ void nf4_table(const float (&q)[16], float ar, uint32_t (&L)[2],
+                                          uint32_t (&H)[2]) {
+  const uint32_t P01 = pack_bf16x2(__fmul_rn(q[8], ar), __fmul_rn(q[9], ar));
+  const uint32_t P23 = pack_bf16x2(__fmul_rn(q[10], ar), __fmul_rn(q[11], ar));
+  const uint32_t P45 = pack_bf16x2(__fmul_rn(q[12], ar), __fmul_rn(q[13], ar));
+  const uint32_t P67 = pack_bf16x2(__fmul_rn(q[14], ar), __fmul_rn(q[15], ar));
+  L[0] = prmt(P01, P23, 0x6420u);
+  H[0] = prmt(P01, P23, 0x7531u);
+  L[1] = prmt(P45, P67, 0x6420u);
+  H[1] = prmt(P45, P67, 0x7531u);
 }
 
-// Decode one block of 64 weight elements (row n of W, block kb of that row) into one
-// 128-byte swizzled smem row (chunk c goes to position c ^ key). Rows past the end
-// of W are written as zeros.
-template <BSrc BS>
-__device__ __forceinline__ void decode_block(const GemmArgs& a, float mean0, int64_t n, int64_t kb,
-                                             uint8_t* dst, uint32_t key) {
-  uint4* d = reinterpret_cast<uint4*>(dst);
-  if (n >= a.Nw || kb >= (a.Kw >> 6)) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) d[c] = make_uint4(0u, 0u, 0u, 0u);
-    return;
-  }
-  const int64_t blk = n * (a.Kw >> 6) + kb;
-  if constexpr (BS == BSrc::NF4) {
-    const uint4* src = reinterpret_cast<const uint4*>(a.codes + blk * 32);
-    const uint4 c0 = __ldg(src), c1 = __ldg(src + 1);
-    // a' = fp32(fp32(c8 * s_g) + mean)
-    const float ar = __fadd_rn(__fmul_rn((float)__ldg(a.qabsmax + blk), __ldg(a.gscale + (blk >> 8))),
-                               mean0);
-    // entries 8..15: bf16(fp32(q_c * a')); entries 0..7 are their exact negatives
-    const uint32_t P01 = pack_bf16x2(__fmul_rn(a.q[8], ar), __fmul_rn(a.q[9], ar));
-    const uint32_t P23 = pack_bf16x2(__fmul_rn(a.q[10], ar), __fmul_rn(a.q[11], ar));
-    const uint32_t P45 = pack_bf16x2(__fmul_rn(a.q[12], ar), __fmul_rn(a.q[13], ar));
-    const uint32_t P67 = pack_bf16x2(__fmul_rn(a.q[14], ar), __fmul_rn(a.q[15], ar));
-    uint32_t L[4], H[4];
-    L[2] = prmt(P01, P23, 0x6420u);
-    H[2] = prmt(P01, P23, 0x7531u);
-    L[3] = prmt(P45, P67, 0x6420u);
-    H[3] = prmt(P45, P67, 0x7531u);
-    L[0] = prmt(L[3], 0u, 0x0123u);
-    H[0] = prmt(H[3], 0u, 0x0123u) ^ 0x80808080u;
-    L[1] = prmt(L[2], 0u, 0x0123u);
-    H[1] = prmt(H[2], 0u, 0x0123u) ^ 0x80808080u;
-    const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      uint4 o;
-      lut4(words[c] & 0xFFFFu, L, H, o.x, o.y);
-      lut4(words[c] >> 16, L, H, o.z, o.w);
-      d[c ^ key] = o;
-    }
-  } else {
-    // int8: w' = bf16(fp32(c * fp32(a/127))); c recovered exactly from a magic float
-    const float sc = __fdiv_rn(__ldg(a.absmax + blk), 127.0f);
-    const uint4* src = reinterpret_cast<const uint4*>(a.codes + blk * 64);
-    const uint4 q0 = __ldg(src), q1 = __ldg(src + 1), q2 = __ldg(src + 2), q3 = __ldg(src + 3);
-    const uint32_t words[16] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w,
-                                q2.x, q2.y, q2.z, q2.w, q3.x, q3.y, q3.z, q3.w};
-    const uint32_t kMagic = 0x4B000000u;   // 2^23: low byte of the mantissa holds c + 128
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      uint32_t o[4];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t wv = words[2 * c + h] ^ 0x80808080u;
-        float f[4];
-        f[0] = __uint_as_float(prmt(wv, kMagic, 0x7540u));
-        f[1] = __uint_as_float(prmt(wv, kMagic, 0x7541u));
-        f[2] = __uint_as_float(prmt(wv, kMagic, 0x7542u));
-        f[3] = __uint_as_float(prmt(wv, kMagic, 0x7543u));
-#pragma unroll
-        for (int i = 0; i < 4; ++i) f[i] = __fmul_rn(__fsub_rn(f[i], 8388736.0f), sc);
-        o[2 * h] = pack_bf16x2(f[0], f[1]);
-        o[2 * h + 1] = pack_bf16x2(f[2], f[3]);
-      }
-      d[c ^ key] = make_uint4(o[0], o[1], o[2], o[3]);
-    }
-  }
+// 8 codes (one 32-bit word, element 0 in the low nibble) -> 8 bf16 (four bf16x2 words).
+__device__ __forceinline__ uint4 nf4_decode8(uint32_t w, const uint32_t (&L)[2], const uint32_t (&H)[2]) {
+  const uint32_t m8 = w & 0x88888888u;                     // bit 3 of every code
+  const uint32_t f = m8 - (m8 >> 3);                       // 7 where the code is >= 8
+  const uint32_t idx = (w ^ f ^ 0x77777777u) & 0x77777777u;  // c-8 (c >= 8) or 7-c (c < 8)
+  const uint32_t m84 = m8 << 4;
+  uint4 o;
+  uint32_t s = prmt(m84, m8, 0xD9C8u);                     // 0xFF in byte i where code i >= 8
+  uint32_t lo = prmt(L[0], L[1], idx);
+  uint32_t hi = prmt(H[0], H[1], idx) ^ (~s & 0x80808080u);  // negate the codes below 8
+  o.x = prmt(lo, hi, 0x5140u);
+  o.y = prmt(lo, hi, 0x7362u);
+  s = prmt(m84, m8, 0xFBEAu);
+  const uint32_t idxh = idx >> 16;
+  lo = prmt(L[0], L[1], idxh);
+  hi = prmt(H[0], H[1], idxh) ^ (~s & 0x80808080u);
+  o.z = prmt(lo, hi, 0x5140u);
+  o.w = prmt(lo, hi, 0x7362u);
+  return o;
 }
 
+// int8: w' = bf16(fp32(c * sc)); c is recovered exactly from a magic float (2^23 + c + 128).
+__device__ __forceinline__ uint4 int8_decode8(uint32_t w0, uint32_t w1, float sc) {
+  uint32_t o[4];
+  const uint32_t kMagic = 0x4B000000u;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t wv = (h ? w1 : w0) ^ 0x80808080u;
+    float f[4];
+    f[0] = __uint_as_float(prmt(wv, kMagic, 0x7540u));
+    f[1] = __uint_as_float(prmt(wv, kMagic, 0x7541u));
+    f[2] = __uint_as_float(prmt(wv, kMagic, 0x7542u));
+    f[3] = __uint_as_float(prmt(wv, kMagic, 0x7543u));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) f[i] = __fmul_rn(__fsub_rn(f[i], 8388736.0f), sc);
+    o[2 * h] = pack_bf16x2(f[0], f[1]);
+    o[2 * h + 1] = pack_bf16x2(f[2], f[3]);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// ---------------------------------------------------------------------------------
+// Epilogues
+// ---------------------------------------------------------------------------------
 template <int EPI>
 __device__ __forceinline__ void epilogue_store(const GemmArgs& a, int64_t row, int64_t col,
                                                const uint32_t (&v)[32]) {
@@ -192,209 +161,403 @@ __device__ __forceinline__ void epilogue_store(const GemmArgs& a, int64_t row, i
   }
 }
 
-template <int BN, int NP, bool A_MN, BSrc BS, bool B_MN, int EPI>
-__global__ void __launch_bounds__((6 + NP) * 32, 1)
-qgemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-             const __grid_constant__ CUtensorMap tmAe, const __grid_constant__ CUtensorMap tmBe,
-             const GemmArgs args) {
-  using Cfg = GemmCfg<BN>;
-  constexpr int S = Cfg::kStages;
-  constexpr bool kDecode = BS != BSrc::TMA;
-  static_assert(!kDecode || NP * 32 == BN, "one decode thread per B row");
+// Epilogue role shared by both kernels: warps 0..3, TMEM lanes 32*warp ..
+template <int BN, int EPI>
+__device__ __forceinline__ void run_epilogue(const GemmArgs& args, uint32_t tmem_base, uint32_t acc_full,
+                                             uint32_t acc_empty, int64_t tiles, int64_t n_tiles,
+                                             volatile int* abort_word) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t tcount = 0;
+  for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++tcount) {
+    const uint32_t acc = tcount & 1, aph = (tcount >> 1) & 1;
+    const bool okw = mbar_wait(acc_full + 8 * acc, aph, args.timeout_ns, abort_word);
+    if (!__all_sync(0xFFFFFFFFu, okw)) break;
+    tc_fence_after();
+    const int64_t r0 = (t / n_tiles) * 128, c0 = (t % n_tiles) * BN;
+    const int64_t row = r0 + warp * 32 + lane;
+#pragma unroll 1
+    for (int cc = 0; cc < BN; cc += 32) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(warp * 32) << 16) + acc * BN + cc, v);
+      if (c0 + cc < args.Cn) epilogue_store<EPI>(args, row, c0 + cc, v);
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(acc_empty + 8 * acc);
+  }
+}
 
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < 200000000ull) {}
+}
+
+// =================================================================================
+// Both operands by TMA
+// =================================================================================
+template <int BN>
+struct TmaCfg {
+  static constexpr int kABytes = 128 * 64 * 2;
+  static constexpr int kBBytes = BN * 128;
+  static constexpr int kStages = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
+  static constexpr int kTmemCols = 2 * BN;
+  static constexpr size_t kSmem = (size_t)kStages * (kABytes + kBBytes) + 2048;
+};
+
+template <int BN, bool A_MN, bool B_MN, int EPI>
+__global__ void __launch_bounds__(192, 1)
+qgemm_tma_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const GemmArgs args) {
+  using Cfg = TmaCfg<BN>;
+  constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + S * Cfg::kABytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sB + S * Cfg::kBBytes);
-  const uint32_t full_a = smem_u32(bars);
-  const uint32_t full_b = full_a + 8 * S;
-  const uint32_t empty = full_a + 16 * S;
-  const uint32_t acc_full = full_a + 24 * S;
+  const uint32_t full = smem_u32(bars);
+  const uint32_t empty = full + 8 * S;
+  const uint32_t acc_full = full + 16 * S;
   const uint32_t acc_empty = acc_full + 16;
   const uint32_t drain = acc_full + 32;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 3 * S + 5);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
   volatile int* abort_word = reinterpret_cast<volatile int*>(tmem_holder + 1);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(full_a + 8 * s, 1);
-      mbar_init(full_b + 8 * s, NP > 0 ? NP : 1);
-      mbar_init(empty + 8 * s, 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(acc_full + 8 * i, 1);
-      mbar_init(acc_empty + 8 * i, 4);
-    }
+    for (int s = 0; s < S; ++s) { mbar_init(full + 8 * s, 1); mbar_init(empty + 8 * s, 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(acc_full + 8 * i, 1); mbar_init(acc_empty + 8 * i, 4); }
     mbar_init(drain, 1);
     *abort_word = 0;
     fence_mbar_init();
   }
-  if (warp == 4 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    if (BS == BSrc::TMA) tma_prefetch_desc(&tmB);
-    if (args.n_ext) { tma_prefetch_desc(&tmAe); tma_prefetch_desc(&tmBe); }
-  }
+  if (warp == 4 && lane == 0) { tma_prefetch_desc(&tmA); tma_prefetch_desc(&tmB); }
   if (warp == 5) tmem_alloc(smem_u32(tmem_holder), Cfg::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  const int64_t m_tiles = (args.R + 127) / 128;
   const int64_t n_tiles = (args.Cn + BN - 1) / BN;
-  const int64_t tiles = m_tiles * n_tiles;
-  const int kc_main = (int)((args.Kc + 63) / 64);
-  const int kc_total = kc_main + args.n_ext;
+  const int64_t tiles = ((args.R + 127) / 128) * n_tiles;
+  const int kc_total = (int)((args.Kc + 63) / 64);
   const uint64_t lim = args.timeout_ns;
 
   if (warp < 4) {
-    // ---------------- epilogue ----------------
-    uint32_t tcount = 0;
-    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++tcount) {
-      const uint32_t acc = tcount & 1, aph = (tcount >> 1) & 1;
-      const bool okw = mbar_wait(acc_full + 8 * acc, aph, lim, abort_word);
-      if (!__all_sync(0xFFFFFFFFu, okw)) break;
-      tc_fence_after();
-      const int64_t r0 = (t / n_tiles) * 128, c0 = (t % n_tiles) * BN;
-      const int64_t row = r0 + warp * 32 + lane;
-#pragma unroll 1
-      for (int cc = 0; cc < BN; cc += 32) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(warp * 32) << 16) + acc * BN + cc, v);
-        if (c0 + cc < args.Cn) epilogue_store<EPI>(args, row, c0 + cc, v);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty + 8 * acc);
-    }
-  } else if (warp == 4) {
-    // ---------------- TMA producer ----------------
-    if (lane == 0) {
-      uint32_t g = 0;
-      bool ok = true;
-      for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-        const int32_t r0 = (int32_t)((t / n_tiles) * 128), c0 = (int32_t)((t % n_tiles) * BN);
-        for (int kc = 0; kc < kc_total; ++kc, ++g) {
-          const uint32_t s = g % S, ph = (g / S) & 1;
-          if (!mbar_wait(empty + 8 * s, ph ^ 1, lim, abort_word)) { ok = false; break; }
-          const uint32_t fa = full_a + 8 * s;
-          const uint32_t dA = smem_u32(sA + s * Cfg::kABytes);
-          const uint32_t dB = smem_u32(sB + s * Cfg::kBBytes);
-          if (kc < kc_main) {
-            mbar_arrive_expect_tx(fa, Cfg::kABytes + (kDecode ? 0 : Cfg::kBBytes));
-            if (!A_MN) {
-              tma_load_2d(dA, &tmA, fa, kc * 64, r0);
-            } else {
-              tma_load_2d(dA, &tmA, fa, r0, kc * 64);
-              tma_load_2d(dA + 8192, &tmA, fa, r0 + 64, kc * 64);
-            }
-            if (!kDecode) {
-              if (!B_MN) {
-                tma_load_2d(dB, &tmB, fa, kc * 64, c0);
-              } else {
-#pragma unroll
-                for (int i = 0; i < BN / 64; ++i) tma_load_2d(dB + i * 8192, &tmB, fa, c0 + 64 * i, kc * 64);
-              }
-            }
-          } else {
-            const int e = kc - kc_main;
-            mbar_arrive_expect_tx(fa, Cfg::kABytes + Cfg::kBBytes);
-            tma_load_2d(dA, &tmAe, fa, e * 64, r0);
-            tma_load_2d(dB, &tmBe, fa, e * 64, c0);
-          }
-        }
-      }
-      if (!ok || *abort_word) {
-        // let our own copies land before the CTA's shared memory goes away
-        for (uint32_t j = (g > (uint32_t)S ? g - S : 0); j < g; ++j) {
-          const uint64_t t0 = globaltimer_ns();
-          while (!mbar_try_wait(full_a + 8 * (j % S), (j / S) & 1) && globaltimer_ns() - t0 < 200000000ull) {}
-        }
-      }
-    }
-  } else if (warp == 5) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      constexpr uint32_t kIdMain = idesc_bf16_f32(128, BN, A_MN ? 1 : 0, B_MN ? 1 : 0);
-      constexpr uint32_t kIdExt = idesc_bf16_f32(128, BN, 0, 0);
-      uint32_t g = 0, tcount = 0;
-      bool ok = true;
-      for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tcount) {
-        const uint32_t acc = tcount & 1, aph = (tcount >> 1) & 1;
-        if (!mbar_wait(acc_empty + 8 * acc, aph ^ 1, lim, abort_word)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kc = 0; kc < kc_total; ++kc, ++g) {
-          const uint32_t s = g % S, ph = (g / S) & 1;
-          if (!mbar_wait(full_a + 8 * s, ph, lim, abort_word)) { ok = false; break; }
-          if (kDecode && !mbar_wait(full_b + 8 * s, ph, lim, abort_word)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a_base = smem_u32(sA + s * Cfg::kABytes);
-          const uint32_t b_base = smem_u32(sB + s * Cfg::kBBytes);
-          const bool ext = kc >= kc_main;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t ad = (!A_MN || ext) ? smem_desc_sw128(a_base + k * 32, 16, 1024)
-                                               : smem_desc_sw128(a_base + k * 2048, 8192, 1024);
-            const uint64_t bd = (!B_MN || ext) ? smem_desc_sw128(b_base + k * 32, 16, 1024)
-                                               : smem_desc_sw128(b_base + k * 2048, 8192, 1024);
-            tc_mma(d_tmem, ad, bd, ext ? kIdExt : kIdMain, (kc > 0 || k > 0) ? 1u : 0u);
-          }
-          tc_commit(empty + 8 * s);
-        }
-        if (!ok) break;
-        tc_commit(acc_full + 8 * acc);
-      }
-      if (!ok || *abort_word) {
-        tc_commit(drain);                       // completes once every issued MMA is done
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < 200000000ull) {}
-      }
-    }
-  } else if (kDecode) {
-    // ---------------- decode producers ----------------
-    const int tid = threadIdx.x - 192;
-    const float mean0 = (BS == BSrc::NF4) ? __ldg(args.mean) : 0.0f;
+    run_epilogue<BN, EPI>(args, tmem_base, acc_full, acc_empty, tiles, n_tiles, abort_word);
+  } else if (warp == 4 && lane == 0) {
     uint32_t g = 0;
     bool ok = true;
     for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-      const int64_t c0 = (t % n_tiles) * BN;
+      const int32_t r0 = (int32_t)((t / n_tiles) * 128), c0 = (int32_t)((t % n_tiles) * BN);
       for (int kc = 0; kc < kc_total; ++kc, ++g) {
         const uint32_t s = g % S, ph = (g / S) & 1;
-        const bool okw = mbar_wait(empty + 8 * s, ph ^ 1, lim, abort_word);
-        if (!__all_sync(0xFFFFFFFFu, okw)) { ok = false; break; }
-        if (kc < kc_main) {
-          uint8_t* bst = sB + s * Cfg::kBBytes;
-          if (!B_MN) {
-            // K-major tile: smem row u = weight row c0 + u, block kc of that row
-            const int u = tid;
-            decode_block<BS>(args, mean0, c0 + u, kc, bst + u * 128, (uint32_t)(u & 7));
-          } else {
-            // MN-major tile: 64-wide groups of output columns (weight input features),
-            // rows = weight rows kc*64 + j
-            const int j = tid & 63, gi = tid >> 6;
-            decode_block<BS>(args, mean0, (int64_t)kc * 64 + j, (c0 >> 6) + gi,
-                             bst + gi * 8192 + (j >> 3) * 1024 + (j & 7) * 128, (uint32_t)(j & 7));
-          }
-          fence_proxy_async_smem();
+        if (!mbar_wait(empty + 8 * s, ph ^ 1, lim, abort_word)) { ok = false; break; }
+        const uint32_t fb = full + 8 * s;
+        const uint32_t dA = smem_u32(sA + s * Cfg::kABytes);
+        const uint32_t dB = smem_u32(sB + s * Cfg::kBBytes);
+        mbar_arrive_expect_tx(fb, Cfg::kABytes + Cfg::kBBytes);
+        if (!A_MN) {
+          tma_load_2d(dA, &tmA, fb, kc * 64, r0);
+        } else {
+          tma_load_2d(dA, &tmA, fb, r0, kc * 64);
+          tma_load_2d(dA + 8192, &tmA, fb, r0 + 64, kc * 64);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(full_b + 8 * s);
+        if (!B_MN) {
+          tma_load_2d(dB, &tmB, fb, kc * 64, c0);
+        } else {
+#pragma unroll
+          for (int i = 0; i < BN / 64; ++i) tma_load_2d(dB + i * 8192, &tmB, fb, c0 + 64 * i, kc * 64);
+        }
       }
     }
+    if (!ok || *abort_word)
+      for (uint32_t j = (g > (uint32_t)S ? g - S : 0); j < g; ++j) drain_wait(full + 8 * (j % S), (j / S) & 1);
+  } else if (warp == 5 && lane == 0) {
+    constexpr uint32_t kId = idesc_bf16_f32(128, BN, A_MN ? 1 : 0, B_MN ? 1 : 0);
+    uint32_t g = 0, tcount = 0;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tcount) {
+      const uint32_t acc = tcount & 1, aph = (tcount >> 1) & 1;
+      if (!mbar_wait(acc_empty + 8 * acc, aph ^ 1, lim, abort_word)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * BN;
+      for (int kc = 0; kc < kc_total; ++kc, ++g) {
+        const uint32_t s = g % S, ph = (g / S) & 1;
+        if (!mbar_wait(full + 8 * s, ph, lim, abort_word)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(sA + s * Cfg::kABytes);
+        const uint32_t b_base = smem_u32(sB + s * Cfg::kBBytes);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint64_t ad = !A_MN ? smem_desc_sw128(a_base + k * 32, 16, 1024)
+                                    : smem_desc_sw128(a_base + k * 2048, 8192, 1024);
+          const uint64_t bd = !B_MN ? smem_desc_sw128(b_base + k * 32, 16, 1024)
+                                    : smem_desc_sw128(b_base + k * 2048, 8192, 1024);
+          tc_mma(d_tmem, ad, bd, kId, (kc > 0 || k > 0) ? 1u : 0u);
+        }
+        tc_commit(empty + 8 * s);
+      }
+      if (!ok) break;
+      tc_commit(acc_full + 8 * acc);
+    }
+    if (!ok || *abort_word) { tc_commit(drain); drain_wait(drain, 0); }
   }
 
   __syncwarp();
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  if (warp == 5) { tc_fence_after(); tmem_dealloc(tmem_base, Cfg::kTmemCols); }
+  if (threadIdx.x == 0 && *abort_word) raise_flag(args.flag, kFlagTimeout);
+}
+
+// =================================================================================
+// Weight operand decoded from NF4 / int8 (BN = 256, one decode thread per B row)
+// =================================================================================
+template <BSrc BS>
+struct DecCfg {
+  static constexpr int BN = 256;
+  static constexpr int NP = 8;                                   // decode warps
+  static constexpr int kABytes = 128 * 64 * 2;                   // activation tile
+  static constexpr int kBBytes = BN * 128;                       // decoded weight tile
+  static constexpr int kCodeBytes = BN * (BS == BSrc::NF4 ? 32 : 64);
+  static constexpr int kCBytes = kCodeBytes + 1024;              // codes + 256 fp32 scales
+  static constexpr int SA = 4, SB = 3, SC = (BS == BSrc::NF4 ? 6 : 3);
+  static constexpr int kTmemCols = 512;
+  static constexpr int kThreads = (7 + NP) * 32;
+  static constexpr size_t kSmem = (size_t)SA * kABytes + (size_t)SB * kBBytes + (size_t)SC * kCBytes + 2048;
+};
+
+// B_MN = false: forward (weight rows are output columns, K-major tile)
+// B_MN = true : dX (weight used transposed, MN-major tile)
+template <BSrc BS, bool B_MN, int EPI>
+__global__ void __launch_bounds__(DecCfg<BS>::kThreads, 1)
+qgemm_dec_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmCodes,
+                 const __grid_constant__ CUtensorMap tmScale, const __grid_constant__ CUtensorMap tmAe,
+                 const __grid_constant__ CUtensorMap tmBe, const GemmArgs args) {
+  using Cfg = DecCfg<BS>;
+  constexpr int BN = Cfg::BN, NP = Cfg::NP, SA = Cfg::SA, SB = Cfg::SB, SC = Cfg::SC;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + SA * Cfg::kABytes;
+  uint8_t* sC = sB + SB * Cfg::kBBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sC + SC * Cfg::kCBytes);
+  const uint32_t full_a = smem_u32(bars);
+  const uint32_t empty_a = full_a + 8 * SA;
+  const uint32_t full_b = empty_a + 8 * SA;
+  const uint32_t empty_b = full_b + 8 * SB;
+  const uint32_t full_c = empty_b + 8 * SB;
+  const uint32_t empty_c = full_c + 8 * SC;
+  const uint32_t acc_full = empty_c + 8 * SC;
+  const uint32_t acc_empty = acc_full + 16;
+  const uint32_t drain = acc_full + 32;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * (SA + SB + SC) + 5);
+  volatile int* abort_word = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SA; ++s) { mbar_init(full_a + 8 * s, 1); mbar_init(empty_a + 8 * s, 1); }
+    for (int s = 0; s < SB; ++s) { mbar_init(full_b + 8 * s, NP); mbar_init(empty_b + 8 * s, 1); }
+    for (int s = 0; s < SC; ++s) { mbar_init(full_c + 8 * s, 1); mbar_init(empty_c + 8 * s, NP); }
+    for (int i = 0; i < 2; ++i) { mbar_init(acc_full + 8 * i, 1); mbar_init(acc_empty + 8 * i, 4); }
+    mbar_init(drain, 1);
+    *abort_word = 0;
+    fence_mbar_init();
   }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    if (args.n_ext) tma_prefetch_desc(&tmAe);
+  }
+  if (warp == 6 && lane == 0) {
+    tma_prefetch_desc(&tmCodes);
+    tma_prefetch_desc(&tmScale);
+  }
+  if (warp == 7 && lane == 0 && args.n_ext) tma_prefetch_desc(&tmBe);
+  if (warp == 5) tmem_alloc(smem_u32(tmem_holder), Cfg::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  const int64_t n_tiles = (args.Cn + BN - 1) / BN;
+  const int64_t tiles = ((args.R + 127) / 128) * n_tiles;
+  const int kc_main = (int)((args.Kc + 63) / 64);
+  const int kc_total = kc_main + args.n_ext;
+  const uint64_t lim = args.timeout_ns;
+
+  if (warp < 4) {
+    run_epilogue<BN, EPI>(args, tmem_base, acc_full, acc_empty, tiles, n_tiles, abort_word);
+  } else if (warp == 4 && lane == 0) {
+    // ---- activation tiles (and the extension's left factor) -> A ring ----
+    uint32_t g = 0;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+      const int32_t r0 = (int32_t)((t / n_tiles) * 128);
+      for (int kc = 0; kc < kc_total; ++kc, ++g) {
+        const uint32_t s = g % SA, ph = (g / SA) & 1;
+        if (!mbar_wait(empty_a + 8 * s, ph ^ 1, lim, abort_word)) { ok = false; break; }
+        const uint32_t fb = full_a + 8 * s;
+        mbar_arrive_expect_tx(fb, Cfg::kABytes);
+        if (kc < kc_main) tma_load_2d(smem_u32(sA + s * Cfg::kABytes), &tmA, fb, kc * 64, r0);
+        else tma_load_2d(smem_u32(sA + s * Cfg::kABytes), &tmAe, fb, (kc - kc_main) * 64, r0);
+      }
+    }
+    if (!ok || *abort_word)
+      for (uint32_t j = (g > (uint32_t)SA ? g - SA : 0); j < g; ++j) drain_wait(full_a + 8 * (j % SA), (j / SA) & 1);
+  } else if (warp == 6 && lane == 0) {
+    // ---- weight codes + block scales -> C ring (main chunks only) ----
+    uint32_t gc = 0;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+      const int32_t c0 = (int32_t)((t % n_tiles) * BN);
+      for (int kc = 0; kc < kc_main; ++kc, ++gc) {
+        const uint32_t s = gc % SC, ph = (gc / SC) & 1;
+        if (!mbar_wait(empty_c + 8 * s, ph ^ 1, lim, abort_word)) { ok = false; break; }
+        const uint32_t fb = full_c + 8 * s;
+        const uint32_t dst = smem_u32(sC + s * Cfg::kCBytes);
+        mbar_arrive_expect_tx(fb, Cfg::kCBytes);
+        if (!B_MN) {
+          // rows c0.. of the weight, k-block kc: codes box {bytes per block, 256 rows},
+          // scales from the block-major copy: 256 consecutive rows of block column kc
+          tma_load_2d(dst, &tmCodes, fb, kc * (BS == BSrc::NF4 ? 32 : 64), c0);
+          tma_load_2d(dst + Cfg::kCodeBytes, &tmScale, fb, c0, kc);
+        } else {
+          // weight rows kc*64 .. +64, weight columns c0 .. c0+256 (4 blocks per row)
+          tma_load_2d(dst, &tmCodes, fb, BS == BSrc::NF4 ? c0 / 2 : c0, kc * 64);
+          tma_load_2d(dst + Cfg::kCodeBytes, &tmScale, fb, c0 / 64, kc * 64);
+        }
+      }
+    }
+    if (!ok || *abort_word)
+      for (uint32_t j = (gc > (uint32_t)SC ? gc - SC : 0); j < gc; ++j) drain_wait(full_c + 8 * (j % SC), (j / SC) & 1);
+  } else if (warp == 5 && lane == 0) {
+    // ---- MMA issuer ----
+    constexpr uint32_t kIdMain = idesc_bf16_f32(128, BN, 0, B_MN ? 1 : 0);
+    constexpr uint32_t kIdExt = idesc_bf16_f32(128, BN, 0, 0);
+    uint32_t g = 0, tcount = 0;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tcount) {
+      const uint32_t acc = tcount & 1, aph = (tcount >> 1) & 1;
+      if (!mbar_wait(acc_empty + 8 * acc, aph ^ 1, lim, abort_word)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * BN;
+      for (int kc = 0; kc < kc_total; ++kc, ++g) {
+        const uint32_t sa = g % SA, pa = (g / SA) & 1;
+        const uint32_t sb = g % SB, pb = (g / SB) & 1;
+        if (!mbar_wait(full_a + 8 * sa, pa, lim, abort_word)) { ok = false; break; }
+        if (!mbar_wait(full_b + 8 * sb, pb, lim, abort_word)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(sA + sa * Cfg::kABytes);
+        const uint32_t b_base = smem_u32(sB + sb * Cfg::kBBytes);
+        const bool ext = kc >= kc_main;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint64_t ad = smem_desc_sw128(a_base + k * 32, 16, 1024);
+          const uint64_t bd = (!B_MN || ext) ? smem_desc_sw128(b_base + k * 32, 16, 1024)
+                                             : smem_desc_sw128(b_base + k * 2048, 8192, 1024);
+          tc_mma(d_tmem, ad, bd, ext ? kIdExt : kIdMain, (kc > 0 || k > 0) ? 1u : 0u);
+        }
+        tc_commit(empty_a + 8 * sa);
+        tc_commit(empty_b + 8 * sb);
+      }
+      if (!ok) break;
+      tc_commit(acc_full + 8 * acc);
+    }
+    if (!ok || *abort_word) { tc_commit(drain); drain_wait(drain, 0); }
+  } else if (warp >= 7) {
+    // ---- decode: C ring (codes, scales) -> B ring (bf16, swizzled UMMA layout) ----
+    const int tid = threadIdx.x - 7 * 32;
+    float q[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) q[i] = args.q[i];
+    // where this thread's block sits in the C stage and in the B tile
+    int code_off, scale_idx;
+    uint32_t b_off, key;
+    if (!B_MN) {
+      code_off = tid * (BS == BSrc::NF4 ? 32 : 64);
+      scale_idx = tid;
+      b_off = tid * 128;
+      key = tid & 7;
+    } else {
+      const int j = tid & 63, gi = tid >> 6;
+      code_off = j * (BS == BSrc::NF4 ? 128 : 256) + gi * (BS == BSrc::NF4 ? 32 : 64);
+      scale_idx = j * 4 + gi;
+      b_off = gi * 8192 + (j >> 3) * 1024 + (j & 7) * 128;
+      key = j & 7;
+    }
+    // The decode warps are the only producers of the B ring, extension stages included
+    // (one of them issues that stage's TMA), so every producer of a stage has waited on
+    // every earlier phase of it and the parity waits stay exact.
+    uint32_t gc = 0, gb = 0, gx = 0, last_sb = 0, last_pb = 0;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+      const int32_t c0 = (int32_t)((t % n_tiles) * BN);
+      for (int kc = 0; kc < kc_total; ++kc, ++gb) {
+        const uint32_t sb = gb % SB, pb = (gb / SB) & 1;
+        if (kc >= kc_main) {
+          const bool wb = mbar_wait(empty_b + 8 * sb, pb ^ 1, lim, abort_word);
+          if (!__all_sync(0xFFFFFFFFu, wb)) { ok = false; break; }
+          if (lane == 0) {
+            const uint32_t fb = full_b + 8 * sb;
+            if (warp == 7) {
+              mbar_arrive_expect_tx(fb, Cfg::kBBytes);
+              tma_load_2d(smem_u32(sB + sb * Cfg::kBBytes), &tmBe, fb, (kc - kc_main) * 64, c0);
+              ++gx;
+              last_sb = sb;
+              last_pb = pb;
+            } else {
+              mbar_arrive(fb);
+            }
+          }
+          continue;
+        }
+        const uint32_t sc = gc % SC, pc = (gc / SC) & 1;
+        const bool w1 = mbar_wait(full_c + 8 * sc, pc, lim, abort_word);
+        const bool w2 = w1 && mbar_wait(empty_b + 8 * sb, pb ^ 1, lim, abort_word);
+        if (!__all_sync(0xFFFFFFFFu, w2)) { ok = false; break; }
+        const uint8_t* cst = sC + sc * Cfg::kCBytes;
+        const float sv = reinterpret_cast<const float*>(cst + Cfg::kCodeBytes)[scale_idx];
+        uint4* d = reinterpret_cast<uint4*>(sB + sb * Cfg::kBBytes + b_off);
+        if constexpr (BS == BSrc::NF4) {
+          const uint4* src = reinterpret_cast<const uint4*>(cst + code_off);
+          const uint4 c0v = src[0], c1v = src[1];
+          uint32_t L[2], H[2];
+          nf4_table(q, sv, L, H);
+          d[0 ^ key] = nf4_decode8(c0v.x, L, H);
+          d[1 ^ key] = nf4_decode8(c0v.y, L, H);
+          d[2 ^ key] = nf4_decode8(c0v.z, L, H);
+          d[3 ^ key] = nf4_decode8(c0v.w, L, H);
+          d[4 ^ key] = nf4_decode8(c1v.x, L, H);
+          d[5 ^ key] = nf4_decode8(c1v.y, L, H);
+          d[6 ^ key] = nf4_decode8(c1v.z, L, H);
+          d[7 ^ key] = nf4_decode8(c1v.w, L, H);
+        } else {
+          const uint4* src = reinterpret_cast<const uint4*>(cst + code_off);
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const uint4 w = src[h];
+            d[(2 * h) ^ key] = int8_decode8(w.x, w.y, sv);
+            d[(2 * h + 1) ^ key] = int8_decode8(w.z, w.w, sv);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(full_b + 8 * sb);
+          mbar_arrive(empty_c + 8 * sc);
+        }
+        ++gc;
+      }
+    }
+    if ((!ok || *abort_word) && warp == 7 && lane == 0 && gx)
+      drain_wait(full_b + 8 * last_sb, last_pb);       // our last extension copy (bounded)
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) { tc_fence_after(); tmem_dealloc(tmem_base, Cfg::kTmemCols); }
   if (threadIdx.x == 0 && *abort_word) raise_flag(args.flag, kFlagTimeout);
 }
 

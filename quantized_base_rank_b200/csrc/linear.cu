@@ -36,32 +36,64 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// bf16 matrix [outer, inner] with row stride `ld` elements; box {64, box_outer} with
-// the 128-byte swizzle (one 128-byte smem row per box row).
-static bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld,
-                     uint32_t box_outer) {
+// 2-D tensor [outer, inner] with row stride `ld_bytes`; box {box_inner, box_outer}.
+static bool make_map_t(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* ptr,
+                       uint64_t inner, uint64_t outer, uint64_t ld_bytes, uint32_t box_inner,
+                       uint32_t box_outer, CUtensorMapSwizzle swz) {
   auto fn = encode_fn();
   if (!fn) return false;
+  (void)esize;
   cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {ld * 2};
-  cuuint32_t box[2] = {64, box_outer};
+  cuuint64_t strides[1] = {ld_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t es[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int NP, bool A_MN, BSrc BS, bool B_MN, int EPI>
-static ql_status launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& ae,
-                             const CUtensorMap& be, const GemmArgs& args, cudaStream_t st) {
-  auto kern = qgemm_kernel<BN, NP, A_MN, BS, B_MN, EPI>;
-  const size_t smem = GemmCfg<BN>::kSmem;
+// bf16 matrix [outer, inner] with row stride `ld` elements; box {64, box_outer} with the
+// 128-byte swizzle (one 128-byte smem row per box row).
+static bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld,
+                     uint32_t box_outer) {
+  return make_map_t(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, inner, outer, ld * 2, 64, box_outer,
+                    CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+template <int BN, bool A_MN, bool B_MN, int EPI>
+static ql_status launch_tma(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args,
+                            cudaStream_t st) {
+  auto kern = qgemm_tma_kernel<BN, A_MN, B_MN, EPI>;
+  const size_t smem = TmaCfg<BN>::kSmem;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return QL_ERR_CUDA;
   const int64_t tiles = ((args.R + 127) / 128) * ((args.Cn + BN - 1) / BN);
   const int grid = (int)imin64(tiles, num_sms());
   if (grid <= 0) return QL_OK;
-  kern<<<grid, (6 + NP) * 32, smem, st>>>(a, b, ae, be, args);
+  kern<<<grid, 192, smem, st>>>(a, b, args);
+  QL_CHECK_LAUNCH();
+  return QL_OK;
+}
+
+template <int EPI, bool A_MN, bool B_MN>
+static ql_status launch_tma_rp(int rp, const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& args,
+                               cudaStream_t st) {
+  if (rp == 64) return launch_tma<64, A_MN, B_MN, EPI>(a, b, args, st);
+  if (rp == 128) return launch_tma<128, A_MN, B_MN, EPI>(a, b, args, st);
+  return launch_tma<256, A_MN, B_MN, EPI>(a, b, args, st);
+}
+
+template <BSrc BS, bool B_MN, int EPI>
+static ql_status launch_dec(const CUtensorMap& a, const CUtensorMap& codes, const CUtensorMap& scale,
+                            const CUtensorMap& ae, const CUtensorMap& be, const GemmArgs& args,
+                            cudaStream_t st) {
+  auto kern = qgemm_dec_kernel<BS, B_MN, EPI>;
+  const size_t smem = DecCfg<BS>::kSmem;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return QL_ERR_CUDA;
+  const int64_t tiles = ((args.R + 127) / 128) * ((args.Cn + 255) / 256);
+  const int grid = (int)imin64(tiles, num_sms());
+  if (grid <= 0) return QL_OK;
+  kern<<<grid, DecCfg<BS>::kThreads, smem, st>>>(a, codes, scale, ae, be, args);
   QL_CHECK_LAUNCH();
   return QL_OK;
 }
@@ -104,32 +136,57 @@ __global__ void transpose_kernel(const uint16_t* __restrict__ src, int64_t rows,
   }
 }
 
+// Rebuilt block scales, fp32, one per block of 64 weight elements:
+//   NF4+DQ: a' = fp32(fp32(c8 * s_g) + mean);  int8: sc = fp32(absmax / 127).
+// major == 0: block-major copy out[kb * N + n] (forward: a stage reads 256 consecutive rows
+// of one block column); major == 1: row-major out[n * ld + kb] (dX: a stage reads 4
+// consecutive blocks of 64 rows). ld is padded so TMA row strides are 16-byte multiples.
+__global__ void block_scale_kernel(int fmt, const int8_t* __restrict__ qabsmax,
+                                   const float* __restrict__ gscale, const float* __restrict__ mean,
+                                   const float* __restrict__ absmax, int64_t N, int64_t KB, int major,
+                                   int64_t ld, float* __restrict__ out) {
+  const int64_t total = N * KB;
+  const float mu = fmt == QL_FMT_NF4_DQ ? *mean : 0.0f;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    int64_t n, kb;
+    if (major == 0) { kb = i / N; n = i % N; } else { n = i / KB; kb = i % KB; }
+    const int64_t blk = n * KB + kb;
+    float v;
+    if (fmt == QL_FMT_NF4_DQ) v = __fadd_rn(__fmul_rn((float)qabsmax[blk], gscale[blk >> 8]), mu);
+    else v = __fdiv_rn(absmax[blk], 127.0f);
+    out[major == 0 ? kb * N + n : n * ld + kb] = v;
+  }
+}
+
 static int small_grid(int64_t n) { return (int)imax64(1, imin64((n + 255) / 256, (int64_t)num_sms() * 8)); }
 
 static int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
 
 struct WsLayout {
-  int64_t off[4];
+  int64_t off[5];
   int64_t total;
 };
 
 static WsLayout ws_layout(int op, int64_t M, int64_t N, int64_t K, int r) {
   WsLayout L{};
   const int64_t rp = round_up(r, 64);
-  int64_t sz[4] = {0, 0, 0, 0};
+  int64_t sz[5] = {0, 0, 0, 0, 0};
   if (op == QL_OP_FWD) {
     sz[0] = M * rp * 2;        // P
     sz[1] = N * rp * 2;        // B padded
+    sz[4] = (K / 64) * N * 4;  // block scales, block-major
   } else if (op == QL_OP_BWD) {
     sz[0] = M * rp * 2;        // Q
     sz[1] = (int64_t)r * N * 2;  // B^T
     sz[2] = K * rp * 2;        // A^T padded
     sz[3] = M * rp * 2;        // T padded
+    sz[4] = N * round_up(K / 64, 4) * 4;  // block scales, row-major (padded rows)
   } else if (op == QL_OP_DQ) {
     sz[0] = 256;
   }
   int64_t o = 0;
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < 5; ++i) {
     L.off[i] = o;
     o += round_up(sz[i], 256);
   }
@@ -137,22 +194,44 @@ static WsLayout ws_layout(int op, int64_t M, int64_t N, int64_t K, int r) {
   return L;
 }
 
-static GemmArgs base_args(const ql_weight* w) {
+static GemmArgs base_args() {
   GemmArgs a{};
   const Nf4Tables& t = nf4_tables();
   for (int i = 0; i < 16; ++i) a.q[i] = t.q[i];
-  if (w) {
-    a.codes = static_cast<const uint8_t*>(w->codes);
-    a.qabsmax = w->qabsmax;
-    a.gscale = w->group_scale;
-    a.mean = w->mean;
-    a.absmax = w->absmax;
-    a.Nw = w->N;
-    a.Kw = w->K;
-  }
   a.timeout_ns = g_wait_timeout_ns.load();
   a.flag = device_flag_ptr();
   return a;
+}
+
+// Tensor maps of the quantised weight for the decode GEMM. Forward (transposed = false):
+// codes box {bytes per block, 256 rows}, scales from the block-major copy, box {256, 1}.
+// dX (transposed = true): codes box {4 blocks of bytes, 64 rows}, scales row-major, box {4, 64}.
+static bool make_weight_maps(const ql_weight* w, const float* scales, bool transposed,
+                             CUtensorMap* mc, CUtensorMap* ms) {
+  const int64_t N = w->N, K = w->K, KB = K / 64;
+  const bool nf4 = w->fmt == QL_FMT_NF4_DQ;
+  const uint64_t row_bytes = nf4 ? K / 2 : K;
+  const uint32_t blk_bytes = nf4 ? 32 : 64;
+  if (!transposed) {
+    return make_map_t(mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, row_bytes, N, row_bytes, blk_bytes,
+                      256, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+           make_map_t(ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, scales, N, KB, N * 4, 256, 1,
+                      CU_TENSOR_MAP_SWIZZLE_NONE);
+  }
+  const int64_t ld = round_up(KB, 4);
+  return make_map_t(mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, row_bytes, N, row_bytes, 4 * blk_bytes,
+                    64, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+         make_map_t(ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, scales, KB, N, ld * 4, 4, 64,
+                    CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+static ql_status launch_block_scales(const ql_weight* w, bool transposed, float* out, cudaStream_t st) {
+  const int64_t N = w->N, KB = w->K / 64;
+  const int64_t ld = transposed ? round_up(KB, 4) : 0;
+  block_scale_kernel<<<small_grid(N * KB), 256, 0, st>>>(w->fmt, w->qabsmax, w->group_scale, w->mean,
+                                                         w->absmax, N, KB, transposed ? 1 : 0, ld, out);
+  QL_CHECK_LAUNCH();
+  return QL_OK;
 }
 
 static ql_status check_weight(const ql_weight* w) {
@@ -200,42 +279,43 @@ ql_status qlora_linear_fwd(const ql_weight* w, const ql_bf16* X, int64_t M, cons
   const int rp = (int)round_up(r, 64);
   const float s = alpha / (float)r;
   cudaStream_t st = as_stream(stream);
-  uint16_t* P = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + L.off[0]);
-  uint16_t* Bp = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + L.off[1]);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  uint16_t* P = reinterpret_cast<uint16_t*>(wsb + L.off[0]);
+  uint16_t* Bp = reinterpret_cast<uint16_t*>(wsb + L.off[1]);
+  float* scales = reinterpret_cast<float*>(wsb + L.off[4]);
 
-  {
-    ProfScope prof(PK_FWD_PREP, st, 1);
-    pad_cols_kernel<<<small_grid(N * rp), 256, 0, st>>>(B, N, r, rp, Bp);
-    QL_CHECK_LAUNCH();
-  }
-
-  CUtensorMap mX, mA, mP, mBp, none;
-  memset(&none, 0, sizeof(none));
+  CUtensorMap mX, mA, mP, mBp, mc, ms;
   if (!make_map(&mX, X, K, M, K, 128) || !make_map(&mA, A, K, r, K, rp) ||
-      !make_map(&mP, P, rp, M, rp, 128) || !make_map(&mBp, Bp, rp, N, rp, 256))
+      !make_map(&mP, P, rp, M, rp, 128) || !make_map(&mBp, Bp, rp, N, rp, 256) ||
+      !make_weight_maps(w, scales, false, &mc, &ms))
     return QL_ERR_CUDA;
 
+  {
+    ProfScope prof(PK_FWD_PREP, st, 2);
+    pad_cols_kernel<<<small_grid(N * rp), 256, 0, st>>>(B, N, r, rp, Bp);
+    QL_CHECK_LAUNCH();
+    ql_status e = launch_block_scales(w, false, scales, st);
+    if (e != QL_OK) return e;
+  }
+
   // [T | P] = X A^T
-  GemmArgs t = base_args(nullptr);
+  GemmArgs t = base_args();
   t.R = M; t.Cn = rp; t.Kc = K; t.n_ext = 0; t.r = r;
   t.out = T_save; t.ld_out = r; t.out2 = P; t.ld_out2 = rp; t.scale = s;
   ql_status e;
   {
-  ProfScope prof(PK_FWD_T, st, 1);
-  if (rp == 64) e = launch_gemm<64, 0, false, BSrc::TMA, false, EPI_LORA_T>(mX, mA, none, none, t, st);
-  else if (rp == 128) e = launch_gemm<128, 0, false, BSrc::TMA, false, EPI_LORA_T>(mX, mA, none, none, t, st);
-  else e = launch_gemm<256, 0, false, BSrc::TMA, false, EPI_LORA_T>(mX, mA, none, none, t, st);
+    ProfScope prof(PK_FWD_T, st, 1);
+    e = launch_tma_rp<EPI_LORA_T, false, false>(rp, mX, mA, t, st);
   }
   if (e != QL_OK) return e;
 
   // Y = X W'^T + P Bp^T
-  GemmArgs y = base_args(w);
+  GemmArgs y = base_args();
   y.R = M; y.Cn = N; y.Kc = K; y.n_ext = rp / 64; y.r = r;
   y.out = Y; y.ld_out = N; y.scale = 1.0f;
   ProfScope prof(PK_FWD_MAIN, st, 1);
-  if (w->fmt == QL_FMT_NF4_DQ)
-    return launch_gemm<256, 8, false, BSrc::NF4, false, EPI_BF16>(mX, none, mP, mBp, y, st);
-  return launch_gemm<256, 8, false, BSrc::INT8, false, EPI_BF16>(mX, none, mP, mBp, y, st);
+  if (w->fmt == QL_FMT_NF4_DQ) return launch_dec<BSrc::NF4, false, EPI_BF16>(mX, mc, ms, mP, mBp, y, st);
+  return launch_dec<BSrc::INT8, false, EPI_BF16>(mX, mc, ms, mP, mBp, y, st);
 }
 
 ql_status qlora_linear_bwd(const ql_weight* w, const ql_bf16* X, const ql_bf16* dY, int64_t M,
@@ -261,66 +341,62 @@ ql_status qlora_linear_bwd(const ql_weight* w, const ql_bf16* X, const ql_bf16* 
   uint16_t* Bt = reinterpret_cast<uint16_t*>(wsb + L.off[1]);
   uint16_t* At = reinterpret_cast<uint16_t*>(wsb + L.off[2]);
   uint16_t* Tp = reinterpret_cast<uint16_t*>(wsb + L.off[3]);
+  float* scales = reinterpret_cast<float*>(wsb + L.off[4]);
+
+  CUtensorMap mdY_k, mBt, mQ_k, mAt, mdY_mn, mTp_mn, mX_mn, mQ_mn, mc, ms;
+  if (!make_map(&mdY_k, dY, N, M, N, 128) || !make_map(&mBt, Bt, N, r, N, rp) ||
+      !make_map(&mQ_k, Q, rp, M, rp, 128) || !make_map(&mAt, At, rp, K, rp, 256) ||
+      !make_map(&mdY_mn, dY, N, M, N, 64) || !make_map(&mTp_mn, Tp, rp, M, rp, 64) ||
+      !make_map(&mX_mn, X, K, M, K, 64) || !make_map(&mQ_mn, Q, rp, M, rp, 64) ||
+      !make_weight_maps(w, scales, true, &mc, &ms))
+    return QL_ERR_CUDA;
 
   {
-    ProfScope prof(PK_BWD_PREP, st, 3);
+    ProfScope prof(PK_BWD_PREP, st, 4);
     transpose_kernel<<<small_grid(N * r), 256, 0, st>>>(B, N, r, Bt);
     QL_CHECK_LAUNCH();
     transpose_pad_kernel<<<small_grid(K * rp), 256, 0, st>>>(A, r, K, rp, At);
     QL_CHECK_LAUNCH();
     pad_cols_kernel<<<small_grid(M * rp), 256, 0, st>>>(T_saved, M, r, rp, Tp);
     QL_CHECK_LAUNCH();
+    ql_status e = launch_block_scales(w, true, scales, st);
+    if (e != QL_OK) return e;
   }
-
-  CUtensorMap mdY_k, mBt, mQ_k, mAt, mdY_mn, mTp_mn, mX_mn, mQ_mn, none;
-  memset(&none, 0, sizeof(none));
-  if (!make_map(&mdY_k, dY, N, M, N, 128) || !make_map(&mBt, Bt, N, r, N, rp) ||
-      !make_map(&mQ_k, Q, rp, M, rp, 128) || !make_map(&mAt, At, rp, K, rp, 256) ||
-      !make_map(&mdY_mn, dY, N, M, N, 64) || !make_map(&mTp_mn, Tp, rp, M, rp, 64) ||
-      !make_map(&mX_mn, X, K, M, K, 64) || !make_map(&mQ_mn, Q, rp, M, rp, 64))
-    return QL_ERR_CUDA;
   ql_status e;
 
   // Q = bf16(s dY B)
-  GemmArgs u = base_args(nullptr);
+  GemmArgs u = base_args();
   u.R = M; u.Cn = rp; u.Kc = N; u.r = r; u.out = Q; u.ld_out = rp; u.scale = s;
   {
-  ProfScope prof(PK_BWD_U, st, 1);
-  if (rp == 64) e = launch_gemm<64, 0, false, BSrc::TMA, false, EPI_LORA_Q>(mdY_k, mBt, none, none, u, st);
-  else if (rp == 128) e = launch_gemm<128, 0, false, BSrc::TMA, false, EPI_LORA_Q>(mdY_k, mBt, none, none, u, st);
-  else e = launch_gemm<256, 0, false, BSrc::TMA, false, EPI_LORA_Q>(mdY_k, mBt, none, none, u, st);
+    ProfScope prof(PK_BWD_U, st, 1);
+    e = launch_tma_rp<EPI_LORA_Q, false, false>(rp, mdY_k, mBt, u, st);
   }
   if (e != QL_OK) return e;
 
   // dB = s dY^T T     (rows n, columns j, contraction over tokens)
-  GemmArgs b = base_args(nullptr);
+  GemmArgs b = base_args();
   b.R = N; b.Cn = rp; b.Kc = M; b.r = r; b.out = dB; b.ld_out = r; b.scale = s;
   {
-  ProfScope prof(PK_BWD_DB, st, 1);
-  if (rp == 64) e = launch_gemm<64, 0, true, BSrc::TMA, true, EPI_DB>(mdY_mn, mTp_mn, none, none, b, st);
-  else if (rp == 128) e = launch_gemm<128, 0, true, BSrc::TMA, true, EPI_DB>(mdY_mn, mTp_mn, none, none, b, st);
-  else e = launch_gemm<256, 0, true, BSrc::TMA, true, EPI_DB>(mdY_mn, mTp_mn, none, none, b, st);
+    ProfScope prof(PK_BWD_DB, st, 1);
+    e = launch_tma_rp<EPI_DB, true, true>(rp, mdY_mn, mTp_mn, b, st);
   }
   if (e != QL_OK) return e;
 
   // dA = Q^T X        (computed as dA^T: rows k, columns j)
-  GemmArgs a = base_args(nullptr);
+  GemmArgs a = base_args();
   a.R = K; a.Cn = rp; a.Kc = M; a.r = r; a.out = dA; a.ld_out = K; a.scale = 1.0f;
   {
-  ProfScope prof(PK_BWD_DA, st, 1);
-  if (rp == 64) e = launch_gemm<64, 0, true, BSrc::TMA, true, EPI_DA>(mX_mn, mQ_mn, none, none, a, st);
-  else if (rp == 128) e = launch_gemm<128, 0, true, BSrc::TMA, true, EPI_DA>(mX_mn, mQ_mn, none, none, a, st);
-  else e = launch_gemm<256, 0, true, BSrc::TMA, true, EPI_DA>(mX_mn, mQ_mn, none, none, a, st);
+    ProfScope prof(PK_BWD_DA, st, 1);
+    e = launch_tma_rp<EPI_DA, true, true>(rp, mX_mn, mQ_mn, a, st);
   }
   if (e != QL_OK) return e;
 
   // dX = dY W' + Q A^T-padded
-  GemmArgs x = base_args(w);
+  GemmArgs x = base_args();
   x.R = M; x.Cn = K; x.Kc = N; x.n_ext = rp / 64; x.r = r; x.out = dX; x.ld_out = K; x.scale = 1.0f;
   ProfScope prof(PK_BWD_DX, st, 1);
-  if (w->fmt == QL_FMT_NF4_DQ)
-    return launch_gemm<256, 8, false, BSrc::NF4, true, EPI_BF16>(mdY_k, none, mQ_k, mAt, x, st);
-  return launch_gemm<256, 8, false, BSrc::INT8, true, EPI_BF16>(mdY_k, none, mQ_k, mAt, x, st);
+  if (w->fmt == QL_FMT_NF4_DQ) return launch_dec<BSrc::NF4, true, EPI_BF16>(mdY_k, mc, ms, mQ_k, mAt, x, st);
+  return launch_dec<BSrc::INT8, true, EPI_BF16>(mdY_k, mc, ms, mQ_k, mAt, x, st);
 }
 
 }  // extern "C"
