@@ -180,6 +180,60 @@ def run_reference(args, case, world, rank):
 # GPU leg
 # --------------------------------------------------------------------------------------
 
+def decode_bench(dev, peaks, reps: int = 20):
+    """Decode-shaped forward (7B 4096x4096 NF4+DQ linear, r=16, M in {1, 4, 16}): GB/s of
+    algorithmic bytes per call. Back-to-back calls rotate over enough quantised weight
+    copies to exceed three times the L2 size, inside one CUDA graph, so each call reads its
+    weight from HBM; the graph is replayed `reps` times and timed with CUDA events."""
+    from quantized_base_rank_b200 import binding as B
+    from quantized_base_rank_b200 import synth
+    out = {}
+    base = synth.CFG2[0]
+    W = synth.weight_with_outliers(base.N, base.K, base.w_std, base.outlier_frac, base.outlier_mult,
+                                   base.seed).to(dev)
+    q0 = B.quantize_weight(W, "nf4_dq")
+    del W
+    n = base.N * base.K
+    wbytes = n * (0.5 + 1.0 / 64) + 4.0 * n / 16384
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    copies = max(4, int(np.ceil(3 * l2 / wbytes)))
+    qws = [B.QuantWeight("nf4_dq", base.N, base.K, q0.codes.clone(), None, q0.qabsmax.clone(),
+                         q0.group_scale.clone(), q0.mean.clone()) for _ in range(copies)]
+    for case in synth.CFG2:
+        M, N, K, r = case.M, case.N, case.K, case.r
+        inp = synth.make_inputs(case)
+        X, A, Bm = (inp[k].to(dev) for k in ("X", "A", "B"))
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        T = torch.empty((M, r), dtype=torch.bfloat16, device=dev)
+        for qw in qws[:2]:
+            B.linear_fwd(qw, X, A, Bm, case.alpha, Y=Y, T=T)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream(dev)
+        s.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                for qw in qws:
+                    B.linear_fwd(qw, X, A, Bm, case.alpha, Y=Y, T=T)
+        torch.cuda.synchronize()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / (reps * copies)
+        nbytes = wbytes + 2 * M * K + 2 * r * K + 2 * N * r + 2 * M * N
+        gbs = nbytes / (us * 1e-6) / 1e9
+        out[f"M{M}"] = {"us_per_call": us, "bytes": nbytes, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
+                        "frac_8tbs": gbs / 8000.0, "weight_copies": copies}
+        del g
+    return out
+
+
 def run_ours(args, case, world, rank, local_rank):
     from quantized_base_rank_b200 import binding as B
     from quantized_base_rank_b200 import synth
@@ -313,6 +367,9 @@ def run_ours(args, case, world, rank, local_rank):
     e2e_ms = timed(e2e_step, e2e_steps)
     e2e_value = world * (fwd_f + bwd_f) / (e2e_ms * 1e-3) / 1e12
 
+    # ---- decode-shaped forward (small M, HBM-bound) ----
+    decode = decode_bench(dev, peaks)
+
     # ---- CPU oracle baseline (rank 0, one GPU only) ----
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -348,6 +405,7 @@ def run_ours(args, case, world, rank, local_rank):
             "fwd_main_gemm": {"ms": main_ms, "TFLOP/s": achieved},
             "bwd_dx_gemm": {"ms": dx_ms, "TFLOP/s": dx_flops / (dx_ms * 1e-3) / 1e12},
             "per_group_ms": {g: avg(g) for g in B.PROFILE_GROUPS if prof[g][1]},
+            "decode_7b_4096x4096_nf4": decode,
         },
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},

@@ -119,7 +119,10 @@ ql_status ql_dequantize(const ql_weight* w, ql_bf16* Wout, void* stream);
  *   T = X A^T (fp32 accumulate); P = bf16(s T);
  *   Y [M, N] bf16 = bf16(X W'^T + P B^T), fp32 accumulation.
  *   T_save [M, r] bf16 = bf16(T) if non-NULL (needed by qlora_linear_bwd).
- * K % 64 == 0, 1 <= r <= 256, M >= 1. ws: ql_workspace_bytes(QL_OP_FWD, M, N, K, r). */
+ * K % 64 == 0, N % 8 == 0, 1 <= r <= 256, M >= 1. ws: ql_workspace_bytes(QL_OP_FWD, M, N, K, r)
+ * bytes (zero, and ws may be NULL, for M <= 16: that decode-shaped case runs as one
+ * kernel that splits K over a cluster of 8 CTAs and adds the adapter term per K-range,
+ * so its rounding differs from the large-M path within the stated tolerance). */
 ql_status qlora_linear_fwd(const ql_weight* w, const ql_bf16* X, int64_t M,
                            const ql_bf16* A, const ql_bf16* B, int32_t r, float alpha,
                            ql_bf16* Y, ql_bf16* T_save, void* ws, size_t ws_bytes,

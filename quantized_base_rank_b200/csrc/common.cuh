@@ -21,6 +21,12 @@ struct Nf4Tables {
 };
 
 const Nf4Tables& nf4_tables();          // host, computed on first use
+
+// Decode-shaped forward (M <= 16), small_m.cu.
+ql_status small_m_forward(const ql_weight* w, const uint16_t* X, int64_t M, const uint16_t* A,
+                          const uint16_t* B, int r, float alpha, uint16_t* Y, uint16_t* T_save,
+                          cudaStream_t st);
+constexpr int64_t kSmallMMax = 16;
 int* device_flag_ptr();                 // device address of the sticky flag (current device)
 int num_sms();                          // SM count of the current device
 

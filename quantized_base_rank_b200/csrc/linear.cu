@@ -256,6 +256,7 @@ extern "C" {
 size_t ql_workspace_bytes(int32_t op, int64_t M, int64_t N, int64_t K, int32_t r) {
   if (op == QL_OP_DQ) return 256;
   if ((op != QL_OP_FWD && op != QL_OP_BWD) || M < 0 || N < 0 || K < 0 || r < 1 || r > 256) return 0;
+  if (op == QL_OP_FWD && M <= kSmallMMax) return 0;      // the decode-shaped path needs none
   return (size_t)ws_layout(op, M, N, K, r).total;
 }
 
@@ -268,17 +269,19 @@ ql_status qlora_linear_fwd(const ql_weight* w, const ql_bf16* X, int64_t M, cons
                            void* ws, size_t ws_bytes, void* stream) {
   ql_status st0 = check_weight(w);
   if (st0 != QL_OK) return st0;
-  if (!X || !A || !B || !Y || !ws || M < 1 || r < 1) return QL_ERR_INVALID_ARG;
+  if (!X || !A || !B || !Y || M < 1 || r < 1) return QL_ERR_INVALID_ARG;
   if (r > 256 || M > (int64_t(1) << 31)) return QL_ERR_UNSUPPORTED;
-  if (!aligned(X, 16) || !aligned(A, 16) || !aligned(B, 2) || !aligned(Y, 16) || !aligned(ws, 256) ||
+  if (!aligned(X, 16) || !aligned(A, 16) || !aligned(B, 2) || !aligned(Y, 16) ||
       (T_save && !aligned(T_save, 2)))
     return QL_ERR_INVALID_ARG;
+  if (M > kSmallMMax && (!ws || !aligned(ws, 256))) return QL_ERR_INVALID_ARG;
   const int64_t N = w->N, K = w->K;
+  cudaStream_t st = as_stream(stream);
+  if (M <= kSmallMMax) return small_m_forward(w, X, M, A, B, r, alpha, Y, T_save, st);
   const WsLayout L = ws_layout(QL_OP_FWD, M, N, K, r);
   if ((int64_t)ws_bytes < L.total) return QL_ERR_WORKSPACE;
   const int rp = (int)round_up(r, 64);
   const float s = alpha / (float)r;
-  cudaStream_t st = as_stream(stream);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   uint16_t* P = reinterpret_cast<uint16_t*>(wsb + L.off[0]);
   uint16_t* Bp = reinterpret_cast<uint16_t*>(wsb + L.off[1]);

@@ -173,6 +173,7 @@ constexpr int kSumBins = 16;
 
 __global__ void __launch_bounds__(256)
 dq_sum_kernel(const float* __restrict__ absmax, int64_t nb, unsigned long long* bins, int* flag) {
+  __shared__ unsigned long long part[8][kSumBins];
   unsigned long long acc[kSumBins];
 #pragma unroll
   for (int i = 0; i < kSumBins; ++i) acc[i] = 0ull;
@@ -190,12 +191,19 @@ dq_sum_kernel(const float* __restrict__ absmax, int64_t nb, unsigned long long* 
     for (int i = 0; i < kSumBins; ++i) acc[i] += (bin == (uint32_t)i) ? c : 0ull;
   }
   if (bad) raise_flag(flag, kFlagNonfinite);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll
   for (int i = 0; i < kSumBins; ++i) {
     unsigned long long x = acc[i];
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) x += __shfl_down_sync(0xFFFFFFFFu, x, off);
-    if ((threadIdx.x & 31) == 0 && x) atomicAdd(bins + i, x);
+    if (lane == 0) part[warp][i] = x;
+  }
+  __syncthreads();
+  if (threadIdx.x < kSumBins) {
+    unsigned long long x = 0ull;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) x += part[w][threadIdx.x];
+    if (x) atomicAdd(bins + threadIdx.x, x);
   }
 }
 
@@ -209,37 +217,37 @@ __global__ void dq_finalize_kernel(const unsigned long long* __restrict__ bins, 
   for (int i = 0; i < kSumBins; ++i) {
     const unsigned long long v = bins[i];
     const int bit = 16 * i;
-    int li = bit / 32;
-    // v << (bit % 32) spans up to three 32-bit limbs
-    unsigned long long lo = (bit % 32) ? (v << 16) : v;
-    uint32_t hi_extra = (bit % 32) ? (uint32_t)(v >> 48) : 0u;
-    uint32_t parts[3] = {(uint32_t)lo, (uint32_t)(lo >> 32), hi_extra};
+    const int li = bit / 32;
+    const unsigned long long lo = (bit % 32) ? (v << 16) : v;
+    const uint32_t parts[3] = {(uint32_t)lo, (uint32_t)(lo >> 32), (bit % 32) ? (uint32_t)(v >> 48) : 0u};
     unsigned long long carry = 0;
     for (int k = 0; li + k < 12; ++k) {
-      unsigned long long s = (unsigned long long)limb[li + k] + (k < 3 ? parts[k] : 0u) + carry;
-      limb[li + k] = (uint32_t)s;
-      carry = s >> 32;
+      const unsigned long long sum = (unsigned long long)limb[li + k] + (k < 3 ? parts[k] : 0u) + carry;
+      limb[li + k] = (uint32_t)sum;
+      carry = sum >> 32;
       if (k >= 2 && carry == 0) break;
     }
   }
   int top = -1;
-  for (int i = 11; i >= 0 && top < 0; --i)
-    if (limb[i]) top = 32 * i + 31 - __clz(limb[i]);
+  for (int i = 11; i >= 0; --i)
+    if (limb[i]) { top = i; break; }
   double S = 0.0;
   if (top >= 0) {
-    auto bit_at = [&](int k) -> uint32_t { return k < 0 ? 0u : (limb[k / 32] >> (k % 32)) & 1u; };
-    const int lsb = top - 52;                          // lowest kept bit position
-    unsigned long long mant = 0;
-    for (int k = top; k >= max(lsb, 0); --k) mant = (mant << 1) | bit_at(k);
-    int exp2 = 0;
-    if (lsb > 0) {
-      const uint32_t round = bit_at(lsb - 1);
-      uint32_t sticky = 0;
-      for (int k = lsb - 2; k >= 0 && !sticky; --k) sticky |= bit_at(k);
-      if (round && (sticky || (mant & 1ull))) mant += 1ull;
-      exp2 = lsb;
+    // 96-bit window of limbs top, top-1, top-2 (missing limbs are zero)
+    const uint32_t l1 = top >= 1 ? limb[top - 1] : 0u, l2 = top >= 2 ? limb[top - 2] : 0u;
+    const unsigned __int128 W = ((unsigned __int128)limb[top] << 64) | ((unsigned __int128)l1 << 32) | l2;
+    const int tb = 95 - __clz(limb[top]);              // top set bit inside W (>= 64)
+    const int base = 32 * (top - 2);                   // weight of bit 0 of W
+    if (base + tb < 53) {
+      S = ldexp((double)(unsigned long long)(W >> (base < 0 ? -base : 0)), base > 0 ? base - 149 : -149);
+    } else {
+      unsigned long long mant = (unsigned long long)(W >> (tb - 52));
+      const uint32_t rbit = (uint32_t)(W >> (tb - 53)) & 1u;
+      bool sticky = (W & ((((unsigned __int128)1) << (tb - 53)) - 1)) != 0;
+      for (int i = 0; i < top - 2 && !sticky; ++i) sticky = limb[i] != 0u;
+      if (rbit && (sticky || (mant & 1ull))) mant += 1ull;
+      S = ldexp((double)mant, base + tb - 52 - 149);   // exact scaling
     }
-    S = ldexp((double)mant, exp2 - 149);               // exact scaling
   }
   *mean = __double2float_rn(__ddiv_rn(S, (double)nb));
 }
@@ -371,7 +379,8 @@ ql_status dq_quantize(const float* absmax, int64_t nblocks, int8_t* qabsmax, flo
   ProfScope prof(PK_DQ, st, 3);
   if (cudaMemsetAsync(bins, 0, kSumBins * sizeof(unsigned long long), st) != cudaSuccess)
     return QL_ERR_CUDA;
-  dq_sum_kernel<<<grid_for(nblocks, 256), 256, 0, st>>>(absmax, nblocks, bins, device_flag_ptr());
+  dq_sum_kernel<<<(int)imin64((nblocks + 255) / 256, num_sms()), 256, 0, st>>>(absmax, nblocks, bins,
+                                                                              device_flag_ptr());
   QL_CHECK_LAUNCH();
   dq_finalize_kernel<<<1, 32, 0, st>>>(bins, nblocks, mean);
   QL_CHECK_LAUNCH();

@@ -148,3 +148,21 @@ def test_timeout_path_reports_and_recovers():
         B.lib().ql_set_wait_timeout_ns(0)
     assert st in (B.QL_OK, B.QL_ERR_TIMEOUT)
     check_case(case, inp)
+
+
+# ---- decode-shaped forward (M <= 16): one cluster-split kernel ------------------------
+
+@pytest.mark.parametrize("case", synth.CFG2, ids=[c.name for c in synth.CFG2])
+def test_cfg2_decode_7b_full(case):
+    """7B decode-shaped linear, 4096x4096 with 0.1% outliers at 20 sigma, r=16: every
+    output of Y and T against the oracle."""
+    check_case(case)
+
+
+@pytest.mark.parametrize("M,N,K,r,fmt", [(1, 256, 256, 8, "nf4_dq"), (3, 200, 320, 20, "int8"),
+                                         (16, 1024, 4160, 64, "nf4_dq"), (9, 136, 704, 1, "nf4_dq"),
+                                         (16, 512, 11008, 16, "int8"), (5, 4096, 64, 33, "nf4_dq")])
+def test_small_m_ragged(M, N, K, r, fmt):
+    case = synth.LinearCase(f"small-{M}-{N}-{K}-{r}", N=N, K=K, M=M, r=r, alpha=16.0, fmt=fmt,
+                            seed=N + K)
+    check_case(case)
