@@ -8,14 +8,10 @@
 //
 // qgemm_tma_kernel — both operands by TMA (the adapter-sized GEMMs). Warps:
 //   0..3 epilogue, 4 TMA, 5 MMA issuer (also owns TMEM).
-// qgemm_dec_kernel — the weight operand is decoded from its quantised form (QLoRA page,
-// "1. NF4" and "2. Double Quantization": w' = q[code] * a'). Warps:
-//   0..3 epilogue, 4 TMA for the activation tiles (and the adapter extension's left
-//   factor), 5 MMA issuer, 6 TMA for the weight codes + rebuilt block scales,
-//   7..14 decode: codes in smem -> bf16 rows written straight into the 128-byte-swizzled
-//   UMMA layout of the weight tile (they also issue the TMA of the extension's right
-//   factor, so each ring keeps a single producer). Nothing in the decode warps reads
-//   global memory, so they never wait on it.
+// qgemm_wdec_kernel — the weight operand is decoded from its quantised form (QLoRA page,
+// "1. NF4" and "2. Double Quantization": w' = q[code] * a') into the swizzled UMMA layout
+// and used as the MMA's M = 128 operand against 256 tokens (see below). Nothing in the
+// decode warps reads global memory, so they never wait on it.
 // The unmerged LoRA term enters as extra contraction chunks of the same accumulator.
 //
 // Every wait is bounded; a wait that gives up raises the CTA's abort word, every role then
@@ -312,53 +308,75 @@ qgemm_tma_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 }
 
 // =================================================================================
-// Weight operand decoded from NF4 / int8 (BN = 256, one decode thread per B row)
+// Weight operand decoded from NF4 / int8, as the M = 128 operand of the MMA
+//
+//   C^T[w, t] = sum_k W'[w, k] * T[t, k]   (w: 128 weight rows per tile, t: 256 tokens)
+//
+// Forward: w = output feature n, contraction over input features (W' K-major).
+// dX:      w = input feature k,  contraction over output features (W'^T, MN-major).
+// Each decoded weight row feeds 256 token columns, so a tile decodes 128 blocks per
+// chunk for 2*128*256*64 flops. The result is stored transposed (lanes are consecutive
+// weight rows, so every store instruction of a warp writes 64 contiguous bytes).
+// Warps: 0..3 epilogue, 4 TMA for the token tiles (and the extension's token factor),
+// 5 MMA issuer, 6 TMA for the weight codes + block scales, 7..14 decode (two lanes per
+// 64-element block; they also issue the TMA of the extension's weight-side factor, so
+// every ring has a single producer).
 // =================================================================================
 template <BSrc BS>
-struct DecCfg {
-  static constexpr int BN = 256;
+struct WdecCfg {
+  static constexpr int BM = 128;                                 // weight rows per tile
+  static constexpr int BN = 256;                                 // tokens per tile
   static constexpr int NP = 8;                                   // decode warps
-  static constexpr int kABytes = 128 * 64 * 2;                   // activation tile
-  static constexpr int kBBytes = BN * 128;                       // decoded weight tile
-  static constexpr int kCodeBytes = BN * (BS == BSrc::NF4 ? 32 : 64);
-  static constexpr int kCBytes = kCodeBytes + 1024;              // codes + 256 fp32 scales
-  static constexpr int SA = 4, SB = 3, SC = (BS == BSrc::NF4 ? 6 : 3);
+  static constexpr int kDBytes = BM * 128;                       // decoded weight stage
+  static constexpr int kTBytes = BN * 128;                       // token stage
+  static constexpr int kCodeBytes = BM * (BS == BSrc::NF4 ? 32 : 64);
+  static constexpr int kCBytes = kCodeBytes + 1024;              // codes + scales
+  static constexpr int SD = 4, ST = 4, SC = (BS == BSrc::NF4 ? 6 : 3);
   static constexpr int kTmemCols = 512;
   static constexpr int kThreads = (7 + NP) * 32;
-  static constexpr size_t kSmem = (size_t)SA * kABytes + (size_t)SB * kBBytes + (size_t)SC * kCBytes + 2048;
+  static constexpr size_t kSmem = (size_t)SD * kDBytes + (size_t)ST * kTBytes + (size_t)SC * kCBytes + 2048;
 };
 
-// B_MN = false: forward (weight rows are output columns, K-major tile)
-// B_MN = true : dX (weight used transposed, MN-major tile)
-template <BSrc BS, bool B_MN, int EPI>
-__global__ void __launch_bounds__(DecCfg<BS>::kThreads, 1)
-qgemm_dec_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmCodes,
-                 const __grid_constant__ CUtensorMap tmScale, const __grid_constant__ CUtensorMap tmAe,
-                 const __grid_constant__ CUtensorMap tmBe, const GemmArgs args) {
-  using Cfg = DecCfg<BS>;
-  constexpr int BN = Cfg::BN, NP = Cfg::NP, SA = Cfg::SA, SB = Cfg::SB, SC = Cfg::SC;
+// EPI_BF16 stored transposed: element (weight row w, token t) -> out[t * ld_out + w]
+__device__ __forceinline__ void epilogue_store_t(const GemmArgs& a, int64_t wrow, int64_t t0,
+                                                 const uint32_t (&v)[32]) {
+  if (wrow >= a.R) return;
+  uint16_t* out = static_cast<uint16_t*>(a.out) + wrow;
+#pragma unroll
+  for (int j = 0; j < 32; ++j)
+    if (t0 + j < a.Cn) out[(t0 + j) * a.ld_out] = (uint16_t)float_to_bf16_bits(__uint_as_float(v[j]));
+}
+
+// W_MN = false: forward; true: dX (weight used transposed)
+template <BSrc BS, bool W_MN>
+__global__ void __launch_bounds__(WdecCfg<BS>::kThreads, 1)
+qgemm_wdec_kernel(const __grid_constant__ CUtensorMap tmT, const __grid_constant__ CUtensorMap tmCodes,
+                  const __grid_constant__ CUtensorMap tmScale, const __grid_constant__ CUtensorMap tmTe,
+                  const __grid_constant__ CUtensorMap tmWe, const GemmArgs args) {
+  using Cfg = WdecCfg<BS>;
+  constexpr int BM = Cfg::BM, BN = Cfg::BN, NP = Cfg::NP, SD = Cfg::SD, ST = Cfg::ST, SC = Cfg::SC;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = smem;
-  uint8_t* sB = sA + SA * Cfg::kABytes;
-  uint8_t* sC = sB + SB * Cfg::kBBytes;
+  uint8_t* sD = smem;                                   // decoded weight (A operand)
+  uint8_t* sT = sD + SD * Cfg::kDBytes;                 // tokens (B operand)
+  uint8_t* sC = sT + ST * Cfg::kTBytes;                 // codes + scales
   uint64_t* bars = reinterpret_cast<uint64_t*>(sC + SC * Cfg::kCBytes);
-  const uint32_t full_a = smem_u32(bars);
-  const uint32_t empty_a = full_a + 8 * SA;
-  const uint32_t full_b = empty_a + 8 * SA;
-  const uint32_t empty_b = full_b + 8 * SB;
-  const uint32_t full_c = empty_b + 8 * SB;
+  const uint32_t full_d = smem_u32(bars);
+  const uint32_t empty_d = full_d + 8 * SD;
+  const uint32_t full_t = empty_d + 8 * SD;
+  const uint32_t empty_t = full_t + 8 * ST;
+  const uint32_t full_c = empty_t + 8 * ST;
   const uint32_t empty_c = full_c + 8 * SC;
   const uint32_t acc_full = empty_c + 8 * SC;
   const uint32_t acc_empty = acc_full + 16;
   const uint32_t drain = acc_full + 32;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * (SA + SB + SC) + 5);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * (SD + ST + SC) + 5);
   volatile int* abort_word = reinterpret_cast<volatile int*>(tmem_holder + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < SA; ++s) { mbar_init(full_a + 8 * s, 1); mbar_init(empty_a + 8 * s, 1); }
-    for (int s = 0; s < SB; ++s) { mbar_init(full_b + 8 * s, NP); mbar_init(empty_b + 8 * s, 1); }
+    for (int s = 0; s < SD; ++s) { mbar_init(full_d + 8 * s, NP); mbar_init(empty_d + 8 * s, 1); }
+    for (int s = 0; s < ST; ++s) { mbar_init(full_t + 8 * s, 1); mbar_init(empty_t + 8 * s, 1); }
     for (int s = 0; s < SC; ++s) { mbar_init(full_c + 8 * s, 1); mbar_init(empty_c + 8 * s, NP); }
     for (int i = 0; i < 2; ++i) { mbar_init(acc_full + 8 * i, 1); mbar_init(acc_empty + 8 * i, 4); }
     mbar_init(drain, 1);
@@ -366,66 +384,83 @@ qgemm_dec_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     fence_mbar_init();
   }
   if (warp == 4 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    if (args.n_ext) tma_prefetch_desc(&tmAe);
+    tma_prefetch_desc(&tmT);
+    if (args.n_ext) tma_prefetch_desc(&tmTe);
   }
-  if (warp == 6 && lane == 0) {
-    tma_prefetch_desc(&tmCodes);
-    tma_prefetch_desc(&tmScale);
-  }
-  if (warp == 7 && lane == 0 && args.n_ext) tma_prefetch_desc(&tmBe);
+  if (warp == 6 && lane == 0) { tma_prefetch_desc(&tmCodes); tma_prefetch_desc(&tmScale); }
+  if (warp == 7 && lane == 0 && args.n_ext) tma_prefetch_desc(&tmWe);
   if (warp == 5) tmem_alloc(smem_u32(tmem_holder), Cfg::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  const int64_t n_tiles = (args.Cn + BN - 1) / BN;
-  const int64_t tiles = ((args.R + 127) / 128) * n_tiles;
+  // tiles: weight-row tiles fastest, so concurrently running CTAs share token tiles
+  const int64_t w_tiles = (args.R + BM - 1) / BM;
+  const int64_t tiles = w_tiles * ((args.Cn + BN - 1) / BN);
   const int kc_main = (int)((args.Kc + 63) / 64);
   const int kc_total = kc_main + args.n_ext;
   const uint64_t lim = args.timeout_ns;
 
   if (warp < 4) {
-    run_epilogue<BN, EPI>(args, tmem_base, acc_full, acc_empty, tiles, n_tiles, abort_word);
+    // ---- epilogue: 128 weight rows (TMEM lanes) x 256 tokens ----
+    uint32_t tcount = 0;
+    for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++tcount) {
+      const uint32_t acc = tcount & 1, aph = (tcount >> 1) & 1;
+      const bool okw = mbar_wait(acc_full + 8 * acc, aph, lim, abort_word);
+      if (!__all_sync(0xFFFFFFFFu, okw)) break;
+      tc_fence_after();
+      const int64_t w0 = (t % w_tiles) * BM, t0 = (t / w_tiles) * BN;
+      const int64_t wrow = w0 + warp * 32 + lane;
+#pragma unroll 1
+      for (int cc = 0; cc < BN; cc += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(warp * 32) << 16) + acc * BN + cc, v);
+        if (t0 + cc < args.Cn) epilogue_store_t(args, wrow, t0 + cc, v);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty + 8 * acc);
+    }
   } else if (warp == 4 && lane == 0) {
-    // ---- activation tiles (and the extension's left factor) -> A ring ----
+    // ---- token tiles -> T ring ----
     uint32_t g = 0;
     bool ok = true;
     for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-      const int32_t r0 = (int32_t)((t / n_tiles) * 128);
+      const int32_t t0 = (int32_t)((t / w_tiles) * BN);
       for (int kc = 0; kc < kc_total; ++kc, ++g) {
-        const uint32_t s = g % SA, ph = (g / SA) & 1;
-        if (!mbar_wait(empty_a + 8 * s, ph ^ 1, lim, abort_word)) { ok = false; break; }
-        const uint32_t fb = full_a + 8 * s;
-        mbar_arrive_expect_tx(fb, Cfg::kABytes);
-        if (kc < kc_main) tma_load_2d(smem_u32(sA + s * Cfg::kABytes), &tmA, fb, kc * 64, r0);
-        else tma_load_2d(smem_u32(sA + s * Cfg::kABytes), &tmAe, fb, (kc - kc_main) * 64, r0);
+        const uint32_t s = g % ST, ph = (g / ST) & 1;
+        if (!mbar_wait(empty_t + 8 * s, ph ^ 1, lim, abort_word)) { ok = false; break; }
+        const uint32_t fb = full_t + 8 * s;
+        mbar_arrive_expect_tx(fb, Cfg::kTBytes);
+        if (kc < kc_main) tma_load_2d(smem_u32(sT + s * Cfg::kTBytes), &tmT, fb, kc * 64, t0);
+        else tma_load_2d(smem_u32(sT + s * Cfg::kTBytes), &tmTe, fb, (kc - kc_main) * 64, t0);
       }
     }
     if (!ok || *abort_word)
-      for (uint32_t j = (g > (uint32_t)SA ? g - SA : 0); j < g; ++j) drain_wait(full_a + 8 * (j % SA), (j / SA) & 1);
+      for (uint32_t j = (g > (uint32_t)ST ? g - ST : 0); j < g; ++j) drain_wait(full_t + 8 * (j % ST), (j / ST) & 1);
   } else if (warp == 6 && lane == 0) {
-    // ---- weight codes + block scales -> C ring (main chunks only) ----
+    // ---- weight codes + block scales -> C ring ----
     uint32_t gc = 0;
     bool ok = true;
     for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-      const int32_t c0 = (int32_t)((t % n_tiles) * BN);
+      const int32_t w0 = (int32_t)((t % w_tiles) * BM);
       for (int kc = 0; kc < kc_main; ++kc, ++gc) {
         const uint32_t s = gc % SC, ph = (gc / SC) & 1;
         if (!mbar_wait(empty_c + 8 * s, ph ^ 1, lim, abort_word)) { ok = false; break; }
         const uint32_t fb = full_c + 8 * s;
         const uint32_t dst = smem_u32(sC + s * Cfg::kCBytes);
-        mbar_arrive_expect_tx(fb, Cfg::kCBytes);
-        if (!B_MN) {
-          // rows c0.. of the weight, k-block kc: codes box {bytes per block, 256 rows},
-          // scales from the block-major copy: 256 consecutive rows of block column kc
-          tma_load_2d(dst, &tmCodes, fb, kc * (BS == BSrc::NF4 ? 32 : 64), c0);
-          tma_load_2d(dst + Cfg::kCodeBytes, &tmScale, fb, c0, kc);
+        if (!W_MN) {
+          // weight rows w0..w0+128, block column kc
+          mbar_arrive_expect_tx(fb, Cfg::kCodeBytes + BM * 4);
+          tma_load_2d(dst, &tmCodes, fb, kc * (BS == BSrc::NF4 ? 32 : 64), w0);
+          tma_load_2d(dst + Cfg::kCodeBytes, &tmScale, fb, w0, kc);
         } else {
-          // weight rows kc*64 .. +64, weight columns c0 .. c0+256 (4 blocks per row)
-          tma_load_2d(dst, &tmCodes, fb, BS == BSrc::NF4 ? c0 / 2 : c0, kc * 64);
-          tma_load_2d(dst + Cfg::kCodeBytes, &tmScale, fb, c0 / 64, kc * 64);
+          // weight rows kc*64..+64, weight columns w0..w0+128 (2 blocks per row); the
+          // scale box starts at a multiple of 4 blocks (16-byte aligned) and spans 4
+          mbar_arrive_expect_tx(fb, Cfg::kCodeBytes + 1024);
+          tma_load_2d(dst, &tmCodes, fb, BS == BSrc::NF4 ? w0 / 2 : w0, kc * 64);
+          tma_load_2d(dst + Cfg::kCodeBytes, &tmScale, fb, (w0 / 64) & ~3, kc * 64);
         }
       }
     }
@@ -433,7 +468,7 @@ qgemm_dec_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       for (uint32_t j = (gc > (uint32_t)SC ? gc - SC : 0); j < gc; ++j) drain_wait(full_c + 8 * (j % SC), (j / SC) & 1);
   } else if (warp == 5 && lane == 0) {
     // ---- MMA issuer ----
-    constexpr uint32_t kIdMain = idesc_bf16_f32(128, BN, 0, B_MN ? 1 : 0);
+    constexpr uint32_t kIdMain = idesc_bf16_f32(128, BN, W_MN ? 1 : 0, 0);
     constexpr uint32_t kIdExt = idesc_bf16_f32(128, BN, 0, 0);
     uint32_t g = 0, tcount = 0;
     bool ok = true;
@@ -443,69 +478,66 @@ qgemm_dec_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + acc * BN;
       for (int kc = 0; kc < kc_total; ++kc, ++g) {
-        const uint32_t sa = g % SA, pa = (g / SA) & 1;
-        const uint32_t sb = g % SB, pb = (g / SB) & 1;
-        if (!mbar_wait(full_a + 8 * sa, pa, lim, abort_word)) { ok = false; break; }
-        if (!mbar_wait(full_b + 8 * sb, pb, lim, abort_word)) { ok = false; break; }
+        const uint32_t sd = g % SD, pd = (g / SD) & 1;
+        const uint32_t st = g % ST, pt = (g / ST) & 1;
+        if (!mbar_wait(full_t + 8 * st, pt, lim, abort_word)) { ok = false; break; }
+        if (!mbar_wait(full_d + 8 * sd, pd, lim, abort_word)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t a_base = smem_u32(sA + sa * Cfg::kABytes);
-        const uint32_t b_base = smem_u32(sB + sb * Cfg::kBBytes);
+        const uint32_t d_base = smem_u32(sD + sd * Cfg::kDBytes);
+        const uint32_t t_base = smem_u32(sT + st * Cfg::kTBytes);
         const bool ext = kc >= kc_main;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const uint64_t ad = smem_desc_sw128(a_base + k * 32, 16, 1024);
-          const uint64_t bd = (!B_MN || ext) ? smem_desc_sw128(b_base + k * 32, 16, 1024)
-                                             : smem_desc_sw128(b_base + k * 2048, 8192, 1024);
+          const uint64_t ad = (!W_MN || ext) ? smem_desc_sw128(d_base + k * 32, 16, 1024)
+                                             : smem_desc_sw128(d_base + k * 2048, 8192, 1024);
+          const uint64_t bd = smem_desc_sw128(t_base + k * 32, 16, 1024);
           tc_mma(d_tmem, ad, bd, ext ? kIdExt : kIdMain, (kc > 0 || k > 0) ? 1u : 0u);
         }
-        tc_commit(empty_a + 8 * sa);
-        tc_commit(empty_b + 8 * sb);
+        tc_commit(empty_d + 8 * sd);
+        tc_commit(empty_t + 8 * st);
       }
       if (!ok) break;
       tc_commit(acc_full + 8 * acc);
     }
     if (!ok || *abort_word) { tc_commit(drain); drain_wait(drain, 0); }
   } else if (warp >= 7) {
-    // ---- decode: C ring (codes, scales) -> B ring (bf16, swizzled UMMA layout) ----
-    const int tid = threadIdx.x - 7 * 32;
+    // ---- decode: C ring -> D ring (bf16, swizzled UMMA layout), two lanes per block ----
+    const int tid = threadIdx.x - 7 * 32;                        // 0..255
+    const int blk = tid >> 1, half = tid & 1;                    // block 0..127
     float q[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) q[i] = args.q[i];
-    // where this thread's block sits in the C stage and in the B tile
-    int code_off, scale_idx;
-    uint32_t b_off, key;
-    if (!B_MN) {
-      code_off = tid * (BS == BSrc::NF4 ? 32 : 64);
-      scale_idx = tid;
-      b_off = tid * 128;
-      key = tid & 7;
+    int code_off, j_row = 0, gi = 0;
+    uint32_t d_off, key;
+    if (!W_MN) {
+      code_off = blk * (BS == BSrc::NF4 ? 32 : 64);
+      d_off = blk * 128;
+      key = blk & 7;
     } else {
-      const int j = tid & 63, gi = tid >> 6;
-      code_off = j * (BS == BSrc::NF4 ? 128 : 256) + gi * (BS == BSrc::NF4 ? 32 : 64);
-      scale_idx = j * 4 + gi;
-      b_off = gi * 8192 + (j >> 3) * 1024 + (j & 7) * 128;
-      key = j & 7;
+      j_row = blk & 63;
+      gi = blk >> 6;
+      code_off = j_row * (BS == BSrc::NF4 ? 64 : 128) + gi * (BS == BSrc::NF4 ? 32 : 64);
+      d_off = gi * 8192 + (j_row >> 3) * 1024 + (j_row & 7) * 128;
+      key = j_row & 7;
     }
-    // The decode warps are the only producers of the B ring, extension stages included
-    // (one of them issues that stage's TMA), so every producer of a stage has waited on
-    // every earlier phase of it and the parity waits stay exact.
-    uint32_t gc = 0, gb = 0, gx = 0, last_sb = 0, last_pb = 0;
-    bool ok = true;
+    uint32_t gc = 0, gd = 0, last_sd = 0, last_pd = 0;
+    bool ok = true, ext_issued = false;
     for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-      const int32_t c0 = (int32_t)((t % n_tiles) * BN);
-      for (int kc = 0; kc < kc_total; ++kc, ++gb) {
-        const uint32_t sb = gb % SB, pb = (gb / SB) & 1;
+      const int32_t w0 = (int32_t)((t % w_tiles) * BM);
+      const int scale_idx = !W_MN ? blk : j_row * 4 + ((w0 / 64) & 3) + gi;
+      for (int kc = 0; kc < kc_total; ++kc, ++gd) {
+        const uint32_t sd = gd % SD, pd = (gd / SD) & 1;
         if (kc >= kc_main) {
-          const bool wb = mbar_wait(empty_b + 8 * sb, pb ^ 1, lim, abort_word);
+          const bool wb = mbar_wait(empty_d + 8 * sd, pd ^ 1, lim, abort_word);
           if (!__all_sync(0xFFFFFFFFu, wb)) { ok = false; break; }
           if (lane == 0) {
-            const uint32_t fb = full_b + 8 * sb;
+            const uint32_t fb = full_d + 8 * sd;
             if (warp == 7) {
-              mbar_arrive_expect_tx(fb, Cfg::kBBytes);
-              tma_load_2d(smem_u32(sB + sb * Cfg::kBBytes), &tmBe, fb, (kc - kc_main) * 64, c0);
-              ++gx;
-              last_sb = sb;
-              last_pb = pb;
+              mbar_arrive_expect_tx(fb, Cfg::kDBytes);
+              tma_load_2d(smem_u32(sD + sd * Cfg::kDBytes), &tmWe, fb, (kc - kc_main) * 64, w0);
+              ext_issued = true;
+              last_sd = sd;
+              last_pd = pd;
             } else {
               mbar_arrive(fb);
             }
@@ -514,44 +546,41 @@ qgemm_dec_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         }
         const uint32_t sc = gc % SC, pc = (gc / SC) & 1;
         const bool w1 = mbar_wait(full_c + 8 * sc, pc, lim, abort_word);
-        const bool w2 = w1 && mbar_wait(empty_b + 8 * sb, pb ^ 1, lim, abort_word);
+        const bool w2 = w1 && mbar_wait(empty_d + 8 * sd, pd ^ 1, lim, abort_word);
         if (!__all_sync(0xFFFFFFFFu, w2)) { ok = false; break; }
         const uint8_t* cst = sC + sc * Cfg::kCBytes;
         const float sv = reinterpret_cast<const float*>(cst + Cfg::kCodeBytes)[scale_idx];
-        uint4* d = reinterpret_cast<uint4*>(sB + sb * Cfg::kBBytes + b_off);
+        uint4* d = reinterpret_cast<uint4*>(sD + sd * Cfg::kDBytes + d_off);
         if constexpr (BS == BSrc::NF4) {
-          const uint4* src = reinterpret_cast<const uint4*>(cst + code_off);
-          const uint4 c0v = src[0], c1v = src[1];
+          const uint4 cv = reinterpret_cast<const uint4*>(cst + code_off)[half];
           uint32_t L[2], H[2];
           nf4_table(q, sv, L, H);
-          d[0 ^ key] = nf4_decode8(c0v.x, L, H);
-          d[1 ^ key] = nf4_decode8(c0v.y, L, H);
-          d[2 ^ key] = nf4_decode8(c0v.z, L, H);
-          d[3 ^ key] = nf4_decode8(c0v.w, L, H);
-          d[4 ^ key] = nf4_decode8(c1v.x, L, H);
-          d[5 ^ key] = nf4_decode8(c1v.y, L, H);
-          d[6 ^ key] = nf4_decode8(c1v.z, L, H);
-          d[7 ^ key] = nf4_decode8(c1v.w, L, H);
+          const int c0i = 4 * half;
+          d[(c0i + 0) ^ key] = nf4_decode8(cv.x, L, H);
+          d[(c0i + 1) ^ key] = nf4_decode8(cv.y, L, H);
+          d[(c0i + 2) ^ key] = nf4_decode8(cv.z, L, H);
+          d[(c0i + 3) ^ key] = nf4_decode8(cv.w, L, H);
         } else {
-          const uint4* src = reinterpret_cast<const uint4*>(cst + code_off);
+          const uint4* src = reinterpret_cast<const uint4*>(cst + code_off) + 2 * half;
 #pragma unroll
-          for (int h = 0; h < 4; ++h) {
+          for (int h = 0; h < 2; ++h) {
             const uint4 w = src[h];
-            d[(2 * h) ^ key] = int8_decode8(w.x, w.y, sv);
-            d[(2 * h + 1) ^ key] = int8_decode8(w.z, w.w, sv);
+            const int c = 4 * half + 2 * h;
+            d[c ^ key] = int8_decode8(w.x, w.y, sv);
+            d[(c + 1) ^ key] = int8_decode8(w.z, w.w, sv);
           }
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(full_b + 8 * sb);
+          mbar_arrive(full_d + 8 * sd);
           mbar_arrive(empty_c + 8 * sc);
         }
         ++gc;
       }
     }
-    if ((!ok || *abort_word) && warp == 7 && lane == 0 && gx)
-      drain_wait(full_b + 8 * last_sb, last_pb);       // our last extension copy (bounded)
+    if ((!ok || *abort_word) && warp == 7 && lane == 0 && ext_issued)
+      drain_wait(full_d + 8 * last_sd, last_pd);       // our last extension copy (bounded)
   }
 
   __syncwarp();

@@ -82,18 +82,18 @@ static ql_status launch_tma_rp(int rp, const CUtensorMap& a, const CUtensorMap& 
   return launch_tma<256, A_MN, B_MN, EPI>(a, b, args, st);
 }
 
-template <BSrc BS, bool B_MN, int EPI>
-static ql_status launch_dec(const CUtensorMap& a, const CUtensorMap& codes, const CUtensorMap& scale,
-                            const CUtensorMap& ae, const CUtensorMap& be, const GemmArgs& args,
-                            cudaStream_t st) {
-  auto kern = qgemm_dec_kernel<BS, B_MN, EPI>;
-  const size_t smem = DecCfg<BS>::kSmem;
+template <BSrc BS, bool W_MN>
+static ql_status launch_wdec(const CUtensorMap& tok, const CUtensorMap& codes, const CUtensorMap& scale,
+                             const CUtensorMap& tok_ext, const CUtensorMap& w_ext, const GemmArgs& args,
+                             cudaStream_t st) {
+  auto kern = qgemm_wdec_kernel<BS, W_MN>;
+  const size_t smem = WdecCfg<BS>::kSmem;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return QL_ERR_CUDA;
   const int64_t tiles = ((args.R + 127) / 128) * ((args.Cn + 255) / 256);
   const int grid = (int)imin64(tiles, num_sms());
   if (grid <= 0) return QL_OK;
-  kern<<<grid, DecCfg<BS>::kThreads, smem, st>>>(a, codes, scale, ae, be, args);
+  kern<<<grid, WdecCfg<BS>::kThreads, smem, st>>>(tok, codes, scale, tok_ext, w_ext, args);
   QL_CHECK_LAUNCH();
   return QL_OK;
 }
@@ -203,23 +203,24 @@ static GemmArgs base_args() {
   return a;
 }
 
-// Tensor maps of the quantised weight for the decode GEMM. Forward (transposed = false):
-// codes box {bytes per block, 256 rows}, scales from the block-major copy, box {256, 1}.
-// dX (transposed = true): codes box {4 blocks of bytes, 64 rows}, scales row-major, box {4, 64}.
+// Tensor maps of the quantised weight for the decode GEMM (tiles of 128 weight rows).
+// Forward: codes box {bytes per block, 128 rows}, scales from the block-major copy, box
+// {128, 1}. dX: codes box {2 blocks of bytes, 64 rows}, scales row-major, box {4, 64}
+// (the kernel starts it at a multiple of 4 blocks to keep TMA coordinates aligned).
 static bool make_weight_maps(const ql_weight* w, const float* scales, bool transposed,
-                             CUtensorMap* mc, CUtensorMap* ms) {
+                                  CUtensorMap* mc, CUtensorMap* ms) {
   const int64_t N = w->N, K = w->K, KB = K / 64;
   const bool nf4 = w->fmt == QL_FMT_NF4_DQ;
   const uint64_t row_bytes = nf4 ? K / 2 : K;
   const uint32_t blk_bytes = nf4 ? 32 : 64;
   if (!transposed) {
     return make_map_t(mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, row_bytes, N, row_bytes, blk_bytes,
-                      256, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-           make_map_t(ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, scales, N, KB, N * 4, 256, 1,
+                      128, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+           make_map_t(ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, scales, N, KB, N * 4, 128, 1,
                       CU_TENSOR_MAP_SWIZZLE_NONE);
   }
   const int64_t ld = round_up(KB, 4);
-  return make_map_t(mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, row_bytes, N, row_bytes, 4 * blk_bytes,
+  return make_map_t(mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, w->codes, row_bytes, N, row_bytes, 2 * blk_bytes,
                     64, CU_TENSOR_MAP_SWIZZLE_NONE) &&
          make_map_t(ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, scales, KB, N, ld * 4, 4, 64,
                     CU_TENSOR_MAP_SWIZZLE_NONE);
@@ -287,10 +288,10 @@ ql_status qlora_linear_fwd(const ql_weight* w, const ql_bf16* X, int64_t M, cons
   uint16_t* Bp = reinterpret_cast<uint16_t*>(wsb + L.off[1]);
   float* scales = reinterpret_cast<float*>(wsb + L.off[4]);
 
-  CUtensorMap mX, mA, mP, mBp, mc, ms;
-  if (!make_map(&mX, X, K, M, K, 128) || !make_map(&mA, A, K, r, K, rp) ||
-      !make_map(&mP, P, rp, M, rp, 128) || !make_map(&mBp, Bp, rp, N, rp, 256) ||
-      !make_weight_maps(w, scales, false, &mc, &ms))
+  CUtensorMap mX, mX256, mA, mP256, mBp, mc, ms;
+  if (!make_map(&mX, X, K, M, K, 128) || !make_map(&mX256, X, K, M, K, 256) ||
+      !make_map(&mA, A, K, r, K, rp) || !make_map(&mP256, P, rp, M, rp, 256) ||
+      !make_map(&mBp, Bp, rp, N, rp, 128) || !make_weight_maps(w, scales, false, &mc, &ms))
     return QL_ERR_CUDA;
 
   {
@@ -312,13 +313,13 @@ ql_status qlora_linear_fwd(const ql_weight* w, const ql_bf16* X, int64_t M, cons
   }
   if (e != QL_OK) return e;
 
-  // Y = X W'^T + P Bp^T
+  // Y^T = W' X^T + Bp P^T  (weight rows as the MMA's M, tokens as its N)
   GemmArgs y = base_args();
-  y.R = M; y.Cn = N; y.Kc = K; y.n_ext = rp / 64; y.r = r;
+  y.R = N; y.Cn = M; y.Kc = K; y.n_ext = rp / 64; y.r = r;
   y.out = Y; y.ld_out = N; y.scale = 1.0f;
   ProfScope prof(PK_FWD_MAIN, st, 1);
-  if (w->fmt == QL_FMT_NF4_DQ) return launch_dec<BSrc::NF4, false, EPI_BF16>(mX, mc, ms, mP, mBp, y, st);
-  return launch_dec<BSrc::INT8, false, EPI_BF16>(mX, mc, ms, mP, mBp, y, st);
+  if (w->fmt == QL_FMT_NF4_DQ) return launch_wdec<BSrc::NF4, false>(mX256, mc, ms, mP256, mBp, y, st);
+  return launch_wdec<BSrc::INT8, false>(mX256, mc, ms, mP256, mBp, y, st);
 }
 
 ql_status qlora_linear_bwd(const ql_weight* w, const ql_bf16* X, const ql_bf16* dY, int64_t M,
@@ -346,9 +347,10 @@ ql_status qlora_linear_bwd(const ql_weight* w, const ql_bf16* X, const ql_bf16* 
   uint16_t* Tp = reinterpret_cast<uint16_t*>(wsb + L.off[3]);
   float* scales = reinterpret_cast<float*>(wsb + L.off[4]);
 
-  CUtensorMap mdY_k, mBt, mQ_k, mAt, mdY_mn, mTp_mn, mX_mn, mQ_mn, mc, ms;
-  if (!make_map(&mdY_k, dY, N, M, N, 128) || !make_map(&mBt, Bt, N, r, N, rp) ||
-      !make_map(&mQ_k, Q, rp, M, rp, 128) || !make_map(&mAt, At, rp, K, rp, 256) ||
+  CUtensorMap mdY_k, mdY256, mBt, mQ256, mAt, mdY_mn, mTp_mn, mX_mn, mQ_mn, mc, ms;
+  if (!make_map(&mdY_k, dY, N, M, N, 128) || !make_map(&mdY256, dY, N, M, N, 256) ||
+      !make_map(&mBt, Bt, N, r, N, rp) ||
+      !make_map(&mQ256, Q, rp, M, rp, 256) || !make_map(&mAt, At, rp, K, rp, 128) ||
       !make_map(&mdY_mn, dY, N, M, N, 64) || !make_map(&mTp_mn, Tp, rp, M, rp, 64) ||
       !make_map(&mX_mn, X, K, M, K, 64) || !make_map(&mQ_mn, Q, rp, M, rp, 64) ||
       !make_weight_maps(w, scales, true, &mc, &ms))
@@ -394,12 +396,12 @@ ql_status qlora_linear_bwd(const ql_weight* w, const ql_bf16* X, const ql_bf16* 
   }
   if (e != QL_OK) return e;
 
-  // dX = dY W' + Q A^T-padded
+  // dX^T = W'^T dY^T + A^T-padded Q^T  (input features as the MMA's M, tokens as its N)
   GemmArgs x = base_args();
-  x.R = M; x.Cn = K; x.Kc = N; x.n_ext = rp / 64; x.r = r; x.out = dX; x.ld_out = K; x.scale = 1.0f;
+  x.R = K; x.Cn = M; x.Kc = N; x.n_ext = rp / 64; x.r = r; x.out = dX; x.ld_out = K; x.scale = 1.0f;
   ProfScope prof(PK_BWD_DX, st, 1);
-  if (w->fmt == QL_FMT_NF4_DQ) return launch_dec<BSrc::NF4, true, EPI_BF16>(mdY_k, mc, ms, mQ_k, mAt, x, st);
-  return launch_dec<BSrc::INT8, true, EPI_BF16>(mdY_k, mc, ms, mQ_k, mAt, x, st);
+  if (w->fmt == QL_FMT_NF4_DQ) return launch_wdec<BSrc::NF4, true>(mdY256, mc, ms, mQ256, mAt, x, st);
+  return launch_wdec<BSrc::INT8, true>(mdY256, mc, ms, mQ256, mAt, x, st);
 }
 
 }  // extern "C"
