@@ -27,6 +27,7 @@ ql_status small_m_forward(const ql_weight* w, const uint16_t* X, int64_t M, cons
                           const uint16_t* B, int r, float alpha, uint16_t* Y, uint16_t* T_save,
                           cudaStream_t st);
 constexpr int64_t kSmallMMax = 16;
+bool small_m_supported(int64_t K, int r);   // rank <= 64 and the staging fits in shared memory
 int* device_flag_ptr();                 // device address of the sticky flag (current device)
 int num_sms();                          // SM count of the current device
 

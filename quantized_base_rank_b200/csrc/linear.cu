@@ -257,7 +257,7 @@ extern "C" {
 size_t ql_workspace_bytes(int32_t op, int64_t M, int64_t N, int64_t K, int32_t r) {
   if (op == QL_OP_DQ) return 256;
   if ((op != QL_OP_FWD && op != QL_OP_BWD) || M < 0 || N < 0 || K < 0 || r < 1 || r > 256) return 0;
-  if (op == QL_OP_FWD && M <= kSmallMMax) return 0;      // the decode-shaped path needs none
+  if (op == QL_OP_FWD && M <= kSmallMMax && small_m_supported(K, r)) return 0;   // decode-shaped path
   return (size_t)ws_layout(op, M, N, K, r).total;
 }
 
@@ -275,10 +275,10 @@ ql_status qlora_linear_fwd(const ql_weight* w, const ql_bf16* X, int64_t M, cons
   if (!aligned(X, 16) || !aligned(A, 16) || !aligned(B, 2) || !aligned(Y, 16) ||
       (T_save && !aligned(T_save, 2)))
     return QL_ERR_INVALID_ARG;
-  if (M > kSmallMMax && (!ws || !aligned(ws, 256))) return QL_ERR_INVALID_ARG;
+  if (!(M <= kSmallMMax && small_m_supported(w->K, r)) && (!ws || !aligned(ws, 256))) return QL_ERR_INVALID_ARG;
   const int64_t N = w->N, K = w->K;
   cudaStream_t st = as_stream(stream);
-  if (M <= kSmallMMax) return small_m_forward(w, X, M, A, B, r, alpha, Y, T_save, st);
+  if (M <= kSmallMMax && small_m_supported(w->K, r)) return small_m_forward(w, X, M, A, B, r, alpha, Y, T_save, st);
   const WsLayout L = ws_layout(QL_OP_FWD, M, N, K, r);
   if ((int64_t)ws_bytes < L.total) return QL_ERR_WORKSPACE;
   const int rp = (int)round_up(r, 64);

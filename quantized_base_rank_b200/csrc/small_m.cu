@@ -12,8 +12,9 @@
 //    (W' rows x k), with X as the 8-token B operand. The contraction order is permuted
 //    consistently for both operands (step s of a unit uses k = 64q + 4s + {0..3}), so a
 //    lane's 64 elements of a block come from one 32-byte code row and one table;
-//  - the adapter term enters per K-range by linearity: each CTA forms T_kr = X_kr A_kr^T
-//    and adds B (s T_kr) to its partial sums;
+//  - the adapter term enters per K-range by linearity: T_kr = X_kr A_kr^T is formed in the
+//    same loop from the same token fragments (adapter rows staged like the tokens), and
+//    B (s T_kr) is added to the partial sums;
 //  - the 8 partial sums of a row group are reduced in fixed rank order through
 //    distributed shared memory, so the result is deterministic and no workspace or atomic
 //    is needed. T = sum of the T_kr is reduced the same way for T_save.
@@ -138,6 +139,9 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// Read a float from the same shared-memory offset in CTA `rank` of the cluster. The loads
+// stay in program order after the cluster barrier; callers issue several before using any,
+// so they are in flight together.
 __device__ __forceinline__ float ld_cluster_f32(const float* local, uint32_t rank) {
   uint32_t addr = static_cast<uint32_t>(__cvta_generic_to_shared(local)), remote;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(addr), "r"(rank));
@@ -146,100 +150,127 @@ __device__ __forceinline__ float ld_cluster_f32(const float* local, uint32_t ran
   return v;
 }
 
-template <int NT, int FMT>
-__global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(256)
+// Shared-memory layout of the token rows and adapter rows of a CTA's K-range: the four
+// elements a lane feeds to one MMA step (k = 64q + 4s + e of unit ul) are 8 contiguous
+// bytes at  row * kRowPitch(units) + ul * 512 + (4s + q) * 8.  With a row pitch of 32 mod 128
+// bytes, the 16 lanes of a half-warp (rows g = 0..3, q = 0..3) hit 16 different bank pairs.
+__host__ __device__ __forceinline__ int small_row_pitch(int units) { return units * 512 + 32; }
+
+template <int NT, int FMT, int JT>
+__global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(256, 2)
 small_m_fwd_kernel(const SmallArgs a) {
   constexpr int NTT = NT / 8;                       // token tiles of 8
+  constexpr int RP = JT * 16;                       // rank padded to j-tiles of 16
   extern __shared__ __align__(16) uint8_t sm[];
-  const int RP = (a.r + 15) & ~15;                  // rank padded to the j-tile of 16
-  uint16_t* sX = reinterpret_cast<uint16_t*>(sm);   // [NT][kr_max] bf16
-  float* sTp = reinterpret_cast<float*>(sm + (size_t)NT * a.kr_max * 2);   // [8 warps][RP][NT]
-  float* sT = sTp + 8 * RP * NT;                    // [RP][NT] this CTA's T_kr
-  float* sD = sT + RP * NT;                         // [128 rows][NT] partial Y
+  const int64_t U = (a.K + 255) / 256;
+  const int units_max = (int)((U + kCS - 1) / kCS);
+  const int pitch = small_row_pitch(units_max);
+  uint8_t* sX = sm;                                 // [NT][pitch]
+  uint8_t* sA = sX + (size_t)NT * pitch;            // [RP][pitch]
+  float* sTw = reinterpret_cast<float*>(sA + (size_t)RP * pitch);   // [8 warps][RP][NT]
+  float* sD = sTw + 8 * RP * NT;                    // [128 rows][NT] partial Y
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, q = lane & 3;
   const uint32_t rank = cluster_rank();
   const int64_t n0 = (int64_t)(blockIdx.x / kCS) * kRowsPerCta;
-  const int64_t U = (a.K + 255) / 256;
   const int64_t u0 = rank * U / kCS, u1 = (rank + 1) * U / kCS;
+  const int nunits = (int)(u1 - u0);
   const int64_t k0 = u0 * 256;
-  const int kr = (int)((u1 - u0) * 256);
   const float mu = FMT == QL_FMT_NF4_DQ ? __ldg(a.mean) : 0.0f;
 
-  // first unit's codes go out before anything else
+  // The next launch on the stream may start now; it will stream its own weight while we
+  // finish. Everything below that reads X, A or B waits for the previous grid first.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  // first unit's codes go out before anything else (weights are never written by the
+  // preceding grid, so they may be read before the dependency wait)
   const int64_t row_g = n0 + warp * 16 + g, row_h = row_g + 8;
   UnitRegs<FMT> cg, ch;
-  if (u0 < u1) {
+  if (nunits > 0) {
     load_block_regs<FMT>(a, row_g, u0 * 4 + q, mu, cg);
     load_block_regs<FMT>(a, row_h, u0 * 4 + q, mu, ch);
   }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  // X[:, k0 : k0 + kr] -> smem, zero beyond M and K
-  for (int i = threadIdx.x; i < NT * kr / 8; i += blockDim.x) {
-    const int tok = i / (kr / 8), kk = (i % (kr / 8)) * 8;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    const int64_t k = k0 + kk;
-    if (tok < a.M && k < a.K) v = *reinterpret_cast<const uint4*>(a.X + tok * a.K + k);
-    *reinterpret_cast<uint4*>(sX + (size_t)tok * a.kr_max + kk) = v;
+  // token rows and adapter rows of the K-range -> smem in fragment order (zero beyond the
+  // tokens, the rank and K): one 16-byte global load feeds two 8-byte fragment slots
+  {
+    const int per_row = nunits * 32;                // 16-byte vectors per row
+    const int total = (NT + RP) * per_row;
+    for (int v = threadIdx.x; v < total; v += blockDim.x) {
+      const int row = v / per_row, rem = v % per_row;
+      const int ul = rem >> 5, qq = (rem >> 3) & 3, ii = rem & 7;
+      const int64_t k = k0 + ul * 256 + 64 * qq + 8 * ii;
+      uint4 val = make_uint4(0u, 0u, 0u, 0u);
+      uint8_t* base;
+      if (row < NT) {
+        if (row < a.M && k < a.K) val = *reinterpret_cast<const uint4*>(a.X + row * a.K + k);
+        base = sX + (size_t)row * pitch;
+      } else {
+        const int j = row - NT;
+        if (j < a.r && k < a.K) val = *reinterpret_cast<const uint4*>(a.A + j * a.K + k);
+        base = sA + (size_t)j * pitch;
+      }
+      uint8_t* p = base + ul * 512;
+      *reinterpret_cast<uint2*>(p + ((2 * ii) * 4 + qq) * 8) = make_uint2(val.x, val.y);
+      *reinterpret_cast<uint2*>(p + ((2 * ii + 1) * 4 + qq) * 8) = make_uint2(val.z, val.w);
+    }
+  }
+  // adapter right factor for this warp's rows (A fragments of the final MMA)
+  auto bload = [&](int64_t row, int j) -> uint32_t {
+    if (row >= a.N) return 0u;
+    const uint32_t lo = j < a.r ? a.B[row * a.r + j] : 0u;
+    const uint32_t hi = j + 1 < a.r ? a.B[row * a.r + j + 1] : 0u;
+    return lo | (hi << 16);
+  };
+  uint32_t bfr[JT][4];
+#pragma unroll
+  for (int jt = 0; jt < JT; ++jt) {
+    {
+      const int j0 = jt * 16 + 2 * q;
+      bfr[jt][0] = bload(row_g, j0);
+      bfr[jt][1] = bload(row_h, j0);
+      bfr[jt][2] = bload(row_g, j0 + 8);
+      bfr[jt][3] = bload(row_h, j0 + 8);
+    }
   }
   __syncthreads();
 
-  // ---- T_kr = X_kr A_kr^T, k16 steps split over the 8 warps ----
-  for (int jt = 0; jt < RP / 16; ++jt) {
-    float dt[NTT][4];
+  // ---- main loop: W' rows (decoded) and, for the adapter, A rows against the tokens ----
+  float d[NTT][4];
+  float dt[JT][NTT][4];                              // T_kr = X_kr A_kr^T, per j-tile
 #pragma unroll
-    for (int t = 0; t < NTT; ++t) dt[t][0] = dt[t][1] = dt[t][2] = dt[t][3] = 0.0f;
-    const int j_g = jt * 16 + g, j_h = j_g + 8;
-    for (int st = warp; st < kr / 16; st += 8) {
-      const int kl = st * 16 + 2 * q;
-      const int64_t k = k0 + kl;
-      uint32_t av[4] = {0u, 0u, 0u, 0u};
-      if (k < a.K) {
-        if (j_g < a.r) {
-          av[0] = *reinterpret_cast<const uint32_t*>(a.A + j_g * a.K + k);
-          av[2] = *reinterpret_cast<const uint32_t*>(a.A + j_g * a.K + k + 8);
-        }
-        if (j_h < a.r) {
-          av[1] = *reinterpret_cast<const uint32_t*>(a.A + j_h * a.K + k);
-          av[3] = *reinterpret_cast<const uint32_t*>(a.A + j_h * a.K + k + 8);
-        }
-      }
+  for (int t = 0; t < NTT; ++t) {
+    d[t][0] = d[t][1] = d[t][2] = d[t][3] = 0.0f;
+#pragma unroll
+    for (int jt = 0; jt < JT; ++jt) dt[jt][t][0] = dt[jt][t][1] = dt[jt][t][2] = dt[jt][t][3] = 0.0f;
+  }
+  for (int ul = 0; ul < nunits; ++ul) {
+    UnitRegs<FMT> ng, nh;
+    if (ul + 1 < nunits) {
+      load_block_regs<FMT>(a, row_g, (u0 + ul + 1) * 4 + q, mu, ng);
+      load_block_regs<FMT>(a, row_h, (u0 + ul + 1) * 4 + q, mu, nh);
+    }
+    const uint8_t* xu = sX + ul * 512 + q * 8;
+    const uint8_t* au = sA + ul * 512 + q * 8;
+    auto step = [&](int s, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
+      uint2 bx[NTT];
 #pragma unroll
       for (int t = 0; t < NTT; ++t) {
-        const uint16_t* xr = sX + (size_t)(t * 8 + g) * a.kr_max + kl;
-        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(xr);
-        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(xr + 8);
-        mma_bf16_16816(dt[t], av[0], av[1], av[2], av[3], b0, b1);
+        bx[t] = *reinterpret_cast<const uint2*>(xu + (size_t)(t * 8 + g) * pitch + s * 32);
+        mma_bf16_16816(d[t], a0, a1, a2, a3, bx[t].x, bx[t].y);
       }
-    }
 #pragma unroll
-    for (int t = 0; t < NTT; ++t) {
-      float* p = sTp + ((size_t)warp * RP) * NT;
-      p[(j_g)*NT + t * 8 + 2 * q] = dt[t][0];
-      p[(j_g)*NT + t * 8 + 2 * q + 1] = dt[t][1];
-      p[(j_h)*NT + t * 8 + 2 * q] = dt[t][2];
-      p[(j_h)*NT + t * 8 + 2 * q + 1] = dt[t][3];
-    }
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < RP * NT; i += blockDim.x) {
-    float acc = 0.0f;
-    for (int w = 0; w < 8; ++w) acc += sTp[(size_t)w * RP * NT + i];
-    sT[i] = acc;
-  }
-
-  // ---- main loop: decode into A fragments, X from smem as the B fragments ----
-  float d[NTT][4];
+      for (int jt = 0; jt < JT; ++jt) {
+        {
+          const uint2 ag = *reinterpret_cast<const uint2*>(au + (size_t)(jt * 16 + g) * pitch + s * 32);
+          const uint2 ah = *reinterpret_cast<const uint2*>(au + (size_t)(jt * 16 + g + 8) * pitch + s * 32);
 #pragma unroll
-  for (int t = 0; t < NTT; ++t) d[t][0] = d[t][1] = d[t][2] = d[t][3] = 0.0f;
-  for (int64_t u = u0; u < u1; ++u) {
-    UnitRegs<FMT> ng, nh;
-    if (u + 1 < u1) {
-      load_block_regs<FMT>(a, row_g, (u + 1) * 4 + q, mu, ng);
-      load_block_regs<FMT>(a, row_h, (u + 1) * 4 + q, mu, nh);
-    }
-    const uint16_t* xb = sX + (u - u0) * 256 + 64 * q;
+          for (int t = 0; t < NTT; ++t) mma_bf16_16816(dt[jt][t], ag.x, ah.x, ag.y, ah.y, bx[t].x, bx[t].y);
+        }
+      }
+    };
     if constexpr (FMT == QL_FMT_NF4_DQ) {
       uint32_t Lg[2], Hg[2], Lh[2], Hh[2];
       small_nf4_table(a.q, cg.sc, Lg, Hg);
@@ -250,17 +281,8 @@ small_m_fwd_kernel(const SmallArgs a) {
       for (int w8 = 0; w8 < 8; ++w8) {
         const uint4 eg = small_nf4_decode8(wg[w8], Lg, Hg);
         const uint4 eh = small_nf4_decode8(wh[w8], Lh, Hh);
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int s = 2 * w8 + half;
-          const uint32_t a0 = half ? eg.z : eg.x, a2 = half ? eg.w : eg.y;
-          const uint32_t a1 = half ? eh.z : eh.x, a3 = half ? eh.w : eh.y;
-#pragma unroll
-          for (int t = 0; t < NTT; ++t) {
-            const uint2 bx = *reinterpret_cast<const uint2*>(xb + (size_t)(t * 8 + g) * a.kr_max + 4 * s);
-            mma_bf16_16816(d[t], a0, a1, a2, a3, bx.x, bx.y);
-          }
-        }
+        step(2 * w8, eg.x, eh.x, eg.y, eh.y);
+        step(2 * w8 + 1, eg.z, eh.z, eg.w, eh.w);
       }
     } else {
       const uint32_t wg[16] = {cg.c[0].x, cg.c[0].y, cg.c[0].z, cg.c[0].w, cg.c[1].x, cg.c[1].y, cg.c[1].z, cg.c[1].w,
@@ -268,37 +290,43 @@ small_m_fwd_kernel(const SmallArgs a) {
       const uint32_t wh[16] = {ch.c[0].x, ch.c[0].y, ch.c[0].z, ch.c[0].w, ch.c[1].x, ch.c[1].y, ch.c[1].z, ch.c[1].w,
                                ch.c[2].x, ch.c[2].y, ch.c[2].z, ch.c[2].w, ch.c[3].x, ch.c[3].y, ch.c[3].z, ch.c[3].w};
 #pragma unroll
-      for (int s = 0; s < 16; ++s) {
-        const uint2 eg = small_int8_decode4(wg[s], cg.sc);
-        const uint2 eh = small_int8_decode4(wh[s], ch.sc);
-#pragma unroll
-        for (int t = 0; t < NTT; ++t) {
-          const uint2 bx = *reinterpret_cast<const uint2*>(xb + (size_t)(t * 8 + g) * a.kr_max + 4 * s);
-          mma_bf16_16816(d[t], eg.x, eh.x, eg.y, eh.y, bx.x, bx.y);
-        }
+      for (int st = 0; st < 16; ++st) {
+        const uint2 eg = small_int8_decode4(wg[st], cg.sc);
+        const uint2 eh = small_int8_decode4(wh[st], ch.sc);
+        step(st, eg.x, eh.x, eg.y, eh.y);
       }
     }
-    if (u + 1 < u1) { cg = ng; ch = nh; }
+    if (ul + 1 < nunits) { cg = ng; ch = nh; }
   }
 
   // ---- adapter term of this K-range: D += B[rows, :] (s T_kr) ----
-  __syncthreads();
-  for (int jt = 0; jt < RP / 16; ++jt) {
-    const int j0 = jt * 16 + 2 * q;
-    auto bload = [&](int64_t row, int j) -> uint32_t {
-      if (row >= a.N) return 0u;
-      const uint32_t lo = j < a.r ? a.B[row * a.r + j] : 0u;
-      const uint32_t hi = j + 1 < a.r ? a.B[row * a.r + j + 1] : 0u;
-      return lo | (hi << 16);
-    };
-    const uint32_t a0 = bload(row_g, j0), a1 = bload(row_h, j0);
-    const uint32_t a2 = bload(row_g, j0 + 8), a3 = bload(row_h, j0 + 8);
+  // every warp holds the same T_kr; it goes through the warp's own smem slice to reach the
+  // B-fragment layout (j along k, tokens along n)
+  float* tw = sTw + (size_t)warp * RP * NT;
 #pragma unroll
-    for (int t = 0; t < NTT; ++t) {
-      const int tok = t * 8 + g;
-      const uint32_t b0 = pack_bf16x2(a.s * sT[j0 * NT + tok], a.s * sT[(j0 + 1) * NT + tok]);
-      const uint32_t b1 = pack_bf16x2(a.s * sT[(j0 + 8) * NT + tok], a.s * sT[(j0 + 9) * NT + tok]);
-      mma_bf16_16816(d[t], a0, a1, a2, a3, b0, b1);
+  for (int jt = 0; jt < JT; ++jt) {
+    {
+#pragma unroll
+      for (int t = 0; t < NTT; ++t) {
+        tw[(jt * 16 + g) * NT + t * 8 + 2 * q] = dt[jt][t][0];
+        tw[(jt * 16 + g) * NT + t * 8 + 2 * q + 1] = dt[jt][t][1];
+        tw[(jt * 16 + g + 8) * NT + t * 8 + 2 * q] = dt[jt][t][2];
+        tw[(jt * 16 + g + 8) * NT + t * 8 + 2 * q + 1] = dt[jt][t][3];
+      }
+    }
+  }
+  __syncwarp();
+#pragma unroll
+  for (int jt = 0; jt < JT; ++jt) {
+    {
+      const int j0 = jt * 16 + 2 * q;
+#pragma unroll
+      for (int t = 0; t < NTT; ++t) {
+        const int tok = t * 8 + g;
+        const uint32_t b0 = pack_bf16x2(a.s * tw[j0 * NT + tok], a.s * tw[(j0 + 1) * NT + tok]);
+        const uint32_t b1 = pack_bf16x2(a.s * tw[(j0 + 8) * NT + tok], a.s * tw[(j0 + 9) * NT + tok]);
+        mma_bf16_16816(d[t], bfr[jt][0], bfr[jt][1], bfr[jt][2], bfr[jt][3], b0, b1);
+      }
     }
   }
 
@@ -316,8 +344,12 @@ small_m_fwd_kernel(const SmallArgs a) {
     constexpr int kRowsPerRank = kRowsPerCta / kCS;    // 16
     for (int i = threadIdx.x; i < kRowsPerRank * NT; i += blockDim.x) {
       const int rr = (int)rank * kRowsPerRank + i / NT, tok = i % NT;
+      float part[kCS];
+#pragma unroll
+      for (int c = 0; c < kCS; ++c) part[c] = ld_cluster_f32(sD + rr * NT + tok, (uint32_t)c);
       float acc = 0.0f;
-      for (uint32_t c = 0; c < kCS; ++c) acc += ld_cluster_f32(sD + rr * NT + tok, c);
+#pragma unroll
+      for (int c = 0; c < kCS; ++c) acc += part[c];
       const int64_t row = n0 + rr;
       if (tok < a.M && row < a.N) a.Y[tok * a.N + row] = (uint16_t)float_to_bf16_bits(acc);
     }
@@ -325,8 +357,12 @@ small_m_fwd_kernel(const SmallArgs a) {
       for (int i = threadIdx.x; i < RP * NT; i += blockDim.x) {
         const int j = i / NT, tok = i % NT;
         if ((int)(j % kCS) != (int)rank) continue;
+        float part[kCS];
+#pragma unroll
+        for (int c = 0; c < kCS; ++c) part[c] = ld_cluster_f32(sTw + j * NT + tok, (uint32_t)c);
         float acc = 0.0f;
-        for (uint32_t c = 0; c < kCS; ++c) acc += ld_cluster_f32(sT + j * NT + tok, c);
+#pragma unroll
+        for (int c = 0; c < kCS; ++c) acc += part[c];
         if (tok < a.M && j < a.r) a.T_save[tok * a.r + j] = (uint16_t)float_to_bf16_bits(acc);
       }
     }
@@ -334,22 +370,43 @@ small_m_fwd_kernel(const SmallArgs a) {
   cluster_sync_all();                                   // keep smem alive for the readers
 }
 
-size_t small_m_smem(int NT, int kr_max, int r) {
-  const int RP = (r + 15) & ~15;
-  return (size_t)NT * kr_max * 2 + (size_t)(8 * RP * NT + RP * NT + kRowsPerCta * NT) * 4;
+size_t small_m_smem(int NT, int units_max, int r) {
+  const int jt = (r + 15) / 16;
+  const int RP = (jt == 3 ? 4 : jt) * 16;
+  return (size_t)(NT + RP) * small_row_pitch(units_max) + (size_t)(8 * RP * NT + kRowsPerCta * NT) * 4;
 }
 
-template <int NT, int FMT>
+template <int NT, int FMT, int JT>
 static ql_status launch_small(const SmallArgs& a, cudaStream_t st) {
-  auto kern = small_m_fwd_kernel<NT, FMT>;
-  const size_t smem = small_m_smem(NT, a.kr_max, a.r);
+  auto kern = small_m_fwd_kernel<NT, FMT, JT>;
+  SmallArgs b = a;
+  const size_t smem = small_m_smem(NT, a.kr_max / 256, JT * 16);
   if (smem > 227 * 1024) return QL_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return QL_ERR_CUDA;
   const int groups = (int)((a.N + kRowsPerCta - 1) / kRowsPerCta);
-  kern<<<groups * kCS, 256, smem, st>>>(a);
+  // programmatic dependent launch: this grid may begin (and prefetch its weight) while the
+  // previous grid on the stream finishes; the kernel waits before touching X, A, B or Y
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(groups * kCS);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, b) != cudaSuccess) return QL_ERR_CUDA;
   QL_CHECK_LAUNCH();
   return QL_OK;
+}
+
+bool small_m_supported(int64_t K, int r) {
+  if (r < 1 || r > 64) return false;
+  const int64_t U = (K + 255) / 256;
+  const int units_max = (int)((U + kCS - 1) / kCS);
+  return small_m_smem(16, units_max, r) <= 200 * 1024;
 }
 
 // Host entry used by qlora_linear_fwd when M <= 16.
@@ -367,9 +424,19 @@ ql_status small_m_forward(const ql_weight* w, const uint16_t* X, int64_t M, cons
   const Nf4Tables& t = nf4_tables();
   for (int i = 0; i < 16; ++i) a.q[i] = t.q[i];
   ProfScope prof(PK_FWD_SMALL, st, 1);
-  if (w->fmt == QL_FMT_NF4_DQ)
-    return M <= 8 ? launch_small<8, QL_FMT_NF4_DQ>(a, st) : launch_small<16, QL_FMT_NF4_DQ>(a, st);
-  return M <= 8 ? launch_small<8, QL_FMT_INT8_B64>(a, st) : launch_small<16, QL_FMT_INT8_B64>(a, st);
+  if (r > 64) return QL_ERR_UNSUPPORTED;
+  const int jt = (r + 15) / 16;
+  const bool nf4 = w->fmt == QL_FMT_NF4_DQ;
+  if (M <= 8) {
+    if (nf4) return jt == 1 ? launch_small<8, QL_FMT_NF4_DQ, 1>(a, st) : jt == 2 ? launch_small<8, QL_FMT_NF4_DQ, 2>(a, st)
+                                                                              : launch_small<8, QL_FMT_NF4_DQ, 4>(a, st);
+    return jt == 1 ? launch_small<8, QL_FMT_INT8_B64, 1>(a, st) : jt == 2 ? launch_small<8, QL_FMT_INT8_B64, 2>(a, st)
+                                                                        : launch_small<8, QL_FMT_INT8_B64, 4>(a, st);
+  }
+  if (nf4) return jt == 1 ? launch_small<16, QL_FMT_NF4_DQ, 1>(a, st) : jt == 2 ? launch_small<16, QL_FMT_NF4_DQ, 2>(a, st)
+                                                                             : launch_small<16, QL_FMT_NF4_DQ, 4>(a, st);
+  return jt == 1 ? launch_small<16, QL_FMT_INT8_B64, 1>(a, st) : jt == 2 ? launch_small<16, QL_FMT_INT8_B64, 2>(a, st)
+                                                                       : launch_small<16, QL_FMT_INT8_B64, 4>(a, st);
 }
 
 }  // namespace qlb
