@@ -139,6 +139,22 @@ ql_status qlora_linear_bwd(const ql_weight* w, const ql_bf16* X, const ql_bf16* 
                            ql_bf16* dX, float* dA, float* dB, void* ws,
                            size_t ws_bytes, void* stream);
 
+/* The forward above, for callers that cannot allocate device memory where they run it
+ * (inside a CUDA graph capture, in a plugin whose host framework owns every allocation,
+ * or in a loop that must not touch the allocator). It has no counterpart on the pages: it
+ * only changes where the scratch lives. Instead of a caller workspace it uses one fixed
+ * 8 MiB array in the library's device image, which every GPU that loads the library holds
+ * until the process exits. Shapes whose ql_workspace_bytes(QL_OP_FWD, ...) exceeds 8 MiB
+ * are refused with QL_ERR_WORKSPACE (M <= 16 needs no scratch at all). The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress) and caches it; make
+ * that first call before any stream capture. All calls share the one array and nothing
+ * in it needs to start at zero (every call rewrites what it reads), but calls that
+ * overlap on the GPU (different streams, or different threads) race on it: serialise
+ * them. Arguments and outputs are as for qlora_linear_fwd. */
+ql_status qlora_linear_fwd_static(const ql_weight* w, const ql_bf16* X, int64_t M,
+                                  const ql_bf16* A, const ql_bf16* B, int32_t r, float alpha,
+                                  ql_bf16* Y, ql_bf16* T_save, void* stream);
+
 enum { QL_OP_DQ = 0, QL_OP_FWD = 1, QL_OP_BWD = 2 };
 
 /* Workspace bytes that op (QL_OP_*) needs for these sizes (0 if none). */

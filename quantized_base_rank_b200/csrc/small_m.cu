@@ -194,27 +194,39 @@ small_m_fwd_kernel(const SmallArgs a) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
   // token rows and adapter rows of the K-range -> smem in fragment order (zero beyond the
-  // tokens, the rank and K): one 16-byte global load feeds two 8-byte fragment slots
+  // tokens, the rank and K): one 16-byte global load feeds two 8-byte fragment slots. The
+  // loads of a batch are all issued before any of its stores, so their latencies overlap.
   {
     const int per_row = nunits * 32;                // 16-byte vectors per row
     const int total = (NT + RP) * per_row;
-    for (int v = threadIdx.x; v < total; v += blockDim.x) {
-      const int row = v / per_row, rem = v % per_row;
-      const int ul = rem >> 5, qq = (rem >> 3) & 3, ii = rem & 7;
-      const int64_t k = k0 + ul * 256 + 64 * qq + 8 * ii;
-      uint4 val = make_uint4(0u, 0u, 0u, 0u);
-      uint8_t* base;
-      if (row < NT) {
-        if (row < a.M && k < a.K) val = *reinterpret_cast<const uint4*>(a.X + row * a.K + k);
-        base = sX + (size_t)row * pitch;
-      } else {
-        const int j = row - NT;
-        if (j < a.r && k < a.K) val = *reinterpret_cast<const uint4*>(a.A + j * a.K + k);
-        base = sA + (size_t)j * pitch;
+    constexpr int kBatch = 8;
+    for (int v0 = 0; v0 < total; v0 += kBatch * 256) {
+      uint4 val[kBatch];
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b) {
+        const int v = v0 + b * 256 + threadIdx.x;
+        val[b] = make_uint4(0u, 0u, 0u, 0u);
+        if (v < total) {
+          const int row = v / per_row, rem = v % per_row;
+          const int64_t k = k0 + (rem >> 5) * 256 + 64 * ((rem >> 3) & 3) + 8 * (rem & 7);
+          if (row < NT) {
+            if (row < a.M && k < a.K) val[b] = __ldg(reinterpret_cast<const uint4*>(a.X + row * a.K + k));
+          } else if (row - NT < a.r && k < a.K) {
+            val[b] = __ldg(reinterpret_cast<const uint4*>(a.A + (row - NT) * a.K + k));
+          }
+        }
       }
-      uint8_t* p = base + ul * 512;
-      *reinterpret_cast<uint2*>(p + ((2 * ii) * 4 + qq) * 8) = make_uint2(val.x, val.y);
-      *reinterpret_cast<uint2*>(p + ((2 * ii + 1) * 4 + qq) * 8) = make_uint2(val.z, val.w);
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b) {
+        const int v = v0 + b * 256 + threadIdx.x;
+        if (v < total) {
+          const int row = v / per_row, rem = v % per_row;
+          const int ul = rem >> 5, qq = (rem >> 3) & 3, ii = rem & 7;
+          uint8_t* p = (row < NT ? sX + (size_t)row * pitch : sA + (size_t)(row - NT) * pitch) + ul * 512;
+          *reinterpret_cast<uint2*>(p + ((2 * ii) * 4 + qq) * 8) = make_uint2(val[b].x, val[b].y);
+          *reinterpret_cast<uint2*>(p + ((2 * ii + 1) * 4 + qq) * 8) = make_uint2(val[b].z, val[b].w);
+        }
+      }
     }
   }
   // adapter right factor for this warp's rows (A fragments of the final MMA)
