@@ -55,6 +55,7 @@ _SIGS = {
     "ql_profile_enable": ([ctypes.c_int], None),
     "ql_profile_read": ([ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)], ctypes.c_int),
     "ql_launch_count": ([], ctypes.c_uint64),
+    "qlora_linear_fwd_static": ([ctypes.POINTER(QLWeight), P, I64, P, P, I32, F32, P, P, P], I32),
 }
 
 # kernel groups of ql_profile_read

@@ -405,3 +405,47 @@ ql_status qlora_linear_bwd(const ql_weight* w, const ql_bf16* X, const ql_bf16* 
 }
 
 }  // extern "C"
+
+// ---- forward without a caller-supplied workspace -------------------------------------
+//
+// Some callers cannot allocate device memory at the point where they run the layer: code
+// executing inside a CUDA graph capture (where cudaMalloc is not allowed), plugins hosted
+// by a framework that owns every device allocation, and real-time loops that must not
+// touch the allocator after start-up. For them the forward can use a fixed scratch array
+// that lives in this library's own device image. It is sized for the fine-tune-shaped
+// layers this library targets (the 8192 x 11008 x 4096, r = 64 forward needs 5.2 MiB);
+// larger shapes are refused with QL_ERR_WORKSPACE.
+namespace qlb {
+
+constexpr size_t kStaticScratchBytes = size_t(8) << 20;
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+// Device address of the scratch array on the current device, looked up once per device.
+static void* static_scratch_ptr() {
+  static std::mutex mu;
+  static void* ptrs[128] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess) return nullptr;
+    ptrs[dev] = p;
+  }
+  return ptrs[dev];
+}
+
+}  // namespace qlb
+
+extern "C" ql_status qlora_linear_fwd_static(const ql_weight* w, const ql_bf16* X, int64_t M,
+                                             const ql_bf16* A, const ql_bf16* B, int32_t r, float alpha,
+                                             ql_bf16* Y, ql_bf16* T_save, void* stream) {
+  ql_status st0 = check_weight(w);
+  if (st0 != QL_OK) return st0;
+  if (M < 1 || r < 1) return QL_ERR_INVALID_ARG;
+  const size_t need = ql_workspace_bytes(QL_OP_FWD, M, w->N, w->K, r);
+  if (need > kStaticScratchBytes) return QL_ERR_WORKSPACE;
+  void* ws = static_scratch_ptr();
+  if (!ws) return QL_ERR_CUDA;
+  return qlora_linear_fwd(w, X, M, A, B, r, alpha, Y, T_save, ws, kStaticScratchBytes, stream);
+}
