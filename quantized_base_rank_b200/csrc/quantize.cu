@@ -26,16 +26,47 @@ namespace qlb {
 // because a*m is never exactly a bf16 value (a has at most 8 significant bits, every
 // nonzero m at least 21), so |x| <= a*m and |x| < a*m agree. a*m is exact in fp64;
 // rounding it up to bf16 gives a boundary C_k with |x| >= a*m  <=>  |x| >= C_k for
-// bf16 |x|, and on positive bf16 values that is an integer comparison of bit patterns.
+// bf16 |x|, an exact bf16 comparison done for two elements per instruction.
 // ---------------------------------------------------------------------------------
 
-__device__ __forceinline__ uint32_t nf4_code(uint32_t x16, const uint32_t (&C)[7]) {
-  const uint32_t mag = x16 & 0x7FFFu;
-  uint32_t cnt = 0;
+// Two elements at a time in bf16x2 arithmetic: every value involved (the compare results
+// 0/1, counts up to 7, codes up to 15, 128 + code) is a small integer, exact in bf16.
+__device__ __forceinline__ uint32_t bf2_set_ge(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("set.ge.bf16x2.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t bf2_set_lt(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("set.lt.bf16x2.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t bf2_add(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t bf2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// Codes of the two elements of one bf16x2 word, as one byte (element 0 in the low
+// nibble). Cp[k] holds the boundary C_k in both halves.
+//   acc  = 8 + #{k : |x| >= C_k}                       (the code of a non-negative x)
+//   code = acc + neg * (15 - 2 acc)  = 7 - #{...} when x < 0 (strictly; -0 is not)
+__device__ __forceinline__ uint32_t nf4_code_pair(uint32_t w, const uint32_t (&Cp)[7]) {
+  constexpr uint32_t kOne8 = 0x41004100u;        // 8.0, 8.0
+  const uint32_t ax = w & 0x7FFF7FFFu;           // |x|, |x|
+  uint32_t acc = bf2_add(kOne8, bf2_set_ge(ax, Cp[0]));
 #pragma unroll
-  for (int k = 0; k < 7; ++k) cnt += (mag >= C[k]) ? 1u : 0u;
-  const bool neg = (x16 & 0x8000u) && mag;
-  return neg ? 7u - cnt : 8u + cnt;
+  for (int k = 1; k < 7; ++k) acc = bf2_add(acc, bf2_set_ge(ax, Cp[k]));
+  const uint32_t neg = bf2_set_lt(w, 0u);                           // 1.0 where x < 0
+  const uint32_t t = bf2_fma(acc, 0xC000C000u /* -2 */, 0x41704170u /* 15 */);
+  const uint32_t code = bf2_fma(neg, t, acc);                        // 0..15
+  const uint32_t r = bf2_add(code, 0x43004300u /* 128 */);           // bits 0x4300 | code
+  return (r & 0xFu) | ((r >> 12) & 0xF0u);
 }
 
 __device__ __forceinline__ void load_block(const uint16_t* __restrict__ W, int64_t base,
@@ -59,10 +90,10 @@ __device__ __forceinline__ void load_block(const uint16_t* __restrict__ W, int64
 }
 
 __device__ __forceinline__ uint32_t block_absmax_bits(const uint32_t (&v)[32]) {
-  uint32_t m = 0;
+  uint32_t m = 0;                                 // two 16-bit lanes of |x| bit patterns
 #pragma unroll
-  for (int i = 0; i < 32; ++i) m = max(m, max(v[i] & 0x7FFFu, (v[i] >> 16) & 0x7FFFu));
-  return m;   // bf16 bits of max |x|; >= 0x7F80 means inf or NaN somewhere
+  for (int i = 0; i < 32; ++i) m = __vmaxu2(m, v[i] & 0x7FFF7FFFu);
+  return max(m & 0xFFFFu, m >> 16);   // bf16 bits of max |x|; >= 0x7F80 means inf or NaN somewhere
 }
 
 __global__ void __launch_bounds__(256)
@@ -79,23 +110,20 @@ nf4_quantize_kernel(const uint16_t* __restrict__ W, int64_t n, uint8_t* __restri
     if (amax >= 0x7F80u) raise_flag(flag, kFlagNonfinite);
     const float a = __uint_as_float(amax << 16);
     absmax[b] = a;
-    uint32_t C[7];
+    uint32_t Cp[7];
 #pragma unroll
     for (int k = 0; k < 7; ++k) {
       const double prod = (double)a * tab.mid_pos[k];            // exact
       const uint32_t fb = __float_as_uint(__double2float_ru(prod));
-      C[k] = amax ? ((fb + 0xFFFFu) >> 16) : 0xFFFFu;           // ceil to bf16
+      const uint32_t c = amax ? ((fb + 0xFFFFu) >> 16) : 0x7FC0u;   // ceil to bf16 (NaN: never >=)
+      Cp[k] = c | (c << 16);
     }
     uint32_t out[8];
 #pragma unroll
     for (int w = 0; w < 8; ++w) {
       uint32_t word = 0;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint32_t pair = v[4 * w + j];
-        const uint32_t byte = nf4_code(pair & 0xFFFFu, C) | (nf4_code(pair >> 16, C) << 4);
-        word |= byte << (8 * j);
-      }
+      for (int j = 0; j < 4; ++j) word |= nf4_code_pair(v[4 * w + j], Cp) << (8 * j);
       out[w] = word;
     }
     if (vec_ok && full) {
@@ -207,11 +235,9 @@ dq_sum_kernel(const float* __restrict__ absmax, int64_t nb, unsigned long long* 
   }
 }
 
-// One thread: turn the bins into the exact integer X (value X * 2^-149), round it to
-// fp64 (nearest, ties to even), and form mean = fp32(fp64(S) / nb).
-__global__ void dq_finalize_kernel(const unsigned long long* __restrict__ bins, int64_t nb,
-                                   float* __restrict__ mean) {
-  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+// Turn the bins into the exact integer X (value X * 2^-149), round it to fp64 (nearest,
+// ties to even), and return mean = fp32(fp64(S) / nb). One thread's work.
+__device__ float dq_mean_from_bins(const unsigned long long* __restrict__ bins, int64_t nb) {
   uint32_t limb[12];                                   // 384-bit little-endian integer
   for (int i = 0; i < 12; ++i) limb[i] = 0u;
   for (int i = 0; i < kSumBins; ++i) {
@@ -249,17 +275,25 @@ __global__ void dq_finalize_kernel(const unsigned long long* __restrict__ bins, 
       S = ldexp((double)mant, base + tb - 52 - 149);   // exact scaling
     }
   }
-  *mean = __double2float_rn(__ddiv_rn(S, (double)nb));
+  return __double2float_rn(__ddiv_rn(S, (double)nb));
 }
 
-// One warp per group of 256 blocks.
+// One warp per group of 256 blocks. Every CTA first rounds the exact sum to the mean
+// itself (a few hundred instructions on one thread), so no separate launch is needed;
+// CTA 0 also stores it.
 __global__ void __launch_bounds__(256)
-dq_encode_kernel(const float* __restrict__ absmax, int64_t nb, const float* __restrict__ mean,
-                 int8_t* __restrict__ qabsmax, float* __restrict__ group_scale) {
+dq_encode_kernel(const float* __restrict__ absmax, int64_t nb, const unsigned long long* __restrict__ bins,
+                 float* __restrict__ mean, int8_t* __restrict__ qabsmax, float* __restrict__ group_scale) {
+  __shared__ float s_mu;
+  if (threadIdx.x == 0) {
+    s_mu = dq_mean_from_bins(bins, nb);
+    if (blockIdx.x == 0) *mean = s_mu;
+  }
+  __syncthreads();
   const int lane = threadIdx.x & 31;
   const int64_t ng = (nb + kGroup - 1) / kGroup;
   const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  const float mu = *mean;
+  const float mu = s_mu;
   for (int64_t g = (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5); g < ng; g += warps) {
     float d[8];
     float mx = 0.0f;
@@ -376,16 +410,14 @@ ql_status dq_quantize(const float* absmax, int64_t nblocks, int8_t* qabsmax, flo
   if (ws_bytes < ql_workspace_bytes(QL_OP_DQ, 0, 0, 0, 0)) return QL_ERR_WORKSPACE;
   cudaStream_t st = as_stream(stream);
   unsigned long long* bins = static_cast<unsigned long long*>(ws);
-  ProfScope prof(PK_DQ, st, 3);
+  ProfScope prof(PK_DQ, st, 2);
   if (cudaMemsetAsync(bins, 0, kSumBins * sizeof(unsigned long long), st) != cudaSuccess)
     return QL_ERR_CUDA;
   dq_sum_kernel<<<(int)imin64((nblocks + 255) / 256, num_sms()), 256, 0, st>>>(absmax, nblocks, bins,
                                                                               device_flag_ptr());
   QL_CHECK_LAUNCH();
-  dq_finalize_kernel<<<1, 32, 0, st>>>(bins, nblocks, mean);
-  QL_CHECK_LAUNCH();
   const int64_t ng = (nblocks + kGroup - 1) / kGroup;
-  dq_encode_kernel<<<grid_for(ng * 32, 256), 256, 0, st>>>(absmax, nblocks, mean, qabsmax, group_scale);
+  dq_encode_kernel<<<grid_for(ng * 32, 256), 256, 0, st>>>(absmax, nblocks, bins, mean, qabsmax, group_scale);
   QL_CHECK_LAUNCH();
   return QL_OK;
 }
