@@ -139,15 +139,17 @@ ql_status qlora_linear_bwd(const ql_weight* w, const ql_bf16* X, const ql_bf16* 
                            ql_bf16* dX, float* dA, float* dB, void* ws,
                            size_t ws_bytes, void* stream);
 
-/* The forward above, for callers that cannot allocate device memory where they run it
- * (inside a CUDA graph capture, in a plugin whose host framework owns every allocation,
- * or in a loop that must not touch the allocator). It has no counterpart on the pages: it
+/* The forward above, for callers that cannot allocate device memory where they run it:
+ * a plugin whose host framework owns every device allocation (a private cudaMalloc would
+ * escape its pool and accounting), or a latency-bound loop that must not touch the
+ * allocator after start-up (cudaMalloc and cudaFree may synchronise the whole device).
+ * It has no counterpart on the pages: it
  * only changes where the scratch lives. Instead of a caller workspace it uses one fixed
  * 8 MiB array in the library's device image, which every GPU that loads the library holds
  * until the process exits. Shapes whose ql_workspace_bytes(QL_OP_FWD, ...) exceeds 8 MiB
  * are refused with QL_ERR_WORKSPACE (M <= 16 needs no scratch at all). The first call on a
- * device looks up the array's device address (cudaGetSymbolAddress) and caches it; make
- * that first call before any stream capture. All calls share the one array and nothing
+ * device looks up the array's device address (cudaGetSymbolAddress) and caches it; a
+ * failed lookup returns QL_ERR_CUDA. All calls share the one array and nothing
  * in it needs to start at zero (every call rewrites what it reads), but calls that
  * overlap on the GPU (different streams, or different threads) race on it: serialise
  * them. Arguments and outputs are as for qlora_linear_fwd. */

@@ -408,10 +408,11 @@ ql_status qlora_linear_bwd(const ql_weight* w, const ql_bf16* X, const ql_bf16* 
 
 // ---- forward without a caller-supplied workspace -------------------------------------
 //
-// Some callers cannot allocate device memory at the point where they run the layer: code
-// executing inside a CUDA graph capture (where cudaMalloc is not allowed), plugins hosted
-// by a framework that owns every device allocation, and real-time loops that must not
-// touch the allocator after start-up. For them the forward can use a fixed scratch array
+// Some callers cannot allocate device memory at the point where they run the layer:
+// plugins hosted by a framework that owns every device allocation (a private cudaMalloc
+// escapes its pool and its memory accounting), and latency-bound loops that must not touch
+// the allocator after start-up (cudaMalloc and cudaFree may synchronise the whole device).
+// For them the forward can use a fixed scratch array
 // that lives in this library's own device image. It is sized for the fine-tune-shaped
 // layers this library targets (the 8192 x 11008 x 4096, r = 64 forward needs 5.2 MiB);
 // larger shapes are refused with QL_ERR_WORKSPACE.

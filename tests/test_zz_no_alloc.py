@@ -1,7 +1,8 @@
 """The forward entry point that allocates nothing (qlora_linear_fwd_static).
 
 It is for callers that cannot allocate device memory where they run the layer, such as
-code inside a CUDA graph capture or a plugin whose host framework owns every allocation.
+a plugin whose host framework owns every allocation or a loop that must not touch the
+allocator.
 It keeps its scratch in one fixed array inside the library. This file is collected last
 so that a failure here comes after every other test has run. Each call goes straight
 through the C ABI and is compared with the workspace-taking qlora_linear_fwd, on two
