@@ -264,8 +264,7 @@ def run_ours(args, case, world, rank, local_rank):
     dB = torch.empty((N, r), dtype=torch.float32, device=dev)
 
     def step():
-        B.nf4_quantize(W, codes, absmax)
-        B.dq_quantize(absmax, qa, gs, mu)
+        B.nf4_dq_quantize(W, codes, absmax, qa, gs, mu)
         B.linear_fwd(qw, X, A, Bm, case.alpha, Y=Y, T=T)
         B.linear_bwd(qw, X, dY, A, Bm, T, case.alpha, dX=dX, dA=dA, dB=dB)
         if dist is not None:

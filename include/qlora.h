@@ -100,6 +100,18 @@ ql_status dq_quantize(const float* absmax, int64_t nblocks, int8_t* qabsmax,
                       float* group_scale, float* mean, void* ws, size_t ws_bytes,
                       void* stream);
 
+/* NF4 with double quantisation in one call (QLoRA page, "1. 4-bit NormalFloat (NF4)"
+ * followed by "2. Double Quantization"): the results are bit-identical to nf4_quantize
+ * followed by dq_quantize on its absmax. The encode pass also accumulates the exact sum
+ * of the block constants, so the constants are not read a second time for the mean.
+ * codes, absmax as in nf4_quantize (absmax is still written: the double quantisation
+ * reads it); qabsmax [ceil(n/64)], group_scale [ceil(ceil(n/64)/256)], mean [1] as in
+ * dq_quantize. ws: at least ql_workspace_bytes(QL_OP_DQ, 0, 0, 0, 0) bytes.
+ * n must be in [1, 2^30] (at most 2^24 blocks). */
+ql_status nf4_dq_quantize(const ql_bf16* W, int64_t n, uint8_t* codes, float* absmax,
+                          int8_t* qabsmax, float* group_scale, float* mean, void* ws,
+                          size_t ws_bytes, void* stream);
+
 /* Blockwise int8 (the 8-bit choice of the per-layer bit-width, AutoQRA page 3.1):
  * absmax[b] as in nf4_quantize; sc = fp32(absmax[b]/127);
  * codes[j] = clamp(rint_half_even(fp32(W_j / sc)), -127, 127) (0 when sc == 0).

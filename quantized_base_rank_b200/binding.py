@@ -44,6 +44,7 @@ _SIGS = {
     "nf4_quantize": ([P, I64, P, P, P], I32),
     "int8_quantize": ([P, I64, P, P, P], I32),
     "dq_quantize": ([P, I64, P, P, P, P, SZ, P], I32),
+    "nf4_dq_quantize": ([P, I64, P, P, P, P, P, P, SZ, P], I32),
     "ql_dequantize": ([ctypes.POINTER(QLWeight), P, P], I32),
     "qlora_linear_fwd": ([ctypes.POINTER(QLWeight), P, I64, P, P, I32, F32, P, P, P, SZ, P], I32),
     "qlora_linear_bwd": ([ctypes.POINTER(QLWeight), P, P, I64, P, P, P, I32, F32, P, P, P, P, SZ, P], I32),
@@ -172,6 +173,29 @@ def dq_quantize(absmax: torch.Tensor, qabsmax=None, group_scale=None, mean=None)
     return qabsmax, group_scale, mean
 
 
+def nf4_dq_quantize(W: torch.Tensor, codes=None, absmax=None, qabsmax=None, group_scale=None,
+                    mean=None):
+    """NF4 + double quantisation in one call; same results as nf4_quantize then dq_quantize."""
+    _need(W, torch.bfloat16, "W")
+    n = W.numel()
+    dev = W.device
+    nb = (n + 63) // 64
+    if codes is None:
+        codes = torch.empty((n + 1) // 2, dtype=torch.uint8, device=dev)
+    if absmax is None:
+        absmax = torch.empty(nb, dtype=torch.float32, device=dev)
+    if qabsmax is None:
+        qabsmax = torch.empty(nb, dtype=torch.int8, device=dev)
+    if group_scale is None:
+        group_scale = torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev)
+    if mean is None:
+        mean = torch.empty(1, dtype=torch.float32, device=dev)
+    ws = workspace(workspace_bytes(QL_OP_DQ, 0, 0, 0, 0), dev)
+    _check(lib().nf4_dq_quantize(_ptr(W), n, _ptr(codes), _ptr(absmax), _ptr(qabsmax), _ptr(group_scale),
+                                 _ptr(mean), _ptr(ws), ws.numel(), _stream(dev)), "nf4_dq_quantize")
+    return codes, absmax, qabsmax, group_scale, mean
+
+
 class QuantWeight:
     """A quantised weight W [N, K] held in device tensors, plus its ABI descriptor."""
 
@@ -197,8 +221,7 @@ def quantize_weight(W: torch.Tensor, fmt: str = "nf4_dq", keep_absmax: bool = Fa
     """Quantise a bf16 [N, K] weight: NF4 + double quantisation, or blockwise int8."""
     N, K = W.shape
     if fmt == "nf4_dq":
-        codes, absmax = nf4_quantize(W)
-        qa, gs, mu = dq_quantize(absmax)
+        codes, absmax, qa, gs, mu = nf4_dq_quantize(W)
         return QuantWeight(fmt, N, K, codes, absmax if keep_absmax else None, qa, gs, mu)
     if fmt == "int8":
         codes, absmax = int8_quantize(W)

@@ -14,13 +14,24 @@ constexpr int kFlagNonfinite = 1;
 constexpr int kFlagTimeout = 2;
 
 // NF4 grid and its exact decision points, computed once on the host by this
-// library (codebook.cu) and passed to kernels by value.
+// library (runtime.cu) and passed to kernels by value.
 struct Nf4Tables {
   float q[16];          // grid points q_0 < ... < q_15, fp32
   double mid_pos[7];    // positive midpoints (q_j + q_{j+1})/2, j = 8..14, exact in fp64
 };
 
 const Nf4Tables& nf4_tables();          // host, computed on first use
+
+// The encoder's decision boundaries for the 128 normal bf16 absmax values in [1, 2),
+// a = 1 + f/128: c[f][k] holds the bf16 bits of ceil_bf16(a * m_{8+k}) (the product is
+// exact in fp64) in both 16-bit halves; c[f][7] = 0. Rounding to bf16 commutes with a
+// power-of-two scale while the result stays normal, so for a = 2^(e-127) (1 + f/128) the
+// boundaries are these bits with (e - 127) added to the exponent field.
+struct Nf4BoundTable {
+  uint32_t c[128][8];
+};
+
+const Nf4BoundTable& nf4_bound_table();  // host, computed on first use
 
 // Decode-shaped forward (M <= 16), small_m.cu.
 ql_status small_m_forward(const ql_weight* w, const uint16_t* X, int64_t M, const uint16_t* A,

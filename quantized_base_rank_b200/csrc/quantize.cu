@@ -6,9 +6,8 @@
 // constants. The int8 format is the 8-bit option of AutoQRA's per-layer bit-width
 // (gist.science/ko/paper/2602.22268, section 3.1).
 //
-// All of these are HBM-bound streaming passes: one thread owns one block of 64
-// elements (128 B of bf16 read with eight 16-byte loads), so the decision data of a
-// block (its absmax and boundaries) lives in registers and nothing is staged.
+// All of these are HBM-bound streaming passes. The decision data of a block (its absmax
+// and boundaries) lives in registers and nothing is staged.
 #include <math.h>
 
 #include "common.cuh"
@@ -52,8 +51,8 @@ __device__ __forceinline__ uint32_t bf2_fma(uint32_t a, uint32_t b, uint32_t c) 
   return d;
 }
 
-// Codes of the two elements of one bf16x2 word, as one byte (element 0 in the low
-// nibble). Cp[k] holds the boundary C_k in both halves.
+// Codes of the two elements of one bf16x2 word, returned as bf16x2 values 128 + code
+// (bits 0x4300 | code in each half). Cp[k] holds the boundary C_k in both halves.
 //   acc  = 8 + #{k : |x| >= C_k}                       (the code of a non-negative x)
 //   code = acc + neg * (15 - 2 acc)  = 7 - #{...} when x < 0 (strictly; -0 is not)
 __device__ __forceinline__ uint32_t nf4_code_pair(uint32_t w, const uint32_t (&Cp)[7]) {
@@ -65,8 +64,52 @@ __device__ __forceinline__ uint32_t nf4_code_pair(uint32_t w, const uint32_t (&C
   const uint32_t neg = bf2_set_lt(w, 0u);                           // 1.0 where x < 0
   const uint32_t t = bf2_fma(acc, 0xC000C000u /* -2 */, 0x41704170u /* 15 */);
   const uint32_t code = bf2_fma(neg, t, acc);                        // 0..15
-  const uint32_t r = bf2_add(code, 0x43004300u /* 128 */);           // bits 0x4300 | code
-  return (r & 0xFu) | ((r >> 12) & 0xF0u);
+  return bf2_add(code, 0x43004300u /* 128 */);
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+// Eight codes (four nf4_code_pair results, elements in order) -> one 32-bit word of
+// nibbles, element i in bits 4i..4i+3. The low byte of each half holds a code.
+__device__ __forceinline__ uint32_t nf4_pack8(uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+  const uint32_t t0 = prmt(r0, r1, 0x6420u);      // bytes: c0 c1 c2 c3
+  const uint32_t t1 = prmt(r2, r3, 0x6420u);      // bytes: c4 c5 c6 c7
+  // t + (t >> 4) == t | (t >> 4) (no overlapping bits): byte 0 = c0 | c1 << 4 and byte 2 =
+  // c2 | c3 << 4; one multiply-add on the FMA pipe instead of a shift and an OR
+  uint32_t y0, y1;
+  asm("mad.hi.u32 %0, %1, 0x10000000, %1;" : "=r"(y0) : "r"(t0));
+  asm("mad.hi.u32 %0, %1, 0x10000000, %1;" : "=r"(y1) : "r"(t1));
+  return prmt(y0, y1, 0x6420u);
+}
+
+// The seven boundaries C_k = ceil_bf16(a * m_{8+k}) of a block with absmax bits `amax`
+// (sign clear), in both halves of Cp[k]. Normal absmax with biased exponent >= 5 come
+// from the shared-memory copy of the [1, 2) table plus an exponent shift (every boundary
+// then stays normal); zero, subnormal, tiny and non-finite absmax take the fp64 product.
+// A zero block gets NaN boundaries, which no comparison passes: every code is 8.
+__device__ __forceinline__ void nf4_boundaries(uint32_t amax, const uint32_t* s_tab, const Nf4Tables& tab,
+                                               uint32_t (&Cp)[7]) {
+  const uint32_t e = amax >> 7;
+  if (e >= 5u && e <= 254u) {
+    const uint4* row = reinterpret_cast<const uint4*>(s_tab + (amax & 0x7Fu) * 8);
+    const uint4 lo = row[0], hi = row[1];
+    const uint32_t d = (uint32_t)(((int32_t)e - 127) * 128) * 0x10001u;
+    Cp[0] = lo.x + d; Cp[1] = lo.y + d; Cp[2] = lo.z + d; Cp[3] = lo.w + d;
+    Cp[4] = hi.x + d; Cp[5] = hi.y + d; Cp[6] = hi.z + d;
+  } else {
+    const float a = __uint_as_float(amax << 16);
+#pragma unroll
+    for (int k = 0; k < 7; ++k) {
+      const double prod = (double)a * tab.mid_pos[k];            // exact
+      const uint32_t fb = __float_as_uint(__double2float_ru(prod));
+      const uint32_t c = amax ? ((fb + 0xFFFFu) >> 16) : 0x7FC0u;   // ceil to bf16 (NaN: never >=)
+      Cp[k] = c | (c << 16);
+    }
+  }
 }
 
 __device__ __forceinline__ void load_block(const uint16_t* __restrict__ W, int64_t base,
@@ -96,49 +139,243 @@ __device__ __forceinline__ uint32_t block_absmax_bits(const uint32_t (&v)[32]) {
   return max(m & 0xFFFFu, m >> 16);   // bf16 bits of max |x|; >= 0x7F80 means inf or NaN somewhere
 }
 
-__global__ void __launch_bounds__(256)
-nf4_quantize_kernel(const uint16_t* __restrict__ W, int64_t n, uint8_t* __restrict__ codes,
-                    float* __restrict__ absmax, const Nf4Tables tab, int vec_ok, int* flag) {
-  const int64_t nb = (n + kBlock - 1) / kBlock;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nb; b += stride) {
-    const int64_t base = b * kBlock;
-    const bool full = base + kBlock <= n;
-    uint32_t v[32];
-    load_block(W, base, n, vec_ok && full, v);
-    const uint32_t amax = block_absmax_bits(v);
-    if (amax >= 0x7F80u) raise_flag(flag, kFlagNonfinite);
-    const float a = __uint_as_float(amax << 16);
-    absmax[b] = a;
-    uint32_t Cp[7];
-#pragma unroll
-    for (int k = 0; k < 7; ++k) {
-      const double prod = (double)a * tab.mid_pos[k];            // exact
-      const uint32_t fb = __float_as_uint(__double2float_ru(prod));
-      const uint32_t c = amax ? ((fb + 0xFFFFu) >> 16) : 0x7FC0u;   // ceil to bf16 (NaN: never >=)
-      Cp[k] = c | (c << 16);
+// ---------------------------------------------------------------------------------
+// Double quantisation.
+//
+// The mean needs the exact sum of the constants, rounded once to fp64. It is
+// accumulated exactly and order-independently in integer bins: a finite v >= 0 is
+// m * 2^(p - 149) with a 24-bit integer m and p in [0, 253]; it adds m << (p % 16)
+// (< 2^39) to bin p / 16, whose weight is 2^(16 * bin - 149). With at most 2^24
+// values a bin stays below 2^63, and integer addition is associative, so thread and
+// atomic order cannot change the result.
+// ---------------------------------------------------------------------------------
+
+constexpr int kSumBins = 16;
+
+// One constant's term of the exact sum, from its fp32 bits u: the bin and the integer
+// added to it. A negative, infinite or NaN constant is left out (c = 0) and sets `bad`.
+__device__ __forceinline__ void dq_term(uint32_t u, uint32_t& bin, unsigned long long& c, bool& bad) {
+  const uint32_t e = (u >> 23) & 0xFFu;
+  const bool ok = !(u >> 31) && e != 0xFFu;
+  bad |= !ok;
+  const uint32_t m = ok ? ((u & 0x7FFFFFu) | (e ? 0x800000u : 0u)) : 0u;
+  const uint32_t p = (e ? e : 1u) - 1u;
+  c = (unsigned long long)m << (p & 15u);
+  bin = p >> 4;
+}
+
+// Adds one group of lanes' terms (all lanes whose `bin` equals the leader's) into the
+// warp's shared bins. A term c < 2^42 is split at bit 20 so that the two 32-bit warp
+// sums cannot wrap (32 * 2^20 and 32 * 2^22 both fit).
+__device__ __forceinline__ void bins_warp_add(unsigned long long* wbins, uint32_t bin, unsigned long long c,
+                                              int lane) {
+  uint32_t pending = __ballot_sync(0xFFFFFFFFu, c != 0ull);
+  while (pending) {                                   // one pass per distinct bin (<= 16)
+    const int leader = __ffs(pending) - 1;
+    const uint32_t lb = __shfl_sync(0xFFFFFFFFu, bin, leader);
+    const bool mine = c != 0ull && bin == lb;
+    const uint32_t lo = __reduce_add_sync(0xFFFFFFFFu, mine ? (uint32_t)(c & 0xFFFFFu) : 0u);
+    const uint32_t hi = __reduce_add_sync(0xFFFFFFFFu, mine ? (uint32_t)(c >> 20) : 0u);
+    if (lane == 0) wbins[lb] += (unsigned long long)lo + ((unsigned long long)hi << 20);
+    pending &= ~__ballot_sync(0xFFFFFFFFu, mine);
+  }
+}
+
+// Turn the bins into the exact integer X (value X * 2^-149), round it to fp64 (nearest,
+// ties to even), and return mean = fp32(fp64(S) / nb). One thread's work.
+__device__ float dq_mean_from_bins(const unsigned long long (&bins)[16], int64_t nb) {
+  uint32_t limb[12];                                   // 384-bit little-endian integer
+  for (int i = 0; i < 12; ++i) limb[i] = 0u;
+  for (int i = 0; i < kSumBins; ++i) {
+    const unsigned long long v = bins[i];
+    const int bit = 16 * i;
+    const int li = bit / 32;
+    const unsigned long long lo = (bit % 32) ? (v << 16) : v;
+    const uint32_t parts[3] = {(uint32_t)lo, (uint32_t)(lo >> 32), (bit % 32) ? (uint32_t)(v >> 48) : 0u};
+    unsigned long long carry = 0;
+    for (int k = 0; li + k < 12; ++k) {
+      const unsigned long long sum = (unsigned long long)limb[li + k] + (k < 3 ? parts[k] : 0u) + carry;
+      limb[li + k] = (uint32_t)sum;
+      carry = sum >> 32;
+      if (k >= 2 && carry == 0) break;
     }
-    uint32_t out[8];
-#pragma unroll
-    for (int w = 0; w < 8; ++w) {
-      uint32_t word = 0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) word |= nf4_code_pair(v[4 * w + j], Cp) << (8 * j);
-      out[w] = word;
-    }
-    if (vec_ok && full) {
-      uint4* dst = reinterpret_cast<uint4*>(codes + b * 32);
-      dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-      dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+  }
+  int top = -1;
+  for (int i = 11; i >= 0; --i)
+    if (limb[i]) { top = i; break; }
+  double S = 0.0;
+  if (top >= 0) {
+    // 96-bit window of limbs top, top-1, top-2 (missing limbs are zero)
+    const uint32_t l1 = top >= 1 ? limb[top - 1] : 0u, l2 = top >= 2 ? limb[top - 2] : 0u;
+    const unsigned __int128 W = ((unsigned __int128)limb[top] << 64) | ((unsigned __int128)l1 << 32) | l2;
+    const int tb = 95 - __clz(limb[top]);              // top set bit inside W (>= 64)
+    const int base = 32 * (top - 2);                   // weight of bit 0 of W
+    if (base + tb < 53) {
+      S = ldexp((double)(unsigned long long)(W >> (base < 0 ? -base : 0)), base > 0 ? base - 149 : -149);
     } else {
-      const int64_t cnt = imin64(kBlock, n - base);
-      const int64_t nbytes = (cnt + 1) / 2;
-      for (int i = 0; i < nbytes; ++i) {
-        uint8_t byte = (uint8_t)(out[i / 4] >> (8 * (i % 4)));
-        if (2 * i + 1 >= cnt) byte &= 0x0F;                  // no element: nibble 0
-        codes[b * 32 + i] = byte;
+      unsigned long long mant = (unsigned long long)(W >> (tb - 52));
+      const uint32_t rbit = (uint32_t)(W >> (tb - 53)) & 1u;
+      bool sticky = (W & ((((unsigned __int128)1) << (tb - 53)) - 1)) != 0;
+      for (int i = 0; i < top - 2 && !sticky; ++i) sticky = limb[i] != 0u;
+      if (rbit && (sticky || (mant & 1ull))) mant += 1ull;
+      S = ldexp((double)mant, base + tb - 52 - 149);   // exact scaling
+    }
+  }
+  return __double2float_rn(__ddiv_rn(S, (double)nb));
+}
+
+// End of the exact sum for one CTA (every thread calls it): the per-warp bins are
+// combined, added to the global bins (one atomic per non-empty bin), and the CTA takes a
+// ticket. The CTA that takes the last of `ctas` tickets (counted over every launch that
+// shares the bins) rounds the sum and writes the mean. No CTA waits for another.
+// ws: bins[16], then the ticket counter; zeroed before the first launch.
+__device__ __forceinline__ void dq_bins_finish(unsigned long long (*s_bins)[kSumBins], int nwarps,
+                                               unsigned long long* ws, unsigned int ctas, int64_t nb,
+                                               float* mean) {
+  __shared__ int s_last;
+  __syncthreads();
+  unsigned int* ticket = reinterpret_cast<unsigned int*>(ws + kSumBins);
+  if (threadIdx.x < kSumBins) {
+    unsigned long long x = 0ull;
+    for (int w = 0; w < nwarps; ++w) x += s_bins[w][threadIdx.x];
+    if (x) atomicAdd(ws + threadIdx.x, x);
+    __threadfence();                                  // the bin atomics before the ticket
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(ticket, 1u) == ctas - 1;
+  __syncthreads();
+  if (s_last && threadIdx.x == 0) {
+    __threadfence();
+    unsigned long long v[kSumBins];
+#pragma unroll
+    for (int i = 0; i < kSumBins; ++i) v[i] = __ldcg(ws + i);
+    *mean = dq_mean_from_bins(v, nb);
+  }
+}
+
+// NF4 encode kernel. Two threads per block of 64: lanes 2t and 2t+1 of a warp take the
+// two halves of one block (32 elements, 64 bytes), combine their partial absmax with one
+// shuffle and each write 16 bytes of codes. The grid is persistent and the loop is
+// warp-uniform, so every lane takes part in the shuffles. VEC = true covers whole blocks
+// with 16-byte aligned input and codes, and loads the next block-half while it encodes
+// the current one; VEC = false (a ragged last block, or unaligned pointers) goes element
+// by element with bounds checks. DQ = true also accumulates the exact sum of the block
+// constants for double quantisation (dq_bins_finish).
+constexpr int kNf4Threads = 256;
+constexpr int kNf4Warps = kNf4Threads / 32;
+
+struct Nf4Args {
+  const uint16_t* W;
+  int64_t n, blk_begin, blk_end;
+  uint8_t* codes;
+  float* absmax;
+  int* flag;
+  unsigned long long* dq_ws;   // DQ: bins + ticket
+  float* mean;                 // DQ: output
+  unsigned int dq_ctas;        // DQ: CTAs over all launches sharing the bins
+  int64_t nb_total;            // DQ: number of constants
+};
+
+__device__ __forceinline__ void nf4_load_vec(const uint16_t* __restrict__ W, int64_t base, bool live,
+                                             uint4 (&x)[4]) {
+  if (live) {
+    const uint4* src = reinterpret_cast<const uint4*>(W + base);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = __ldg(src + i);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+template <bool VEC, bool DQ>
+__global__ void __launch_bounds__(kNf4Threads, VEC ? 4 : 1)
+nf4_quantize_kernel(const Nf4Args args, const Nf4Tables tab, const Nf4BoundTable btab) {
+  __shared__ __align__(16) uint32_t s_tab[128 * 8];
+  __shared__ unsigned long long s_bins[DQ ? kNf4Warps : 1][kSumBins];
+  for (int i = threadIdx.x; i < 128 * 8 / 4; i += blockDim.x)
+    reinterpret_cast<uint4*>(s_tab)[i] = reinterpret_cast<const uint4*>(&btab.c[0][0])[i];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (DQ) {
+    if (lane < kSumBins) s_bins[warp][lane] = 0ull;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  }
+  __syncthreads();
+
+  const uint16_t* __restrict__ W = args.W;
+  const int64_t n = args.n;
+  const int64_t items = 2 * (args.blk_end - args.blk_begin);
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  bool bad = false;
+  int64_t w0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
+  uint4 nx[4];
+  if (VEC) {
+    const int64_t it = w0 + lane;
+    nf4_load_vec(W, (args.blk_begin + (it >> 1)) * kBlock + 32 * (it & 1), it < items, nx);
+  }
+  for (; w0 < items; w0 += stride) {
+    const int64_t it = w0 + lane;
+    const bool live = it < items;
+    const int64_t b = args.blk_begin + (it >> 1);
+    const int h = (int)(it & 1);
+    const int64_t base = b * kBlock + 32 * h;
+    uint32_t v[16];
+    if (VEC) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        v[4 * i + 0] = nx[i].x; v[4 * i + 1] = nx[i].y; v[4 * i + 2] = nx[i].z; v[4 * i + 3] = nx[i].w;
+      }
+      const int64_t it1 = it + stride;                 // next block-half of this lane
+      nf4_load_vec(W, (args.blk_begin + (it1 >> 1)) * kBlock + 32 * (it1 & 1), it1 < items, nx);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int64_t e = base + 2 * i;
+        const uint32_t lo = live && e < n ? (uint32_t)W[e] : 0u;
+        const uint32_t hi = live && e + 1 < n ? (uint32_t)W[e + 1] : 0u;
+        v[i] = lo | (hi << 16);
       }
     }
+    uint32_t m = 0;                                  // two 16-bit lanes of |x| bit patterns
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m = __vmaxu2(m, v[i] & 0x7FFF7FFFu);
+    m = __vmaxu2(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+    const uint32_t amax = max(m & 0xFFFFu, m >> 16);   // bf16 bits of the block's max |x|
+    const bool owner = live && h == 0;
+    if (owner) {
+      if (amax >= 0x7F80u) raise_flag(args.flag, kFlagNonfinite);
+      args.absmax[b] = __uint_as_float(amax << 16);
+    }
+    if (DQ) {
+      uint32_t bin = 0;
+      unsigned long long c = 0ull;
+      if (owner) dq_term(amax << 16, bin, c, bad);
+      bins_warp_add(s_bins[warp], bin, c, lane);
+    }
+    uint32_t Cp[7];
+    nf4_boundaries(amax, s_tab, tab, Cp);
+    uint32_t out[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w)
+      out[w] = nf4_pack8(nf4_code_pair(v[4 * w + 0], Cp), nf4_code_pair(v[4 * w + 1], Cp),
+                         nf4_code_pair(v[4 * w + 2], Cp), nf4_code_pair(v[4 * w + 3], Cp));
+    uint8_t* dst = args.codes + b * 32 + 16 * h;
+    if (VEC) {
+      if (live) *reinterpret_cast<uint4*>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
+    } else if (live) {
+      const int64_t cnt = imin64(32, n - base);        // elements of this half (may be <= 0)
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        if (2 * i >= cnt) break;
+        uint8_t byte = (uint8_t)(out[i / 4] >> (8 * (i % 4)));
+        if (2 * i + 1 >= cnt) byte &= 0x0F;              // no element: nibble 0
+        dst[i] = byte;
+      }
+    }
+  }
+  if (DQ) {
+    (void)bad;                                         // a non-finite absmax already raised the flag
+    dq_bins_finish(s_bins, kNf4Warps, args.dq_ws, args.dq_ctas, args.nb_total, args.mean);
   }
 }
 
@@ -186,114 +423,73 @@ int8_quantize_kernel(const uint16_t* __restrict__ W, int64_t n, int8_t* __restri
   }
 }
 
-// ---------------------------------------------------------------------------------
-// Double quantisation.
-//
-// The mean needs the exact sum of the constants, rounded once to fp64. It is
-// accumulated exactly and order-independently in integer bins: a finite v >= 0 is
-// m * 2^(p - 149) with a 24-bit integer m and p in [0, 253]; it adds m << (p % 16)
-// (< 2^39) to bin p / 16, whose weight is 2^(16 * bin - 149). With at most 2^24
-// values a bin stays below 2^63, and integer addition is associative, so thread and
-// atomic order cannot change the result.
-// ---------------------------------------------------------------------------------
+// Exact integer-bin sum of an array of constants (dq_quantize). Each thread reads
+// kSumPerThread constants; a lane whose constants share one bin adds them first, and a
+// warp whose lanes all use one bin needs one pass of bins_warp_add.
+constexpr int kSumThreads = 256;
+constexpr int kSumPerThread = 8;          // constants per thread (two 16-byte loads)
 
-constexpr int kSumBins = 16;
+__global__ void __launch_bounds__(kSumThreads)
+dq_sum_kernel(const float* __restrict__ absmax, int64_t nb, unsigned long long* ws, float* mean, int vec,
+              int* flag) {
+  __shared__ unsigned long long s_bins[kSumThreads / 32][kSumBins];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane < kSumBins) s_bins[warp][lane] = 0ull;
+  __syncwarp();
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-__global__ void __launch_bounds__(256)
-dq_sum_kernel(const float* __restrict__ absmax, int64_t nb, unsigned long long* bins, int* flag) {
-  __shared__ unsigned long long part[8][kSumBins];
-  unsigned long long acc[kSumBins];
-#pragma unroll
-  for (int i = 0; i < kSumBins; ++i) acc[i] = 0ull;
   bool bad = false;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nb; b += stride) {
-    const uint32_t u = __float_as_uint(absmax[b]);
-    const uint32_t e = (u >> 23) & 0xFFu;
-    if ((u >> 31) || e == 0xFFu) { bad = true; continue; }
-    const uint32_t m = (u & 0x7FFFFFu) | (e ? 0x800000u : 0u);
-    const uint32_t p = (e ? e : 1u) - 1u;
-    const unsigned long long c = (unsigned long long)m << (p & 15u);
-    const uint32_t bin = p >> 4;
+  const int64_t chunk = (int64_t)kSumThreads * kSumPerThread;
+  for (int64_t c0 = (int64_t)blockIdx.x * chunk; c0 < nb; c0 += (int64_t)gridDim.x * chunk) {
+    const int64_t i0 = c0 + (int64_t)threadIdx.x * kSumPerThread;
+    uint32_t u[kSumPerThread];
+    if (vec && i0 + kSumPerThread <= nb) {
+      const uint4* src = reinterpret_cast<const uint4*>(absmax + i0);
+      const uint4 x = __ldg(src), y = __ldg(src + 1);
+      u[0] = x.x; u[1] = x.y; u[2] = x.z; u[3] = x.w; u[4] = y.x; u[5] = y.y; u[6] = y.z; u[7] = y.w;
+    } else {
 #pragma unroll
-    for (int i = 0; i < kSumBins; ++i) acc[i] += (bin == (uint32_t)i) ? c : 0ull;
+      for (int k = 0; k < kSumPerThread; ++k) u[k] = i0 + k < nb ? __float_as_uint(absmax[i0 + k]) : 0u;
+    }
+    uint32_t bin[kSumPerThread];
+    unsigned long long c[kSumPerThread];
+#pragma unroll
+    for (int k = 0; k < kSumPerThread; ++k) dq_term(u[k], bin[k], c[k], bad);
+    // lane-level merge when every non-zero term of the lane falls in one bin
+    uint32_t b0 = 0u;
+    bool have = false;
+#pragma unroll
+    for (int k = 0; k < kSumPerThread; ++k)
+      if (c[k] != 0ull && !have) { b0 = bin[k]; have = true; }
+    bool one = true;
+    unsigned long long csum = 0ull;
+#pragma unroll
+    for (int k = 0; k < kSumPerThread; ++k) {
+      one &= (c[k] == 0ull) || (bin[k] == b0);
+      csum += c[k];                                   // < 8 * 2^39 = 2^42: fits the split in bins_warp_add
+    }
+    if (__all_sync(0xFFFFFFFFu, one)) {
+      bins_warp_add(s_bins[warp], b0, csum, lane);
+    } else {
+#pragma unroll
+      for (int k = 0; k < kSumPerThread; ++k) bins_warp_add(s_bins[warp], bin[k], c[k], lane);
+    }
   }
   if (bad) raise_flag(flag, kFlagNonfinite);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-#pragma unroll
-  for (int i = 0; i < kSumBins; ++i) {
-    unsigned long long x = acc[i];
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) x += __shfl_down_sync(0xFFFFFFFFu, x, off);
-    if (lane == 0) part[warp][i] = x;
-  }
-  __syncthreads();
-  if (threadIdx.x < kSumBins) {
-    unsigned long long x = 0ull;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) x += part[w][threadIdx.x];
-    if (x) atomicAdd(bins + threadIdx.x, x);
-  }
+  dq_bins_finish(s_bins, kSumThreads / 32, ws, gridDim.x, nb, mean);
 }
 
-// Turn the bins into the exact integer X (value X * 2^-149), round it to fp64 (nearest,
-// ties to even), and return mean = fp32(fp64(S) / nb). One thread's work.
-__device__ float dq_mean_from_bins(const unsigned long long* __restrict__ bins, int64_t nb) {
-  uint32_t limb[12];                                   // 384-bit little-endian integer
-  for (int i = 0; i < 12; ++i) limb[i] = 0u;
-  for (int i = 0; i < kSumBins; ++i) {
-    const unsigned long long v = bins[i];
-    const int bit = 16 * i;
-    const int li = bit / 32;
-    const unsigned long long lo = (bit % 32) ? (v << 16) : v;
-    const uint32_t parts[3] = {(uint32_t)lo, (uint32_t)(lo >> 32), (bit % 32) ? (uint32_t)(v >> 48) : 0u};
-    unsigned long long carry = 0;
-    for (int k = 0; li + k < 12; ++k) {
-      const unsigned long long sum = (unsigned long long)limb[li + k] + (k < 3 ? parts[k] : 0u) + carry;
-      limb[li + k] = (uint32_t)sum;
-      carry = sum >> 32;
-      if (k >= 2 && carry == 0) break;
-    }
-  }
-  int top = -1;
-  for (int i = 11; i >= 0; --i)
-    if (limb[i]) { top = i; break; }
-  double S = 0.0;
-  if (top >= 0) {
-    // 96-bit window of limbs top, top-1, top-2 (missing limbs are zero)
-    const uint32_t l1 = top >= 1 ? limb[top - 1] : 0u, l2 = top >= 2 ? limb[top - 2] : 0u;
-    const unsigned __int128 W = ((unsigned __int128)limb[top] << 64) | ((unsigned __int128)l1 << 32) | l2;
-    const int tb = 95 - __clz(limb[top]);              // top set bit inside W (>= 64)
-    const int base = 32 * (top - 2);                   // weight of bit 0 of W
-    if (base + tb < 53) {
-      S = ldexp((double)(unsigned long long)(W >> (base < 0 ? -base : 0)), base > 0 ? base - 149 : -149);
-    } else {
-      unsigned long long mant = (unsigned long long)(W >> (tb - 52));
-      const uint32_t rbit = (uint32_t)(W >> (tb - 53)) & 1u;
-      bool sticky = (W & ((((unsigned __int128)1) << (tb - 53)) - 1)) != 0;
-      for (int i = 0; i < top - 2 && !sticky; ++i) sticky = limb[i] != 0u;
-      if (rbit && (sticky || (mant & 1ull))) mant += 1ull;
-      S = ldexp((double)mant, base + tb - 52 - 149);   // exact scaling
-    }
-  }
-  return __double2float_rn(__ddiv_rn(S, (double)nb));
-}
-
-// One warp per group of 256 blocks. Every CTA first rounds the exact sum to the mean
-// itself (a few hundred instructions on one thread), so no separate launch is needed;
-// CTA 0 also stores it.
+// One warp per group of 256 blocks: d = a - mean, s_g = max|d| / 127, code =
+// clamp(rint(d / s_g)). Launched as a programmatic dependent of dq_sum_kernel; it waits
+// for that grid (and its mean) before reading anything.
 __global__ void __launch_bounds__(256)
-dq_encode_kernel(const float* __restrict__ absmax, int64_t nb, const unsigned long long* __restrict__ bins,
-                 float* __restrict__ mean, int8_t* __restrict__ qabsmax, float* __restrict__ group_scale) {
-  __shared__ float s_mu;
-  if (threadIdx.x == 0) {
-    s_mu = dq_mean_from_bins(bins, nb);
-    if (blockIdx.x == 0) *mean = s_mu;
-  }
-  __syncthreads();
+dq_encode_kernel(const float* __restrict__ absmax, int64_t nb, const float* __restrict__ mean,
+                 int8_t* __restrict__ qabsmax, float* __restrict__ group_scale) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int lane = threadIdx.x & 31;
   const int64_t ng = (nb + kGroup - 1) / kGroup;
   const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  const float mu = s_mu;
+  const float mu = *mean;
   for (int64_t g = (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5); g < ng; g += warps) {
     float d[8];
     float mx = 0.0f;
@@ -361,10 +557,84 @@ dequant_int8_kernel(const int8_t* __restrict__ codes, const float* __restrict__ 
   }
 }
 
+// CTAs of `kernel` that fit on one SM at `threads` threads (at least 1), per device.
+template <typename Kernel>
+static int resident_ctas(Kernel kernel, int threads) {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, 0) != cudaSuccess || n < 1) return 1;
+  return n;
+}
+
 static int grid_for(int64_t items, int threads) {
   const int64_t need = (items + threads - 1) / threads;
   const int64_t cap = (int64_t)num_sms() * 16;
   return (int)imax64(1, imin64(need, cap));
+}
+
+// Kernels nf4_quantize launches: the vector kernel over whole blocks when W and codes are
+// 16-byte aligned, and the element-wise kernel over the rest (a ragged last block, or
+// everything when unaligned).
+static int nf4_launches(const void* W, int64_t n, const void* codes) {
+  const bool vec = aligned(W, 16) && aligned(codes, 16);
+  const int64_t nb = (n + kBlock - 1) / kBlock, nb_vec = vec ? n / kBlock : 0;
+  return (nb_vec > 0) + (nb_vec < nb);
+}
+
+// NF4 encode of W[0, n); with dq_ws (zeroed bins + ticket) also the exact sum of the block
+// constants and, from the last CTA, the double-quantisation mean.
+static ql_status launch_nf4(const uint16_t* W, int64_t n, uint8_t* codes, float* absmax,
+                            unsigned long long* dq_ws, float* mean, cudaStream_t st) {
+  const bool vec = aligned(W, 16) && aligned(codes, 16);
+  const int64_t nb = (n + kBlock - 1) / kBlock;
+  const int64_t nb_vec = vec ? n / kBlock : 0;
+  const bool dq = dq_ws != nullptr;
+  int g_vec = 0, g_tail = 0;
+  if (nb_vec > 0) {
+    static const int per_sm = resident_ctas(nf4_quantize_kernel<true, true>, kNf4Threads);
+    const int64_t need = (2 * nb_vec + kNf4Threads - 1) / kNf4Threads;
+    g_vec = (int)imax64(1, imin64(need, (int64_t)num_sms() * per_sm));
+  }
+  if (nb_vec < nb) {
+    const int64_t need = (2 * (nb - nb_vec) + kNf4Threads - 1) / kNf4Threads;
+    g_tail = (int)imax64(1, imin64(need, (int64_t)num_sms() * 4));
+  }
+  Nf4Args a;
+  a.W = W; a.n = n; a.codes = codes; a.absmax = absmax; a.flag = device_flag_ptr();
+  a.dq_ws = dq_ws; a.mean = mean; a.dq_ctas = (unsigned)(g_vec + g_tail); a.nb_total = nb;
+  const Nf4Tables& tab = nf4_tables();
+  const Nf4BoundTable& btab = nf4_bound_table();
+  if (g_vec) {
+    a.blk_begin = 0; a.blk_end = nb_vec;
+    if (dq) nf4_quantize_kernel<true, true><<<g_vec, kNf4Threads, 0, st>>>(a, tab, btab);
+    else nf4_quantize_kernel<true, false><<<g_vec, kNf4Threads, 0, st>>>(a, tab, btab);
+    QL_CHECK_LAUNCH();
+  }
+  if (g_tail) {
+    a.blk_begin = nb_vec; a.blk_end = nb;
+    if (dq) nf4_quantize_kernel<false, true><<<g_tail, kNf4Threads, 0, st>>>(a, tab, btab);
+    else nf4_quantize_kernel<false, false><<<g_tail, kNf4Threads, 0, st>>>(a, tab, btab);
+    QL_CHECK_LAUNCH();
+  }
+  return QL_OK;
+}
+
+// The encode pass of double quantisation, launched as a programmatic dependent of the
+// kernel before it on the stream (it waits for that grid before reading anything).
+static ql_status launch_dq_encode(const float* absmax, int64_t nb, const float* mean, int8_t* qabsmax,
+                                  float* group_scale, cudaStream_t st) {
+  const int64_t ng = (nb + kGroup - 1) / kGroup;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid_for(ng * 32, 256));
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, dq_encode_kernel, absmax, nb, mean, qabsmax, group_scale) != cudaSuccess)
+    return QL_ERR_CUDA;
+  return QL_OK;
 }
 
 }  // namespace qlb
@@ -378,13 +648,8 @@ ql_status nf4_quantize(const ql_bf16* W, int64_t n, uint8_t* codes, float* absma
   if (n == 0) return QL_OK;
   if (!W || !codes || !absmax) return QL_ERR_INVALID_ARG;
   if (!aligned(W, 2) || !aligned(codes, 4) || !aligned(absmax, 4)) return QL_ERR_INVALID_ARG;
-  const int vec = aligned(W, 16) && aligned(codes, 16);
-  const int64_t nb = (n + kBlock - 1) / kBlock;
-  ProfScope prof(PK_NF4, as_stream(stream), 1);
-  nf4_quantize_kernel<<<grid_for(nb, 256), 256, 0, as_stream(stream)>>>(
-      W, n, codes, absmax, nf4_tables(), vec, device_flag_ptr());
-  QL_CHECK_LAUNCH();
-  return QL_OK;
+  ProfScope prof(PK_NF4, as_stream(stream), nf4_launches(W, n, codes));
+  return launch_nf4(W, n, codes, absmax, nullptr, nullptr, as_stream(stream));
 }
 
 ql_status int8_quantize(const ql_bf16* W, int64_t n, int8_t* codes, float* absmax, void* stream) {
@@ -411,15 +676,36 @@ ql_status dq_quantize(const float* absmax, int64_t nblocks, int8_t* qabsmax, flo
   cudaStream_t st = as_stream(stream);
   unsigned long long* bins = static_cast<unsigned long long*>(ws);
   ProfScope prof(PK_DQ, st, 2);
-  if (cudaMemsetAsync(bins, 0, kSumBins * sizeof(unsigned long long), st) != cudaSuccess)
+  if (cudaMemsetAsync(bins, 0, (kSumBins + 1) * sizeof(unsigned long long), st) != cudaSuccess)
     return QL_ERR_CUDA;
-  dq_sum_kernel<<<(int)imin64((nblocks + 255) / 256, num_sms()), 256, 0, st>>>(absmax, nblocks, bins,
-                                                                              device_flag_ptr());
+  const int64_t chunk = (int64_t)kSumThreads * kSumPerThread;
+  const int sum_grid = (int)imax64(1, imin64((nblocks + chunk - 1) / chunk, (int64_t)num_sms() * 8));
+  dq_sum_kernel<<<sum_grid, kSumThreads, 0, st>>>(absmax, nblocks, bins, mean, aligned(absmax, 16) ? 1 : 0,
+                                                  device_flag_ptr());
   QL_CHECK_LAUNCH();
-  const int64_t ng = (nblocks + kGroup - 1) / kGroup;
-  dq_encode_kernel<<<grid_for(ng * 32, 256), 256, 0, st>>>(absmax, nblocks, bins, mean, qabsmax, group_scale);
-  QL_CHECK_LAUNCH();
-  return QL_OK;
+  return launch_dq_encode(absmax, nblocks, mean, qabsmax, group_scale, st);
+}
+
+ql_status nf4_dq_quantize(const ql_bf16* W, int64_t n, uint8_t* codes, float* absmax, int8_t* qabsmax,
+                          float* group_scale, float* mean, void* ws, size_t ws_bytes, void* stream) {
+  if (n < 1 || !W || !codes || !absmax || !qabsmax || !group_scale || !mean || !ws) return QL_ERR_INVALID_ARG;
+  const int64_t nb = (n + kBlock - 1) / kBlock;
+  if (nb > (int64_t(1) << 24)) return QL_ERR_UNSUPPORTED;
+  if (!aligned(W, 2) || !aligned(codes, 4) || !aligned(absmax, 4) || !aligned(group_scale, 4) ||
+      !aligned(mean, 4) || !aligned(ws, 16))
+    return QL_ERR_INVALID_ARG;
+  if (ws_bytes < ql_workspace_bytes(QL_OP_DQ, 0, 0, 0, 0)) return QL_ERR_WORKSPACE;
+  cudaStream_t st = as_stream(stream);
+  unsigned long long* bins = static_cast<unsigned long long*>(ws);
+  {
+    ProfScope prof(PK_NF4, st, nf4_launches(W, n, codes));
+    if (cudaMemsetAsync(bins, 0, (kSumBins + 1) * sizeof(unsigned long long), st) != cudaSuccess)
+      return QL_ERR_CUDA;
+    const ql_status s = launch_nf4(W, n, codes, absmax, bins, mean, st);
+    if (s != QL_OK) return s;
+  }
+  ProfScope prof(PK_DQ, st, 1);
+  return launch_dq_encode(absmax, nb, mean, qabsmax, group_scale, st);
 }
 
 ql_status ql_dequantize(const ql_weight* w, ql_bf16* Wout, void* stream) {

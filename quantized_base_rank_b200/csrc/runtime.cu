@@ -1,5 +1,6 @@
 // Host-side runtime pieces: the NF4 tables, the sticky device flag, status strings.
 #include <math.h>
+#include <string.h>
 
 #include <atomic>
 #include <mutex>
@@ -40,6 +41,35 @@ static Nf4Tables build_tables() {
 const Nf4Tables& nf4_tables() {
   static const Nf4Tables t = build_tables();
   return t;
+}
+
+// Smallest bf16 value >= d, for a positive double d whose bf16 rounding is normal: round
+// the fp64 bit pattern up at the 8th significant bit (a carry moves into the exponent
+// on its own), then move the exponent from the fp64 bias to the bf16 bias.
+static uint32_t ceil_bf16_bits(double d) {
+  uint64_t bits;
+  memcpy(&bits, &d, sizeof bits);
+  const uint64_t r = (bits + ((uint64_t(1) << 45) - 1)) >> 45;   // sign | exp11 | top 7 bits
+  return (uint32_t)(r - (uint64_t(1023 - 127) << 7));
+}
+
+static Nf4BoundTable build_bound_table() {
+  const Nf4Tables& t = nf4_tables();
+  Nf4BoundTable b;
+  for (int f = 0; f < 128; ++f) {
+    const double a = 1.0 + f / 128.0;
+    for (int k = 0; k < 7; ++k) {
+      const uint32_t c = ceil_bf16_bits(a * t.mid_pos[k]);          // exact product
+      b.c[f][k] = c | (c << 16);
+    }
+    b.c[f][7] = 0u;
+  }
+  return b;
+}
+
+const Nf4BoundTable& nf4_bound_table() {
+  static const Nf4BoundTable b = build_bound_table();
+  return b;
 }
 
 __device__ int g_ql_flag;

@@ -20,7 +20,7 @@ def lib():
 
 def test_header_declares_the_boundary():
     names = set(B.header_functions())
-    for required in ("nf4_quantize", "dq_quantize", "int8_quantize", "ql_dequantize",
+    for required in ("nf4_quantize", "dq_quantize", "nf4_dq_quantize", "int8_quantize", "ql_dequantize",
                      "qlora_linear_fwd", "qlora_linear_bwd", "ql_workspace_bytes",
                      "ql_get_device_status", "ql_status_string", "ql_nf4_codebook"):
         assert required in names, required
@@ -51,6 +51,12 @@ def test_argument_validation_without_a_device(lib):
     assert lib.nf4_quantize(None, 0, None, None, None) == B.QL_OK
     assert lib.int8_quantize(None, 64, None, None, None) == B.QL_ERR_INVALID_ARG
     assert lib.dq_quantize(None, 4, None, None, None, None, 0, None) == B.QL_ERR_INVALID_ARG
+    assert lib.nf4_dq_quantize(None, 64, None, None, None, None, None, None, 0, None) == B.QL_ERR_INVALID_ARG
+    assert lib.nf4_dq_quantize(16, 0, 16, 16, 16, 16, 16, 16, 256, None) == B.QL_ERR_INVALID_ARG
+    # more than 2^24 blocks
+    assert lib.nf4_dq_quantize(16, 64 * (1 << 24) + 1, 16, 16, 16, 16, 16, 16, 256, None) == B.QL_ERR_UNSUPPORTED
+    # workspace too small
+    assert lib.nf4_dq_quantize(16, 64, 16, 16, 16, 16, 16, 16, 8, None) == B.QL_ERR_WORKSPACE
     assert lib.ql_dequantize(None, None, None) == B.QL_ERR_INVALID_ARG
     w = B.QLWeight(0, 0, 64, 64, 16, 0, 16, 16, 16)
     # misaligned or null pointers, bad shapes: all rejected synchronously

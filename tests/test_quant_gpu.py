@@ -30,6 +30,40 @@ def _weights():
     special[384:384 + 2048] = np.resize(vals, 2048) * np.resize([1, -1], 2048)
     special[2432:] = rng.standard_normal(special.size - 2432) * 0.05
     yield "special-values", synth.to_bf16(special)
+    yield "boundary-sweep", _boundary_sweep()
+
+
+def _ceil_bf16_bits(d):
+    """Bits of the smallest bf16 >= d, elementwise (d > 0, fp64): round up to fp32, then
+    round the fp32 bit pattern up to bf16."""
+    f = d.astype(np.float32)
+    f = np.where(f.astype(np.float64) < d, np.nextafter(f, np.float32(np.inf)), f)
+    return ((f.view(np.uint32).astype(np.uint64) + 0xFFFF) >> 16).astype(np.uint32)
+
+
+def _boundary_sweep():
+    """One block for every positive finite bf16 absmax a (all exponents, all mantissas,
+    subnormals included). Each block holds +a, then, for each positive midpoint m of the
+    grid, the bf16 values at and just below ceil_bf16(a*m), each with both signs; the
+    rest of the block is uniform in [-a, a]. Every element sits on or next to a decision
+    point, so a wrong boundary for any absmax changes a code."""
+    mids = o.nf4_midpoints()[8:]                     # the 7 positive midpoints (fp64, exact)
+    assert len(mids) == 7 and min(mids) > 0
+    rng = np.random.default_rng(11)
+    abits = np.arange(1, 0x7F80, dtype=np.uint32)
+    a = (abits << 16).view(np.float32).astype(np.float64)
+    blocks = np.zeros((abits.size, 64), np.uint32)
+    blocks[:, 0] = abits
+    for k, m in enumerate(mids):
+        c = _ceil_bf16_bits(a * m)
+        below = np.where(c > 0, c - 1, 0)
+        blocks[:, 1 + 4 * k] = c
+        blocks[:, 2 + 4 * k] = c | 0x8000
+        blocks[:, 3 + 4 * k] = below
+        blocks[:, 4 + 4 * k] = below | 0x8000
+    rest = (rng.uniform(-1.0, 1.0, (abits.size, 64 - 29)) * a[:, None]).astype(np.float32)
+    blocks[:, 29:] = synth.to_bf16(rest).view(torch.int16).numpy().astype(np.uint32) & 0xFFFF
+    return torch.from_numpy(blocks.astype(np.uint16).view(np.int16).ravel()).view(torch.bfloat16)
 
 
 WEIGHTS = list(_weights())
@@ -54,6 +88,25 @@ def test_nf4_dq_bitexact(name, W):
         wd = B.dequantize(qw).float().cpu().numpy().ravel()
         ref_wd = o.nf4_dequant(ref_codes, o.dq_decode(ref_qa, ref_gs, ref_mu), n)
         assert np.array_equal(_u32(wd), _u32(ref_wd))
+    assert B.device_status() == B.QL_OK
+
+
+@pytest.mark.parametrize("name,W", WEIGHTS, ids=[w[0] for w in WEIGHTS])
+def test_nf4_dq_fused_matches_two_step(name, W):
+    """The one-call NF4 + double quantisation gives the same bits as the two calls, and
+    the oracle's."""
+    Wd = W.cuda().contiguous().view(-1)
+    codes, absmax, qa, gs, mu = B.nf4_dq_quantize(Wd)
+    c2, a2 = B.nf4_quantize(Wd)
+    qa2, gs2, mu2 = B.dq_quantize(a2)
+    for x, y in ((codes, c2), (absmax, a2), (qa, qa2), (gs, gs2), (mu, mu2)):
+        assert torch.equal(x.view(torch.uint8), y.view(torch.uint8))
+    ref_codes, ref_a = o.nf4_quantize(W.float().numpy().ravel())
+    ref_qa, ref_gs, ref_mu = o.dq_encode(ref_a)
+    assert np.array_equal(codes.cpu().numpy(), ref_codes)
+    assert np.array_equal(qa.cpu().numpy(), ref_qa)
+    assert np.array_equal(_u32(gs.cpu().numpy()), _u32(ref_gs))
+    assert _u32(mu.cpu().numpy())[0] == _u32(np.float32(ref_mu))
     assert B.device_status() == B.QL_OK
 
 
