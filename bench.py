@@ -31,6 +31,27 @@ sys.path.insert(0, ROOT)
 METRIC = "fused NF4+LoRA linear TFLOP/s & HBM GB/s (% of roofline); quantize GB/s"
 NF4_DQ_BYTES_PER_PARAM = 2.0 + 0.5 + 1.0 / 64 + 4.0 / 16384   # bf16 read + codes + consts
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the fused
+# forward GEMM on this workload, from one ncu capture (profiles/fwd_main_gemm_upproj_11008x4096_M8192.md),
+# valid only for the kernel sources it was taken on: reported as null once they change.
+FWD_MAIN_TRAFFIC = {"bytes": 105957376 + 150237952, "sources_sha256_16": "c9105cab3bd39074"}
+FWD_MAIN_SOURCES = ("quantized_base_rank_b200/csrc/gemm.cuh", "quantized_base_rank_b200/csrc/sm100.cuh",
+                    "quantized_base_rank_b200/csrc/linear.cu", "quantized_base_rank_b200/csrc/common.cuh")
+
+
+def sources_sha256_16(paths) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in paths:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def fwd_main_traffic():
+    ok = sources_sha256_16(FWD_MAIN_SOURCES) == FWD_MAIN_TRAFFIC["sources_sha256_16"]
+    return FWD_MAIN_TRAFFIC["bytes"] if ok else None
+
 
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -392,7 +413,8 @@ def run_ours(args, case, world, rank, local_rank):
                    "parallelism": f"dp{world}" if world > 1 else "single"},
         "roofline": {"kernel": "fused forward GEMM (NF4 decode + X W'^T + P B^T)", "bound": "tensor",
                      "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                     "frac": achieved / peaks["bf16_tflops"], "traffic": fwd_main_traffic(),
+                     "traffic_unit": "bytes per launch (ncu dram read + write)",
                      "peak_source": f"{peaks['source']} bf16 burst",
                      "frac_of_sustained": (achieved / peaks["bf16_tflops_sustained"]
                                            if peaks["bf16_tflops_sustained"] else None)},
@@ -422,6 +444,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--part", choices=["all", "decode"], default="all",
+                    help="decode: only the decode-shaped forward component (a short run for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -439,6 +463,13 @@ def main():
         import torch.distributed as dist
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if args.part == "decode":
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        out = decode_bench(dev, load_peaks(), reps=args.steps)
+        if rank == 0:
+            print(json.dumps({"part": "decode", "decode_7b_4096x4096_nf4": out}), flush=True)
+        return
     try:
         run_ours(args, case, world, rank, local_rank)
     finally:
