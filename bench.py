@@ -257,7 +257,7 @@ def decode_bench(dev, peaks, reps: int = 20):
 
 def run_ours(args, case, world, rank, local_rank):
     from quantized_base_rank_b200 import binding as B
-    from quantized_base_rank_b200 import synth
+    from quantized_base_rank_b200 import dp, synth
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -289,8 +289,7 @@ def run_ours(args, case, world, rank, local_rank):
         B.linear_fwd(qw, X, A, Bm, case.alpha, Y=Y, T=T)
         B.linear_bwd(qw, X, dY, A, Bm, T, case.alpha, dX=dX, dA=dA, dB=dB)
         if dist is not None:
-            dist.all_reduce(dA)
-            dist.all_reduce(dB)
+            dp.allreduce_adapter_grads(dA, dB)
 
     def barrier():
         if dist is not None:

@@ -327,23 +327,34 @@ def linear_fwd(X, Wd, A, B, alpha: float, r: int):
     return Y, T
 
 
-def linear_bwd(X, dY, Wd, A, B, alpha: float, r: int):
-    """Gradients of Y = X Wd^T + s (X A^T) B^T with Wd frozen, fp64.
-
-    U = dY B;  dX = dY Wd + s U A;  dA = s U^T X;  dB = s dY^T T  (T = X A^T).
-    Returns (dX, dA, dB).
-    """
+def adapter_grads(X, dY, A, B, alpha: float, r: int):
+    """The adapter gradients alone, fp64: dA = s U^T X and dB = s dY^T T, with
+    U = dY B and T = X A^T. They need no weight, so large layers can be checked in full
+    without the dX product."""
     X = np.asarray(X, np.float64)
     dY = np.asarray(dY, np.float64)
-    Wd = np.asarray(Wd, np.float64)
     A = np.asarray(A, np.float64)
     B = np.asarray(B, np.float64)
     s = alpha / r
     T = X @ A.T
     U = dY @ B
+    return s * (U.T @ X), s * (dY.T @ T)
+
+
+def linear_bwd(X, dY, Wd, A, B, alpha: float, r: int):
+    """Gradients of Y = X Wd^T + s (X A^T) B^T with Wd frozen, fp64.
+
+    U = dY B;  dX = dY Wd + s U A;  dA = s U^T X;  dB = s dY^T T  (T = X A^T).
+    Returns (dX, dA, dB). dX of a subset of rows needs only those rows of dY.
+    """
+    dY = np.asarray(dY, np.float64)
+    Wd = np.asarray(Wd, np.float64)
+    A = np.asarray(A, np.float64)
+    B = np.asarray(B, np.float64)
+    s = alpha / r
+    U = dY @ B
     dX = dY @ Wd + s * (U @ A)
-    dA = s * (U.T @ X)
-    dB = s * (dY.T @ T)
+    dA, dB = adapter_grads(X, dY, A, B, alpha, r)
     return dX, dA, dB
 
 

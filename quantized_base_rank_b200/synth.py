@@ -119,3 +119,24 @@ def layer_mix_65b(n_layers: int = 80, seed: int = 0):
     fmts = g.integers(0, 2, size=n_layers)
     ranks = g.integers(0, 4, size=n_layers)
     return [("nf4_dq" if f == 0 else "int8", (8, 16, 32, 64)[r]) for f, r in zip(fmts, ranks)]
+
+
+def stack_index(layer: int, which: int, slot: int) -> int:
+    """Sub-stream of tensor `slot` (W_IDX, X_IDX, A_IDX, B_IDX or DY_IDX) of linear `which`
+    of decoder layer `layer` in a multi-layer stack."""
+    return 100000 + (layer * 8 + which) * 8 + slot
+
+
+def stack_linear_inputs(layer: int, which: int, N: int, K: int, M: int, r: int, seed: int = 0,
+                        device="cuda", backward: bool = True) -> dict:
+    """Device bf16 tensors of one linear of a stack: W ~ N(0, 0.02) [N, K], X ~ N(0, 1)
+    [M, K], A ~ N(0, 1/K) [r, K], B ~ N(0, 0.01) [N, r] and dY ~ N(0, 1) [M, N], each from
+    its own Philox sub-stream."""
+    idx = lambda slot: stack_index(layer, which, slot)
+    out = {"W": device_normal_bf16((N, K), 0.02, seed, idx(W_IDX), device),
+           "X": device_normal_bf16((M, K), 1.0, seed, idx(X_IDX), device),
+           "A": device_normal_bf16((r, K), 1.0 / K, seed, idx(A_IDX), device),
+           "B": device_normal_bf16((N, r), 0.01, seed, idx(B_IDX), device)}
+    if backward:
+        out["dY"] = device_normal_bf16((M, N), 1.0, seed, idx(DY_IDX), device)
+    return out

@@ -1,0 +1,80 @@
+"""Data parallelism over tokens, world size 2 on CPU with the gloo backend.
+
+Each rank takes its token shard, computes its partial adapter gradients with the oracle
+(fp64 on the host; the GPU kernels compute the same partial sums on the device), and the
+ranks exchange them with dp.allreduce_adapter_grads. The sum must equal the full-batch
+gradients, and each rank's dX rows must equal the full-batch rows of its shard."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import oracle.qlora_oracle as o
+from quantized_base_rank_b200 import dp, synth
+
+
+def test_shards_cover_every_row_once():
+    for M in (0, 1, 2, 3, 7, 64, 8191, 8192):
+        for world in (1, 2, 3, 4, 8):
+            spans = [dp.shard_rows(M, world, r) for r in range(world)]
+            assert spans[0][0] == 0 and spans[-1][1] == M
+            assert all(a[1] == b[0] for a, b in zip(spans, spans[1:]))
+            sizes = [e - s for s, e in spans]
+            assert max(sizes) - min(sizes) <= 1
+    with pytest.raises(ValueError):
+        dp.shard_rows(8, 2, 2)
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+CASE = synth.LinearCase("dp-ragged", N=192, K=256, M=131, r=8, alpha=16.0, seed=3)
+
+
+def _worker(rank, world, port, results):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        inp = synth.make_inputs(CASE)
+        wd = o.quantize_weight(inp["W"].float().numpy(), CASE.fmt)["wdeq"].reshape(CASE.N, CASE.K)
+        s0, s1 = dp.shard_rows(CASE.M, world, rank)
+        f = lambda t: t.float().numpy().astype(np.float64)
+        X, dY, A, B = f(inp["X"])[s0:s1], f(inp["dY"])[s0:s1], f(inp["A"]), f(inp["B"])
+        dX, dA, dB = o.linear_bwd(X, dY, wd, A, B, CASE.alpha, CASE.r)
+        tA = torch.from_numpy(dA.astype(np.float32))
+        tB = torch.from_numpy(dB.astype(np.float32))
+        dp.allreduce_adapter_grads(tA, tB)
+        results[rank] = (s0, s1, dX, tA.numpy(), tB.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_allreduce_of_partial_gradients_equals_full_batch():
+    world = 2
+    mgr = mp.get_context("spawn").Manager()
+    results = mgr.dict()
+    mp.start_processes(_worker, args=(world, _free_port(), results), nprocs=world, join=True,
+                       start_method="spawn")
+    inp = synth.make_inputs(CASE)
+    wd = o.quantize_weight(inp["W"].float().numpy(), CASE.fmt)["wdeq"].reshape(CASE.N, CASE.K)
+    f = lambda t: t.float().numpy().astype(np.float64)
+    dX, dA, dB = o.linear_bwd(f(inp["X"]), f(inp["dY"]), wd, f(inp["A"]), f(inp["B"]), CASE.alpha, CASE.r)
+    covered = 0
+    for rank in range(world):
+        s0, s1, dXr, dAr, dBr = results[rank]
+        covered += s1 - s0
+        np.testing.assert_allclose(dXr, dX[s0:s1], rtol=0, atol=1e-12)
+        # the exchange sums fp32 partials; the reference is the fp64 full batch
+        np.testing.assert_allclose(dAr, dA, rtol=1e-5, atol=1e-6 * np.abs(dA).max())
+        np.testing.assert_allclose(dBr, dB, rtol=1e-5, atol=1e-6 * np.abs(dB).max())
+        if rank:
+            assert np.array_equal(dAr, results[0][3]) and np.array_equal(dBr, results[0][4])
+    assert covered == CASE.M
