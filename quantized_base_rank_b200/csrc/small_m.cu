@@ -36,6 +36,7 @@ struct SmallArgs {
   const float* absmax;
   uint16_t* Y; uint16_t* T_save;
   int kr_max;                      // max K-range per CTA, in elements
+  int b_pairs;                     // r even and B 4-byte aligned
   float q[16];
 };
 
@@ -101,32 +102,46 @@ __device__ __forceinline__ uint2 small_int8_decode4(uint32_t w, float sc) {
   return make_uint2(pack_bf16x2(f0, f1), pack_bf16x2(f2, f3));
 }
 
-// The codes and scale of one block (row, block index) for one lane.
+// The codes and the raw constants of one block (row, block index) for one lane. Loading
+// does no arithmetic on the loaded values, so several units' loads can be in flight at
+// once; unit_scale() turns the constants into the block scale at first use.
 template <int FMT>
 struct UnitRegs {
   uint4 c[FMT == QL_FMT_NF4_DQ ? 2 : 4];
-  float sc;
+  int qa;         // NF4: the int8 double-quantised constant
+  float f;        // NF4: the group scale; int8: the fp32 absmax
 };
 
 template <int FMT>
-__device__ __forceinline__ void load_block_regs(const SmallArgs& a, int64_t row, int64_t kb, float mu,
-                                                UnitRegs<FMT>& u) {
+__device__ __forceinline__ void load_block_regs(const SmallArgs& a, int64_t row, int64_t kb, UnitRegs<FMT>& u) {
   const int64_t KB = a.K >> 6;
   constexpr int NV = FMT == QL_FMT_NF4_DQ ? 2 : 4;
   if (row >= a.N || kb >= KB) {
 #pragma unroll
     for (int i = 0; i < NV; ++i) u.c[i] = make_uint4(0u, 0u, 0u, 0u);
-    u.sc = 0.0f;
+    u.qa = 0;
+    u.f = 0.0f;
     return;
   }
   const int64_t blk = row * KB + kb;
   const uint4* src = reinterpret_cast<const uint4*>(a.codes + blk * (FMT == QL_FMT_NF4_DQ ? 32 : 64));
 #pragma unroll
   for (int i = 0; i < NV; ++i) u.c[i] = __ldg(src + i);
-  if (FMT == QL_FMT_NF4_DQ)
-    u.sc = __fadd_rn(__fmul_rn((float)__ldg(a.qabsmax + blk), __ldg(a.gscale + (blk >> 8))), mu);
-  else
-    u.sc = __fdiv_rn(__ldg(a.absmax + blk), 127.0f);
+  if (FMT == QL_FMT_NF4_DQ) {
+    u.qa = __ldg(a.qabsmax + blk);
+    u.f = __ldg(a.gscale + (blk >> 8));
+  } else {
+    u.qa = 0;
+    u.f = __ldg(a.absmax + blk);
+  }
+}
+
+// NF4: a' = fp32(fp32(qabsmax * group_scale) + mean); int8: fp32(absmax / 127). Zero for a
+// block outside the weight.
+template <int FMT>
+__device__ __forceinline__ float unit_scale(const UnitRegs<FMT>& u, float mu) {
+  if (FMT == QL_FMT_NF4_DQ) return __fadd_rn(__fmul_rn((float)u.qa, u.f), mu);
+  return __fdiv_rn(u.f, 127.0f);
 }
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -179,26 +194,49 @@ small_m_fwd_kernel(const SmallArgs a) {
   const int64_t k0 = u0 * 256;
   const float mu = FMT == QL_FMT_NF4_DQ ? __ldg(a.mean) : 0.0f;
 
-  // The next launch on the stream may start now; it will stream its own weight while we
-  // finish. Everything below that reads X, A or B waits for the previous grid first.
+  // The next launch on the stream may start now and stream its own weight while this
+  // one finishes.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-  // first unit's codes go out before anything else (weights are never written by the
-  // preceding grid, so they may be read before the dependency wait)
+  // Everything that depends only on the weight and the adapter goes out before the
+  // dependency wait (the preceding grid never writes them): the codes of the first two
+  // units, the adapter rows in fragment order, and this warp's rows of B. Only the token
+  // rows wait.
   const int64_t row_g = n0 + warp * 16 + g, row_h = row_g + 8;
-  UnitRegs<FMT> cg, ch;
-  if (nunits > 0) {
-    load_block_regs<FMT>(a, row_g, u0 * 4 + q, mu, cg);
-    load_block_regs<FMT>(a, row_h, u0 * 4 + q, mu, ch);
+  // adapter right factor for this warp's rows (A fragments of the final MMA)
+  auto bload = [&](int64_t row, int j) -> uint32_t {
+    if (a.b_pairs)                                  // even r, 4-byte aligned B: j, j+1 in one word
+      return row < a.N && j < a.r ? __ldg(reinterpret_cast<const uint32_t*>(a.B + row * a.r + j)) : 0u;
+    if (row >= a.N) return 0u;
+    const uint32_t lo = j < a.r ? a.B[row * a.r + j] : 0u;
+    const uint32_t hi = j + 1 < a.r ? a.B[row * a.r + j + 1] : 0u;
+    return lo | (hi << 16);
+  };
+  uint32_t bfr[JT][4];
+#pragma unroll
+  for (int jt = 0; jt < JT; ++jt) {
+    const int j0 = jt * 16 + 2 * q;
+    bfr[jt][0] = bload(row_g, j0);
+    bfr[jt][1] = bload(row_h, j0);
+    bfr[jt][2] = bload(row_g, j0 + 8);
+    bfr[jt][3] = bload(row_h, j0 + 8);
   }
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-
-  // token rows and adapter rows of the K-range -> smem in fragment order (zero beyond the
-  // tokens, the rank and K): one 16-byte global load feeds two 8-byte fragment slots. The
-  // loads of a batch are all issued before any of its stores, so their latencies overlap.
-  {
-    const int per_row = nunits * 32;                // 16-byte vectors per row
-    const int total = (NT + RP) * per_row;
+  UnitRegs<FMT> cg, ch, ng, nh;
+  if (nunits > 0) {
+    load_block_regs<FMT>(a, row_g, u0 * 4 + q, cg);
+    load_block_regs<FMT>(a, row_h, u0 * 4 + q, ch);
+  }
+  if (nunits > 1) {
+    load_block_regs<FMT>(a, row_g, (u0 + 1) * 4 + q, ng);
+    load_block_regs<FMT>(a, row_h, (u0 + 1) * 4 + q, nh);
+  }
+  // rows [row_begin, row_end) of the staged block (tokens 0..NT-1, then adapter rows) ->
+  // smem in fragment order (zero beyond the tokens, the rank and K): one 16-byte global
+  // load feeds two 8-byte fragment slots. The loads of a batch are all issued before any
+  // of its stores, so their latencies overlap.
+  const int per_row = nunits * 32;                  // 16-byte vectors per row
+  auto stage_rows = [&](int row_begin, int row_end) {
+    const int total = (row_end - row_begin) * per_row;
     constexpr int kBatch = 8;
     for (int v0 = 0; v0 < total; v0 += kBatch * 256) {
       uint4 val[kBatch];
@@ -207,7 +245,7 @@ small_m_fwd_kernel(const SmallArgs a) {
         const int v = v0 + b * 256 + threadIdx.x;
         val[b] = make_uint4(0u, 0u, 0u, 0u);
         if (v < total) {
-          const int row = v / per_row, rem = v % per_row;
+          const int row = row_begin + v / per_row, rem = v % per_row;
           const int64_t k = k0 + (rem >> 5) * 256 + 64 * ((rem >> 3) & 3) + 8 * (rem & 7);
           if (row < NT) {
             if (row < a.M && k < a.K) val[b] = __ldg(reinterpret_cast<const uint4*>(a.X + row * a.K + k));
@@ -220,7 +258,7 @@ small_m_fwd_kernel(const SmallArgs a) {
       for (int b = 0; b < kBatch; ++b) {
         const int v = v0 + b * 256 + threadIdx.x;
         if (v < total) {
-          const int row = v / per_row, rem = v % per_row;
+          const int row = row_begin + v / per_row, rem = v % per_row;
           const int ul = rem >> 5, qq = (rem >> 3) & 3, ii = rem & 7;
           uint8_t* p = (row < NT ? sX + (size_t)row * pitch : sA + (size_t)(row - NT) * pitch) + ul * 512;
           *reinterpret_cast<uint2*>(p + ((2 * ii) * 4 + qq) * 8) = make_uint2(val[b].x, val[b].y);
@@ -228,25 +266,10 @@ small_m_fwd_kernel(const SmallArgs a) {
         }
       }
     }
-  }
-  // adapter right factor for this warp's rows (A fragments of the final MMA)
-  auto bload = [&](int64_t row, int j) -> uint32_t {
-    if (row >= a.N) return 0u;
-    const uint32_t lo = j < a.r ? a.B[row * a.r + j] : 0u;
-    const uint32_t hi = j + 1 < a.r ? a.B[row * a.r + j + 1] : 0u;
-    return lo | (hi << 16);
   };
-  uint32_t bfr[JT][4];
-#pragma unroll
-  for (int jt = 0; jt < JT; ++jt) {
-    {
-      const int j0 = jt * 16 + 2 * q;
-      bfr[jt][0] = bload(row_g, j0);
-      bfr[jt][1] = bload(row_h, j0);
-      bfr[jt][2] = bload(row_g, j0 + 8);
-      bfr[jt][3] = bload(row_h, j0 + 8);
-    }
-  }
+  stage_rows(NT, NT + RP);                          // adapter rows
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  stage_rows(0, NT);                                // token rows
   __syncthreads();
 
   // ---- main loop: W' rows (decoded) and, for the adapter, A rows against the tokens ----
@@ -258,11 +281,14 @@ small_m_fwd_kernel(const SmallArgs a) {
 #pragma unroll
     for (int jt = 0; jt < JT; ++jt) dt[jt][t][0] = dt[jt][t][1] = dt[jt][t][2] = dt[jt][t][3] = 0.0f;
   }
+  // Register ring of the codes: units ul and ul + 1 are held; with DEPTH 3 unit ul + 2 is
+  // loaded at the top of iteration ul, with DEPTH 2 at its end (fewer registers).
+  constexpr int DEPTH = (FMT == QL_FMT_NF4_DQ && NT * JT <= 16) ? 3 : 2;
   for (int ul = 0; ul < nunits; ++ul) {
-    UnitRegs<FMT> ng, nh;
-    if (ul + 1 < nunits) {
-      load_block_regs<FMT>(a, row_g, (u0 + ul + 1) * 4 + q, mu, ng);
-      load_block_regs<FMT>(a, row_h, (u0 + ul + 1) * 4 + q, mu, nh);
+    UnitRegs<FMT> mg, mh;                            // unit ul + 2
+    if (DEPTH == 3 && ul + 2 < nunits) {
+      load_block_regs<FMT>(a, row_g, (u0 + ul + 2) * 4 + q, mg);
+      load_block_regs<FMT>(a, row_h, (u0 + ul + 2) * 4 + q, mh);
     }
     const uint8_t* xu = sX + ul * 512 + q * 8;
     const uint8_t* au = sA + ul * 512 + q * 8;
@@ -285,8 +311,8 @@ small_m_fwd_kernel(const SmallArgs a) {
     };
     if constexpr (FMT == QL_FMT_NF4_DQ) {
       uint32_t Lg[2], Hg[2], Lh[2], Hh[2];
-      small_nf4_table(a.q, cg.sc, Lg, Hg);
-      small_nf4_table(a.q, ch.sc, Lh, Hh);
+      small_nf4_table(a.q, unit_scale<FMT>(cg, mu), Lg, Hg);
+      small_nf4_table(a.q, unit_scale<FMT>(ch, mu), Lh, Hh);
       const uint32_t wg[8] = {cg.c[0].x, cg.c[0].y, cg.c[0].z, cg.c[0].w, cg.c[1].x, cg.c[1].y, cg.c[1].z, cg.c[1].w};
       const uint32_t wh[8] = {ch.c[0].x, ch.c[0].y, ch.c[0].z, ch.c[0].w, ch.c[1].x, ch.c[1].y, ch.c[1].z, ch.c[1].w};
 #pragma unroll
@@ -301,14 +327,23 @@ small_m_fwd_kernel(const SmallArgs a) {
                                cg.c[2].x, cg.c[2].y, cg.c[2].z, cg.c[2].w, cg.c[3].x, cg.c[3].y, cg.c[3].z, cg.c[3].w};
       const uint32_t wh[16] = {ch.c[0].x, ch.c[0].y, ch.c[0].z, ch.c[0].w, ch.c[1].x, ch.c[1].y, ch.c[1].z, ch.c[1].w,
                                ch.c[2].x, ch.c[2].y, ch.c[2].z, ch.c[2].w, ch.c[3].x, ch.c[3].y, ch.c[3].z, ch.c[3].w};
+      const float scg = unit_scale<FMT>(cg, mu), sch = unit_scale<FMT>(ch, mu);
 #pragma unroll
       for (int st = 0; st < 16; ++st) {
-        const uint2 eg = small_int8_decode4(wg[st], cg.sc);
-        const uint2 eh = small_int8_decode4(wh[st], ch.sc);
+        const uint2 eg = small_int8_decode4(wg[st], scg);
+        const uint2 eh = small_int8_decode4(wh[st], sch);
         step(st, eg.x, eh.x, eg.y, eh.y);
       }
     }
     if (ul + 1 < nunits) { cg = ng; ch = nh; }
+    if (ul + 2 < nunits) {
+      if (DEPTH == 3) {
+        ng = mg; nh = mh;
+      } else {
+        load_block_regs<FMT>(a, row_g, (u0 + ul + 2) * 4 + q, ng);
+        load_block_regs<FMT>(a, row_h, (u0 + ul + 2) * 4 + q, nh);
+      }
+    }
   }
 
   // ---- adapter term of this K-range: D += B[rows, :] (s T_kr) ----
@@ -433,6 +468,7 @@ ql_status small_m_forward(const ql_weight* w, const uint16_t* X, int64_t M, cons
   a.Y = Y; a.T_save = T_save;
   const int64_t U = (w->K + 255) / 256;
   a.kr_max = (int)(((U + kCS - 1) / kCS) * 256);
+  a.b_pairs = (r % 2 == 0 && aligned(B, 4)) ? 1 : 0;
   const Nf4Tables& t = nf4_tables();
   for (int i = 0; i < 16; ++i) a.q[i] = t.q[i];
   ProfScope prof(PK_FWD_SMALL, st, 1);
