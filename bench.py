@@ -261,6 +261,7 @@ def run_ours(args, case, world, rank, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
+    B.lib().ql_set_gemm_pair(1 if args.gemm == "pair" else 0)
     dist = None
     if world > 1:
         import torch.distributed as dist
@@ -409,7 +410,8 @@ def run_ours(args, case, world, rank, local_rank):
         "config": {"workload": case.name, "M": M, "N": N, "K": K, "r": r, "alpha": case.alpha,
                    "format": "nf4_dq", "step": "quantise(NF4+DQ) + fwd + bwd(dX,dA,dB)",
                    "l2": "inputs larger than L2 (X 64 MB, W 90 MB, dY 180 MB > 126 MB)",
-                   "parallelism": f"dp{world}" if world > 1 else "single"},
+                   "parallelism": f"dp{world}" if world > 1 else "single",
+                   "fused_gemm": "cta_pair" if args.gemm == "pair" else "single_cta"},
         "roofline": {"kernel": "fused forward GEMM (NF4 decode + X W'^T + P B^T)", "bound": "tensor",
                      "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": achieved / peaks["bf16_tflops"], "traffic": fwd_main_traffic(),
@@ -443,6 +445,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gemm", choices=["pair", "single"], default="single",
+                    help="fused weight GEMM on CTA pairs (cta_group::2) or on single CTAs")
     ap.add_argument("--part", choices=["all", "decode"], default="all",
                     help="decode: only the decode-shaped forward component (a short run for profiling)")
     args = ap.parse_args()

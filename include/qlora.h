@@ -178,6 +178,12 @@ size_t ql_workspace_bytes(int32_t op, int64_t M, int64_t N, int64_t K, int32_t r
  * device (QL_OK, QL_ERR_NONFINITE or QL_ERR_TIMEOUT). */
 ql_status ql_get_device_status(void* stream);
 
+/* Which fused weight GEMM the linear uses for M > 16: 0 (the default) runs it on single
+ * CTAs (128 weight rows x 256 tokens per tile), 1 on CTA pairs (two SMs share each tcgen05
+ * MMA, cta_group::2, 256 weight rows x 256 tokens). Both give the same results up to fp32
+ * summation order. Process-wide; meant for comparisons. */
+void ql_set_gemm_pair(int on);
+
 /* Upper bound, in nanoseconds, on every wait inside the GEMM kernels (0 restores the
  * default of 2 s). A wait that exceeds it makes the kernel give up cleanly and report
  * QL_ERR_TIMEOUT through ql_get_device_status. Process-wide; meant for diagnostics. */

@@ -53,6 +53,7 @@ _SIGS = {
     "ql_status_string": ([I32], ctypes.c_char_p),
     "ql_nf4_codebook": ([ctypes.POINTER(ctypes.c_float)], None),
     "ql_set_wait_timeout_ns": ([ctypes.c_uint64], None),
+    "ql_set_gemm_pair": ([ctypes.c_int], None),
     "ql_profile_enable": ([ctypes.c_int], None),
     "ql_profile_read": ([ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)], ctypes.c_int),
     "ql_launch_count": ([], ctypes.c_uint64),

@@ -195,8 +195,8 @@ template <int BN>
 struct TmaCfg {
   static constexpr int kABytes = 128 * 64 * 2;
   static constexpr int kBBytes = BN * 128;
-  static constexpr int kStages = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
-  static constexpr int kTmemCols = 2 * BN;
+  static constexpr int kStages = BN >= 192 ? 4 : (BN == 128 ? 6 : 8);
+  static constexpr int kTmemCols = 2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512);   // power of two
   static constexpr size_t kSmem = (size_t)kStages * (kABytes + kBBytes) + 2048;
 };
 
@@ -587,6 +587,307 @@ qgemm_wdec_kernel(const __grid_constant__ CUtensorMap tmT, const __grid_constant
   tc_fence_before();
   __syncthreads();
   if (warp == 5) { tc_fence_after(); tmem_dealloc(tmem_base, Cfg::kTmemCols); }
+  if (threadIdx.x == 0 && *abort_word) raise_flag(args.flag, kFlagTimeout);
+}
+
+// =================================================================================
+// The same decode GEMM on a CTA pair (cta_group::2): one MMA of 256 weight rows x 256
+// tokens per 16-wide k step, issued by the even CTA. Each CTA decodes its own 128 weight
+// rows into its own shared memory and loads its own 128 token rows by TMA, so per SM the
+// token tile and its tensor-core reads are half of the single-CTA kernel's, which is
+// what bounds that kernel (shared-memory bandwidth). Every ring stays local to its CTA;
+// the odd CTA's MMA warp relays "stage s is full here" to the even CTA with one
+// cluster-scope arrive per stage, and the even CTA's commits free the stages of both.
+// =================================================================================
+template <BSrc BS>
+struct WpairCfg {
+  static constexpr int BM = 128;                                 // weight rows per CTA
+  static constexpr int BN = 256;                                 // tokens per pair tile
+  static constexpr int BNH = 128;                                // tokens per CTA
+  static constexpr int NP = 8;                                   // decode warps
+  static constexpr int kDBytes = BM * 128;                       // decoded weight stage
+  static constexpr int kTBytes = BNH * 128;                      // token stage (this CTA's half)
+  static constexpr int kCodeBytes = BM * (BS == BSrc::NF4 ? 32 : 64);
+  static constexpr int kCBytes = kCodeBytes + 1024;              // codes + scales
+  // decoded-weight stages (filled on this SM, short latency), token stages (TMA from L2,
+  // long latency: the deeper ring), code stages
+  static constexpr int SD = 4, ST = 8, SC = (BS == BSrc::NF4 ? 6 : 3);
+  static constexpr int kTmemCols = 512;
+  static constexpr int kThreads = (7 + NP) * 32;
+  static constexpr size_t kSmem = (size_t)SD * kDBytes + (size_t)ST * kTBytes + (size_t)SC * kCBytes + 2048;
+  static_assert(kSmem + 1024 <= 232448, "shared memory");
+};
+
+// First weight row (or input feature, for dX) that a CTA of the pair loads. When the odd
+// CTA's whole 128-row half lies past the end (R not a multiple of 256), it loads the even
+// CTA's rows instead, so no box starts past the end of a tensor; the outputs of those
+// rows are never stored.
+__device__ __forceinline__ int32_t load_row0(int32_t w0, int64_t R) {
+  return (int64_t)w0 >= R ? w0 - 128 : w0;
+}
+
+template <BSrc BS, bool W_MN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(WpairCfg<BS>::kThreads, 1)
+qgemm_wpair_kernel(const __grid_constant__ CUtensorMap tmT, const __grid_constant__ CUtensorMap tmCodes,
+                   const __grid_constant__ CUtensorMap tmScale, const __grid_constant__ CUtensorMap tmTe,
+                   const __grid_constant__ CUtensorMap tmWe, const GemmArgs args) {
+  using Cfg = WpairCfg<BS>;
+  constexpr int BM = Cfg::BM, BN = Cfg::BN, BNH = Cfg::BNH, NP = Cfg::NP, SD = Cfg::SD, ST = Cfg::ST,
+                SC = Cfg::SC;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sD = smem;                                   // decoded weight (A operand rows of this CTA)
+  uint8_t* sT = sD + SD * Cfg::kDBytes;                 // tokens (this CTA's half of B)
+  uint8_t* sC = sT + ST * Cfg::kTBytes;                 // codes + scales
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sC + SC * Cfg::kCBytes);
+  const uint32_t full_d = smem_u32(bars);
+  const uint32_t empty_d = full_d + 8 * SD;
+  const uint32_t full_t = empty_d + 8 * SD;
+  const uint32_t empty_t = full_t + 8 * ST;
+  const uint32_t peer_ready = empty_t + 8 * ST;         // even CTA: the odd CTA's chunk g is in
+  const uint32_t full_c = peer_ready + 8 * ST;
+  const uint32_t empty_c = full_c + 8 * SC;
+  const uint32_t acc_full = empty_c + 8 * SC;
+  const uint32_t acc_empty = acc_full + 16;             // even CTA: epilogue warps of both CTAs
+  const uint32_t drain = acc_full + 32;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * SD + 3 * ST + 2 * SC + 5);
+  volatile int* abort_word = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SD; ++s) { mbar_init(full_d + 8 * s, NP); mbar_init(empty_d + 8 * s, 1); }
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(full_t + 8 * s, 1); mbar_init(empty_t + 8 * s, 1); mbar_init(peer_ready + 8 * s, 1);
+    }
+    for (int s = 0; s < SC; ++s) { mbar_init(full_c + 8 * s, 1); mbar_init(empty_c + 8 * s, NP); }
+    for (int i = 0; i < 2; ++i) { mbar_init(acc_full + 8 * i, 1); mbar_init(acc_empty + 8 * i, 8); }
+    mbar_init(drain, 1);
+    *abort_word = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&tmT);
+    if (args.n_ext) tma_prefetch_desc(&tmTe);
+  }
+  if (warp == 6 && lane == 0) { tma_prefetch_desc(&tmCodes); tma_prefetch_desc(&tmScale); }
+  if (warp == 7 && lane == 0 && args.n_ext) tma_prefetch_desc(&tmWe);
+  if (warp == 5) tmem_alloc_pair(smem_u32(tmem_holder), Cfg::kTmemCols);
+  tc_fence_before();
+  cluster_sync();                                       // barriers of both CTAs initialised
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  // pair tiles: 256 weight rows x 256 tokens, weight-row tiles fastest
+  const int64_t w_tiles = (args.R + 2 * BM - 1) / (2 * BM);
+  const int64_t tiles = w_tiles * ((args.Cn + BN - 1) / BN);
+  const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int kc_main = (int)((args.Kc + 63) / 64);
+  const int kc_total = kc_main + args.n_ext;
+  const uint64_t lim = args.timeout_ns;
+  const uint32_t row_off = rank * BM;                   // this CTA's rows within the pair tile
+
+  if (warp < 4) {
+    // ---- epilogue: this CTA's 128 weight rows (TMEM lanes) x the tile's 256 tokens ----
+    const uint32_t acc_empty_lead = mapa_shared(acc_empty, 0);
+    uint32_t tcount = 0;
+    for (int64_t t = pair; t < tiles; t += npairs, ++tcount) {
+      const uint32_t acc = tcount & 1, aph = (tcount >> 1) & 1;
+      const bool okw = mbar_wait(acc_full + 8 * acc, aph, lim, abort_word);
+      if (!__all_sync(0xFFFFFFFFu, okw)) break;
+      tc_fence_after();
+      const int64_t w0 = (t % w_tiles) * 2 * BM + row_off, t0 = (t / w_tiles) * BN;
+      const int64_t wrow = w0 + warp * 32 + lane;
+#pragma unroll 1
+      for (int cc = 0; cc < BN; cc += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(warp * 32) << 16) + acc * BN + cc, v);
+        if (t0 + cc < args.Cn) epilogue_store_t(args, wrow, t0 + cc, v);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(acc_empty_lead + 8 * acc);
+    }
+  } else if (warp == 4 && lane == 0) {
+    // ---- this CTA's token rows -> T ring ----
+    uint32_t g = 0;
+    bool ok = true;
+    for (int64_t t = pair; t < tiles && ok; t += npairs) {
+      int32_t t0 = (int32_t)((t / w_tiles) * BN + rank * BNH);
+      if (t0 >= args.Cn) t0 -= BNH;                      // whole half past the tokens: as load_row0
+      for (int kc = 0; kc < kc_total; ++kc, ++g) {
+        const uint32_t s = g % ST, ph = (g / ST) & 1;
+        if (!mbar_wait(empty_t + 8 * s, ph ^ 1, lim, abort_word)) { ok = false; break; }
+        const uint32_t fb = full_t + 8 * s;
+        mbar_arrive_expect_tx(fb, Cfg::kTBytes);
+        if (kc < kc_main) tma_load_2d(smem_u32(sT + s * Cfg::kTBytes), &tmT, fb, kc * 64, t0);
+        else tma_load_2d(smem_u32(sT + s * Cfg::kTBytes), &tmTe, fb, (kc - kc_main) * 64, t0);
+      }
+    }
+    if (!ok || *abort_word)
+      for (uint32_t j = (g > (uint32_t)ST ? g - ST : 0); j < g; ++j) drain_wait(full_t + 8 * (j % ST), (j / ST) & 1);
+  } else if (warp == 6 && lane == 0) {
+    // ---- this CTA's weight codes + block scales -> C ring ----
+    uint32_t gc = 0;
+    bool ok = true;
+    for (int64_t t = pair; t < tiles && ok; t += npairs) {
+      const int32_t w0 = load_row0((int32_t)((t % w_tiles) * 2 * BM + row_off), args.R);
+      for (int kc = 0; kc < kc_main; ++kc, ++gc) {
+        const uint32_t s = gc % SC, ph = (gc / SC) & 1;
+        if (!mbar_wait(empty_c + 8 * s, ph ^ 1, lim, abort_word)) { ok = false; break; }
+        const uint32_t fb = full_c + 8 * s;
+        const uint32_t dst = smem_u32(sC + s * Cfg::kCBytes);
+        if (!W_MN) {
+          mbar_arrive_expect_tx(fb, Cfg::kCodeBytes + BM * 4);
+          tma_load_2d(dst, &tmCodes, fb, kc * (BS == BSrc::NF4 ? 32 : 64), w0);
+          tma_load_2d(dst + Cfg::kCodeBytes, &tmScale, fb, w0, kc);
+        } else {
+          mbar_arrive_expect_tx(fb, Cfg::kCodeBytes + 1024);
+          tma_load_2d(dst, &tmCodes, fb, BS == BSrc::NF4 ? w0 / 2 : w0, kc * 64);
+          tma_load_2d(dst + Cfg::kCodeBytes, &tmScale, fb, (w0 / 64) & ~3, kc * 64);
+        }
+      }
+    }
+    if (!ok || *abort_word)
+      for (uint32_t j = (gc > (uint32_t)SC ? gc - SC : 0); j < gc; ++j) drain_wait(full_c + 8 * (j % SC), (j / SC) & 1);
+  } else if (warp == 5 && lane == 0 && leader) {
+    // ---- MMA issuer (even CTA) ----
+    constexpr uint32_t kIdMain = idesc_bf16_f32(2 * BM, BN, W_MN ? 1 : 0, 0);
+    constexpr uint32_t kIdExt = idesc_bf16_f32(2 * BM, BN, 0, 0);
+    uint32_t g = 0, tcount = 0;
+    bool ok = true;
+    for (int64_t t = pair; t < tiles && ok; t += npairs, ++tcount) {
+      const uint32_t acc = tcount & 1, aph = (tcount >> 1) & 1;
+      if (!mbar_wait(acc_empty + 8 * acc, aph ^ 1, lim, abort_word)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * BN;
+      for (int kc = 0; kc < kc_total; ++kc, ++g) {
+        const uint32_t sd = g % SD, pd = (g / SD) & 1, st = g % ST, pt = (g / ST) & 1;
+        if (!mbar_wait(full_t + 8 * st, pt, lim, abort_word)) { ok = false; break; }
+        if (!mbar_wait(full_d + 8 * sd, pd, lim, abort_word)) { ok = false; break; }
+        if (!mbar_wait(peer_ready + 8 * st, pt, lim, abort_word)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_base = smem_u32(sD + sd * Cfg::kDBytes);
+        const uint32_t t_base = smem_u32(sT + st * Cfg::kTBytes);
+        const bool ext = kc >= kc_main;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint64_t ad = (!W_MN || ext) ? smem_desc_sw128(d_base + k * 32, 16, 1024)
+                                             : smem_desc_sw128(d_base + k * 2048, 8192, 1024);
+          const uint64_t bd = smem_desc_sw128(t_base + k * 32, 16, 1024);
+          tc_mma_pair(d_tmem, ad, bd, ext ? kIdExt : kIdMain, (kc > 0 || k > 0) ? 1u : 0u);
+        }
+        tc_commit_pair_mc(empty_d + 8 * sd, 0x3);
+        tc_commit_pair_mc(empty_t + 8 * st, 0x3);
+      }
+      if (!ok) break;
+      tc_commit_pair_mc(acc_full + 8 * acc, 0x3);
+    }
+    if (!ok || *abort_word) { tc_commit_pair(drain); drain_wait(drain, 0); }
+  } else if (warp == 5 && lane == 0) {
+    // ---- relay (odd CTA): tell the even CTA when a stage is full here ----
+    const uint32_t ready_lead = mapa_shared(peer_ready, 0);
+    uint32_t g = 0;
+    bool ok = true;
+    for (int64_t t = pair; t < tiles && ok; t += npairs) {
+      for (int kc = 0; kc < kc_total; ++kc, ++g) {
+        const uint32_t sd = g % SD, pd = (g / SD) & 1, st = g % ST, pt = (g / ST) & 1;
+        if (!mbar_wait(full_t + 8 * st, pt, lim, abort_word)) { ok = false; break; }
+        if (!mbar_wait(full_d + 8 * sd, pd, lim, abort_word)) { ok = false; break; }
+        mbar_arrive_remote(ready_lead + 8 * st);      // never laps: the MMA frees slots first
+      }
+    }
+  } else if (warp >= 7) {
+    // ---- decode: C ring -> D ring (bf16, swizzled UMMA layout), two lanes per block ----
+    const int tid = threadIdx.x - 7 * 32;                        // 0..255
+    const int blk = tid >> 1, half = tid & 1;                    // block 0..127
+    float q[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) q[i] = args.q[i];
+    int code_off, j_row = 0, gi = 0;
+    uint32_t d_off, key;
+    if (!W_MN) {
+      code_off = blk * (BS == BSrc::NF4 ? 32 : 64);
+      d_off = blk * 128;
+      key = blk & 7;
+    } else {
+      j_row = blk & 63;
+      gi = blk >> 6;
+      code_off = j_row * (BS == BSrc::NF4 ? 64 : 128) + gi * (BS == BSrc::NF4 ? 32 : 64);
+      d_off = gi * 8192 + (j_row >> 3) * 1024 + (j_row & 7) * 128;
+      key = j_row & 7;
+    }
+    uint32_t gc = 0, gd = 0, last_s = 0, last_p = 0;
+    bool ok = true, ext_issued = false;
+    for (int64_t t = pair; t < tiles && ok; t += npairs) {
+      const int32_t w0 = load_row0((int32_t)((t % w_tiles) * 2 * BM + row_off), args.R);
+      const int scale_idx = !W_MN ? blk : j_row * 4 + ((w0 / 64) & 3) + gi;
+      for (int kc = 0; kc < kc_total; ++kc, ++gd) {
+        const uint32_t sd = gd % SD, pd = (gd / SD) & 1;
+        if (kc >= kc_main) {
+          const bool wb = mbar_wait(empty_d + 8 * sd, pd ^ 1, lim, abort_word);
+          if (!__all_sync(0xFFFFFFFFu, wb)) { ok = false; break; }
+          if (lane == 0) {
+            const uint32_t fb = full_d + 8 * sd;
+            if (warp == 7) {
+              mbar_arrive_expect_tx(fb, Cfg::kDBytes);
+              tma_load_2d(smem_u32(sD + sd * Cfg::kDBytes), &tmWe, fb, (kc - kc_main) * 64, w0);
+              ext_issued = true;
+              last_s = sd;
+              last_p = pd;
+            } else {
+              mbar_arrive(fb);
+            }
+          }
+          continue;
+        }
+        const uint32_t sc = gc % SC, pc = (gc / SC) & 1;
+        const bool w1 = mbar_wait(full_c + 8 * sc, pc, lim, abort_word);
+        const bool w2 = w1 && mbar_wait(empty_d + 8 * sd, pd ^ 1, lim, abort_word);
+        if (!__all_sync(0xFFFFFFFFu, w2)) { ok = false; break; }
+        const uint8_t* cst = sC + sc * Cfg::kCBytes;
+        const float sv = reinterpret_cast<const float*>(cst + Cfg::kCodeBytes)[scale_idx];
+        uint4* d = reinterpret_cast<uint4*>(sD + sd * Cfg::kDBytes + d_off);
+        if constexpr (BS == BSrc::NF4) {
+          const uint4 cv = reinterpret_cast<const uint4*>(cst + code_off)[half];
+          uint32_t L[2], H[2];
+          nf4_table(q, sv, L, H);
+          const int c0i = 4 * half;
+          d[(c0i + 0) ^ key] = nf4_decode8(cv.x, L, H);
+          d[(c0i + 1) ^ key] = nf4_decode8(cv.y, L, H);
+          d[(c0i + 2) ^ key] = nf4_decode8(cv.z, L, H);
+          d[(c0i + 3) ^ key] = nf4_decode8(cv.w, L, H);
+        } else {
+          const uint4* src = reinterpret_cast<const uint4*>(cst + code_off) + 2 * half;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint4 w = src[h];
+            const int c = 4 * half + 2 * h;
+            d[c ^ key] = int8_decode8(w.x, w.y, sv);
+            d[(c + 1) ^ key] = int8_decode8(w.z, w.w, sv);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(full_d + 8 * sd);
+          mbar_arrive(empty_c + 8 * sc);
+        }
+        ++gc;
+      }
+    }
+    if ((!ok || *abort_word) && warp == 7 && lane == 0 && ext_issued)
+      drain_wait(full_d + 8 * last_s, last_p);           // our last extension copy (bounded)
+  }
+
+  // Neither CTA leaves (or frees TMEM) while the pair's MMAs may still read its shared
+  // memory or the other CTA may still arrive on its barriers.
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  if (warp == 5) tmem_dealloc_pair(tmem_base, Cfg::kTmemCols);
   if (threadIdx.x == 0 && *abort_word) raise_flag(args.flag, kFlagTimeout);
 }
 

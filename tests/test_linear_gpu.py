@@ -166,3 +166,20 @@ def test_small_m_ragged(M, N, K, r, fmt):
     case = synth.LinearCase(f"small-{M}-{N}-{K}-{r}", N=N, K=K, M=M, r=r, alpha=16.0, fmt=fmt,
                             seed=N + K)
     check_case(case)
+
+
+# ---- both fused-GEMM variants: single CTAs (default) and CTA pairs -------------------
+
+@pytest.mark.parametrize("pair", [1, 0], ids=["pair", "single"])
+@pytest.mark.parametrize("fmt", ["nf4_dq", "int8"])
+@pytest.mark.parametrize("M,N,K,r", [(300, 1024, 768, 64), (517, 392, 1344, 24), (257, 640, 512, 130)])
+def test_gemm_variants(pair, fmt, M, N, K, r):
+    """Ragged weight rows and tokens (pair tiles of 256 x 256 leave an idle half), both
+    formats, adapter ranks that need one, one and three extension chunks."""
+    B.lib().ql_set_gemm_pair(pair)
+    try:
+        case = synth.LinearCase(f"variant-{M}-{N}-{K}-{r}", N=N, K=K, M=M, r=r, alpha=2.0 * r,
+                                fmt=fmt, seed=M + N)
+        check_case(case)
+    finally:
+        B.lib().ql_set_gemm_pair(0)
