@@ -38,6 +38,12 @@ struct GemmArgs {
   float scale;
   uint64_t timeout_ns;
   int* flag;
+  // split-K (TMA GEMM only): ksplit > 1 splits the contraction into slices of kc_per
+  // 64-wide chunks; each (tile, slice) stores its fp32 partial into part [ksplit][R][ldp]
+  // and reduce_partials_kernel applies the epilogue to their sum
+  int32_t ksplit, kc_per;
+  float* part;
+  int64_t ldp;
 };
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
@@ -160,22 +166,34 @@ __device__ __forceinline__ void epilogue_store(const GemmArgs& a, int64_t row, i
 // Epilogue role shared by both kernels: warps 0..3, TMEM lanes 32*warp ..
 template <int BN, int EPI>
 __device__ __forceinline__ void run_epilogue(const GemmArgs& args, uint32_t tmem_base, uint32_t acc_full,
-                                             uint32_t acc_empty, int64_t tiles, int64_t n_tiles,
+                                             uint32_t acc_empty, int64_t items, int64_t n_tiles,
                                              volatile int* abort_word) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ks = args.ksplit > 1 ? args.ksplit : 1;
   uint32_t tcount = 0;
-  for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++tcount) {
+  for (int64_t it = blockIdx.x; it < items; it += gridDim.x, ++tcount) {
     const uint32_t acc = tcount & 1, aph = (tcount >> 1) & 1;
     const bool okw = mbar_wait(acc_full + 8 * acc, aph, args.timeout_ns, abort_word);
     if (!__all_sync(0xFFFFFFFFu, okw)) break;
     tc_fence_after();
+    const int64_t t = it / ks, split = it % ks;
     const int64_t r0 = (t / n_tiles) * 128, c0 = (t % n_tiles) * BN;
     const int64_t row = r0 + warp * 32 + lane;
 #pragma unroll 1
     for (int cc = 0; cc < BN; cc += 32) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(warp * 32) << 16) + acc * BN + cc, v);
-      if (c0 + cc < args.Cn) epilogue_store<EPI>(args, row, c0 + cc, v);
+      if (ks > 1) {
+        if (row < args.R) {                          // the slice's partial, all BN columns
+          float4* dst = reinterpret_cast<float4*>(args.part + (split * args.R + row) * args.ldp + c0 + cc);
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                 __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+        }
+      } else if (c0 + cc < args.Cn) {
+        epilogue_store<EPI>(args, row, c0 + cc, v);
+      }
     }
     tc_fence_before();
     __syncwarp();
@@ -186,6 +204,32 @@ __device__ __forceinline__ void run_epilogue(const GemmArgs& args, uint32_t tmem
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < 200000000ull) {}
+}
+
+// Sum of the split-K partials in slice order (so the result does not depend on which CTA
+// ran which slice), then the GEMM's own epilogue. One thread per (row, 32 columns).
+template <int EPI>
+__global__ void __launch_bounds__(256)
+reduce_partials_kernel(const GemmArgs args) {
+  const int64_t chunks = (args.Cn + 31) / 32;
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= args.R * chunks) return;
+  const int64_t row = i / chunks, c0 = (i % chunks) * 32;
+  float acc[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) acc[j] = 0.0f;
+  for (int s = 0; s < args.ksplit; ++s) {
+    const float4* src = reinterpret_cast<const float4*>(args.part + (s * args.R + row) * args.ldp + c0);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float4 v = src[j];
+      acc[4 * j] += v.x; acc[4 * j + 1] += v.y; acc[4 * j + 2] += v.z; acc[4 * j + 3] += v.w;
+    }
+  }
+  uint32_t v[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(acc[j]);
+  epilogue_store<EPI>(args, row, c0, v);
 }
 
 // =================================================================================
@@ -237,16 +281,22 @@ qgemm_tma_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
   const int64_t n_tiles = (args.Cn + BN - 1) / BN;
   const int64_t tiles = ((args.R + 127) / 128) * n_tiles;
   const int kc_total = (int)((args.Kc + 63) / 64);
+  // work items: (tile, contraction slice); one slice of all chunks without split-K
+  const int ks = args.ksplit > 1 ? args.ksplit : 1;
+  const int kc_per = ks > 1 ? args.kc_per : kc_total;
+  const int64_t items = tiles * ks;
   const uint64_t lim = args.timeout_ns;
 
   if (warp < 4) {
-    run_epilogue<BN, EPI>(args, tmem_base, acc_full, acc_empty, tiles, n_tiles, abort_word);
+    run_epilogue<BN, EPI>(args, tmem_base, acc_full, acc_empty, items, n_tiles, abort_word);
   } else if (warp == 4 && lane == 0) {
     uint32_t g = 0;
     bool ok = true;
-    for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+    for (int64_t it = blockIdx.x; it < items && ok; it += gridDim.x) {
+      const int64_t t = it / ks;
+      const int kb = (int)(it % ks) * kc_per, ke = kb + kc_per < kc_total ? kb + kc_per : kc_total;
       const int32_t r0 = (int32_t)((t / n_tiles) * 128), c0 = (int32_t)((t % n_tiles) * BN);
-      for (int kc = 0; kc < kc_total; ++kc, ++g) {
+      for (int kc = kb; kc < ke; ++kc, ++g) {
         const uint32_t s = g % S, ph = (g / S) & 1;
         if (!mbar_wait(empty + 8 * s, ph ^ 1, lim, abort_word)) { ok = false; break; }
         const uint32_t fb = full + 8 * s;
@@ -273,12 +323,13 @@ qgemm_tma_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
     constexpr uint32_t kId = idesc_bf16_f32(128, BN, A_MN ? 1 : 0, B_MN ? 1 : 0);
     uint32_t g = 0, tcount = 0;
     bool ok = true;
-    for (int64_t t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tcount) {
+    for (int64_t it = blockIdx.x; it < items && ok; it += gridDim.x, ++tcount) {
       const uint32_t acc = tcount & 1, aph = (tcount >> 1) & 1;
       if (!mbar_wait(acc_empty + 8 * acc, aph ^ 1, lim, abort_word)) { ok = false; break; }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + acc * BN;
-      for (int kc = 0; kc < kc_total; ++kc, ++g) {
+      const int kb = (int)(it % ks) * kc_per, ke = kb + kc_per < kc_total ? kb + kc_per : kc_total;
+      for (int kc = kb; kc < ke; ++kc, ++g) {
         const uint32_t s = g % S, ph = (g / S) & 1;
         if (!mbar_wait(full + 8 * s, ph, lim, abort_word)) { ok = false; break; }
         tc_fence_after();
@@ -290,7 +341,7 @@ qgemm_tma_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                                     : smem_desc_sw128(a_base + k * 2048, 8192, 1024);
           const uint64_t bd = !B_MN ? smem_desc_sw128(b_base + k * 32, 16, 1024)
                                     : smem_desc_sw128(b_base + k * 2048, 8192, 1024);
-          tc_mma(d_tmem, ad, bd, kId, (kc > 0 || k > 0) ? 1u : 0u);
+          tc_mma(d_tmem, ad, bd, kId, (kc > kb || k > 0) ? 1u : 0u);
         }
         tc_commit(empty + 8 * s);
       }

@@ -66,11 +66,16 @@ static ql_status launch_tma(const CUtensorMap& a, const CUtensorMap& b, const Ge
   const size_t smem = TmaCfg<BN>::kSmem;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return QL_ERR_CUDA;
-  const int64_t tiles = ((args.R + 127) / 128) * ((args.Cn + BN - 1) / BN);
-  const int grid = (int)imin64(tiles, num_sms());
+  const int64_t items = ((args.R + 127) / 128) * ((args.Cn + BN - 1) / BN) * (args.ksplit > 1 ? args.ksplit : 1);
+  const int grid = (int)imin64(items, num_sms());
   if (grid <= 0) return QL_OK;
   kern<<<grid, 192, smem, st>>>(a, b, args);
   QL_CHECK_LAUNCH();
+  if (args.ksplit > 1) {
+    const int64_t threads = args.R * ((args.Cn + 31) / 32);
+    reduce_partials_kernel<EPI><<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(args);
+    QL_CHECK_LAUNCH();
+  }
   return QL_OK;
 }
 
@@ -186,14 +191,59 @@ static int small_grid(int64_t n) { return (int)imax64(1, imin64((n + 255) / 256,
 static int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
 
 struct WsLayout {
-  int64_t off[5];
+  int64_t off[6];
   int64_t total;
 };
+
+// Split-K for the adapter GEMMs of the backward, which stream a whole activation (dY or
+// X) against a narrow factor and have few 128-row tiles: the number of contraction
+// slices ks <= 8 that minimises the busiest CTA's share, ceil(tiles * ks / 148) / ks
+// (148 SMs; a fixed count keeps the workspace size independent of the device), the
+// smaller ks on ties, and never more slices than 64-wide chunks.
+struct SplitK {
+  int ks, kc_per;
+};
+
+static SplitK split_k(int64_t R, int64_t Cn, int64_t Kc, int BN) {
+  const int64_t tiles = ((R + 127) / 128) * ((Cn + BN - 1) / BN);
+  const int64_t kc_total = (Kc + 63) / 64;
+  int best = 1;
+  double best_share = 1.0;
+  for (int ks = 2; ks <= 8; ++ks) {
+    const double share = (double)((tiles * ks + 147) / 148) / ks;
+    if (share < best_share - 1e-9) { best = ks; best_share = share; }
+  }
+  if (best > kc_total) best = (int)imax64(1, kc_total);
+  const int kc_per = (int)((kc_total + best - 1) / best);
+  SplitK k{(int)((kc_total + kc_per - 1) / kc_per), kc_per};   // no empty slice
+  return k;
+}
+
+static int rp_bn(int64_t rp) { return rp <= 64 ? 64 : rp <= 128 ? 128 : rp <= 192 ? 192 : 256; }
+
+// Bytes of split-K partials of one adapter GEMM: [ks][R][columns of its tiles] fp32.
+static int64_t partial_bytes(int64_t R, int64_t rp, int64_t Kc) {
+  const int bn = rp_bn(rp);
+  const SplitK k = split_k(R, rp, Kc, bn);
+  return k.ks > 1 ? (int64_t)k.ks * R * round_up(rp, bn) * 4 : 0;
+}
+
+// Turn on split-K for an adapter GEMM of padded rank rp, with its partials at `part`.
+// Returns the number of kernels the GEMM then launches (1 or 2).
+static int apply_split(GemmArgs& a, float* part, int64_t rp) {
+  const int bn = rp_bn(rp);
+  const SplitK k = split_k(a.R, a.Cn, a.Kc, bn);
+  a.ksplit = k.ks;
+  a.kc_per = k.kc_per;
+  a.part = part;
+  a.ldp = round_up(a.Cn, bn);
+  return k.ks > 1 ? 2 : 1;
+}
 
 static WsLayout ws_layout(int op, int64_t M, int64_t N, int64_t K, int r) {
   WsLayout L{};
   const int64_t rp = round_up(r, 64);
-  int64_t sz[5] = {0, 0, 0, 0, 0};
+  int64_t sz[6] = {0, 0, 0, 0, 0, 0};
   if (op == QL_OP_FWD) {
     sz[0] = M * rp * 2;        // P
     sz[1] = N * rp * 2;        // B padded
@@ -204,11 +254,14 @@ static WsLayout ws_layout(int op, int64_t M, int64_t N, int64_t K, int r) {
     sz[2] = K * rp * 2;        // A^T padded
     sz[3] = M * rp * 2;        // T padded
     sz[4] = N * round_up(K / 64, 4) * 4;  // block scales, row-major (padded rows)
+    // split-K partials, shared by dY B (rows M, contraction N), dB (rows N, over M) and
+    // dA (rows K, over M), which run one after another
+    sz[5] = imax64(partial_bytes(M, rp, N), imax64(partial_bytes(N, rp, M), partial_bytes(K, rp, M)));
   } else if (op == QL_OP_DQ) {
     sz[0] = 256;
   }
   int64_t o = 0;
-  for (int i = 0; i < 5; ++i) {
+  for (int i = 0; i < 6; ++i) {
     L.off[i] = o;
     o += round_up(sz[i], 256);
   }
@@ -377,6 +430,7 @@ ql_status qlora_linear_bwd(const ql_weight* w, const ql_bf16* X, const ql_bf16* 
   uint16_t* At = reinterpret_cast<uint16_t*>(wsb + L.off[2]);
   uint16_t* Tp = reinterpret_cast<uint16_t*>(wsb + L.off[3]);
   float* scales = reinterpret_cast<float*>(wsb + L.off[4]);
+  float* part = reinterpret_cast<float*>(wsb + L.off[5]);
 
   const bool pair = g_gemm_pair.load() != 0;
   const uint32_t tbox = pair ? 128 : 256;
@@ -406,7 +460,7 @@ ql_status qlora_linear_bwd(const ql_weight* w, const ql_bf16* X, const ql_bf16* 
   GemmArgs u = base_args();
   u.R = M; u.Cn = rp; u.Kc = N; u.r = r; u.out = Q; u.ld_out = rp; u.scale = s;
   {
-    ProfScope prof(PK_BWD_U, st, 1);
+    ProfScope prof(PK_BWD_U, st, apply_split(u, part, rp));
     e = launch_tma_rp<EPI_LORA_Q, false, false>(rp, mdY_k, mBt, u, st);
   }
   if (e != QL_OK) return e;
@@ -415,7 +469,7 @@ ql_status qlora_linear_bwd(const ql_weight* w, const ql_bf16* X, const ql_bf16* 
   GemmArgs b = base_args();
   b.R = N; b.Cn = rp; b.Kc = M; b.r = r; b.out = dB; b.ld_out = r; b.scale = s;
   {
-    ProfScope prof(PK_BWD_DB, st, 1);
+    ProfScope prof(PK_BWD_DB, st, apply_split(b, part, rp));
     e = launch_tma_rp<EPI_DB, true, true>(rp, mdY_mn, mTp_mn, b, st);
   }
   if (e != QL_OK) return e;
@@ -424,7 +478,7 @@ ql_status qlora_linear_bwd(const ql_weight* w, const ql_bf16* X, const ql_bf16* 
   GemmArgs a = base_args();
   a.R = K; a.Cn = rp; a.Kc = M; a.r = r; a.out = dA; a.ld_out = K; a.scale = 1.0f;
   {
-    ProfScope prof(PK_BWD_DA, st, 1);
+    ProfScope prof(PK_BWD_DA, st, apply_split(a, part, rp));
     e = launch_tma_rp<EPI_DA, true, true>(rp, mX_mn, mQ_mn, a, st);
   }
   if (e != QL_OK) return e;
