@@ -112,6 +112,25 @@ ql_status nf4_dq_quantize(const ql_bf16* W, int64_t n, uint8_t* codes, float* ab
                           int8_t* qabsmax, float* group_scale, float* mean, void* ws,
                           size_t ws_bytes, void* stream);
 
+/* NF4 + double quantisation of a weight split across ranks (QLoRA page, "2. Double
+ * Quantization": one mean per tensor, so the ranks must agree on the sum of all block
+ * constants). Every rank holds a contiguous shard of the flattened weight; every shard
+ * but the last holds a multiple of 16384 elements (whole groups of 256 blocks).
+ *  1. nf4_quantize_shard: NF4 codes and absmax of the shard as in nf4_quantize, and the
+ *     exact sum of its block constants as 16 unsigned 64-bit bins: a finite v >= 0 is
+ *     m * 2^(p - 149) with 24-bit m and p in [0, 253], and adds m << (p % 16) to bin
+ *     p / 16. bins: device uint64 [16], overwritten. ws as for nf4_dq_quantize.
+ *  2. The caller sums the bins over the ranks: an integer all-reduce, exact whatever
+ *     the order (each bin stays below 2^63 for at most 2^24 blocks in all).
+ *  3. dq_quantize_shard: the mean from the summed bins and the total block count, as in
+ *     dq_quantize, then the shard's groups.
+ * The result on every rank is bit-identical to nf4_dq_quantize of the whole weight. */
+ql_status nf4_quantize_shard(const ql_bf16* W, int64_t n, uint8_t* codes, float* absmax,
+                             uint64_t* bins, void* ws, size_t ws_bytes, void* stream);
+ql_status dq_quantize_shard(const float* absmax, int64_t nblocks, const uint64_t* bins,
+                            int64_t nblocks_total, int8_t* qabsmax, float* group_scale,
+                            float* mean, void* stream);
+
 /* Blockwise int8 (the 8-bit choice of the per-layer bit-width, AutoQRA page 3.1):
  * absmax[b] as in nf4_quantize; sc = fp32(absmax[b]/127);
  * codes[j] = clamp(rint_half_even(fp32(W_j / sc)), -127, 127) (0 when sc == 0).

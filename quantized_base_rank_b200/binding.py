@@ -45,6 +45,8 @@ _SIGS = {
     "int8_quantize": ([P, I64, P, P, P], I32),
     "dq_quantize": ([P, I64, P, P, P, P, SZ, P], I32),
     "nf4_dq_quantize": ([P, I64, P, P, P, P, P, P, SZ, P], I32),
+    "nf4_quantize_shard": ([P, I64, P, P, P, P, SZ, P], I32),
+    "dq_quantize_shard": ([P, I64, P, I64, P, P, P, P], I32),
     "ql_dequantize": ([ctypes.POINTER(QLWeight), P, P], I32),
     "qlora_linear_fwd": ([ctypes.POINTER(QLWeight), P, I64, P, P, I32, F32, P, P, P, SZ, P], I32),
     "qlora_linear_bwd": ([ctypes.POINTER(QLWeight), P, P, I64, P, P, P, I32, F32, P, P, P, P, SZ, P], I32),
@@ -195,6 +197,42 @@ def nf4_dq_quantize(W: torch.Tensor, codes=None, absmax=None, qabsmax=None, grou
     _check(lib().nf4_dq_quantize(_ptr(W), n, _ptr(codes), _ptr(absmax), _ptr(qabsmax), _ptr(group_scale),
                                  _ptr(mean), _ptr(ws), ws.numel(), _stream(dev)), "nf4_dq_quantize")
     return codes, absmax, qabsmax, group_scale, mean
+
+
+def nf4_quantize_shard(W: torch.Tensor, codes=None, absmax=None, bins=None):
+    """Step 1 of the sharded NF4 + double quantisation: codes, absmax and the shard's exact
+    DQ bins (int64 [16] holding the unsigned 64-bit sums, each below 2^63)."""
+    _need(W, torch.bfloat16, "W")
+    n = W.numel()
+    dev = W.device
+    if codes is None:
+        codes = torch.empty((n + 1) // 2, dtype=torch.uint8, device=dev)
+    if absmax is None:
+        absmax = torch.empty((n + 63) // 64, dtype=torch.float32, device=dev)
+    if bins is None:
+        bins = torch.empty(16, dtype=torch.int64, device=dev)
+    ws = workspace(workspace_bytes(QL_OP_DQ, 0, 0, 0, 0), dev)
+    _check(lib().nf4_quantize_shard(_ptr(W), n, _ptr(codes), _ptr(absmax), _ptr(bins), _ptr(ws),
+                                    ws.numel(), _stream(dev)), "nf4_quantize_shard")
+    return codes, absmax, bins
+
+
+def dq_quantize_shard(absmax: torch.Tensor, bins: torch.Tensor, nblocks_total: int, qabsmax=None,
+                      group_scale=None, mean=None):
+    """Step 3: the mean from bins summed over all shards, then this shard's groups."""
+    _need(absmax, torch.float32, "absmax")
+    _need(bins, torch.int64, "bins")
+    nb = absmax.numel()
+    dev = absmax.device
+    if qabsmax is None:
+        qabsmax = torch.empty(nb, dtype=torch.int8, device=dev)
+    if group_scale is None:
+        group_scale = torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev)
+    if mean is None:
+        mean = torch.empty(1, dtype=torch.float32, device=dev)
+    _check(lib().dq_quantize_shard(_ptr(absmax), nb, _ptr(bins), int(nblocks_total), _ptr(qabsmax),
+                                   _ptr(group_scale), _ptr(mean), _stream(dev)), "dq_quantize_shard")
+    return qabsmax, group_scale, mean
 
 
 class QuantWeight:

@@ -227,11 +227,12 @@ __device__ float dq_mean_from_bins(const unsigned long long (&bins)[16], int64_t
 // End of the exact sum for one CTA (every thread calls it): the per-warp bins are
 // combined, added to the global bins (one atomic per non-empty bin), and the CTA takes a
 // ticket. The CTA that takes the last of `ctas` tickets (counted over every launch that
-// shares the bins) rounds the sum and writes the mean. No CTA waits for another.
-// ws: bins[16], then the ticket counter; zeroed before the first launch.
+// shares the bins) rounds the sum and writes the mean, or, with bins_out (one shard of a
+// weight split across ranks), copies the shard's exact bins out instead. No CTA waits
+// for another. ws: bins[16], then the ticket counter; zeroed before the first launch.
 __device__ __forceinline__ void dq_bins_finish(unsigned long long (*s_bins)[kSumBins], int nwarps,
                                                unsigned long long* ws, unsigned int ctas, int64_t nb,
-                                               float* mean) {
+                                               float* mean, unsigned long long* bins_out) {
   __shared__ int s_last;
   __syncthreads();
   unsigned int* ticket = reinterpret_cast<unsigned int*>(ws + kSumBins);
@@ -249,8 +250,22 @@ __device__ __forceinline__ void dq_bins_finish(unsigned long long (*s_bins)[kSum
     unsigned long long v[kSumBins];
 #pragma unroll
     for (int i = 0; i < kSumBins; ++i) v[i] = __ldcg(ws + i);
-    *mean = dq_mean_from_bins(v, nb);
+    if (bins_out) {
+      for (int i = 0; i < kSumBins; ++i) bins_out[i] = v[i];
+    } else {
+      *mean = dq_mean_from_bins(v, nb);
+    }
   }
+}
+
+// The mean from bins summed over the shards of a weight: one thread.
+__global__ void dq_mean_kernel(const unsigned long long* __restrict__ bins, int64_t nb_total, float* mean) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  unsigned long long v[kSumBins];
+#pragma unroll
+  for (int i = 0; i < kSumBins; ++i) v[i] = bins[i];
+  *mean = dq_mean_from_bins(v, nb_total);
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // NF4 encode kernel. Two threads per block of 64: lanes 2t and 2t+1 of a warp take the
@@ -272,6 +287,7 @@ struct Nf4Args {
   int* flag;
   unsigned long long* dq_ws;   // DQ: bins + ticket
   float* mean;                 // DQ: output
+  unsigned long long* bins_out;  // DQ, one shard: its exact bins instead of the mean
   unsigned int dq_ctas;        // DQ: CTAs over all launches sharing the bins
   int64_t nb_total;            // DQ: number of constants
 };
@@ -375,7 +391,7 @@ nf4_quantize_kernel(const Nf4Args args, const Nf4Tables tab, const Nf4BoundTable
   }
   if (DQ) {
     (void)bad;                                         // a non-finite absmax already raised the flag
-    dq_bins_finish(s_bins, kNf4Warps, args.dq_ws, args.dq_ctas, args.nb_total, args.mean);
+    dq_bins_finish(s_bins, kNf4Warps, args.dq_ws, args.dq_ctas, args.nb_total, args.mean, args.bins_out);
   }
 }
 
@@ -476,7 +492,7 @@ dq_sum_kernel(const float* __restrict__ absmax, int64_t nb, unsigned long long* 
     }
   }
   if (bad) raise_flag(flag, kFlagNonfinite);
-  dq_bins_finish(s_bins, kSumThreads / 32, ws, gridDim.x, nb, mean);
+  dq_bins_finish(s_bins, kSumThreads / 32, ws, gridDim.x, nb, mean, nullptr);
 }
 
 // One warp per group of 256 blocks: d = a - mean, s_g = max|d| / 127, code =
@@ -583,7 +599,8 @@ static int nf4_launches(const void* W, int64_t n, const void* codes) {
 // NF4 encode of W[0, n); with dq_ws (zeroed bins + ticket) also the exact sum of the block
 // constants and, from the last CTA, the double-quantisation mean.
 static ql_status launch_nf4(const uint16_t* W, int64_t n, uint8_t* codes, float* absmax,
-                            unsigned long long* dq_ws, float* mean, cudaStream_t st) {
+                            unsigned long long* dq_ws, float* mean, cudaStream_t st,
+                            unsigned long long* bins_out = nullptr) {
   const bool vec = aligned(W, 16) && aligned(codes, 16);
   const int64_t nb = (n + kBlock - 1) / kBlock;
   const int64_t nb_vec = vec ? n / kBlock : 0;
@@ -600,7 +617,8 @@ static ql_status launch_nf4(const uint16_t* W, int64_t n, uint8_t* codes, float*
   }
   Nf4Args a;
   a.W = W; a.n = n; a.codes = codes; a.absmax = absmax; a.flag = device_flag_ptr();
-  a.dq_ws = dq_ws; a.mean = mean; a.dq_ctas = (unsigned)(g_vec + g_tail); a.nb_total = nb;
+  a.dq_ws = dq_ws; a.mean = mean; a.bins_out = bins_out; a.dq_ctas = (unsigned)(g_vec + g_tail);
+  a.nb_total = nb;
   const Nf4Tables& tab = nf4_tables();
   const Nf4BoundTable& btab = nf4_bound_table();
   if (g_vec) {
@@ -706,6 +724,36 @@ ql_status nf4_dq_quantize(const ql_bf16* W, int64_t n, uint8_t* codes, float* ab
   }
   ProfScope prof(PK_DQ, st, 1);
   return launch_dq_encode(absmax, nb, mean, qabsmax, group_scale, st);
+}
+
+ql_status nf4_quantize_shard(const ql_bf16* W, int64_t n, uint8_t* codes, float* absmax, uint64_t* bins,
+                             void* ws, size_t ws_bytes, void* stream) {
+  if (n < 1 || !W || !codes || !absmax || !bins || !ws) return QL_ERR_INVALID_ARG;
+  const int64_t nb = (n + kBlock - 1) / kBlock;
+  if (nb > (int64_t(1) << 24)) return QL_ERR_UNSUPPORTED;
+  if (!aligned(W, 2) || !aligned(codes, 4) || !aligned(absmax, 4) || !aligned(bins, 8) || !aligned(ws, 16))
+    return QL_ERR_INVALID_ARG;
+  if (ws_bytes < ql_workspace_bytes(QL_OP_DQ, 0, 0, 0, 0)) return QL_ERR_WORKSPACE;
+  cudaStream_t st = as_stream(stream);
+  unsigned long long* wsb = static_cast<unsigned long long*>(ws);
+  ProfScope prof(PK_NF4, st, nf4_launches(W, n, codes));
+  if (cudaMemsetAsync(wsb, 0, (kSumBins + 1) * sizeof(unsigned long long), st) != cudaSuccess)
+    return QL_ERR_CUDA;
+  return launch_nf4(W, n, codes, absmax, wsb, nullptr, st, reinterpret_cast<unsigned long long*>(bins));
+}
+
+ql_status dq_quantize_shard(const float* absmax, int64_t nblocks, const uint64_t* bins, int64_t nblocks_total,
+                            int8_t* qabsmax, float* group_scale, float* mean, void* stream) {
+  if (nblocks < 1 || nblocks_total < nblocks || !absmax || !bins || !qabsmax || !group_scale || !mean)
+    return QL_ERR_INVALID_ARG;
+  if (nblocks_total > (int64_t(1) << 24)) return QL_ERR_UNSUPPORTED;
+  if (!aligned(absmax, 4) || !aligned(bins, 8) || !aligned(group_scale, 4) || !aligned(mean, 4))
+    return QL_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  ProfScope prof(PK_DQ, st, 2);
+  dq_mean_kernel<<<1, 32, 0, st>>>(reinterpret_cast<const unsigned long long*>(bins), nblocks_total, mean);
+  QL_CHECK_LAUNCH();
+  return launch_dq_encode(absmax, nblocks, mean, qabsmax, group_scale, st);
 }
 
 ql_status ql_dequantize(const ql_weight* w, ql_bf16* Wout, void* stream) {

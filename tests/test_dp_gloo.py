@@ -78,3 +78,34 @@ def test_allreduce_of_partial_gradients_equals_full_batch():
         if rank:
             assert np.array_equal(dAr, results[0][3]) and np.array_equal(dBr, results[0][4])
     assert covered == CASE.M
+
+
+def test_quantise_shards_are_whole_groups():
+    for n in (1, 64, 16384, 16385, 3 * 16384 + 5, 4096 * 4096, 22016 * 8192):
+        for world in (1, 2, 3, 8):
+            spans = [dp.shard_elems(n, world, r) for r in range(world)]
+            assert spans[0][0] == 0 and spans[-1][1] == n
+            assert all(a[1] == b[0] for a, b in zip(spans, spans[1:]))
+            assert all(a % dp.GROUP_ELEMS == 0 for a, b in spans if b > a)   # empty shards are refused
+
+
+def _bins_worker(rank, world, port, results):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # values near 2^62: the sum must stay exact in int64
+        bins = torch.tensor([(1 << 61) + 12345 * (rank + 1) + i for i in range(16)], dtype=torch.int64)
+        dp.allreduce_bins(bins)
+        results[rank] = bins.tolist()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bin_allreduce_is_exact():
+    world = 2
+    results = mp.get_context("spawn").Manager().dict()
+    mp.start_processes(_bins_worker, args=(world, _free_port(), results), nprocs=world, join=True,
+                       start_method="spawn")
+    want = [sum((1 << 61) + 12345 * (r + 1) + i for r in range(world)) for i in range(16)]
+    assert results[0] == want and results[1] == want

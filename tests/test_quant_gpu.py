@@ -172,3 +172,32 @@ def test_full_size_65b_shapes(N, K):
     c8, a8 = B.int8_quantize(W.view(-1))
     rc8, ra8 = o.int8_quantize(w)
     assert np.array_equal(c8.cpu().numpy(), rc8)
+
+
+# ---- quantisation sharded across ranks (run here as shards in sequence) -------------
+
+@pytest.mark.parametrize("shards", [2, 3])
+@pytest.mark.parametrize("name,W", [w for w in WEIGHTS if w[0] in ("cfg2-4096x4096-outliers", "ragged-odd",
+                                                                 "boundary-sweep")],
+                         ids=lambda v: v if isinstance(v, str) else "")
+def test_sharded_nf4_dq_matches_whole(shards, name, W):
+    """Each shard quantised on its own with its exact DQ bins, the bins summed as integers
+    (the all-reduce), the double quantisation finished per shard: every array is the
+    whole-weight nf4_dq_quantize result, bit for bit."""
+    from quantized_base_rank_b200 import dp
+    flat = W.cuda().contiguous().view(-1)
+    n = flat.numel()
+    codes, absmax, qa, gs, mu = B.nf4_dq_quantize(flat)
+    spans = [dp.shard_elems(n, shards, r) for r in range(shards)]
+    parts = [B.nf4_quantize_shard(flat[a:b]) for a, b in spans]
+    total = sum(p[2] for p in parts)                       # integer sum of the bins
+    nb_total = (n + 63) // 64
+    for (a, b), (c, am, _) in zip(spans, parts):
+        q, g, m = B.dq_quantize_shard(am, total, nb_total)
+        assert a % 2 == 0 and a % 64 == 0
+        assert torch.equal(c[: (b - a + 1) // 2], codes[a // 2: a // 2 + (b - a + 1) // 2])
+        assert torch.equal(am.view(torch.int32), absmax[a // 64: a // 64 + am.numel()].view(torch.int32))
+        assert torch.equal(q, qa[a // 64: a // 64 + q.numel()])
+        assert torch.equal(g.view(torch.int32), gs[a // 16384: a // 16384 + g.numel()].view(torch.int32))
+        assert torch.equal(m.view(torch.int32), mu.view(torch.int32))
+    assert B.device_status() == B.QL_OK
