@@ -18,6 +18,9 @@ It is a plain, slow, obviously correct restatement of what the method computes:
   gradients, computed in fp64 (QLoRA page, section "memory decomposition": frozen
   4-bit base plus bf16 LoRA adapters; LoRDBA page, gist.science/ko/paper/2605.24058,
   "adapter mode", for the unmerged branch).
+* The low-rank double-binary adapter of the LoRDBA page (section "2. Methodology",
+  core architecture): Delta W = sum_i diag(alpha_i) B1 diag(beta_i) B2 diag(gamma_i)
+  with sign carriers B1, B2 in {+-1}, in fp64.
 
 Where the pages are silent the reading taken is stated in the docstring of the
 function that takes it. Floating-point steps are written with numpy float32 scalars
@@ -373,3 +376,36 @@ def quantize_weight(w: np.ndarray, fmt: str):
         c, a = int8_quantize(w)
         return {"codes": c, "absmax": a, "wdeq": int8_dequant(c, a)}
     raise ValueError(fmt)
+
+
+# --------------------------------------------------------------------------------------
+# LoRDBA: low-rank double-binary adapter (LoRDBA page, gist.science/ko/paper/2605.24058,
+# section "2. Methodology", core architecture: the parameterisation, 1-bit carriers and
+# fp16 channel scales, and the two-stage sign-accumulate inference kernel)
+# --------------------------------------------------------------------------------------
+
+def lordba_delta(alpha, beta, gamma, B1, B2):
+    """Delta W = sum_{i < l} diag(alpha[i]) B1 diag(beta[i]) B2 diag(gamma[i]), fp64.
+
+    B1 [N, R] and B2 [R, K] hold +-1 (the carriers are shared by the l envelope terms;
+    only the scale vectors carry the index i). alpha [l, N], beta [l, R], gamma [l, K]
+    are the channel scales. Returns Delta W [N, K], the update to the frozen weight
+    [out, in]."""
+    B1 = np.asarray(B1, np.float64)
+    B2 = np.asarray(B2, np.float64)
+    alpha = np.atleast_2d(np.asarray(alpha, np.float64))
+    beta = np.atleast_2d(np.asarray(beta, np.float64))
+    gamma = np.atleast_2d(np.asarray(gamma, np.float64))
+    assert set(np.unique(B1)) <= {-1.0, 1.0} and set(np.unique(B2)) <= {-1.0, 1.0}
+    D = np.zeros((B1.shape[0], B2.shape[1]))
+    for i in range(alpha.shape[0]):
+        D += (alpha[i][:, None] * B1 * beta[i][None, :]) @ (B2 * gamma[i][None, :])
+    return D
+
+
+def lordba_linear_fwd(X, Wd, alpha, beta, gamma, B1, B2):
+    """Y = X Wd^T + X Delta W^T in fp64: the frozen (dequantised) base plus the unmerged
+    double-binary adapter branch (the page's "adapter mode")."""
+    X = np.asarray(X, np.float64)
+    Wd = np.asarray(Wd, np.float64)
+    return X @ Wd.T + X @ lordba_delta(alpha, beta, gamma, B1, B2).T

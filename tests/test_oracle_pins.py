@@ -380,3 +380,80 @@ def test_forward_backward_against_torch_autograd():
     assert np.allclose(Yo, Y.detach().numpy(), rtol=1e-12, atol=1e-12)
     for a, b in ((dX, tX.grad), (dA, tA.grad), (dB, tB.grad)):
         assert np.allclose(a, b.numpy(), rtol=1e-12, atol=1e-12)
+
+
+# ---- LoRDBA double-binary adapter ----------------------------------------------------
+
+def _lordba_case(N=24, K=40, R=6, ell=2, seed=5):
+    rng = np.random.default_rng(seed)
+    B1 = np.where(rng.random((N, R)) < 0.5, -1.0, 1.0)
+    B2 = np.where(rng.random((R, K)) < 0.5, -1.0, 1.0)
+    alpha = rng.uniform(0.1, 1.0, (ell, N))
+    beta = rng.uniform(0.1, 1.0, (ell, R))
+    gamma = rng.uniform(0.1, 1.0, (ell, K))
+    return alpha, beta, gamma, B1, B2
+
+
+def test_lordba_two_stage_sign_accumulate():
+    """The page's inference kernel: gamma-scale x, accumulate with B2's signs (adds and
+    subtracts only), beta-scale, accumulate with B1's signs, alpha-scale. Written as
+    plain loops over Python floats, it must equal the oracle's Delta W x."""
+    alpha, beta, gamma, B1, B2 = _lordba_case()
+    ell, N = alpha.shape
+    R, K = B2.shape
+    x = np.random.default_rng(6).standard_normal(K)
+    y = [0.0] * N
+    for i in range(ell):
+        u = []
+        for j in range(R):
+            acc = 0.0
+            for k in range(K):
+                v = gamma[i][k] * x[k]
+                acc = acc + v if B2[j][k] > 0 else acc - v
+            u.append(beta[i][j] * acc)
+        for n in range(N):
+            acc = 0.0
+            for j in range(R):
+                acc = acc + u[j] if B1[n][j] > 0 else acc - u[j]
+            y[n] += alpha[i][n] * acc
+    ref = o.lordba_delta(alpha, beta, gamma, B1, B2) @ x
+    np.testing.assert_allclose(np.array(y), ref, rtol=1e-12, atol=1e-12)
+
+
+def test_lordba_all_plus_carriers_closed_form():
+    """B1 = B2 = all +1: Delta W[n, k] = sum_i alpha_i[n] (sum_j beta_i[j]) gamma_i[k]."""
+    alpha, beta, gamma, B1, B2 = _lordba_case()
+    B1 = np.ones_like(B1)
+    B2 = np.ones_like(B2)
+    D = o.lordba_delta(alpha, beta, gamma, B1, B2)
+    want = sum(np.outer(alpha[i], gamma[i]) * beta[i].sum() for i in range(alpha.shape[0]))
+    np.testing.assert_allclose(D, want, rtol=1e-13)
+
+
+def test_lordba_terms_add_and_sign_flips():
+    """Envelope terms add; flipping every sign of B1 (or of B2) negates Delta W; zero
+    alpha (or beta, or gamma) removes the branch."""
+    alpha, beta, gamma, B1, B2 = _lordba_case()
+    D = o.lordba_delta(alpha, beta, gamma, B1, B2)
+    D0 = o.lordba_delta(alpha[:1], beta[:1], gamma[:1], B1, B2)
+    D1 = o.lordba_delta(alpha[1:], beta[1:], gamma[1:], B1, B2)
+    np.testing.assert_allclose(D, D0 + D1, rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(o.lordba_delta(alpha, beta, gamma, -B1, B2), -D, rtol=1e-13)
+    np.testing.assert_allclose(o.lordba_delta(alpha, beta, gamma, B1, -B2), -D, rtol=1e-13)
+    assert np.all(o.lordba_delta(0 * alpha, beta, gamma, B1, B2) == 0)
+    # rank: with one envelope term, Delta W has rank <= R
+    assert np.linalg.matrix_rank(D0) <= B1.shape[1]
+
+
+def test_lordba_linear_is_base_plus_branch():
+    alpha, beta, gamma, B1, B2 = _lordba_case()
+    rng = np.random.default_rng(7)
+    X = rng.standard_normal((5, B2.shape[1]))
+    Wd = rng.standard_normal((B1.shape[0], B2.shape[1]))
+    Y = o.lordba_linear_fwd(X, Wd, alpha, beta, gamma, B1, B2)
+    naive = np.zeros_like(Y)
+    D = o.lordba_delta(alpha, beta, gamma, B1, B2)
+    for t in range(X.shape[0]):
+        for n in range(Wd.shape[0]):
+            naive[t, n] = sum(X[t, k] * (Wd[n, k] + D[n, k]) for k in range(X.shape[1]))
+    np.testing.assert_allclose(Y, naive, rtol=1e-12)
