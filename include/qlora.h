@@ -188,7 +188,39 @@ ql_status qlora_linear_fwd_static(const ql_weight* w, const ql_bf16* X, int64_t 
                                   const ql_bf16* A, const ql_bf16* B, int32_t r, float alpha,
                                   ql_bf16* Y, ql_bf16* T_save, void* stream);
 
-enum { QL_OP_DQ = 0, QL_OP_FWD = 1, QL_OP_BWD = 2 };
+/* A LoRDBA double-binary adapter (LoRDBA page, gist.science/ko/paper/2605.24058, section
+ * "2. Methodology", core architecture):
+ *     Delta W = sum_{i < ell} diag(alpha_i) B1 diag(beta_i) B2 diag(gamma_i)
+ * with sign carriers B1 in {+-1}^{N x R} and B2 in {+-1}^{R x K} shared by the ell
+ * envelope terms, stored 1 bit per entry, and fp16 channel scales (the page's storage).
+ *   B1:    device uint32 [N][ceil(R/32)]: bit j%32 of word j/32 of row n is B1[n][j]
+ *          (1 = +1, 0 = -1); unused high bits of a row's last word are ignored.
+ *   B2:    device uint32 [R][ceil(K/32)], the same packing for B2[j][k].
+ *   alpha: device fp16 bits [ell][N]; beta: [ell][R]; gamma: [ell][K].          */
+typedef struct {
+  int32_t R, ell;
+  const uint32_t* B1;
+  const uint32_t* B2;
+  const uint16_t* alpha;
+  const uint16_t* beta;
+  const uint16_t* gamma;
+} ql_lordba;
+
+/* Forward of the quantised linear with a LoRDBA adapter branch, unmerged (the page's
+ * "adapter mode"): Y [M, N] bf16 = bf16(X W'^T + X Delta W^T), fp32 accumulation.
+ * The carriers are expanded with their scales into the bf16 operands of the same
+ * fused GEMM as qlora_linear_fwd, at rank ell*R with s = 1:
+ *   A_eff[i*R + j][k] = sign(B2[j][k]) * bf16(beta_i[j] * gamma_i[k])
+ *   B_eff[n][i*R + j] = sign(B1[n][j]) * bf16(alpha_i[n])
+ * (the fp16 x fp16 product is exact in fp32; one rounding to bf16). The adapter's
+ * left factor X A_eff^T is rounded to bf16 as in qlora_linear_fwd. Shapes as in
+ * qlora_linear_fwd with r = ell*R in [1, 256] (at most 64 for M <= 16).
+ * ws: ql_workspace_bytes(QL_OP_FWD_LORDBA, M, N, K, ell*R) bytes. */
+ql_status qlora_linear_fwd_lordba(const ql_weight* w, const ql_bf16* X, int64_t M,
+                                  const ql_lordba* adapter, ql_bf16* Y, void* ws,
+                                  size_t ws_bytes, void* stream);
+
+enum { QL_OP_DQ = 0, QL_OP_FWD = 1, QL_OP_BWD = 2, QL_OP_FWD_LORDBA = 3 };
 
 /* Workspace bytes that op (QL_OP_*) needs for these sizes (0 if none). */
 size_t ql_workspace_bytes(int32_t op, int64_t M, int64_t N, int64_t K, int32_t r);

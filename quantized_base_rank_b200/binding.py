@@ -19,7 +19,7 @@ HEADER = os.path.join(os.path.dirname(_PKG), "include", "qlora.h")
 QL_OK, QL_ERR_INVALID_ARG, QL_ERR_UNSUPPORTED, QL_ERR_WORKSPACE, QL_ERR_NONFINITE, \
     QL_ERR_TIMEOUT, QL_ERR_CUDA = range(7)
 QL_FMT_NF4_DQ, QL_FMT_INT8_B64 = 0, 1
-QL_OP_DQ, QL_OP_FWD, QL_OP_BWD = 0, 1, 2
+QL_OP_DQ, QL_OP_FWD, QL_OP_BWD, QL_OP_FWD_LORDBA = 0, 1, 2, 3
 FORMATS = {"nf4_dq": QL_FMT_NF4_DQ, "int8": QL_FMT_INT8_B64}
 
 
@@ -37,6 +37,13 @@ class QLWeight(ctypes.Structure):
                 ("mean", ctypes.c_void_p)]
 
 
+class QLLordba(ctypes.Structure):
+    """ql_lordba: packed sign carriers and fp16 channel scales of a LoRDBA adapter."""
+    _fields_ = [("R", ctypes.c_int32), ("ell", ctypes.c_int32), ("B1", ctypes.c_void_p),
+                ("B2", ctypes.c_void_p), ("alpha", ctypes.c_void_p), ("beta", ctypes.c_void_p),
+                ("gamma", ctypes.c_void_p)]
+
+
 _lib = None
 _lock = threading.Lock()
 P, I64, I32, F32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
@@ -46,6 +53,7 @@ _SIGS = {
     "dq_quantize": ([P, I64, P, P, P, P, SZ, P], I32),
     "nf4_dq_quantize": ([P, I64, P, P, P, P, P, P, SZ, P], I32),
     "nf4_quantize_shard": ([P, I64, P, P, P, P, SZ, P], I32),
+    "qlora_linear_fwd_lordba": ([ctypes.POINTER(QLWeight), P, I64, ctypes.c_void_p, P, P, SZ, P], I32),
     "dq_quantize_shard": ([P, I64, P, I64, P, P, P, P], I32),
     "ql_dequantize": ([ctypes.POINTER(QLWeight), P, P], I32),
     "qlora_linear_fwd": ([ctypes.POINTER(QLWeight), P, I64, P, P, I32, F32, P, P, P, SZ, P], I32),
@@ -233,6 +241,42 @@ def dq_quantize_shard(absmax: torch.Tensor, bins: torch.Tensor, nblocks_total: i
     _check(lib().dq_quantize_shard(_ptr(absmax), nb, _ptr(bins), int(nblocks_total), _ptr(qabsmax),
                                    _ptr(group_scale), _ptr(mean), _stream(dev)), "dq_quantize_shard")
     return qabsmax, group_scale, mean
+
+
+def pack_signs(S: torch.Tensor) -> torch.Tensor:
+    """Pack a +-1 matrix [rows, cols] 1 bit per entry, the ql_lordba carrier layout:
+    bit j%32 of word j/32 of a row is 1 for +1. Returns int32 [rows, ceil(cols/32)]."""
+    rows, cols = S.shape
+    words = (cols + 31) // 32
+    bits = torch.zeros((rows, words * 32), dtype=torch.int64, device=S.device)
+    bits[:, :cols] = (S > 0).to(torch.int64)
+    shifts = torch.arange(32, device=S.device, dtype=torch.int64)
+    packed = (bits.view(rows, words, 32) << shifts).sum(dim=2)
+    packed = torch.where(packed >= 2 ** 31, packed - 2 ** 32, packed)
+    return packed.to(torch.int32).contiguous()
+
+
+def linear_fwd_lordba(qw: "QuantWeight", X: torch.Tensor, B1p: torch.Tensor, B2p: torch.Tensor,
+                      alpha: torch.Tensor, beta: torch.Tensor, gamma: torch.Tensor, R: int,
+                      Y: torch.Tensor | None = None) -> torch.Tensor:
+    """Y = X W'^T + X Delta W^T with the LoRDBA adapter given by packed carriers B1p
+    [N, ceil(R/32)], B2p [R, ceil(K/32)] (int32 words) and fp16 scales alpha [ell, N],
+    beta [ell, R], gamma [ell, K]."""
+    _need(X, torch.bfloat16, "X")
+    for t, nm in ((alpha, "alpha"), (beta, "beta"), (gamma, "gamma")):
+        _need(t, torch.float16, nm)
+    for t, nm in ((B1p, "B1"), (B2p, "B2")):
+        _need(t, torch.int32, nm)
+    M, K = X.shape
+    ell = alpha.shape[0]
+    dev = X.device
+    if Y is None:
+        Y = torch.empty((M, qw.N), dtype=torch.bfloat16, device=dev)
+    ad = QLLordba(R, ell, _ptr(B1p), _ptr(B2p), _ptr(alpha), _ptr(beta), _ptr(gamma))
+    ws = workspace(workspace_bytes(QL_OP_FWD_LORDBA, M, qw.N, K, R * ell), dev)
+    _check(lib().qlora_linear_fwd_lordba(ctypes.byref(qw.desc), _ptr(X), M, ctypes.addressof(ad), _ptr(Y),
+                                         _ptr(ws), ws.numel(), _stream(dev)), "qlora_linear_fwd_lordba")
+    return Y
 
 
 class QuantWeight:

@@ -39,6 +39,7 @@ ql_status small_m_forward(const ql_weight* w, const uint16_t* X, int64_t M, cons
                           cudaStream_t st);
 constexpr int64_t kSmallMMax = 16;
 bool small_m_supported(int64_t K, int r);   // rank <= 64 and the staging fits in shared memory
+int64_t lordba_ws_bytes(int64_t M, int64_t N, int64_t K, int r);   // lordba.cu
 int* device_flag_ptr();                 // device address of the sticky flag (current device)
 int num_sms();                          // SM count of the current device
 

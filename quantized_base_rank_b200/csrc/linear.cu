@@ -331,6 +331,10 @@ extern "C" {
 
 size_t ql_workspace_bytes(int32_t op, int64_t M, int64_t N, int64_t K, int32_t r) {
   if (op == QL_OP_DQ) return 256;
+  if (op == QL_OP_FWD_LORDBA) {
+    if (M < 0 || N < 0 || K < 0 || r < 1 || r > 256) return 0;
+    return (size_t)lordba_ws_bytes(M, N, K, r);
+  }
   if ((op != QL_OP_FWD && op != QL_OP_BWD) || M < 0 || N < 0 || K < 0 || r < 1 || r > 256) return 0;
   if (op == QL_OP_FWD && M <= kSmallMMax && small_m_supported(K, r)) return 0;   // decode-shaped path
   return (size_t)ws_layout(op, M, N, K, r).total;

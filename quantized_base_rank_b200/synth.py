@@ -140,3 +140,18 @@ def stack_linear_inputs(layer: int, which: int, N: int, K: int, M: int, r: int, 
     if backward:
         out["dY"] = device_normal_bf16((M, N), 1.0, seed, idx(DY_IDX), device)
     return out
+
+
+def lordba_inputs(N: int, K: int, R: int, ell: int, seed: int = 0) -> dict:
+    """A LoRDBA adapter for a weight [N, K]: sign carriers B1 [N, R], B2 [R, K] (+-1,
+    fp32) and fp16 channel scales alpha [ell, N] ~ U(0.5, 1) * 0.02 / sqrt(R),
+    beta [ell, R] ~ U(0.5, 1), gamma [ell, K] ~ U(0.5, 1), so that the branch is of the
+    same order as a N(0, 0.02) weight."""
+    g = _rng(seed, 40)
+    B1 = np.where(g.random((N, R)) < 0.5, -1.0, 1.0).astype(np.float32)
+    B2 = np.where(g.random((R, K)) < 0.5, -1.0, 1.0).astype(np.float32)
+    alpha = (g.uniform(0.5, 1.0, (ell, N)) * 0.02 / np.sqrt(R)).astype(np.float16)
+    beta = g.uniform(0.5, 1.0, (ell, R)).astype(np.float16)
+    gamma = g.uniform(0.5, 1.0, (ell, K)).astype(np.float16)
+    return {"B1": torch.from_numpy(B1), "B2": torch.from_numpy(B2), "alpha": torch.from_numpy(alpha),
+            "beta": torch.from_numpy(beta), "gamma": torch.from_numpy(gamma)}

@@ -57,6 +57,15 @@ def test_argument_validation_without_a_device(lib):
     assert lib.nf4_dq_quantize(16, 64 * (1 << 24) + 1, 16, 16, 16, 16, 16, 16, 256, None) == B.QL_ERR_UNSUPPORTED
     # workspace too small
     assert lib.nf4_dq_quantize(16, 64, 16, 16, 16, 16, 16, 16, 8, None) == B.QL_ERR_WORKSPACE
+    # LoRDBA forward: missing adapter, empty rank, rank beyond 256
+    w = B.QLWeight(0, 0, 64, 64, 16, 0, 16, 16, 16)
+    assert lib.qlora_linear_fwd_lordba(ctypes.byref(w), 16, 1, None, 16, 16, 1 << 20, None) == B.QL_ERR_INVALID_ARG
+    ad = B.QLLordba(0, 1, 16, 16, 16, 16, 16)
+    assert lib.qlora_linear_fwd_lordba(ctypes.byref(w), 16, 1, ctypes.addressof(ad), 16, 256, 1 << 20,
+                                       None) == B.QL_ERR_INVALID_ARG
+    ad = B.QLLordba(100, 3, 16, 16, 16, 16, 16)
+    assert lib.qlora_linear_fwd_lordba(ctypes.byref(w), 16, 1, ctypes.addressof(ad), 16, 256, 1 << 20,
+                                       None) == B.QL_ERR_UNSUPPORTED
     assert lib.ql_dequantize(None, None, None) == B.QL_ERR_INVALID_ARG
     w = B.QLWeight(0, 0, 64, 64, 16, 0, 16, 16, 16)
     # misaligned or null pointers, bad shapes: all rejected synchronously
