@@ -34,7 +34,7 @@ NF4_DQ_BYTES_PER_PARAM = 2.0 + 0.5 + 1.0 / 64 + 4.0 / 16384   # bf16 read + code
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the fused
 # forward GEMM on this workload, from one ncu capture (profiles/fwd_main_gemm_upproj_11008x4096_M8192.md),
 # valid only for the kernel sources it was taken on: reported as null once they change.
-FWD_MAIN_TRAFFIC = {"bytes": 112405248 + 149725184, "sources_sha256_16": "ec0d6b3a8f4fb70d"}
+FWD_MAIN_TRAFFIC = {"bytes": 103397120 + 149664000, "sources_sha256_16": "2a34a12501ce4503"}
 FWD_MAIN_SOURCES = ("quantized_base_rank_b200/csrc/gemm.cuh", "quantized_base_rank_b200/csrc/sm100.cuh",
                     "quantized_base_rank_b200/csrc/linear.cu", "quantized_base_rank_b200/csrc/common.cuh")
 
@@ -255,6 +255,79 @@ def decode_bench(dev, peaks, reps: int = 20):
     return out
 
 
+def lordba_bench(dev, peaks, qw_up, X_up, reps: int = 10):
+    """The LoRDBA double-binary adapter branch: (1) the up-projection forward (8192 tokens,
+    R = 64, one envelope term) against the same forward with a dense r = 64 adapter;
+    (2) the decode-shaped 4096x4096 NF4+DQ layer at M = 1, R = 16, timed like the dense
+    decode component (a CUDA graph over weight copies exceeding 3x L2)."""
+    from quantized_base_rank_b200 import binding as B
+    from quantized_base_rank_b200 import synth
+    out = {}
+    N, K = qw_up.N, qw_up.K
+    ad = synth.lordba_inputs(N, K, 64, 1, 3)
+    B1p, B2p = B.pack_signs(ad["B1"].to(dev)), B.pack_signs(ad["B2"].to(dev))
+    al, be, ga = (ad[k].to(dev) for k in ("alpha", "beta", "gamma"))
+    Y = torch.empty((X_up.shape[0], N), dtype=torch.bfloat16, device=dev)
+    for _ in range(3):
+        B.linear_fwd_lordba(qw_up, X_up, B1p, B2p, al, be, ga, 64, Y=Y)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        B.linear_fwd_lordba(qw_up, X_up, B1p, B2p, al, be, ga, 64, Y=Y)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    M = X_up.shape[0]
+    flops = 2 * M * N * K + 2 * M * K * 64 + 2 * M * N * 64
+    carrier_bytes = (N * 64 + 64 * K) / 8 + 2 * (N + 64 + K)
+    out["upproj_R64"] = {"ms": ms, "TFLOP/s": flops / (ms * 1e-3) / 1e12, "adapter_bytes": carrier_bytes,
+                         "dense_adapter_bytes": 2 * 64 * (N + K)}
+    # decode-shaped
+    base = synth.CFG2[0]
+    W = synth.weight_with_outliers(base.N, base.K, base.w_std, base.outlier_frac, base.outlier_mult,
+                                   base.seed).to(dev)
+    q0 = B.quantize_weight(W, "nf4_dq")
+    del W
+    n = base.N * base.K
+    ad = synth.lordba_inputs(base.N, base.K, 16, 1, 4)
+    B1p, B2p = B.pack_signs(ad["B1"].to(dev)), B.pack_signs(ad["B2"].to(dev))
+    al, be, ga = (ad[k].to(dev) for k in ("alpha", "beta", "gamma"))
+    wbytes = n * (0.5 + 1.0 / 64) + 4.0 * n / 16384
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    copies = max(4, int(np.ceil(3 * l2 / wbytes)))
+    qws = [B.QuantWeight("nf4_dq", base.N, base.K, q0.codes.clone(), None, q0.qabsmax.clone(),
+                         q0.group_scale.clone(), q0.mean.clone()) for _ in range(copies)]
+    X = synth.normal_bf16((1, base.K), 1.0, 5, 0).to(dev)
+    Y = torch.empty((1, base.N), dtype=torch.bfloat16, device=dev)
+    for qw in qws[:2]:
+        B.linear_fwd_lordba(qw, X, B1p, B2p, al, be, ga, 16, Y=Y)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    st = torch.cuda.Stream(dev)
+    st.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(st):
+        with torch.cuda.graph(g, stream=st):
+            for qw in qws:
+                B.linear_fwd_lordba(qw, X, B1p, B2p, al, be, ga, 16, Y=Y)
+    torch.cuda.synchronize()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / (reps * copies)
+    nbytes = wbytes + 2 * base.K + (base.N * 16 + 16 * base.K) / 8 + 2 * (base.N + 16 + base.K) + 2 * base.N
+    out["decode_7b_4096x4096_M1_R16"] = {"us_per_call": us, "bytes": nbytes,
+                                        "GB/s": nbytes / (us * 1e-6) / 1e9,
+                                        "frac_hbm": nbytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"]}
+    del g
+    return out
+
+
 def run_ours(args, case, world, rank, local_rank):
     from quantized_base_rank_b200 import binding as B
     from quantized_base_rank_b200 import dp, synth
@@ -390,6 +463,9 @@ def run_ours(args, case, world, rank, local_rank):
     # ---- decode-shaped forward (small M, HBM-bound) ----
     decode = decode_bench(dev, peaks)
 
+    # ---- LoRDBA double-binary adapter branch ----
+    lordba = lordba_bench(dev, peaks, qw, X)
+
     # ---- CPU oracle baseline (rank 0, one GPU only) ----
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -428,6 +504,7 @@ def run_ours(args, case, world, rank, local_rank):
             "bwd_dx_gemm": {"ms": dx_ms, "TFLOP/s": dx_flops / (dx_ms * 1e-3) / 1e12},
             "per_group_ms": {g: avg(g) for g in B.PROFILE_GROUPS if prof[g][1]},
             "decode_7b_4096x4096_nf4": decode,
+            "lordba": lordba,
         },
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},

@@ -25,34 +25,34 @@ __device__ __forceinline__ uint32_t sign_bit(const uint32_t* __restrict__ row, i
   return (__ldg(row + (j >> 5)) >> (j & 31)) & 1u;
 }
 
-// A_eff [ell*R, K] bf16: element (i*R + j, k) = sign(B2[j][k]) * bf16(beta_i[j] * gamma_i[k]).
+// One launch expands both operands, A_eff first, then B_eff (grid-stride over the two
+// ranges): the branch costs one small kernel before the GEMM, not two.
+//   A_eff [ell*R, K]: element (i*R + j, k) = sign(B2[j][k]) * bf16(beta_i[j] * gamma_i[k])
+//   B_eff [N, ell*R]: element (n, i*R + j) = sign(B1[n][j]) * bf16(alpha_i[n])
 // The fp16 x fp16 product is exact in fp32; negating a rounded value is exact.
 __global__ void __launch_bounds__(256)
-lordba_expand_a_kernel(const uint32_t* __restrict__ B2, const uint16_t* __restrict__ beta,
-                       const uint16_t* __restrict__ gamma, int R, int ell, int64_t K, uint16_t* __restrict__ A) {
-  const int64_t words = (K + 31) / 32;
-  const int64_t total = (int64_t)ell * R * K;
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t row = e / K, k = e % K;
-    const int i = (int)(row / R), j = (int)(row % R);
-    const float v = __fmul_rn(half_bits_to_float(beta[i * R + j]), half_bits_to_float(gamma[(int64_t)i * K + k]));
-    const uint32_t b = float_to_bf16_bits(v);
-    A[e] = (uint16_t)(sign_bit(B2 + j * words, (int)k) ? b : (b ^ 0x8000u));
-  }
-}
-
-// B_eff [N, ell*R] bf16: element (n, i*R + j) = sign(B1[n][j]) * bf16(alpha_i[n]).
-__global__ void __launch_bounds__(256)
-lordba_expand_b_kernel(const uint32_t* __restrict__ B1, const uint16_t* __restrict__ alpha, int R, int ell,
-                       int64_t N, uint16_t* __restrict__ Bo) {
-  const int words = (R + 31) / 32;
+lordba_expand_kernel(const uint32_t* __restrict__ B1, const uint32_t* __restrict__ B2,
+                     const uint16_t* __restrict__ alpha, const uint16_t* __restrict__ beta,
+                     const uint16_t* __restrict__ gamma, int R, int ell, int64_t N, int64_t K,
+                     uint16_t* __restrict__ A, uint16_t* __restrict__ Bo) {
+  const int64_t wk = (K + 31) / 32;
+  const int wr = (R + 31) / 32;
   const int r = ell * R;
-  const int64_t total = N * r;
+  const int64_t ea = (int64_t)r * K, total = ea + N * r;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t n = e / r;
-    const int c = (int)(e % r), i = c / R, j = c % R;
-    const uint32_t b = float_to_bf16_bits(half_bits_to_float(alpha[(int64_t)i * N + n]));
-    Bo[e] = (uint16_t)(sign_bit(B1 + n * words, j) ? b : (b ^ 0x8000u));
+    if (e < ea) {
+      const int64_t row = e / K, k = e % K;
+      const int i = (int)(row / R), j = (int)(row % R);
+      const float v = __fmul_rn(half_bits_to_float(beta[i * R + j]), half_bits_to_float(gamma[(int64_t)i * K + k]));
+      const uint32_t b = float_to_bf16_bits(v);
+      A[e] = (uint16_t)(sign_bit(B2 + j * wk, (int)k) ? b : (b ^ 0x8000u));
+    } else {
+      const int64_t f = e - ea;
+      const int64_t n = f / r;
+      const int c = (int)(f % r), i = c / R, j = c % R;
+      const uint32_t b = float_to_bf16_bits(half_bits_to_float(alpha[(int64_t)i * N + n]));
+      Bo[f] = (uint16_t)(sign_bit(B1 + n * wr, j) ? b : (b ^ 0x8000u));
+    }
   }
 }
 
@@ -90,13 +90,10 @@ extern "C" ql_status qlora_linear_fwd_lordba(const ql_weight* w, const ql_bf16* 
   uint8_t* fwd_ws = wsb + round256(r * K * 2) + round256(N * r * 2);
   const size_t fwd_bytes = ws_bytes - (size_t)(fwd_ws - wsb);
   {
-    ProfScope prof(PK_FWD_PREP, st, 2);
-    const int64_t ea = r64 * K, eb = N * r64;
-    lordba_expand_a_kernel<<<(int)imin64((ea + 255) / 256, (int64_t)num_sms() * 8), 256, 0, st>>>(
-        ad->B2, ad->beta, ad->gamma, ad->R, ad->ell, K, A_eff);
-    QL_CHECK_LAUNCH();
-    lordba_expand_b_kernel<<<(int)imin64((eb + 255) / 256, (int64_t)num_sms() * 8), 256, 0, st>>>(
-        ad->B1, ad->alpha, ad->R, ad->ell, N, B_eff);
+    ProfScope prof(PK_FWD_PREP, st, 1);
+    const int64_t total = r64 * K + N * r64;
+    lordba_expand_kernel<<<(int)imin64((total + 255) / 256, (int64_t)num_sms() * 8), 256, 0, st>>>(
+        ad->B1, ad->B2, ad->alpha, ad->beta, ad->gamma, ad->R, ad->ell, N, K, A_eff, B_eff);
     QL_CHECK_LAUNCH();
   }
   // s = alpha / r = 1: the scales are already in A_eff and B_eff

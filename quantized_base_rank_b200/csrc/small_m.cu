@@ -144,6 +144,25 @@ __device__ __forceinline__ float unit_scale(const UnitRegs<FMT>& u, float mu) {
   return __fdiv_rn(u.f, 127.0f);
 }
 
+// Warm L2 with bytes [lo, hi) of each of rows [0, rows) of a byte array whose rows are
+// `pitch` bytes apart: one prefetch per 128-byte line, threads t, t + nt, ... taking
+// successive lines. Every prefetched address lies inside a requested span.
+__device__ __forceinline__ void l2_prefetch_rows(const void* p, int64_t pitch, int64_t rows, int64_t lo,
+                                                 int64_t hi, int t, int nt) {
+  if (rows <= 0 || hi <= lo) return;
+  const int lpr = (int)((hi - lo + 127) >> 7) + 1;   // lines that can touch one row's span
+  const int total = (int)rows * lpr;
+  for (int i = t; i < total; i += nt) {
+    const int row = i / lpr, l = i - row * lpr;
+    const uintptr_t b = reinterpret_cast<uintptr_t>(p) + (uintptr_t)(row * pitch + lo);
+    const uintptr_t e = b + (uintptr_t)(hi - lo);
+    uintptr_t x = ((b >> 7) + (uintptr_t)l) << 7;
+    if (x >= e) continue;
+    if (x < b) x = b;
+    asm volatile("prefetch.global.L2 [%0];" :: "l"(x));
+  }
+}
+
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -192,16 +211,37 @@ small_m_fwd_kernel(const SmallArgs a) {
   const int64_t u0 = rank * U / kCS, u1 = (rank + 1) * U / kCS;
   const int nunits = (int)(u1 - u0);
   const int64_t k0 = u0 * 256;
-  const float mu = FMT == QL_FMT_NF4_DQ ? __ldg(a.mean) : 0.0f;
 
-  // The next launch on the stream may start now and stream its own weight while this
-  // one finishes.
+  // The next launch on the stream may start now and warm L2 with its own weight while
+  // this one finishes.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-  // Everything that depends only on the weight and the adapter goes out before the
-  // dependency wait (the preceding grid never writes them): the codes of the first two
-  // units, the adapter rows in fragment order, and this warp's rows of B. Only the token
-  // rows wait.
+  // Before the dependency wait this grid only warms L2 with what it is about to read: the
+  // codes and constants of its blocks, the adapter rows of its K-range, its rows of B and
+  // the token rows. The grid before it on the stream (a quantise, an adapter expansion,
+  // the previous layer) may still be writing any of these, and its writes are visible
+  // only after the wait; L2 is the point of coherence, so a prefetch never makes a later
+  // load return stale data. Every load proper comes after the wait.
+  {
+    const int64_t rows = a.N - n0 < kRowsPerCta ? a.N - n0 : kRowsPerCta;
+    const int64_t KB = a.K >> 6, kend = u1 * 256 < a.K ? u1 * 256 : a.K;
+    const int t = threadIdx.x;
+    if (FMT == QL_FMT_NF4_DQ) {
+      l2_prefetch_rows(a.codes + n0 * (a.K >> 1), a.K >> 1, rows, k0 >> 1, kend >> 1, t, 256);
+      l2_prefetch_rows(a.qabsmax + n0 * KB, KB, rows, u0 * 4, (kend + 63) >> 6, t, 256);
+      const int64_t g0 = (n0 * KB) >> 8, g1 = ((n0 + rows) * KB - 1) >> 8;
+      l2_prefetch_rows(a.gscale, 0, 1, g0 * 4, g1 * 4 + 4, t, 256);
+    } else {
+      l2_prefetch_rows(a.codes + n0 * a.K, a.K, rows, k0, kend, t, 256);
+      l2_prefetch_rows(a.absmax + n0 * KB, KB * 4, rows, u0 * 16, ((kend + 63) >> 6) * 4, t, 256);
+    }
+    l2_prefetch_rows(a.A, a.K * 2, a.r, k0 * 2, kend * 2, t, 256);
+    l2_prefetch_rows(a.B + n0 * a.r, 0, 1, 0, rows * a.r * 2, t, 256);
+    l2_prefetch_rows(a.X, a.K * 2, a.M < NT ? a.M : NT, k0 * 2, kend * 2, t, 256);
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const float mu = FMT == QL_FMT_NF4_DQ ? __ldg(a.mean) : 0.0f;
+
   const int64_t row_g = n0 + warp * 16 + g, row_h = row_g + 8;
   // adapter right factor for this warp's rows (A fragments of the final MMA)
   auto bload = [&](int64_t row, int j) -> uint32_t {
@@ -267,9 +307,7 @@ small_m_fwd_kernel(const SmallArgs a) {
       }
     }
   };
-  stage_rows(NT, NT + RP);                          // adapter rows
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  stage_rows(0, NT);                                // token rows
+  stage_rows(0, NT + RP);                           // token rows, then adapter rows
   __syncthreads();
 
   // ---- main loop: W' rows (decoded) and, for the adapter, A rows against the tokens ----
@@ -432,8 +470,8 @@ static ql_status launch_small(const SmallArgs& a, cudaStream_t st) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return QL_ERR_CUDA;
   const int groups = (int)((a.N + kRowsPerCta - 1) / kRowsPerCta);
-  // programmatic dependent launch: this grid may begin (and prefetch its weight) while the
-  // previous grid on the stream finishes; the kernel waits before touching X, A, B or Y
+  // programmatic dependent launch: this grid may begin (and warm L2 with its inputs) while
+  // the previous grid on the stream finishes; the kernel waits before loading any input
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(groups * kCS);
   cfg.blockDim = dim3(256);
