@@ -21,6 +21,9 @@ It is a plain, slow, obviously correct restatement of what the method computes:
 * The low-rank double-binary adapter of the LoRDBA page (section "2. Methodology",
   core architecture): Delta W = sum_i diag(alpha_i) B1 diag(beta_i) B2 diag(gamma_i)
   with sign carriers B1, B2 in {+-1}, in fp64.
+* The Walsh-Hadamard adapter of the QWHA page (gist.science/ko/paper/2509.17428,
+  section 2.1): Delta W = F H^{-1} with a sparse coefficient matrix F and the
+  Walsh-Hadamard matrix H, in fp64.
 
 Where the pages are silent the reading taken is stated in the docstring of the
 function that takes it. Floating-point steps are written with numpy float32 scalars
@@ -409,3 +412,88 @@ def lordba_linear_fwd(X, Wd, alpha, beta, gamma, B1, B2):
     X = np.asarray(X, np.float64)
     Wd = np.asarray(Wd, np.float64)
     return X @ Wd.T + X @ lordba_delta(alpha, beta, gamma, B1, B2).T
+
+
+# --------------------------------------------------------------------------------------
+# QWHA: Walsh-Hadamard adapter (QWHA page, gist.science/ko/paper/2509.17428, section
+# "2.1 Adapter design: Walsh-Hadamard adaptation"): Delta W = F H^{-1} with a sparse
+# coefficient matrix F (values c at the positions of an index list E) and the
+# predefined Walsh-Hadamard transform H
+# --------------------------------------------------------------------------------------
+
+def wht_block_size(K: int) -> int:
+    """Order of the Walsh-Hadamard blocks of H for an input width K.
+
+    Reading: a Walsh-Hadamard matrix exists only for power-of-two orders and the page
+    does not say what H is when K is not one (LLaMA's 11008 and 22016 are 2^8 * 43 and
+    2^9 * 43). H is taken as the block-diagonal matrix whose blocks are the Walsh-Hadamard
+    matrix of the largest power of two dividing K, which keeps Delta W = F H^{-1} a K x K
+    product; for a power-of-two K it is the single full-width transform."""
+    assert K >= 1
+    return K & (-K)
+
+
+def walsh_hadamard(K: int) -> np.ndarray:
+    """H [K, K] in fp64: block-diagonal with blocks of order b = wht_block_size(K),
+    entry (i, j) of a block = (-1)^popcount(i & j) / sqrt(b).
+
+    Reading: the page names H only as the predefined WHT matrix. Sylvester's (natural)
+    ordering is taken, the one the recursion H_2n = [[H_n, H_n], [H_n, -H_n]] produces,
+    and the orthonormal scaling 1/sqrt(b), so that H is symmetric and orthogonal. Another
+    ordering of the same Walsh functions only relabels the columns of F (the positions
+    E), and another scale only rescales c."""
+    b = wht_block_size(K)
+    i = np.arange(b)
+    par = np.zeros((b, b), dtype=np.int64)
+    ij = i[:, None] & i[None, :]
+    while np.any(ij):
+        par ^= ij & 1
+        ij = ij >> 1
+    blk = np.where(par == 1, -1.0, 1.0) / math.sqrt(b)
+    H = np.zeros((K, K))
+    for s in range(0, K, b):
+        H[s:s + b, s:s + b] = blk
+    return H
+
+
+def qwha_dense_F(N: int, K: int, row_ptr, col, c) -> np.ndarray:
+    """The sparse coefficient matrix F [N, K] written out densely: row n holds the values
+    c[j] at columns col[j] for j in [row_ptr[n], row_ptr[n+1]).
+
+    Reading: the page gives F as a value vector c and an index list E. E is taken in
+    compressed-row form (row offsets plus column indices), the position (n, col[j]) of
+    each value; every position appears at most once."""
+    row_ptr = np.asarray(row_ptr, np.int64)
+    col = np.asarray(col, np.int64)
+    c = np.asarray(c, np.float64)
+    assert row_ptr.shape == (N + 1,) and row_ptr[0] == 0 and np.all(np.diff(row_ptr) >= 0)
+    assert col.shape == c.shape == (row_ptr[-1],)
+    F = np.zeros((N, K))
+    for n in range(N):
+        for j in range(row_ptr[n], row_ptr[n + 1]):
+            assert 0 <= col[j] < K and F[n, col[j]] == 0.0
+            F[n, col[j]] = c[j]
+    return F
+
+
+def qwha_delta(N: int, K: int, row_ptr, col, c) -> np.ndarray:
+    """Delta W = F H^{-1} [N, K] in fp64 (the page's single-transform formula). H is
+    orthogonal, so H^{-1} is its transpose."""
+    return qwha_dense_F(N, K, row_ptr, col, c) @ walsh_hadamard(K).T
+
+
+def qwha_transform(X) -> np.ndarray:
+    """Z = X H^{-T} in fp64: each token row x becomes H^{-1} x, the transformed input that
+    F multiplies in Delta W x = F (H^{-1} x)."""
+    X = np.asarray(X, np.float64)
+    H_inv = walsh_hadamard(X.shape[1]).T          # H is orthogonal
+    return X @ H_inv.T
+
+
+def qwha_linear_fwd(X, Wd, row_ptr, col, c) -> np.ndarray:
+    """Y = X Wd^T + X Delta W^T in fp64: the frozen (dequantised) base plus the unmerged
+    Walsh-Hadamard adapter, with Delta W = F H^{-1} [N, K]."""
+    X = np.asarray(X, np.float64)
+    Wd = np.asarray(Wd, np.float64)
+    N, K = Wd.shape
+    return X @ Wd.T + X @ qwha_delta(N, K, row_ptr, col, c).T

@@ -155,3 +155,37 @@ def lordba_inputs(N: int, K: int, R: int, ell: int, seed: int = 0) -> dict:
     gamma = g.uniform(0.5, 1.0, (ell, K)).astype(np.float16)
     return {"B1": torch.from_numpy(B1), "B2": torch.from_numpy(B2), "alpha": torch.from_numpy(alpha),
             "beta": torch.from_numpy(beta), "gamma": torch.from_numpy(gamma)}
+
+
+def qwha_inputs(N: int, K: int, r_equiv: int, seed: int = 0, c_std: float = 0.02) -> dict:
+    """A Walsh-Hadamard adapter for a weight [N, K] in compressed-row form.
+
+    Budget: p = r_equiv * (N + K) coefficients, the trainable-parameter count of a rank
+    r_equiv LoRA adapter on the same weight. Per-row counts: a floor of max(1, p / (4N))
+    per output channel, the rest spread in proportion to a log-normal(0, 1) channel weight
+    (a heavy-tailed stand-in for a per-channel error magnitude), each capped at K.
+    Positions: distinct columns drawn uniformly per row, sorted ascending. Values:
+    c ~ N(0, c_std) rounded to bf16.
+
+    Returns row_ptr (int32 [N+1]), col (uint16 [nnz]), c (bf16 [nnz]) as CPU tensors."""
+    assert 1 <= K <= 65536 and N >= 1
+    g = _rng(seed, 50)
+    p = min(r_equiv * (N + K), N * K)
+    floor = max(1, p // (4 * N))
+    w = g.lognormal(0.0, 1.0, N)
+    extra = max(p - floor * N, 0)
+    share = extra * w / w.sum()
+    cnt = floor + np.floor(share).astype(np.int64)
+    short = p - int(cnt.sum())
+    if short > 0:                                   # largest remainders take the rest
+        order = np.argsort(-(share - np.floor(share)), kind="stable")
+        cnt[order[:short]] += 1
+    cnt = np.minimum(cnt, K)
+    row_ptr = np.zeros(N + 1, np.int64)
+    row_ptr[1:] = np.cumsum(cnt)
+    col = np.empty(int(row_ptr[-1]), np.uint16)
+    for n in range(N):
+        col[row_ptr[n]:row_ptr[n + 1]] = np.sort(g.choice(K, int(cnt[n]), replace=False))
+    c = g.standard_normal(int(row_ptr[-1]), dtype=np.float32) * np.float32(c_std)
+    return {"row_ptr": torch.from_numpy(row_ptr.astype(np.int32)), "col": torch.from_numpy(col),
+            "c": to_bf16(c)}

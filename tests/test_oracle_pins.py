@@ -457,3 +457,112 @@ def test_lordba_linear_is_base_plus_branch():
         for n in range(Wd.shape[0]):
             naive[t, n] = sum(X[t, k] * (Wd[n, k] + D[n, k]) for k in range(X.shape[1]))
     np.testing.assert_allclose(Y, naive, rtol=1e-12)
+
+
+# ---------------------------------------------------------------- QWHA adapter
+
+def _walsh_butterflies(x, b):
+    """The fast recursive Walsh-Hadamard transform of each length-b block of x, written
+    as in-place butterflies of adds and subtracts (the page's fast kernel), then scaled
+    by 1/sqrt(b). Plain Python floats."""
+    x = [float(v) for v in x]
+    for s in range(0, len(x), b):
+        h = 1
+        while h < b:
+            for i in range(s, s + b, 2 * h):
+                for j in range(i, i + h):
+                    u, v = x[j], x[j + h]
+                    x[j], x[j + h] = u + v, u - v
+            h *= 2
+    return [v / math.sqrt(b) for v in x]
+
+
+def _qwha_case(N=7, K=192, seed=5):
+    rng = np.random.default_rng(seed)
+    cnt = rng.integers(0, 6, N)
+    row_ptr = np.concatenate([[0], np.cumsum(cnt)])
+    col = np.concatenate([np.sort(rng.choice(K, k, replace=False)) for k in cnt]).astype(np.int64)
+    c = rng.standard_normal(int(row_ptr[-1]))
+    return row_ptr, col, c
+
+
+@pytest.mark.parametrize("b", [1, 2, 4, 8, 16, 32, 64, 128, 256])
+def test_qwha_hadamard_is_sylvester(b):
+    """H for a power-of-two width is scipy's Sylvester-construction Hadamard matrix / sqrt(b)."""
+    import scipy.linalg
+    np.testing.assert_array_equal(o.walsh_hadamard(b) * math.sqrt(b), scipy.linalg.hadamard(b))
+
+
+def test_qwha_block_structure():
+    """Non-power-of-two widths: H = I (x) H_b with b the largest power of two dividing K
+    (11008 = 2^8 * 43, 22016 = 2^9 * 43)."""
+    import scipy.linalg
+    assert [o.wht_block_size(K) for K in (4096, 8192, 11008, 22016, 192)] == [4096, 8192, 256, 512, 64]
+    want = np.kron(np.eye(3), scipy.linalg.hadamard(64) / 8.0)
+    np.testing.assert_array_equal(o.walsh_hadamard(192), want)
+
+
+def test_qwha_H_is_orthogonal_and_inverts():
+    H = o.walsh_hadamard(96)
+    np.testing.assert_allclose(H @ H.T, np.eye(96), atol=1e-14)
+    np.testing.assert_allclose(np.linalg.inv(H), H.T, atol=1e-13)
+
+
+def test_qwha_single_coefficient_is_a_walsh_function():
+    """One value c at (n, k): row n of Delta W = F H^{-1} is c times the Walsh function
+    j -> (-1)^popcount(k & j) / sqrt(b) on the block holding k, zero elsewhere; every
+    other row is zero."""
+    N, K, n, k, c = 4, 192, 2, 77, 0.375
+    row_ptr = [0, 0, 0, 1, 1]
+    D = o.qwha_delta(N, K, row_ptr, [k], [c])
+    b = 64
+    want = np.zeros((N, K))
+    s = (k // b) * b
+    for j in range(s, s + b):
+        want[n, j] = c * (-1) ** bin((k - s) & (j - s)).count("1") / math.sqrt(b)
+    np.testing.assert_allclose(D, want, rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("K", [64, 128, 192])
+def test_qwha_transform_equals_butterflies_and_keeps_norms(K):
+    """Z = H^{-1} x per token equals the add/subtract recursion, and the orthonormal
+    transform keeps each block's Euclidean norm."""
+    rng = np.random.default_rng(K)
+    X = rng.standard_normal((3, K))
+    Z = o.qwha_transform(X)
+    b = o.wht_block_size(K)
+    for t in range(3):
+        np.testing.assert_allclose(Z[t], _walsh_butterflies(X[t], b), rtol=0, atol=1e-12)
+        for s in range(0, K, b):
+            assert math.isclose(np.linalg.norm(Z[t, s:s + b]), np.linalg.norm(X[t, s:s + b]), rel_tol=1e-13)
+
+
+def test_qwha_linear_as_sparse_gather_of_the_transformed_input():
+    """Y = X Wd^T + X (F H^{-1})^T equals the page's association Delta W x = F (H^{-1} x):
+    the butterfly transform of x, then for every stored value c at (n, k) an add of
+    c * z_k into y_n (loops)."""
+    N, K = 7, 192
+    row_ptr, col, c = _qwha_case(N, K)
+    rng = np.random.default_rng(11)
+    X = rng.standard_normal((4, K))
+    Wd = rng.standard_normal((N, K))
+    Y = o.qwha_linear_fwd(X, Wd, row_ptr, col, c)
+    for t in range(4):
+        z = _walsh_butterflies(X[t], o.wht_block_size(K))
+        for n in range(N):
+            y = sum(X[t, k] * Wd[n, k] for k in range(K))
+            for j in range(row_ptr[n], row_ptr[n + 1]):
+                y += c[j] * z[col[j]]
+            assert math.isclose(Y[t, n], y, rel_tol=1e-11, abs_tol=1e-11)
+
+
+def test_qwha_zero_and_linear_in_c():
+    N, K = 7, 192
+    row_ptr, col, c = _qwha_case(N, K)
+    rng = np.random.default_rng(3)
+    X = rng.standard_normal((2, K))
+    Wd = rng.standard_normal((N, K))
+    np.testing.assert_allclose(o.qwha_linear_fwd(X, Wd, row_ptr, col, 0 * c), X @ Wd.T, rtol=1e-13)
+    D1 = o.qwha_delta(N, K, row_ptr, col, c)
+    D2 = o.qwha_delta(N, K, row_ptr, col, -2.5 * c)
+    np.testing.assert_allclose(D2, -2.5 * D1, rtol=1e-13, atol=1e-15)
