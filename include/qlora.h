@@ -220,13 +220,53 @@ ql_status qlora_linear_fwd_lordba(const ql_weight* w, const ql_bf16* X, int64_t 
                                   const ql_lordba* adapter, ql_bf16* Y, void* ws,
                                   size_t ws_bytes, void* stream);
 
-enum { QL_OP_DQ = 0, QL_OP_FWD = 1, QL_OP_BWD = 2, QL_OP_FWD_LORDBA = 3 };
+/* A Walsh-Hadamard adapter (QWHA page, gist.science/ko/paper/2509.17428, section 2.1
+ * "Walsh-Hadamard adaptation"): Delta W = F H^{-1}, F [N, K] sparse with values c at the
+ * positions of an index list E, H the Walsh-Hadamard transform. E is held in
+ * compressed-row form:
+ *   row_ptr: device int32 [N + 1], row_ptr[0] = 0, nondecreasing, row_ptr[N] = nnz;
+ *   col:     device uint16 [nnz], the column k of each value; within a row, distinct;
+ *   c:       device bf16 [nnz], the values (row n holds j in [row_ptr[n], row_ptr[n+1])).
+ * H is the orthonormal Sylvester-order Walsh-Hadamard matrix when K is a power of two;
+ * otherwise block-diagonal, with blocks of the largest power of two dividing K (so
+ * H = H^T = H^{-1}). The caller keeps the arrays alive until the stream passes the call;
+ * nothing is copied. col and c may be NULL when nnz = 0. */
+typedef struct {
+  const int32_t* row_ptr;
+  const uint16_t* col;
+  const ql_bf16* c;
+  int64_t nnz;
+} ql_qwha;
+
+/* Forward of the quantised linear with a Walsh-Hadamard adapter, unmerged:
+ *   Y [M, N] = bf16( bf16(X W'^T) + sum over row n's values of c_j * Z[m, col_j] ),
+ *   Z = X H^{-T} = X H  (H^{-1} x per token), computed in fp32 by the add/subtract
+ *   recursion and rounded once to bf16; the sparse sums accumulate in fp32.
+ * Shapes and formats as qlora_linear_fwd (K a multiple of 64, K <= 65536, N a multiple
+ * of 8). The base product takes the same kernels as qlora_linear_fwd without a LoRA
+ * branch. Column indices >= K and row offsets outside [0, nnz] are skipped on the
+ * device and reported as QL_ERR_INVALID_ARG by ql_get_device_status; the contents of
+ * the index arrays are not read on the host.
+ * ws: ql_workspace_bytes(QL_OP_FWD_QWHA, M, N, K, 0) bytes, 256-byte aligned (it holds
+ * Z in slabs of 16 tokens, [ceil(M/16)][K][16] bf16, and the base product's scratch). */
+ql_status qlora_linear_fwd_qwha(const ql_weight* w, const ql_bf16* X, int64_t M,
+                                const ql_qwha* adapter, ql_bf16* Y, void* ws,
+                                size_t ws_bytes, void* stream);
+
+/* The Walsh-Hadamard transform of each token row alone: Z [M, K] bf16 = bf16(X H^{-T})
+ * with the H of ql_qwha (orthonormal, blockwise for K not a power of two), by the
+ * add/subtract recursion in fp32 (QWHA page, section 2.1, the fast WHT kernel).
+ * X and Z are 16-byte aligned, K a multiple of 64. */
+ql_status ql_wht(const ql_bf16* X, int64_t M, int64_t K, ql_bf16* Z, void* stream);
+
+enum { QL_OP_DQ = 0, QL_OP_FWD = 1, QL_OP_BWD = 2, QL_OP_FWD_LORDBA = 3, QL_OP_FWD_QWHA = 4 };
 
 /* Workspace bytes that op (QL_OP_*) needs for these sizes (0 if none). */
 size_t ql_workspace_bytes(int32_t op, int64_t M, int64_t N, int64_t K, int32_t r);
 
 /* Synchronise `stream`, then return and clear the sticky device flag of the current
- * device (QL_OK, QL_ERR_NONFINITE or QL_ERR_TIMEOUT). */
+ * device (QL_OK, QL_ERR_NONFINITE, QL_ERR_TIMEOUT, or QL_ERR_INVALID_ARG when a sparse
+ * index read on the device was out of range). */
 ql_status ql_get_device_status(void* stream);
 
 /* Which fused weight GEMM the linear uses for M > 16: 0 (the default) runs it on single
@@ -245,7 +285,8 @@ void ql_set_wait_timeout_ns(uint64_t ns);
  * them and returns (then forgets) the summed milliseconds and the number of launches of
  * one group. Groups: 0 nf4 encode, 1 double quantisation, 2 int8 encode, 3 dequantise,
  * 4 forward layout prep, 5 forward X A^T, 6 forward main GEMM, 7 backward layout prep,
- * 8 backward dY B, 9 dB, 10 dA, 11 dX, 12 small-M forward. ql_launch_count is the
+ * 8 backward dY B, 9 dB, 10 dA, 11 dX, 12 small-M forward, 13 Walsh-Hadamard adapter
+ * (transform and sparse product). ql_launch_count is the
  * running number of kernels the library has launched in this process. Returns 0, or -1
  * for an unknown group. */
 void ql_profile_enable(int on);

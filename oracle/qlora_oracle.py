@@ -37,6 +37,7 @@ flattening, group = 256 consecutive blocks.
 """
 from __future__ import annotations
 
+import functools
 import math
 import statistics
 
@@ -433,23 +434,31 @@ def wht_block_size(K: int) -> int:
     return K & (-K)
 
 
-def walsh_hadamard(K: int) -> np.ndarray:
-    """H [K, K] in fp64: block-diagonal with blocks of order b = wht_block_size(K),
-    entry (i, j) of a block = (-1)^popcount(i & j) / sqrt(b).
+@functools.lru_cache(maxsize=4)
+def walsh_hadamard_block(b: int) -> np.ndarray:
+    """One Walsh-Hadamard block [b, b] in fp64: entry (i, j) = (-1)^popcount(i & j) / sqrt(b).
 
     Reading: the page names H only as the predefined WHT matrix. Sylvester's (natural)
     ordering is taken, the one the recursion H_2n = [[H_n, H_n], [H_n, -H_n]] produces,
     and the orthonormal scaling 1/sqrt(b), so that H is symmetric and orthogonal. Another
     ordering of the same Walsh functions only relabels the columns of F (the positions
     E), and another scale only rescales c."""
-    b = wht_block_size(K)
+    assert b >= 1 and b & (b - 1) == 0
     i = np.arange(b)
     par = np.zeros((b, b), dtype=np.int64)
     ij = i[:, None] & i[None, :]
     while np.any(ij):
         par ^= ij & 1
         ij = ij >> 1
-    blk = np.where(par == 1, -1.0, 1.0) / math.sqrt(b)
+    H = np.where(par == 1, -1.0, 1.0) / math.sqrt(b)
+    H.flags.writeable = False                       # shared by the cache
+    return H
+
+
+def walsh_hadamard(K: int) -> np.ndarray:
+    """H [K, K] in fp64: block-diagonal with blocks walsh_hadamard_block(wht_block_size(K))."""
+    b = wht_block_size(K)
+    blk = walsh_hadamard_block(b)
     H = np.zeros((K, K))
     for s in range(0, K, b):
         H[s:s + b, s:s + b] = blk
@@ -479,15 +488,50 @@ def qwha_dense_F(N: int, K: int, row_ptr, col, c) -> np.ndarray:
 def qwha_delta(N: int, K: int, row_ptr, col, c) -> np.ndarray:
     """Delta W = F H^{-1} [N, K] in fp64 (the page's single-transform formula). H is
     orthogonal, so H^{-1} is its transpose."""
-    return qwha_dense_F(N, K, row_ptr, col, c) @ walsh_hadamard(K).T
+    H_inv = walsh_hadamard(K).T
+    return qwha_dense_F(N, K, row_ptr, col, c) @ H_inv
 
 
 def qwha_transform(X) -> np.ndarray:
     """Z = X H^{-T} in fp64: each token row x becomes H^{-1} x, the transformed input that
-    F multiplies in Delta W x = F (H^{-1} x)."""
+    F multiplies in Delta W x = F (H^{-1} x). H is block-diagonal, so the product is taken
+    one diagonal block at a time (the same numbers as the full K x K product without
+    forming it); each block is orthogonal, so its inverse is its transpose."""
     X = np.asarray(X, np.float64)
-    H_inv = walsh_hadamard(X.shape[1]).T          # H is orthogonal
-    return X @ H_inv.T
+    K = X.shape[1]
+    b = wht_block_size(K)
+    H_inv = walsh_hadamard_block(b).T
+    Z = np.empty_like(X)
+    for s in range(0, K, b):
+        Z[:, s:s + b] = X[:, s:s + b] @ H_inv.T
+    return Z
+
+
+def qwha_adapter_out(Z, N: int, row_ptr, col, c) -> np.ndarray:
+    """Z F^T [M, N] in fp64: for each token, F applied to its transformed input, i.e. the
+    page's F (H^{-1} x), with F given by its compressed rows (a scipy sparse product)."""
+    import scipy.sparse
+    Z = np.asarray(Z, np.float64)
+    row_ptr = np.asarray(row_ptr, np.int64)
+    col = np.asarray(col, np.int64)
+    c = np.asarray(c, np.float64)
+    K = Z.shape[1]
+    assert row_ptr.shape == (N + 1,) and row_ptr[0] == 0 and np.all(np.diff(row_ptr) >= 0)
+    assert col.shape == c.shape == (row_ptr[-1],) and np.all((col >= 0) & (col < K))
+    for n in range(N):                              # positions within a row are distinct
+        seg = col[row_ptr[n]:row_ptr[n + 1]]
+        assert np.unique(seg).size == seg.size
+    F = scipy.sparse.csr_matrix((c, col, row_ptr), shape=(N, K))
+    return np.asarray((F @ Z.T).T)
+
+
+def qwha_linear_fwd_factored(X, Wd, row_ptr, col, c) -> np.ndarray:
+    """The same Y as qwha_linear_fwd in the page's order Delta W x = F (H^{-1} x): the
+    transform of each token, then the sparse product. For widths where forming
+    Delta W [N, K] or H [K, K] would be too large."""
+    X = np.asarray(X, np.float64)
+    Wd = np.asarray(Wd, np.float64)
+    return X @ Wd.T + qwha_adapter_out(qwha_transform(X), Wd.shape[0], row_ptr, col, c)
 
 
 def qwha_linear_fwd(X, Wd, row_ptr, col, c) -> np.ndarray:

@@ -19,7 +19,7 @@ HEADER = os.path.join(os.path.dirname(_PKG), "include", "qlora.h")
 QL_OK, QL_ERR_INVALID_ARG, QL_ERR_UNSUPPORTED, QL_ERR_WORKSPACE, QL_ERR_NONFINITE, \
     QL_ERR_TIMEOUT, QL_ERR_CUDA = range(7)
 QL_FMT_NF4_DQ, QL_FMT_INT8_B64 = 0, 1
-QL_OP_DQ, QL_OP_FWD, QL_OP_BWD, QL_OP_FWD_LORDBA = 0, 1, 2, 3
+QL_OP_DQ, QL_OP_FWD, QL_OP_BWD, QL_OP_FWD_LORDBA, QL_OP_FWD_QWHA = 0, 1, 2, 3, 4
 FORMATS = {"nf4_dq": QL_FMT_NF4_DQ, "int8": QL_FMT_INT8_B64}
 
 
@@ -35,6 +35,12 @@ class QLWeight(ctypes.Structure):
                 ("codes", ctypes.c_void_p), ("absmax", ctypes.c_void_p),
                 ("qabsmax", ctypes.c_void_p), ("group_scale", ctypes.c_void_p),
                 ("mean", ctypes.c_void_p)]
+
+
+class QLQwha(ctypes.Structure):
+    """ql_qwha: the sparse coefficients of a Walsh-Hadamard adapter in compressed rows."""
+    _fields_ = [("row_ptr", ctypes.c_void_p), ("col", ctypes.c_void_p), ("c", ctypes.c_void_p),
+                ("nnz", ctypes.c_int64)]
 
 
 class QLLordba(ctypes.Structure):
@@ -54,6 +60,8 @@ _SIGS = {
     "nf4_dq_quantize": ([P, I64, P, P, P, P, P, P, SZ, P], I32),
     "nf4_quantize_shard": ([P, I64, P, P, P, P, SZ, P], I32),
     "qlora_linear_fwd_lordba": ([ctypes.POINTER(QLWeight), P, I64, ctypes.c_void_p, P, P, SZ, P], I32),
+    "qlora_linear_fwd_qwha": ([ctypes.POINTER(QLWeight), P, I64, ctypes.c_void_p, P, P, SZ, P], I32),
+    "ql_wht": ([P, I64, I64, P, P], I32),
     "dq_quantize_shard": ([P, I64, P, I64, P, P, P, P], I32),
     "ql_dequantize": ([ctypes.POINTER(QLWeight), P, P], I32),
     "qlora_linear_fwd": ([ctypes.POINTER(QLWeight), P, I64, P, P, I32, F32, P, P, P, SZ, P], I32),
@@ -72,7 +80,7 @@ _SIGS = {
 
 # kernel groups of ql_profile_read
 PROFILE_GROUPS = ["nf4", "dq", "int8", "dequant", "fwd_prep", "fwd_xa", "fwd_main", "bwd_prep",
-                  "bwd_dyb", "bwd_db", "bwd_da", "bwd_dx", "fwd_small"]
+                  "bwd_dyb", "bwd_db", "bwd_da", "bwd_dx", "fwd_small", "fwd_adapter"]
 
 
 def lib() -> ctypes.CDLL:
@@ -277,6 +285,36 @@ def linear_fwd_lordba(qw: "QuantWeight", X: torch.Tensor, B1p: torch.Tensor, B2p
     _check(lib().qlora_linear_fwd_lordba(ctypes.byref(qw.desc), _ptr(X), M, ctypes.addressof(ad), _ptr(Y),
                                          _ptr(ws), ws.numel(), _stream(dev)), "qlora_linear_fwd_lordba")
     return Y
+
+
+def linear_fwd_qwha(qw: "QuantWeight", X: torch.Tensor, row_ptr: torch.Tensor, col: torch.Tensor,
+                    c: torch.Tensor, Y: torch.Tensor | None = None) -> torch.Tensor:
+    """Y = X W'^T + X (F H^{-1})^T with the Walsh-Hadamard adapter F given in compressed
+    rows: row_ptr int32 [N+1], col uint16 [nnz], c bf16 [nnz]."""
+    _need(X, torch.bfloat16, "X")
+    _need(row_ptr, torch.int32, "row_ptr")
+    _need(col, torch.uint16, "col")
+    _need(c, torch.bfloat16, "c")
+    M, K = X.shape
+    dev = X.device
+    if Y is None:
+        Y = torch.empty((M, qw.N), dtype=torch.bfloat16, device=dev)
+    nnz = c.numel()
+    ad = QLQwha(_ptr(row_ptr), _ptr(col) if nnz else None, _ptr(c) if nnz else None, nnz)
+    ws = workspace(workspace_bytes(QL_OP_FWD_QWHA, M, qw.N, K, 0), dev)
+    _check(lib().qlora_linear_fwd_qwha(ctypes.byref(qw.desc), _ptr(X), M, ctypes.addressof(ad), _ptr(Y),
+                                       _ptr(ws), ws.numel(), _stream(dev)), "qlora_linear_fwd_qwha")
+    return Y
+
+
+def wht(X: torch.Tensor, Z: torch.Tensor | None = None) -> torch.Tensor:
+    """Z = X H^{-T}: the orthonormal (blockwise) Walsh-Hadamard transform of each row."""
+    _need(X, torch.bfloat16, "X")
+    M, K = X.shape
+    if Z is None:
+        Z = torch.empty_like(X)
+    _check(lib().ql_wht(_ptr(X), M, K, _ptr(Z), _stream(X.device)), "ql_wht")
+    return Z
 
 
 class QuantWeight:

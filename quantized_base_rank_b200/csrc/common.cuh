@@ -12,6 +12,7 @@ constexpr int kBlock = 64;        // elements per quantisation block
 constexpr int kGroup = 256;       // blocks per double-quantisation group
 constexpr int kFlagNonfinite = 1;
 constexpr int kFlagTimeout = 2;
+constexpr int kFlagBadIndex = 4;    // a sparse index read on the device was out of range
 
 // NF4 grid and its exact decision points, computed once on the host by this
 // library (runtime.cu) and passed to kernels by value.
@@ -38,8 +39,16 @@ ql_status small_m_forward(const ql_weight* w, const uint16_t* X, int64_t M, cons
                           const uint16_t* B, int r, float alpha, uint16_t* Y, uint16_t* T_save,
                           cudaStream_t st);
 constexpr int64_t kSmallMMax = 16;
-bool small_m_supported(int64_t K, int r);   // rank <= 64 and the staging fits in shared memory
+bool small_m_supported(int64_t K, int r);   // 0 <= rank <= 64 (0: no adapter), staging fits in smem
 int64_t lordba_ws_bytes(int64_t M, int64_t N, int64_t K, int r);   // lordba.cu
+// Y = X deq(W)^T + Zext Wext^T (linear.cu): the fused forward GEMM with caller-given
+// extension operands [M, kext] and [N, kext] (kext % 64 == 0; 0 = the base product alone);
+// scratch of ext_fwd_ws_bytes, 256-aligned
+int64_t ext_fwd_ws_bytes(int64_t M, int64_t N, int64_t K, int64_t kext);
+ql_status ext_forward(const ql_weight* w, const uint16_t* X, int64_t M, const uint16_t* Zext,
+                      const uint16_t* Wext, int64_t kext, uint16_t* Y, void* ws, size_t ws_bytes,
+                      cudaStream_t st);
+int64_t qwha_ws_bytes(int64_t M, int64_t N, int64_t K);             // qwha.cu
 int* device_flag_ptr();                 // device address of the sticky flag (current device)
 int num_sms();                          // SM count of the current device
 
@@ -50,7 +59,7 @@ __host__ __device__ __forceinline__ int64_t imax64(int64_t a, int64_t b) { retur
 enum ProfKind : int {
   PK_NF4 = 0, PK_DQ = 1, PK_INT8 = 2, PK_DEQ = 3, PK_FWD_PREP = 4, PK_FWD_T = 5, PK_FWD_MAIN = 6,
   PK_BWD_PREP = 7, PK_BWD_U = 8, PK_BWD_DB = 9, PK_BWD_DA = 10, PK_BWD_DX = 11, PK_FWD_SMALL = 12,
-  PK_COUNT = 13
+  PK_FWD_ADAPTER = 13, PK_COUNT = 14
 };
 
 // Counts the kernels a scope launches and, when profiling is on, brackets them with a
@@ -67,6 +76,7 @@ class ProfScope {
 };
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+inline int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
 
 inline bool aligned(const void* p, uintptr_t a) {
   return (reinterpret_cast<uintptr_t>(p) % a) == 0;

@@ -188,7 +188,6 @@ __global__ void block_scale_kernel(int fmt, const int8_t* __restrict__ qabsmax,
 
 static int small_grid(int64_t n) { return (int)imax64(1, imin64((n + 255) / 256, (int64_t)num_sms() * 8)); }
 
-static int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
 
 struct WsLayout {
   int64_t off[6];
@@ -323,6 +322,57 @@ static ql_status check_weight(const ql_weight* w) {
   return QL_OK;
 }
 
+// Y = X deq(W)^T + Zext Wext^T, with Zext [M, kext] and Wext [N, kext] bf16 row-major
+// (kext a multiple of 64, 0 for the base product alone): the fused GEMM of the forward,
+// its extension chunks taken from the caller's operands. M <= 16 with kext = 0 runs the
+// decode-shaped kernel without its adapter part. The only scratch is the block-scale copy.
+int64_t ext_fwd_ws_bytes(int64_t M, int64_t N, int64_t K, int64_t kext) {
+  if (kext == 0 && M <= kSmallMMax && small_m_supported(K, 0)) return 0;
+  return round_up((K / 64) * N * 4, 256);
+}
+
+ql_status ext_forward(const ql_weight* w, const uint16_t* X, int64_t M, const uint16_t* Zext,
+                      const uint16_t* Wext, int64_t kext, uint16_t* Y, void* ws, size_t ws_bytes,
+                      cudaStream_t st) {
+  ql_status e = check_weight(w);
+  if (e != QL_OK) return e;
+  if (!X || !Y || M < 1 || !aligned(X, 16) || !aligned(Y, 16)) return QL_ERR_INVALID_ARG;
+  if (kext < 0 || kext % 64 != 0 || (kext > 0 && (!Zext || !Wext || !aligned(Zext, 16) || !aligned(Wext, 16))))
+    return QL_ERR_INVALID_ARG;
+  if (M > (int64_t(1) << 31)) return QL_ERR_UNSUPPORTED;
+  const int64_t N = w->N, K = w->K;
+  if (kext == 0 && M <= kSmallMMax && small_m_supported(K, 0))
+    return small_m_forward(w, X, M, nullptr, nullptr, 0, 0.0f, Y, nullptr, st);
+  if (!ws || !aligned(ws, 256)) return QL_ERR_INVALID_ARG;
+  if ((int64_t)ws_bytes < ext_fwd_ws_bytes(M, N, K, kext)) return QL_ERR_WORKSPACE;
+  float* scales = static_cast<float*>(ws);
+  const bool pair = g_gemm_pair.load() != 0;
+  const uint32_t tbox = pair ? 128 : 256;
+  CUtensorMap mXt, mc, ms, mZt, mWe;
+  if (!make_map(&mXt, X, K, M, K, tbox) || !make_weight_maps(w, scales, false, &mc, &ms)) return QL_ERR_CUDA;
+  if (kext > 0) {
+    if (!make_map(&mZt, Zext, kext, M, kext, tbox) || !make_map(&mWe, Wext, kext, N, kext, 128)) return QL_ERR_CUDA;
+  } else {
+    mZt = mXt;                                      // never read with no extension chunks
+    mWe = mXt;
+  }
+  {
+    ProfScope prof(PK_FWD_PREP, st, 1);
+    e = launch_block_scales(w, false, scales, st);
+    if (e != QL_OK) return e;
+  }
+  GemmArgs y = base_args();
+  y.R = N; y.Cn = M; y.Kc = K; y.n_ext = (int32_t)(kext / 64); y.r = 0;
+  y.out = Y; y.ld_out = N; y.scale = 1.0f;
+  ProfScope prof(PK_FWD_MAIN, st, 1);
+  if (pair) {
+    if (w->fmt == QL_FMT_NF4_DQ) return launch_wpair<BSrc::NF4, false>(mXt, mc, ms, mZt, mWe, y, st);
+    return launch_wpair<BSrc::INT8, false>(mXt, mc, ms, mZt, mWe, y, st);
+  }
+  if (w->fmt == QL_FMT_NF4_DQ) return launch_wdec<BSrc::NF4, false>(mXt, mc, ms, mZt, mWe, y, st);
+  return launch_wdec<BSrc::INT8, false>(mXt, mc, ms, mZt, mWe, y, st);
+}
+
 }  // namespace qlb
 
 using namespace qlb;
@@ -331,6 +381,10 @@ extern "C" {
 
 size_t ql_workspace_bytes(int32_t op, int64_t M, int64_t N, int64_t K, int32_t r) {
   if (op == QL_OP_DQ) return 256;
+  if (op == QL_OP_FWD_QWHA) {
+    if (M < 1 || N < 1 || K < 64 || K % 64 != 0) return 0;
+    return (size_t)qwha_ws_bytes(M, N, K);
+  }
   if (op == QL_OP_FWD_LORDBA) {
     if (M < 0 || N < 0 || K < 0 || r < 1 || r > 256) return 0;
     return (size_t)lordba_ws_bytes(M, N, K, r);

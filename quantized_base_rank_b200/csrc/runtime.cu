@@ -184,6 +184,7 @@ ql_status ql_get_device_status(void* stream) {
   }
   if (v & qlb::kFlagTimeout) return QL_ERR_TIMEOUT;
   if (v & qlb::kFlagNonfinite) return QL_ERR_NONFINITE;
+  if (v & qlb::kFlagBadIndex) return QL_ERR_INVALID_ARG;
   return QL_OK;
 }
 

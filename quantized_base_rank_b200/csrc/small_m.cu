@@ -252,7 +252,7 @@ small_m_fwd_kernel(const SmallArgs a) {
     const uint32_t hi = j + 1 < a.r ? a.B[row * a.r + j + 1] : 0u;
     return lo | (hi << 16);
   };
-  uint32_t bfr[JT][4];
+  uint32_t bfr[JT > 0 ? JT : 1][4];                 // JT = 0: no adapter
 #pragma unroll
   for (int jt = 0; jt < JT; ++jt) {
     const int j0 = jt * 16 + 2 * q;
@@ -312,7 +312,7 @@ small_m_fwd_kernel(const SmallArgs a) {
 
   // ---- main loop: W' rows (decoded) and, for the adapter, A rows against the tokens ----
   float d[NTT][4];
-  float dt[JT][NTT][4];                              // T_kr = X_kr A_kr^T, per j-tile
+  float dt[JT > 0 ? JT : 1][NTT][4];                 // T_kr = X_kr A_kr^T, per j-tile
 #pragma unroll
   for (int t = 0; t < NTT; ++t) {
     d[t][0] = d[t][1] = d[t][2] = d[t][3] = 0.0f;
@@ -488,7 +488,7 @@ static ql_status launch_small(const SmallArgs& a, cudaStream_t st) {
 }
 
 bool small_m_supported(int64_t K, int r) {
-  if (r < 1 || r > 64) return false;
+  if (r < 0 || r > 64) return false;
   const int64_t U = (K + 255) / 256;
   const int units_max = (int)((U + kCS - 1) / kCS);
   return small_m_smem(16, units_max, r) <= 200 * 1024;
@@ -499,7 +499,7 @@ ql_status small_m_forward(const ql_weight* w, const uint16_t* X, int64_t M, cons
                           const uint16_t* B, int r, float alpha, uint16_t* Y, uint16_t* T_save,
                           cudaStream_t st) {
   SmallArgs a{};
-  a.X = X; a.A = A; a.B = B; a.M = M; a.N = w->N; a.K = w->K; a.r = r; a.s = alpha / (float)r;
+  a.X = X; a.A = A; a.B = B; a.M = M; a.N = w->N; a.K = w->K; a.r = r; a.s = r > 0 ? alpha / (float)r : 0.0f;
   a.fmt = w->fmt;
   a.codes = static_cast<const uint8_t*>(w->codes);
   a.qabsmax = w->qabsmax; a.gscale = w->group_scale; a.mean = w->mean; a.absmax = w->absmax;
@@ -510,9 +510,13 @@ ql_status small_m_forward(const ql_weight* w, const uint16_t* X, int64_t M, cons
   const Nf4Tables& t = nf4_tables();
   for (int i = 0; i < 16; ++i) a.q[i] = t.q[i];
   ProfScope prof(PK_FWD_SMALL, st, 1);
-  if (r > 64) return QL_ERR_UNSUPPORTED;
+  if (r < 0 || r > 64) return QL_ERR_UNSUPPORTED;
   const int jt = (r + 15) / 16;
   const bool nf4 = w->fmt == QL_FMT_NF4_DQ;
+  if (jt == 0) {                                   // no adapter: the base product alone
+    if (M <= 8) return nf4 ? launch_small<8, QL_FMT_NF4_DQ, 0>(a, st) : launch_small<8, QL_FMT_INT8_B64, 0>(a, st);
+    return nf4 ? launch_small<16, QL_FMT_NF4_DQ, 0>(a, st) : launch_small<16, QL_FMT_INT8_B64, 0>(a, st);
+  }
   if (M <= 8) {
     if (nf4) return jt == 1 ? launch_small<8, QL_FMT_NF4_DQ, 1>(a, st) : jt == 2 ? launch_small<8, QL_FMT_NF4_DQ, 2>(a, st)
                                                                               : launch_small<8, QL_FMT_NF4_DQ, 4>(a, st);

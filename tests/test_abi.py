@@ -66,6 +66,23 @@ def test_argument_validation_without_a_device(lib):
     ad = B.QLLordba(100, 3, 16, 16, 16, 16, 16)
     assert lib.qlora_linear_fwd_lordba(ctypes.byref(w), 16, 1, ctypes.addressof(ad), 16, 256, 1 << 20,
                                        None) == B.QL_ERR_UNSUPPORTED
+    # Walsh-Hadamard adapter: missing or inconsistent index arrays, oversize K
+    assert lib.qlora_linear_fwd_qwha(ctypes.byref(w), 16, 1, None, 16, 256, 1 << 20, None) == B.QL_ERR_INVALID_ARG
+    for ad in (B.QLQwha(None, 16, 16, 4), B.QLQwha(16, None, 16, 4), B.QLQwha(16, 16, 16, -1),
+               B.QLQwha(18, 16, 16, 4), B.QLQwha(16, 17, 16, 4)):
+        assert lib.qlora_linear_fwd_qwha(ctypes.byref(w), 16, 1, ctypes.addressof(ad), 16, 256, 1 << 20,
+                                         None) == B.QL_ERR_INVALID_ARG
+    ad = B.QLQwha(16, 16, 16, 4)
+    assert lib.qlora_linear_fwd_qwha(ctypes.byref(w), 16, 1, ctypes.addressof(ad), 16, None, 1 << 20,
+                                     None) == B.QL_ERR_INVALID_ARG
+    assert lib.qlora_linear_fwd_qwha(ctypes.byref(w), 16, 1, ctypes.addressof(ad), 16, 256, 16,
+                                     None) == B.QL_ERR_WORKSPACE
+    wk = B.QLWeight(0, 0, 64, 65600, 16, 0, 16, 16, 16)
+    assert lib.qlora_linear_fwd_qwha(ctypes.byref(wk), 16, 1, ctypes.addressof(ad), 16, 256, 1 << 30,
+                                     None) == B.QL_ERR_UNSUPPORTED
+    assert lib.ql_wht(None, 1, 64, 16, None) == B.QL_ERR_INVALID_ARG
+    assert lib.ql_wht(16, 1, 100, 16, None) == B.QL_ERR_UNSUPPORTED
+    assert lib.ql_wht(24, 1, 64, 16, None) == B.QL_ERR_INVALID_ARG
     assert lib.ql_dequantize(None, None, None) == B.QL_ERR_INVALID_ARG
     w = B.QLWeight(0, 0, 64, 64, 16, 0, 16, 16, 16)
     # misaligned or null pointers, bad shapes: all rejected synchronously
@@ -75,3 +92,10 @@ def test_argument_validation_without_a_device(lib):
 
 def test_workspace_query(lib):
     assert B.workspace_bytes(B.QL_OP_DQ, 0, 0, 0, 0) >= 128
+    # Walsh-Hadamard adapter: decode-shaped, one slab of Z (16 tokens); otherwise Z [M, K],
+    # the dense F [N, K] and the fused GEMM's block scales
+    assert B.workspace_bytes(B.QL_OP_FWD_QWHA, 1, 4096, 4096, 0) == 4096 * 16 * 2
+    assert B.workspace_bytes(B.QL_OP_FWD_QWHA, 8192, 11008, 4096, 0) == \
+        8192 * 4096 * 2 + 11008 * 4096 * 2 + 64 * 11008 * 4
+    assert B.workspace_bytes(B.QL_OP_FWD_QWHA, 17, 64, 192, 0) == 6656 + 64 * 192 * 2 + 3 * 64 * 4
+    assert B.workspace_bytes(B.QL_OP_FWD_QWHA, 1, 64, 100, 0) == 0

@@ -554,6 +554,17 @@ def test_qwha_linear_as_sparse_gather_of_the_transformed_input():
             for j in range(row_ptr[n], row_ptr[n + 1]):
                 y += c[j] * z[col[j]]
             assert math.isclose(Y[t, n], y, rel_tol=1e-11, abs_tol=1e-11)
+    # the factored form (block transform, then the sparse product) is the same Y
+    np.testing.assert_allclose(o.qwha_linear_fwd_factored(X, Wd, row_ptr, col, c), Y, rtol=1e-12, atol=1e-12)
+
+
+def test_qwha_block_transform_equals_full_matrix():
+    """The transform taken one diagonal block at a time equals the product with the full
+    K x K matrix, for a width with 7 blocks."""
+    rng = np.random.default_rng(2)
+    X = rng.standard_normal((3, 448))
+    np.testing.assert_allclose(o.qwha_transform(X), X @ np.linalg.inv(o.walsh_hadamard(448)).T,
+                               rtol=0, atol=1e-12)
 
 
 def test_qwha_zero_and_linear_in_c():
