@@ -15,6 +15,7 @@ Rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -336,6 +337,101 @@ def lordba_bench(dev, peaks, qw_up, X_up, reps: int = 10):
     return out
 
 
+def qwha_bench(dev, peaks, qw_up, X_up, reps: int = 10):
+    """The Walsh-Hadamard adapter (Delta W = F H^{-1}, sparse F): (1) the up-projection
+    forward at 8192 tokens with a budget of a rank-64 LoRA (64 (N + K) values), beside the
+    dense rank-64 forward timed the same way, and the transform kernel alone; (2) the
+    decode-shaped 4096x4096 NF4+DQ layer at M = 1 with a rank-16 budget, timed like the
+    dense decode component (a CUDA graph over weight copies exceeding 3x L2), beside the
+    dense rank-16 adapter timed the same way."""
+    from quantized_base_rank_b200 import binding as B
+    from quantized_base_rank_b200 import synth
+    out = {}
+    N, K = qw_up.N, qw_up.K
+    M = X_up.shape[0]
+    ad = synth.qwha_inputs(N, K, 64, 5)
+    rp, col, c = ad["row_ptr"].to(dev), ad["col"].to(dev), ad["c"].to(dev)
+    nnz = c.numel()
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    A_d = synth.normal_bf16((64, K), 0.02, 7, 0).to(dev)
+    B_d = synth.normal_bf16((N, 64), 0.02, 7, 1).to(dev)
+    Z = torch.empty_like(X_up)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def timed(call, n=reps):
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(n):
+            call()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    ms_dense = timed(lambda: B.linear_fwd(qw_up, X_up, A_d, B_d, 64.0, save_T=False, Y=Y))
+    ms = timed(lambda: B.linear_fwd_qwha(qw_up, X_up, rp, col, c, Y=Y))
+    ms_wht = timed(lambda: B.wht(X_up, Z))
+    wht_bytes = 2 * M * K * 2
+    useful = 2 * M * N * K + 2 * M * nnz
+    out["upproj_r64_budget"] = {
+        "ms": ms, "TFLOP/s_useful": useful / (ms * 1e-3) / 1e12, "dense_lora_r64_ms": ms_dense, "nnz": nnz,
+        "adapter_bytes": nnz * 4 + (N + 1) * 4, "dense_lora_bytes": 2 * 64 * (N + K),
+        "wht_us": ms_wht * 1e3, "wht_GB/s": wht_bytes / (ms_wht * 1e-3) / 1e9,
+        "wht_frac_hbm": wht_bytes / (ms_wht * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    del Y, Z
+    # decode-shaped
+    base = synth.CFG2[0]
+    W = synth.weight_with_outliers(base.N, base.K, base.w_std, base.outlier_frac, base.outlier_mult,
+                                   base.seed).to(dev)
+    q0 = B.quantize_weight(W, "nf4_dq")
+    del W
+    n = base.N * base.K
+    ad = synth.qwha_inputs(base.N, base.K, 16, 6)
+    rp, col, c = ad["row_ptr"].to(dev), ad["col"].to(dev), ad["c"].to(dev)
+    nnz = c.numel()
+    A16 = synth.normal_bf16((16, base.K), 0.02, 8, 0).to(dev)
+    B16 = synth.normal_bf16((base.N, 16), 0.02, 8, 1).to(dev)
+    wbytes = n * (0.5 + 1.0 / 64) + 4.0 * n / 16384
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    copies = max(4, int(np.ceil(3 * l2 / wbytes)))
+    qws = [B.QuantWeight("nf4_dq", base.N, base.K, q0.codes.clone(), None, q0.qabsmax.clone(),
+                         q0.group_scale.clone(), q0.mean.clone()) for _ in range(copies)]
+    X = synth.normal_bf16((1, base.K), 1.0, 5, 0).to(dev)
+    Y = torch.empty((1, base.N), dtype=torch.bfloat16, device=dev)
+
+    def graph_us(call):
+        for qw in qws[:2]:
+            call(qw)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        st = torch.cuda.Stream(dev)
+        st.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(st):
+            with torch.cuda.graph(g, stream=st):
+                for qw in qws:
+                    call(qw)
+        torch.cuda.synchronize()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(2 * reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        del g
+        return e0.elapsed_time(e1) * 1e3 / (2 * reps * copies)
+
+    us = graph_us(lambda qw: B.linear_fwd_qwha(qw, X, rp, col, c, Y=Y))
+    us_lora = graph_us(lambda qw: B.linear_fwd(qw, X, A16, B16, 32.0, save_T=False, Y=Y))
+    nbytes = wbytes + 2 * base.K + nnz * 4 + (base.N + 1) * 4 + 2 * base.N
+    out["decode_7b_4096x4096_M1_r16_budget"] = {
+        "us_per_call": us, "dense_lora_r16_us": us_lora, "nnz": nnz, "bytes": nbytes,
+        "GB/s": nbytes / (us * 1e-6) / 1e9, "frac_hbm": nbytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"]}
+    return out
+
+
 def run_ours(args, case, world, rank, local_rank):
     from quantized_base_rank_b200 import binding as B
     from quantized_base_rank_b200 import dp, synth
@@ -474,6 +570,9 @@ def run_ours(args, case, world, rank, local_rank):
     # ---- LoRDBA double-binary adapter branch ----
     lordba = lordba_bench(dev, peaks, qw, X)
 
+    # ---- Walsh-Hadamard (QWHA) adapter ----
+    qwha = qwha_bench(dev, peaks, qw, X)
+
     # ---- CPU oracle baseline (rank 0, one GPU only) ----
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -513,6 +612,7 @@ def run_ours(args, case, world, rank, local_rank):
             "per_group_ms": {g: avg(g) for g in B.PROFILE_GROUPS if prof[g][1]},
             "decode_7b_4096x4096_nf4": decode,
             "lordba": lordba,
+            "qwha": qwha,
         },
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
@@ -532,8 +632,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--gemm", choices=["pair", "single"], default="single",
                     help="fused weight GEMM on CTA pairs (cta_group::2) or on single CTAs")
-    ap.add_argument("--part", choices=["all", "decode"], default="all",
-                    help="decode: only the decode-shaped forward component (a short run for profiling)")
+    ap.add_argument("--part", choices=["all", "decode", "qwha"], default="all",
+                    help="decode / qwha: only that component (a short run for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -557,6 +657,16 @@ def main():
         out = decode_bench(dev, load_peaks(), reps=args.steps)
         if rank == 0:
             print(json.dumps({"part": "decode", "decode_7b_4096x4096_nf4": out}), flush=True)
+        return
+    if args.part == "qwha":
+        from quantized_base_rank_b200 import binding as B
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        inp = synth.make_inputs(dataclasses.replace(case, backward=False))
+        qw = B.quantize_weight(inp["W"].to(dev), "nf4_dq")
+        out = qwha_bench(dev, load_peaks(), qw, inp["X"].to(dev), reps=args.steps)
+        if rank == 0:
+            print(json.dumps({"part": "qwha", "qwha": out}), flush=True)
         return
     try:
         run_ours(args, case, world, rank, local_rank)

@@ -243,12 +243,16 @@ typedef struct {
  *   Z = X H^{-T} = X H  (H^{-1} x per token), computed in fp32 by the add/subtract
  *   recursion and rounded once to bf16; the sparse sums accumulate in fp32.
  * Shapes and formats as qlora_linear_fwd (K a multiple of 64, K <= 65536, N a multiple
- * of 8). The base product takes the same kernels as qlora_linear_fwd without a LoRA
- * branch. Column indices >= K and row offsets outside [0, nnz] are skipped on the
+ * of 8); the Walsh-Hadamard block (the largest power of two dividing K) is at most
+ * 16384, else QL_ERR_UNSUPPORTED. M <= 16: the base product of the decode-shaped kernel,
+ * then the transform and a sparse product that gathers Z by column index; M > 16: F is
+ * written out as a dense bf16 [N, K] and Z F^T runs on the tensor cores as K/64
+ * extension chunks of the same fused GEMM as qlora_linear_fwd. Column indices >= K and row offsets outside [0, nnz] are skipped on the
  * device and reported as QL_ERR_INVALID_ARG by ql_get_device_status; the contents of
  * the index arrays are not read on the host.
- * ws: ql_workspace_bytes(QL_OP_FWD_QWHA, M, N, K, 0) bytes, 256-byte aligned (it holds
- * Z in slabs of 16 tokens, [ceil(M/16)][K][16] bf16, and the base product's scratch). */
+ * ws: ql_workspace_bytes(QL_OP_FWD_QWHA, M, N, K, 0) bytes, 256-byte aligned (M <= 16:
+ * one slab of Z, [K][16] bf16; otherwise Z [M, K], the dense F [N, K] and the GEMM's
+ * block scales). */
 ql_status qlora_linear_fwd_qwha(const ql_weight* w, const ql_bf16* X, int64_t M,
                                 const ql_qwha* adapter, ql_bf16* Y, void* ws,
                                 size_t ws_bytes, void* stream);
@@ -256,7 +260,7 @@ ql_status qlora_linear_fwd_qwha(const ql_weight* w, const ql_bf16* X, int64_t M,
 /* The Walsh-Hadamard transform of each token row alone: Z [M, K] bf16 = bf16(X H^{-T})
  * with the H of ql_qwha (orthonormal, blockwise for K not a power of two), by the
  * add/subtract recursion in fp32 (QWHA page, section 2.1, the fast WHT kernel).
- * X and Z are 16-byte aligned, K a multiple of 64. */
+ * X and Z are 16-byte aligned, K a multiple of 64, the block at most 16384. */
 ql_status ql_wht(const ql_bf16* X, int64_t M, int64_t K, ql_bf16* Z, void* stream);
 
 enum { QL_OP_DQ = 0, QL_OP_FWD = 1, QL_OP_BWD = 2, QL_OP_FWD_LORDBA = 3, QL_OP_FWD_QWHA = 4 };

@@ -53,13 +53,24 @@ __device__ __forceinline__ void butterflies(float* v) {
 __device__ __forceinline__ int phys(int e) { return e + (e >> 4); }
 __host__ __device__ __forceinline__ int qwha_pitch(int b) { return b + (b >> 4) + 4; }
 
-// One pass over the index bits [lo, lo + NB) of every length-b row held in shared memory
+// Where element e of the transformed row of token m lands in global memory: row-major
+// Z [M][K], or the token slabs Zs[m / 16][k][m % 16].
+template <bool SLAB>
+__device__ __forceinline__ size_t z_index(int64_t m, int64_t k, int64_t K) {
+  return SLAB ? (size_t)(((m / kQwSlab) * K + k) * kQwSlab + (m % kQwSlab)) : (size_t)(m * K + k);
+}
+
+// One pass over the index bits [lo, lo + NB) of every length-bs row held in shared memory
 // (rows of `pitch` floats, TT rows). A group is the 2^NB elements that differ only in
 // those bits; consecutive threads take groups with consecutive low bits, so a warp's
-// accesses to one element of its groups are consecutive words.
-template <int NB>
-__device__ __forceinline__ void smem_pass(float* sm, int TT, int b, int pitch, int lo) {
-  const int per_row = b >> NB;                   // groups per row
+// accesses to one element of its groups are consecutive words. FINAL: the pass that
+// completes the transform writes its results (times `scale`, rounded to bf16) straight
+// to global memory instead of back to shared memory; a warp's 32 stores of one element
+// index are then 32 consecutive columns.
+template <int NB, bool FINAL, bool SLAB>
+__device__ __forceinline__ void smem_pass(float* sm, int TT, int bs, int pitch, int lo, float scale,
+                                          uint16_t* Z, int64_t m0, int64_t M, int64_t K, int64_t kbase) {
+  const int per_row = bs >> NB;                  // groups per row
   const int total = TT * per_row;
   const int low_mask = (1 << lo) - 1;
   for (int gi = threadIdx.x; gi < total; gi += blockDim.x) {
@@ -70,201 +81,225 @@ __device__ __forceinline__ void smem_pass(float* sm, int TT, int b, int pitch, i
 #pragma unroll
     for (int j = 0; j < (1 << NB); ++j) v[j] = row[phys(base + (j << lo))];
     butterflies<NB>(v);
+    if (FINAL) {
+      const int64_t m = m0 + t;
+      if (m < M) {
 #pragma unroll
-    for (int j = 0; j < (1 << NB); ++j) row[phys(base + (j << lo))] = v[j];
+        for (int j = 0; j < (1 << NB); ++j)
+          Z[z_index<SLAB>(m, kbase + base + (j << lo), K)] = float_to_bf16_bits(v[j] * scale);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < (1 << NB); ++j) row[phys(base + (j << lo))] = v[j];
+    }
   }
 }
 
-// Z = X H for TT tokens [m0, m0 + TT) and one Walsh-Hadamard block [bi*b, bi*b + b) of the
-// input width. L = log2(b) >= 6 (K is a multiple of 64). Tokens at or past M read as zero,
-// so a slab's tail is written as zeros. SLAB: Zs[m / 16][k][m % 16]; otherwise Z [M][K].
+template <bool FINAL, bool SLAB>
+__device__ __forceinline__ void smem_pass_n(int nb, float* sm, int TT, int bs, int pitch, int lo, float scale,
+                                            uint16_t* Z, int64_t m0, int64_t M, int64_t K, int64_t kbase) {
+  switch (nb) {
+    case 4: smem_pass<4, FINAL, SLAB>(sm, TT, bs, pitch, lo, scale, Z, m0, M, K, kbase); break;
+    case 3: smem_pass<3, FINAL, SLAB>(sm, TT, bs, pitch, lo, scale, Z, m0, M, K, kbase); break;
+    case 2: smem_pass<2, FINAL, SLAB>(sm, TT, bs, pitch, lo, scale, Z, m0, M, K, kbase); break;
+    default: smem_pass<1, FINAL, SLAB>(sm, TT, bs, pitch, lo, scale, Z, m0, M, K, kbase); break;
+  }
+}
+
+// Z = X H for TT tokens [m0, m0 + TT) and one slice of one Walsh-Hadamard block of the
+// input width: block blockIdx.y >> SL (b = 2^L elements), slice j = blockIdx.y & (2^SL - 1)
+// of its outputs (bs = b / 2^SL consecutive columns). Sylvester's matrix factors as
+// H_b = H_{2^SL} (x) H_bs, so slice j is H_bs applied to u_j = sum_r (-1)^popcount(j & r)
+// x[r * bs ...]: the 2^SL input slices combined with signs, then a transform of length bs
+// (2^SL CTAs share one token's block; SL = 0 is the plain transform). log2(bs) >= 5.
+// Tokens at or past M read as zero and are not written.
 template <bool SLAB>
 __global__ void __launch_bounds__(256)
-qwha_wht_kernel(const uint16_t* __restrict__ X, int64_t M, int64_t K, int L, int TT, float scale,
+qwha_wht_kernel(const uint16_t* __restrict__ X, int64_t M, int64_t K, int L, int SL, int TT, float scale,
                 uint16_t* __restrict__ Z) {
   extern __shared__ __align__(16) float wsm[];
+  const int Ls = L - SL, bs = 1 << Ls;
   const int b = 1 << L;
-  const int pitch = qwha_pitch(b);
+  const int pitch = qwha_pitch(bs);
   const int64_t m0 = (int64_t)blockIdx.x * TT;
-  const int64_t k0 = (int64_t)blockIdx.y * b;
-
-  // pass 0: 16 contiguous elements per thread from global, bits 0..3 in registers
+  const int j = (int)(blockIdx.y & ((1u << SL) - 1));
+  const int64_t kblk = (int64_t)(blockIdx.y >> SL) << L;
+  const int S = 1 << SL;
+  // the raw bf16 input tile [TT][b] sits after the fp32 rows; every thread issues all of
+  // its 16-byte copies before any is waited for (tokens past M are zero-filled)
+  uint16_t* raw = reinterpret_cast<uint16_t*>(wsm + (size_t)TT * pitch);
   {
-    const int per_row = b >> 4;
+    const int per_row = b >> 3;
     for (int gi = threadIdx.x; gi < TT * per_row; gi += blockDim.x) {
-      const int t = gi / per_row, e0 = (gi - t * per_row) << 4;
+      const int t = gi / per_row, e = (gi - t * per_row) << 3;
       const int64_t m = m0 + t;
-      uint4 u0 = make_uint4(0u, 0u, 0u, 0u), u1 = u0;
-      if (m < M) {
-        const uint4* src = reinterpret_cast<const uint4*>(X + m * K + k0 + e0);
-        u0 = __ldg(src);
-        u1 = __ldg(src + 1);
-      }
-      float v[16] = {bf16_lo(u0.x), bf16_hi(u0.x), bf16_lo(u0.y), bf16_hi(u0.y),
-                     bf16_lo(u0.z), bf16_hi(u0.z), bf16_lo(u0.w), bf16_hi(u0.w),
-                     bf16_lo(u1.x), bf16_hi(u1.x), bf16_lo(u1.y), bf16_hi(u1.y),
-                     bf16_lo(u1.z), bf16_hi(u1.z), bf16_lo(u1.w), bf16_hi(u1.w)};
-      butterflies<4>(v);
-      float* dst = wsm + (size_t)t * pitch + phys(e0);
-#pragma unroll
-      for (int j = 0; j < 16; ++j) dst[j] = v[j];
+      const uint16_t* src = m < M ? X + m * K + kblk + e : X;
+      const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(raw + (size_t)t * b + e));
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(dst), "l"(src), "r"(m < M ? 16 : 0)
+                   : "memory");
     }
-  }
-  __syncthreads();
-  // the remaining bits, up to four per pass
-  for (int lo = 4; lo < L; lo += 4) {
-    switch (L - lo >= 4 ? 4 : L - lo) {
-      case 4: smem_pass<4>(wsm, TT, b, pitch, lo); break;
-      case 3: smem_pass<3>(wsm, TT, b, pitch, lo); break;
-      case 2: smem_pass<2>(wsm, TT, b, pitch, lo); break;
-      default: smem_pass<1>(wsm, TT, b, pitch, lo); break;
-    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
   }
 
-  if (SLAB) {
-    // one column k per thread: the TT tokens' values, contiguous in the slab
-    const int64_t slab = m0 / kQwSlab;
-    const int t0 = (int)(m0 % kQwSlab);
-    for (int k = threadIdx.x; k < b; k += blockDim.x) {
-      uint32_t w[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float a = 2 * i < TT ? wsm[(size_t)(2 * i) * pitch + phys(k)] * scale : 0.0f;
-        const float c = 2 * i + 1 < TT ? wsm[(size_t)(2 * i + 1) * pitch + phys(k)] * scale : 0.0f;
-        w[i] = f2_to_bf16x2(a, c);
-      }
-      uint16_t* dst = Z + ((slab * K + k0 + k) * kQwSlab + t0);
-      if (TT == 16) {
-        reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
-        reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
-      } else if (TT == 8) {
-        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-      } else if (TT == 4) {
-        *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
-      } else if (TT == 2) {
-        *reinterpret_cast<uint32_t*>(dst) = w[0];
-      } else {
-        *dst = (uint16_t)(w[0] & 0xFFFFu);
-      }
-    }
-  } else {
-    // eight consecutive k of one token per thread
-    const int per_row = b >> 3;
+  // pass 0: 16 contiguous elements of u per thread, bits 0..3 in registers
+  {
+    const int per_row = bs >> 4;
     for (int gi = threadIdx.x; gi < TT * per_row; gi += blockDim.x) {
-      const int t = gi / per_row, e0 = (gi - t * per_row) << 3;
-      const int64_t m = m0 + t;
-      if (m >= M) continue;
-      const float* src = wsm + (size_t)t * pitch + phys(e0);   // e0 % 8 == 0: no gap inside
-      const uint4 o = make_uint4(f2_to_bf16x2(src[0] * scale, src[1] * scale),
-                                 f2_to_bf16x2(src[2] * scale, src[3] * scale),
-                                 f2_to_bf16x2(src[4] * scale, src[5] * scale),
-                                 f2_to_bf16x2(src[6] * scale, src[7] * scale));
-      *reinterpret_cast<uint4*>(Z + m * K + k0 + e0) = o;
+      const int t = gi / per_row, e0 = (gi - t * per_row) << 4;
+      float v[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] = 0.0f;
+      {
+        for (int r = 0; r < S; ++r) {
+          const uint4* src = reinterpret_cast<const uint4*>(raw + (size_t)t * b + r * bs + e0);
+          const uint4 u0 = src[0], u1 = src[1];
+          const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+          if (__popc(j & r) & 1) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              v[2 * i] -= bf16_lo(w[i]);
+              v[2 * i + 1] -= bf16_hi(w[i]);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              v[2 * i] += bf16_lo(w[i]);
+              v[2 * i + 1] += bf16_hi(w[i]);
+            }
+          }
+        }
+      }
+      butterflies<4>(v);
+      float* dst = wsm + (size_t)t * pitch + phys(e0);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) dst[i] = v[i];
+    }
+  }
+  __syncthreads();
+  // the remaining bits of the slice, up to four per pass; the last pass stores to global
+  const int64_t kbase = kblk + (int64_t)j * bs;
+  for (int lo = 4; lo < Ls; lo += 4) {
+    const int nb = Ls - lo >= 4 ? 4 : Ls - lo;
+    if (lo + nb < Ls) {
+      smem_pass_n<false, SLAB>(nb, wsm, TT, bs, pitch, lo, scale, Z, m0, M, K, kbase);
+      __syncthreads();
+    } else {
+      smem_pass_n<true, SLAB>(nb, wsm, TT, bs, pitch, lo, scale, Z, m0, M, K, kbase);
     }
   }
 }
 
-// Decode-shaped sparse product (M <= 16, one slab):
+// Decode-shaped sparse product (M <= 16, one slab of Z):
 //   Y[m, n] += sum_j c_j Z[m, col_j], j over row n's stored values.
-// A warp takes 8 consecutive rows (N is a multiple of 8). Each row's values are read 32 at
-// a time, one (col, c) pair per lane, and handed out by shuffles: lane = (stream
-// s = lane / 8, token pair tp = lane % 8), stream s takes values s, s + 4, ... of the
-// chunk, so each chunk issues 8 independent 4-byte gathers of Z per lane. Each lane keeps
-// two tokens' fp32 sums per row; the streams are combined by a fixed xor butterfly (the
-// result does not depend on scheduling) and the sum is added to the base product with
-// one bf16 rounding. Columns at or past K, or row offsets outside [0, nnz], are skipped
-// and raise the device's bad-index flag.
+// One warp per row. Lane = (stream, token pair tp): TP = ceil(M / 2) token pairs and
+// 32 / TP streams, so at M <= 2 every lane takes its own value. A row's values are read
+// 32 per chunk and four chunks at a time (one (col, c) pair per lane and chunk, all four
+// loads issued together), handed to the streams by shuffles; each lane gathers the two
+// tokens' Z values of its value (one 4-byte load) and keeps their fp32 sums. The streams
+// are combined by a fixed xor butterfly (the result does not depend on scheduling) and
+// added to the base product with one bf16 rounding. Columns at or past K, or row offsets
+// outside [0, nnz], are skipped and raise the device's bad-index flag.
+template <int TP>
 __global__ void __launch_bounds__(256)
 qwha_spmm_kernel(const uint16_t* __restrict__ Zs, int64_t M, int64_t N, int64_t K,
                  const int32_t* __restrict__ row_ptr, const uint16_t* __restrict__ col,
                  const uint16_t* __restrict__ cval, int64_t nnz, uint16_t* __restrict__ Y, int* flag) {
-  const int64_t slab = blockIdx.y;
-  const uint16_t* zsrc = Zs + slab * K * kQwSlab;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int s = lane >> 3, tp = lane & 7;
-  const int64_t rg = (int64_t)blockIdx.x * 64 + warp * 8;
-  if (rg >= N) return;                               // whole warp: its 8 rows are all outside
+  constexpr int NS = 32 / TP;                        // streams
+  constexpr int U = 4;                               // chunks in flight
+  const int lane = threadIdx.x & 31;
+  const int stream = lane / TP, tp = lane % TP;
+  const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   bool bad = false;
-  int off = 0;                                       // lanes 0..8: the 9 row offsets
-  if (lane < 9) off = __ldg(row_ptr + rg + lane);
-  float acc[8][2];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    acc[i][0] = acc[i][1] = 0.0f;
-    int j0 = __shfl_sync(0xffffffffu, off, i), j1 = __shfl_sync(0xffffffffu, off, i + 1);
+  for (int64_t n = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; n < N; n += warps) {
+    int j0 = __ldg(row_ptr + n), j1 = __ldg(row_ptr + n + 1);
     if (j0 < 0 || (int64_t)j1 > nnz || j0 > j1) {
       bad = true;
       j0 = j1 = 0;
     }
-    for (int jc = j0; jc < j1; jc += 32) {
-      uint32_t wv = 0u;                              // col | c << 16; 0 adds nothing
-      if (jc + lane < j1) wv = (uint32_t)__ldg(col + jc + lane) | ((uint32_t)__ldg(cval + jc + lane) << 16);
-      if ((int64_t)(wv & 0xFFFFu) >= K) {
-        bad = true;
-        wv = 0u;
+    float a0 = 0.0f, a1 = 0.0f;
+    for (int jc = j0; jc < j1; jc += 32 * U) {
+      const int nch = (j1 - jc + 31) >> 5;           // chunks of this batch that hold values
+      uint32_t wv[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int jj = jc + 32 * u + lane;
+        wv[u] = jj < j1 ? (uint32_t)__ldg(col + jj) | ((uint32_t)__ldg(cval + jj) << 16) : 0u;
+        if ((int64_t)(wv[u] & 0xFFFFu) >= K) {
+          bad = true;
+          wv[u] = 0u;
+        }
       }
 #pragma unroll
-      for (int it = 0; it < 8; ++it) {
-        const uint32_t we = __shfl_sync(0xffffffffu, wv, 4 * it + s);
-        const uint32_t z = __ldg(reinterpret_cast<const uint32_t*>(zsrc + (size_t)(we & 0xFFFFu) * kQwSlab) + tp);
-        const float cv = __uint_as_float(we & 0xFFFF0000u);
-        acc[i][0] = fmaf(cv, bf16_lo(z), acc[i][0]);
-        acc[i][1] = fmaf(cv, bf16_hi(z), acc[i][1]);
+      for (int u = 0; u < U; ++u) {
+        if (u >= nch) break;                         // warp-uniform
+#pragma unroll
+        for (int it = 0; it < TP; ++it) {
+          const uint32_t we = __shfl_sync(0xffffffffu, wv[u], it * NS + stream);
+          const uint32_t z = __ldg(reinterpret_cast<const uint32_t*>(Zs + (size_t)(we & 0xFFFFu) * kQwSlab) + tp);
+          const float cv = __uint_as_float(we & 0xFFFF0000u);
+          a0 = fmaf(cv, bf16_lo(z), a0);
+          a1 = fmaf(cv, bf16_hi(z), a1);
+        }
       }
     }
-  }
-  // combine the four streams (lanes tp, tp + 8, tp + 16, tp + 24)
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      acc[i][e] += __shfl_xor_sync(0xffffffffu, acc[i][e], 8);
-      acc[i][e] += __shfl_xor_sync(0xffffffffu, acc[i][e], 16);
+    for (int off = TP; off < 32; off <<= 1) {
+      a0 += __shfl_xor_sync(0xffffffffu, a0, off);
+      a1 += __shfl_xor_sync(0xffffffffu, a1, off);
     }
-  }
-  // stream 0 adds token 2tp, stream 1 token 2tp + 1 into the base product (8 rows = 16 B)
-  if (s < 2) {
-    const int64_t m = slab * kQwSlab + 2 * tp + s;
-    if (m < M) {
-      uint4* py = reinterpret_cast<uint4*>(Y + m * N + rg);
-      const uint4 y = *py;
-      const uint32_t yw[4] = {y.x, y.y, y.z, y.w};
-      uint32_t o[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        o[q] = f2_to_bf16x2(bf16_lo(yw[q]) + (s ? acc[2 * q][1] : acc[2 * q][0]),
-                            bf16_hi(yw[q]) + (s ? acc[2 * q + 1][1] : acc[2 * q + 1][0]));
-      *py = make_uint4(o[0], o[1], o[2], o[3]);
+    if (stream == 0) {
+      const int64_t m = 2 * tp;
+      if (m < M) Y[m * N + n] = float_to_bf16_bits(bf16_lo(Y[m * N + n]) + a0);
+      if (m + 1 < M) Y[(m + 1) * N + n] = float_to_bf16_bits(bf16_lo(Y[(m + 1) * N + n]) + a1);
     }
   }
   if (bad) raise_flag(flag, kFlagBadIndex);
 }
 
-// F written out densely for the tensor cores: Fd [N, K] bf16 (zeroed beforehand) gets c_j
-// at (n, col_j). One warp per row; the same index checks as the sparse product.
+// F written out densely for the tensor cores: Fd [N, K] bf16 holds c_j at (n, col_j) and
+// zero elsewhere. A CTA builds `rows` (<= 64) consecutive rows in shared memory: zero,
+// then all its threads scatter the rows' values together (the values of the CTA's rows
+// are one contiguous range, so a long row is spread over every thread), then the rows go
+// out once with 16-byte stores. The same index checks as the sparse product.
 __global__ void __launch_bounds__(256)
 qwha_densify_kernel(const int32_t* __restrict__ row_ptr, const uint16_t* __restrict__ col,
-                    const uint16_t* __restrict__ cval, int64_t nnz, int64_t N, int64_t K,
+                    const uint16_t* __restrict__ cval, int64_t nnz, int64_t N, int64_t K, int rows,
                     uint16_t* __restrict__ Fd, int* flag) {
-  const int lane = threadIdx.x & 31;
-  const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  extern __shared__ __align__(16) uint16_t drow[];
+  __shared__ int s_off[65];
+  const int64_t n0 = (int64_t)blockIdx.x * rows;
+  const int nr = (int)imin64(rows, N - n0);
+  const int64_t n16 = (int64_t)nr * K / 8;             // 16-byte words (K % 64 == 0)
+  uint4* d4 = reinterpret_cast<uint4*>(drow);
+  for (int64_t i = threadIdx.x; i < n16; i += blockDim.x) d4[i] = make_uint4(0u, 0u, 0u, 0u);
+  if (threadIdx.x <= nr) s_off[threadIdx.x] = __ldg(row_ptr + n0 + threadIdx.x);
+  __syncthreads();
   bool bad = false;
-  for (int64_t n = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; n < N; n += warps) {
-    int64_t j0 = __ldg(row_ptr + n), j1 = __ldg(row_ptr + n + 1);
-    if (j0 < 0 || j1 > nnz || j0 > j1) {
-      bad = true;
-      continue;
-    }
-    for (int64_t j = j0 + lane; j < j1; j += 32) {
-      const uint32_t k = __ldg(col + j);
+  {
+    const int t = threadIdx.x;
+    const bool row_bad = t < nr && (s_off[t] < 0 || s_off[t] > s_off[t + 1] || (int64_t)s_off[t + 1] > nnz);
+    bad = __syncthreads_or(row_bad) != 0;             // inconsistent offsets: scatter nothing
+  }
+  if (!bad) {
+    const int jb = s_off[0], je = s_off[nr];
+    for (int jj = jb + (int)threadIdx.x; jj < je; jj += blockDim.x) {
+      int lo = 0, hi = nr - 1;                         // the row holding jj: s_off[lo] <= jj < s_off[lo + 1]
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_off[mid] <= jj) lo = mid; else hi = mid - 1;
+      }
+      const uint32_t k = __ldg(col + jj);
       if (k >= (uint64_t)K) {
         bad = true;
         continue;
       }
-      Fd[n * K + k] = __ldg(cval + j);
+      drow[(int64_t)lo * K + k] = __ldg(cval + jj);
     }
   }
+  __syncthreads();
+  uint4* g4 = reinterpret_cast<uint4*>(Fd + n0 * K);
+  for (int64_t i = threadIdx.x; i < n16; i += blockDim.x) g4[i] = d4[i];
   if (bad) raise_flag(flag, kFlagBadIndex);
 }
 
@@ -283,7 +318,10 @@ static int wht_tokens(int64_t b) {
   return tt;
 }
 
-static size_t wht_smem(int64_t b, int tt) { return (size_t)tt * qwha_pitch((int)b) * 4; }
+// fp32 rows of the transform (length bs) plus the raw bf16 input tile (length b)
+static size_t wht_smem(int64_t b, int64_t bs, int tt) {
+  return (size_t)tt * qwha_pitch((int)bs) * 4 + (size_t)tt * b * 2;
+}
 
 static bool qwha_decode_shaped(int64_t M, int64_t K) { return M <= kSmallMMax && small_m_supported(K, 0); }
 
@@ -294,25 +332,30 @@ int64_t qwha_ws_bytes(int64_t M, int64_t N, int64_t K) {
   return round_up(M * K * 2, 256) + round_up(N * K * 2, 256) + ext_fwd_ws_bytes(M, N, K, K);
 }
 
-// Z = X H: SLAB (decode-shaped, one token per CTA, tokens < M only: the slab's other
-// columns are never added to Y) or row-major [M, K].
+// Z = X H, SLAB (decode-shaped: one token per CTA and blocks of more than 512 split into
+// 512-column slices over several CTAs, so one token's transform is spread over the GPU;
+// tokens < M only, the slab's other columns are never added to Y) or row-major [M, K].
 template <bool SLAB>
 static ql_status launch_wht(const uint16_t* X, int64_t M, int64_t K, uint16_t* Z, cudaStream_t st) {
   const int64_t b = K & (-K);
   const int L = log2_exact(b);
+  const int SL = SLAB && L > 9 ? L - 9 : 0;
   const int tt = SLAB ? 1 : wht_tokens(b);
-  const size_t smem = wht_smem(b, tt);
-  if (L < 6 || L > 15 || smem > 200 * 1024) return QL_ERR_UNSUPPORTED;
+  const size_t smem = wht_smem(b, b >> SL, tt);
+  if (L < 6 || L > 16 || L - SL < 5 || smem > 200 * 1024) return QL_ERR_UNSUPPORTED;
   auto kern = qwha_wht_kernel<SLAB>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return QL_ERR_CUDA;
-  const dim3 grid((unsigned)((M + tt - 1) / tt), (unsigned)(K / b));
-  if ((M + tt - 1) / tt > 0x7fffffff) return QL_ERR_UNSUPPORTED;
+  if ((M + tt - 1) / tt > 0x7fffffff || (K / b) << SL > 65535) return QL_ERR_UNSUPPORTED;
+  const dim3 grid((unsigned)((M + tt - 1) / tt), (unsigned)((K / b) << SL));
   const float scale = (float)(1.0 / std::sqrt((double)b));
-  kern<<<grid, 256, smem, st>>>(X, M, K, L, tt, scale, Z);
+  kern<<<grid, 256, smem, st>>>(X, M, K, L, SL, tt, scale, Z);
   QL_CHECK_LAUNCH();
   return QL_OK;
 }
+
+// rows of the dense F per CTA: about 64 KB of shared memory
+static int densify_rows(int64_t K) { return (int)imax64(1, imin64(64, 65536 / (2 * K))); }
 
 }  // namespace qlb
 
@@ -322,7 +365,7 @@ extern "C" {
 
 ql_status qlora_linear_fwd_qwha(const ql_weight* w, const ql_bf16* X, int64_t M, const ql_qwha* f, ql_bf16* Y,
                                 void* ws, size_t ws_bytes, void* stream) {
-  if (!w || !f || !X || !Y || M < 1) return QL_ERR_INVALID_ARG;
+  if (!w || !f || !X || !Y || M < 1 || !aligned(X, 16) || !aligned(Y, 16)) return QL_ERR_INVALID_ARG;
   if (!f->row_ptr || f->nnz < 0 || (f->nnz > 0 && (!f->col || !f->c))) return QL_ERR_INVALID_ARG;
   if (!aligned(f->row_ptr, 4) || !aligned(f->col, 2) || !aligned(f->c, 2)) return QL_ERR_INVALID_ARG;
   if (f->nnz >= (int64_t(1) << 31) || w->K > 65536) return QL_ERR_UNSUPPORTED;
@@ -332,7 +375,7 @@ ql_status qlora_linear_fwd_qwha(const ql_weight* w, const ql_bf16* X, int64_t M,
   if ((int64_t)ws_bytes < qwha_ws_bytes(M, N, K)) return QL_ERR_WORKSPACE;
   {
     const int64_t b = K & (-K);
-    if (wht_smem(b, wht_tokens(b)) > 200 * 1024) return QL_ERR_UNSUPPORTED;
+    if (wht_smem(b, b, wht_tokens(b)) > 200 * 1024) return QL_ERR_UNSUPPORTED;
   }
   cudaStream_t st = as_stream(stream);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
@@ -345,8 +388,16 @@ ql_status qlora_linear_fwd_qwha(const ql_weight* w, const ql_bf16* X, int64_t M,
     ProfScope prof(PK_FWD_ADAPTER, st, 2);
     e = launch_wht<true>(X, M, K, Zs, st);
     if (e != QL_OK || f->nnz == 0) return e;
-    const dim3 grid((unsigned)((N + 63) / 64), 1u);
-    qwha_spmm_kernel<<<grid, 256, 0, st>>>(Zs, M, N, K, f->row_ptr, f->col, f->c, f->nnz, Y, device_flag_ptr());
+    const unsigned grid = (unsigned)imin64((N + 7) / 8, (int64_t)num_sms() * 8);   // a warp per row
+    const int tp = (int)((M + 1) / 2);
+    if (tp <= 1)
+      qwha_spmm_kernel<1><<<grid, 256, 0, st>>>(Zs, M, N, K, f->row_ptr, f->col, f->c, f->nnz, Y, device_flag_ptr());
+    else if (tp <= 2)
+      qwha_spmm_kernel<2><<<grid, 256, 0, st>>>(Zs, M, N, K, f->row_ptr, f->col, f->c, f->nnz, Y, device_flag_ptr());
+    else if (tp <= 4)
+      qwha_spmm_kernel<4><<<grid, 256, 0, st>>>(Zs, M, N, K, f->row_ptr, f->col, f->c, f->nnz, Y, device_flag_ptr());
+    else
+      qwha_spmm_kernel<8><<<grid, 256, 0, st>>>(Zs, M, N, K, f->row_ptr, f->col, f->c, f->nnz, Y, device_flag_ptr());
     QL_CHECK_LAUNCH();
     return QL_OK;
   }
@@ -356,15 +407,17 @@ ql_status qlora_linear_fwd_qwha(const ql_weight* w, const ql_bf16* X, int64_t M,
   uint16_t* Fd = reinterpret_cast<uint16_t*>(wsb + zb);
   const int64_t fb = round_up(N * K * 2, 256);
   {
-    ProfScope prof(PK_FWD_ADAPTER, st, 3);
+    ProfScope prof(PK_FWD_ADAPTER, st, 2);
     e = launch_wht<false>(X, M, K, Z, st);
     if (e != QL_OK) return e;
-    if (cudaMemsetAsync(Fd, 0, (size_t)(N * K * 2), st) != cudaSuccess) return QL_ERR_CUDA;
-    if (f->nnz > 0) {
-      qwha_densify_kernel<<<(unsigned)imin64((N + 7) / 8, (int64_t)num_sms() * 8), 256, 0, st>>>(
-          f->row_ptr, f->col, f->c, f->nnz, N, K, Fd, device_flag_ptr());
-      QL_CHECK_LAUNCH();
-    }
+    const int rows = densify_rows(K);
+    const size_t dsm = (size_t)rows * K * 2;
+    if (cudaFuncSetAttribute(qwha_densify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsm) !=
+        cudaSuccess)
+      return QL_ERR_CUDA;
+    qwha_densify_kernel<<<(unsigned)((N + rows - 1) / rows), 256, dsm, st>>>(f->row_ptr, f->col, f->c, f->nnz,
+                                                                          N, K, rows, Fd, device_flag_ptr());
+    QL_CHECK_LAUNCH();
   }
   return ext_forward(w, X, M, Z, Fd, K, Y, wsb + zb + fb, ws_bytes - (size_t)(zb + fb), st);
 }
@@ -374,7 +427,7 @@ ql_status ql_wht(const ql_bf16* X, int64_t M, int64_t K, ql_bf16* Z, void* strea
   if (K % 64 != 0 || M > (int64_t(1) << 31)) return QL_ERR_UNSUPPORTED;
   if (!aligned(X, 16) || !aligned(Z, 16)) return QL_ERR_INVALID_ARG;
   const int64_t b = K & (-K);
-  if (wht_smem(b, wht_tokens(b)) > 200 * 1024) return QL_ERR_UNSUPPORTED;
+  if (wht_smem(b, b, wht_tokens(b)) > 200 * 1024) return QL_ERR_UNSUPPORTED;
   ProfScope prof(PK_FWD_ADAPTER, as_stream(stream), 1);
   return launch_wht<false>(X, M, K, Z, as_stream(stream));
 }
