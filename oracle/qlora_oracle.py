@@ -24,6 +24,8 @@ It is a plain, slow, obviously correct restatement of what the method computes:
 * The Walsh-Hadamard adapter of the QWHA page (gist.science/ko/paper/2509.17428,
   section 2.1): Delta W = F H^{-1} with a sparse coefficient matrix F and the
   Walsh-Hadamard matrix H, in fp64.
+* The adapter optimiser step whose states the QLoRA page pages to host memory (section
+  "3. Paged Optimizer"): AdamW on the flat adapter vector, in fp64.
 
 Where the pages are silent the reading taken is stated in the docstring of the
 function that takes it. Floating-point steps are written with numpy float32 scalars
@@ -541,3 +543,34 @@ def qwha_linear_fwd(X, Wd, row_ptr, col, c) -> np.ndarray:
     Wd = np.asarray(Wd, np.float64)
     N, K = Wd.shape
     return X @ Wd.T + X @ qwha_delta(N, K, row_ptr, col, c).T
+
+
+# --------------------------------------------------------------------------------------
+# The adapter optimiser step with paged states (QLoRA page, aizip.shop/methodologies/qlora,
+# section "3. Paged Optimizer": optimiser states held in unified memory, paged to host RAM
+# when device memory runs short, with the memory decomposition listing the optimiser
+# states as the pageable part)
+# --------------------------------------------------------------------------------------
+
+def adamw_step(master, grad, m, v, step: int, lr: float, beta1: float, beta2: float, eps: float,
+               weight_decay: float, grad_scale: float = 1.0):
+    """One AdamW step on a flat adapter parameter vector, fp64.
+
+    Reading: the page names no optimiser, only that its states are pageable. AdamW is
+    taken: Adam's bias-corrected first and second moments with weight decay decoupled from
+    the gradient. With g = grad_scale * grad and t = step (1 for the first step):
+        m <- beta1 m + (1 - beta1) g
+        v <- beta2 v + (1 - beta2) g^2
+        theta <- theta (1 - lr weight_decay) - lr (m / (1 - beta1^t)) / (sqrt(v / (1 - beta2^t)) + eps)
+    The trained copy theta (`master`) is kept in full precision; the bf16 copy the linear
+    layer reads is RNbf(theta). grad_scale folds a data-parallel average (1/world) into
+    the step. Returns (master, m, v, param_bf16_bits)."""
+    assert step >= 1
+    theta = np.asarray(master, np.float64).copy()
+    g = np.asarray(grad, np.float64) * grad_scale
+    m = beta1 * np.asarray(m, np.float64) + (1.0 - beta1) * g
+    v = beta2 * np.asarray(v, np.float64) + (1.0 - beta2) * g * g
+    m_hat = m / (1.0 - beta1 ** step)
+    v_hat = v / (1.0 - beta2 ** step)
+    theta = theta * (1.0 - lr * weight_decay) - lr * m_hat / (np.sqrt(v_hat) + eps)
+    return theta, m, v, f32_to_bf16_bits(theta.astype(np.float32))

@@ -577,3 +577,48 @@ def test_qwha_zero_and_linear_in_c():
     D1 = o.qwha_delta(N, K, row_ptr, col, c)
     D2 = o.qwha_delta(N, K, row_ptr, col, -2.5 * c)
     np.testing.assert_allclose(D2, -2.5 * D1, rtol=1e-13, atol=1e-15)
+
+
+# ---------------------------------------------------------------- AdamW step (paged states)
+
+def test_adamw_matches_torch_over_several_steps():
+    """The oracle's step equals torch.optim.AdamW (fp64) over six steps with weight decay
+    and a gradient scale folded into the gradient."""
+    rng = np.random.default_rng(21)
+    n = 257
+    theta0 = rng.standard_normal(n) * 0.05
+    hp = dict(lr=2e-3, beta1=0.9, beta2=0.995, eps=1e-8, weight_decay=0.05)
+    p = torch.nn.Parameter(torch.tensor(theta0, dtype=torch.float64))
+    opt = torch.optim.AdamW([p], lr=hp["lr"], betas=(hp["beta1"], hp["beta2"]), eps=hp["eps"],
+                            weight_decay=hp["weight_decay"])
+    theta, m, v = theta0.copy(), np.zeros(n), np.zeros(n)
+    for t in range(1, 7):
+        g = rng.standard_normal(n)
+        p.grad = torch.tensor(g * 0.5, dtype=torch.float64)
+        opt.step()
+        theta, m, v, bits = o.adamw_step(theta, g, m, v, t, grad_scale=0.5, **hp)
+        np.testing.assert_allclose(theta, p.detach().numpy(), rtol=1e-13, atol=1e-15)
+        st = opt.state[p]
+        np.testing.assert_allclose(m, st["exp_avg"].numpy(), rtol=1e-13, atol=1e-16)
+        np.testing.assert_allclose(v, st["exp_avg_sq"].numpy(), rtol=1e-13, atol=1e-18)
+    assert np.array_equal(bits, o.f32_to_bf16_bits(theta.astype(np.float32)))
+
+
+def test_adamw_first_step_closed_form():
+    """Step 1 without weight decay: m_hat = g and v_hat = g^2, so the update is
+    -lr g / (|g| + eps), a step of lr against the sign of g."""
+    g = np.array([3.0, -0.25, 1e-3, -7.5])
+    lr, eps = 1e-2, 1e-8
+    theta, m, v, _ = o.adamw_step(np.zeros(4), g, np.zeros(4), np.zeros(4), 1, lr, 0.9, 0.999, eps, 0.0)
+    np.testing.assert_allclose(theta, -lr * g / (np.abs(g) + eps), rtol=1e-14)
+    np.testing.assert_allclose(m, 0.1 * g, rtol=1e-15)
+    np.testing.assert_allclose(v, 0.001 * g * g, rtol=1e-14)
+
+
+def test_adamw_zero_gradient_only_decays():
+    """g = 0: the moments decay by beta1 and beta2 and, without weight decay, theta moves by
+    the remaining momentum alone; with m = 0 too it stays where it is except for decay."""
+    theta0 = np.array([0.5, -1.0])
+    theta, m, v, _ = o.adamw_step(theta0, np.zeros(2), np.zeros(2), np.zeros(2), 3, 1e-3, 0.9, 0.99, 1e-8, 0.1)
+    np.testing.assert_allclose(theta, theta0 * (1 - 1e-4), rtol=1e-15)
+    assert np.all(m == 0) and np.all(v == 0)
