@@ -432,6 +432,58 @@ def qwha_bench(dev, peaks, qw_up, X_up, reps: int = 10):
     return out
 
 
+def optim_bench(dev, peaks, reps: int = 10):
+    """The adapter optimiser step (AdamW) over every adapter parameter of the 7B stack at
+    rank 64 (one flat vector), 30 bytes per parameter. States (theta, m, v) in paged
+    (managed) memory resident on the device, beside the same step on plain device memory;
+    and once with the states paged out to the host before the step (the migration cost)."""
+    from quantized_base_rank_b200 import binding as B
+    from quantized_base_rank_b200 import stack
+    n = sum(sp.r * (sp.N + sp.K) for sp in stack.stack_7b())
+    n = (n + 3) // 4 * 4
+    g = torch.empty(n, device=dev).normal_(0.0, 1e-3, generator=torch.Generator(dev).manual_seed(3))
+    param = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    hp = dict(lr=1e-4, beta1=0.9, beta2=0.999, eps=1e-8, weight_decay=0.0)
+
+    def timed(theta, m, v, before=None, n_steps=reps):
+        B.adamw_step(theta, param, g, m, v, 1, **hp)
+        torch.cuda.synchronize()
+        total = 0.0
+        for t in range(n_steps):
+            if before is not None:
+                before()
+                torch.cuda.synchronize()
+            e0.record()
+            B.adamw_step(theta, param, g, m, v, t + 2, **hp)
+            e1.record()
+            torch.cuda.synchronize()
+            total += e0.elapsed_time(e1)
+        return total / n_steps
+
+    dense = [torch.zeros(n, device=dev) for _ in range(3)]
+    ms_dev = timed(*dense)
+    del dense
+    buf = B.PagedBuffer(3 * n * 4)
+    th, m, v = (buf.view(torch.float32, n, i * n * 4) for i in range(3))
+    th.zero_()
+    m.zero_()
+    v.zero_()
+    buf.prefetch(to_host=False)
+    ms_paged = timed(th, m, v)
+    ms_paged_in = timed(th, m, v, before=lambda: buf.prefetch(to_host=True), n_steps=2)
+    buf.prefetch(to_host=False)
+    torch.cuda.synchronize()
+    del th, m, v
+    buf.free()
+    nbytes = 30 * n
+    return {"params": n, "bytes_per_step": nbytes,
+            "paged_resident": {"ms": ms_paged, "GB/s": nbytes / (ms_paged * 1e-3) / 1e9,
+                               "frac_hbm": nbytes / (ms_paged * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+            "device_memory": {"ms": ms_dev, "GB/s": nbytes / (ms_dev * 1e-3) / 1e9},
+            "paged_in_from_host": {"ms": ms_paged_in, "state_bytes_migrated": 12 * n}}
+
+
 def run_ours(args, case, world, rank, local_rank):
     from quantized_base_rank_b200 import binding as B
     from quantized_base_rank_b200 import dp, synth
@@ -573,6 +625,9 @@ def run_ours(args, case, world, rank, local_rank):
     # ---- Walsh-Hadamard (QWHA) adapter ----
     qwha = qwha_bench(dev, peaks, qw, X)
 
+    # ---- adapter optimiser step with paged states ----
+    optim = optim_bench(dev, peaks)
+
     # ---- CPU oracle baseline (rank 0, one GPU only) ----
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -613,6 +668,7 @@ def run_ours(args, case, world, rank, local_rank):
             "decode_7b_4096x4096_nf4": decode,
             "lordba": lordba,
             "qwha": qwha,
+            "optimizer_adamw_7b_r64": optim,
         },
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
@@ -632,8 +688,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--gemm", choices=["pair", "single"], default="single",
                     help="fused weight GEMM on CTA pairs (cta_group::2) or on single CTAs")
-    ap.add_argument("--part", choices=["all", "decode", "qwha"], default="all",
-                    help="decode / qwha: only that component (a short run for profiling)")
+    ap.add_argument("--part", choices=["all", "decode", "qwha", "optim"], default="all",
+                    help="decode / qwha / optim: only that component (a short run for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -657,6 +713,13 @@ def main():
         out = decode_bench(dev, load_peaks(), reps=args.steps)
         if rank == 0:
             print(json.dumps({"part": "decode", "decode_7b_4096x4096_nf4": out}), flush=True)
+        return
+    if args.part == "optim":
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        out = optim_bench(dev, load_peaks(), reps=args.steps)
+        if rank == 0:
+            print(json.dumps({"part": "optim", "optimizer_adamw_7b_r64": out}), flush=True)
         return
     if args.part == "qwha":
         from quantized_base_rank_b200 import binding as B

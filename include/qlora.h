@@ -265,6 +265,43 @@ ql_status ql_wht(const ql_bf16* X, int64_t M, int64_t K, ql_bf16* Z, void* strea
 
 enum { QL_OP_DQ = 0, QL_OP_FWD = 1, QL_OP_BWD = 2, QL_OP_FWD_LORDBA = 3, QL_OP_FWD_QWHA = 4 };
 
+/* The adapter optimiser step with paged states (QLoRA page, aizip.shop/methodologies/qlora,
+ * section "3. Paged Optimizer": optimiser states held in unified memory, paged to host RAM
+ * when device memory runs short). The page names no optimiser; the step is AdamW with
+ * bias-corrected moments and weight decay decoupled from the gradient. With
+ * g = grad_scale * grad and t = step (1 for the first):
+ *   m <- beta1 m + (1 - beta1) g,   v <- beta2 v + (1 - beta2) g^2,
+ *   theta <- theta (1 - lr weight_decay) - (lr / (1 - beta1^t)) m / (sqrt(v / (1 - beta2^t)) + eps),
+ *   param <- bf16(theta)  (round to nearest even),
+ * all in fp32 (the bias corrections are formed on the host in fp64). grad_scale folds a
+ * data-parallel average (1/world) into the step. */
+typedef struct {
+  float lr, beta1, beta2, eps, weight_decay, grad_scale;
+  int64_t step;
+} ql_adamw;
+
+/* One step over n adapter parameters held as one flat vector: theta, grad, m, v fp32
+ * [n] (theta the trained copy, m and v zero before step 1), param bf16 [n] (written).
+ * Every array is device memory or managed memory from ql_paged_alloc; 4-byte aligned
+ * (2 for param); 16-byte alignment and n % 4 == 0 take the vector path. The arrays must
+ * not overlap. A non-finite gradient element sets QL_ERR_NONFINITE on the device flag
+ * (the step still runs). Hyperparameters outside their domain (step < 1, beta not in
+ * [0, 1), eps <= 0, negative lr or weight decay) return QL_ERR_INVALID_ARG. */
+ql_status ql_adamw_step(float* theta, ql_bf16* param, const float* grad, float* m, float* v, int64_t n,
+                        const ql_adamw* hparams, void* stream);
+
+/* Paged memory for optimiser states: `bytes` of CUDA managed (unified) memory, usable by
+ * the kernels and the host alike, whose pages the driver migrates between device and host
+ * memory on demand (and evicts to the host when device memory is oversubscribed).
+ * *out = NULL for bytes = 0. Free with ql_paged_free. The caller owns the memory. */
+ql_status ql_paged_alloc(size_t bytes, void** out);
+ql_status ql_paged_free(void* ptr);
+
+/* Move the pages of [ptr, ptr + bytes) of paged memory to the host (to_host != 0) or to
+ * the current device, asynchronously on `stream`: the explicit form of the paging, ahead
+ * of the step that touches them (or away from the device between steps). */
+ql_status ql_paged_prefetch(const void* ptr, size_t bytes, int32_t to_host, void* stream);
+
 /* Workspace bytes that op (QL_OP_*) needs for these sizes (0 if none). */
 size_t ql_workspace_bytes(int32_t op, int64_t M, int64_t N, int64_t K, int32_t r);
 
@@ -290,7 +327,7 @@ void ql_set_wait_timeout_ns(uint64_t ns);
  * one group. Groups: 0 nf4 encode, 1 double quantisation, 2 int8 encode, 3 dequantise,
  * 4 forward layout prep, 5 forward X A^T, 6 forward main GEMM, 7 backward layout prep,
  * 8 backward dY B, 9 dB, 10 dA, 11 dX, 12 small-M forward, 13 Walsh-Hadamard adapter
- * (transform and sparse product). ql_launch_count is the
+ * (transform and sparse product), 14 optimiser step. ql_launch_count is the
  * running number of kernels the library has launched in this process. Returns 0, or -1
  * for an unknown group. */
 void ql_profile_enable(int on);

@@ -10,6 +10,7 @@ import os
 import re
 import threading
 
+import numpy as np
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -50,6 +51,13 @@ class QLLordba(ctypes.Structure):
                 ("gamma", ctypes.c_void_p)]
 
 
+class QLAdamw(ctypes.Structure):
+    """ql_adamw: the hyperparameters of one AdamW step."""
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
+                ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float), ("grad_scale", ctypes.c_float),
+                ("step", ctypes.c_int64)]
+
+
 _lib = None
 _lock = threading.Lock()
 P, I64, I32, F32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
@@ -62,6 +70,10 @@ _SIGS = {
     "qlora_linear_fwd_lordba": ([ctypes.POINTER(QLWeight), P, I64, ctypes.c_void_p, P, P, SZ, P], I32),
     "qlora_linear_fwd_qwha": ([ctypes.POINTER(QLWeight), P, I64, ctypes.c_void_p, P, P, SZ, P], I32),
     "ql_wht": ([P, I64, I64, P, P], I32),
+    "ql_adamw_step": ([P, P, P, P, P, I64, ctypes.c_void_p, P], I32),
+    "ql_paged_alloc": ([SZ, ctypes.POINTER(ctypes.c_void_p)], I32),
+    "ql_paged_free": ([ctypes.c_void_p], I32),
+    "ql_paged_prefetch": ([ctypes.c_void_p, SZ, I32, P], I32),
     "dq_quantize_shard": ([P, I64, P, I64, P, P, P, P], I32),
     "ql_dequantize": ([ctypes.POINTER(QLWeight), P, P], I32),
     "qlora_linear_fwd": ([ctypes.POINTER(QLWeight), P, I64, P, P, I32, F32, P, P, P, SZ, P], I32),
@@ -80,7 +92,7 @@ _SIGS = {
 
 # kernel groups of ql_profile_read
 PROFILE_GROUPS = ["nf4", "dq", "int8", "dequant", "fwd_prep", "fwd_xa", "fwd_main", "bwd_prep",
-                  "bwd_dyb", "bwd_db", "bwd_da", "bwd_dx", "fwd_small", "fwd_adapter"]
+                  "bwd_dyb", "bwd_db", "bwd_da", "bwd_dx", "fwd_small", "fwd_adapter", "optim"]
 
 
 def lib() -> ctypes.CDLL:
@@ -315,6 +327,80 @@ def wht(X: torch.Tensor, Z: torch.Tensor | None = None) -> torch.Tensor:
         Z = torch.empty_like(X)
     _check(lib().ql_wht(_ptr(X), M, K, _ptr(Z), _stream(X.device)), "ql_wht")
     return Z
+
+
+def adamw_step(theta: torch.Tensor, param: torch.Tensor, grad: torch.Tensor, m: torch.Tensor,
+               v: torch.Tensor, step: int, lr: float, beta1: float = 0.9, beta2: float = 0.999,
+               eps: float = 1e-8, weight_decay: float = 0.0, grad_scale: float = 1.0):
+    """One AdamW step over flat adapter parameters: theta, grad, m, v fp32 [n] (theta the
+    trained copy), param bf16 [n] (rewritten as bf16(theta)). Tensors may be views of a
+    PagedBuffer."""
+    n = theta.numel()
+    for t, nm in ((theta, "theta"), (grad, "grad"), (m, "m"), (v, "v")):
+        _need(t, torch.float32, nm)
+        if t.numel() != n:
+            raise ValueError(f"{nm} must have {n} elements")
+    _need(param, torch.bfloat16, "param")
+    if param.numel() != n:
+        raise ValueError(f"param must have {n} elements")
+    h = QLAdamw(lr, beta1, beta2, eps, weight_decay, grad_scale, step)
+    _check(lib().ql_adamw_step(_ptr(theta), _ptr(param), _ptr(grad), _ptr(m), _ptr(v), n, ctypes.addressof(h),
+                               _stream(theta.device)), "ql_adamw_step")
+
+
+class _CudaArray:
+    """A CUDA Array Interface view of memory the library owns (torch.as_tensor reads it
+    without a copy)."""
+
+    def __init__(self, ptr: int, shape, typestr: str):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr, "data": (ptr, False),
+                                         "version": 3, "strides": None, "stream": None}
+
+
+class PagedBuffer:
+    """Paged (CUDA managed) memory from ql_paged_alloc, for optimiser states: the driver
+    moves its pages between device and host memory on demand; prefetch() moves them
+    explicitly. float32 views are plain CUDA tensors over the same memory, valid while the
+    buffer is alive."""
+
+    _TYPES = {torch.float32: ("<f4", 4), torch.int8: ("|i1", 1), torch.int32: ("<i4", 4)}
+
+    def __init__(self, nbytes: int):
+        self.nbytes = int(nbytes)
+        p = ctypes.c_void_p()
+        _check(lib().ql_paged_alloc(self.nbytes, ctypes.byref(p)), "ql_paged_alloc")
+        self.ptr = p.value or 0
+
+    def view(self, dtype: torch.dtype, numel: int, offset_bytes: int = 0) -> torch.Tensor:
+        code, size = self._TYPES[dtype]
+        if offset_bytes < 0 or offset_bytes % size or offset_bytes + numel * size > self.nbytes:
+            raise ValueError("view outside the buffer")
+        return torch.as_tensor(_CudaArray(self.ptr + offset_bytes, (numel,), code), device="cuda")
+
+    def prefetch(self, to_host: bool, stream_device: torch.device | None = None, offset_bytes: int = 0,
+                 nbytes: int | None = None):
+        n = self.nbytes - offset_bytes if nbytes is None else nbytes
+        _check(lib().ql_paged_prefetch(self.ptr + offset_bytes, n, 1 if to_host else 0, _stream(stream_device)),
+               "ql_paged_prefetch")
+
+    def host_array(self, dtype=np.float32, numel: int | None = None, offset_bytes: int = 0) -> np.ndarray:
+        """The same memory read from the host (unified memory): a numpy view, valid after
+        the stream that wrote it has been synchronised."""
+        item = np.dtype(dtype).itemsize
+        n = (self.nbytes - offset_bytes) // item if numel is None else numel
+        buf = (ctypes.c_char * (n * item)).from_address(self.ptr + offset_bytes)
+        return np.frombuffer(buf, dtype=dtype, count=n)
+
+    def free(self):
+        if self.ptr:
+            _check(lib().ql_paged_free(self.ptr), "ql_paged_free")
+            self.ptr = 0
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
 
 
 class QuantWeight:

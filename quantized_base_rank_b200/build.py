@@ -18,7 +18,7 @@ BUILD_DIR = os.path.join(ROOT, "_build")
 LIB_NAME = "libqlora_b200.so"
 LIB_PATH = os.path.join(PKG, LIB_NAME)
 
-SOURCES = ["runtime.cu", "quantize.cu", "linear.cu", "small_m.cu", "lordba.cu", "qwha.cu"]
+SOURCES = ["runtime.cu", "quantize.cu", "linear.cu", "small_m.cu", "lordba.cu", "qwha.cu", "optim.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "--std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-O3",
          "-I", INCLUDE, "-I", CSRC]

@@ -59,7 +59,7 @@ __host__ __device__ __forceinline__ int64_t imax64(int64_t a, int64_t b) { retur
 enum ProfKind : int {
   PK_NF4 = 0, PK_DQ = 1, PK_INT8 = 2, PK_DEQ = 3, PK_FWD_PREP = 4, PK_FWD_T = 5, PK_FWD_MAIN = 6,
   PK_BWD_PREP = 7, PK_BWD_U = 8, PK_BWD_DB = 9, PK_BWD_DA = 10, PK_BWD_DX = 11, PK_FWD_SMALL = 12,
-  PK_FWD_ADAPTER = 13, PK_COUNT = 14
+  PK_FWD_ADAPTER = 13, PK_OPTIM = 14, PK_COUNT = 15
 };
 
 // Counts the kernels a scope launches and, when profiling is on, brackets them with a

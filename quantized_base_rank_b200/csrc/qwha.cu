@@ -17,6 +17,8 @@
 // The gather of Z by column index has no tensor-core form (F's positions are arbitrary),
 // so the second kernel runs on the FMA pipes, its slab of Z staged in shared memory when
 // it fits.
+#include <cmath>
+
 #include "common.cuh"
 
 namespace qlb {

@@ -83,6 +83,23 @@ def test_argument_validation_without_a_device(lib):
     assert lib.ql_wht(None, 1, 64, 16, None) == B.QL_ERR_INVALID_ARG
     assert lib.ql_wht(16, 1, 100, 16, None) == B.QL_ERR_UNSUPPORTED
     assert lib.ql_wht(24, 1, 64, 16, None) == B.QL_ERR_INVALID_ARG
+    # optimiser step and paged memory: argument checks happen before any CUDA call
+    h = B.QLAdamw(1e-3, 0.9, 0.999, 1e-8, 0.0, 1.0, 1)
+    assert lib.ql_adamw_step(16, 16, 16, 16, 16, 0, ctypes.addressof(h), None) == B.QL_OK
+    assert lib.ql_adamw_step(16, 16, 16, 16, 16, -1, ctypes.addressof(h), None) == B.QL_ERR_INVALID_ARG
+    assert lib.ql_adamw_step(None, 16, 16, 16, 16, 8, ctypes.addressof(h), None) == B.QL_ERR_INVALID_ARG
+    assert lib.ql_adamw_step(18, 16, 16, 16, 16, 8, ctypes.addressof(h), None) == B.QL_ERR_INVALID_ARG
+    for bad in (B.QLAdamw(1e-3, 0.9, 0.999, 1e-8, 0.0, 1.0, 0), B.QLAdamw(1e-3, 1.0, 0.999, 1e-8, 0.0, 1.0, 1),
+                B.QLAdamw(1e-3, 0.9, 0.999, 0.0, 0.0, 1.0, 1), B.QLAdamw(-1e-3, 0.9, 0.999, 1e-8, 0.0, 1.0, 1),
+                B.QLAdamw(1e-3, 0.9, 0.999, 1e-8, -0.1, 1.0, 1),
+                B.QLAdamw(1e-3, 0.9, 0.999, 1e-8, 0.0, float("nan"), 1)):
+        assert lib.ql_adamw_step(16, 16, 16, 16, 16, 8, ctypes.addressof(bad), None) == B.QL_ERR_INVALID_ARG
+    out = ctypes.c_void_p(1)
+    assert lib.ql_paged_alloc(0, ctypes.byref(out)) == B.QL_OK and not out.value
+    assert lib.ql_paged_alloc(16, None) == B.QL_ERR_INVALID_ARG
+    assert lib.ql_paged_free(None) == B.QL_OK
+    assert lib.ql_paged_prefetch(None, 0, 1, None) == B.QL_OK
+    assert lib.ql_paged_prefetch(None, 64, 1, None) == B.QL_ERR_INVALID_ARG
     assert lib.ql_dequantize(None, None, None) == B.QL_ERR_INVALID_ARG
     w = B.QLWeight(0, 0, 64, 64, 16, 0, 16, 16, 16)
     # misaligned or null pointers, bad shapes: all rejected synchronously
