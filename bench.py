@@ -641,6 +641,12 @@ def run_ours(args, case, world, rank, local_rank):
 
     if rank != 0:
         return
+    if peaks.get("bf16_tflops_sustained"):
+        peak_fwd = peaks["bf16_tflops_sustained"]
+        peak_fwd_source = f"{peaks['source']} bf16 sustained (kernel timed inside {args.steps} steps)"
+    else:
+        peak_fwd = peaks["bf16_tflops"]
+        peak_fwd_source = f"{peaks['source']} bf16 burst (no sustained figure)"
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -650,13 +656,14 @@ def run_ours(args, case, world, rank, local_rank):
                    "l2": "inputs larger than L2 (X 64 MB, W 90 MB, dY 180 MB > 126 MB)",
                    "parallelism": f"dp{world}" if world > 1 else "single",
                    "fused_gemm": "cta_pair" if args.gemm == "pair" else "single_cta"},
+        # the kernel is timed inside a long run of steps under the power cap, so its
+        # denominator is the measured sustained bf16 throughput; the burst figure is beside it
         "roofline": {"kernel": "fused forward GEMM (NF4 decode + X W'^T + P B^T)", "bound": "tensor",
-                     "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": achieved / peaks["bf16_tflops"], "traffic": fwd_main_traffic(),
+                     "achieved": achieved, "peak": peak_fwd, "unit": "TFLOP/s",
+                     "frac": achieved / peak_fwd, "traffic": fwd_main_traffic(),
                      "traffic_unit": "bytes per launch (ncu dram read + write)",
-                     "peak_source": f"{peaks['source']} bf16 burst",
-                     "frac_of_sustained": (achieved / peaks["bf16_tflops_sustained"]
-                                           if peaks["bf16_tflops_sustained"] else None)},
+                     "peak_source": peak_fwd_source,
+                     "frac_of_burst": achieved / peaks["bf16_tflops"]},
         "components": {
             "quantize_nf4_dq": {"ms": q_ms, "GB/s": n * NF4_DQ_BYTES_PER_PARAM / (q_ms * 1e-3) / 1e9,
                                 "frac_hbm": n * NF4_DQ_BYTES_PER_PARAM / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},

@@ -26,6 +26,8 @@ It is a plain, slow, obviously correct restatement of what the method computes:
   Walsh-Hadamard matrix H, in fp64.
 * The adapter optimiser step whose states the QLoRA page pages to host memory (section
   "3. Paged Optimizer"): AdamW on the flat adapter vector, in fp64.
+* The Lion step with INT8 momentum of the QFT page (section 2.1), in fp32 one operation
+  at a time, since the new momentum codes are integer decisions.
 
 Where the pages are silent the reading taken is stated in the docstring of the
 function that takes it. Floating-point steps are written with numpy float32 scalars
@@ -574,3 +576,48 @@ def adamw_step(master, grad, m, v, step: int, lr: float, beta1: float, beta2: fl
     v_hat = v / (1.0 - beta2 ** step)
     theta = theta * (1.0 - lr * weight_decay) - lr * m_hat / (np.sqrt(v_hat) + eps)
     return theta, m, v, f32_to_bf16_bits(theta.astype(np.float32))
+
+
+# --------------------------------------------------------------------------------------
+# Lion with INT8 momentum (QFT page, gist.science/ko/paper/2310.07147, section 2.1:
+# the Lion optimiser tracks only a momentum, its update is a sign so the update size is
+# fixed, and the momentum is stored in INT8)
+# --------------------------------------------------------------------------------------
+
+def lion_int8_step(theta, grad, m_codes, m_absmax, lr: float, beta1: float, beta2: float,
+                   weight_decay: float):
+    """One Lion step with the momentum held as blockwise INT8, in fp32, one IEEE operation
+    at a time (the new momentum codes are integer decisions, so the arithmetic is fixed).
+
+    Lion (the published update): c = beta1 m + (1 - beta1) g, theta <- theta (1 - lr
+    weight_decay) - lr sign(c), m <- beta2 m + (1 - beta2) g. Reading: the page gives no
+    INT8 scheme for the momentum; the blockwise absmax code of the int8 weight format is
+    taken (blocks of 64, fp32 absmax per block, codes in [-127, 127]): before the step
+    m_j = RN32(code_j * RN32(a_b / 127)); after it the blocks are re-encoded with their new
+    absmax. With f32 values: omb = RN32(1 - beta), decay = RN32(1 - RN32(lr wd)),
+        c      = RN32(RN32(beta1 m) + RN32(omb1 g))
+        theta' = RN32(RN32(theta decay) - lr sign(c))        (sign(0) = 0)
+        m'     = RN32(RN32(beta2 m) + RN32(omb2 g))
+    The trained copy theta is fp32; the bf16 copy is RNbf(theta'). The last block may be
+    partial. Returns (theta', m_codes', m_absmax', param_bf16_bits)."""
+    f = np.float32
+    theta = np.asarray(theta, np.float32).ravel()
+    g = np.asarray(grad, np.float32).ravel()
+    n = theta.size
+    codes = np.asarray(m_codes, np.int8).ravel()[:n]
+    absmax = np.asarray(m_absmax, np.float32).ravel()
+    b1, b2 = f(beta1), f(beta2)
+    omb1, omb2 = f(f(1.0) - b1), f(f(1.0) - b2)
+    decay = f(f(1.0) - f(f(lr) * f(weight_decay)))
+    blk = np.arange(n) // BLOCK
+    sc = (absmax / f(INT8_QMAX)).astype(np.float32)
+    m = (codes.astype(np.float32) * sc[blk]).astype(np.float32)
+    c = (b1 * m).astype(np.float32) + (omb1 * g).astype(np.float32)
+    u = np.where(c > 0, f(1.0), np.where(c < 0, f(-1.0), f(0.0))).astype(np.float32)
+    theta_new = (theta * decay).astype(np.float32) - (f(lr) * u).astype(np.float32)
+    m_new = ((b2 * m).astype(np.float32) + (omb2 * g).astype(np.float32)).astype(np.float32)
+    nb = (n + BLOCK - 1) // BLOCK
+    a_new = np.zeros(nb, np.float32)
+    np.maximum.at(a_new, blk, np.abs(m_new))
+    codes_new = int8_encode(m_new, a_new)
+    return theta_new.astype(np.float32), codes_new, a_new, f32_to_bf16_bits(theta_new)

@@ -622,3 +622,63 @@ def test_adamw_zero_gradient_only_decays():
     theta, m, v, _ = o.adamw_step(theta0, np.zeros(2), np.zeros(2), np.zeros(2), 3, 1e-3, 0.9, 0.99, 1e-8, 0.1)
     np.testing.assert_allclose(theta, theta0 * (1 - 1e-4), rtol=1e-15)
     assert np.all(m == 0) and np.all(v == 0)
+
+
+# ---------------------------------------------------------------- Lion with INT8 momentum
+
+def _lion_case(n=300, seed=4):
+    rng = np.random.default_rng(seed)
+    th = (rng.standard_normal(n) * 0.02).astype(np.float32)
+    g = (rng.standard_normal(n) * 1e-3).astype(np.float32)
+    m_exact = (rng.standard_normal(n) * 1e-4).astype(np.float32)
+    codes, am = o.int8_quantize(m_exact)
+    return th, g, codes, am
+
+
+def test_lion_first_step_closed_form():
+    """From a zero momentum: c = (1 - beta1) g, so theta' = RN32(theta decay) - lr sign(g),
+    and the new momentum is the blockwise INT8 code of RN32((1 - beta2) g)."""
+    th, g, _, _ = _lion_case()
+    n = th.size
+    lr, wd = 1e-4, 0.1
+    t2, c2, a2, _ = o.lion_int8_step(th, g, np.zeros(n, np.int8), np.zeros(5, np.float32), lr, 0.9, 0.99, wd)
+    decay = np.float32(np.float32(1) - np.float32(np.float32(lr) * np.float32(wd)))
+    want = (th * decay).astype(np.float32) - np.float32(lr) * np.sign(g).astype(np.float32)
+    assert np.array_equal(t2, want.astype(np.float32))
+    m_new = (np.float32(np.float32(1) - np.float32(0.99)) * g).astype(np.float32)
+    c_ref, a_ref = o.int8_quantize(m_new)
+    assert np.array_equal(c2, c_ref) and np.array_equal(a2, a_ref)
+
+
+def test_lion_update_size_is_fixed():
+    """Without weight decay every element moves by lr (the sign update's fixed size, the
+    property the page relies on), up to one fp32 rounding of theta, against the direction
+    of c computed independently in fp64."""
+    th, g, codes, am = _lion_case()
+    lr = 3e-4
+    t2, _, _, _ = o.lion_int8_step(th, g, codes, am, lr, 0.9, 0.99, 0.0)
+    m = codes.astype(np.float64) * (am.astype(np.float64) / 127.0)[np.arange(th.size) // 64]
+    c64 = 0.9 * m + 0.1 * g.astype(np.float64)
+    sure = np.abs(c64) > 1e-9
+    step = t2.astype(np.float64) - th.astype(np.float64)
+    # one rounding of theta' (at the larger of |theta|, |theta'|), against lr as an fp32
+    ulp = np.spacing(np.maximum(np.abs(th), np.abs(t2))).astype(np.float64)
+    lr32 = float(np.float32(lr))
+    assert np.all(np.abs(np.abs(step[sure]) - lr32) <= ulp[sure])
+    assert np.all(np.sign(step[sure]) == -np.sign(c64[sure]))
+
+
+def test_lion_momentum_round_trip_bound():
+    """The stored momentum is within half a code step of the exact new momentum, and each
+    block's largest element is stored as +-127."""
+    th, g, codes, am = _lion_case(n=640)
+    b1, b2 = 0.9, 0.95
+    _, c2, a2, _ = o.lion_int8_step(th, g, codes, am, 1e-4, b1, b2, 0.0)
+    blk = np.arange(th.size) // 64
+    m = codes.astype(np.float64) * (am.astype(np.float64) / 127.0)[blk]
+    m_new = b2 * m + (1 - b2) * g.astype(np.float64)
+    step = (a2.astype(np.float64) / 127.0)[blk]
+    got = c2.astype(np.float64) * step
+    assert np.all(np.abs(got - m_new) <= 0.5 * step * (1 + 1e-5) + 1e-12)
+    for b in range(a2.size):
+        assert np.max(np.abs(c2[blk == b])) == 127
