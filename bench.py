@@ -476,8 +476,26 @@ def optim_bench(dev, peaks, reps: int = 10):
     torch.cuda.synchronize()
     del th, m, v
     buf.free()
+    # Lion with INT8 momentum on the same parameters: 16 bytes per parameter
+    theta = torch.zeros(n, device=dev)
+    codes = torch.zeros(n, dtype=torch.int8, device=dev)
+    amax = torch.zeros((n + 63) // 64, device=dev)
+    for _ in range(3):
+        B.lion_int8_step(theta, param, g, codes, amax, 1e-4)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(reps):
+        B.lion_int8_step(theta, param, g, codes, amax, 1e-4)
+    e1.record()
+    torch.cuda.synchronize()
+    ms_lion = e0.elapsed_time(e1) / reps
+    lion_bytes = 16 * n + 8 * ((n + 63) // 64)
+    del theta, codes, amax
     nbytes = 30 * n
     return {"params": n, "bytes_per_step": nbytes,
+            "lion_int8": {"ms": ms_lion, "bytes_per_step": lion_bytes,
+                          "GB/s": lion_bytes / (ms_lion * 1e-3) / 1e9,
+                          "frac_hbm": lion_bytes / (ms_lion * 1e-3) / 1e9 / peaks["hbm_gbs"]},
             "paged_resident": {"ms": ms_paged, "GB/s": nbytes / (ms_paged * 1e-3) / 1e9,
                                "frac_hbm": nbytes / (ms_paged * 1e-3) / 1e9 / peaks["hbm_gbs"]},
             "device_memory": {"ms": ms_dev, "GB/s": nbytes / (ms_dev * 1e-3) / 1e9},

@@ -290,6 +290,28 @@ typedef struct {
 ql_status ql_adamw_step(float* theta, ql_bf16* param, const float* grad, float* m, float* v, int64_t n,
                         const ql_adamw* hparams, void* stream);
 
+/* Lion with INT8 momentum (QFT page, gist.science/ko/paper/2310.07147, section 2.1: Lion
+ * keeps only a momentum, its update is a sign of fixed size, and the momentum is stored in
+ * INT8). With fp32 values and one IEEE rounding per operation, omb = 1 - beta and
+ * decay = 1 - lr * weight_decay:
+ *   m      = code * (absmax_block / 127)           (the stored momentum, decoded)
+ *   c      = beta1 m + omb1 g
+ *   theta <- theta decay - lr sign(c)              (sign(0) = 0)
+ *   m'     = beta2 m + omb2 g, re-encoded per block of 64: absmax' = max |m'|,
+ *            code' = clamp(rint(m' / (absmax' / 127)), -127, 127) (0 for a zero block)
+ *   param <- bf16(theta)                          (round to nearest even)
+ * The page names no INT8 scheme for the momentum; this is the blockwise absmax code of the
+ * int8 weight format. */
+typedef struct {
+  float lr, beta1, beta2, weight_decay;
+} ql_lion;
+
+/* One step over n parameters: theta, grad fp32 [n]; m_codes int8 [n] and m_absmax fp32
+ * [ceil(n/64)] (all zero before the first step), both updated; param bf16 [n] written.
+ * Device or paged memory. A non-finite gradient sets QL_ERR_NONFINITE on the device flag. */
+ql_status ql_lion_int8_step(float* theta, ql_bf16* param, const float* grad, int8_t* m_codes,
+                            float* m_absmax, int64_t n, const ql_lion* hparams, void* stream);
+
 /* Paged memory for optimiser states: `bytes` of CUDA managed (unified) memory, usable by
  * the kernels and the host alike, whose pages the driver migrates between device and host
  * memory on demand (and evicts to the host when device memory is oversubscribed).

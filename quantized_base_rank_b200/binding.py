@@ -58,6 +58,12 @@ class QLAdamw(ctypes.Structure):
                 ("step", ctypes.c_int64)]
 
 
+class QLLion(ctypes.Structure):
+    """ql_lion: the hyperparameters of one Lion step."""
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
+                ("weight_decay", ctypes.c_float)]
+
+
 _lib = None
 _lock = threading.Lock()
 P, I64, I32, F32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
@@ -71,6 +77,7 @@ _SIGS = {
     "qlora_linear_fwd_qwha": ([ctypes.POINTER(QLWeight), P, I64, ctypes.c_void_p, P, P, SZ, P], I32),
     "ql_wht": ([P, I64, I64, P, P], I32),
     "ql_adamw_step": ([P, P, P, P, P, I64, ctypes.c_void_p, P], I32),
+    "ql_lion_int8_step": ([P, P, P, P, P, I64, ctypes.c_void_p, P], I32),
     "ql_paged_alloc": ([SZ, ctypes.POINTER(ctypes.c_void_p)], I32),
     "ql_paged_free": ([ctypes.c_void_p], I32),
     "ql_paged_prefetch": ([ctypes.c_void_p, SZ, I32, P], I32),
@@ -346,6 +353,26 @@ def adamw_step(theta: torch.Tensor, param: torch.Tensor, grad: torch.Tensor, m: 
     h = QLAdamw(lr, beta1, beta2, eps, weight_decay, grad_scale, step)
     _check(lib().ql_adamw_step(_ptr(theta), _ptr(param), _ptr(grad), _ptr(m), _ptr(v), n, ctypes.addressof(h),
                                _stream(theta.device)), "ql_adamw_step")
+
+
+def lion_int8_step(theta: torch.Tensor, param: torch.Tensor, grad: torch.Tensor, m_codes: torch.Tensor,
+                   m_absmax: torch.Tensor, lr: float, beta1: float = 0.9, beta2: float = 0.99,
+                   weight_decay: float = 0.0):
+    """One Lion step with INT8 momentum: theta, grad fp32 [n]; m_codes int8 [n] and m_absmax
+    fp32 [ceil(n/64)] updated in place; param bf16 [n] rewritten as bf16(theta)."""
+    n = theta.numel()
+    for t, nm in ((theta, "theta"), (grad, "grad")):
+        _need(t, torch.float32, nm)
+        if t.numel() != n:
+            raise ValueError(f"{nm} must have {n} elements")
+    _need(param, torch.bfloat16, "param")
+    _need(m_codes, torch.int8, "m_codes")
+    _need(m_absmax, torch.float32, "m_absmax")
+    if param.numel() != n or m_codes.numel() != n or m_absmax.numel() != (n + 63) // 64:
+        raise ValueError("param, m_codes or m_absmax has the wrong size")
+    h = QLLion(lr, beta1, beta2, weight_decay)
+    _check(lib().ql_lion_int8_step(_ptr(theta), _ptr(param), _ptr(grad), _ptr(m_codes), _ptr(m_absmax), n,
+                                   ctypes.addressof(h), _stream(theta.device)), "ql_lion_int8_step")
 
 
 class _CudaArray:

@@ -94,6 +94,12 @@ def test_argument_validation_without_a_device(lib):
                 B.QLAdamw(1e-3, 0.9, 0.999, 1e-8, -0.1, 1.0, 1),
                 B.QLAdamw(1e-3, 0.9, 0.999, 1e-8, 0.0, float("nan"), 1)):
         assert lib.ql_adamw_step(16, 16, 16, 16, 16, 8, ctypes.addressof(bad), None) == B.QL_ERR_INVALID_ARG
+    hl = B.QLLion(1e-4, 0.9, 0.99, 0.0)
+    assert lib.ql_lion_int8_step(16, 16, 16, 16, 16, 0, ctypes.addressof(hl), None) == B.QL_OK
+    assert lib.ql_lion_int8_step(16, 16, 16, None, 16, 8, ctypes.addressof(hl), None) == B.QL_ERR_INVALID_ARG
+    for bad in (B.QLLion(-1e-4, 0.9, 0.99, 0.0), B.QLLion(1e-4, 1.5, 0.99, 0.0), B.QLLion(1e-4, 0.9, -0.1, 0.0),
+                B.QLLion(1e-4, 0.9, 0.99, float("inf"))):
+        assert lib.ql_lion_int8_step(16, 16, 16, 16, 16, 8, ctypes.addressof(bad), None) == B.QL_ERR_INVALID_ARG
     out = ctypes.c_void_p(1)
     assert lib.ql_paged_alloc(0, ctypes.byref(out)) == B.QL_OK and not out.value
     assert lib.ql_paged_alloc(16, None) == B.QL_ERR_INVALID_ARG

@@ -102,3 +102,59 @@ def test_adamw_nonfinite_gradient_is_flagged():
     assert B.device_status() == B.QL_ERR_NONFINITE
     B.adamw_step(theta, param, torch.zeros_like(g), torch.zeros_like(m), torch.zeros_like(v), 1, **HP)
     assert B.device_status() == B.QL_OK
+
+
+# ---- Lion with INT8 momentum (QFT page, section 2.1) -----------------------------------
+
+@pytest.mark.parametrize("n", [64 * 4096, 1_000_003, 37])
+def test_lion_int8_bit_exact(n):
+    """Four steps: theta, the momentum codes and absmax, and the bf16 copy are bit-identical
+    to the oracle (the step is fixed fp32 arithmetic; the codes are integer decisions)."""
+    theta0 = synth.normal_bf16((n,), 0.02, 9, 59).float()
+    grads = _grads(n, 4, 9)
+    nb = (n + 63) // 64
+    theta = theta0.cuda()
+    codes = torch.zeros(n, dtype=torch.int8, device="cuda")
+    amax = torch.zeros(nb, dtype=torch.float32, device="cuda")
+    param = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+    tr, cr, ar = theta0.numpy(), np.zeros(n, np.int8), np.zeros(nb, np.float32)
+    hp = dict(lr=1e-4, beta1=0.9, beta2=0.99, weight_decay=0.1)
+    for g in grads:
+        B.lion_int8_step(theta, param, g.cuda(), codes, amax, **hp)
+        tr, cr, ar, br = o.lion_int8_step(tr, g.numpy(), cr, ar, **hp)
+    torch.cuda.synchronize()
+    assert B.device_status() == B.QL_OK
+    assert np.array_equal(theta.cpu().numpy().view(np.uint32), tr.view(np.uint32))
+    assert np.array_equal(codes.cpu().numpy(), cr)
+    assert np.array_equal(amax.cpu().numpy().view(np.uint32), ar.view(np.uint32))
+    assert np.array_equal(param.view(torch.int16).cpu().numpy().view(np.uint16), br)
+
+
+def test_lion_int8_paged_states():
+    """The INT8 momentum and theta in paged memory, moved to the host between steps, give
+    the same bits as device memory."""
+    n = 200_000
+    nb = (n + 63) // 64
+    theta0 = synth.normal_bf16((n,), 0.02, 10, 59).float()
+    grads = _grads(n, 3, 10)
+    buf = B.PagedBuffer(n * 4 + nb * 4 + n)
+    pt = buf.view(torch.float32, n)
+    pa = buf.view(torch.float32, nb, n * 4)
+    pc = buf.view(torch.int8, n, n * 4 + nb * 4)
+    pt.copy_(theta0.cuda())
+    pa.zero_()
+    pc.zero_()
+    theta, codes = theta0.cuda(), torch.zeros(n, dtype=torch.int8, device="cuda")
+    amax = torch.zeros(nb, device="cuda")
+    p1 = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+    p2 = torch.empty_like(p1)
+    for g in grads:
+        gd = g.cuda()
+        B.lion_int8_step(theta, p1, gd, codes, amax, 1e-4)
+        buf.prefetch(to_host=True)
+        B.lion_int8_step(pt, p2, gd, pc, pa, 1e-4)
+    torch.cuda.synchronize()
+    assert B.device_status() == B.QL_OK
+    assert torch.equal(theta, pt) and torch.equal(codes, pc) and torch.equal(amax, pa)
+    del pt, pa, pc
+    buf.free()
