@@ -35,9 +35,11 @@ struct Nf4BoundTable {
 const Nf4BoundTable& nf4_bound_table();  // host, computed on first use
 
 // Decode-shaped forward (M <= 16), small_m.cu.
+// Yadd (optional, fp32 [M][N]) is added to the product before its bf16 rounding; it may be
+// written by the grid just before on the stream (it is read after the dependency wait).
 ql_status small_m_forward(const ql_weight* w, const uint16_t* X, int64_t M, const uint16_t* A,
                           const uint16_t* B, int r, float alpha, uint16_t* Y, uint16_t* T_save,
-                          cudaStream_t st);
+                          cudaStream_t st, const float* Yadd = nullptr);
 constexpr int64_t kSmallMMax = 16;
 bool small_m_supported(int64_t K, int r);   // 0 <= rank <= 64 (0: no adapter), staging fits in smem
 int64_t lordba_ws_bytes(int64_t M, int64_t N, int64_t K, int r);   // lordba.cu
@@ -47,7 +49,7 @@ int64_t lordba_ws_bytes(int64_t M, int64_t N, int64_t K, int r);   // lordba.cu
 int64_t ext_fwd_ws_bytes(int64_t M, int64_t N, int64_t K, int64_t kext);
 ql_status ext_forward(const ql_weight* w, const uint16_t* X, int64_t M, const uint16_t* Zext,
                       const uint16_t* Wext, int64_t kext, uint16_t* Y, void* ws, size_t ws_bytes,
-                      cudaStream_t st);
+                      cudaStream_t st, const float* Yadd = nullptr);
 int64_t qwha_ws_bytes(int64_t M, int64_t N, int64_t K);             // qwha.cu
 int* device_flag_ptr();                 // device address of the sticky flag (current device)
 int num_sms();                          // SM count of the current device

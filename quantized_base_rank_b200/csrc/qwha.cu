@@ -5,18 +5,19 @@
 //
 // H is the orthonormal Sylvester-order Walsh-Hadamard matrix, block-diagonal in blocks of
 // b = the largest power of two dividing K (H = H^T = H^{-1}); F [N, K] is sparse, held as
-// compressed rows (row_ptr, col, c). The adapter stays unmerged: after the base product,
+// compressed rows (row_ptr, col, c). The adapter stays unmerged.
 //
 //  * qwha_wht_kernel forms Z = X H per token and block by the fast butterfly recursion,
-//    adds and subtracts only, in fp32 (the page's point: no multiplies by H), and writes
-//    it once as bf16 in a token-slab layout Zs[slab][k][16]: the 16 tokens of a slab are
-//    contiguous, so column k of a slab is one 32-byte sector;
-//  * qwha_spmm_kernel adds, for every output row n and token m,
-//    sum_j c_j Z[m, col_j] over row n's stored values, in fp32, into Y in place.
-//
-// The gather of Z by column index has no tensor-core form (F's positions are arbitrary),
-// so the second kernel runs on the FMA pipes, its slab of Z staged in shared memory when
-// it fits.
+//    adds and subtracts only, in fp32 (the page's point: no multiplies by H).
+//  * Decode-shaped calls (M <= 16): Z goes to one token slab Zs[k][16] (a column of the
+//    slab is one 32-byte sector); qwha_spmm_kernel gathers it by column index into fp32
+//    sums Yad[m, n] = sum_j c_j Z[m, col_j]; the decode-shaped base kernel adds Yad before
+//    its one bf16 rounding of Y.
+//  * Larger M: Z row-major; qwha_densify_kernel writes F as a dense bf16 [N, K] and the
+//    fused tcgen05 GEMM takes Z F^T as K/64 extension chunks, beside X W'^T. The gather
+//    has no tensor-core form (F's positions are arbitrary), and on the FMA pipes it needs
+//    a shared-memory read per multiply-add; the extension chunks are faster at the
+//    budgets of a rank-64 LoRA.
 #include <cmath>
 
 #include "common.cuh"
@@ -193,26 +194,33 @@ qwha_wht_kernel(const uint16_t* __restrict__ X, int64_t M, int64_t K, int L, int
 }
 
 // Decode-shaped sparse product (M <= 16, one slab of Z):
-//   Y[m, n] += sum_j c_j Z[m, col_j], j over row n's stored values.
+//   Yad[m, n] = sum_j c_j Z[m, col_j], j over row n's stored values (fp32, [M][N]),
+// which the decode-shaped base kernel then adds before its one bf16 rounding of Y.
 // One warp per row. Lane = (stream, token pair tp): TP = ceil(M / 2) token pairs and
 // 32 / TP streams, so at M <= 2 every lane takes its own value. A row's values are read
-// 32 per chunk and four chunks at a time (one (col, c) pair per lane and chunk, all four
-// loads issued together), handed to the streams by shuffles; each lane gathers the two
-// tokens' Z values of its value (one 4-byte load) and keeps their fp32 sums. The streams
-// are combined by a fixed xor butterfly (the result does not depend on scheduling) and
-// added to the base product with one bf16 rounding. Columns at or past K, or row offsets
+// 32 per chunk and U chunks at a time (one (col, c) pair per lane and chunk, all loads
+// issued together), handed to the streams by shuffles; each lane gathers the two tokens'
+// Z values of its value (one 4-byte load) and keeps their fp32 sums. The streams are
+// combined by a fixed xor butterfly (the result does not depend on scheduling).
+//
+// It runs as a programmatic dependent of the transform. The transform is launched without
+// programmatic serialisation, so every grid before it has completed when this one starts:
+// the row offsets and the first chunks of (col, c) are loaded before the dependency wait,
+// and only Z, which the transform writes, after it. Columns at or past K, or row offsets
 // outside [0, nnz], are skipped and raise the device's bad-index flag.
 template <int TP>
 __global__ void __launch_bounds__(256)
 qwha_spmm_kernel(const uint16_t* __restrict__ Zs, int64_t M, int64_t N, int64_t K,
                  const int32_t* __restrict__ row_ptr, const uint16_t* __restrict__ col,
-                 const uint16_t* __restrict__ cval, int64_t nnz, uint16_t* __restrict__ Y, int* flag) {
+                 const uint16_t* __restrict__ cval, int64_t nnz, float* __restrict__ Yad, int* flag) {
   constexpr int NS = 32 / TP;                        // streams
-  constexpr int U = 4;                               // chunks in flight
+  constexpr int U = TP <= 2 ? 16 : (TP == 4 ? 8 : 4);   // chunks in flight: 512, 256 or 128 values
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int lane = threadIdx.x & 31;
   const int stream = lane / TP, tp = lane % TP;
   const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   bool bad = false;
+  bool waited = false;
   for (int64_t n = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; n < N; n += warps) {
     int j0 = __ldg(row_ptr + n), j1 = __ldg(row_ptr + n + 1);
     if (j0 < 0 || (int64_t)j1 > nnz || j0 > j1) {
@@ -231,6 +239,10 @@ qwha_spmm_kernel(const uint16_t* __restrict__ Zs, int64_t M, int64_t N, int64_t 
           bad = true;
           wv[u] = 0u;
         }
+      }
+      if (!waited) {                                 // Z is the transform's output
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        waited = true;
       }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
@@ -252,8 +264,8 @@ qwha_spmm_kernel(const uint16_t* __restrict__ Zs, int64_t M, int64_t N, int64_t 
     }
     if (stream == 0) {
       const int64_t m = 2 * tp;
-      if (m < M) Y[m * N + n] = float_to_bf16_bits(bf16_lo(Y[m * N + n]) + a0);
-      if (m + 1 < M) Y[(m + 1) * N + n] = float_to_bf16_bits(bf16_lo(Y[(m + 1) * N + n]) + a1);
+      if (m < M) Yad[m * N + n] = a0;
+      if (m + 1 < M) Yad[(m + 1) * N + n] = a1;
     }
   }
   if (bad) raise_flag(flag, kFlagBadIndex);
@@ -327,10 +339,10 @@ static size_t wht_smem(int64_t b, int64_t bs, int tt) {
 
 static bool qwha_decode_shaped(int64_t M, int64_t K) { return M <= kSmallMMax && small_m_supported(K, 0); }
 
-// Workspace: decode-shaped, the one slab of Z; otherwise Z [M, K] and the dense F [N, K]
-// (bf16) plus the fused GEMM's scratch.
+// Workspace: decode-shaped, the one slab of Z and the fp32 sparse sums [M][N]; otherwise
+// Z [M, K] and the dense F [N, K] (bf16) plus the fused GEMM's scratch.
 int64_t qwha_ws_bytes(int64_t M, int64_t N, int64_t K) {
-  if (qwha_decode_shaped(M, K)) return round_up(K * kQwSlab * 2, 256);
+  if (qwha_decode_shaped(M, K)) return round_up(K * kQwSlab * 2, 256) + round_up(M * N * 4, 256);
   return round_up(M * K * 2, 256) + round_up(N * K * 2, 256) + ext_fwd_ws_bytes(M, N, K, K);
 }
 
@@ -383,25 +395,44 @@ ql_status qlora_linear_fwd_qwha(const ql_weight* w, const ql_bf16* X, int64_t M,
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   ql_status e;
   if (qwha_decode_shaped(M, K)) {
-    // the base product (decode-shaped kernel), then Z = X H and the sparse product
+    // Z = X H, then the sparse sums into fp32 Yad (a programmatic dependent of the
+    // transform), then the decode-shaped base product, which adds Yad before rounding
+    // (a programmatic dependent of the sparse product: it warms L2 with its weight while
+    // the two run)
     uint16_t* Zs = reinterpret_cast<uint16_t*>(wsb);
-    e = ext_forward(w, X, M, nullptr, nullptr, 0, Y, nullptr, 0, st);
-    if (e != QL_OK) return e;
-    ProfScope prof(PK_FWD_ADAPTER, st, 2);
-    e = launch_wht<true>(X, M, K, Zs, st);
-    if (e != QL_OK || f->nnz == 0) return e;
-    const unsigned grid = (unsigned)imin64((N + 7) / 8, (int64_t)num_sms() * 8);   // a warp per row
-    const int tp = (int)((M + 1) / 2);
-    if (tp <= 1)
-      qwha_spmm_kernel<1><<<grid, 256, 0, st>>>(Zs, M, N, K, f->row_ptr, f->col, f->c, f->nnz, Y, device_flag_ptr());
-    else if (tp <= 2)
-      qwha_spmm_kernel<2><<<grid, 256, 0, st>>>(Zs, M, N, K, f->row_ptr, f->col, f->c, f->nnz, Y, device_flag_ptr());
-    else if (tp <= 4)
-      qwha_spmm_kernel<4><<<grid, 256, 0, st>>>(Zs, M, N, K, f->row_ptr, f->col, f->c, f->nnz, Y, device_flag_ptr());
-    else
-      qwha_spmm_kernel<8><<<grid, 256, 0, st>>>(Zs, M, N, K, f->row_ptr, f->col, f->c, f->nnz, Y, device_flag_ptr());
-    QL_CHECK_LAUNCH();
-    return QL_OK;
+    float* Yad = reinterpret_cast<float*>(wsb + round_up(K * kQwSlab * 2, 256));
+    {
+      ProfScope prof(PK_FWD_ADAPTER, st, 2);
+      e = launch_wht<true>(X, M, K, Zs, st);
+      if (e != QL_OK) return e;
+      const unsigned grid = (unsigned)imin64((N + 7) / 8, (int64_t)num_sms() * 8);   // a warp per row
+      const int tp = (int)((M + 1) / 2);
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(grid);
+      cfg.blockDim = dim3(256);
+      cfg.stream = st;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int* flag = device_flag_ptr();
+      const int32_t* rp = f->row_ptr;
+      const uint16_t* cl = f->col;
+      const uint16_t* cv = reinterpret_cast<const uint16_t*>(f->c);
+      cudaError_t ce;
+      if (tp <= 1)
+        ce = cudaLaunchKernelEx(&cfg, qwha_spmm_kernel<1>, (const uint16_t*)Zs, M, N, K, rp, cl, cv, f->nnz, Yad, flag);
+      else if (tp <= 2)
+        ce = cudaLaunchKernelEx(&cfg, qwha_spmm_kernel<2>, (const uint16_t*)Zs, M, N, K, rp, cl, cv, f->nnz, Yad, flag);
+      else if (tp <= 4)
+        ce = cudaLaunchKernelEx(&cfg, qwha_spmm_kernel<4>, (const uint16_t*)Zs, M, N, K, rp, cl, cv, f->nnz, Yad, flag);
+      else
+        ce = cudaLaunchKernelEx(&cfg, qwha_spmm_kernel<8>, (const uint16_t*)Zs, M, N, K, rp, cl, cv, f->nnz, Yad, flag);
+      if (ce != cudaSuccess) return QL_ERR_CUDA;
+      QL_CHECK_LAUNCH();
+    }
+    return ext_forward(w, X, M, nullptr, nullptr, 0, Y, nullptr, 0, st, Yad);
   }
   // tensor cores: Y = [X | Z] [W' | F]^T, the adapter as K extension chunks of the fused GEMM
   uint16_t* Z = reinterpret_cast<uint16_t*>(wsb);

@@ -35,6 +35,7 @@ struct SmallArgs {
   const uint8_t* codes; const int8_t* qabsmax; const float* gscale; const float* mean;
   const float* absmax;
   uint16_t* Y; uint16_t* T_save;
+  const float* Yadd;               // optional fp32 [M][N] added before the bf16 rounding of Y
   int kr_max;                      // max K-range per CTA, in elements
   int b_pairs;                     // r even and B 4-byte aligned
   float q[16];
@@ -238,6 +239,8 @@ small_m_fwd_kernel(const SmallArgs a) {
     l2_prefetch_rows(a.A, a.K * 2, a.r, k0 * 2, kend * 2, t, 256);
     l2_prefetch_rows(a.B + n0 * a.r, 0, 1, 0, rows * a.r * 2, t, 256);
     l2_prefetch_rows(a.X, a.K * 2, a.M < NT ? a.M : NT, k0 * 2, kend * 2, t, 256);
+    if (a.Yadd && rank == 0)
+      l2_prefetch_rows(a.Yadd + n0, a.N * 4, a.M < NT ? a.M : NT, 0, rows * 4, t, 256);
   }
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const float mu = FMT == QL_FMT_NF4_DQ ? __ldg(a.mean) : 0.0f;
@@ -436,7 +439,10 @@ small_m_fwd_kernel(const SmallArgs a) {
 #pragma unroll
       for (int c = 0; c < kCS; ++c) acc += part[c];
       const int64_t row = n0 + rr;
-      if (tok < a.M && row < a.N) a.Y[tok * a.N + row] = (uint16_t)float_to_bf16_bits(acc);
+      if (tok < a.M && row < a.N) {
+        if (a.Yadd) acc += a.Yadd[tok * a.N + row];
+        a.Y[tok * a.N + row] = (uint16_t)float_to_bf16_bits(acc);
+      }
     }
     if (a.T_save && blockIdx.x < (unsigned)kCS) {        // first cluster also reduces T
       for (int i = threadIdx.x; i < RP * NT; i += blockDim.x) {
@@ -497,8 +503,9 @@ bool small_m_supported(int64_t K, int r) {
 // Host entry used by qlora_linear_fwd when M <= 16.
 ql_status small_m_forward(const ql_weight* w, const uint16_t* X, int64_t M, const uint16_t* A,
                           const uint16_t* B, int r, float alpha, uint16_t* Y, uint16_t* T_save,
-                          cudaStream_t st) {
+                          cudaStream_t st, const float* Yadd) {
   SmallArgs a{};
+  a.Yadd = Yadd;
   a.X = X; a.A = A; a.B = B; a.M = M; a.N = w->N; a.K = w->K; a.r = r; a.s = r > 0 ? alpha / (float)r : 0.0f;
   a.fmt = w->fmt;
   a.codes = static_cast<const uint8_t*>(w->codes);
