@@ -35,11 +35,21 @@ struct Nf4BoundTable {
 const Nf4BoundTable& nf4_bound_table();  // host, computed on first use
 
 // Decode-shaped forward (M <= 16), small_m.cu.
-// Yadd (optional, fp32 [M][N]) is added to the product before its bf16 rounding; it may be
-// written by the grid just before on the stream (it is read after the dependency wait).
+// A Walsh-Hadamard adapter's rows of F (compressed rows) and the transformed tokens Zs
+// ([K][16] bf16, token-contiguous) for the decode-shaped kernel.
+struct QwhaRows {
+  const int32_t* row_ptr;
+  const uint16_t* col;
+  const uint16_t* c;
+  int64_t nnz;
+  const uint16_t* Zs;
+};
+// qw (optional, r = 0 only): the adapter's sparse sums are added before Y's rounding; Zs
+// may be written by the grid just before on the stream (it is read after the dependency
+// wait), provided that grid was launched without programmatic serialisation.
 ql_status small_m_forward(const ql_weight* w, const uint16_t* X, int64_t M, const uint16_t* A,
                           const uint16_t* B, int r, float alpha, uint16_t* Y, uint16_t* T_save,
-                          cudaStream_t st, const float* Yadd = nullptr);
+                          cudaStream_t st, const QwhaRows* qw = nullptr);
 constexpr int64_t kSmallMMax = 16;
 bool small_m_supported(int64_t K, int r);   // 0 <= rank <= 64 (0: no adapter), staging fits in smem
 int64_t lordba_ws_bytes(int64_t M, int64_t N, int64_t K, int r);   // lordba.cu
@@ -49,7 +59,7 @@ int64_t lordba_ws_bytes(int64_t M, int64_t N, int64_t K, int r);   // lordba.cu
 int64_t ext_fwd_ws_bytes(int64_t M, int64_t N, int64_t K, int64_t kext);
 ql_status ext_forward(const ql_weight* w, const uint16_t* X, int64_t M, const uint16_t* Zext,
                       const uint16_t* Wext, int64_t kext, uint16_t* Y, void* ws, size_t ws_bytes,
-                      cudaStream_t st, const float* Yadd = nullptr);
+                      cudaStream_t st, const QwhaRows* qw = nullptr);
 int64_t qwha_ws_bytes(int64_t M, int64_t N, int64_t K);             // qwha.cu
 int* device_flag_ptr();                 // device address of the sticky flag (current device)
 int num_sms();                          // SM count of the current device

@@ -325,8 +325,8 @@ static ql_status check_weight(const ql_weight* w) {
 // Y = X deq(W)^T + Zext Wext^T, with Zext [M, kext] and Wext [N, kext] bf16 row-major
 // (kext a multiple of 64, 0 for the base product alone): the fused GEMM of the forward,
 // its extension chunks taken from the caller's operands. M <= 16 with kext = 0 runs the
-// decode-shaped kernel without its adapter part, adding Yadd (fp32 [M][N], optional)
-// before the rounding. The only scratch is the block-scale copy.
+// decode-shaped kernel without its adapter part, adding a Walsh-Hadamard adapter's sparse
+// sums when qw is given. The only scratch is the block-scale copy.
 int64_t ext_fwd_ws_bytes(int64_t M, int64_t N, int64_t K, int64_t kext) {
   if (kext == 0 && M <= kSmallMMax && small_m_supported(K, 0)) return 0;
   return round_up((K / 64) * N * 4, 256);
@@ -334,7 +334,7 @@ int64_t ext_fwd_ws_bytes(int64_t M, int64_t N, int64_t K, int64_t kext) {
 
 ql_status ext_forward(const ql_weight* w, const uint16_t* X, int64_t M, const uint16_t* Zext,
                       const uint16_t* Wext, int64_t kext, uint16_t* Y, void* ws, size_t ws_bytes,
-                      cudaStream_t st, const float* Yadd) {
+                      cudaStream_t st, const QwhaRows* qw) {
   ql_status e = check_weight(w);
   if (e != QL_OK) return e;
   if (!X || !Y || M < 1 || !aligned(X, 16) || !aligned(Y, 16)) return QL_ERR_INVALID_ARG;
@@ -343,8 +343,8 @@ ql_status ext_forward(const ql_weight* w, const uint16_t* X, int64_t M, const ui
   if (M > (int64_t(1) << 31)) return QL_ERR_UNSUPPORTED;
   const int64_t N = w->N, K = w->K;
   if (kext == 0 && M <= kSmallMMax && small_m_supported(K, 0))
-    return small_m_forward(w, X, M, nullptr, nullptr, 0, 0.0f, Y, nullptr, st, Yadd);
-  if (Yadd) return QL_ERR_UNSUPPORTED;              // the addend exists on the decode-shaped path only
+    return small_m_forward(w, X, M, nullptr, nullptr, 0, 0.0f, Y, nullptr, st, qw);
+  if (qw) return QL_ERR_UNSUPPORTED;                // the sparse sums exist on the decode-shaped path only
   if (!ws || !aligned(ws, 256)) return QL_ERR_INVALID_ARG;
   if ((int64_t)ws_bytes < ext_fwd_ws_bytes(M, N, K, kext)) return QL_ERR_WORKSPACE;
   float* scales = static_cast<float*>(ws);

@@ -10,9 +10,9 @@
 //  * qwha_wht_kernel forms Z = X H per token and block by the fast butterfly recursion,
 //    adds and subtracts only, in fp32 (the page's point: no multiplies by H).
 //  * Decode-shaped calls (M <= 16): Z goes to one token slab Zs[k][16] (a column of the
-//    slab is one 32-byte sector); qwha_spmm_kernel gathers it by column index into fp32
-//    sums Yad[m, n] = sum_j c_j Z[m, col_j]; the decode-shaped base kernel adds Yad before
-//    its one bf16 rounding of Y.
+//    slab is one 32-byte sector); the decode-shaped base kernel gathers it by column index
+//    for its rows (sum_j c_j Z[m, col_j]) and adds the sums before the cluster reduction,
+//    so they reach Y with its one bf16 rounding (small_m.cu, qwha_rows_add).
 //  * Larger M: Z row-major; qwha_densify_kernel writes F as a dense bf16 [N, K] and the
 //    fused tcgen05 GEMM takes Z F^T as K/64 extension chunks, beside X W'^T. The gather
 //    has no tensor-core form (F's positions are arbitrary), and on the FMA pipes it needs
@@ -128,6 +128,9 @@ qwha_wht_kernel(const uint16_t* __restrict__ X, int64_t M, int64_t K, int L, int
   const int j = (int)(blockIdx.y & ((1u << SL) - 1));
   const int64_t kblk = (int64_t)(blockIdx.y >> SL) << L;
   const int S = 1 << SL;
+  // the next grid (the decode-shaped base kernel) may start now and warm L2 with its own
+  // inputs; it waits for this grid before reading Z
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // the raw bf16 input tile [TT][b] sits after the fp32 rows; every thread issues all of
   // its 16-byte copies before any is waited for (tokens past M are zero-filled)
   uint16_t* raw = reinterpret_cast<uint16_t*>(wsm + (size_t)TT * pitch);
@@ -191,84 +194,6 @@ qwha_wht_kernel(const uint16_t* __restrict__ X, int64_t M, int64_t K, int L, int
       smem_pass_n<true, SLAB>(nb, wsm, TT, bs, pitch, lo, scale, Z, m0, M, K, kbase);
     }
   }
-}
-
-// Decode-shaped sparse product (M <= 16, one slab of Z):
-//   Yad[m, n] = sum_j c_j Z[m, col_j], j over row n's stored values (fp32, [M][N]),
-// which the decode-shaped base kernel then adds before its one bf16 rounding of Y.
-// One warp per row. Lane = (stream, token pair tp): TP = ceil(M / 2) token pairs and
-// 32 / TP streams, so at M <= 2 every lane takes its own value. A row's values are read
-// 32 per chunk and U chunks at a time (one (col, c) pair per lane and chunk, all loads
-// issued together), handed to the streams by shuffles; each lane gathers the two tokens'
-// Z values of its value (one 4-byte load) and keeps their fp32 sums. The streams are
-// combined by a fixed xor butterfly (the result does not depend on scheduling).
-//
-// It runs as a programmatic dependent of the transform. The transform is launched without
-// programmatic serialisation, so every grid before it has completed when this one starts:
-// the row offsets and the first chunks of (col, c) are loaded before the dependency wait,
-// and only Z, which the transform writes, after it. Columns at or past K, or row offsets
-// outside [0, nnz], are skipped and raise the device's bad-index flag.
-template <int TP>
-__global__ void __launch_bounds__(256)
-qwha_spmm_kernel(const uint16_t* __restrict__ Zs, int64_t M, int64_t N, int64_t K,
-                 const int32_t* __restrict__ row_ptr, const uint16_t* __restrict__ col,
-                 const uint16_t* __restrict__ cval, int64_t nnz, float* __restrict__ Yad, int* flag) {
-  constexpr int NS = 32 / TP;                        // streams
-  constexpr int U = TP <= 2 ? 16 : (TP == 4 ? 8 : 4);   // chunks in flight: 512, 256 or 128 values
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int lane = threadIdx.x & 31;
-  const int stream = lane / TP, tp = lane % TP;
-  const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  bool bad = false;
-  bool waited = false;
-  for (int64_t n = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; n < N; n += warps) {
-    int j0 = __ldg(row_ptr + n), j1 = __ldg(row_ptr + n + 1);
-    if (j0 < 0 || (int64_t)j1 > nnz || j0 > j1) {
-      bad = true;
-      j0 = j1 = 0;
-    }
-    float a0 = 0.0f, a1 = 0.0f;
-    for (int jc = j0; jc < j1; jc += 32 * U) {
-      const int nch = (j1 - jc + 31) >> 5;           // chunks of this batch that hold values
-      uint32_t wv[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int jj = jc + 32 * u + lane;
-        wv[u] = jj < j1 ? (uint32_t)__ldg(col + jj) | ((uint32_t)__ldg(cval + jj) << 16) : 0u;
-        if ((int64_t)(wv[u] & 0xFFFFu) >= K) {
-          bad = true;
-          wv[u] = 0u;
-        }
-      }
-      if (!waited) {                                 // Z is the transform's output
-        asm volatile("griddepcontrol.wait;" ::: "memory");
-        waited = true;
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        if (u >= nch) break;                         // warp-uniform
-#pragma unroll
-        for (int it = 0; it < TP; ++it) {
-          const uint32_t we = __shfl_sync(0xffffffffu, wv[u], it * NS + stream);
-          const uint32_t z = __ldg(reinterpret_cast<const uint32_t*>(Zs + (size_t)(we & 0xFFFFu) * kQwSlab) + tp);
-          const float cv = __uint_as_float(we & 0xFFFF0000u);
-          a0 = fmaf(cv, bf16_lo(z), a0);
-          a1 = fmaf(cv, bf16_hi(z), a1);
-        }
-      }
-    }
-#pragma unroll
-    for (int off = TP; off < 32; off <<= 1) {
-      a0 += __shfl_xor_sync(0xffffffffu, a0, off);
-      a1 += __shfl_xor_sync(0xffffffffu, a1, off);
-    }
-    if (stream == 0) {
-      const int64_t m = 2 * tp;
-      if (m < M) Yad[m * N + n] = a0;
-      if (m + 1 < M) Yad[(m + 1) * N + n] = a1;
-    }
-  }
-  if (bad) raise_flag(flag, kFlagBadIndex);
 }
 
 // F written out densely for the tensor cores: Fd [N, K] bf16 holds c_j at (n, col_j) and
@@ -339,10 +264,10 @@ static size_t wht_smem(int64_t b, int64_t bs, int tt) {
 
 static bool qwha_decode_shaped(int64_t M, int64_t K) { return M <= kSmallMMax && small_m_supported(K, 0); }
 
-// Workspace: decode-shaped, the one slab of Z and the fp32 sparse sums [M][N]; otherwise
-// Z [M, K] and the dense F [N, K] (bf16) plus the fused GEMM's scratch.
+// Workspace: decode-shaped, the one slab of Z; otherwise Z [M, K] and the dense F [N, K]
+// (bf16) plus the fused GEMM's scratch.
 int64_t qwha_ws_bytes(int64_t M, int64_t N, int64_t K) {
-  if (qwha_decode_shaped(M, K)) return round_up(K * kQwSlab * 2, 256) + round_up(M * N * 4, 256);
+  if (qwha_decode_shaped(M, K)) return round_up(K * kQwSlab * 2, 256);
   return round_up(M * K * 2, 256) + round_up(N * K * 2, 256) + ext_fwd_ws_bytes(M, N, K, K);
 }
 
@@ -395,44 +320,18 @@ ql_status qlora_linear_fwd_qwha(const ql_weight* w, const ql_bf16* X, int64_t M,
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   ql_status e;
   if (qwha_decode_shaped(M, K)) {
-    // Z = X H, then the sparse sums into fp32 Yad (a programmatic dependent of the
-    // transform), then the decode-shaped base product, which adds Yad before rounding
-    // (a programmatic dependent of the sparse product: it warms L2 with its weight while
-    // the two run)
+    // Z = X H into one token slab, then the decode-shaped base kernel, which adds the
+    // sparse sums of its rows before the cluster reduction (a programmatic dependent of
+    // the transform: it warms L2 with its weight and its rows of F while the transform
+    // runs)
     uint16_t* Zs = reinterpret_cast<uint16_t*>(wsb);
-    float* Yad = reinterpret_cast<float*>(wsb + round_up(K * kQwSlab * 2, 256));
     {
-      ProfScope prof(PK_FWD_ADAPTER, st, 2);
+      ProfScope prof(PK_FWD_ADAPTER, st, 1);
       e = launch_wht<true>(X, M, K, Zs, st);
       if (e != QL_OK) return e;
-      const unsigned grid = (unsigned)imin64((N + 7) / 8, (int64_t)num_sms() * 8);   // a warp per row
-      const int tp = (int)((M + 1) / 2);
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(grid);
-      cfg.blockDim = dim3(256);
-      cfg.stream = st;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-      attr[0].val.programmaticStreamSerializationAllowed = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      int* flag = device_flag_ptr();
-      const int32_t* rp = f->row_ptr;
-      const uint16_t* cl = f->col;
-      const uint16_t* cv = reinterpret_cast<const uint16_t*>(f->c);
-      cudaError_t ce;
-      if (tp <= 1)
-        ce = cudaLaunchKernelEx(&cfg, qwha_spmm_kernel<1>, (const uint16_t*)Zs, M, N, K, rp, cl, cv, f->nnz, Yad, flag);
-      else if (tp <= 2)
-        ce = cudaLaunchKernelEx(&cfg, qwha_spmm_kernel<2>, (const uint16_t*)Zs, M, N, K, rp, cl, cv, f->nnz, Yad, flag);
-      else if (tp <= 4)
-        ce = cudaLaunchKernelEx(&cfg, qwha_spmm_kernel<4>, (const uint16_t*)Zs, M, N, K, rp, cl, cv, f->nnz, Yad, flag);
-      else
-        ce = cudaLaunchKernelEx(&cfg, qwha_spmm_kernel<8>, (const uint16_t*)Zs, M, N, K, rp, cl, cv, f->nnz, Yad, flag);
-      if (ce != cudaSuccess) return QL_ERR_CUDA;
-      QL_CHECK_LAUNCH();
     }
-    return ext_forward(w, X, M, nullptr, nullptr, 0, Y, nullptr, 0, st, Yad);
+    const QwhaRows rows{f->row_ptr, f->col, reinterpret_cast<const uint16_t*>(f->c), f->nnz, Zs};
+    return ext_forward(w, X, M, nullptr, nullptr, 0, Y, nullptr, 0, st, &rows);
   }
   // tensor cores: Y = [X | Z] [W' | F]^T, the adapter as K extension chunks of the fused GEMM
   uint16_t* Z = reinterpret_cast<uint16_t*>(wsb);

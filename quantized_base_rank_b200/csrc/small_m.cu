@@ -35,7 +35,11 @@ struct SmallArgs {
   const uint8_t* codes; const int8_t* qabsmax; const float* gscale; const float* mean;
   const float* absmax;
   uint16_t* Y; uint16_t* T_save;
-  const float* Yadd;               // optional fp32 [M][N] added before the bf16 rounding of Y
+  // Walsh-Hadamard adapter (QW instantiations): F in compressed rows and the transformed
+  // tokens Zs [K][16] (bf16, token-contiguous), written by the grid just before
+  const int32_t* q_row_ptr; const uint16_t* q_col; const uint16_t* q_c; int64_t q_nnz;
+  const uint16_t* q_Zs;
+  int* flag;                       // the device status flag (bad sparse indices)
   int kr_max;                      // max K-range per CTA, in elements
   int b_pairs;                     // r even and B 4-byte aligned
   float q[16];
@@ -191,7 +195,107 @@ __device__ __forceinline__ float ld_cluster_f32(const float* local, uint32_t ran
 // bytes, the 16 lanes of a half-warp (rows g = 0..3, q = 0..3) hit 16 different bank pairs.
 __host__ __device__ __forceinline__ int small_row_pitch(int units) { return units * 512 + 32; }
 
-template <int NT, int FMT, int JT>
+// Adds sum_j c_j Zs[col_j][tok] over each of the 16 rows [r0, r0 + 16) of F (compressed
+// rows) to out[(row - r0) * NT + tok] for the NT tokens. Each warp takes two rows, and the
+// first batch of both is requested before either is used. Lane = (stream, token pair tp),
+// NT/2 token pairs and 64/NT streams; a row's values are read 32 per chunk, U chunks at a
+// time, and handed to the streams by shuffles; each lane gathers
+// its value's two tokens (one 4-byte load from the token-contiguous Zs) and keeps their
+// fp32 sums; a fixed xor butterfly combines the streams. Columns at or past K and row
+// offsets outside [0, nnz] are skipped and raise the bad-index flag. Call after the
+// dependency wait (Zs is the previous grid's output) and a __syncthreads.
+template <int NT>
+__device__ __forceinline__ void qwha_rows_add(const SmallArgs& a, int64_t r0, float* out) {
+  constexpr int TP = NT / 2, NS = 32 / TP;
+  constexpr int U = NT == 8 ? 8 : 4;                 // chunks in flight per row: 256 / 128 values
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int stream = lane / TP, tp = lane % TP;
+  bool bad = false;
+  // the warp's two rows: bounds, then the first batch of both rows, before any is used
+  int jb[2], je[2];
+  uint32_t wv[2][U];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int64_t n = r0 + 2 * warp + i;
+    jb[i] = je[i] = 0;
+    if (n < a.N) {
+      jb[i] = __ldg(a.q_row_ptr + n);
+      je[i] = __ldg(a.q_row_ptr + n + 1);
+      if (jb[i] < 0 || (int64_t)je[i] > a.q_nnz || jb[i] > je[i]) {
+        bad = true;
+        jb[i] = je[i] = 0;
+      }
+    }
+  }
+  auto load_batch = [&](int i, int jc, uint32_t (&w)[U]) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int jj = jc + 32 * u + lane;
+      w[u] = jj < je[i] ? (uint32_t)__ldg(a.q_col + jj) | ((uint32_t)__ldg(a.q_c + jj) << 16) : 0u;
+      if ((int64_t)(w[u] & 0xFFFFu) >= a.K) {
+        bad = true;
+        w[u] = 0u;
+      }
+    }
+  };
+  load_batch(0, jb[0], wv[0]);
+  load_batch(1, jb[1], wv[1]);
+  // the gathers of CH chunks, all issued before any is used (a value of 0 gathers column 0
+  // and adds nothing)
+  auto gather = [&](const uint32_t* w, int CHn, float& a0, float& a1) {
+    uint32_t z[U * TP];
+    uint32_t we[U * TP];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+#pragma unroll
+      for (int it = 0; it < TP; ++it) {
+        if (u < CHn) {
+          we[u * TP + it] = __shfl_sync(0xffffffffu, w[u], it * NS + stream);
+          z[u * TP + it] =
+              __ldg(reinterpret_cast<const uint32_t*>(a.q_Zs + (size_t)(we[u * TP + it] & 0xFFFFu) * 16) + tp);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+#pragma unroll
+      for (int it = 0; it < TP; ++it) {
+        if (u < CHn) {
+          const float cv = __uint_as_float(we[u * TP + it] & 0xFFFF0000u);
+          a0 = fmaf(cv, __uint_as_float(z[u * TP + it] << 16), a0);
+          a1 = fmaf(cv, __uint_as_float(z[u * TP + it] & 0xFFFF0000u), a1);
+        }
+      }
+    }
+  };
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    float a0 = 0.0f, a1 = 0.0f;
+    for (int jc = jb[i]; jc < je[i]; jc += 32 * U) {
+      if (jc != jb[i]) load_batch(i, jc, wv[i]);
+      // warp-uniform: a short batch (most rows) takes the two-chunk form
+      if (je[i] - jc <= 64) gather(wv[i], 2, a0, a1);
+      else gather(wv[i], U, a0, a1);
+    }
+#pragma unroll
+    for (int off = TP; off < 32; off <<= 1) {
+      a0 += __shfl_xor_sync(0xffffffffu, a0, off);
+      a1 += __shfl_xor_sync(0xffffffffu, a1, off);
+    }
+    const int rr = 2 * warp + i;
+    if (stream == 0 && r0 + rr < a.N) {
+      out[rr * NT + 2 * tp] += a0;
+      out[rr * NT + 2 * tp + 1] += a1;
+    }
+  }
+  if (bad) raise_flag(a.flag, kFlagBadIndex);
+}
+
+// QW: the Walsh-Hadamard adapter's sparse sums (QWHA page, gist.science/ko/paper/2509.17428,
+// section 2.1: Delta W x = F (H^{-1} x)) for the 16 rows this CTA reduces are added to its
+// partial sums before the cluster reduction, so they reach Y with its one rounding. Only
+// with JT = 0 (no LoRA part).
+template <int NT, int FMT, int JT, bool QW = false>
 __global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(256, 2)
 small_m_fwd_kernel(const SmallArgs a) {
   constexpr int NTT = NT / 8;                       // token tiles of 8
@@ -239,8 +343,22 @@ small_m_fwd_kernel(const SmallArgs a) {
     l2_prefetch_rows(a.A, a.K * 2, a.r, k0 * 2, kend * 2, t, 256);
     l2_prefetch_rows(a.B + n0 * a.r, 0, 1, 0, rows * a.r * 2, t, 256);
     l2_prefetch_rows(a.X, a.K * 2, a.M < NT ? a.M : NT, k0 * 2, kend * 2, t, 256);
-    if (a.Yadd && rank == 0)
-      l2_prefetch_rows(a.Yadd + n0, a.N * 4, a.M < NT ? a.M : NT, 0, rows * 4, t, 256);
+    if (QW) {
+      // this CTA's rows of F: the offsets, then the values they bound. The grid before
+      // this one (the transform) never writes F, and it is launched without programmatic
+      // serialisation, so everything that wrote F has completed: reading two offsets
+      // here is safe. Only Zs waits.
+      const int64_t r0 = n0 + rank * (kRowsPerCta / kCS);
+      const int64_t r1 = imin64(r0 + kRowsPerCta / kCS, a.N);
+      if (r0 < r1) {
+        l2_prefetch_rows(a.q_row_ptr + r0, 0, 1, 0, (r1 - r0 + 1) * 4, t, 256);
+        const int64_t j0 = __ldg(a.q_row_ptr + r0), j1 = __ldg(a.q_row_ptr + r1);
+        if (j0 >= 0 && j1 <= a.q_nnz && j0 < j1) {
+          l2_prefetch_rows(a.q_col, 0, 1, j0 * 2, j1 * 2, t, 256);
+          l2_prefetch_rows(a.q_c, 0, 1, j0 * 2, j1 * 2, t, 256);
+        }
+      }
+    }
   }
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const float mu = FMT == QL_FMT_NF4_DQ ? __ldg(a.mean) : 0.0f;
@@ -427,6 +545,10 @@ small_m_fwd_kernel(const SmallArgs a) {
     sD[(rg + 8) * NT + t * 8 + 2 * q] = d[t][2];
     sD[(rg + 8) * NT + t * 8 + 2 * q + 1] = d[t][3];
   }
+  if (QW) {
+    __syncthreads();
+    qwha_rows_add<NT>(a, n0 + rank * (kRowsPerCta / kCS), sD + (size_t)rank * (kRowsPerCta / kCS) * NT);
+  }
   cluster_sync_all();
   {
     constexpr int kRowsPerRank = kRowsPerCta / kCS;    // 16
@@ -439,10 +561,7 @@ small_m_fwd_kernel(const SmallArgs a) {
 #pragma unroll
       for (int c = 0; c < kCS; ++c) acc += part[c];
       const int64_t row = n0 + rr;
-      if (tok < a.M && row < a.N) {
-        if (a.Yadd) acc += a.Yadd[tok * a.N + row];
-        a.Y[tok * a.N + row] = (uint16_t)float_to_bf16_bits(acc);
-      }
+      if (tok < a.M && row < a.N) a.Y[tok * a.N + row] = (uint16_t)float_to_bf16_bits(acc);
     }
     if (a.T_save && blockIdx.x < (unsigned)kCS) {        // first cluster also reduces T
       for (int i = threadIdx.x; i < RP * NT; i += blockDim.x) {
@@ -467,9 +586,9 @@ size_t small_m_smem(int NT, int units_max, int r) {
   return (size_t)(NT + RP) * small_row_pitch(units_max) + (size_t)(8 * RP * NT + kRowsPerCta * NT) * 4;
 }
 
-template <int NT, int FMT, int JT>
+template <int NT, int FMT, int JT, bool QW = false>
 static ql_status launch_small(const SmallArgs& a, cudaStream_t st) {
-  auto kern = small_m_fwd_kernel<NT, FMT, JT>;
+  auto kern = small_m_fwd_kernel<NT, FMT, JT, QW>;
   SmallArgs b = a;
   const size_t smem = small_m_smem(NT, a.kr_max / 256, JT * 16);
   if (smem > 227 * 1024) return QL_ERR_UNSUPPORTED;
@@ -503,9 +622,13 @@ bool small_m_supported(int64_t K, int r) {
 // Host entry used by qlora_linear_fwd when M <= 16.
 ql_status small_m_forward(const ql_weight* w, const uint16_t* X, int64_t M, const uint16_t* A,
                           const uint16_t* B, int r, float alpha, uint16_t* Y, uint16_t* T_save,
-                          cudaStream_t st, const float* Yadd) {
+                          cudaStream_t st, const QwhaRows* qw) {
   SmallArgs a{};
-  a.Yadd = Yadd;
+  a.flag = device_flag_ptr();
+  if (qw) {
+    if (r != 0) return QL_ERR_UNSUPPORTED;
+    a.q_row_ptr = qw->row_ptr; a.q_col = qw->col; a.q_c = qw->c; a.q_nnz = qw->nnz; a.q_Zs = qw->Zs;
+  }
   a.X = X; a.A = A; a.B = B; a.M = M; a.N = w->N; a.K = w->K; a.r = r; a.s = r > 0 ? alpha / (float)r : 0.0f;
   a.fmt = w->fmt;
   a.codes = static_cast<const uint8_t*>(w->codes);
@@ -520,6 +643,11 @@ ql_status small_m_forward(const ql_weight* w, const uint16_t* X, int64_t M, cons
   if (r < 0 || r > 64) return QL_ERR_UNSUPPORTED;
   const int jt = (r + 15) / 16;
   const bool nf4 = w->fmt == QL_FMT_NF4_DQ;
+  if (jt == 0 && qw) {                             // no LoRA part; the Walsh-Hadamard sums
+    if (M <= 8)
+      return nf4 ? launch_small<8, QL_FMT_NF4_DQ, 0, true>(a, st) : launch_small<8, QL_FMT_INT8_B64, 0, true>(a, st);
+    return nf4 ? launch_small<16, QL_FMT_NF4_DQ, 0, true>(a, st) : launch_small<16, QL_FMT_INT8_B64, 0, true>(a, st);
+  }
   if (jt == 0) {                                   // no adapter: the base product alone
     if (M <= 8) return nf4 ? launch_small<8, QL_FMT_NF4_DQ, 0>(a, st) : launch_small<8, QL_FMT_INT8_B64, 0>(a, st);
     return nf4 ? launch_small<16, QL_FMT_NF4_DQ, 0>(a, st) : launch_small<16, QL_FMT_INT8_B64, 0>(a, st);
