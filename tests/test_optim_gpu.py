@@ -41,7 +41,7 @@ def _check(theta_g, m_g, v_g, p_g, theta_r, m_r, v_r, lr):
     assert np.all(np.abs(got - ref) <= 2.0 ** -7 * np.abs(ref) + 1e-6 * np.abs(theta_r) + 1e-5 * lr)
 
 
-@pytest.mark.parametrize("n", [4096 * 64, 1_000_003, 5])
+@pytest.mark.parametrize("n", [4096 * 64, 1_000_003, 5, 1, 63, 65])
 def test_adamw_matches_oracle(n):
     theta0 = synth.normal_bf16((n,), 0.02, 7, 59).float()
     grads = _grads(n, 5, 7)
@@ -106,7 +106,7 @@ def test_adamw_nonfinite_gradient_is_flagged():
 
 # ---- Lion with INT8 momentum (QFT page, section 2.1) -----------------------------------
 
-@pytest.mark.parametrize("n", [64 * 4096, 1_000_003, 37])
+@pytest.mark.parametrize("n", [64 * 4096, 1_000_003, 37, 1, 63, 65, 127])
 def test_lion_int8_bit_exact(n):
     """Four steps: theta, the momentum codes and absmax, and the bf16 copy are bit-identical
     to the oracle (the step is fixed fp32 arithmetic; the codes are integer decisions)."""

@@ -151,3 +151,49 @@ def test_wht_of_unit_vectors_is_exact():
     for t, k in enumerate(ks):
         par = np.array([bin(k & v).count("1") & 1 for v in j])
         assert np.array_equal(Z[t], np.where(par == 1, -1.0, 1.0) / 64.0)
+
+
+# ---- edge cases ------------------------------------------------------------------------
+
+def _run_custom(M, N, K, row_ptr, col, c, fmt="nf4_dq", seed=12):
+    case = synth.LinearCase(f"qwha-edge-{M}-{N}-{K}", N=N, K=K, M=M, r=8, alpha=8.0, fmt=fmt, seed=seed,
+                            backward=False)
+    inp = synth.make_inputs(case)
+    qw = B.quantize_weight(inp["W"].cuda(), fmt)
+    Y = B.linear_fwd_qwha(qw, inp["X"].cuda(), torch.tensor(row_ptr, dtype=torch.int32).cuda(),
+                          torch.tensor(np.asarray(col, np.uint16)).cuda(),
+                          synth.to_bf16(np.asarray(c, np.float32)).cuda())
+    torch.cuda.synchronize()
+    assert B.device_status() == B.QL_OK
+    wd = o.quantize_weight(inp["W"].float().numpy(), fmt)["wdeq"].reshape(N, K)
+    cv = synth.to_bf16(np.asarray(c, np.float32)).float().numpy()
+    ref = o.qwha_linear_fwd(inp["X"].float().numpy(), wd, row_ptr, np.asarray(col, np.int64), cv)
+    _close(Y.float().cpu().numpy(), ref, f"edge M={M} N={N} K={K}")
+
+
+@pytest.mark.parametrize("M", [1, 16, 17])
+def test_qwha_smallest_width(M):
+    """K = 64 (one 64-point block), N = 8: the smallest shape the format allows."""
+    rng = np.random.default_rng(M)
+    cnt = [3, 0, 64, 1, 0, 7, 2, 5]                   # an empty row and a full row
+    row_ptr = np.concatenate([[0], np.cumsum(cnt)]).astype(np.int32)
+    col = np.concatenate([np.sort(rng.choice(64, k, replace=False)) for k in cnt])
+    c = rng.standard_normal(int(row_ptr[-1])) * 0.05
+    _run_custom(M, 8, 64, row_ptr, col, c)
+
+
+@pytest.mark.parametrize("M", [1, 8, 16, 40])
+def test_qwha_dense_row_spans_several_batches(M):
+    """One row holds all 1024 columns (several gather batches on the decode-shaped path,
+    and a full dense row on the tensor-core path); the others hold one value or none."""
+    N, K = 24, 1024
+    rng = np.random.default_rng(40 + M)
+    cnt = [0] * N
+    cnt[5] = K
+    for i in range(0, N, 3):
+        if i != 5:
+            cnt[i] = 1
+    row_ptr = np.concatenate([[0], np.cumsum(cnt)]).astype(np.int32)
+    col = np.concatenate([np.sort(rng.choice(K, k, replace=False)) for k in cnt])
+    c = rng.standard_normal(int(row_ptr[-1])) * 0.02
+    _run_custom(M, N, K, row_ptr, col, c)
