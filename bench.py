@@ -141,14 +141,25 @@ def oracle_step(inp_np, case, m_rows: int, n_rows: int):
 
 
 def oracle_inputs(case):
+    """The oracle's inputs, with the full-weight quantisations timed on the way (NF4+DQ,
+    which also gives the dequantised weight, and blockwise int8), as GB/s of algorithmic
+    bytes (2.516 and 3.0625 B/param) on the host's cores."""
     import oracle.qlora_oracle as o
     from quantized_base_rank_b200 import synth
     inp = synth.make_inputs(case)
     f = lambda t: t.float().numpy()
     w = f(inp["W"])
+    t0 = time.perf_counter()
     wd = o.quantize_weight(w, "nf4_dq")["wdeq"].reshape(case.N, case.K).astype(np.float64)
+    t_nf4 = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    o.quantize_weight(w, "int8")
+    t_i8 = time.perf_counter() - t0
+    n = w.size
+    timing = {"nf4_dq_quantize_and_dequant": {"s": t_nf4, "GB/s": NF4_DQ_BYTES_PER_PARAM * n / t_nf4 / 1e9},
+              "int8_quantize_and_dequant": {"s": t_i8, "GB/s": 3.0625 * n / t_i8 / 1e9}}
     return {"W": w, "Wd": wd, "X": f(inp["X"]).astype(np.float64), "A": f(inp["A"]).astype(np.float64),
-            "B": f(inp["B"]).astype(np.float64), "dY": f(inp["dY"]).astype(np.float64)}
+            "B": f(inp["B"]).astype(np.float64), "dY": f(inp["dY"]).astype(np.float64), "timing": timing}
 
 
 def blas_threads() -> int:
@@ -193,7 +204,8 @@ def run_reference(args, case, world, rank):
             "config": {"workload": case.name, "M": case.M, "N": case.N, "K": case.K, "r": case.r,
                        "alpha": case.alpha, "format": "nf4_dq"},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(),
-                             "kind": "oracle", "sample": sample, "cpu": cpu_model()},
+                             "kind": "oracle", "sample": sample, "cpu": cpu_model(),
+                             "components": inp["timing"]},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -655,7 +667,7 @@ def run_ours(args, case, world, rank, local_rank):
         cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
                "sample": (f"one step with the full {N}x{K} weight quantised (NF4+DQ) and fp64 "
                           f"forward + backward for {m_rows} of {M} tokens; {dt:.1f} s"),
-               "cpu": cpu_model()}
+               "cpu": cpu_model(), "components": o_inp["timing"]}
 
     if rank != 0:
         return
@@ -681,10 +693,12 @@ def run_ours(args, case, world, rank, local_rank):
                      "frac": achieved / peak_fwd, "traffic": fwd_main_traffic(),
                      "traffic_unit": "bytes per launch (ncu dram read + write)",
                      "peak_source": peak_fwd_source,
-                     "frac_of_burst": achieved / peaks["bf16_tflops"]},
+                     "frac_of_burst": achieved / peaks["bf16_tflops"],
+                     "frac_of_datasheet_2250": achieved / 2250.0},
         "components": {
             "quantize_nf4_dq": {"ms": q_ms, "GB/s": n * NF4_DQ_BYTES_PER_PARAM / (q_ms * 1e-3) / 1e9,
-                                "frac_hbm": n * NF4_DQ_BYTES_PER_PARAM / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+                                "frac_hbm": n * NF4_DQ_BYTES_PER_PARAM / (q_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                "frac_8tbs": n * NF4_DQ_BYTES_PER_PARAM / (q_ms * 1e-3) / 1e9 / 8000.0},
             "forward": {"ms": fwd_ms, "TFLOP/s": fwd_f / (fwd_ms * 1e-3) / 1e12},
             "backward": {"ms": bwd_ms, "TFLOP/s": bwd_f / (bwd_ms * 1e-3) / 1e12},
             "fwd_main_gemm": {"ms": main_ms, "TFLOP/s": achieved},
