@@ -109,3 +109,62 @@ def test_bin_allreduce_is_exact():
                        start_method="spawn")
     want = [sum((1 << 61) + 12345 * (r + 1) + i for r in range(world)) for i in range(16)]
     assert results[0] == want and results[1] == want
+
+
+def _step_worker(rank, world, port, results):
+    """A data-parallel training step of the adapter: partial gradients of the shard, the
+    all-reduce, then the optimiser step with the 1/world gradient scale (AdamW) and the
+    Lion INT8 step on the averaged gradient, both with the oracle on the host."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        inp = synth.make_inputs(CASE)
+        wd = o.quantize_weight(inp["W"].float().numpy(), CASE.fmt)["wdeq"].reshape(CASE.N, CASE.K)
+        s0, s1 = dp.shard_rows(CASE.M, world, rank)
+        f = lambda t: t.float().numpy().astype(np.float64)
+        A, B = f(inp["A"]), f(inp["B"])
+        _, dA, dB = o.linear_bwd(f(inp["X"])[s0:s1], f(inp["dY"])[s0:s1], wd, A, B, CASE.alpha, CASE.r)
+        tA = torch.from_numpy(dA.astype(np.float32))
+        tB = torch.from_numpy(dB.astype(np.float32))
+        dp.allreduce_adapter_grads(tA, tB)
+        g = np.concatenate([tA.numpy().ravel(), tB.numpy().ravel()])
+        theta0 = np.concatenate([A.ravel(), B.ravel()]).astype(np.float32)
+        n = theta0.size
+        th_adam = o.adamw_step(theta0, g, np.zeros(n), np.zeros(n), 1, 1e-3, 0.9, 0.999, 1e-8, 0.01,
+                               grad_scale=1.0 / world)[0]
+        g_mean = (g / np.float32(world)).astype(np.float32)
+        th_lion, codes, amax, _ = o.lion_int8_step(theta0, g_mean, np.zeros(n, np.int8),
+                                                   np.zeros((n + 63) // 64, np.float32), 1e-4, 0.9, 0.99, 0.1)
+        results[rank] = (th_adam, th_lion, codes, amax)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_data_parallel_step_with_optimisers_keeps_replicas_identical():
+    """After the exchange every rank takes the same optimiser step: the replicas are
+    bit-identical, and equal (within the fp32 exchange's rounding) to one process stepping
+    on the averaged full-batch gradient."""
+    world = 2
+    mgr = mp.get_context("spawn").Manager()
+    results = mgr.dict()
+    mp.start_processes(_step_worker, args=(world, _free_port(), results), nprocs=world, join=True,
+                       start_method="spawn")
+    r0, r1 = results[0], results[1]
+    for a, b in zip(r0, r1):
+        assert np.array_equal(np.asarray(a), np.asarray(b))
+    inp = synth.make_inputs(CASE)
+    wd = o.quantize_weight(inp["W"].float().numpy(), CASE.fmt)["wdeq"].reshape(CASE.N, CASE.K)
+    f = lambda t: t.float().numpy().astype(np.float64)
+    A, B = f(inp["A"]), f(inp["B"])
+    _, dA, dB = o.linear_bwd(f(inp["X"]), f(inp["dY"]), wd, A, B, CASE.alpha, CASE.r)
+    g = np.concatenate([dA.ravel(), dB.ravel()]) / world
+    theta0 = np.concatenate([A.ravel(), B.ravel()])
+    n = theta0.size
+    th_ref = o.adamw_step(theta0, g, np.zeros(n), np.zeros(n), 1, 1e-3, 0.9, 0.999, 1e-8, 0.01)[0]
+    np.testing.assert_allclose(r0[0], th_ref, rtol=1e-6, atol=1e-9)
+    # Lion moves every element by lr against sign(c); the same signs as the single process
+    # wherever the averaged gradient is not within the exchange's rounding of zero
+    sure = np.abs(g) > 1e-6 * np.abs(g).max()
+    step = r0[1].astype(np.float64) - theta0.astype(np.float32).astype(np.float64) * (1 - 1e-5)
+    assert np.all(np.sign(step[sure]) == -np.sign(g[sure]))
