@@ -15,10 +15,18 @@
  * The per-layer choice of bit-width and rank is the allocation C = {(q_l, r_l)} of the
  * AutoQRA page (gist.science/ko/paper/2602.22268), section 3.1.
  *
+ * Beside the low-rank adapter, the same quantised linear takes two other unmerged
+ * adapters in its forward: LoRDBA's double-binary adapter (qlora_linear_fwd_lordba) and
+ * QWHA's Walsh-Hadamard adapter (qlora_linear_fwd_qwha, ql_wht). The adapter's training
+ * step has two optimisers: AdamW with states in paged (managed) memory, after the QLoRA
+ * page's paged optimiser (ql_adamw_step, ql_paged_*), and Lion with INT8 momentum, after
+ * the QFT page (ql_lion_int8_step).
+ *
  * Conventions, for every entry point:
- *  - Pointers named "device" are CUDA device pointers owned by the caller. The library
- *    never allocates or frees caller-visible memory; scratch comes from the caller's
- *    workspace (size from ql_workspace_bytes).
+ *  - Pointers named "device" are CUDA device pointers owned by the caller. Apart from
+ *    ql_paged_alloc / ql_paged_free, which allocate and free managed memory when asked,
+ *    the library never allocates or frees caller-visible memory; scratch comes from the
+ *    caller's workspace (size from ql_workspace_bytes).
  *  - bf16 tensors are passed as uint16_t bit patterns, row-major, densely packed.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream). All work is
  *    asynchronous on it; outputs are valid once the stream reaches that point.
