@@ -230,7 +230,7 @@ __device__ float dq_mean_from_bins(const unsigned long long (&bins)[16], int64_t
 // shares the bins) rounds the sum and writes the mean, or, with bins_out (one shard of a
 // weight split across ranks), copies the shard's exact bins out instead. No CTA waits
 // for another. ws: bins[16], then the ticket counter; zeroed before the first launch.
-__device__ __forceinline__ void dq_bins_finish(unsigned long long (*s_bins)[kSumBins], int nwarps,
+__device__ __forceinline__ bool dq_bins_finish(unsigned long long (*s_bins)[kSumBins], int nwarps,
                                                unsigned long long* ws, unsigned int ctas, int64_t nb,
                                                float* mean, unsigned long long* bins_out) {
   __shared__ int s_last;
@@ -256,6 +256,7 @@ __device__ __forceinline__ void dq_bins_finish(unsigned long long (*s_bins)[kSum
       *mean = dq_mean_from_bins(v, nb);
     }
   }
+  return s_last != 0;
 }
 
 // The mean from bins summed over the shards of a weight: one thread.
@@ -268,6 +269,40 @@ __global__ void dq_mean_kernel(const unsigned long long* __restrict__ bins, int6
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// One group of 256 constants by one warp: d = a - mean, s_g = max|d| / 127, code =
+// clamp(rint(d / s_g)). CG: read the constants from L2 (they were written by other CTAs
+// of the same grid).
+template <bool CG>
+__device__ __forceinline__ void dq_encode_group(const float* __restrict__ absmax, int64_t nb, float mu,
+                                                int8_t* __restrict__ qabsmax, float* __restrict__ group_scale,
+                                                int64_t g, int lane) {
+  {
+    float d[8];
+    float mx = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int64_t b = g * kGroup + i * 32 + lane;
+      d[i] = b < nb ? __fsub_rn(CG ? __ldcg(absmax + b) : absmax[b], mu) : 0.0f;
+      mx = fmaxf(mx, fabsf(d[i]));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+    const float s = __fdiv_rn(mx, 127.0f);
+    if (lane == 0) group_scale[g] = s;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int64_t b = g * kGroup + i * 32 + lane;
+      if (b >= nb) continue;
+      int8_t c = 0;
+      if (s != 0.0f) {
+        float t = rintf(__fdiv_rn(d[i], s));
+        c = (int8_t)(int32_t)fminf(fmaxf(t, -127.0f), 127.0f);
+      }
+      qabsmax[b] = c;
+    }
+  }
+}
+
 // NF4 encode kernel. Two threads per block of 64: lanes 2t and 2t+1 of a warp take the
 // two halves of one block (32 elements, 64 bytes), combine their partial absmax with one
 // shuffle and each write 16 bytes of codes. The grid is persistent and the loop is
@@ -277,6 +312,13 @@ __global__ void dq_mean_kernel(const unsigned long long* __restrict__ bins, int6
 // by element with bounds checks. DQ = true also accumulates the exact sum of the block
 // constants for double quantisation (dq_bins_finish).
 constexpr int kNf4Threads = 256;
+constexpr uint64_t kDqWaitNs = 2000000000ull;   // bound of the fused quantise's wait for the mean
+
+__device__ __forceinline__ uint64_t qt_globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 constexpr int kNf4Warps = kNf4Threads / 32;
 
 struct Nf4Args {
@@ -290,6 +332,8 @@ struct Nf4Args {
   unsigned long long* bins_out;  // DQ, one shard: its exact bins instead of the mean
   unsigned int dq_ctas;        // DQ: CTAs over all launches sharing the bins
   int64_t nb_total;            // DQ: number of constants
+  int8_t* qabsmax;             // FUSED: the DQ codes
+  float* group_scale;          // FUSED: the group scales
 };
 
 __device__ __forceinline__ void nf4_load_vec(const uint16_t* __restrict__ W, int64_t base, bool live,
@@ -304,7 +348,12 @@ __device__ __forceinline__ void nf4_load_vec(const uint16_t* __restrict__ W, int
   }
 }
 
-template <bool VEC, bool DQ>
+// FUSED (a cooperative launch of the single whole-block VEC grid, with DQ): after the
+// exact sum, the last CTA publishes the mean through a ready flag in the workspace; every
+// CTA waits for it (bounded by globaltimer; all CTAs are co-resident by the cooperative
+// launch) and the grid's warps then encode the groups of 256 constants, so no second
+// launch is needed. The constants written by other CTAs are read from L2.
+template <bool VEC, bool DQ, bool FUSED = false>
 __global__ void __launch_bounds__(kNf4Threads, VEC ? 4 : 1)
 nf4_quantize_kernel(const Nf4Args args, const Nf4Tables tab, const Nf4BoundTable btab) {
   __shared__ __align__(16) uint32_t s_tab[128 * 8];
@@ -314,7 +363,7 @@ nf4_quantize_kernel(const Nf4Args args, const Nf4Tables tab, const Nf4BoundTable
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (DQ) {
     if (lane < kSumBins) s_bins[warp][lane] = 0ull;
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (!FUSED) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   }
   __syncthreads();
 
@@ -391,7 +440,34 @@ nf4_quantize_kernel(const Nf4Args args, const Nf4Tables tab, const Nf4BoundTable
   }
   if (DQ) {
     (void)bad;                                         // a non-finite absmax already raised the flag
-    dq_bins_finish(s_bins, kNf4Warps, args.dq_ws, args.dq_ctas, args.nb_total, args.mean, args.bins_out);
+    const bool last =
+        dq_bins_finish(s_bins, kNf4Warps, args.dq_ws, args.dq_ctas, args.nb_total, args.mean, args.bins_out);
+    if (FUSED) {
+      __shared__ int s_ok;
+      unsigned int* ready = reinterpret_cast<unsigned int*>(args.dq_ws + kSumBins + 1);
+      if (threadIdx.x == 0) {
+        if (last) {
+          __threadfence();                             // the mean before the flag
+          atomicExch(ready, 1u);
+        }
+        unsigned int v = 0u;
+        const uint64_t t0 = qt_globaltimer_ns();
+        for (;;) {
+          asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ready) : "memory");
+          if (v || qt_globaltimer_ns() - t0 > kDqWaitNs) break;
+          __nanosleep(64);
+        }
+        s_ok = v != 0u;
+        if (!v) raise_flag(args.flag, kFlagTimeout);
+      }
+      __syncthreads();
+      if (!s_ok) return;
+      const float mu = __ldcg(args.mean);
+      const int64_t ng = (args.nb_total + kGroup - 1) / kGroup;
+      const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+      for (int64_t g = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; g < ng; g += warps)
+        dq_encode_group<true>(args.absmax, args.nb_total, mu, args.qabsmax, args.group_scale, g, lane);
+    }
   }
 }
 
@@ -506,31 +582,8 @@ dq_encode_kernel(const float* __restrict__ absmax, int64_t nb, const float* __re
   const int64_t ng = (nb + kGroup - 1) / kGroup;
   const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   const float mu = *mean;
-  for (int64_t g = (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5); g < ng; g += warps) {
-    float d[8];
-    float mx = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int64_t b = g * kGroup + i * 32 + lane;
-      d[i] = b < nb ? __fsub_rn(absmax[b], mu) : 0.0f;
-      mx = fmaxf(mx, fabsf(d[i]));
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
-    const float s = __fdiv_rn(mx, 127.0f);
-    if (lane == 0) group_scale[g] = s;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int64_t b = g * kGroup + i * 32 + lane;
-      if (b >= nb) continue;
-      int8_t c = 0;
-      if (s != 0.0f) {
-        float t = rintf(__fdiv_rn(d[i], s));
-        c = (int8_t)(int32_t)fminf(fmaxf(t, -127.0f), 127.0f);
-      }
-      qabsmax[b] = c;
-    }
-  }
+  for (int64_t g = (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5); g < ng; g += warps)
+    dq_encode_group<false>(absmax, nb, mu, qabsmax, group_scale, g, lane);
 }
 
 // ---------------------------------------------------------------------------------
@@ -618,7 +671,7 @@ static ql_status launch_nf4(const uint16_t* W, int64_t n, uint8_t* codes, float*
   Nf4Args a;
   a.W = W; a.n = n; a.codes = codes; a.absmax = absmax; a.flag = device_flag_ptr();
   a.dq_ws = dq_ws; a.mean = mean; a.bins_out = bins_out; a.dq_ctas = (unsigned)(g_vec + g_tail);
-  a.nb_total = nb;
+  a.nb_total = nb; a.qabsmax = nullptr; a.group_scale = nullptr;
   const Nf4Tables& tab = nf4_tables();
   const Nf4BoundTable& btab = nf4_bound_table();
   if (g_vec) {
@@ -632,6 +685,35 @@ static ql_status launch_nf4(const uint16_t* W, int64_t n, uint8_t* codes, float*
     if (dq) nf4_quantize_kernel<false, true><<<g_tail, kNf4Threads, 0, st>>>(a, tab, btab);
     else nf4_quantize_kernel<false, false><<<g_tail, kNf4Threads, 0, st>>>(a, tab, btab);
     QL_CHECK_LAUNCH();
+  }
+  return QL_OK;
+}
+
+// NF4 + DQ in one cooperative launch: whole blocks, 16-byte aligned W and codes (the
+// single VEC grid). The workspace holds the bins, the ticket and the ready flag, zeroed
+// here. A refused cooperative launch (grid not co-resident) returns QL_ERR_UNSUPPORTED
+// and the caller takes the two-kernel path.
+static ql_status launch_nf4_dq_fused(const uint16_t* W, int64_t n, uint8_t* codes, float* absmax,
+                                     int8_t* qabsmax, float* group_scale, float* mean,
+                                     unsigned long long* dq_ws, cudaStream_t st) {
+  auto kern = nf4_quantize_kernel<true, true, true>;
+  static const int per_sm = resident_ctas(kern, kNf4Threads);
+  const int64_t nb = n / kBlock;
+  const int64_t need = (2 * nb + kNf4Threads - 1) / kNf4Threads;
+  const int grid = (int)imax64(1, imin64(need, (int64_t)num_sms() * per_sm));
+  Nf4Args a;
+  a.W = W; a.n = n; a.blk_begin = 0; a.blk_end = nb; a.codes = codes; a.absmax = absmax;
+  a.flag = device_flag_ptr(); a.dq_ws = dq_ws; a.mean = mean; a.bins_out = nullptr;
+  a.dq_ctas = (unsigned)grid; a.nb_total = nb; a.qabsmax = qabsmax; a.group_scale = group_scale;
+  const Nf4Tables& tab = nf4_tables();
+  const Nf4BoundTable& btab = nf4_bound_table();
+  if (cudaMemsetAsync(dq_ws, 0, (kSumBins + 2) * sizeof(unsigned long long), st) != cudaSuccess)
+    return QL_ERR_CUDA;
+  void* params[] = {&a, const_cast<Nf4Tables*>(&tab), const_cast<Nf4BoundTable*>(&btab)};
+  if (cudaLaunchCooperativeKernel(reinterpret_cast<void*>(kern), dim3(grid), dim3(kNf4Threads), params, 0, st) !=
+      cudaSuccess) {
+    (void)cudaGetLastError();                          // clear it; the two-kernel path follows
+    return QL_ERR_UNSUPPORTED;
   }
   return QL_OK;
 }
@@ -715,6 +797,12 @@ ql_status nf4_dq_quantize(const ql_bf16* W, int64_t n, uint8_t* codes, float* ab
   if (ws_bytes < ql_workspace_bytes(QL_OP_DQ, 0, 0, 0, 0)) return QL_ERR_WORKSPACE;
   cudaStream_t st = as_stream(stream);
   unsigned long long* bins = static_cast<unsigned long long*>(ws);
+  if (n % kBlock == 0 && aligned(W, 16) && aligned(codes, 16)) {
+    // one cooperative launch: encode, exact sum, mean and DQ codes
+    ProfScope prof(PK_NF4, st, 1);
+    const ql_status s = launch_nf4_dq_fused(W, n, codes, absmax, qabsmax, group_scale, mean, bins, st);
+    if (s != QL_ERR_UNSUPPORTED) return s;
+  }
   {
     ProfScope prof(PK_NF4, st, nf4_launches(W, n, codes));
     if (cudaMemsetAsync(bins, 0, (kSumBins + 1) * sizeof(unsigned long long), st) != cudaSuccess)
