@@ -401,9 +401,13 @@ nf4_quantize_kernel(const Nf4Args args, const Nf4Tables tab, const Nf4BoundTable
         v[i] = lo | (hi << 16);
       }
     }
-    uint32_t m = 0;                                  // two 16-bit lanes of |x| bit patterns
+    // two 16-bit lanes of max |x| by packed bf16 max (NaN-propagating; the sign bits of the
+    // running value are meaningless and cleared after the loop): for non-NaN values the
+    // order of |x| is the order of its bit patterns, so this is the bitwise maximum
+    uint32_t m = 0;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) m = __vmaxu2(m, v[i] & 0x7FFF7FFFu);
+    for (int i = 0; i < 16; ++i) asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(m), "r"(v[i]));
+    m &= 0x7FFF7FFFu;
     m = __vmaxu2(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
     const uint32_t amax = max(m & 0xFFFFu, m >> 16);   // bf16 bits of the block's max |x|
     const bool owner = live && h == 0;
