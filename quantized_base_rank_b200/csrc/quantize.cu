@@ -849,23 +849,23 @@ ql_status dq_quantize_shard(const float* absmax, int64_t nblocks, const uint64_t
 }
 
 ql_status ql_dequantize(const ql_weight* w, ql_bf16* Wout, void* stream) {
-  if (!w || !Wout || w->N < 1 || w->K < 1 || !w->codes) return QL_ERR_INVALID_ARG;
+  if (!w || !Wout || w->N < 1 || w->K < 1 || !w->codes || !aligned(Wout, 2)) return QL_ERR_INVALID_ARG;
+  if (w->N > (int64_t(1) << 40) / w->K) return QL_ERR_UNSUPPORTED;   // N*K stays far from overflow
+  const bool nf4 = w->fmt == QL_FMT_NF4_DQ;
+  if (nf4 ? !w->qabsmax || !w->group_scale || !w->mean || !aligned(w->group_scale, 4) || !aligned(w->mean, 4)
+          : w->fmt != QL_FMT_INT8_B64 || !w->absmax || !aligned(w->absmax, 4))
+    return QL_ERR_INVALID_ARG;
   const int64_t n = w->N * w->K;
   const int64_t nb = (n + kBlock - 1) / kBlock;
   cudaStream_t st = as_stream(stream);
-  ProfScope prof(PK_DEQ, st, 1);
-  if (w->fmt == QL_FMT_NF4_DQ) {
-    if (!w->qabsmax || !w->group_scale || !w->mean) return QL_ERR_INVALID_ARG;
+  ProfScope prof(PK_DEQ, st, 1);                      // counts a launch: every check is above
+  if (nf4)
     dequant_nf4_kernel<<<grid_for(nb, 256), 256, 0, st>>>(
         static_cast<const uint8_t*>(w->codes), w->qabsmax, w->group_scale, w->mean, n, Wout,
         nf4_tables());
-  } else if (w->fmt == QL_FMT_INT8_B64) {
-    if (!w->absmax) return QL_ERR_INVALID_ARG;
+  else
     dequant_int8_kernel<<<grid_for(nb, 256), 256, 0, st>>>(
         static_cast<const int8_t*>(w->codes), w->absmax, n, Wout);
-  } else {
-    return QL_ERR_INVALID_ARG;
-  }
   QL_CHECK_LAUNCH();
   return QL_OK;
 }

@@ -107,7 +107,17 @@ def test_argument_validation_without_a_device(lib):
     assert lib.ql_paged_prefetch(None, 0, 1, None) == B.QL_OK
     assert lib.ql_paged_prefetch(None, 64, 1, None) == B.QL_ERR_INVALID_ARG
     assert lib.ql_dequantize(None, None, None) == B.QL_ERR_INVALID_ARG
+    # dequantise: a bad format, a missing constant, an odd output address or an oversize
+    # shape is refused before anything is launched or counted
+    c0 = lib.ql_launch_count()
+    for bad in (B.QLWeight(7, 0, 64, 64, 16, 16, 16, 16, 16), B.QLWeight(0, 0, 64, 64, 16, 0, None, 16, 16),
+                B.QLWeight(1, 0, 64, 64, 16, None, 16, 16, 16), B.QLWeight(1, 0, 64, 64, 16, 18, 16, 16, 16)):
+        assert lib.ql_dequantize(ctypes.byref(bad), 16, None) == B.QL_ERR_INVALID_ARG
     w = B.QLWeight(0, 0, 64, 64, 16, 0, 16, 16, 16)
+    assert lib.ql_dequantize(ctypes.byref(w), 17, None) == B.QL_ERR_INVALID_ARG
+    big = B.QLWeight(1, 0, 1 << 21, 1 << 21, 16, 16, 16, 16, 16)
+    assert lib.ql_dequantize(ctypes.byref(big), 16, None) == B.QL_ERR_UNSUPPORTED
+    assert lib.ql_launch_count() == c0
     # misaligned or null pointers, bad shapes: all rejected synchronously
     assert lib.qlora_linear_fwd(ctypes.byref(w), None, 1, None, None, 8, 16.0, None, None,
                                 None, 0, None) == B.QL_ERR_INVALID_ARG
