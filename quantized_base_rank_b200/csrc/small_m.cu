@@ -630,6 +630,7 @@ bool small_m_supported(int64_t K, int r) {
 ql_status small_m_forward(const ql_weight* w, const uint16_t* X, int64_t M, const uint16_t* A,
                           const uint16_t* B, int r, float alpha, uint16_t* Y, uint16_t* T_save,
                           cudaStream_t st, const QwhaRows* qw) {
+  if (r < 0 || r > 64) return QL_ERR_UNSUPPORTED;
   SmallArgs a{};
   a.flag = device_flag_ptr();
   if (qw) {
@@ -647,7 +648,6 @@ ql_status small_m_forward(const ql_weight* w, const uint16_t* X, int64_t M, cons
   const Nf4Tables& t = nf4_tables();
   for (int i = 0; i < 16; ++i) a.q[i] = t.q[i];
   ProfScope prof(PK_FWD_SMALL, st, 1);
-  if (r < 0 || r > 64) return QL_ERR_UNSUPPORTED;
   const int jt = (r + 15) / 16;
   const bool nf4 = w->fmt == QL_FMT_NF4_DQ;
   if (jt == 0 && qw) {                             // no LoRA part; the Walsh-Hadamard sums
