@@ -144,9 +144,23 @@ def _stream(device: torch.device | None = None) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
 
-def _need(t: torch.Tensor, dtype: torch.dtype, name: str):
-    if not isinstance(t, torch.Tensor) or t.dtype != dtype or not t.is_cuda or not t.is_contiguous():
+def _is_cuda(t: torch.Tensor) -> bool:
+    return t.is_cuda
+
+
+def _need(t: torch.Tensor, dtype: torch.dtype, name: str, shape=None, device=None):
+    """Refuse, before the library is called, what its kernels would read or write out of
+    bounds: t must be a contiguous CUDA tensor of `dtype`; with `shape`, of exactly that
+    shape (an int: that many elements, any shape); with `device`, on that device. The C
+    entry points take bare pointers and cannot see a buffer's size."""
+    if not isinstance(t, torch.Tensor) or t.dtype != dtype or not _is_cuda(t) or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+    if shape is not None:
+        ok = t.numel() == shape if isinstance(shape, int) else tuple(t.shape) == tuple(shape)
+        if not ok:
+            raise ValueError(f"{name} has shape {tuple(t.shape)}; expected {shape}")
+    if device is not None and t.device != torch.device(device):
+        raise ValueError(f"{name} is on {t.device}; expected {device}")
 
 
 # ---- workspace: caller-owned device memory, allocated by torch, reused ----------------
@@ -166,6 +180,19 @@ def workspace_bytes(op: int, M: int, N: int, K: int, r: int) -> int:
     return int(lib().ql_workspace_bytes(op, M, N, K, r))
 
 
+def _need_dq_outputs(nb: int, qabsmax, group_scale, mean, dev):
+    _need(qabsmax, torch.int8, "qabsmax", nb, dev)
+    _need(group_scale, torch.float32, "group_scale", (nb + 255) // 256, dev)
+    _need(mean, torch.float32, "mean", 1, dev)
+
+
+def _need_weight(qw: "QuantWeight", K: int, dev):
+    if qw.K != K:
+        raise ValueError(f"X has {K} columns; the weight has K = {qw.K}")
+    if qw.device != dev:
+        raise ValueError(f"the weight is on {qw.device}; X is on {dev}")
+
+
 # ---- entry points ---------------------------------------------------------------------
 
 def nf4_quantize(W: torch.Tensor, codes: torch.Tensor | None = None,
@@ -176,6 +203,8 @@ def nf4_quantize(W: torch.Tensor, codes: torch.Tensor | None = None,
         codes = torch.empty((n + 1) // 2, dtype=torch.uint8, device=W.device)
     if absmax is None:
         absmax = torch.empty((n + 63) // 64, dtype=torch.float32, device=W.device)
+    _need(codes, torch.uint8, "codes", (n + 1) // 2, W.device)
+    _need(absmax, torch.float32, "absmax", (n + 63) // 64, W.device)
     _check(lib().nf4_quantize(_ptr(W), n, _ptr(codes), _ptr(absmax), _stream(W.device)),
            "nf4_quantize")
     return codes, absmax
@@ -189,6 +218,8 @@ def int8_quantize(W: torch.Tensor, codes: torch.Tensor | None = None,
         codes = torch.empty(n, dtype=torch.int8, device=W.device)
     if absmax is None:
         absmax = torch.empty((n + 63) // 64, dtype=torch.float32, device=W.device)
+    _need(codes, torch.int8, "codes", n, W.device)
+    _need(absmax, torch.float32, "absmax", (n + 63) // 64, W.device)
     _check(lib().int8_quantize(_ptr(W), n, _ptr(codes), _ptr(absmax), _stream(W.device)),
            "int8_quantize")
     return codes, absmax
@@ -204,6 +235,7 @@ def dq_quantize(absmax: torch.Tensor, qabsmax=None, group_scale=None, mean=None)
         group_scale = torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev)
     if mean is None:
         mean = torch.empty(1, dtype=torch.float32, device=dev)
+    _need_dq_outputs(nb, qabsmax, group_scale, mean, dev)
     nws = workspace_bytes(QL_OP_DQ, 0, 0, 0, 0)
     ws = workspace(nws, dev)
     _check(lib().dq_quantize(_ptr(absmax), nb, _ptr(qabsmax), _ptr(group_scale), _ptr(mean),
@@ -228,6 +260,9 @@ def nf4_dq_quantize(W: torch.Tensor, codes=None, absmax=None, qabsmax=None, grou
         group_scale = torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev)
     if mean is None:
         mean = torch.empty(1, dtype=torch.float32, device=dev)
+    _need(codes, torch.uint8, "codes", (n + 1) // 2, dev)
+    _need(absmax, torch.float32, "absmax", nb, dev)
+    _need_dq_outputs(nb, qabsmax, group_scale, mean, dev)
     ws = workspace(workspace_bytes(QL_OP_DQ, 0, 0, 0, 0), dev)
     _check(lib().nf4_dq_quantize(_ptr(W), n, _ptr(codes), _ptr(absmax), _ptr(qabsmax), _ptr(group_scale),
                                  _ptr(mean), _ptr(ws), ws.numel(), _stream(dev)), "nf4_dq_quantize")
@@ -246,6 +281,9 @@ def nf4_quantize_shard(W: torch.Tensor, codes=None, absmax=None, bins=None):
         absmax = torch.empty((n + 63) // 64, dtype=torch.float32, device=dev)
     if bins is None:
         bins = torch.empty(16, dtype=torch.int64, device=dev)
+    _need(codes, torch.uint8, "codes", (n + 1) // 2, dev)
+    _need(absmax, torch.float32, "absmax", (n + 63) // 64, dev)
+    _need(bins, torch.int64, "bins", 16, dev)
     ws = workspace(workspace_bytes(QL_OP_DQ, 0, 0, 0, 0), dev)
     _check(lib().nf4_quantize_shard(_ptr(W), n, _ptr(codes), _ptr(absmax), _ptr(bins), _ptr(ws),
                                     ws.numel(), _stream(dev)), "nf4_quantize_shard")
@@ -256,15 +294,16 @@ def dq_quantize_shard(absmax: torch.Tensor, bins: torch.Tensor, nblocks_total: i
                       group_scale=None, mean=None):
     """Step 3: the mean from bins summed over all shards, then this shard's groups."""
     _need(absmax, torch.float32, "absmax")
-    _need(bins, torch.int64, "bins")
     nb = absmax.numel()
     dev = absmax.device
+    _need(bins, torch.int64, "bins", 16, dev)
     if qabsmax is None:
         qabsmax = torch.empty(nb, dtype=torch.int8, device=dev)
     if group_scale is None:
         group_scale = torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev)
     if mean is None:
         mean = torch.empty(1, dtype=torch.float32, device=dev)
+    _need_dq_outputs(nb, qabsmax, group_scale, mean, dev)
     _check(lib().dq_quantize_shard(_ptr(absmax), nb, _ptr(bins), int(nblocks_total), _ptr(qabsmax),
                                    _ptr(group_scale), _ptr(mean), _stream(dev)), "dq_quantize_shard")
     return qabsmax, group_scale, mean
@@ -297,8 +336,16 @@ def linear_fwd_lordba(qw: "QuantWeight", X: torch.Tensor, B1p: torch.Tensor, B2p
     M, K = X.shape
     ell = alpha.shape[0]
     dev = X.device
+    N = qw.N
+    _need_weight(qw, K, dev)
+    _need(B1p, torch.int32, "B1", (N, (R + 31) // 32), dev)
+    _need(B2p, torch.int32, "B2", (R, (K + 31) // 32), dev)
+    _need(alpha, torch.float16, "alpha", (ell, N), dev)
+    _need(beta, torch.float16, "beta", (ell, R), dev)
+    _need(gamma, torch.float16, "gamma", (ell, K), dev)
     if Y is None:
-        Y = torch.empty((M, qw.N), dtype=torch.bfloat16, device=dev)
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    _need(Y, torch.bfloat16, "Y", (M, N), dev)
     ad = QLLordba(R, ell, _ptr(B1p), _ptr(B2p), _ptr(alpha), _ptr(beta), _ptr(gamma))
     ws = workspace(workspace_bytes(QL_OP_FWD_LORDBA, M, qw.N, K, R * ell), dev)
     _check(lib().qlora_linear_fwd_lordba(ctypes.byref(qw.desc), _ptr(X), M, ctypes.addressof(ad), _ptr(Y),
@@ -316,9 +363,14 @@ def linear_fwd_qwha(qw: "QuantWeight", X: torch.Tensor, row_ptr: torch.Tensor, c
     _need(c, torch.bfloat16, "c")
     M, K = X.shape
     dev = X.device
+    nnz = c.numel()
+    _need_weight(qw, K, dev)
+    _need(row_ptr, torch.int32, "row_ptr", qw.N + 1, dev)
+    _need(col, torch.uint16, "col", nnz, dev)
+    _need(c, torch.bfloat16, "c", nnz, dev)
     if Y is None:
         Y = torch.empty((M, qw.N), dtype=torch.bfloat16, device=dev)
-    nnz = c.numel()
+    _need(Y, torch.bfloat16, "Y", (M, qw.N), dev)
     ad = QLQwha(_ptr(row_ptr), _ptr(col) if nnz else None, _ptr(c) if nnz else None, nnz)
     ws = workspace(workspace_bytes(QL_OP_FWD_QWHA, M, qw.N, K, 0), dev)
     _check(lib().qlora_linear_fwd_qwha(ctypes.byref(qw.desc), _ptr(X), M, ctypes.addressof(ad), _ptr(Y),
@@ -332,6 +384,7 @@ def wht(X: torch.Tensor, Z: torch.Tensor | None = None) -> torch.Tensor:
     M, K = X.shape
     if Z is None:
         Z = torch.empty_like(X)
+    _need(Z, torch.bfloat16, "Z", (M, K), X.device)
     _check(lib().ql_wht(_ptr(X), M, K, _ptr(Z), _stream(X.device)), "ql_wht")
     return Z
 
@@ -344,12 +397,8 @@ def adamw_step(theta: torch.Tensor, param: torch.Tensor, grad: torch.Tensor, m: 
     PagedBuffer."""
     n = theta.numel()
     for t, nm in ((theta, "theta"), (grad, "grad"), (m, "m"), (v, "v")):
-        _need(t, torch.float32, nm)
-        if t.numel() != n:
-            raise ValueError(f"{nm} must have {n} elements")
-    _need(param, torch.bfloat16, "param")
-    if param.numel() != n:
-        raise ValueError(f"param must have {n} elements")
+        _need(t, torch.float32, nm, n, theta.device)
+    _need(param, torch.bfloat16, "param", n, theta.device)
     h = QLAdamw(lr, beta1, beta2, eps, weight_decay, grad_scale, step)
     _check(lib().ql_adamw_step(_ptr(theta), _ptr(param), _ptr(grad), _ptr(m), _ptr(v), n, ctypes.addressof(h),
                                _stream(theta.device)), "ql_adamw_step")
@@ -361,15 +410,12 @@ def lion_int8_step(theta: torch.Tensor, param: torch.Tensor, grad: torch.Tensor,
     """One Lion step with INT8 momentum: theta, grad fp32 [n]; m_codes int8 [n] and m_absmax
     fp32 [ceil(n/64)] updated in place; param bf16 [n] rewritten as bf16(theta)."""
     n = theta.numel()
+    dev = theta.device
     for t, nm in ((theta, "theta"), (grad, "grad")):
-        _need(t, torch.float32, nm)
-        if t.numel() != n:
-            raise ValueError(f"{nm} must have {n} elements")
-    _need(param, torch.bfloat16, "param")
-    _need(m_codes, torch.int8, "m_codes")
-    _need(m_absmax, torch.float32, "m_absmax")
-    if param.numel() != n or m_codes.numel() != n or m_absmax.numel() != (n + 63) // 64:
-        raise ValueError("param, m_codes or m_absmax has the wrong size")
+        _need(t, torch.float32, nm, n, dev)
+    _need(param, torch.bfloat16, "param", n, dev)
+    _need(m_codes, torch.int8, "m_codes", n, dev)
+    _need(m_absmax, torch.float32, "m_absmax", (n + 63) // 64, dev)
     h = QLLion(lr, beta1, beta2, weight_decay)
     _check(lib().ql_lion_int8_step(_ptr(theta), _ptr(param), _ptr(grad), _ptr(m_codes), _ptr(m_absmax), n,
                                    ctypes.addressof(h), _stream(theta.device)), "ql_lion_int8_step")
@@ -479,10 +525,16 @@ def linear_fwd(qw: QuantWeight, X: torch.Tensor, A: torch.Tensor, B: torch.Tenso
     M, K = X.shape
     r = A.shape[0]
     dev = X.device
+    _need_weight(qw, K, dev)
+    _need(A, torch.bfloat16, "A", (r, K), dev)
+    _need(B, torch.bfloat16, "B", (qw.N, r), dev)
     if Y is None:
         Y = torch.empty((M, qw.N), dtype=torch.bfloat16, device=dev)
     if T is None and save_T:
         T = torch.empty((M, r), dtype=torch.bfloat16, device=dev)
+    _need(Y, torch.bfloat16, "Y", (M, qw.N), dev)
+    if T is not None:
+        _need(T, torch.bfloat16, "T", (M, r), dev)
     ws = workspace(workspace_bytes(QL_OP_FWD, M, qw.N, K, r), dev)
     _check(lib().qlora_linear_fwd(ctypes.byref(qw.desc), _ptr(X), M, _ptr(A), _ptr(B), r,
                                   float(alpha), _ptr(Y), _ptr(T), _ptr(ws), ws.numel(),
@@ -497,12 +549,19 @@ def linear_bwd(qw: QuantWeight, X, dY, A, B, T, alpha: float, dX=None, dA=None, 
     M, K = X.shape
     r = A.shape[0]
     dev = X.device
+    N = qw.N
+    _need_weight(qw, K, dev)
+    for t, nm, shape in ((dY, "dY", (M, N)), (A, "A", (r, K)), (B, "B", (N, r)), (T, "T", (M, r))):
+        _need(t, torch.bfloat16, nm, shape, dev)
     if dX is None:
         dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
     if dA is None:
         dA = torch.empty((r, K), dtype=torch.float32, device=dev)
     if dB is None:
-        dB = torch.empty((qw.N, r), dtype=torch.float32, device=dev)
+        dB = torch.empty((N, r), dtype=torch.float32, device=dev)
+    _need(dX, torch.bfloat16, "dX", (M, K), dev)
+    _need(dA, torch.float32, "dA", (r, K), dev)
+    _need(dB, torch.float32, "dB", (N, r), dev)
     ws = workspace(workspace_bytes(QL_OP_BWD, M, qw.N, K, r), dev)
     _check(lib().qlora_linear_bwd(ctypes.byref(qw.desc), _ptr(X), _ptr(dY), M, _ptr(A), _ptr(B),
                                   _ptr(T), r, float(alpha), _ptr(dX), _ptr(dA), _ptr(dB),
