@@ -547,6 +547,74 @@ def qwha_linear_fwd(X, Wd, row_ptr, col, c) -> np.ndarray:
     return X @ Wd.T + X @ qwha_delta(N, K, row_ptr, col, c).T
 
 
+def _qwha_value_rows(N: int, row_ptr) -> np.ndarray:
+    """The row n of every stored value, in storage order."""
+    row_ptr = np.asarray(row_ptr, np.int64)
+    assert row_ptr.shape == (N + 1,) and row_ptr[0] == 0 and np.all(np.diff(row_ptr) >= 0)
+    return np.repeat(np.arange(N), np.diff(row_ptr))
+
+
+def qwha_linear_bwd(X, dY, Wd, row_ptr, col, c):
+    """Gradients of the QWHA linear Y = X Wd^T + X Delta W^T, Delta W = F H^{-1}, in fp64,
+    for an upstream gradient dY [M, N]:
+        dX  = dY (Wd + Delta W)                          [M, K]
+        dc_j = (dY^T Z)[n_j, col_j],  Z = X H^{-T}        [nnz]
+    where value j sits at (n_j, col_j). Returns (dX, dc).
+
+    Reading: the page trains the values c of F at positions E chosen once at
+    initialisation (AdaAlloc, then the refinement of c), and the frozen quantised base
+    gets no gradient. So the trainable gradient is that of c alone: the gradient of F,
+    dY^T X H^{-T}, read at the positions E and nowhere else."""
+    X = np.asarray(X, np.float64)
+    dY = np.asarray(dY, np.float64)
+    Wd = np.asarray(Wd, np.float64)
+    N, K = Wd.shape
+    dX = dY @ (Wd + qwha_delta(N, K, row_ptr, col, c))
+    G = dY.T @ qwha_transform(X)                    # gradient of the dense F [N, K]
+    rows = _qwha_value_rows(N, row_ptr)
+    dc = G[rows, np.asarray(col, np.int64)]
+    return dX, dc
+
+
+def qwha_inverse_transform_rows(U) -> np.ndarray:
+    """U H^{-1} in fp64 for rows U [M, K], one diagonal block of H at a time (the same
+    numbers as the full K x K product without forming it)."""
+    U = np.asarray(U, np.float64)
+    K = U.shape[1]
+    b = wht_block_size(K)
+    H_inv = walsh_hadamard_block(b).T
+    out = np.empty_like(U)
+    for s in range(0, K, b):
+        out[:, s:s + b] = U[:, s:s + b] @ H_inv
+    return out
+
+
+def qwha_linear_bwd_factored(X, dY, Wd, row_ptr, col, c, chunk: int = 4096):
+    """The same (dX, dc) as qwha_linear_bwd without forming Delta W or the dense gradient of
+    F, for widths where those [N, K] matrices are too large:
+        dX   = dY Wd + (dY F) H^{-1}     (the sparse product, then the blockwise inverse
+                                          transform of each token row)
+        dc_j = sum_m dY[m, n_j] Z[m, col_j]   with Z = X H^{-T} (taken in chunks of values)."""
+    import scipy.sparse
+    X = np.asarray(X, np.float64)
+    dY = np.asarray(dY, np.float64)
+    Wd = np.asarray(Wd, np.float64)
+    N, K = Wd.shape
+    row_ptr = np.asarray(row_ptr, np.int64)
+    col = np.asarray(col, np.int64)
+    c = np.asarray(c, np.float64)
+    assert col.shape == c.shape == (row_ptr[-1],) and np.all((col >= 0) & (col < K))
+    F = scipy.sparse.csr_matrix((c, col, row_ptr), shape=(N, K))
+    dX = dY @ Wd + qwha_inverse_transform_rows(np.asarray((F.T @ dY.T).T))
+    Z = qwha_transform(X)
+    rows = _qwha_value_rows(N, row_ptr)
+    dc = np.empty(c.shape[0])
+    for s in range(0, c.shape[0], chunk):
+        e = min(s + chunk, c.shape[0])
+        dc[s:e] = np.einsum("mj,mj->j", dY[:, rows[s:e]], Z[:, col[s:e]])
+    return dX, dc
+
+
 # --------------------------------------------------------------------------------------
 # The adapter optimiser step with paged states (QLoRA page, aizip.shop/methodologies/qlora,
 # section "3. Paged Optimizer": optimiser states held in unified memory, paged to host RAM

@@ -579,6 +579,102 @@ def test_qwha_zero_and_linear_in_c():
     np.testing.assert_allclose(D2, -2.5 * D1, rtol=1e-13, atol=1e-15)
 
 
+def _qwha_bwd_case(N=7, K=192, M=5, seed=5):
+    row_ptr, col, c = _qwha_case(N, K, seed)
+    rng = np.random.default_rng(seed + 100)
+    return (rng.standard_normal((M, K)), rng.standard_normal((M, N)), rng.standard_normal((N, K)),
+            row_ptr, col, c)
+
+
+def test_qwha_backward_matches_torch_autograd():
+    """dX and dc equal torch's fp64 autograd of sum(dY * Y), with F scattered from c by
+    torch, H built from scipy's Sylvester matrix block by block, and its inverse taken by
+    torch.linalg.inv."""
+    import scipy.linalg
+    X, dY, Wd, row_ptr, col, c = _qwha_bwd_case()
+    N, K = Wd.shape
+    b = 64                                            # 192 = 3 * 64
+    H = torch.block_diag(*[torch.tensor(scipy.linalg.hadamard(b) / math.sqrt(b))] * (K // b))
+    rows = torch.repeat_interleave(torch.arange(N), torch.tensor(np.diff(row_ptr)))
+    Xt = torch.tensor(X, requires_grad=True)
+    ct = torch.tensor(c, requires_grad=True)
+    F = torch.zeros((N, K), dtype=torch.float64).index_put((rows, torch.tensor(col)), ct)
+    Y = Xt @ torch.tensor(Wd).T + Xt @ (F @ torch.linalg.inv(H)).T
+    (Y * torch.tensor(dY)).sum().backward()
+    dX, dc = o.qwha_linear_bwd(X, dY, Wd, row_ptr, col, c)
+    np.testing.assert_allclose(dX, Xt.grad.numpy(), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dc, ct.grad.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_qwha_backward_central_differences():
+    """Y is linear in X and in c, so a central difference of sum(dY * Y) with a unit step
+    is the exact derivative up to rounding: checked for every value c_j and a spread of
+    entries of X."""
+    X, dY, Wd, row_ptr, col, c = _qwha_bwd_case(N=5, K=128, M=3, seed=9)
+    dX, dc = o.qwha_linear_bwd(X, dY, Wd, row_ptr, col, c)
+    L = lambda Xv, cv: float(np.sum(dY * o.qwha_linear_fwd(Xv, Wd, row_ptr, col, cv)))
+    for j in range(c.size):
+        e = np.zeros_like(c)
+        e[j] = 1.0
+        assert math.isclose((L(X, c + e) - L(X, c - e)) / 2, dc[j], rel_tol=1e-9, abs_tol=1e-9)
+    for m, k in [(0, 0), (1, 37), (2, 127), (0, 64), (2, 90)]:
+        E = np.zeros_like(X)
+        E[m, k] = 1.0
+        assert math.isclose((L(X + E, c) - L(X - E, c)) / 2, dX[m, k], rel_tol=1e-9, abs_tol=1e-9)
+
+
+def test_qwha_backward_adjoint_identities():
+    """The adapter branch A(X, c) = X Delta W^T is bilinear, so Euler's identity fixes
+    both gradients against the forward: <dc, c> = <dY, A> and <dX - dY Wd, X> = <dY, A>."""
+    X, dY, Wd, row_ptr, col, c = _qwha_bwd_case(N=9, K=448, M=4, seed=13)
+    dX, dc = o.qwha_linear_bwd(X, dY, Wd, row_ptr, col, c)
+    A = o.qwha_linear_fwd(X, Wd, row_ptr, col, c) - X @ Wd.T
+    pair = float(np.sum(dY * A))
+    assert math.isclose(float(dc @ c), pair, rel_tol=1e-11)
+    assert math.isclose(float(np.sum((dX - dY @ Wd) * X)), pair, rel_tol=1e-11)
+
+
+def test_qwha_backward_single_coefficient_is_a_walsh_correlation():
+    """One value at (n, k): dc = sum over tokens m and block columns j of
+    dY[m, n] X[m, j] (-1)^popcount((k - s) & (j - s)) / sqrt(b), s the start of k's
+    block; and the adapter's part of dX is dY[:, n] c times that Walsh function (loops)."""
+    N, K, n, k, cv = 4, 192, 2, 77, 0.625
+    rng = np.random.default_rng(17)
+    X, dY, Wd = rng.standard_normal((3, K)), rng.standard_normal((3, N)), rng.standard_normal((N, K))
+    dX, dc = o.qwha_linear_bwd(X, dY, Wd, [0, 0, 0, 1, 1], [k], [cv])
+    b, s = 64, 64
+    walsh = lambda j: (-1) ** bin((k - s) & (j - s)).count("1") / math.sqrt(b)
+    want = sum(dY[m, n] * X[m, j] * walsh(j) for m in range(3) for j in range(s, s + b))
+    assert math.isclose(dc[0], want, rel_tol=1e-12)
+    for m in range(3):
+        for j in range(K):
+            ad = dY[m, n] * cv * walsh(j) if s <= j < s + b else 0.0
+            assert math.isclose(dX[m, j] - float(dY[m] @ Wd[:, j]), ad, abs_tol=1e-12)
+
+
+@pytest.mark.parametrize("K", [192, 256, 448])
+def test_qwha_backward_factored_equals_dense(K):
+    X, dY, Wd, row_ptr, col, c = _qwha_bwd_case(N=11, K=K, M=6, seed=K)
+    dX, dc = o.qwha_linear_bwd(X, dY, Wd, row_ptr, col, c)
+    fX, fc = o.qwha_linear_bwd_factored(X, dY, Wd, row_ptr, col, c, chunk=7)
+    np.testing.assert_allclose(fX, dX, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(fc, dc, rtol=1e-12, atol=1e-12)
+
+
+def test_qwha_backward_empty_and_zero():
+    """No stored values: dc is empty and dX is the base's dY Wd. c = 0: dX is the base's
+    and dc is unchanged (it does not depend on c)."""
+    X, dY, Wd, row_ptr, col, c = _qwha_bwd_case(seed=21)
+    N = Wd.shape[0]
+    dX0, dc0 = o.qwha_linear_bwd(X, dY, Wd, np.zeros(N + 1, np.int64), np.zeros(0, np.int64), np.zeros(0))
+    assert dc0.shape == (0,)
+    np.testing.assert_allclose(dX0, dY @ Wd, rtol=1e-13)
+    dX, dc = o.qwha_linear_bwd(X, dY, Wd, row_ptr, col, c)
+    dXz, dcz = o.qwha_linear_bwd(X, dY, Wd, row_ptr, col, 0 * c)
+    np.testing.assert_allclose(dXz, dY @ Wd, rtol=1e-13)
+    np.testing.assert_array_equal(dcz, dc)
+
+
 # ---------------------------------------------------------------- AdamW step (paged states)
 
 def test_adamw_matches_torch_over_several_steps():
