@@ -284,6 +284,51 @@ def test_int8_format():
     assert np.all(c0 == 0) and o.int8_dequant(c0, a0).tolist() == [0.0] * 64
 
 
+def _rn32_exact(q: Fraction) -> Fraction:
+    """q rounded to the nearest fp32 value, ties to even, subnormals included (exact
+    rational arithmetic, no floating point)."""
+    if q == 0:
+        return Fraction(0)
+    s, q = (-1 if q < 0 else 1), abs(q)
+    e = q.numerator.bit_length() - q.denominator.bit_length()
+    if Fraction(2) ** e > q:
+        e -= 1                                            # now 2^e <= q < 2^(e+1)
+    ulp = Fraction(2) ** (max(e, -126) - 23)
+    m = q / ulp
+    k = m.numerator // m.denominator
+    rem = m - k
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and k % 2 == 1):
+        k += 1
+    return s * k * ulp
+
+
+@pytest.mark.parametrize("a_bits", [0x3F80, 0x417E, 0x7F7F, 0x0080, 0x0003, 0x4123])
+def test_int8_encoder_matches_exact_rational(a_bits):
+    """Every bf16 w with |w| <= a (or a 3000-sample of them) against the definition in
+    exact rationals: sc = RN32(a / 127), code = clamp(round_half_even(RN32(w / sc)), +-127),
+    0 when sc = 0. a = 15.875 = 127/8 makes sc = 1/8, so w = 2.5/8 and 3.5/8 are exact
+    half-way cases: half-even gives 2 and 4 (half away from zero would give 3 and 4)."""
+    a = float(np.array([a_bits << 16], np.uint32).view(np.float32)[0])
+    xs = _all_bf16_upto(a)
+    rng = np.random.default_rng(a_bits + 1)
+    if xs.size > 3000:
+        keep = rng.choice(xs.size, 3000, replace=False)
+        xs = np.concatenate([xs[keep], np.float32([0.0, -0.0, a, -a])])
+    if a == 15.875:
+        xs = np.concatenate([xs, np.float32([2.5 / 8, 3.5 / 8, -2.5 / 8, 0.5 / 8, 1.5 / 8])])
+    nb = (xs.size + 63) // 64
+    absmax = np.full(nb, a, np.float32)
+    sc = _rn32_exact(Fraction(a) / 127)
+    assert Fraction(float(np.float32(a) / np.float32(127))) == sc
+    codes = o.int8_encode(xs, absmax)
+    for w, c in zip(xs.tolist(), codes.tolist()):
+        want = 0 if sc == 0 else max(-127, min(127, round(_rn32_exact(Fraction(w) / sc))))
+        assert c == want, (w, a, c, want)
+    if a == 15.875:
+        got = dict(zip(xs[-5:].tolist(), codes[-5:].tolist()))
+        assert got == {2.5 / 8: 2, 3.5 / 8: 4, -2.5 / 8: -2, 0.5 / 8: 0, 1.5 / 8: 2}
+
+
 # ---------------------------------------------------------------- bf16 rounding
 
 def test_rn_bf16_matches_torch():
