@@ -24,3 +24,12 @@ def test_reference_arm_prints_one_json_line():
     assert set(cb["components"]) == {"nf4_dq_quantize_and_dequant", "int8_quantize_and_dequant"}
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["config"]["workload"] == "upproj-11008x4096-M8192"
+
+
+def test_reference_arm_runs_on_rank_0_only():
+    """Under torchrun with N > 1, a rank other than 0 exits 0 without work or output."""
+    env = dict(os.environ, RANK="1", LOCAL_RANK="1", WORLD_SIZE="2")
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--gpus", "2", "--steps", "1",
+                          "--warmup", "3"], cwd=ROOT, capture_output=True, text=True, timeout=300, env=env)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert not [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
