@@ -257,13 +257,43 @@ def test_dq_roundtrip_bound_and_mean():
     assert np.all(np.abs(qa.astype(int)) <= 127) and np.max(np.abs(qa.astype(int))) == 127
 
 
-def test_rint_half_even_in_dq():
-    # d/s = 2.5 exactly -> 2 ; 3.5 -> 4 (round half to even)
-    a = np.float32([0.0, 2.5, 3.5, -127.0 + 0.0]) + np.float32(127.0)
+def _dq_tie_groups():
+    """Two groups of 256 constants built so that every DQ quantity is exact: each group is
+    symmetric about 1 (so the tensor mean is exactly 1), its largest |a - 1| is 127 * 2^-k
+    (so the group scale is exactly 2^-k), and the other offsets are small multiples of
+    2^-(k+1), so a - 1 and (a - 1) / 2^-k are exact in fp32. The quotients include the
+    half-way cases +-0.5, +-1.5, +-2.5, +-3.5 and +-126.5."""
+    groups, want = [], []
+    for k in (7, 5):
+        s = Fraction(1, 2 ** k)
+        qs = [Fraction(127), Fraction(5, 2), Fraction(7, 2), Fraction(1, 2), Fraction(3, 2),
+              Fraction(253, 2), Fraction(0), Fraction(3), Fraction(41, 4)]
+        offs = []
+        for qv in qs:
+            offs += [qv, -qv]
+        offs += [Fraction(0)] * (256 - len(offs))
+        groups.append([1 + qv * s for qv in offs])
+        # the code each half-way quotient must take under round-half-to-even (by hand)
+        hand = {Fraction(127): 127, Fraction(5, 2): 2, Fraction(7, 2): 4, Fraction(1, 2): 0,
+                Fraction(3, 2): 2, Fraction(253, 2): 126, Fraction(0): 0, Fraction(3): 3,
+                Fraction(41, 4): 10}
+        want.append([hand[abs(qv)] * (1 if qv >= 0 else -1) for qv in offs])
+    return groups, want
+
+
+def test_dq_encode_rounds_half_to_even_on_exact_ties():
+    """Double quantisation's code is round-half-to-even of d / s_g (QLoRA page, "2. Double
+    Quantization", with the half-even reading): constructed exact ties 2.5 -> 2, 3.5 -> 4,
+    0.5 -> 0, 1.5 -> 2, 126.5 -> 126 and their negatives, with the mean and the group
+    scales exact. Half-away-from-zero, truncation or a floor would each fail here."""
+    groups, want = _dq_tie_groups()
+    a = np.array([float(v) for g in groups for v in g], dtype=np.float64)
+    assert all(Fraction(float(np.float32(v))) == v for g in groups for v in g)   # exact in fp32
+    a = a.astype(np.float32)
     qa, sc, mu = o.dq_encode(a)
-    d = a - mu
-    t = d / sc[0]
-    assert np.array_equal(qa, np.clip(np.rint(t), -127, 127).astype(np.int8))
+    assert mu == np.float32(1.0)
+    assert sc.tolist() == [2.0 ** -7, 2.0 ** -5]
+    assert qa.astype(int).tolist() == [c for w in want for c in w]
 
 
 # ---------------------------------------------------------------- int8 format
