@@ -135,19 +135,29 @@ def test_cfg3_upproj_full_size_sampled():
 def test_timeout_path_reports_and_recovers():
     """Force every bounded wait to give up almost at once: the kernels must return,
     report QL_ERR_TIMEOUT through the device flag, free their TMEM, and leave the
-    context usable for a normal run afterwards."""
-    case = synth.CFG1
+    context usable for a normal run afterwards.
+
+    With a 1 ns bound, any mbarrier wait that is not satisfied on its first poll gives
+    up at the next tick of the global timer. The epilogue warps of the fused GEMM wait
+    for the first accumulator during the whole first tile (the TMA loads from HBM, the
+    decode and 12 contraction chunks of 64), which spans many timer ticks, so the
+    timeout must be reported."""
+    case = synth.LinearCase("timeout-300x1024x768", N=1024, K=768, M=300, r=64, alpha=16.0, seed=4)
     inp = synth.make_inputs(case)
     qw = B.quantize_weight(inp["W"].cuda(), case.fmt)
     X, A, Bm = inp["X"].cuda(), inp["A"].cuda(), inp["B"].cuda()
+    torch.cuda.synchronize()
+    assert B.device_status() == B.QL_OK
     B.lib().ql_set_wait_timeout_ns(1)
     try:
         B.linear_fwd(qw, X, A, Bm, case.alpha)
         st = B.device_status()
     finally:
         B.lib().ql_set_wait_timeout_ns(0)
-    assert st in (B.QL_OK, B.QL_ERR_TIMEOUT)
+    assert st == B.QL_ERR_TIMEOUT, B.status_string(st)
+    assert B.device_status() == B.QL_OK                     # the flag was read and cleared
     check_case(case, inp)
+    check_case(synth.CFG1)
 
 
 # ---- decode-shaped forward (M <= 16): one cluster-split kernel ------------------------
