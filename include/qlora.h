@@ -36,6 +36,9 @@
  *    gave up) set a sticky device flag instead of trapping; ql_get_device_status
  *    reads and clears it.
  *  - Device pointers must be 16-byte aligned unless stated otherwise.
+ *  - The library looks up the device addresses of its own device-side objects (the
+ *    status flag, the no-allocation forward's scratch) once per device and keeps them
+ *    for the life of the process: do not use it across a cudaDeviceReset.
  */
 #ifndef QLORA_B200_H
 #define QLORA_B200_H
@@ -186,9 +189,13 @@ ql_status qlora_linear_bwd(const ql_weight* w, const ql_bf16* X, const ql_bf16* 
  * only changes where the scratch lives. Instead of a caller workspace it uses one fixed
  * 8 MiB array in the library's device image, which every GPU that loads the library holds
  * until the process exits. Shapes whose ql_workspace_bytes(QL_OP_FWD, ...) exceeds 8 MiB
- * are refused with QL_ERR_WORKSPACE (M <= 16 needs no scratch at all). The first call on a
- * device looks up the array's device address (cudaGetSymbolAddress) and caches it; a
- * failed lookup returns QL_ERR_CUDA. All calls share the one array and nothing
+ * are refused with QL_ERR_WORKSPACE, after the same argument checks as qlora_linear_fwd
+ * (so both return the same status for arguments that both refuse). A decode-shaped call
+ * (M <= 16, with a K and r that the decode-shaped path supports, i.e. where
+ * ql_workspace_bytes returns 0) needs no scratch at all. The first call on a device looks
+ * up the array's device address (cudaGetSymbolAddress) and caches it for the life of the
+ * process, so the library must not be used across a cudaDeviceReset; make that first call
+ * before any stream capture. A failed lookup returns QL_ERR_CUDA. All calls share the one array and nothing
  * in it needs to start at zero (every call rewrites what it reads), but calls that
  * overlap on the GPU (different streams, or different threads) race on it: serialise
  * them. Arguments and outputs are as for qlora_linear_fwd. */

@@ -572,7 +572,9 @@ namespace qlb {
 constexpr size_t kStaticScratchBytes = size_t(8) << 20;
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
-// Device address of the scratch array on the current device, looked up once per device.
+// Device address of the scratch array on the current device, looked up once per device and
+// kept for the life of the process (so the library must not be used across a
+// cudaDeviceReset, which may load the module at a new address).
 static void* static_scratch_ptr() {
   static std::mutex mu;
   static void* ptrs[128] = {nullptr};
@@ -592,9 +594,15 @@ static void* static_scratch_ptr() {
 extern "C" ql_status qlora_linear_fwd_static(const ql_weight* w, const ql_bf16* X, int64_t M,
                                              const ql_bf16* A, const ql_bf16* B, int32_t r, float alpha,
                                              ql_bf16* Y, ql_bf16* T_save, void* stream) {
+  // the same refusals, in the same order, as qlora_linear_fwd, so the two entry points
+  // return the same status for the same arguments; only then the scratch-size limit
   ql_status st0 = check_weight(w);
   if (st0 != QL_OK) return st0;
-  if (M < 1 || r < 1) return QL_ERR_INVALID_ARG;
+  if (!X || !A || !B || !Y || M < 1 || r < 1) return QL_ERR_INVALID_ARG;
+  if (r > 256 || M > (int64_t(1) << 31)) return QL_ERR_UNSUPPORTED;
+  if (!aligned(X, 16) || !aligned(A, 16) || !aligned(B, 2) || !aligned(Y, 16) ||
+      (T_save && !aligned(T_save, 2)))
+    return QL_ERR_INVALID_ARG;
   const size_t need = ql_workspace_bytes(QL_OP_FWD, M, w->N, w->K, r);
   if (need > kStaticScratchBytes) return QL_ERR_WORKSPACE;
   void* ws = static_scratch_ptr();
