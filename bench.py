@@ -808,15 +808,24 @@ def run_ours(args, case, world, rank, local_rank):
     Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     T = torch.empty((M, r), dtype=torch.bfloat16, device=dev)
     dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
-    dA = torch.empty((r, K), dtype=torch.float32, device=dev)
-    dB = torch.empty((N, r), dtype=torch.float32, device=dev)
+    # the adapter gradients live in the data-parallel exchange's bucket (written in place)
+    exchange = dp.BucketedGradExchange([(r, K, N)], device=dev) if dist is not None else None
+    if exchange is not None:
+        dA, dB = exchange.grads(0)
+    else:
+        dA = torch.empty((r, K), dtype=torch.float32, device=dev)
+        dB = torch.empty((N, r), dtype=torch.float32, device=dev)
+
+    def exchange_grads():
+        if exchange is not None:
+            exchange.ready(0)
+            exchange.finish()
 
     def step():
         B.nf4_dq_quantize(W, codes, absmax, qa, gs, mu)
         B.linear_fwd(qw, X, A, Bm, case.alpha, Y=Y, T=T)
         B.linear_bwd(qw, X, dY, A, Bm, T, case.alpha, dX=dX, dA=dA, dB=dB)
-        if dist is not None:
-            dp.allreduce_adapter_grads(dA, dB)
+        exchange_grads()
 
     def barrier():
         if dist is not None:
@@ -931,8 +940,7 @@ def run_ours(args, case, world, rank, local_rank):
         B.nf4_dq_quantize(Wj, codes, absmax, qa, gs, mu)
         B.linear_fwd(qw, Xj, Aj, Bj, case.alpha, Y=Y, T=T)
         B.linear_bwd(qw, Xj, dYj, Aj, Bj, T, case.alpha, dX=dX, dA=dA, dB=dB)
-        if dist is not None:
-            dp.allreduce_adapter_grads(dA, dB)
+        exchange_grads()
         used[j].record(cur)
         hdA.copy_(dA, non_blocking=True)
         hdB.copy_(dB, non_blocking=True)

@@ -4,8 +4,11 @@ quantisation sharded over ranks.
 Every rank holds the same quantised weight and adapter and its own shard of the tokens.
 The forward and dX need nothing from other ranks. The adapter gradients are sums over
 tokens (dA = s U^T X, dB = s dY^T T), so the full-batch gradients are the sums of the
-ranks' partial gradients: the only exchange is one all-reduce of dA and dB. Both go in
-one flat fp32 bucket, so the exchange is one collective per layer.
+ranks' partial gradients: the only exchange is one all-reduce of dA and dB. For one layer
+both go in one flat fp32 bucket (allreduce_adapter_grads). For a stack of layers,
+BucketedGradExchange puts several layers' gradients in each bucket and issues each
+bucket's all-reduce as soon as its layers' backward has been issued, so the exchange
+overlaps the backward of the layers that follow.
 """
 from __future__ import annotations
 
@@ -32,6 +35,82 @@ def allreduce_adapter_grads(dA: torch.Tensor, dB: torch.Tensor, group=None) -> N
     dist.all_reduce(bucket, op=dist.ReduceOp.SUM, group=group)
     dA.copy_(bucket[:dA.numel()].view_as(dA))
     dB.copy_(bucket[dA.numel():].view_as(dB))
+
+
+class BucketedGradExchange:
+    """The adapter-gradient exchange of a whole stack, bucketed across layers and
+    overlapped with the rest of the backward.
+
+    The backward visits the layers last to first. Each layer's dA [r, K] and dB [N, r]
+    (fp32) are views into one flat bucket, so the backward kernels write them in place
+    and nothing is copied. Buckets are filled in the order the gradients become ready,
+    up to `bucket_cap_bytes` each (a layer never straddles two buckets). As soon as every
+    layer of a bucket has reported ready(), the bucket's sum over ranks is issued as an
+    asynchronous all-reduce. With NCCL it runs on the library's communication stream after
+    the work already queued on the current stream, while the following layers' backward
+    kernels run. finish() makes the current stream wait for every bucket. Each bucket is
+    summed in one collective with the same element layout on every rank, and a sum of
+    world-size-2 contributions has one rounding, so the result is the same bit for bit as
+    one all-reduce per layer (allreduce_adapter_grads).
+
+    layers: (r, K, N) per layer, in the order their gradients become ready.
+    """
+
+    def __init__(self, layers, bucket_cap_bytes: int = 25 << 20, group=None, device=None):
+        if bucket_cap_bytes <= 0:
+            raise ValueError("bucket_cap_bytes must be positive")
+        self.group = group
+        sizes = [r * K + N * r for (r, K, N) in layers]
+        if any(r < 1 or K < 1 or N < 1 for (r, K, N) in layers):
+            raise ValueError("every layer needs r, K, N >= 1")
+        self.layer_bucket, self.layer_offset = [], []
+        bucket_elems = []
+        for n in sizes:
+            if not bucket_elems or (bucket_elems[-1] > 0 and 4 * (bucket_elems[-1] + n) > bucket_cap_bytes):
+                bucket_elems.append(0)
+            self.layer_bucket.append(len(bucket_elems) - 1)
+            self.layer_offset.append(bucket_elems[-1])
+            bucket_elems[-1] += n
+        self.buckets = [torch.zeros(n, dtype=torch.float32, device=device) for n in bucket_elems]
+        self._views = []
+        for (r, K, N), b, off in zip(layers, self.layer_bucket, self.layer_offset):
+            flat = self.buckets[b]
+            self._views.append((flat[off:off + r * K].view(r, K), flat[off + r * K:off + r * K + N * r].view(N, r)))
+        self._members = [sum(1 for b in self.layer_bucket if b == i) for i in range(len(self.buckets))]
+        self._left = list(self._members)
+        self._reported = [False] * len(layers)
+        self.works = [None] * len(self.buckets)
+        self.launch_order = []                   # bucket indices, in the order they were issued
+
+    def grads(self, layer: int):
+        """(dA, dB) of `layer`: the views its backward writes."""
+        return self._views[layer]
+
+    def ready(self, layer: int) -> None:
+        """The backward of `layer` has been issued on the current stream."""
+        if self._reported[layer]:
+            raise RuntimeError(f"layer {layer} reported twice in one step")
+        self._reported[layer] = True
+        b = self.layer_bucket[layer]
+        self._left[b] -= 1
+        if self._left[b] == 0:
+            if dist.is_initialized() and dist.get_world_size(self.group) > 1:
+                self.works[b] = dist.all_reduce(self.buckets[b], op=dist.ReduceOp.SUM, group=self.group,
+                                                async_op=True)
+            self.launch_order.append(b)
+
+    def finish(self) -> None:
+        """Wait (on the current stream) for every bucket, then reset for the next step."""
+        if not all(self._reported):
+            missing = [i for i, r in enumerate(self._reported) if not r]
+            raise RuntimeError(f"layers {missing} never reported ready")
+        for w in self.works:
+            if w is not None:
+                w.wait()
+        self.works = [None] * len(self.buckets)
+        self._left = list(self._members)
+        self._reported = [False] * len(self._reported)
+        self.launch_order = []
 
 
 GROUP_ELEMS = 64 * 256        # elements per double-quantisation group

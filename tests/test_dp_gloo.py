@@ -168,3 +168,91 @@ def test_data_parallel_step_with_optimisers_keeps_replicas_identical():
     sure = np.abs(g) > 1e-6 * np.abs(g).max()
     step = r0[1].astype(np.float64) - theta0.astype(np.float32).astype(np.float64) * (1 - 1e-5)
     assert np.all(np.sign(step[sure]) == -np.sign(g[sure]))
+
+
+# ---- bucketed, overlapped exchange across the layers of a stack ----------------------
+
+STACK = [synth.LinearCase(f"dp-stack-{i}", N=N, K=K, M=97, r=r, alpha=16.0, seed=20 + i)
+         for i, (N, K, r) in enumerate([(128, 192, 8), (256, 128, 16), (64, 256, 4), (192, 64, 32),
+                                        (128, 128, 8)])]
+CAP = 4 * (8 * 192 + 128 * 8 + 16 * 128 + 256 * 16)   # the first two layers fill one bucket
+
+
+def _stack_worker(rank, world, port, results):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        order = list(reversed(range(len(STACK))))          # the backward goes last layer first
+        ex = dp.BucketedGradExchange([(STACK[i].r, STACK[i].K, STACK[i].N) for i in order], CAP)
+        partial = {}
+        issued_before_last = []
+        for j, i in enumerate(order):
+            c = STACK[i]
+            inp = synth.make_inputs(c)
+            wd = o.quantize_weight(inp["W"].float().numpy(), c.fmt)["wdeq"].reshape(c.N, c.K)
+            s0, s1 = dp.shard_rows(c.M, world, rank)
+            f = lambda t: t.float().numpy().astype(np.float64)
+            _, dA, dB = o.linear_bwd(f(inp["X"])[s0:s1], f(inp["dY"])[s0:s1], wd, f(inp["A"]), f(inp["B"]),
+                                     c.alpha, c.r)
+            gA, gB = ex.grads(j)
+            gA.copy_(torch.from_numpy(dA.astype(np.float32)))
+            gB.copy_(torch.from_numpy(dB.astype(np.float32)))
+            partial[i] = (gA.clone(), gB.clone())
+            ex.ready(j)
+            if j < len(order) - 1:
+                issued_before_last.append(list(ex.launch_order))
+        ex.finish()
+        seq = {}
+        for i in order:                                      # one all-reduce per layer
+            tA, tB = partial[i]
+            dp.allreduce_adapter_grads(tA, tB)
+            seq[i] = (tA.numpy(), tB.numpy())
+        got = {i: tuple(t.clone().numpy() for t in ex.grads(j)) for j, i in enumerate(order)}
+        results[rank] = (got, seq, issued_before_last, ex.layer_bucket, len(ex.buckets))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bucketed_overlapped_exchange_equals_per_layer_allreduce():
+    world = 2
+    mgr = mp.get_context("spawn").Manager()
+    results = mgr.dict()
+    mp.start_processes(_stack_worker, args=(world, _free_port(), results), nprocs=world, join=True,
+                       start_method="spawn")
+    for rank in range(world):
+        got, seq, issued, layer_bucket, nb = results[rank]
+        assert nb >= 3 and layer_bucket == sorted(layer_bucket)
+        # each bucket's collective is issued as soon as its last layer is ready, before the
+        # backward of the remaining layers has been issued
+        assert issued[-1] == list(range(nb - 1))
+        for i in got:
+            assert np.array_equal(got[i][0], seq[i][0]) and np.array_equal(got[i][1], seq[i][1])
+            if rank:
+                assert np.array_equal(got[i][0], results[0][0][i][0])
+    # and the summed gradients are the full-batch ones
+    got = results[0][0]
+    for i, c in enumerate(STACK):
+        inp = synth.make_inputs(c)
+        wd = o.quantize_weight(inp["W"].float().numpy(), c.fmt)["wdeq"].reshape(c.N, c.K)
+        f = lambda t: t.float().numpy().astype(np.float64)
+        _, dA, dB = o.linear_bwd(f(inp["X"]), f(inp["dY"]), wd, f(inp["A"]), f(inp["B"]), c.alpha, c.r)
+        np.testing.assert_allclose(got[i][0], dA, rtol=1e-5, atol=1e-6 * np.abs(dA).max())
+        np.testing.assert_allclose(got[i][1], dB, rtol=1e-5, atol=1e-6 * np.abs(dB).max())
+
+
+def test_bucket_plan_without_a_process_group():
+    layers = [(8, 192, 128), (16, 128, 256), (4, 256, 64)]
+    ex = dp.BucketedGradExchange(layers, bucket_cap_bytes=1)      # one layer per bucket
+    assert ex.layer_bucket == [0, 1, 2]
+    ex = dp.BucketedGradExchange(layers, bucket_cap_bytes=1 << 30)
+    assert ex.layer_bucket == [0, 0, 0] and ex.buckets[0].numel() == sum(r * (K + N) for r, K, N in layers)
+    dA, dB = ex.grads(1)
+    assert dA.shape == (16, 128) and dB.shape == (256, 16) and dA.is_contiguous() and dB.is_contiguous()
+    for i in range(3):
+        ex.ready(i)
+    with pytest.raises(RuntimeError):
+        ex.ready(0)
+    ex.finish()
+    with pytest.raises(RuntimeError):
+        ex.finish()                                              # nothing reported this step
