@@ -28,43 +28,48 @@ namespace qlb {
 // bf16 |x|, an exact bf16 comparison done for two elements per instruction.
 // ---------------------------------------------------------------------------------
 
-// Two elements at a time in bf16x2 arithmetic: every value involved (the compare results
-// 0/1, counts up to 7, codes up to 15, 128 + code) is a small integer, exact in bf16.
-__device__ __forceinline__ uint32_t bf2_set_ge(uint32_t a, uint32_t b) {
+// Packed compares that return masks: 0xFFFF in each half where the comparison holds.
+__device__ __forceinline__ uint32_t bf2_ge_mask(uint32_t a, uint32_t b) {
   uint32_t d;
-  asm("set.ge.bf16x2.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  asm("set.ge.u32.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
 }
-__device__ __forceinline__ uint32_t bf2_set_lt(uint32_t a, uint32_t b) {
+__device__ __forceinline__ uint32_t bf2_lt_mask(uint32_t a, uint32_t b) {
   uint32_t d;
-  asm("set.lt.bf16x2.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  asm("set.lt.u32.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
 }
-__device__ __forceinline__ uint32_t bf2_add(uint32_t a, uint32_t b) {
+// m ? a : b, bit by bit (one LOP3)
+__device__ __forceinline__ uint32_t bit_select(uint32_t m, uint32_t a, uint32_t b) {
   uint32_t d;
-  asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  asm("lop3.b32 %0, %1, %2, %3, 0xCA;" : "=r"(d) : "r"(m), "r"(a), "r"(b));
   return d;
 }
-__device__ __forceinline__ uint32_t bf2_fma(uint32_t a, uint32_t b, uint32_t c) {
+// (a & b) ^ c (one LOP3)
+__device__ __forceinline__ uint32_t and_xor(uint32_t a, uint32_t b, uint32_t c) {
   uint32_t d;
-  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
   return d;
 }
 
-// Codes of the two elements of one bf16x2 word, returned as bf16x2 values 128 + code
-// (bits 0x4300 | code in each half). Cp[k] holds the boundary C_k in both halves.
-//   acc  = 8 + #{k : |x| >= C_k}                       (the code of a non-negative x)
-//   code = acc + neg * (15 - 2 acc)  = 7 - #{...} when x < 0 (strictly; -0 is not)
+// Codes of the two elements of one bf16x2 word, each in the low nibble of its half (the
+// rest of the half zero). Cp[k] holds the boundary C_{k+1} in both halves, C_1 < ... < C_7.
+// cnt = #{k : |x| >= C_k} by a three-step binary search over the sorted boundaries (three
+// packed compares; the next boundary is chosen by bit selects), then
+//   code = 8 + cnt = 8 ^ cnt  for x >= 0 (and -0),   7 - cnt = 7 ^ cnt  for x < 0.
+// A zero block has NaN boundaries, which no compare passes: cnt = 0 and every code is 8.
 __device__ __forceinline__ uint32_t nf4_code_pair(uint32_t w, const uint32_t (&Cp)[7]) {
-  constexpr uint32_t kOne8 = 0x41004100u;        // 8.0, 8.0
-  const uint32_t ax = w & 0x7FFF7FFFu;           // |x|, |x|
-  uint32_t acc = bf2_add(kOne8, bf2_set_ge(ax, Cp[0]));
-#pragma unroll
-  for (int k = 1; k < 7; ++k) acc = bf2_add(acc, bf2_set_ge(ax, Cp[k]));
-  const uint32_t neg = bf2_set_lt(w, 0u);                           // 1.0 where x < 0
-  const uint32_t t = bf2_fma(acc, 0xC000C000u /* -2 */, 0x41704170u /* 15 */);
-  const uint32_t code = bf2_fma(neg, t, acc);                        // 0..15
-  return bf2_add(code, 0x43004300u /* 128 */);
+  const uint32_t ax = w & 0x7FFF7FFFu;                       // |x|, |x|
+  const uint32_t f1 = bf2_ge_mask(ax, Cp[3]);               // cnt >= 4
+  const uint32_t t2 = bit_select(f1, Cp[5], Cp[1]);
+  const uint32_t u = bit_select(f1, Cp[6], Cp[2]);
+  const uint32_t v = bit_select(f1, Cp[4], Cp[0]);
+  const uint32_t f2 = bf2_ge_mask(ax, t2);                  // the next bit of cnt
+  const uint32_t f3 = bf2_ge_mask(ax, bit_select(f2, u, v));
+  // bit 2 from f1, bit 1 from f2, bit 0 from f3 (higher bits hold copies, masked below)
+  const uint32_t cnt = bit_select(0x00060006u, bit_select(0x00040004u, f1, f2), f3);
+  const uint32_t base = and_xor(bf2_lt_mask(w, 0u), 0x000F000Fu, 0x00080008u);   // 7 if x < 0, else 8
+  return and_xor(cnt, 0x00070007u, base);
 }
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
@@ -112,33 +117,6 @@ __device__ __forceinline__ void nf4_boundaries(uint32_t amax, const uint32_t* s_
   }
 }
 
-__device__ __forceinline__ void load_block(const uint16_t* __restrict__ W, int64_t base,
-                                           int64_t n, bool vec, uint32_t (&v)[32]) {
-  if (vec) {
-    const uint4* p = reinterpret_cast<const uint4*>(W + base);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      uint4 t = __ldg(p + i);
-      v[4 * i + 0] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int64_t e = base + 2 * i;
-      const uint32_t lo = e < n ? (uint32_t)W[e] : 0u;
-      const uint32_t hi = e + 1 < n ? (uint32_t)W[e + 1] : 0u;
-      v[i] = lo | (hi << 16);
-    }
-  }
-}
-
-__device__ __forceinline__ uint32_t block_absmax_bits(const uint32_t (&v)[32]) {
-  uint32_t m = 0;                                 // two 16-bit lanes of |x| bit patterns
-#pragma unroll
-  for (int i = 0; i < 32; ++i) m = __vmaxu2(m, v[i] & 0x7FFF7FFFu);
-  return max(m & 0xFFFFu, m >> 16);   // bf16 bits of max |x|; >= 0x7F80 means inf or NaN somewhere
-}
-
 // ---------------------------------------------------------------------------------
 // Double quantisation.
 //
@@ -165,8 +143,8 @@ __device__ __forceinline__ void dq_term(uint32_t u, uint32_t& bin, unsigned long
 }
 
 // Adds one group of lanes' terms (all lanes whose `bin` equals the leader's) into the
-// warp's shared bins. A term c < 2^42 is split at bit 20 so that the two 32-bit warp
-// sums cannot wrap (32 * 2^20 and 32 * 2^22 both fit).
+// warp's shared bins. A lane's value c < 2^63 (a running sum of terms below 2^39) is split
+// into 27-bit parts so that no 32-bit warp sum can wrap (32 * 2^27 = 2^32).
 __device__ __forceinline__ void bins_warp_add(unsigned long long* wbins, uint32_t bin, unsigned long long c,
                                               int lane) {
   uint32_t pending = __ballot_sync(0xFFFFFFFFu, c != 0ull);
@@ -174,9 +152,12 @@ __device__ __forceinline__ void bins_warp_add(unsigned long long* wbins, uint32_
     const int leader = __ffs(pending) - 1;
     const uint32_t lb = __shfl_sync(0xFFFFFFFFu, bin, leader);
     const bool mine = c != 0ull && bin == lb;
-    const uint32_t lo = __reduce_add_sync(0xFFFFFFFFu, mine ? (uint32_t)(c & 0xFFFFFu) : 0u);
-    const uint32_t hi = __reduce_add_sync(0xFFFFFFFFu, mine ? (uint32_t)(c >> 20) : 0u);
-    if (lane == 0) wbins[lb] += (unsigned long long)lo + ((unsigned long long)hi << 20);
+    constexpr unsigned long long kPart = (1ull << 27) - 1ull;
+    const uint32_t p0 = __reduce_add_sync(0xFFFFFFFFu, mine ? (uint32_t)(c & kPart) : 0u);
+    const uint32_t p1 = __reduce_add_sync(0xFFFFFFFFu, mine ? (uint32_t)((c >> 27) & kPart) : 0u);
+    const uint32_t p2 = __reduce_add_sync(0xFFFFFFFFu, mine ? (uint32_t)(c >> 54) : 0u);
+    if (lane == 0)
+      wbins[lb] += (unsigned long long)p0 + ((unsigned long long)p1 << 27) + ((unsigned long long)p2 << 54);
     pending &= ~__ballot_sync(0xFFFFFFFFu, mine);
   }
 }
@@ -303,14 +284,15 @@ __device__ __forceinline__ void dq_encode_group(const float* __restrict__ absmax
   }
 }
 
-// NF4 encode kernel. Two threads per block of 64: lanes 2t and 2t+1 of a warp take the
-// two halves of one block (32 elements, 64 bytes), combine their partial absmax with one
-// shuffle and each write 16 bytes of codes. The grid is persistent and the loop is
-// warp-uniform, so every lane takes part in the shuffles. VEC = true covers whole blocks
-// with 16-byte aligned input and codes, and loads the next block-half while it encodes
-// the current one; VEC = false (a ragged last block, or unaligned pointers) goes element
-// by element with bounds checks. DQ = true also accumulates the exact sum of the block
-// constants for double quantisation (dq_bins_finish).
+// NF4 encode kernel. One lane per block of 64 elements (128 bytes in, 32 bytes of codes
+// out); the grid is persistent and the loop warp-uniform, so every lane takes part in the
+// warp collectives. VEC = true covers whole blocks with 16-byte aligned input and codes,
+// and each lane loads its next block while it encodes the current one; VEC = false (a
+// ragged last block, or unaligned pointers) goes element by element with bounds checks.
+// DQ = true also accumulates the exact sum of the block constants for double
+// quantisation: each lane keeps a running sum for one bin of the exact integer sum (the
+// constants of a weight rarely span more than one bin of 16 binades) and the warp adds it
+// into its shared bins only when some lane's bin changes, and at the end (dq_bins_finish).
 constexpr int kNf4Threads = 256;
 constexpr uint64_t kDqWaitNs = 2000000000ull;   // bound of the fused quantise's wait for the mean
 
@@ -354,7 +336,7 @@ __device__ __forceinline__ void nf4_load_vec(const uint16_t* __restrict__ W, int
 // launch) and the grid's warps then encode the groups of 256 constants, so no second
 // launch is needed. The constants written by other CTAs are read from L2.
 template <bool VEC, bool DQ, bool FUSED = false>
-__global__ void __launch_bounds__(kNf4Threads, VEC ? 4 : 1)
+__global__ void __launch_bounds__(kNf4Threads, VEC ? 2 : 1)
 nf4_quantize_kernel(const Nf4Args args, const Nf4Tables tab, const Nf4BoundTable btab) {
   __shared__ __align__(16) uint32_t s_tab[128 * 8];
   __shared__ unsigned long long s_bins[DQ ? kNf4Warps : 1][kSumBins];
@@ -369,32 +351,40 @@ nf4_quantize_kernel(const Nf4Args args, const Nf4Tables tab, const Nf4BoundTable
 
   const uint16_t* __restrict__ W = args.W;
   const int64_t n = args.n;
-  const int64_t items = 2 * (args.blk_end - args.blk_begin);
+  const int64_t nblk = args.blk_end - args.blk_begin;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   bool bad = false;
+  uint32_t lbin = 0;                                  // DQ: this lane's running bin and sum
+  unsigned long long lsum = 0ull;
   int64_t w0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
-  uint4 nx[4];
+  uint4 nx[8];
   if (VEC) {
     const int64_t it = w0 + lane;
-    nf4_load_vec(W, (args.blk_begin + (it >> 1)) * kBlock + 32 * (it & 1), it < items, nx);
+    if (it < nblk) {
+      const uint4* src = reinterpret_cast<const uint4*>(W + (args.blk_begin + it) * kBlock);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) nx[i] = __ldg(src + i);
+    }
   }
-  for (; w0 < items; w0 += stride) {
+  for (; w0 < nblk; w0 += stride) {
     const int64_t it = w0 + lane;
-    const bool live = it < items;
-    const int64_t b = args.blk_begin + (it >> 1);
-    const int h = (int)(it & 1);
-    const int64_t base = b * kBlock + 32 * h;
-    uint32_t v[16];
+    const bool live = it < nblk;
+    const int64_t b = args.blk_begin + it;
+    const int64_t base = b * kBlock;
+    uint32_t v[32];
     if (VEC) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < 8; ++i) {
         v[4 * i + 0] = nx[i].x; v[4 * i + 1] = nx[i].y; v[4 * i + 2] = nx[i].z; v[4 * i + 3] = nx[i].w;
       }
-      const int64_t it1 = it + stride;                 // next block-half of this lane
-      nf4_load_vec(W, (args.blk_begin + (it1 >> 1)) * kBlock + 32 * (it1 & 1), it1 < items, nx);
+      if (it + stride < nblk) {                        // this lane's next block
+        const uint4* src = reinterpret_cast<const uint4*>(W + (b + stride) * kBlock);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) nx[i] = __ldg(src + i);
+      }
     } else {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < 32; ++i) {
         const int64_t e = base + 2 * i;
         const uint32_t lo = live && e < n ? (uint32_t)W[e] : 0u;
         const uint32_t hi = live && e + 1 < n ? (uint32_t)W[e + 1] : 0u;
@@ -406,35 +396,44 @@ nf4_quantize_kernel(const Nf4Args args, const Nf4Tables tab, const Nf4BoundTable
     // order of |x| is the order of its bit patterns, so this is the bitwise maximum
     uint32_t m = 0;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(m), "r"(v[i]));
+    for (int i = 0; i < 32; ++i) asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(m), "r"(v[i]));
     m &= 0x7FFF7FFFu;
-    m = __vmaxu2(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
     const uint32_t amax = max(m & 0xFFFFu, m >> 16);   // bf16 bits of the block's max |x|
-    const bool owner = live && h == 0;
-    if (owner) {
+    if (live) {
       if (amax >= 0x7F80u) raise_flag(args.flag, kFlagNonfinite);
       args.absmax[b] = __uint_as_float(amax << 16);
     }
     if (DQ) {
       uint32_t bin = 0;
       unsigned long long c = 0ull;
-      if (owner) dq_term(amax << 16, bin, c, bad);
-      bins_warp_add(s_bins[warp], bin, c, lane);
+      if (live) dq_term(amax << 16, bin, c, bad);
+      const bool move = c != 0ull && bin != lbin && lsum != 0ull;
+      if (__any_sync(0xFFFFFFFFu, move)) {           // some lane changes bin: flush the old sums
+        bins_warp_add(s_bins[warp], lbin, move ? lsum : 0ull, lane);
+        if (move) lsum = 0ull;
+      }
+      if (c != 0ull) {
+        lbin = bin;
+        lsum += c;                                      // < 2^63: at most 2^24 terms below 2^39
+      }
     }
     uint32_t Cp[7];
     nf4_boundaries(amax, s_tab, tab, Cp);
-    uint32_t out[4];
+    uint32_t out[8];
 #pragma unroll
-    for (int w = 0; w < 4; ++w)
+    for (int w = 0; w < 8; ++w)
       out[w] = nf4_pack8(nf4_code_pair(v[4 * w + 0], Cp), nf4_code_pair(v[4 * w + 1], Cp),
                          nf4_code_pair(v[4 * w + 2], Cp), nf4_code_pair(v[4 * w + 3], Cp));
-    uint8_t* dst = args.codes + b * 32 + 16 * h;
+    uint8_t* dst = args.codes + b * 32;
     if (VEC) {
-      if (live) *reinterpret_cast<uint4*>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
+      if (live) {
+        *reinterpret_cast<uint4*>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
+        *reinterpret_cast<uint4*>(dst + 16) = make_uint4(out[4], out[5], out[6], out[7]);
+      }
     } else if (live) {
-      const int64_t cnt = imin64(32, n - base);        // elements of this half (may be <= 0)
+      const int64_t cnt = imin64(64, n - base);        // elements of this block
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < 32; ++i) {
         if (2 * i >= cnt) break;
         uint8_t byte = (uint8_t)(out[i / 4] >> (8 * (i % 4)));
         if (2 * i + 1 >= cnt) byte &= 0x0F;              // no element: nibble 0
@@ -444,6 +443,7 @@ nf4_quantize_kernel(const Nf4Args args, const Nf4Tables tab, const Nf4BoundTable
   }
   if (DQ) {
     (void)bad;                                         // a non-finite absmax already raised the flag
+    bins_warp_add(s_bins[warp], lbin, lsum, lane);
     const bool last =
         dq_bins_finish(s_bins, kNf4Warps, args.dq_ws, args.dq_ctas, args.nb_total, args.mean, args.bins_out);
     if (FUSED) {
@@ -477,38 +477,93 @@ nf4_quantize_kernel(const Nf4Args args, const Nf4Tables tab, const Nf4BoundTable
 
 // ---------------------------------------------------------------------------------
 // Blockwise int8: sc = fp32(a/127); c = clamp(rint_half_even(fp32(x/sc)), -127, 127).
+//
+// One lane per block of 64 elements. The quotient fp32(x/sc) is formed from the block's
+// reciprocal r = fp32(1/sc) with one residual correction (Markstein's method: q0 = x r,
+// e = x - q0 sc exactly by FMA, q = q0 + e r rounded once), which yields the correctly
+// rounded quotient when nothing under- or overflows; blocks whose scale is below 2^-100
+// take the IEEE division instead. Rounding to an integer, half to even, is one add of
+// 1.5 * 2^23, after which the low byte of the sum's bits is the code in two's complement.
+// All of it runs on the FMA pipe except the bf16 unpacking and the byte packing.
 // ---------------------------------------------------------------------------------
 
-__device__ __forceinline__ uint32_t int8_code(uint32_t x16, float sc) {
-  if (sc == 0.0f) return 0u;
-  float t = rintf(__fdiv_rn(bf16_bits_to_float(x16), sc));
-  t = fminf(fmaxf(t, -127.0f), 127.0f);
-  return (uint32_t)((int32_t)t) & 0xFFu;
+constexpr float kInt8FastMinScale = 7.888609052210118e-31f;   // 2^-100
+constexpr float kRoundMagic = 12582912.0f;                     // 1.5 * 2^23
+
+// Code byte (low 8 bits) of the element x given the block scale.
+__device__ __forceinline__ uint32_t int8_byte(float x, float sc, float r, bool fast) {
+  float q;
+  if (fast) {
+    const float q0 = __fmul_rn(x, r);
+    const float e = __fmaf_rn(-q0, sc, x);
+    q = __fmaf_rn(e, r, q0);
+  } else {
+    q = sc == 0.0f ? 0.0f : __fdiv_rn(x, sc);
+  }
+  return __float_as_uint(__fadd_rn(fminf(fmaxf(q, -127.0f), 127.0f), kRoundMagic));
 }
 
+// Four elements in two bf16x2 words -> one word of four code bytes, element order kept.
+__device__ __forceinline__ uint32_t int8_word(uint32_t p0, uint32_t p1, float sc, float r, bool fast) {
+  const uint32_t b0 = int8_byte(__uint_as_float(p0 << 16), sc, r, fast);
+  const uint32_t b1 = int8_byte(__uint_as_float(p0 & 0xFFFF0000u), sc, r, fast);
+  const uint32_t b2 = int8_byte(__uint_as_float(p1 << 16), sc, r, fast);
+  const uint32_t b3 = int8_byte(__uint_as_float(p1 & 0xFFFF0000u), sc, r, fast);
+  return __byte_perm(__byte_perm(b0, b1, 0x0040u), __byte_perm(b2, b3, 0x0040u), 0x5410u);
+}
+
+// VEC: whole blocks, 16-byte aligned W and codes; each lane loads its next block while it
+// encodes the current one. Otherwise element loads with bounds checks (a ragged last
+// block, or unaligned pointers).
+template <bool VEC>
 __global__ void __launch_bounds__(256)
-int8_quantize_kernel(const uint16_t* __restrict__ W, int64_t n, int8_t* __restrict__ codes,
-                     float* __restrict__ absmax, int vec_ok, int* flag) {
-  const int64_t nb = (n + kBlock - 1) / kBlock;
+int8_quantize_kernel(const uint16_t* __restrict__ W, int64_t n, int64_t nb, int8_t* __restrict__ codes,
+                     float* __restrict__ absmax, int* flag) {
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nb; b += stride) {
-    const int64_t base = b * kBlock;
-    const bool full = base + kBlock <= n;
+  int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  uint4 nx[8];
+  if (VEC && b < nb) {
+    const uint4* src = reinterpret_cast<const uint4*>(W + b * kBlock);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) nx[i] = __ldg(src + i);
+  }
+  for (; b < nb; b += stride) {
     uint32_t v[32];
-    load_block(W, base, n, vec_ok && full, v);
-    const uint32_t amax = block_absmax_bits(v);
+    const int64_t base = b * kBlock;
+    if (VEC) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[4 * i] = nx[i].x; v[4 * i + 1] = nx[i].y; v[4 * i + 2] = nx[i].z; v[4 * i + 3] = nx[i].w;
+      }
+      if (b + stride < nb) {
+        const uint4* src = reinterpret_cast<const uint4*>(W + (b + stride) * kBlock);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) nx[i] = __ldg(src + i);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int64_t e = base + 2 * i;
+        const uint32_t lo = e < n ? (uint32_t)W[e] : 0u;
+        const uint32_t hi = e + 1 < n ? (uint32_t)W[e + 1] : 0u;
+        v[i] = lo | (hi << 16);
+      }
+    }
+    uint32_t m = 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(m), "r"(v[i]));
+    m &= 0x7FFF7FFFu;
+    const uint32_t amax = max(m & 0xFFFFu, m >> 16);
     if (amax >= 0x7F80u) raise_flag(flag, kFlagNonfinite);
     const float a = __uint_as_float(amax << 16);
     absmax[b] = a;
     const float sc = __fdiv_rn(a, 127.0f);
+    const bool fast = sc >= kInt8FastMinScale && sc < 3.0e38f;
+    const float r = fast ? __frcp_rn(sc) : 0.0f;
     uint32_t out[16];
 #pragma unroll
-    for (int w = 0; w < 16; ++w) {
-      const uint32_t p0 = v[2 * w], p1 = v[2 * w + 1];
-      out[w] = int8_code(p0 & 0xFFFFu, sc) | (int8_code(p0 >> 16, sc) << 8) |
-               (int8_code(p1 & 0xFFFFu, sc) << 16) | (int8_code(p1 >> 16, sc) << 24);
-    }
-    if (vec_ok && full) {
+    for (int w = 0; w < 16; ++w) out[w] = int8_word(v[2 * w], v[2 * w + 1], sc, r, fast);
+    if (VEC) {
       uint4* dst = reinterpret_cast<uint4*>(codes + base);
 #pragma unroll
       for (int i = 0; i < 4; ++i) dst[i] = make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
@@ -665,11 +720,11 @@ static ql_status launch_nf4(const uint16_t* W, int64_t n, uint8_t* codes, float*
   int g_vec = 0, g_tail = 0;
   if (nb_vec > 0) {
     static const int per_sm = resident_ctas(nf4_quantize_kernel<true, true>, kNf4Threads);
-    const int64_t need = (2 * nb_vec + kNf4Threads - 1) / kNf4Threads;
+    const int64_t need = (nb_vec + kNf4Threads - 1) / kNf4Threads;
     g_vec = (int)imax64(1, imin64(need, (int64_t)num_sms() * per_sm));
   }
   if (nb_vec < nb) {
-    const int64_t need = (2 * (nb - nb_vec) + kNf4Threads - 1) / kNf4Threads;
+    const int64_t need = (nb - nb_vec + kNf4Threads - 1) / kNf4Threads;
     g_tail = (int)imax64(1, imin64(need, (int64_t)num_sms() * 4));
   }
   Nf4Args a;
@@ -703,7 +758,7 @@ static ql_status launch_nf4_dq_fused(const uint16_t* W, int64_t n, uint8_t* code
   auto kern = nf4_quantize_kernel<true, true, true>;
   static const int per_sm = resident_ctas(kern, kNf4Threads);
   const int64_t nb = n / kBlock;
-  const int64_t need = (2 * nb + kNf4Threads - 1) / kNf4Threads;
+  const int64_t need = (nb + kNf4Threads - 1) / kNf4Threads;
   const int grid = (int)imax64(1, imin64(need, (int64_t)num_sms() * per_sm));
   Nf4Args a;
   a.W = W; a.n = n; a.blk_begin = 0; a.blk_end = nb; a.codes = codes; a.absmax = absmax;
@@ -761,12 +816,23 @@ ql_status int8_quantize(const ql_bf16* W, int64_t n, int8_t* codes, float* absma
   if (n == 0) return QL_OK;
   if (!W || !codes || !absmax) return QL_ERR_INVALID_ARG;
   if (!aligned(W, 2) || !aligned(absmax, 4)) return QL_ERR_INVALID_ARG;
-  const int vec = aligned(W, 16) && aligned(codes, 16);
+  const bool vec = aligned(W, 16) && aligned(codes, 16);
   const int64_t nb = (n + kBlock - 1) / kBlock;
-  ProfScope prof(PK_INT8, as_stream(stream), 1);
-  int8_quantize_kernel<<<grid_for(nb, 256), 256, 0, as_stream(stream)>>>(
-      W, n, codes, absmax, vec, device_flag_ptr());
-  QL_CHECK_LAUNCH();
+  const int64_t nb_full = vec ? n / kBlock : 0;       // whole blocks on the vector path
+  cudaStream_t st = as_stream(stream);
+  ProfScope prof(PK_INT8, st, (nb_full > 0) + (nb_full < nb));
+  if (nb_full > 0) {
+    int8_quantize_kernel<true><<<grid_for(nb_full, 256), 256, 0, st>>>(W, n, nb_full, codes, absmax,
+                                                                      device_flag_ptr());
+    QL_CHECK_LAUNCH();
+  }
+  if (nb_full < nb) {
+    // the rest (a ragged last block, or every block when unaligned), offset to its first block
+    const int64_t off = nb_full * kBlock;
+    int8_quantize_kernel<false><<<grid_for(nb - nb_full, 256), 256, 0, st>>>(
+        W + off, n - off, nb - nb_full, codes + off, absmax + nb_full, device_flag_ptr());
+    QL_CHECK_LAUNCH();
+  }
   return QL_OK;
 }
 

@@ -124,6 +124,44 @@ def test_int8_bitexact(name, W):
     assert B.device_status() == B.QL_OK
 
 
+def _int8_exhaustive_blocks():
+    """For each of 473 absmax values a (43 mantissas at each of 11 exponents, the
+    subnormal range, the smallest normals and the largest finite included), every bf16
+    magnitude <= a in both signs, 63 to a block with +a first so that each block's absmax
+    is a. Every quotient x / (a/127) an element of such a block can produce is covered."""
+    rows = []
+    for e in (0, 1, 2, 20, 60, 100, 120, 127, 140, 200, 254):
+        for m in range(0, 128, 3):
+            ab = (e << 7) | m
+            if ab == 0:
+                continue
+            mags = np.arange(0, ab + 1, dtype=np.uint32)
+            vals = np.concatenate([mags, mags | 0x8000])
+            pad = (-vals.size) % 63
+            vals = np.concatenate([vals, np.zeros(pad, np.uint32)]).reshape(-1, 63)
+            blk = np.empty((vals.shape[0], 64), np.uint32)
+            blk[:, 0] = ab
+            blk[:, 1:] = vals
+            rows.append(blk)
+    bits = np.concatenate(rows).ravel().astype(np.uint16)
+    return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+
+
+def test_int8_every_bf16_below_many_absmax():
+    """The fast quotient (reciprocal plus one residual correction) and the add-based
+    half-even rounding give the oracle's codes, bit for bit, on every element value."""
+    W = _int8_exhaustive_blocks()
+    w = W.float().numpy()
+    codes, absmax = B.int8_quantize(W.cuda())
+    ref_c, ref_a = o.int8_quantize(w)
+    got = codes.cpu().numpy()
+    bad = np.flatnonzero(got != ref_c)
+    assert bad.size == 0, (f"{bad.size} codes differ; first at {bad[0]}: x={w[bad[0]]!r} "
+                           f"a={ref_a[bad[0] // 64]!r} got {got[bad[0]]} want {ref_c[bad[0]]}")
+    assert np.array_equal(_u32(absmax.cpu().numpy()), _u32(ref_a))
+    assert B.device_status() == B.QL_OK
+
+
 def test_unaligned_input_takes_scalar_path():
     W = synth.normal_bf16((64 * 300 + 3,), 0.02, 6, 0).cuda()
     Wu = W[1:]                                   # 2-byte aligned, not 16
