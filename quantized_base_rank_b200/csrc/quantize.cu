@@ -163,44 +163,47 @@ __device__ __forceinline__ void bins_warp_add(unsigned long long* wbins, uint32_
 }
 
 // Turn the bins into the exact integer X (value X * 2^-149), round it to fp64 (nearest,
-// ties to even), and return mean = fp32(fp64(S) / nb). One thread's work.
+// ties to even), and return mean = fp32(fp64(S) / nb). One thread's work. Every array
+// index is a compile-time constant (the loops are unrolled), so the big integer stays in
+// registers: X < 16 * 2^63 * 2^240 = 2^307 fits five 64-bit limbs.
 __device__ float dq_mean_from_bins(const unsigned long long (&bins)[16], int64_t nb) {
-  uint32_t limb[12];                                   // 384-bit little-endian integer
-  for (int i = 0; i < 12; ++i) limb[i] = 0u;
-  for (int i = 0; i < kSumBins; ++i) {
-    const unsigned long long v = bins[i];
-    const int bit = 16 * i;
-    const int li = bit / 32;
-    const unsigned long long lo = (bit % 32) ? (v << 16) : v;
-    const uint32_t parts[3] = {(uint32_t)lo, (uint32_t)(lo >> 32), (bit % 32) ? (uint32_t)(v >> 48) : 0u};
-    unsigned long long carry = 0;
-    for (int k = 0; li + k < 12; ++k) {
-      const unsigned long long sum = (unsigned long long)limb[li + k] + (k < 3 ? parts[k] : 0u) + carry;
-      limb[li + k] = (uint32_t)sum;
-      carry = sum >> 32;
-      if (k >= 2 && carry == 0) break;
-    }
+  unsigned __int128 acc[6] = {0, 0, 0, 0, 0, 0};
+#pragma unroll
+  for (int i = 0; i < kSumBins; ++i) {                // bin i has weight 2^(16 i)
+    const unsigned __int128 v = (unsigned __int128)bins[i] << (16 * (i % 4));   // < 2^111
+    acc[i / 4] += (unsigned long long)v;
+    acc[i / 4 + 1] += (unsigned long long)(v >> 64);
+  }
+  unsigned long long limb[6];
+#pragma unroll
+  for (int j = 0; j < 6; ++j) {                       // each acc < 2^67 before its carry-in
+    limb[j] = (unsigned long long)acc[j];
+    if (j < 5) acc[j + 1] += acc[j] >> 64;
   }
   int top = -1;
-  for (int i = 11; i >= 0; --i)
-    if (limb[i]) { top = i; break; }
+#pragma unroll
+  for (int j = 0; j < 6; ++j)
+    if (limb[j]) top = j;
   double S = 0.0;
-  if (top >= 0) {
-    // 96-bit window of limbs top, top-1, top-2 (missing limbs are zero)
-    const uint32_t l1 = top >= 1 ? limb[top - 1] : 0u, l2 = top >= 2 ? limb[top - 2] : 0u;
-    const unsigned __int128 W = ((unsigned __int128)limb[top] << 64) | ((unsigned __int128)l1 << 32) | l2;
-    const int tb = 95 - __clz(limb[top]);              // top set bit inside W (>= 64)
-    const int base = 32 * (top - 2);                   // weight of bit 0 of W
-    if (base + tb < 53) {
-      S = ldexp((double)(unsigned long long)(W >> (base < 0 ? -base : 0)), base > 0 ? base - 149 : -149);
-    } else {
-      unsigned long long mant = (unsigned long long)(W >> (tb - 52));
-      const uint32_t rbit = (uint32_t)(W >> (tb - 53)) & 1u;
-      bool sticky = (W & ((((unsigned __int128)1) << (tb - 53)) - 1)) != 0;
-      for (int i = 0; i < top - 2 && !sticky; ++i) sticky = limb[i] != 0u;
-      if (rbit && (sticky || (mant & 1ull))) mant += 1ull;
-      S = ldexp((double)mant, base + tb - 52 - 149);   // exact scaling
+  if (top == 0) {
+    S = ldexp(__ull2double_rn(limb[0]), -149);        // one rounding of a 64-bit integer
+  } else if (top > 0) {
+    // the 128-bit window of limbs top and top - 1, and whether anything below it is set
+    unsigned long long hi = 0, lo = 0;
+    bool sticky = false;
+#pragma unroll
+    for (int j = 0; j < 6; ++j) {
+      if (j == top) hi = limb[j];
+      if (j == top - 1) lo = limb[j];
+      if (j < top - 1 && limb[j]) sticky = true;
     }
+    const unsigned __int128 W = ((unsigned __int128)hi << 64) | lo;
+    const int tb = 127 - __clzll((long long)hi);     // top set bit of W, >= 64
+    unsigned long long mant = (unsigned long long)(W >> (tb - 52));
+    const unsigned rbit = (unsigned)(W >> (tb - 53)) & 1u;
+    sticky = sticky || (W & ((((unsigned __int128)1) << (tb - 53)) - 1)) != 0;
+    if (rbit && (sticky || (mant & 1ull))) mant += 1ull;
+    S = ldexp((double)mant, 64 * (top - 1) + tb - 52 - 149);   // exact scaling
   }
   return __double2float_rn(__ddiv_rn(S, (double)nb));
 }
