@@ -118,6 +118,32 @@ __device__ __forceinline__ void nf4_boundaries(uint32_t amax, const uint32_t* s_
 }
 
 // ---------------------------------------------------------------------------------
+// Integer codes clamp(rint_half_even(fp32(x / sc)), -127, 127), shared by the blockwise
+// int8 format and the double-quantised constants. The quotient comes from the reciprocal
+// r = fp32(1/sc) and one residual correction (Markstein's method: q0 = x r, e = x - q0 sc
+// exactly by FMA, q = q0 + e r rounded once), the correctly rounded quotient when nothing
+// under- or overflows; scales below 2^-100 take the IEEE division. Rounding to an integer,
+// half to even, is one add of 1.5 * 2^23, after which the low byte of the sum's bits is the
+// code in two's complement.
+// ---------------------------------------------------------------------------------
+
+constexpr float kInt8FastMinScale = 7.888609052210118e-31f;   // 2^-100
+constexpr float kRoundMagic = 12582912.0f;                     // 1.5 * 2^23
+
+// Code byte (low 8 bits) of the element x given the block scale.
+__device__ __forceinline__ uint32_t int8_byte(float x, float sc, float r, bool fast) {
+  float q;
+  if (fast) {
+    const float q0 = __fmul_rn(x, r);
+    const float e = __fmaf_rn(-q0, sc, x);
+    q = __fmaf_rn(e, r, q0);
+  } else {
+    q = sc == 0.0f ? 0.0f : __fdiv_rn(x, sc);
+  }
+  return __float_as_uint(__fadd_rn(fminf(fmaxf(q, -127.0f), 127.0f), kRoundMagic));
+}
+
+// ---------------------------------------------------------------------------------
 // Double quantisation.
 //
 // The mean needs the exact sum of the constants, rounded once to fp64. It is
@@ -273,16 +299,52 @@ __device__ __forceinline__ void dq_encode_group(const float* __restrict__ absmax
     for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
     const float s = __fdiv_rn(mx, 127.0f);
     if (lane == 0) group_scale[g] = s;
+    const bool fast = s >= kInt8FastMinScale && s < 3.0e38f;
+    const float r = fast ? __frcp_rn(s) : 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int64_t b = g * kGroup + i * 32 + lane;
       if (b >= nb) continue;
-      int8_t c = 0;
-      if (s != 0.0f) {
-        float t = rintf(__fdiv_rn(d[i], s));
-        c = (int8_t)(int32_t)fminf(fmaxf(t, -127.0f), 127.0f);
-      }
-      qabsmax[b] = c;
+      qabsmax[b] = (int8_t)int8_byte(d[i], s, r, fast);
+    }
+  }
+}
+
+// Groups g[0..G-1] (a value >= ng is skipped) by one warp, as dq_encode_group<true>, with
+// the loads of every group issued before any is used, so their round trips to L2 overlap.
+template <int G>
+__device__ __forceinline__ void dq_encode_groups_cg(const float* __restrict__ absmax, int64_t nb, float mu,
+                                                    int8_t* __restrict__ qabsmax, float* __restrict__ group_scale,
+                                                    const int64_t (&g)[G], int lane) {
+  float d[G][8];
+#pragma unroll
+  for (int j = 0; j < G; ++j)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int64_t b = g[j] * kGroup + i * 32 + lane;
+      d[j][i] = b < nb ? __ldcg(absmax + b) : mu;     // a value past the end gives d = 0
+    }
+#pragma unroll
+  for (int j = 0; j < G; ++j) {
+    float mx = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      d[j][i] = __fsub_rn(d[j][i], mu);
+      mx = fmaxf(mx, fabsf(d[j][i]));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+    const float s = __fdiv_rn(mx, 127.0f);
+    const int64_t ng = (nb + kGroup - 1) / kGroup;
+    if (g[j] >= ng) continue;                        // warp-uniform
+    if (lane == 0) group_scale[g[j]] = s;
+    const bool fast = s >= kInt8FastMinScale && s < 3.0e38f;
+    const float r = fast ? __frcp_rn(s) : 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int64_t b = g[j] * kGroup + i * 32 + lane;
+      if (b >= nb) continue;
+      qabsmax[b] = (int8_t)int8_byte(d[j][i], s, r, fast);
     }
   }
 }
@@ -450,30 +512,36 @@ nf4_quantize_kernel(const Nf4Args args, const Nf4Tables tab, const Nf4BoundTable
     const bool last =
         dq_bins_finish(s_bins, kNf4Warps, args.dq_ws, args.dq_ctas, args.nb_total, args.mean, args.bins_out);
     if (FUSED) {
+      // the ready word: 1 in the low half once the mean is written, the mean's bits in the
+      // high half, so the waiting CTAs get the mean with the same acquire load
       __shared__ int s_ok;
-      unsigned int* ready = reinterpret_cast<unsigned int*>(args.dq_ws + kSumBins + 1);
+      __shared__ float s_mu;
+      unsigned long long* ready = args.dq_ws + kSumBins + 1;
       if (threadIdx.x == 0) {
         if (last) {
-          __threadfence();                             // the mean before the flag
-          atomicExch(ready, 1u);
+          const unsigned long long word = 1ull | ((unsigned long long)__float_as_uint(*args.mean) << 32);
+          asm volatile("st.release.gpu.global.u64 [%0], %1;" :: "l"(ready), "l"(word) : "memory");
         }
-        unsigned int v = 0u;
+        unsigned long long v = 0ull;
         const uint64_t t0 = qt_globaltimer_ns();
         for (;;) {
-          asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ready) : "memory");
-          if (v || qt_globaltimer_ns() - t0 > kDqWaitNs) break;
+          asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(ready) : "memory");
+          if ((v & 1ull) || qt_globaltimer_ns() - t0 > kDqWaitNs) break;
           __nanosleep(64);
         }
-        s_ok = v != 0u;
-        if (!v) raise_flag(args.flag, kFlagTimeout);
+        s_ok = (v & 1ull) != 0ull;
+        s_mu = __uint_as_float((uint32_t)(v >> 32));
+        if (!s_ok) raise_flag(args.flag, kFlagTimeout);
       }
       __syncthreads();
       if (!s_ok) return;
-      const float mu = __ldcg(args.mean);
+      const float mu = s_mu;
       const int64_t ng = (args.nb_total + kGroup - 1) / kGroup;
       const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-      for (int64_t g = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; g < ng; g += warps)
-        dq_encode_group<true>(args.absmax, args.nb_total, mu, args.qabsmax, args.group_scale, g, lane);
+      for (int64_t g = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; g < ng; g += 2 * warps) {
+        const int64_t gg[2] = {g, g + warps};
+        dq_encode_groups_cg<2>(args.absmax, args.nb_total, mu, args.qabsmax, args.group_scale, gg, lane);
+      }
     }
   }
 }
@@ -489,22 +557,6 @@ nf4_quantize_kernel(const Nf4Args args, const Nf4Tables tab, const Nf4BoundTable
 // 1.5 * 2^23, after which the low byte of the sum's bits is the code in two's complement.
 // All of it runs on the FMA pipe except the bf16 unpacking and the byte packing.
 // ---------------------------------------------------------------------------------
-
-constexpr float kInt8FastMinScale = 7.888609052210118e-31f;   // 2^-100
-constexpr float kRoundMagic = 12582912.0f;                     // 1.5 * 2^23
-
-// Code byte (low 8 bits) of the element x given the block scale.
-__device__ __forceinline__ uint32_t int8_byte(float x, float sc, float r, bool fast) {
-  float q;
-  if (fast) {
-    const float q0 = __fmul_rn(x, r);
-    const float e = __fmaf_rn(-q0, sc, x);
-    q = __fmaf_rn(e, r, q0);
-  } else {
-    q = sc == 0.0f ? 0.0f : __fdiv_rn(x, sc);
-  }
-  return __float_as_uint(__fadd_rn(fminf(fmaxf(q, -127.0f), 127.0f), kRoundMagic));
-}
 
 // Four elements in two bf16x2 words -> one word of four code bytes, element order kept.
 __device__ __forceinline__ uint32_t int8_word(uint32_t p0, uint32_t p1, float sc, float r, bool fast) {
@@ -825,8 +877,11 @@ ql_status int8_quantize(const ql_bf16* W, int64_t n, int8_t* codes, float* absma
   cudaStream_t st = as_stream(stream);
   ProfScope prof(PK_INT8, st, (nb_full > 0) + (nb_full < nb));
   if (nb_full > 0) {
-    int8_quantize_kernel<true><<<grid_for(nb_full, 256), 256, 0, st>>>(W, n, nb_full, codes, absmax,
-                                                                      device_flag_ptr());
+    // persistent: the CTAs that fit at once, each lane loading its next block while it
+    // encodes the current one
+    static const int per_sm = resident_ctas(int8_quantize_kernel<true>, 256);
+    const int grid = (int)imax64(1, imin64((nb_full + 255) / 256, (int64_t)num_sms() * per_sm));
+    int8_quantize_kernel<true><<<grid, 256, 0, st>>>(W, n, nb_full, codes, absmax, device_flag_ptr());
     QL_CHECK_LAUNCH();
   }
   if (nb_full < nb) {
