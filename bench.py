@@ -378,6 +378,60 @@ def as_weight(fmt, N, K, outs):
     return B.QuantWeight(fmt, N, K, codes, absmax)
 
 
+def graph_us(fn, reps: int = 20) -> float:
+    """Device time of one fn() call: reps calls captured in one CUDA graph and replayed, so
+    the host's launch overhead is not in the figure."""
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    st = torch.cuda.Stream()
+    st.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(st):
+        with torch.cuda.graph(g, stream=st):
+            for _ in range(reps):
+                fn()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) * 1e3 / reps
+
+
+def quant_bench(dev, peaks, reps: int = 20, shapes=((4096, 4096), (11008, 4096), (22016, 8192))):
+    """Quantise alone, device time per weight (CUDA-graph replay of back-to-back calls over
+    three bf16 source copies, so each call reads its source from HBM): NF4 + double
+    quantisation in one call, and blockwise int8, on the 7B-shaped 4096x4096 and 11008x4096
+    weights and the 65B-shaped 22016x8192 one. GB/s of algorithmic bytes (2.516 and 3.0625
+    B/param)."""
+    from quantized_base_rank_b200 import synth
+    out = {}
+    for (N, K) in shapes:
+        n = N * K
+        Ws = [synth.device_normal_bf16((N, K), 0.02, 0, 400 + c, dev) for c in range(3)]
+        i = [0]
+
+        def nxt():
+            i[0] += 1
+            return Ws[i[0] % 3]
+
+        for fmt, bpp in (("nf4_dq", NF4_DQ_BYTES_PER_PARAM), ("int8", INT8_BYTES_PER_PARAM)):
+            outs = quant_outputs(fmt, n, dev)
+            us = graph_us(lambda: quantize_into(fmt, nxt(), outs), reps)
+            gbs = bpp * n / (us * 1e-6) / 1e9
+            out[f"{N}x{K}_{fmt}"] = {"us": us, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
+                                     "hbm_floor_us": bpp * n / (peaks["hbm_gbs"] * 1e3)}
+            del outs
+        del Ws
+        torch.cuda.empty_cache()
+    return out
+
+
 def layer_bench(dev, peaks, N, K, M, r, fmt, reps: int = 5, seed: int = 0, idx: int = 0):
     """One quantised linear W [N, K] in format `fmt` at M tokens and rank r: the quantise
     (GB/s of algorithmic bytes; the bf16 source rotates over enough copies to exceed 3x
@@ -391,16 +445,13 @@ def layer_bench(dev, peaks, N, K, M, r, fmt, reps: int = 5, seed: int = 0, idx: 
     Ws = [synth.device_normal_bf16((N, K), 0.02, seed, idx + c, dev) for c in range(copies)]
     outs = quant_outputs(fmt, n, dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for Wc in Ws:
-        quantize_into(fmt, Wc, outs)
-    torch.cuda.synchronize()
-    e0.record()
-    for _ in range(reps):
-        for Wc in Ws:
-            quantize_into(fmt, Wc, outs)
-    e1.record()
-    torch.cuda.synchronize()
-    q_us = e0.elapsed_time(e1) * 1e3 / (reps * copies)
+    qi = [0]
+
+    def nxt():
+        qi[0] += 1
+        return Ws[qi[0] % copies]
+
+    q_us = graph_us(lambda: quantize_into(fmt, nxt(), outs), max(4, reps * copies))
     bpp = NF4_DQ_BYTES_PER_PARAM if fmt == "nf4_dq" else INT8_BYTES_PER_PARAM
     q_gbs = bpp * n / (q_us * 1e-6) / 1e9
     del Ws
@@ -470,9 +521,10 @@ def layers_bench(dev, peaks, reps: int = 5):
 
 def stack_bench(dev, peaks, M: int = 4096, reps: int = 2):
     """The 32-layer 7B-shaped stack: every one of its 224 bf16 weights is drawn on the
-    device (13 GB of sources), then (1) the whole stack is quantised to NF4+DQ, timed as one
-    region (16.3 GB of algorithmic traffic), and (2) every linear runs its forward at M
-    tokens with a rank-64 adapter, timed as one region."""
+    device (13 GB of sources), then (1) the whole stack is quantised to NF4+DQ by the batched
+    entry, timed as one region (16.3 GB of algorithmic traffic), with one call per weight
+    timed beside it, and (2) every linear runs its forward at M tokens with a rank-64
+    adapter, timed as one region."""
     from quantized_base_rank_b200 import binding as B
     from quantized_base_rank_b200 import stack, synth
     specs = stack.stack_7b()
@@ -481,16 +533,21 @@ def stack_bench(dev, peaks, M: int = 4096, reps: int = 2):
     outs = [quant_outputs("nf4_dq", sp.N * sp.K, dev) for sp in specs]
     n_total = sum(sp.N * sp.K for sp in specs)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for Wc, o in zip(srcs, outs):
-        quantize_into("nf4_dq", Wc, o)
-    torch.cuda.synchronize()
-    e0.record()
-    for _ in range(reps):
-        for Wc, o in zip(srcs, outs):
-            quantize_into("nf4_dq", Wc, o)
-    e1.record()
-    torch.cuda.synchronize()
-    q_ms = e0.elapsed_time(e1) / reps
+
+    def timed_ms(fn):
+        fn()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    # the whole stack in one batched call (three launches per 128 weights), and, beside it,
+    # one nf4_dq_quantize call per weight
+    q_ms = timed_ms(lambda: B.nf4_dq_quantize_batch(srcs, outs))
+    q_ms_each = timed_ms(lambda: [quantize_into("nf4_dq", Wc, o) for Wc, o in zip(srcs, outs)])
     q_gbs = NF4_DQ_BYTES_PER_PARAM * n_total / (q_ms * 1e-3) / 1e9
     del srcs
     torch.cuda.empty_cache()
@@ -527,7 +584,8 @@ def stack_bench(dev, peaks, M: int = 4096, reps: int = 2):
     return {"linears": len(specs), "params": n_total, "stored_bytes": acct["weight_bytes"],
             "bits_per_param": acct["bits_per_param"],
             "quantize_all": {"ms": q_ms, "GB/s": q_gbs, "frac_hbm": q_gbs / peaks["hbm_gbs"],
-                             "algorithmic_bytes": NF4_DQ_BYTES_PER_PARAM * n_total},
+                             "algorithmic_bytes": NF4_DQ_BYTES_PER_PARAM * n_total, "call": "nf4_dq_quantize_batch",
+                             "one_call_per_weight_ms": q_ms_each},
             "forward_all_M4096_r64": {"ms": f_ms, "TFLOP": flops / 1e12, "TFLOP/s": flops / (f_ms * 1e-3) / 1e12,
                                       "main_gemm_ms": main_ms,
                                       "main_gemm_TFLOP/s": main_flops / (main_ms * 1e-3) / 1e12,
@@ -965,6 +1023,9 @@ def run_ours(args, case, world, rank, local_rank):
     # ---- adapter optimiser step with paged states ----
     optim = optim_bench(dev, peaks)
 
+    # ---- quantise alone, device time (CUDA graphs) ----
+    quant = quant_bench(dev, peaks)
+
     # ---- the int8 format and the 65B-shaped layers; the whole 7B stack ----
     layers = layers_bench(dev, peaks) if not args.skip_extra else None
     torch.cuda.empty_cache()
@@ -1027,6 +1088,7 @@ def run_ours(args, case, world, rank, local_rank):
             "lordba": lordba,
             "qwha": qwha,
             "optimizer_adamw_7b_r64": optim,
+            "quantize_alone": quant,
             "layers": layers,
             "stack_7b_32x7": stack7b,
         },
@@ -1048,9 +1110,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--gemm", choices=["pair", "single"], default="single",
                     help="fused weight GEMM on CTA pairs (cta_group::2) or on single CTAs")
-    ap.add_argument("--part", choices=["all", "decode", "qwha", "optim", "layers", "stack"], default="all",
-                    help="decode / qwha / optim / layers / stack: only that component (a short run "
-                         "for profiling)")
+    ap.add_argument("--part", choices=["all", "decode", "qwha", "optim", "layers", "stack", "quantize"],
+                    default="all", help="decode / qwha / optim / layers / stack / quantize: only that "
+                                        "component (a short run for profiling)")
+    ap.add_argument("--shape", default=None, help="NxK: the one weight shape of --part quantize")
     ap.add_argument("--skip-extra", action="store_true",
                     help="leave out the int8, 65B-shaped and whole-stack components")
     args = ap.parse_args()
@@ -1077,11 +1140,14 @@ def main():
         if rank == 0:
             print(json.dumps({"part": "decode", "decode_7b_4096x4096_nf4": out}), flush=True)
         return
-    if args.part in ("layers", "stack"):
+    if args.part in ("layers", "stack", "quantize"):
         dev = torch.device("cuda", local_rank)
         torch.cuda.set_device(dev)
-        fn = layers_bench if args.part == "layers" else stack_bench
-        out = fn(dev, load_peaks(), reps=max(1, args.steps))
+        fn = {"layers": layers_bench, "stack": stack_bench, "quantize": quant_bench}[args.part]
+        kw = {}
+        if args.part == "quantize" and args.shape:
+            kw["shapes"] = (tuple(int(v) for v in args.shape.lower().split("x")),)
+        out = fn(dev, load_peaks(), reps=max(1, args.steps), **kw)
         if rank == 0:
             print(json.dumps({"part": args.part, args.part: out}), flush=True)
         return

@@ -123,6 +123,34 @@ ql_status nf4_dq_quantize(const ql_bf16* W, int64_t n, uint8_t* codes, float* ab
                           int8_t* qabsmax, float* group_scale, float* mean, void* ws,
                           size_t ws_bytes, void* stream);
 
+/* One weight of nf4_dq_quantize_batch: the arguments of nf4_dq_quantize (device
+ * pointers; W bf16 [n], codes uint8 [ceil(n/2)], absmax fp32 [ceil(n/64)], qabsmax int8
+ * [ceil(n/64)], group_scale fp32 [ceil(ceil(n/64)/256)], mean fp32 [1]).               */
+typedef struct {
+  const ql_bf16* W;
+  int64_t n;
+  uint8_t* codes;
+  float*   absmax;
+  int8_t*  qabsmax;
+  float*   group_scale;
+  float*   mean;
+} ql_nf4_dq_item;
+
+/* NF4 + double quantisation of `count` weights, each exactly as nf4_dq_quantize would
+ * quantise it (QLoRA page, "1. 4-bit NormalFloat (NF4)" and "2. Double Quantization": one
+ * mean per tensor), for quantising a model's linears together. Weights with whole blocks
+ * and 16-byte aligned W and codes share three launches per 128 weights: one pass over all
+ * their blocks (codes, absmax and each weight's exact DQ sum), the means, and the group
+ * encode; any other weight takes the single-weight path on the stream. Every output is
+ * bit-identical to nf4_dq_quantize of that weight.
+ * items: HOST array of count descriptors (read before the call returns). count = 0 is a
+ * no-op. Each item is checked as nf4_dq_quantize checks its arguments; a bad item returns
+ * an error before anything is launched.
+ * ws: device workspace of ql_workspace_bytes(QL_OP_DQ_BATCH, count, 0, 0, 0) bytes,
+ * 16-byte aligned. */
+ql_status nf4_dq_quantize_batch(const ql_nf4_dq_item* items, int32_t count, void* ws,
+                                size_t ws_bytes, void* stream);
+
 /* NF4 + double quantisation of a weight split across ranks (QLoRA page, "2. Double
  * Quantization": one mean per tensor, so the ranks must agree on the sum of all block
  * constants). Every rank holds a contiguous shard of the flattened weight; every shard
@@ -278,7 +306,8 @@ ql_status qlora_linear_fwd_qwha(const ql_weight* w, const ql_bf16* X, int64_t M,
  * X and Z are 16-byte aligned, K a multiple of 64, the block at most 16384. */
 ql_status ql_wht(const ql_bf16* X, int64_t M, int64_t K, ql_bf16* Z, void* stream);
 
-enum { QL_OP_DQ = 0, QL_OP_FWD = 1, QL_OP_BWD = 2, QL_OP_FWD_LORDBA = 3, QL_OP_FWD_QWHA = 4 };
+enum { QL_OP_DQ = 0, QL_OP_FWD = 1, QL_OP_BWD = 2, QL_OP_FWD_LORDBA = 3, QL_OP_FWD_QWHA = 4,
+       QL_OP_DQ_BATCH = 5 /* M = the number of weights */ };
 
 /* The adapter optimiser step with paged states (QLoRA page, aizip.shop/methodologies/qlora,
  * section "3. Paged Optimizer": optimiser states held in unified memory, paged to host RAM

@@ -20,7 +20,7 @@ HEADER = os.path.join(os.path.dirname(_PKG), "include", "qlora.h")
 QL_OK, QL_ERR_INVALID_ARG, QL_ERR_UNSUPPORTED, QL_ERR_WORKSPACE, QL_ERR_NONFINITE, \
     QL_ERR_TIMEOUT, QL_ERR_CUDA = range(7)
 QL_FMT_NF4_DQ, QL_FMT_INT8_B64 = 0, 1
-QL_OP_DQ, QL_OP_FWD, QL_OP_BWD, QL_OP_FWD_LORDBA, QL_OP_FWD_QWHA = 0, 1, 2, 3, 4
+QL_OP_DQ, QL_OP_FWD, QL_OP_BWD, QL_OP_FWD_LORDBA, QL_OP_FWD_QWHA, QL_OP_DQ_BATCH = 0, 1, 2, 3, 4, 5
 FORMATS = {"nf4_dq": QL_FMT_NF4_DQ, "int8": QL_FMT_INT8_B64}
 
 
@@ -35,6 +35,13 @@ class QLWeight(ctypes.Structure):
                 ("N", ctypes.c_int64), ("K", ctypes.c_int64),
                 ("codes", ctypes.c_void_p), ("absmax", ctypes.c_void_p),
                 ("qabsmax", ctypes.c_void_p), ("group_scale", ctypes.c_void_p),
+                ("mean", ctypes.c_void_p)]
+
+
+class QLNf4DqItem(ctypes.Structure):
+    """ql_nf4_dq_item: one weight of nf4_dq_quantize_batch."""
+    _fields_ = [("W", ctypes.c_void_p), ("n", ctypes.c_int64), ("codes", ctypes.c_void_p),
+                ("absmax", ctypes.c_void_p), ("qabsmax", ctypes.c_void_p), ("group_scale", ctypes.c_void_p),
                 ("mean", ctypes.c_void_p)]
 
 
@@ -72,6 +79,7 @@ _SIGS = {
     "int8_quantize": ([P, I64, P, P, P], I32),
     "dq_quantize": ([P, I64, P, P, P, P, SZ, P], I32),
     "nf4_dq_quantize": ([P, I64, P, P, P, P, P, P, SZ, P], I32),
+    "nf4_dq_quantize_batch": ([P, I32, P, SZ, P], I32),
     "nf4_quantize_shard": ([P, I64, P, P, P, P, SZ, P], I32),
     "qlora_linear_fwd_lordba": ([ctypes.POINTER(QLWeight), P, I64, ctypes.c_void_p, P, P, SZ, P], I32),
     "qlora_linear_fwd_qwha": ([ctypes.POINTER(QLWeight), P, I64, ctypes.c_void_p, P, P, SZ, P], I32),
@@ -267,6 +275,41 @@ def nf4_dq_quantize(W: torch.Tensor, codes=None, absmax=None, qabsmax=None, grou
     _check(lib().nf4_dq_quantize(_ptr(W), n, _ptr(codes), _ptr(absmax), _ptr(qabsmax), _ptr(group_scale),
                                  _ptr(mean), _ptr(ws), ws.numel(), _stream(dev)), "nf4_dq_quantize")
     return codes, absmax, qabsmax, group_scale, mean
+
+
+def nf4_dq_quantize_batch(Ws, outs=None):
+    """NF4 + double quantisation of several weights in one call (three launches per 128
+    weights). Ws: list of bf16 tensors on one device. outs: optional list of (codes,
+    absmax, qabsmax, group_scale, mean) per weight. Returns that list; each entry equals
+    nf4_dq_quantize of its weight bit for bit."""
+    if not Ws:
+        return []
+    dev = Ws[0].device
+    if outs is None:
+        outs = []
+        for W in Ws:
+            n = W.numel()
+            nb = (n + 63) // 64
+            outs.append((torch.empty((n + 1) // 2, dtype=torch.uint8, device=dev),
+                         torch.empty(nb, dtype=torch.float32, device=dev),
+                         torch.empty(nb, dtype=torch.int8, device=dev),
+                         torch.empty((nb + 255) // 256, dtype=torch.float32, device=dev),
+                         torch.empty(1, dtype=torch.float32, device=dev)))
+    if len(outs) != len(Ws):
+        raise ValueError("one output tuple per weight")
+    items = (QLNf4DqItem * len(Ws))()
+    for i, (W, (codes, absmax, qa, gs, mu)) in enumerate(zip(Ws, outs)):
+        _need(W, torch.bfloat16, f"W[{i}]", None, dev)
+        n = W.numel()
+        nb = (n + 63) // 64
+        _need(codes, torch.uint8, f"codes[{i}]", (n + 1) // 2, dev)
+        _need(absmax, torch.float32, f"absmax[{i}]", nb, dev)
+        _need_dq_outputs(nb, qa, gs, mu, dev)
+        items[i] = QLNf4DqItem(_ptr(W), n, _ptr(codes), _ptr(absmax), _ptr(qa), _ptr(gs), _ptr(mu))
+    ws = workspace(workspace_bytes(QL_OP_DQ_BATCH, len(Ws), 0, 0, 0), dev)
+    _check(lib().nf4_dq_quantize_batch(items, len(Ws), _ptr(ws), ws.numel(), _stream(dev)),
+           "nf4_dq_quantize_batch")
+    return outs
 
 
 def nf4_quantize_shard(W: torch.Tensor, codes=None, absmax=None, bins=None):

@@ -383,6 +383,10 @@ extern "C" {
 
 size_t ql_workspace_bytes(int32_t op, int64_t M, int64_t N, int64_t K, int32_t r) {
   if (op == QL_OP_DQ) return 256;
+  if (op == QL_OP_DQ_BATCH) {                         // 16 exact-sum bins per weight of a launch
+    if (M < 0) return 0;
+    return (size_t)imax64(256, imin64(M, 128) * 16 * 8);
+  }
   if (op == QL_OP_FWD_QWHA) {
     if (M < 1 || N < 1 || K < 64 || K % 64 != 0) return 0;
     return (size_t)qwha_ws_bytes(M, N, K);

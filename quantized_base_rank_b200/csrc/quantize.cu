@@ -10,6 +10,9 @@
 // and boundaries) lives in registers and nothing is staged.
 #include <math.h>
 
+#include <algorithm>
+#include <vector>
+
 #include "common.cuh"
 
 namespace qlb {
@@ -701,6 +704,162 @@ dq_encode_kernel(const float* __restrict__ absmax, int64_t nb, const float* __re
 }
 
 // ---------------------------------------------------------------------------------
+// NF4 + double quantisation of a batch of weights (a model's linears at load time) in
+// three launches instead of two per weight: one persistent pass over every block of every
+// weight (NF4 codes, absmax, and each weight's exact DQ sum), one thread per weight for
+// the means, and the group encode over every weight's groups. The arithmetic of each weight
+// is that of nf4_dq_quantize, so the results are the same bit for bit.
+// ---------------------------------------------------------------------------------
+
+constexpr int kBatchMax = 128;      // weights per launch (the table travels as a kernel parameter)
+
+struct BatchItem {
+  const uint16_t* W;
+  int64_t n;
+  uint8_t* codes;
+  float* absmax;
+  int8_t* qabsmax;
+  float* group_scale;
+  float* mean;
+};
+
+struct BatchArgs {
+  BatchItem item[kBatchMax];
+  int64_t blk_start[kBatchMax + 1];   // prefix sums of the weights' blocks
+  int64_t grp_start[kBatchMax + 1];   // prefix sums of their DQ groups
+  int count;
+  unsigned long long* bins;           // [count][16] exact sums, zeroed before the pass
+  int* flag;
+};
+
+// Weight of flattened block (or group) x, starting the search at w (prefix sums ascending).
+__device__ __forceinline__ int batch_find(const int64_t* start, int count, int64_t x, int w) {
+  while (w + 1 < count && x >= start[w + 1]) ++w;
+  return w;
+}
+
+// Adds the lanes' running sums, keyed by (weight, bin), into the global bins: one pass per
+// distinct key, a three-part warp reduction (as bins_warp_add), one atomic per key.
+__device__ __forceinline__ void batch_bins_flush(unsigned long long* gbins, uint32_t key, unsigned long long c) {
+  uint32_t pending = __ballot_sync(0xFFFFFFFFu, c != 0ull);
+  while (pending) {
+    const int leader = __ffs(pending) - 1;
+    const uint32_t lk = __shfl_sync(0xFFFFFFFFu, key, leader);
+    const bool mine = c != 0ull && key == lk;
+    constexpr unsigned long long kPart = (1ull << 27) - 1ull;
+    const uint32_t p0 = __reduce_add_sync(0xFFFFFFFFu, mine ? (uint32_t)(c & kPart) : 0u);
+    const uint32_t p1 = __reduce_add_sync(0xFFFFFFFFu, mine ? (uint32_t)((c >> 27) & kPart) : 0u);
+    const uint32_t p2 = __reduce_add_sync(0xFFFFFFFFu, mine ? (uint32_t)(c >> 54) : 0u);
+    if ((threadIdx.x & 31) == 0)
+      atomicAdd(gbins + lk, (unsigned long long)p0 + ((unsigned long long)p1 << 27) + ((unsigned long long)p2 << 54));
+    pending &= ~__ballot_sync(0xFFFFFFFFu, mine);
+  }
+}
+
+// Every weight of the batch holds whole blocks, with 16-byte aligned source and codes. Each
+// CTA takes a contiguous range of the flattened blocks, so it touches one or two weights;
+// its lanes take consecutive blocks and load their next block while they encode.
+__global__ void __launch_bounds__(kNf4Threads, 2)
+nf4_batch_kernel(const __grid_constant__ BatchArgs args, const Nf4Tables tab, const Nf4BoundTable btab) {
+  __shared__ __align__(16) uint32_t s_tab[128 * 8];
+  for (int i = threadIdx.x; i < 128 * 8 / 4; i += blockDim.x)
+    reinterpret_cast<uint4*>(s_tab)[i] = reinterpret_cast<const uint4*>(&btab.c[0][0])[i];
+  __syncthreads();
+  const int64_t total = args.blk_start[args.count];
+  const int64_t per = (total + gridDim.x - 1) / gridDim.x;
+  const int64_t c0 = imin64(total, per * blockIdx.x), c1 = imin64(total, c0 + per);
+  bool bad = false;
+  uint32_t lkey = 0;                                  // this lane's running (weight, bin) and sum
+  unsigned long long lsum = 0ull;
+  int w = batch_find(args.blk_start, args.count, c0, 0);
+  int64_t it = c0 + threadIdx.x;
+  uint4 nx[8];
+  if (it < c1) {
+    w = batch_find(args.blk_start, args.count, it, w);
+    const uint4* src = reinterpret_cast<const uint4*>(args.item[w].W + (it - args.blk_start[w]) * kBlock);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) nx[i] = __ldg(src + i);
+  }
+  for (int64_t w0 = c0 + (threadIdx.x & ~31); w0 < c1; w0 += kNf4Threads, it += kNf4Threads) {
+    const bool live = it < c1;
+    uint32_t v[32];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[4 * i] = nx[i].x; v[4 * i + 1] = nx[i].y; v[4 * i + 2] = nx[i].z; v[4 * i + 3] = nx[i].w;
+    }
+    const int wc = w;                                 // this block's weight
+    const int64_t b = it - args.blk_start[wc];
+    if (it + kNf4Threads < c1) {                      // the next block, possibly of the next weight
+      w = batch_find(args.blk_start, args.count, it + kNf4Threads, w);
+      const uint4* src =
+          reinterpret_cast<const uint4*>(args.item[w].W + (it + kNf4Threads - args.blk_start[w]) * kBlock);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) nx[i] = __ldg(src + i);
+    }
+    uint32_t m = 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(m), "r"(v[i]));
+    m &= 0x7FFF7FFFu;
+    const uint32_t amax = max(m & 0xFFFFu, m >> 16);
+    uint32_t bin = 0;
+    unsigned long long c = 0ull;
+    if (live) {
+      if (amax >= 0x7F80u) raise_flag(args.flag, kFlagNonfinite);
+      args.item[wc].absmax[b] = __uint_as_float(amax << 16);
+      dq_term(amax << 16, bin, c, bad);
+    }
+    const uint32_t key = (uint32_t)wc * kSumBins + bin;
+    const bool move = c != 0ull && key != lkey && lsum != 0ull;
+    if (__any_sync(0xFFFFFFFFu, move)) {
+      batch_bins_flush(args.bins, lkey, move ? lsum : 0ull);
+      if (move) lsum = 0ull;
+    }
+    if (c != 0ull) {
+      lkey = key;
+      lsum += c;
+    }
+    uint32_t Cp[7];
+    nf4_boundaries(amax, s_tab, tab, Cp);
+    uint32_t out[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      out[q] = nf4_pack8(nf4_code_pair(v[4 * q + 0], Cp), nf4_code_pair(v[4 * q + 1], Cp),
+                         nf4_code_pair(v[4 * q + 2], Cp), nf4_code_pair(v[4 * q + 3], Cp));
+    if (live) {
+      uint8_t* dst = args.item[wc].codes + b * 32;
+      *reinterpret_cast<uint4*>(dst) = make_uint4(out[0], out[1], out[2], out[3]);
+      *reinterpret_cast<uint4*>(dst + 16) = make_uint4(out[4], out[5], out[6], out[7]);
+    }
+  }
+  (void)bad;                                          // a non-finite absmax already raised the flag
+  batch_bins_flush(args.bins, lkey, lsum);
+}
+
+// One thread per weight: the mean from its exact bins.
+__global__ void nf4_batch_mean_kernel(const __grid_constant__ BatchArgs args) {
+  const int w = blockIdx.x * blockDim.x + threadIdx.x;
+  if (w >= args.count) return;
+  unsigned long long v[kSumBins];
+#pragma unroll
+  for (int i = 0; i < kSumBins; ++i) v[i] = args.bins[w * kSumBins + i];
+  *args.item[w].mean = dq_mean_from_bins(v, args.blk_start[w + 1] - args.blk_start[w]);
+}
+
+// One warp per DQ group, over every weight's groups.
+__global__ void __launch_bounds__(256) nf4_batch_dq_kernel(const __grid_constant__ BatchArgs args) {
+  const int lane = threadIdx.x & 31;
+  const int64_t total = args.grp_start[args.count];
+  const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  int w = 0;
+  for (int64_t gg = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; gg < total; gg += warps) {
+    w = batch_find(args.grp_start, args.count, gg, w);
+    const BatchItem& it = args.item[w];
+    dq_encode_group<false>(it.absmax, args.blk_start[w + 1] - args.blk_start[w], *it.mean, it.qabsmax,
+                           it.group_scale, gg - args.grp_start[w], lane);
+  }
+}
+
+// ---------------------------------------------------------------------------------
 // Standalone dequantisation (checks only; the linear kernels decode on the fly).
 // ---------------------------------------------------------------------------------
 
@@ -940,6 +1099,68 @@ ql_status nf4_dq_quantize(const ql_bf16* W, int64_t n, uint8_t* codes, float* ab
   }
   ProfScope prof(PK_DQ, st, 1);
   return launch_dq_encode(absmax, nb, mean, qabsmax, group_scale, st);
+}
+
+ql_status nf4_dq_quantize_batch(const ql_nf4_dq_item* items, int32_t count, void* ws, size_t ws_bytes,
+                                void* stream) {
+  if (count < 0 || (count > 0 && (!items || !ws))) return QL_ERR_INVALID_ARG;
+  if (count == 0) return QL_OK;
+  if (!aligned(ws, 16)) return QL_ERR_INVALID_ARG;
+  if (ws_bytes < ql_workspace_bytes(QL_OP_DQ_BATCH, count, 0, 0, 0)) return QL_ERR_WORKSPACE;
+  for (int32_t i = 0; i < count; ++i) {
+    const ql_nf4_dq_item& t = items[i];
+    if (t.n < 1 || !t.W || !t.codes || !t.absmax || !t.qabsmax || !t.group_scale || !t.mean)
+      return QL_ERR_INVALID_ARG;
+    if ((t.n + kBlock - 1) / kBlock > (int64_t(1) << 24)) return QL_ERR_UNSUPPORTED;
+    if (!aligned(t.W, 2) || !aligned(t.codes, 4) || !aligned(t.absmax, 4) || !aligned(t.group_scale, 4) ||
+        !aligned(t.mean, 4))
+      return QL_ERR_INVALID_ARG;
+  }
+  cudaStream_t st = as_stream(stream);
+  unsigned long long* bins = static_cast<unsigned long long*>(ws);
+  // items the batch kernel does not take (a ragged last block, unaligned source or codes)
+  // go through the single-weight path, one after another on the stream
+  std::vector<int32_t> batch;
+  for (int32_t i = 0; i < count; ++i) {
+    const ql_nf4_dq_item& t = items[i];
+    if (t.n % kBlock == 0 && aligned(t.W, 16) && aligned(t.codes, 16)) {
+      batch.push_back(i);
+    } else {
+      const ql_status e = nf4_dq_quantize(t.W, t.n, t.codes, t.absmax, t.qabsmax, t.group_scale, t.mean, ws,
+                                          ql_workspace_bytes(QL_OP_DQ, 0, 0, 0, 0), stream);
+      if (e != QL_OK) return e;
+    }
+  }
+  static const int per_sm = resident_ctas(nf4_batch_kernel, kNf4Threads);
+  const Nf4Tables& tab = nf4_tables();
+  const Nf4BoundTable& btab = nf4_bound_table();
+  for (size_t s0 = 0; s0 < batch.size(); s0 += kBatchMax) {
+    const int cnt = (int)std::min(batch.size() - s0, (size_t)kBatchMax);
+    BatchArgs a{};
+    a.count = cnt;
+    a.bins = bins;
+    a.flag = device_flag_ptr();
+    a.blk_start[0] = a.grp_start[0] = 0;
+    for (int j = 0; j < cnt; ++j) {
+      const ql_nf4_dq_item& t = items[batch[s0 + j]];
+      a.item[j] = BatchItem{t.W, t.n, t.codes, t.absmax, t.qabsmax, t.group_scale, t.mean};
+      const int64_t nb = t.n / kBlock;
+      a.blk_start[j + 1] = a.blk_start[j] + nb;
+      a.grp_start[j + 1] = a.grp_start[j] + (nb + kGroup - 1) / kGroup;
+    }
+    ProfScope prof(PK_NF4, st, 3);
+    if (cudaMemsetAsync(bins, 0, (size_t)cnt * kSumBins * sizeof(unsigned long long), st) != cudaSuccess)
+      return QL_ERR_CUDA;
+    const int64_t total = a.blk_start[cnt];
+    const int grid = (int)imax64(1, imin64((total + kNf4Threads - 1) / kNf4Threads, (int64_t)num_sms() * per_sm));
+    nf4_batch_kernel<<<grid, kNf4Threads, 0, st>>>(a, tab, btab);
+    QL_CHECK_LAUNCH();
+    nf4_batch_mean_kernel<<<(cnt + 31) / 32, 32, 0, st>>>(a);
+    QL_CHECK_LAUNCH();
+    nf4_batch_dq_kernel<<<grid_for(a.grp_start[cnt] * 32, 256), 256, 0, st>>>(a);
+    QL_CHECK_LAUNCH();
+  }
+  return QL_OK;
 }
 
 ql_status nf4_quantize_shard(const ql_bf16* W, int64_t n, uint8_t* codes, float* absmax, uint64_t* bins,

@@ -118,6 +118,19 @@ def test_argument_validation_without_a_device(lib):
     big = B.QLWeight(1, 0, 1 << 21, 1 << 21, 16, 16, 16, 16, 16)
     assert lib.ql_dequantize(ctypes.byref(big), 16, None) == B.QL_ERR_UNSUPPORTED
     assert lib.ql_launch_count() == c0
+    # batched NF4 + DQ: nothing to do, a null table, a bad item, a short workspace
+    assert lib.nf4_dq_quantize_batch(None, 0, None, 0, None) == B.QL_OK
+    assert lib.nf4_dq_quantize_batch(None, 2, 16, 1 << 20, None) == B.QL_ERR_INVALID_ARG
+    items = (B.QLNf4DqItem * 2)(B.QLNf4DqItem(16, 64, 16, 16, 16, 16, 16),
+                                B.QLNf4DqItem(16, 64, 16, None, 16, 16, 16))
+    c0 = lib.ql_launch_count()
+    assert lib.nf4_dq_quantize_batch(items, 2, 16, 1 << 20, None) == B.QL_ERR_INVALID_ARG
+    items[1] = B.QLNf4DqItem(16, 64 * (1 << 24) + 64, 16, 16, 16, 16, 16)
+    assert lib.nf4_dq_quantize_batch(items, 2, 16, 1 << 20, None) == B.QL_ERR_UNSUPPORTED
+    assert lib.nf4_dq_quantize_batch(items, 2, 16, 8, None) == B.QL_ERR_WORKSPACE
+    assert lib.ql_launch_count() == c0
+    assert B.workspace_bytes(B.QL_OP_DQ_BATCH, 224, 0, 0, 0) == 128 * 16 * 8
+    assert B.workspace_bytes(B.QL_OP_DQ_BATCH, 1, 0, 0, 0) == 256
     # misaligned or null pointers, bad shapes: all rejected synchronously
     assert lib.qlora_linear_fwd(ctypes.byref(w), None, 1, None, None, 8, 16.0, None, None,
                                 None, 0, None) == B.QL_ERR_INVALID_ARG

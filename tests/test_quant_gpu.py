@@ -239,3 +239,33 @@ def test_sharded_nf4_dq_matches_whole(shards, name, W):
         assert torch.equal(g.view(torch.int32), gs[a // 16384: a // 16384 + g.numel()].view(torch.int32))
         assert torch.equal(m.view(torch.int32), mu.view(torch.int32))
     assert B.device_status() == B.QL_OK
+
+
+def test_nf4_dq_batch_matches_single_weight_calls():
+    """The batched entry equals nf4_dq_quantize of each weight bit for bit: every output
+    (codes, absmax, DQ codes, group scales, mean). The mix spans the batch kernel (whole
+    blocks, aligned), the single-weight path inside the batch (a ragged block count, an
+    unaligned source), weights of one to thousands of groups, the outlier weight, the
+    special values, and more than 128 weights so that the batch runs in two launches."""
+    specials = dict(_weights())
+    Ws = [specials["cfg1-256x256"], specials["cfg2-4096x4096-outliers"], specials["special-values"],
+          specials["ragged-odd"], synth.normal_bf16((11008 * 64,), 0.02, 21, 0)]
+    Ws += [synth.normal_bf16((64 * (1 + (i * 37) % 300),), 0.01 * (1 + i % 5), 30 + i, 0) for i in range(127)]
+    dev_Ws = [W.cuda().contiguous().view(-1) for W in Ws]
+    base = torch.empty(64 * 500 + 1, dtype=torch.bfloat16, device="cuda")
+    base[1:].copy_(synth.normal_bf16((64 * 500,), 0.02, 99, 0).cuda())
+    dev_Ws.append(base[1:])                                  # 2-byte aligned only
+    got = B.nf4_dq_quantize_batch(dev_Ws)
+    torch.cuda.synchronize()
+    assert B.device_status() == B.QL_OK
+    for i, (W, g) in enumerate(zip(dev_Ws, got)):
+        ref = B.nf4_dq_quantize(W)
+        for name, a, b in zip(("codes", "absmax", "qabsmax", "group_scale", "mean"), g, ref):
+            assert torch.equal(a.view(torch.uint8) if a.dtype != torch.uint8 else a,
+                               b.view(torch.uint8) if b.dtype != torch.uint8 else b), (i, name)
+    # and two of them against the oracle
+    for i in (0, 1):
+        w = Ws[i].float().numpy().ravel()
+        ref = o.quantize_weight(w, "nf4_dq")
+        assert np.array_equal(got[i][0].cpu().numpy(), ref["codes"])
+        assert np.array_equal(got[i][2].cpu().numpy(), ref["qabsmax"])
