@@ -60,6 +60,10 @@ int64_t ext_fwd_ws_bytes(int64_t M, int64_t N, int64_t K, int64_t kext);
 ql_status ext_forward(const ql_weight* w, const uint16_t* X, int64_t M, const uint16_t* Zext,
                       const uint16_t* Wext, int64_t kext, uint16_t* Y, void* ws, size_t ws_bytes,
                       cudaStream_t st, const QwhaRows* qw = nullptr);
+// Y = X bf16(deq(W) + dW)^T, dW a dense bf16 [N, K] update added to the decoded weight in
+// the fused GEMM (M > 16); scratch of ext_fwd_ws_bytes(M, N, K, 0), 256-aligned (linear.cu)
+ql_status dw_forward(const ql_weight* w, const uint16_t* X, int64_t M, const uint16_t* dW, uint16_t* Y, void* ws,
+                     size_t ws_bytes, cudaStream_t st);
 int64_t qwha_ws_bytes(int64_t M, int64_t N, int64_t K);             // qwha.cu
 int* device_flag_ptr();                 // device address of the sticky flag (current device)
 int num_sms();                          // SM count of the current device

@@ -373,7 +373,9 @@ qgemm_tma_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
 // 64-element block; they also issue the TMA of the extension's weight-side factor, so
 // every ring has a single producer).
 // =================================================================================
-template <BSrc BS>
+// DW: a ring of SW stages for the dense update's chunks, paid for with one token stage and
+// fewer code stages.
+template <BSrc BS, bool DW = false>
 struct WdecCfg {
   static constexpr int BM = 128;                                 // weight rows per tile
   static constexpr int BN = 256;                                 // tokens per tile
@@ -382,10 +384,13 @@ struct WdecCfg {
   static constexpr int kTBytes = BN * 128;                       // token stage
   static constexpr int kCodeBytes = BM * (BS == BSrc::NF4 ? 32 : 64);
   static constexpr int kCBytes = kCodeBytes + 1024;              // codes + scales
-  static constexpr int SD = 4, ST = 4, SC = (BS == BSrc::NF4 ? 6 : 3);
+  static constexpr int SD = 4, ST = DW ? 3 : 4;
+  static constexpr int SC = DW ? (BS == BSrc::NF4 ? 3 : 2) : (BS == BSrc::NF4 ? 6 : 3);
+  static constexpr int SW = DW ? (BS == BSrc::NF4 ? 3 : 2) : 0;  // update stages (kDBytes each)
   static constexpr int kTmemCols = 512;
   static constexpr int kThreads = (7 + NP) * 32;
-  static constexpr size_t kSmem = (size_t)SD * kDBytes + (size_t)ST * kTBytes + (size_t)SC * kCBytes + 2048;
+  static constexpr size_t kSmem =
+      (size_t)SD * kDBytes + (size_t)ST * kTBytes + (size_t)SC * kCBytes + (size_t)SW * kDBytes + 2048;
 };
 
 // EPI_BF16 stored transposed: element (weight row w, token t) -> out[t * ld_out + w]
@@ -398,20 +403,35 @@ __device__ __forceinline__ void epilogue_store_t(const GemmArgs& a, int64_t wrow
     if (t0 + j < a.Cn) out[(t0 + j) * a.ld_out] = (uint16_t)float_to_bf16_bits(__uint_as_float(v[j]));
 }
 
-// W_MN = false: forward; true: dX (weight used transposed)
-template <BSrc BS, bool W_MN>
-__global__ void __launch_bounds__(WdecCfg<BS>::kThreads, 1)
+// bf16x2 sum with one rounding to nearest even per half.
+__device__ __forceinline__ uint32_t add_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// W_MN = false: forward; true: dX (weight used transposed). DW (forward only, no extension
+// chunks): a dense bf16 update dW [R, Kc] (tmDW, box 64 x 128 with the 128-byte swizzle, the
+// decoded stage's own layout) is added to the decoded weight before the MMA, bf16(W' + dW)
+// with one rounding: the codes' producer also loads each chunk of dW into a ring of its own,
+// and the decode warps add it to their decoded values before storing them.
+template <BSrc BS, bool W_MN, bool DW = false>
+__global__ void __launch_bounds__(WdecCfg<BS, DW>::kThreads, 1)
 qgemm_wdec_kernel(const __grid_constant__ CUtensorMap tmT, const __grid_constant__ CUtensorMap tmCodes,
                   const __grid_constant__ CUtensorMap tmScale, const __grid_constant__ CUtensorMap tmTe,
-                  const __grid_constant__ CUtensorMap tmWe, const GemmArgs args) {
-  using Cfg = WdecCfg<BS>;
+                  const __grid_constant__ CUtensorMap tmWe, const __grid_constant__ CUtensorMap tmDW,
+                  const GemmArgs args) {
+  static_assert(!(DW && W_MN), "the dense update is a forward-only operand");
+  using Cfg = WdecCfg<BS, DW>;
   constexpr int BM = Cfg::BM, BN = Cfg::BN, NP = Cfg::NP, SD = Cfg::SD, ST = Cfg::ST, SC = Cfg::SC;
+  constexpr int SW = Cfg::SW;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sD = smem;                                   // decoded weight (A operand)
   uint8_t* sT = sD + SD * Cfg::kDBytes;                 // tokens (B operand)
   uint8_t* sC = sT + ST * Cfg::kTBytes;                 // codes + scales
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sC + SC * Cfg::kCBytes);
+  uint8_t* sW = sC + SC * Cfg::kCBytes;                 // DW: the update's chunks
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sW + SW * Cfg::kDBytes);
   const uint32_t full_d = smem_u32(bars);
   const uint32_t empty_d = full_d + 8 * SD;
   const uint32_t full_t = empty_d + 8 * SD;
@@ -421,7 +441,9 @@ qgemm_wdec_kernel(const __grid_constant__ CUtensorMap tmT, const __grid_constant
   const uint32_t acc_full = empty_c + 8 * SC;
   const uint32_t acc_empty = acc_full + 16;
   const uint32_t drain = acc_full + 32;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * (SD + ST + SC) + 5);
+  const uint32_t dw_full = drain + 8;                  // DW: the update's chunk has landed
+  const uint32_t dw_empty = dw_full + 8 * SW;          // DW: the decode warps have read it
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * (SD + ST + SC) + 5 + 2 * SW);
   volatile int* abort_word = reinterpret_cast<volatile int*>(tmem_holder + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -431,6 +453,7 @@ qgemm_wdec_kernel(const __grid_constant__ CUtensorMap tmT, const __grid_constant
     for (int s = 0; s < SC; ++s) { mbar_init(full_c + 8 * s, 1); mbar_init(empty_c + 8 * s, NP); }
     for (int i = 0; i < 2; ++i) { mbar_init(acc_full + 8 * i, 1); mbar_init(acc_empty + 8 * i, 4); }
     mbar_init(drain, 1);
+    for (int s = 0; s < SW; ++s) { mbar_init(dw_full + 8 * s, 1); mbar_init(dw_empty + 8 * s, NP); }
     *abort_word = 0;
     fence_mbar_init();
   }
@@ -438,7 +461,11 @@ qgemm_wdec_kernel(const __grid_constant__ CUtensorMap tmT, const __grid_constant
     tma_prefetch_desc(&tmT);
     if (args.n_ext) tma_prefetch_desc(&tmTe);
   }
-  if (warp == 6 && lane == 0) { tma_prefetch_desc(&tmCodes); tma_prefetch_desc(&tmScale); }
+  if (warp == 6 && lane == 0) {
+    tma_prefetch_desc(&tmCodes);
+    tma_prefetch_desc(&tmScale);
+    if (DW) tma_prefetch_desc(&tmDW);
+  }
   if (warp == 7 && lane == 0 && args.n_ext) tma_prefetch_desc(&tmWe);
   if (warp == 5) tmem_alloc(smem_u32(tmem_holder), Cfg::kTmemCols);
   tc_fence_before();
@@ -513,10 +540,24 @@ qgemm_wdec_kernel(const __grid_constant__ CUtensorMap tmT, const __grid_constant
           tma_load_2d(dst, &tmCodes, fb, BS == BSrc::NF4 ? w0 / 2 : w0, kc * 64);
           tma_load_2d(dst + Cfg::kCodeBytes, &tmScale, fb, (w0 / 64) & ~3, kc * 64);
         }
+        if (DW) {
+          // the update's rows w0..w0+128, columns kc*64..+64, into its own ring (the chunk
+          // sequence, there being no extension chunks)
+          const uint32_t sw = gc % SW, pw = (gc / SW) & 1;
+          if (!mbar_wait(dw_empty + 8 * sw, pw ^ 1, lim, abort_word)) { ok = false; ++gc; break; }
+          mbar_arrive_expect_tx(dw_full + 8 * sw, Cfg::kDBytes);
+          tma_load_2d(smem_u32(sW + sw * Cfg::kDBytes), &tmDW, dw_full + 8 * sw, kc * 64, w0);
+        }
       }
     }
-    if (!ok || *abort_word)
+    if (!ok || *abort_word) {
       for (uint32_t j = (gc > (uint32_t)SC ? gc - SC : 0); j < gc; ++j) drain_wait(full_c + 8 * (j % SC), (j / SC) & 1);
+      if (DW) {
+        // the update chunks issued: all but the last when a wait for the stage gave up
+        const uint32_t gdw = ok ? gc : gc - 1;
+        for (uint32_t j = (gdw > (uint32_t)SW ? gdw - SW : 0); j < gdw; ++j) drain_wait(dw_full + 8 * (j % SW), (j / SW) & 1);
+      }
+    }
   } else if (warp == 5 && lane == 0) {
     // ---- MMA issuer ----
     constexpr uint32_t kIdMain = idesc_bf16_f32(128, BN, W_MN ? 1 : 0, 0);
@@ -597,28 +638,39 @@ qgemm_wdec_kernel(const __grid_constant__ CUtensorMap tmT, const __grid_constant
         }
         const uint32_t sc = gc % SC, pc = (gc / SC) & 1;
         const bool w1 = mbar_wait(full_c + 8 * sc, pc, lim, abort_word);
-        const bool w2 = w1 && mbar_wait(empty_d + 8 * sd, pd ^ 1, lim, abort_word);
+        // DW: the update's chunk gc has landed in its ring
+        const uint32_t sw = DW ? gc % SW : 0, pw = DW ? (gc / SW) & 1 : 0;
+        const bool w3 = w1 && (!DW || mbar_wait(dw_full + 8 * sw, pw, lim, abort_word));
+        const bool w2 = w3 && mbar_wait(empty_d + 8 * sd, pd ^ 1, lim, abort_word);
         if (!__all_sync(0xFFFFFFFFu, w2)) { ok = false; break; }
         const uint8_t* cst = sC + sc * Cfg::kCBytes;
         const float sv = reinterpret_cast<const float*>(cst + Cfg::kCodeBytes)[scale_idx];
         uint4* d = reinterpret_cast<uint4*>(sD + sd * Cfg::kDBytes + d_off);
+        const uint4* u = reinterpret_cast<const uint4*>(sW + sw * Cfg::kDBytes + d_off);
+        auto put = [&](int i, uint4 v) {
+          if (DW) {
+            const uint4 x = u[i];
+            v = make_uint4(add_bf16x2(v.x, x.x), add_bf16x2(v.y, x.y), add_bf16x2(v.z, x.z), add_bf16x2(v.w, x.w));
+          }
+          d[i] = v;
+        };
         if constexpr (BS == BSrc::NF4) {
           const uint4 cv = reinterpret_cast<const uint4*>(cst + code_off)[half];
           uint32_t L[2], H[2];
           nf4_table(q, sv, L, H);
           const int c0i = 4 * half;
-          d[(c0i + 0) ^ key] = nf4_decode8(cv.x, L, H);
-          d[(c0i + 1) ^ key] = nf4_decode8(cv.y, L, H);
-          d[(c0i + 2) ^ key] = nf4_decode8(cv.z, L, H);
-          d[(c0i + 3) ^ key] = nf4_decode8(cv.w, L, H);
+          put((c0i + 0) ^ key, nf4_decode8(cv.x, L, H));
+          put((c0i + 1) ^ key, nf4_decode8(cv.y, L, H));
+          put((c0i + 2) ^ key, nf4_decode8(cv.z, L, H));
+          put((c0i + 3) ^ key, nf4_decode8(cv.w, L, H));
         } else {
           const uint4* src = reinterpret_cast<const uint4*>(cst + code_off) + 2 * half;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const uint4 w = src[h];
             const int c = 4 * half + 2 * h;
-            d[c ^ key] = int8_decode8(w.x, w.y, sv);
-            d[(c + 1) ^ key] = int8_decode8(w.z, w.w, sv);
+            put(c ^ key, int8_decode8(w.x, w.y, sv));
+            put((c + 1) ^ key, int8_decode8(w.z, w.w, sv));
           }
         }
         fence_proxy_async_smem();
@@ -626,6 +678,7 @@ qgemm_wdec_kernel(const __grid_constant__ CUtensorMap tmT, const __grid_constant
         if (lane == 0) {
           mbar_arrive(full_d + 8 * sd);
           mbar_arrive(empty_c + 8 * sc);
+          if (DW) mbar_arrive(dw_empty + 8 * sw);
         }
         ++gc;
       }

@@ -109,18 +109,20 @@ static ql_status launch_wpair(const CUtensorMap& tok, const CUtensorMap& codes, 
   return QL_OK;
 }
 
-template <BSrc BS, bool W_MN>
+// dw: the dense update added to the decoded weight (forward, no extension chunks), or null
+template <BSrc BS, bool W_MN, bool DW = false>
 static ql_status launch_wdec(const CUtensorMap& tok, const CUtensorMap& codes, const CUtensorMap& scale,
                              const CUtensorMap& tok_ext, const CUtensorMap& w_ext, const GemmArgs& args,
-                             cudaStream_t st) {
-  auto kern = qgemm_wdec_kernel<BS, W_MN>;
-  const size_t smem = WdecCfg<BS>::kSmem;
+                             cudaStream_t st, const CUtensorMap* dw = nullptr) {
+  auto kern = qgemm_wdec_kernel<BS, W_MN, DW>;
+  if (DW && (!dw || args.n_ext != 0)) return QL_ERR_INVALID_ARG;
+  const size_t smem = WdecCfg<BS, DW>::kSmem;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return QL_ERR_CUDA;
   const int64_t tiles = ((args.R + 127) / 128) * ((args.Cn + 255) / 256);
   const int grid = (int)imin64(tiles, num_sms());
   if (grid <= 0) return QL_OK;
-  kern<<<grid, WdecCfg<BS>::kThreads, smem, st>>>(tok, codes, scale, tok_ext, w_ext, args);
+  kern<<<grid, WdecCfg<BS, DW>::kThreads, smem, st>>>(tok, codes, scale, tok_ext, w_ext, dw ? *dw : tok, args);
   QL_CHECK_LAUNCH();
   return QL_OK;
 }
@@ -373,6 +375,36 @@ ql_status ext_forward(const ql_weight* w, const uint16_t* X, int64_t M, const ui
   }
   if (w->fmt == QL_FMT_NF4_DQ) return launch_wdec<BSrc::NF4, false>(mXt, mc, ms, mZt, mWe, y, st);
   return launch_wdec<BSrc::INT8, false>(mXt, mc, ms, mZt, mWe, y, st);
+}
+
+// Y = X bf16(deq(W) + dW)^T with a dense bf16 update dW [N, K] (row-major, 16-byte
+// aligned) added to the decoded weight inside the fused GEMM (M > 16 only; the scratch is
+// the block-scale copy of ext_fwd_ws_bytes(M, N, K, 0)).
+ql_status dw_forward(const ql_weight* w, const uint16_t* X, int64_t M, const uint16_t* dW, uint16_t* Y, void* ws,
+                     size_t ws_bytes, cudaStream_t st) {
+  ql_status e = check_weight(w);
+  if (e != QL_OK) return e;
+  if (!X || !Y || !dW || M < 1 || !aligned(X, 16) || !aligned(Y, 16) || !aligned(dW, 16)) return QL_ERR_INVALID_ARG;
+  if (M > (int64_t(1) << 31)) return QL_ERR_UNSUPPORTED;
+  const int64_t N = w->N, K = w->K;
+  if (!ws || !aligned(ws, 256)) return QL_ERR_INVALID_ARG;
+  if ((int64_t)ws_bytes < ext_fwd_ws_bytes(M, N, K, 0)) return QL_ERR_WORKSPACE;
+  float* scales = static_cast<float*>(ws);
+  CUtensorMap mXt, mc, ms, mdw;
+  if (!make_map(&mXt, X, K, M, K, 256) || !make_weight_maps(w, scales, false, &mc, &ms) ||
+      !make_map(&mdw, dW, K, N, K, 128))
+    return QL_ERR_CUDA;
+  {
+    ProfScope prof(PK_FWD_PREP, st, 1);
+    e = launch_block_scales(w, false, scales, st);
+    if (e != QL_OK) return e;
+  }
+  GemmArgs y = base_args();
+  y.R = N; y.Cn = M; y.Kc = K; y.n_ext = 0; y.r = 0;
+  y.out = Y; y.ld_out = N; y.scale = 1.0f;
+  ProfScope prof(PK_FWD_MAIN, st, 1);
+  if (w->fmt == QL_FMT_NF4_DQ) return launch_wdec<BSrc::NF4, false, true>(mXt, mc, ms, mXt, mXt, y, st, &mdw);
+  return launch_wdec<BSrc::INT8, false, true>(mXt, mc, ms, mXt, mXt, y, st, &mdw);
 }
 
 }  // namespace qlb

@@ -13,11 +13,13 @@
 //    slab is one 32-byte sector); the decode-shaped base kernel gathers it by column index
 //    for its rows (sum_j c_j Z[m, col_j]) and adds the sums before the cluster reduction,
 //    so they reach Y with its one bf16 rounding (small_m.cu, qwha_rows_add).
-//  * Larger M: Z row-major; qwha_densify_kernel writes F as a dense bf16 [N, K] and the
-//    fused tcgen05 GEMM takes Z F^T as K/64 extension chunks, beside X W'^T. The gather
-//    has no tensor-core form (F's positions are arbitrary), and on the FMA pipes it needs
-//    a shared-memory read per multiply-add; the extension chunks are faster at the
-//    budgets of a rank-64 LoRA.
+//  * Larger M: Z F^T = X (F H)^T since H is symmetric. qwha_update_kernel forms dW = F H
+//    [N, K] bf16 straight from the compressed rows (blocks up to 4096 wide; wider blocks:
+//    qwha_densify_kernel writes the dense F and the row transform follows), and the fused
+//    tcgen05 GEMM adds dW to the decoded weight in shared memory before the MMA, so the
+//    adapter costs one bf16 add per weight element instead of a second contraction of K.
+//    The gather has no tensor-core form (F's positions are arbitrary), and on the FMA
+//    pipes it needs a shared-memory read per multiply-add.
 #include <cmath>
 
 #include "common.cuh"
@@ -242,6 +244,206 @@ qwha_densify_kernel(const int32_t* __restrict__ row_ptr, const uint16_t* __restr
   if (bad) raise_flag(flag, kFlagBadIndex);
 }
 
+// The update dW = F H (QWHA page, section 2.1: Delta W = F H^{-1}, H symmetric and
+// orthogonal) straight from the compressed rows of F, for transform blocks of b = 64 << LB
+// columns (b <= 4096), on the tensor cores. Each warp takes one (row n, super-tile st) item:
+// the 4096 columns [4096 st, 4096 st + 4096) of row n as a 64 x 64 tile R[a][j] (column
+// 4096 st + 64 a + j), which holds 64 >> LB whole blocks of 2^LB tile rows. In Sylvester
+// order H_b = H_{2^LB} (x) H_64, so the tile's transform is Q = G R H_64 with G = I (x) H_{2^LB}
+// (64 x 64, entries 0 and +-1) and H_64 the 64-point matrix: two 64 x 64 x 64 products by
+// mma.sync (m16n8k16, bf16 in, fp32 out). R holds F's bf16 values and G, H_64 are exact in
+// bf16, so P = G R is exact up to fp32 summation; P enters the second product as
+// bf16 hi + lo (hi = bf16(P), lo = bf16(P - hi)), a relative error near 2^-16. Q is scaled
+// by 1 / sqrt(b), rounded to bf16 and stored. The scatter writes F's values into a zeroed
+// bf16 tile and writes zeros back to the same places afterwards. The same index checks as
+// the densified form; a repeated column keeps one of its values, as there.
+constexpr int kUpdPitch = 72;            // bf16 per tile row (144 bytes): conflict-free ldmatrix rows
+constexpr int kUpdWarps = 6;
+constexpr int kUpdWarpBytes = (64 + 16) * kUpdPitch * 2;   // the tile, then 16 output rows
+
+__device__ __forceinline__ void upd_mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// +-1 (or 0) as bf16 bits
+__device__ __forceinline__ uint32_t pm1_bf16(bool nonzero, int parity) {
+  return nonzero ? (parity & 1 ? 0xBF80u : 0x3F80u) : 0u;
+}
+
+template <int LB>
+__global__ void __launch_bounds__(kUpdWarps * 32)
+qwha_update_kernel(const int32_t* __restrict__ row_ptr, const uint16_t* __restrict__ col,
+                   const uint16_t* __restrict__ cval, int64_t nnz, int64_t N, int64_t K, float scale,
+                   uint16_t* __restrict__ dW, int* flag) {
+  extern __shared__ __align__(16) uint16_t usm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, q = lane & 3;
+  uint16_t* R = usm + (size_t)warp * (kUpdWarpBytes / 2);
+  uint16_t* O = R + 64 * kUpdPitch;                      // one 16-row block of Q, bf16
+  for (int i = lane; i < 64 * kUpdPitch / 8; i += 32) reinterpret_cast<uint4*>(R)[i] = make_uint4(0u, 0u, 0u, 0u);
+  __syncwarp();
+  // G's 16 x 16 diagonal-position block as an A fragment: element (r, c) is nonzero when r
+  // and c lie in the same 2^LB block, with sign (-1)^popcount(r & c & (2^LB - 1)); a block
+  // (ib, ka) of G is this one with the sign (-1)^popcount(ib & ka & (2^(LB-4) - 1)) when
+  // LB >= 4 and ib, ka share a 2^LB block, and zero otherwise.
+  constexpr int m = (1 << LB) - 1;
+  auto gel = [&](int r, int c) -> uint32_t { return pm1_bf16(((r ^ c) & ~m & 15) == 0, __popc(r & c & m)); };
+  uint32_t Ad[4];
+  Ad[0] = gel(g, 2 * q) | (gel(g, 2 * q + 1) << 16);
+  Ad[1] = gel(g + 8, 2 * q) | (gel(g + 8, 2 * q + 1) << 16);
+  Ad[2] = gel(g, 2 * q + 8) | (gel(g, 2 * q + 9) << 16);
+  Ad[3] = gel(g + 8, 2 * q + 8) | (gel(g + 8, 2 * q + 9) << 16);
+  // H_64 as the B operand: rows 16 kn + {2q, 2q+1} (b0) and 16 kn + 8 + {2q, 2q+1} (b1) of
+  // column 8 jt + g carry the signs of H_8 entries (2q.., g) times (-1)^popcount(kn & (jt >> 1))
+  // (and (-1)^(jt & 1) for b1).
+  const uint32_t B0 = pm1_bf16(true, __popc((2 * q) & g)) | (pm1_bf16(true, __popc((2 * q + 1) & g)) << 16);
+  const int64_t ST = (K + 4095) / 4096;
+  const int64_t items = N * ST;
+  const int64_t stride = (int64_t)gridDim.x * kUpdWarps;
+  const uint32_t rbase = static_cast<uint32_t>(__cvta_generic_to_shared(R));
+  bool bad = false;
+  // The warp's items it0, it0 + stride, ... are software-pipelined so that no global load
+  // waits in front of the tensor cores: the row bounds are requested two items ahead, and
+  // the first 64 (column, value) pairs of a row (two per lane) one item ahead; a longer
+  // row loads the rest when it is scattered.
+  auto row_bounds = [&](int64_t it, int& jb, int& je) {
+    jb = je = 0;
+    if (it < items) {
+      const int64_t n = it / ST;
+      jb = __ldg(row_ptr + n);
+      je = __ldg(row_ptr + n + 1);
+    }
+  };
+  auto first_pairs = [&](int jb, int je, uint32_t (&kv)[2]) {
+    const bool ok = jb >= 0 && jb <= je && (int64_t)je <= nnz;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int jj = jb + 32 * u + lane;
+      kv[u] = ok && jj < je ? (uint32_t)__ldg(col + jj) | ((uint32_t)__ldg(cval + jj) << 16) : 0xFFFFFFFFu;
+    }
+  };
+  int64_t it = (int64_t)blockIdx.x * kUpdWarps + warp;
+  int jb_c, je_c, jb_n, je_n;
+  uint32_t kv_c[2];
+  row_bounds(it, jb_c, je_c);
+  row_bounds(it + stride, jb_n, je_n);
+  first_pairs(jb_c, je_c, kv_c);
+  for (; it < items; it += stride) {
+    int jb_nn, je_nn;
+    uint32_t kv_n[2];
+    row_bounds(it + 2 * stride, jb_nn, je_nn);
+    first_pairs(jb_n, je_n, kv_n);
+    const int64_t n = it / ST, c0 = (it % ST) * 4096;
+    const int rows = (int)imin64(64, (K - c0) >> 6);     // tile rows present: whole blocks (b | K)
+    int jb = jb_c, je = je_c;
+    if (jb < 0 || je < jb || (int64_t)je > nnz) {
+      bad = true;
+      jb = je = 0;
+    }
+    auto scatter = [&](uint32_t kc) {
+      const uint32_t k = kc & 0xFFFFu;
+      if ((int64_t)k >= K) {
+        bad = true;
+        return;
+      }
+      const int64_t e = (int64_t)k - c0;
+      if (e >= 0 && e < 4096) R[(e >> 6) * kUpdPitch + (e & 63)] = (uint16_t)(kc >> 16);
+    };
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+      if (jb + 32 * u + lane < je) scatter(kv_c[u]);
+    for (int jj = jb + 64 + lane; jj < je; jj += 32)
+      scatter((uint32_t)__ldg(col + jj) | ((uint32_t)__ldg(cval + jj) << 16));
+    __syncwarp();
+#pragma unroll 1
+    for (int ib = 0; ib < 4; ++ib) {
+      if (16 * ib >= rows) break;
+      // P[ib] (16 x 64) = sum over ka of G[ib, ka] R[ka, :]
+      float P[8][4];
+#pragma unroll
+      for (int jt = 0; jt < 8; ++jt) P[jt][0] = P[jt][1] = P[jt][2] = P[jt][3] = 0.f;
+#pragma unroll
+      for (int ka = 0; ka < 4; ++ka) {
+        if (LB < 6 && ((ib ^ ka) >> (LB > 4 ? LB - 4 : 0)) != 0) continue;   // a zero block of G
+        if (LB < 4 && ka != ib) continue;
+        const int sg = LB >= 4 ? __popc(ib & ka & ((1 << (LB > 4 ? LB - 4 : 0)) - 1)) & 1 : 0;
+        uint32_t A[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) A[i] = Ad[i] ^ (sg ? 0x80008000u : 0u);
+#pragma unroll
+        for (int jp = 0; jp < 4; ++jp) {                 // j-tiles 2 jp, 2 jp + 1
+          const int mi = lane >> 3, r = lane & 7;
+          const uint32_t addr = rbase + (uint32_t)(((16 * ka + 8 * (mi & 1) + r) * kUpdPitch + 8 * (2 * jp + (mi >> 1))) * 2);
+          uint32_t b[4];
+          asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3]) : "r"(addr));
+          upd_mma(P[2 * jp], A, b[0], b[1]);
+          upd_mma(P[2 * jp + 1], A, b[2], b[3]);
+        }
+      }
+      // P as A fragments of the second product, split into bf16 hi + lo
+      uint32_t Ah[4][4], Al[4][4];
+#pragma unroll
+      for (int kn = 0; kn < 4; ++kn) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float* c = P[2 * kn + h];
+          const uint32_t hi01 = pack_bf16x2(c[0], c[1]), hi23 = pack_bf16x2(c[2], c[3]);
+          const uint32_t lo01 = pack_bf16x2(c[0] - __uint_as_float(hi01 << 16), c[1] - __uint_as_float(hi01 & 0xFFFF0000u));
+          const uint32_t lo23 = pack_bf16x2(c[2] - __uint_as_float(hi23 << 16), c[3] - __uint_as_float(hi23 & 0xFFFF0000u));
+          Ah[kn][2 * h] = hi01; Ah[kn][2 * h + 1] = hi23;
+          Al[kn][2 * h] = lo01; Al[kn][2 * h + 1] = lo23;
+        }
+      }
+      // Q[ib] (16 x 64) = P[ib] H_64, eight independent accumulators per step, then scaled
+      // and stored
+      float Q[8][4];
+#pragma unroll
+      for (int jt = 0; jt < 8; ++jt) Q[jt][0] = Q[jt][1] = Q[jt][2] = Q[jt][3] = 0.f;
+#pragma unroll
+      for (int kn = 0; kn < 4; ++kn) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int jt = 0; jt < 8; ++jt) {
+            const int s0 = __popc(kn & (jt >> 1)) & 1, s1 = (s0 + (jt & 1)) & 1;
+            const uint32_t b0 = B0 ^ (s0 ? 0x80008000u : 0u), b1 = B0 ^ (s1 ? 0x80008000u : 0u);
+            upd_mma(Q[jt], h ? Al[kn] : Ah[kn], b0, b1);
+          }
+        }
+      }
+      // through shared memory, so that the block's 16 tile rows (2 KB, contiguous in dW) go
+      // out as whole 16-byte vectors, 512 contiguous bytes per warp store
+#pragma unroll
+      for (int jt = 0; jt < 8; ++jt) {
+        const int col0 = 8 * jt + 2 * q;
+        *reinterpret_cast<uint32_t*>(O + g * kUpdPitch + col0) = pack_bf16x2(Q[jt][0] * scale, Q[jt][1] * scale);
+        *reinterpret_cast<uint32_t*>(O + (g + 8) * kUpdPitch + col0) = pack_bf16x2(Q[jt][2] * scale, Q[jt][3] * scale);
+      }
+      __syncwarp();
+      const int vrows = rows - 16 * ib < 16 ? rows - 16 * ib : 16;
+      uint4* dst = reinterpret_cast<uint4*>(dW + n * K + c0 + 64 * 16 * ib);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int idx = v * 32 + lane, r = idx >> 3, c = idx & 7;   // row r, 16-byte column c
+        if (r < vrows) dst[idx] = *reinterpret_cast<const uint4*>(O + r * kUpdPitch + 8 * c);
+      }
+      __syncwarp();
+    }
+    __syncwarp();
+    for (int i = lane; i < 64 * kUpdPitch / 8; i += 32)   // the tile back to zero
+      reinterpret_cast<uint4*>(R)[i] = make_uint4(0u, 0u, 0u, 0u);
+    __syncwarp();
+    jb_c = jb_n; je_c = je_n; jb_n = jb_nn; je_n = je_nn;
+    kv_c[0] = kv_n[0]; kv_c[1] = kv_n[1];
+  }
+  if (bad) raise_flag(flag, kFlagBadIndex);
+}
+
 // ---- host side -------------------------------------------------------------------------
 
 static int log2_exact(int64_t b) {
@@ -266,11 +468,15 @@ static size_t wht_smem(int64_t b, int64_t bs, int tt) {
 
 static bool qwha_decode_shaped(int64_t M, int64_t K) { return M <= kSmallMMax && small_m_supported(K, 0); }
 
-// Workspace: decode-shaped, the one slab of Z; otherwise Z [M, K] and the dense F [N, K]
-// (bf16) plus the fused GEMM's scratch.
+// dW straight from the compressed rows when the transform blocks are at most 4096 wide;
+// wider blocks go through the densified F and the row transform.
+static bool qwha_update_direct(int64_t K) { return (K & (-K)) <= 4096; }
+
+// Workspace: decode-shaped, the one slab of Z; otherwise dW = F H (bf16 [N, K]), the dense
+// F as well when the blocks are wider than 4096, plus the fused GEMM's scratch.
 int64_t qwha_ws_bytes(int64_t M, int64_t N, int64_t K) {
   if (qwha_decode_shaped(M, K)) return round_up(K * kQwSlab * 2, 256);
-  return round_up(M * K * 2, 256) + round_up(N * K * 2, 256) + ext_fwd_ws_bytes(M, N, K, K);
+  return (qwha_update_direct(K) ? 1 : 2) * round_up(N * K * 2, 256) + ext_fwd_ws_bytes(M, N, K, 0);
 }
 
 // Z = X H, SLAB (decode-shaped: one token per CTA and blocks of more than 512 split into
@@ -336,15 +542,45 @@ ql_status qlora_linear_fwd_qwha(const ql_weight* w, const ql_bf16* X, int64_t M,
     const QwhaRows rows{f->row_ptr, f->col, reinterpret_cast<const uint16_t*>(f->c), f->nnz, Zs};
     return ext_forward(w, X, M, nullptr, nullptr, 0, Y, nullptr, 0, st, &rows);
   }
-  // tensor cores: Y = [X | Z] [W' | F]^T, the adapter as K extension chunks of the fused GEMM
-  uint16_t* Z = reinterpret_cast<uint16_t*>(wsb);
-  const int64_t zb = round_up(M * K * 2, 256);
-  uint16_t* Fd = reinterpret_cast<uint16_t*>(wsb + zb);
+  // tensor cores: Z F^T = X (F H)^T (H symmetric), so the update dW = F H is formed once
+  // (straight from the compressed rows for blocks up to 4096 wide, else F densified and
+  // then the row transform) and added to the decoded weight inside the fused GEMM:
+  // Y = X bf16(W' + dW)^T, one contraction of K.
   const int64_t fb = round_up(N * K * 2, 256);
+  uint16_t* dW = reinterpret_cast<uint16_t*>(wsb);
+  if (qwha_update_direct(K)) {
+    const int64_t b = K & (-K);
+    const int LB = log2_exact(b) - 6;
+    const size_t usm = (size_t)kUpdWarps * kUpdWarpBytes;
+    const float scale = (float)(1.0 / std::sqrt((double)b));
+    const int64_t items = N * ((K + 4095) / 4096);
+    const int grid = (int)imin64((items + kUpdWarps - 1) / kUpdWarps, (int64_t)num_sms() * 3);
+    auto launch = [&](auto kern) -> ql_status {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)usm) != cudaSuccess)
+        return QL_ERR_CUDA;
+      kern<<<grid, kUpdWarps * 32, usm, st>>>(f->row_ptr, f->col, reinterpret_cast<const uint16_t*>(f->c), f->nnz,
+                                              N, K, scale, dW, device_flag_ptr());
+      QL_CHECK_LAUNCH();
+      return QL_OK;
+    };
+    {
+      ProfScope prof(PK_FWD_ADAPTER, st, 1);
+      switch (LB) {
+        case 0: e = launch(qwha_update_kernel<0>); break;
+        case 1: e = launch(qwha_update_kernel<1>); break;
+        case 2: e = launch(qwha_update_kernel<2>); break;
+        case 3: e = launch(qwha_update_kernel<3>); break;
+        case 4: e = launch(qwha_update_kernel<4>); break;
+        case 5: e = launch(qwha_update_kernel<5>); break;
+        default: e = launch(qwha_update_kernel<6>); break;
+      }
+    }
+    if (e != QL_OK) return e;
+    return dw_forward(w, X, M, dW, Y, wsb + fb, ws_bytes - (size_t)fb, st);
+  }
+  uint16_t* Fd = reinterpret_cast<uint16_t*>(wsb + fb);
   {
     ProfScope prof(PK_FWD_ADAPTER, st, 2);
-    e = launch_wht<false>(X, M, K, Z, st);
-    if (e != QL_OK) return e;
     const int rows = densify_rows(K);
     const size_t dsm = (size_t)rows * K * 2;
     if (cudaFuncSetAttribute(qwha_densify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsm) !=
@@ -353,8 +589,10 @@ ql_status qlora_linear_fwd_qwha(const ql_weight* w, const ql_bf16* X, int64_t M,
     qwha_densify_kernel<<<(unsigned)((N + rows - 1) / rows), 256, dsm, st>>>(f->row_ptr, f->col, f->c, f->nnz,
                                                                           N, K, rows, Fd, device_flag_ptr());
     QL_CHECK_LAUNCH();
+    e = launch_wht<false>(Fd, N, K, dW, st);
+    if (e != QL_OK) return e;
   }
-  return ext_forward(w, X, M, Z, Fd, K, Y, wsb + zb + fb, ws_bytes - (size_t)(zb + fb), st);
+  return dw_forward(w, X, M, dW, Y, wsb + 2 * fb, ws_bytes - (size_t)(2 * fb), st);
 }
 
 ql_status ql_wht(const ql_bf16* X, int64_t M, int64_t K, ql_bf16* Z, void* stream) {

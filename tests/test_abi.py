@@ -138,10 +138,11 @@ def test_argument_validation_without_a_device(lib):
 
 def test_workspace_query(lib):
     assert B.workspace_bytes(B.QL_OP_DQ, 0, 0, 0, 0) >= 128
-    # Walsh-Hadamard adapter: decode-shaped, one slab of Z (16 tokens); otherwise Z [M, K],
-    # the dense F [N, K] and the fused GEMM's block scales
+    # Walsh-Hadamard adapter: decode-shaped, one slab of Z (16 tokens); otherwise the update
+    # F H [N, K], the dense F [N, K] too when the transform blocks are wider than 4096, and
+    # the fused GEMM's block scales
     assert B.workspace_bytes(B.QL_OP_FWD_QWHA, 1, 4096, 4096, 0) == 4096 * 16 * 2
-    assert B.workspace_bytes(B.QL_OP_FWD_QWHA, 8192, 11008, 4096, 0) == \
-        8192 * 4096 * 2 + 11008 * 4096 * 2 + 64 * 11008 * 4
-    assert B.workspace_bytes(B.QL_OP_FWD_QWHA, 17, 64, 192, 0) == 6656 + 64 * 192 * 2 + 3 * 64 * 4
+    assert B.workspace_bytes(B.QL_OP_FWD_QWHA, 8192, 11008, 4096, 0) == 11008 * 4096 * 2 + 64 * 11008 * 4
+    assert B.workspace_bytes(B.QL_OP_FWD_QWHA, 17, 64, 192, 0) == 64 * 192 * 2 + 3 * 64 * 4
+    assert B.workspace_bytes(B.QL_OP_FWD_QWHA, 40, 128, 8192, 0) == 2 * 128 * 8192 * 2 + 128 * 128 * 4
     assert B.workspace_bytes(B.QL_OP_FWD_QWHA, 1, 64, 100, 0) == 0

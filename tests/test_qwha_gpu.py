@@ -56,11 +56,15 @@ def _run(M, N, K, r_equiv, fmt, zero_w=False, zero_c=False, seed=1, rows=None):
     (1, 4096, 4096, 16),        # decode-shaped sparse path, one full-width block
     (5, 136, 704, 8),           # decode-shaped, 11 blocks of 64
     (16, 512, 1024, 64),        # decode-shaped, 16 tokens
-    (17, 256, 256, 8),          # smallest tensor-core case (4 extension chunks)
-    (300, 392, 512, 20),
-    (200, 512, 4096, 64),       # 64 extension chunks
-    (70, 264, 11008, 16),       # 43 blocks of 256, 172 extension chunks
-    (40, 128, 8192, 8),         # one block of 8192
+    (17, 256, 256, 8),          # smallest tensor-core case: dW = F H in blocks of 256
+    (300, 392, 512, 20),        # blocks of 512
+    (33, 64, 192, 4),           # blocks of 64 (the tile transform is the row transform alone)
+    (33, 64, 384, 4),           # blocks of 128
+    (24, 128, 1024, 8),         # blocks of 1024
+    (24, 128, 2048, 8),         # blocks of 2048
+    (200, 512, 4096, 64),       # full 4096-wide blocks
+    (70, 264, 11008, 16),       # 43 blocks of 256 over three 4096-column tiles, the last partial
+    (40, 128, 8192, 8),         # one block of 8192: dW through the dense F and the row transform
 ])
 def test_qwha_forward(M, N, K, r_equiv, fmt):
     _run(M, N, K, r_equiv, fmt)
