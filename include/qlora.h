@@ -139,9 +139,10 @@ typedef struct {
 /* NF4 + double quantisation of `count` weights, each exactly as nf4_dq_quantize would
  * quantise it (QLoRA page, "1. 4-bit NormalFloat (NF4)" and "2. Double Quantization": one
  * mean per tensor), for quantising a model's linears together. Weights with whole blocks
- * and 16-byte aligned W and codes share three launches per 128 weights: one pass over all
- * their blocks (codes, absmax and each weight's exact DQ sum), the means, and the group
- * encode; any other weight takes the single-weight path on the stream. Every output is
+ * and 16-byte aligned W and codes share four launches per 128 weights: the workspace's
+ * sums zeroed, one pass over all their blocks (codes, absmax and each weight's exact DQ
+ * sum), the means, and the group encode; any other weight takes the single-weight path on
+ * the stream. Every output is
  * bit-identical to nf4_dq_quantize of that weight.
  * items: HOST array of count descriptors (read before the call returns). count = 0 is a
  * no-op. Each item is checked as nf4_dq_quantize checks its arguments; a bad item returns

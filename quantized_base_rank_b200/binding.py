@@ -278,7 +278,7 @@ def nf4_dq_quantize(W: torch.Tensor, codes=None, absmax=None, qabsmax=None, grou
 
 
 def nf4_dq_quantize_batch(Ws, outs=None):
-    """NF4 + double quantisation of several weights in one call (three launches per 128
+    """NF4 + double quantisation of several weights in one call (four launches per 128
     weights). Ws: list of bf16 tensors on one device. outs: optional list of (codes,
     absmax, qabsmax, group_scale, mean) per weight. Returns that list; each entry equals
     nf4_dq_quantize of its weight bit for bit."""

@@ -425,6 +425,7 @@ qgemm_wdec_kernel(const __grid_constant__ CUtensorMap tmT, const __grid_constant
   using Cfg = WdecCfg<BS, DW>;
   constexpr int BM = Cfg::BM, BN = Cfg::BN, NP = Cfg::NP, SD = Cfg::SD, ST = Cfg::ST, SC = Cfg::SC;
   constexpr int SW = Cfg::SW;
+  constexpr int SWm = SW > 0 ? SW : 1;                 // the update ring's modulus (DW only)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sD = smem;                                   // decoded weight (A operand)
@@ -543,7 +544,7 @@ qgemm_wdec_kernel(const __grid_constant__ CUtensorMap tmT, const __grid_constant
         if (DW) {
           // the update's rows w0..w0+128, columns kc*64..+64, into its own ring (the chunk
           // sequence, there being no extension chunks)
-          const uint32_t sw = gc % SW, pw = (gc / SW) & 1;
+          const uint32_t sw = gc % SWm, pw = (gc / SWm) & 1;
           if (!mbar_wait(dw_empty + 8 * sw, pw ^ 1, lim, abort_word)) { ok = false; ++gc; break; }
           mbar_arrive_expect_tx(dw_full + 8 * sw, Cfg::kDBytes);
           tma_load_2d(smem_u32(sW + sw * Cfg::kDBytes), &tmDW, dw_full + 8 * sw, kc * 64, w0);
@@ -555,7 +556,7 @@ qgemm_wdec_kernel(const __grid_constant__ CUtensorMap tmT, const __grid_constant
       if (DW) {
         // the update chunks issued: all but the last when a wait for the stage gave up
         const uint32_t gdw = ok ? gc : gc - 1;
-        for (uint32_t j = (gdw > (uint32_t)SW ? gdw - SW : 0); j < gdw; ++j) drain_wait(dw_full + 8 * (j % SW), (j / SW) & 1);
+        for (uint32_t j = (gdw > (uint32_t)SWm ? gdw - SWm : 0); j < gdw; ++j) drain_wait(dw_full + 8 * (j % SWm), (j / SWm) & 1);
       }
     }
   } else if (warp == 5 && lane == 0) {
@@ -639,7 +640,7 @@ qgemm_wdec_kernel(const __grid_constant__ CUtensorMap tmT, const __grid_constant
         const uint32_t sc = gc % SC, pc = (gc / SC) & 1;
         const bool w1 = mbar_wait(full_c + 8 * sc, pc, lim, abort_word);
         // DW: the update's chunk gc has landed in its ring
-        const uint32_t sw = DW ? gc % SW : 0, pw = DW ? (gc / SW) & 1 : 0;
+        const uint32_t sw = DW ? gc % SWm : 0, pw = DW ? (gc / SWm) & 1 : 0;
         const bool w3 = w1 && (!DW || mbar_wait(dw_full + 8 * sw, pw, lim, abort_word));
         const bool w2 = w3 && mbar_wait(empty_d + 8 * sd, pd ^ 1, lim, abort_word);
         if (!__all_sync(0xFFFFFFFFu, w2)) { ok = false; break; }

@@ -962,9 +962,23 @@ static ql_status launch_nf4(const uint16_t* W, int64_t n, uint8_t* codes, float*
   return QL_OK;
 }
 
+// Zeroes n 64-bit words of a workspace. A one-CTA kernel node costs about a microsecond
+// in a chain of launches, a memset node about five (measured in a CUDA graph on B200).
+__global__ void __launch_bounds__(256) ws_zero_kernel(unsigned long long* __restrict__ p, int64_t n) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    p[i] = 0ull;
+}
+
+static ql_status zero_ws(unsigned long long* p, int64_t n, cudaStream_t st) {
+  if (n <= 0) return QL_OK;
+  ws_zero_kernel<<<(unsigned)imin64((n + 255) / 256, 64), 256, 0, st>>>(p, n);
+  QL_CHECK_LAUNCH();
+  return QL_OK;
+}
+
 // NF4 + DQ in one cooperative launch: whole blocks, 16-byte aligned W and codes (the
 // single VEC grid). The workspace holds the bins, the ticket and the ready flag, zeroed
-// here. A refused cooperative launch (grid not co-resident) returns QL_ERR_UNSUPPORTED
+// here by ws_zero_kernel. A refused cooperative launch (grid not co-resident) returns QL_ERR_UNSUPPORTED
 // and the caller takes the two-kernel path.
 static ql_status launch_nf4_dq_fused(const uint16_t* W, int64_t n, uint8_t* codes, float* absmax,
                                      int8_t* qabsmax, float* group_scale, float* mean,
@@ -980,8 +994,7 @@ static ql_status launch_nf4_dq_fused(const uint16_t* W, int64_t n, uint8_t* code
   a.dq_ctas = (unsigned)grid; a.nb_total = nb; a.qabsmax = qabsmax; a.group_scale = group_scale;
   const Nf4Tables& tab = nf4_tables();
   const Nf4BoundTable& btab = nf4_bound_table();
-  if (cudaMemsetAsync(dq_ws, 0, (kSumBins + 2) * sizeof(unsigned long long), st) != cudaSuccess)
-    return QL_ERR_CUDA;
+  if (zero_ws(dq_ws, kSumBins + 2, st) != QL_OK) return QL_ERR_CUDA;
   void* params[] = {&a, const_cast<Nf4Tables*>(&tab), const_cast<Nf4BoundTable*>(&btab)};
   if (cudaLaunchCooperativeKernel(reinterpret_cast<void*>(kern), dim3(grid), dim3(kNf4Threads), params, 0, st) !=
       cudaSuccess) {
@@ -1062,9 +1075,8 @@ ql_status dq_quantize(const float* absmax, int64_t nblocks, int8_t* qabsmax, flo
   if (ws_bytes < ql_workspace_bytes(QL_OP_DQ, 0, 0, 0, 0)) return QL_ERR_WORKSPACE;
   cudaStream_t st = as_stream(stream);
   unsigned long long* bins = static_cast<unsigned long long*>(ws);
-  ProfScope prof(PK_DQ, st, 2);
-  if (cudaMemsetAsync(bins, 0, (kSumBins + 1) * sizeof(unsigned long long), st) != cudaSuccess)
-    return QL_ERR_CUDA;
+  ProfScope prof(PK_DQ, st, 3);
+  if (zero_ws(bins, kSumBins + 1, st) != QL_OK) return QL_ERR_CUDA;
   const int64_t chunk = (int64_t)kSumThreads * kSumPerThread;
   const int sum_grid = (int)imax64(1, imin64((nblocks + chunk - 1) / chunk, (int64_t)num_sms() * 8));
   dq_sum_kernel<<<sum_grid, kSumThreads, 0, st>>>(absmax, nblocks, bins, mean, aligned(absmax, 16) ? 1 : 0,
@@ -1086,14 +1098,13 @@ ql_status nf4_dq_quantize(const ql_bf16* W, int64_t n, uint8_t* codes, float* ab
   unsigned long long* bins = static_cast<unsigned long long*>(ws);
   if (n % kBlock == 0 && aligned(W, 16) && aligned(codes, 16)) {
     // one cooperative launch: encode, exact sum, mean and DQ codes
-    ProfScope prof(PK_NF4, st, 1);
+    ProfScope prof(PK_NF4, st, 2);
     const ql_status s = launch_nf4_dq_fused(W, n, codes, absmax, qabsmax, group_scale, mean, bins, st);
     if (s != QL_ERR_UNSUPPORTED) return s;
   }
   {
-    ProfScope prof(PK_NF4, st, nf4_launches(W, n, codes));
-    if (cudaMemsetAsync(bins, 0, (kSumBins + 1) * sizeof(unsigned long long), st) != cudaSuccess)
-      return QL_ERR_CUDA;
+    ProfScope prof(PK_NF4, st, nf4_launches(W, n, codes) + 1);
+    if (zero_ws(bins, kSumBins + 1, st) != QL_OK) return QL_ERR_CUDA;
     const ql_status s = launch_nf4(W, n, codes, absmax, bins, mean, st);
     if (s != QL_OK) return s;
   }
@@ -1148,8 +1159,8 @@ ql_status nf4_dq_quantize_batch(const ql_nf4_dq_item* items, int32_t count, void
       a.blk_start[j + 1] = a.blk_start[j] + nb;
       a.grp_start[j + 1] = a.grp_start[j] + (nb + kGroup - 1) / kGroup;
     }
-    ProfScope prof(PK_NF4, st, 3);
-    if (cudaMemsetAsync(bins, 0, (size_t)cnt * kSumBins * sizeof(unsigned long long), st) != cudaSuccess)
+    ProfScope prof(PK_NF4, st, 4);
+    if (zero_ws(reinterpret_cast<unsigned long long*>(bins), (int64_t)cnt * kSumBins, st) != QL_OK)
       return QL_ERR_CUDA;
     const int64_t total = a.blk_start[cnt];
     const int grid = (int)imax64(1, imin64((total + kNf4Threads - 1) / kNf4Threads, (int64_t)num_sms() * per_sm));
@@ -1173,9 +1184,8 @@ ql_status nf4_quantize_shard(const ql_bf16* W, int64_t n, uint8_t* codes, float*
   if (ws_bytes < ql_workspace_bytes(QL_OP_DQ, 0, 0, 0, 0)) return QL_ERR_WORKSPACE;
   cudaStream_t st = as_stream(stream);
   unsigned long long* wsb = static_cast<unsigned long long*>(ws);
-  ProfScope prof(PK_NF4, st, nf4_launches(W, n, codes));
-  if (cudaMemsetAsync(wsb, 0, (kSumBins + 1) * sizeof(unsigned long long), st) != cudaSuccess)
-    return QL_ERR_CUDA;
+  ProfScope prof(PK_NF4, st, nf4_launches(W, n, codes) + 1);
+  if (zero_ws(wsb, kSumBins + 1, st) != QL_OK) return QL_ERR_CUDA;
   return launch_nf4(W, n, codes, absmax, wsb, nullptr, st, reinterpret_cast<unsigned long long*>(bins));
 }
 
