@@ -704,7 +704,9 @@ qgemm_wdec_kernel(const __grid_constant__ CUtensorMap tmT, const __grid_constant
 // the odd CTA's MMA warp relays "stage s is full here" to the even CTA with one
 // cluster-scope arrive per stage, and the even CTA's commits free the stages of both.
 // =================================================================================
-template <BSrc BS>
+// DW: as WdecCfg, a ring of SW stages for the dense update's chunks (this CTA's 128 rows),
+// paid for with token and code stages.
+template <BSrc BS, bool DW = false>
 struct WpairCfg {
   static constexpr int BM = 128;                                 // weight rows per CTA
   static constexpr int BN = 256;                                 // tokens per pair tile
@@ -716,10 +718,13 @@ struct WpairCfg {
   static constexpr int kCBytes = kCodeBytes + 1024;              // codes + scales
   // decoded-weight stages (filled on this SM, short latency), token stages (TMA from L2,
   // long latency: the deeper ring), code stages
-  static constexpr int SD = 4, ST = 8, SC = (BS == BSrc::NF4 ? 6 : 3);
+  static constexpr int SD = 4, ST = DW ? (BS == BSrc::NF4 ? 6 : 5) : 8;
+  static constexpr int SC = DW ? 3 : (BS == BSrc::NF4 ? 6 : 3);
+  static constexpr int SW = DW ? 3 : 0;                          // update stages (kDBytes each)
   static constexpr int kTmemCols = 512;
   static constexpr int kThreads = (7 + NP) * 32;
-  static constexpr size_t kSmem = (size_t)SD * kDBytes + (size_t)ST * kTBytes + (size_t)SC * kCBytes + 2048;
+  static constexpr size_t kSmem =
+      (size_t)SD * kDBytes + (size_t)ST * kTBytes + (size_t)SC * kCBytes + (size_t)SW * kDBytes + 2048;
   static_assert(kSmem + 1024 <= 232448, "shared memory");
 };
 
@@ -731,20 +736,24 @@ __device__ __forceinline__ int32_t load_row0(int32_t w0, int64_t R) {
   return (int64_t)w0 >= R ? w0 - 128 : w0;
 }
 
-template <BSrc BS, bool W_MN>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(WpairCfg<BS>::kThreads, 1)
+template <BSrc BS, bool W_MN, bool DW = false>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(WpairCfg<BS, DW>::kThreads, 1)
 qgemm_wpair_kernel(const __grid_constant__ CUtensorMap tmT, const __grid_constant__ CUtensorMap tmCodes,
                    const __grid_constant__ CUtensorMap tmScale, const __grid_constant__ CUtensorMap tmTe,
-                   const __grid_constant__ CUtensorMap tmWe, const GemmArgs args) {
-  using Cfg = WpairCfg<BS>;
+                   const __grid_constant__ CUtensorMap tmWe, const __grid_constant__ CUtensorMap tmDW,
+                   const GemmArgs args) {
+  static_assert(!(DW && W_MN), "the dense update is a forward-only operand");
+  using Cfg = WpairCfg<BS, DW>;
   constexpr int BM = Cfg::BM, BN = Cfg::BN, BNH = Cfg::BNH, NP = Cfg::NP, SD = Cfg::SD, ST = Cfg::ST,
                 SC = Cfg::SC;
+  constexpr int SW = Cfg::SW, SWm = SW > 0 ? SW : 1;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sD = smem;                                   // decoded weight (A operand rows of this CTA)
   uint8_t* sT = sD + SD * Cfg::kDBytes;                 // tokens (this CTA's half of B)
   uint8_t* sC = sT + ST * Cfg::kTBytes;                 // codes + scales
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sC + SC * Cfg::kCBytes);
+  uint8_t* sW = sC + SC * Cfg::kCBytes;                 // DW: this CTA's update chunks
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sW + SW * Cfg::kDBytes);
   const uint32_t full_d = smem_u32(bars);
   const uint32_t empty_d = full_d + 8 * SD;
   const uint32_t full_t = empty_d + 8 * SD;
@@ -755,7 +764,8 @@ qgemm_wpair_kernel(const __grid_constant__ CUtensorMap tmT, const __grid_constan
   const uint32_t acc_full = empty_c + 8 * SC;
   const uint32_t acc_empty = acc_full + 16;             // even CTA: epilogue warps of both CTAs
   const uint32_t drain = acc_full + 32;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * SD + 3 * ST + 2 * SC + 5);
+  const uint32_t dw_full = drain + 8, dw_empty = dw_full + 8 * SW;   // DW
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * SD + 3 * ST + 2 * SC + 5 + 2 * SW);
   volatile int* abort_word = reinterpret_cast<volatile int*>(tmem_holder + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -769,6 +779,7 @@ qgemm_wpair_kernel(const __grid_constant__ CUtensorMap tmT, const __grid_constan
     for (int s = 0; s < SC; ++s) { mbar_init(full_c + 8 * s, 1); mbar_init(empty_c + 8 * s, NP); }
     for (int i = 0; i < 2; ++i) { mbar_init(acc_full + 8 * i, 1); mbar_init(acc_empty + 8 * i, 8); }
     mbar_init(drain, 1);
+    for (int s = 0; s < SW; ++s) { mbar_init(dw_full + 8 * s, 1); mbar_init(dw_empty + 8 * s, NP); }
     *abort_word = 0;
     fence_mbar_init();
   }
@@ -776,7 +787,11 @@ qgemm_wpair_kernel(const __grid_constant__ CUtensorMap tmT, const __grid_constan
     tma_prefetch_desc(&tmT);
     if (args.n_ext) tma_prefetch_desc(&tmTe);
   }
-  if (warp == 6 && lane == 0) { tma_prefetch_desc(&tmCodes); tma_prefetch_desc(&tmScale); }
+  if (warp == 6 && lane == 0) {
+    tma_prefetch_desc(&tmCodes);
+    tma_prefetch_desc(&tmScale);
+    if (DW) tma_prefetch_desc(&tmDW);
+  }
   if (warp == 7 && lane == 0 && args.n_ext) tma_prefetch_desc(&tmWe);
   if (warp == 5) tmem_alloc_pair(smem_u32(tmem_holder), Cfg::kTmemCols);
   tc_fence_before();
@@ -852,10 +867,22 @@ qgemm_wpair_kernel(const __grid_constant__ CUtensorMap tmT, const __grid_constan
           tma_load_2d(dst, &tmCodes, fb, BS == BSrc::NF4 ? w0 / 2 : w0, kc * 64);
           tma_load_2d(dst + Cfg::kCodeBytes, &tmScale, fb, (w0 / 64) & ~3, kc * 64);
         }
+        if (DW) {
+          // this CTA's 128 rows of the update, columns kc*64..+64, into its own ring
+          const uint32_t sw = gc % SWm, pw = (gc / SWm) & 1;
+          if (!mbar_wait(dw_empty + 8 * sw, pw ^ 1, lim, abort_word)) { ok = false; ++gc; break; }
+          mbar_arrive_expect_tx(dw_full + 8 * sw, Cfg::kDBytes);
+          tma_load_2d(smem_u32(sW + sw * Cfg::kDBytes), &tmDW, dw_full + 8 * sw, kc * 64, w0);
+        }
       }
     }
-    if (!ok || *abort_word)
+    if (!ok || *abort_word) {
       for (uint32_t j = (gc > (uint32_t)SC ? gc - SC : 0); j < gc; ++j) drain_wait(full_c + 8 * (j % SC), (j / SC) & 1);
+      if (DW) {
+        const uint32_t gdw = ok ? gc : gc - 1;
+        for (uint32_t j = (gdw > (uint32_t)SWm ? gdw - SWm : 0); j < gdw; ++j) drain_wait(dw_full + 8 * (j % SWm), (j / SWm) & 1);
+      }
+    }
   } else if (warp == 5 && lane == 0 && leader) {
     // ---- MMA issuer (even CTA) ----
     constexpr uint32_t kIdMain = idesc_bf16_f32(2 * BM, BN, W_MN ? 1 : 0, 0);
@@ -949,28 +976,38 @@ qgemm_wpair_kernel(const __grid_constant__ CUtensorMap tmT, const __grid_constan
         }
         const uint32_t sc = gc % SC, pc = (gc / SC) & 1;
         const bool w1 = mbar_wait(full_c + 8 * sc, pc, lim, abort_word);
-        const bool w2 = w1 && mbar_wait(empty_d + 8 * sd, pd ^ 1, lim, abort_word);
+        const uint32_t sw = DW ? gc % SWm : 0, pw = DW ? (gc / SWm) & 1 : 0;
+        const bool w3 = w1 && (!DW || mbar_wait(dw_full + 8 * sw, pw, lim, abort_word));
+        const bool w2 = w3 && mbar_wait(empty_d + 8 * sd, pd ^ 1, lim, abort_word);
         if (!__all_sync(0xFFFFFFFFu, w2)) { ok = false; break; }
         const uint8_t* cst = sC + sc * Cfg::kCBytes;
         const float sv = reinterpret_cast<const float*>(cst + Cfg::kCodeBytes)[scale_idx];
         uint4* d = reinterpret_cast<uint4*>(sD + sd * Cfg::kDBytes + d_off);
+        const uint4* u = reinterpret_cast<const uint4*>(sW + sw * Cfg::kDBytes + d_off);
+        auto put = [&](int i, uint4 v) {
+          if (DW) {
+            const uint4 x = u[i];
+            v = make_uint4(add_bf16x2(v.x, x.x), add_bf16x2(v.y, x.y), add_bf16x2(v.z, x.z), add_bf16x2(v.w, x.w));
+          }
+          d[i] = v;
+        };
         if constexpr (BS == BSrc::NF4) {
           const uint4 cv = reinterpret_cast<const uint4*>(cst + code_off)[half];
           uint32_t L[2], H[2];
           nf4_table(q, sv, L, H);
           const int c0i = 4 * half;
-          d[(c0i + 0) ^ key] = nf4_decode8(cv.x, L, H);
-          d[(c0i + 1) ^ key] = nf4_decode8(cv.y, L, H);
-          d[(c0i + 2) ^ key] = nf4_decode8(cv.z, L, H);
-          d[(c0i + 3) ^ key] = nf4_decode8(cv.w, L, H);
+          put((c0i + 0) ^ key, nf4_decode8(cv.x, L, H));
+          put((c0i + 1) ^ key, nf4_decode8(cv.y, L, H));
+          put((c0i + 2) ^ key, nf4_decode8(cv.z, L, H));
+          put((c0i + 3) ^ key, nf4_decode8(cv.w, L, H));
         } else {
           const uint4* src = reinterpret_cast<const uint4*>(cst + code_off) + 2 * half;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const uint4 w = src[h];
             const int c = 4 * half + 2 * h;
-            d[c ^ key] = int8_decode8(w.x, w.y, sv);
-            d[(c + 1) ^ key] = int8_decode8(w.z, w.w, sv);
+            put(c ^ key, int8_decode8(w.x, w.y, sv));
+            put((c + 1) ^ key, int8_decode8(w.z, w.w, sv));
           }
         }
         fence_proxy_async_smem();
@@ -978,6 +1015,7 @@ qgemm_wpair_kernel(const __grid_constant__ CUtensorMap tmT, const __grid_constan
         if (lane == 0) {
           mbar_arrive(full_d + 8 * sd);
           mbar_arrive(empty_c + 8 * sc);
+          if (DW) mbar_arrive(dw_empty + 8 * sw);
         }
         ++gc;
       }

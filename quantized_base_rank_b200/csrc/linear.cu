@@ -93,18 +93,19 @@ static ql_status launch_tma_rp(int rp, const CUtensorMap& a, const CUtensorMap& 
 // percent of each other, the single-CTA kernel ahead).
 static std::atomic<int> g_gemm_pair{0};
 
-template <BSrc BS, bool W_MN>
+template <BSrc BS, bool W_MN, bool DW = false>
 static ql_status launch_wpair(const CUtensorMap& tok, const CUtensorMap& codes, const CUtensorMap& scale,
                               const CUtensorMap& tok_ext, const CUtensorMap& w_ext, const GemmArgs& args,
-                              cudaStream_t st) {
-  auto kern = qgemm_wpair_kernel<BS, W_MN>;
-  const size_t smem = WpairCfg<BS>::kSmem;
+                              cudaStream_t st, const CUtensorMap* dw = nullptr) {
+  auto kern = qgemm_wpair_kernel<BS, W_MN, DW>;
+  if (DW && (!dw || args.n_ext != 0)) return QL_ERR_INVALID_ARG;
+  const size_t smem = WpairCfg<BS, DW>::kSmem;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return QL_ERR_CUDA;
   const int64_t tiles = ((args.R + 255) / 256) * ((args.Cn + 255) / 256);
   const int pairs = (int)imin64(tiles, num_sms() / 2);
   if (pairs <= 0) return QL_OK;
-  kern<<<2 * pairs, WpairCfg<BS>::kThreads, smem, st>>>(tok, codes, scale, tok_ext, w_ext, args);
+  kern<<<2 * pairs, WpairCfg<BS, DW>::kThreads, smem, st>>>(tok, codes, scale, tok_ext, w_ext, dw ? *dw : tok, args);
   QL_CHECK_LAUNCH();
   return QL_OK;
 }
@@ -390,8 +391,9 @@ ql_status dw_forward(const ql_weight* w, const uint16_t* X, int64_t M, const uin
   if (!ws || !aligned(ws, 256)) return QL_ERR_INVALID_ARG;
   if ((int64_t)ws_bytes < ext_fwd_ws_bytes(M, N, K, 0)) return QL_ERR_WORKSPACE;
   float* scales = static_cast<float*>(ws);
+  const bool pair = g_gemm_pair.load() != 0;
   CUtensorMap mXt, mc, ms, mdw;
-  if (!make_map(&mXt, X, K, M, K, 256) || !make_weight_maps(w, scales, false, &mc, &ms) ||
+  if (!make_map(&mXt, X, K, M, K, pair ? 128 : 256) || !make_weight_maps(w, scales, false, &mc, &ms) ||
       !make_map(&mdw, dW, K, N, K, 128))
     return QL_ERR_CUDA;
   {
@@ -403,6 +405,10 @@ ql_status dw_forward(const ql_weight* w, const uint16_t* X, int64_t M, const uin
   y.R = N; y.Cn = M; y.Kc = K; y.n_ext = 0; y.r = 0;
   y.out = Y; y.ld_out = N; y.scale = 1.0f;
   ProfScope prof(PK_FWD_MAIN, st, 1);
+  if (pair) {
+    if (w->fmt == QL_FMT_NF4_DQ) return launch_wpair<BSrc::NF4, false, true>(mXt, mc, ms, mXt, mXt, y, st, &mdw);
+    return launch_wpair<BSrc::INT8, false, true>(mXt, mc, ms, mXt, mXt, y, st, &mdw);
+  }
   if (w->fmt == QL_FMT_NF4_DQ) return launch_wdec<BSrc::NF4, false, true>(mXt, mc, ms, mXt, mXt, y, st, &mdw);
   return launch_wdec<BSrc::INT8, false, true>(mXt, mc, ms, mXt, mXt, y, st, &mdw);
 }

@@ -70,6 +70,18 @@ def test_qwha_forward(M, N, K, r_equiv, fmt):
     _run(M, N, K, r_equiv, fmt)
 
 
+@pytest.mark.parametrize("fmt", ["nf4_dq", "int8"])
+@pytest.mark.parametrize("M,N,K,r_equiv", [(300, 392, 512, 20), (70, 264, 11008, 16), (257, 128, 4096, 32)])
+def test_qwha_forward_pair_gemm(M, N, K, r_equiv, fmt):
+    """The update merged into the decoded weight by the CTA-pair GEMM (256 weight rows x
+    256 tokens per MMA): ragged rows and tokens leave idle halves of pair tiles."""
+    B.lib().ql_set_gemm_pair(1)
+    try:
+        _run(M, N, K, r_equiv, fmt)
+    finally:
+        B.lib().ql_set_gemm_pair(0)
+
+
 @pytest.mark.parametrize("M", [3, 77])
 def test_qwha_adapter_alone(M):
     """W = 0: Y is the Walsh-Hadamard branch alone."""
