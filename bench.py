@@ -35,7 +35,7 @@ NF4_DQ_BYTES_PER_PARAM = 2.0 + 0.5 + 1.0 / 64 + 4.0 / 16384   # bf16 read + code
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the fused
 # forward GEMM on this workload, from one ncu capture (profiles/fwd_main_gemm_upproj_11008x4096_M8192.md),
 # valid only for the kernel sources it was taken on: reported as null once they change.
-FWD_MAIN_TRAFFIC = {"bytes": 102475264 + 149658624, "sources_sha256_16": "03b07d0db5c18512"}
+FWD_MAIN_TRAFFIC = {"bytes": 112071168 + 149585664, "sources_sha256_16": "24736b26d741c823"}
 FWD_MAIN_SOURCES = ("quantized_base_rank_b200/csrc/gemm.cuh", "quantized_base_rank_b200/csrc/sm100.cuh",
                     "quantized_base_rank_b200/csrc/linear.cu", "quantized_base_rank_b200/csrc/common.cuh")
 
