@@ -35,7 +35,7 @@ NF4_DQ_BYTES_PER_PARAM = 2.0 + 0.5 + 1.0 / 64 + 4.0 / 16384   # bf16 read + code
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the fused
 # forward GEMM on this workload, from one ncu capture (profiles/fwd_main_gemm_upproj_11008x4096_M8192.md),
 # valid only for the kernel sources it was taken on: reported as null once they change.
-FWD_MAIN_TRAFFIC = {"bytes": 111643904 + 149806080, "sources_sha256_16": "f35c10c464f05fea"}
+FWD_MAIN_TRAFFIC = {"bytes": 112071168 + 149585664, "sources_sha256_16": "24736b26d741c823"}
 FWD_MAIN_SOURCES = ("quantized_base_rank_b200/csrc/gemm.cuh", "quantized_base_rank_b200/csrc/sm100.cuh",
                     "quantized_base_rank_b200/csrc/linear.cu", "quantized_base_rank_b200/csrc/common.cuh")
 
@@ -345,26 +345,6 @@ def decode_bench(dev, peaks, reps: int = 20):
         out[f"M{M}"] = {"us_per_call": us, "bytes": nbytes, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
                         "frac_8tbs": gbs / 8000.0, "weight_copies": copies}
         del g
-        # the query, key and value projections of one 7B layer (three 4096x4096 weights, each
-        # with its own rank-16 adapter, all reading X): one grouped launch against three calls
-        triples = [qws[3 * i:3 * i + 3] for i in range(copies // 3)]
-        Ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(3)]
-
-        def grouped():
-            for tri in triples:
-                B.linear_fwd_group([(qw, A, Bm, case.alpha) for qw in tri], X, Ys=Ys)
-
-        def singles():
-            for tri in triples:
-                for qw, Yq in zip(tri, Ys):
-                    B.linear_fwd(qw, X, A, Bm, case.alpha, save_T=False, Y=Yq)
-
-        gu = graph_us(grouped, reps=max(1, reps // 4)) / len(triples)
-        su = graph_us(singles, reps=max(1, reps // 4)) / len(triples)
-        qkv_bytes = 3 * (wbytes + 2 * r * K + 2 * N * r + 2 * M * N) + 2 * M * K
-        out[f"qkv_M{M}"] = {"us_grouped": gu, "us_three_calls": su, "bytes": qkv_bytes,
-                            "GB/s_grouped": qkv_bytes / (gu * 1e-6) / 1e9,
-                            "frac_hbm_grouped": qkv_bytes / (gu * 1e-6) / 1e9 / peaks["hbm_gbs"]}
     return out
 
 

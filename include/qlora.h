@@ -232,30 +232,6 @@ ql_status qlora_linear_fwd_static(const ql_weight* w, const ql_bf16* X, int64_t 
                                   const ql_bf16* A, const ql_bf16* B, int32_t r, float alpha,
                                   ql_bf16* Y, ql_bf16* T_save, void* stream);
 
-/* One linear of a group that shares its input (the projections of one layer that read
- * the same tokens, as a decoder's query, key and value projections do). */
-typedef struct {
-  const ql_weight* w;   /* N_g x K, the group's common K and format */
-  const ql_bf16* A;     /* [r, K] bf16, 16-byte aligned; may be NULL when r == 0 */
-  const ql_bf16* B;     /* [N_g, r] bf16, 2-byte aligned; may be NULL when r == 0 */
-  int32_t r;            /* 0 <= r <= 64 (0: the base product alone) */
-  float alpha;          /* the adapter's scale is alpha / r */
-  ql_bf16* Y;           /* [M, N_g] bf16 out, 16-byte aligned */
-} ql_group_item;
-
-/* The decode-shaped forward (M <= 16 tokens) of `count` linears that share X, in one
- * launch: Y_g = bf16(X W'_g^T + (alpha_g / r_g) (X A_g^T) B_g^T) for g < count (QLoRA page,
- * "limitations": the cost of dequantisation at inference; the layer's projections read
- * the same tokens, so their weights stream through one grid instead of one chain link
- * each). Every Y_g equals qlora_linear_fwd of that linear on the same X bit for bit.
- * items: HOST array of count descriptors (read before the call returns), 1 <= count <= 8,
- * every weight with the same K and format, each passing qlora_linear_fwd's weight checks;
- * X [M, K] bf16, 16-byte aligned, 1 <= M <= 16. No workspace. Bad arguments return
- * QL_ERR_INVALID_ARG, shapes the decode-shaped kernel does not take QL_ERR_UNSUPPORTED,
- * before anything is launched. */
-ql_status qlora_linear_fwd_group(const ql_group_item* items, int32_t count, const ql_bf16* X,
-                                 int64_t M, void* stream);
-
 /* A LoRDBA double-binary adapter (LoRDBA page, gist.science/ko/paper/2605.24058, section
  * "2. Methodology", core architecture):
  *     Delta W = sum_{i < ell} diag(alpha_i) B1 diag(beta_i) B2 diag(gamma_i)

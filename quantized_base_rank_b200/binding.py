@@ -45,12 +45,6 @@ class QLNf4DqItem(ctypes.Structure):
                 ("mean", ctypes.c_void_p)]
 
 
-class QLGroupItem(ctypes.Structure):
-    """ql_group_item: one linear of a group that shares its input (qlora_linear_fwd_group)."""
-    _fields_ = [("w", ctypes.c_void_p), ("A", ctypes.c_void_p), ("B", ctypes.c_void_p),
-                ("r", ctypes.c_int32), ("alpha", ctypes.c_float), ("Y", ctypes.c_void_p)]
-
-
 class QLQwha(ctypes.Structure):
     """ql_qwha: the sparse coefficients of a Walsh-Hadamard adapter in compressed rows."""
     _fields_ = [("row_ptr", ctypes.c_void_p), ("col", ctypes.c_void_p), ("c", ctypes.c_void_p),
@@ -109,7 +103,6 @@ _SIGS = {
     "ql_profile_read": ([ctypes.c_int, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)], ctypes.c_int),
     "ql_launch_count": ([], ctypes.c_uint64),
     "qlora_linear_fwd_static": ([ctypes.POINTER(QLWeight), P, I64, P, P, I32, F32, P, P, P], I32),
-    "qlora_linear_fwd_group": ([P, I32, P, I64, P], I32),
 }
 
 # kernel groups of ql_profile_read
@@ -590,34 +583,6 @@ def linear_fwd(qw: QuantWeight, X: torch.Tensor, A: torch.Tensor, B: torch.Tenso
                                   float(alpha), _ptr(Y), _ptr(T), _ptr(ws), ws.numel(),
                                   _stream(dev)), "qlora_linear_fwd")
     return Y, T
-
-
-def linear_fwd_group(items, X: torch.Tensor, Ys=None):
-    """The decode-shaped forward (M <= 16) of several linears sharing X in one launch.
-    items: list of (qw, A, B, alpha), A [r, K] and B [N, r] bf16 (r = 0: A and B may be
-    None). Returns the list of Y [M, N] bf16; each equals linear_fwd of its linear bit for
-    bit."""
-    _need(X, torch.bfloat16, "X")
-    M, K = X.shape
-    dev = X.device
-    arr = (QLGroupItem * max(1, len(items)))()
-    keep = []
-    out = []
-    for g, (qw, A, B, alpha) in enumerate(items):
-        _need_weight(qw, K, dev)
-        r = 0 if A is None else A.shape[0]
-        if r:
-            _need(A, torch.bfloat16, "A", (r, K), dev)
-            _need(B, torch.bfloat16, "B", (qw.N, r), dev)
-        Y = Ys[g] if Ys is not None else torch.empty((M, qw.N), dtype=torch.bfloat16, device=dev)
-        _need(Y, torch.bfloat16, "Y", (M, qw.N), dev)
-        keep.append(qw.desc)
-        arr[g] = QLGroupItem(ctypes.addressof(qw.desc), _ptr(A) if r else None, _ptr(B) if r else None,
-                             r, float(alpha), _ptr(Y))
-        out.append(Y)
-    _check(lib().qlora_linear_fwd_group(ctypes.addressof(arr), len(items), _ptr(X), M, _stream(dev)),
-           "qlora_linear_fwd_group")
-    return out
 
 
 def linear_bwd(qw: QuantWeight, X, dY, A, B, T, alpha: float, dX=None, dA=None, dB=None):

@@ -50,11 +50,6 @@ struct QwhaRows {
 ql_status small_m_forward(const ql_weight* w, const uint16_t* X, int64_t M, const uint16_t* A,
                           const uint16_t* B, int r, float alpha, uint16_t* Y, uint16_t* T_save,
                           cudaStream_t st, const QwhaRows* qw = nullptr);
-// A group of linears sharing X on the decode-shaped path, one launch (checked by the
-// caller as qlora_linear_fwd_group documents).
-ql_status small_m_forward_group(const ql_group_item* items, int count, const uint16_t* X, int64_t M,
-                                cudaStream_t st);
-ql_status check_weight(const ql_weight* w);       // qlora_linear_fwd's weight checks (linear.cu)
 constexpr int64_t kSmallMMax = 16;
 bool small_m_supported(int64_t K, int r);   // 0 <= rank <= 64 (0: no adapter), staging fits in smem
 int64_t lordba_ws_bytes(int64_t M, int64_t N, int64_t K, int r);   // lordba.cu

@@ -312,7 +312,7 @@ static ql_status launch_block_scales(const ql_weight* w, bool transposed, float*
   return QL_OK;
 }
 
-ql_status check_weight(const ql_weight* w) {
+static ql_status check_weight(const ql_weight* w) {
   if (!w || w->N < 1 || w->K < 64 || !w->codes || !aligned(w->codes, 16)) return QL_ERR_INVALID_ARG;
   if (w->K % 64 != 0 || w->N % 8 != 0) return QL_ERR_UNSUPPORTED;
   if (w->fmt == QL_FMT_NF4_DQ) {
@@ -650,20 +650,4 @@ extern "C" ql_status qlora_linear_fwd_static(const ql_weight* w, const ql_bf16* 
   void* ws = static_scratch_ptr();
   if (!ws) return QL_ERR_CUDA;
   return qlora_linear_fwd(w, X, M, A, B, r, alpha, Y, T_save, ws, kStaticScratchBytes, stream);
-}
-
-ql_status qlora_linear_fwd_group(const ql_group_item* items, int32_t count, const ql_bf16* X, int64_t M,
-                                 void* stream) {
-  if (!items || !X || count < 1 || M < 1 || !aligned(X, 16)) return QL_ERR_INVALID_ARG;
-  if (count > 8 || M > kSmallMMax) return QL_ERR_UNSUPPORTED;
-  for (int g = 0; g < count; ++g) {
-    const ql_group_item& it = items[g];
-    const ql_status e = check_weight(it.w);
-    if (e != QL_OK) return e;
-    if (it.w->K != items[0].w->K || it.w->fmt != items[0].w->fmt) return QL_ERR_INVALID_ARG;
-    if (!it.Y || !aligned(it.Y, 16) || it.r < 0) return QL_ERR_INVALID_ARG;
-    if (it.r > 0 && (!it.A || !it.B || !aligned(it.A, 16) || !aligned(it.B, 2))) return QL_ERR_INVALID_ARG;
-    if (it.r > 64 || !small_m_supported(it.w->K, it.r)) return QL_ERR_UNSUPPORTED;
-  }
-  return small_m_forward_group(items, count, X, M, as_stream(stream));
 }

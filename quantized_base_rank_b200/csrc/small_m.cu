@@ -19,8 +19,6 @@
 //    distributed shared memory, so the result is deterministic and no workspace or atomic
 //    is needed. T = sum of the T_kr is reduced the same way for T_save.
 // The codes of the next unit are loaded while the current one is decoded.
-#include <atomic>
-
 #include "common.cuh"
 
 namespace qlb {
@@ -176,29 +174,6 @@ __device__ __forceinline__ uint32_t cluster_rank() {
   return r;
 }
 
-// Warm L2 with the part of one weight that a CTA reads: rows [n0, n0 + 128) over the
-// K-units [u0, u1) (codes and block scales), the adapter rows of that K-range and the
-// CTA's rows of B. Thread t of 256.
-template <int FMT>
-__device__ __forceinline__ void l2_prefetch_tile(const uint8_t* codes, const int8_t* qabsmax, const float* gscale,
-                                                 const float* absmax, const uint16_t* A, const uint16_t* B,
-                                                 int64_t N, int64_t K, int r, int64_t n0, int64_t u0, int64_t u1,
-                                                 int t) {
-  const int64_t rows = N - n0 < kRowsPerCta ? N - n0 : kRowsPerCta;
-  const int64_t KB = K >> 6, k0 = u0 * 256, kend = u1 * 256 < K ? u1 * 256 : K;
-  if (FMT == QL_FMT_NF4_DQ) {
-    l2_prefetch_rows(codes + n0 * (K >> 1), K >> 1, rows, k0 >> 1, kend >> 1, t, 256);
-    l2_prefetch_rows(qabsmax + n0 * KB, KB, rows, u0 * 4, (kend + 63) >> 6, t, 256);
-    const int64_t g0 = (n0 * KB) >> 8, g1 = ((n0 + rows) * KB - 1) >> 8;
-    l2_prefetch_rows(gscale, 0, 1, g0 * 4, g1 * 4 + 4, t, 256);
-  } else {
-    l2_prefetch_rows(codes + n0 * K, K, rows, k0, kend, t, 256);
-    l2_prefetch_rows(absmax + n0 * KB, KB * 4, rows, u0 * 16, ((kend + 63) >> 6) * 4, t, 256);
-  }
-  l2_prefetch_rows(A, K * 2, r, k0 * 2, kend * 2, t, 256);
-  l2_prefetch_rows(B + n0 * r, 0, 1, 0, rows * r * 2, t, 256);
-}
-
 // The last barrier only keeps every CTA's shared memory alive until the other CTAs have
 // read it; each of those remote loads is consumed (summed) before the arrive, so the
 // arrive needs no release ordering.
@@ -327,9 +302,9 @@ __device__ __forceinline__ void qwha_rows_add(const SmallArgs& a, int64_t r0, fl
 // section 2.1: Delta W x = F (H^{-1} x)) for the 16 rows this CTA reduces are added to its
 // partial sums before the cluster reduction, so they reach Y with its one rounding. Only
 // with JT = 0 (no LoRA part).
-// The body of one CTA: cluster index `cluster` (128 weight rows of the weight in `a`).
-template <int NT, int FMT, int JT, bool QW>
-__device__ __forceinline__ void small_m_body(const SmallArgs& a, int64_t cluster) {
+template <int NT, int FMT, int JT, bool QW = false>
+__global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(256, 2)
+small_m_fwd_kernel(const SmallArgs a) {
   constexpr int NTT = NT / 8;                       // token tiles of 8
   constexpr int RP = JT * 16;                       // rank padded to j-tiles of 16
   extern __shared__ __align__(16) uint8_t sm[];
@@ -344,7 +319,7 @@ __device__ __forceinline__ void small_m_body(const SmallArgs& a, int64_t cluster
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, q = lane & 3;
   const uint32_t rank = cluster_rank();
-  const int64_t n0 = cluster * kRowsPerCta;
+  const int64_t n0 = (int64_t)(blockIdx.x / kCS) * kRowsPerCta;
   const int64_t u0 = rank * U / kCS, u1 = (rank + 1) * U / kCS;
   const int nunits = (int)(u1 - u0);
   const int64_t k0 = u0 * 256;
@@ -360,9 +335,20 @@ __device__ __forceinline__ void small_m_body(const SmallArgs& a, int64_t cluster
   // only after the wait; L2 is the point of coherence, so a prefetch never makes a later
   // load return stale data. Every load proper comes after the wait.
   {
-    const int64_t kend = u1 * 256 < a.K ? u1 * 256 : a.K;
+    const int64_t rows = a.N - n0 < kRowsPerCta ? a.N - n0 : kRowsPerCta;
+    const int64_t KB = a.K >> 6, kend = u1 * 256 < a.K ? u1 * 256 : a.K;
     const int t = threadIdx.x;
-    l2_prefetch_tile<FMT>(a.codes, a.qabsmax, a.gscale, a.absmax, a.A, a.B, a.N, a.K, a.r, n0, u0, u1, t);
+    if (FMT == QL_FMT_NF4_DQ) {
+      l2_prefetch_rows(a.codes + n0 * (a.K >> 1), a.K >> 1, rows, k0 >> 1, kend >> 1, t, 256);
+      l2_prefetch_rows(a.qabsmax + n0 * KB, KB, rows, u0 * 4, (kend + 63) >> 6, t, 256);
+      const int64_t g0 = (n0 * KB) >> 8, g1 = ((n0 + rows) * KB - 1) >> 8;
+      l2_prefetch_rows(a.gscale, 0, 1, g0 * 4, g1 * 4 + 4, t, 256);
+    } else {
+      l2_prefetch_rows(a.codes + n0 * a.K, a.K, rows, k0, kend, t, 256);
+      l2_prefetch_rows(a.absmax + n0 * KB, KB * 4, rows, u0 * 16, ((kend + 63) >> 6) * 4, t, 256);
+    }
+    l2_prefetch_rows(a.A, a.K * 2, a.r, k0 * 2, kend * 2, t, 256);
+    l2_prefetch_rows(a.B + n0 * a.r, 0, 1, 0, rows * a.r * 2, t, 256);
     l2_prefetch_rows(a.X, a.K * 2, a.M < NT ? a.M : NT, k0 * 2, kend * 2, t, 256);
     if (QW) {
       // this CTA's rows of F: the offsets, then the values they bound. The grid before
@@ -584,7 +570,7 @@ __device__ __forceinline__ void small_m_body(const SmallArgs& a, int64_t cluster
       const int64_t row = n0 + rr;
       if (tok < a.M && row < a.N) a.Y[tok * a.N + row] = (uint16_t)float_to_bf16_bits(acc);
     }
-    if (a.T_save && cluster == 0) {                       // first cluster also reduces T
+    if (a.T_save && blockIdx.x < (unsigned)kCS) {        // first cluster also reduces T
       for (int i = threadIdx.x; i < RP * NT; i += blockDim.x) {
         const int j = i / NT, tok = i % NT;
         if ((int)(j % kCS) != (int)rank) continue;
@@ -599,72 +585,6 @@ __device__ __forceinline__ void small_m_body(const SmallArgs& a, int64_t cluster
     }
   }
   cluster_sync_relaxed();                               // keep smem alive for the readers
-}
-
-template <int NT, int FMT, int JT, bool QW = false>
-__global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(256, 2)
-small_m_fwd_kernel(const SmallArgs a) {
-  small_m_body<NT, FMT, JT, QW>(a, blockIdx.x / kCS);
-}
-
-// Several weights that share the tokens (the projections of one layer that read the same
-// input) in one launch. Tile c (128 rows of one weight) belongs to the weight g with
-// cl_begin[g] <= c < cl_begin[g + 1]. The grid holds no more clusters than can be resident
-// at once, and each cluster walks the tiles c, c + G, c + 2G, ... (G clusters): before it
-// works on one tile it warms L2 with its next, so from the second tile on its loads find
-// their data on chip. For each tile the weight's fields replace those of `a` in a
-// shared-memory copy of the arguments and the cluster runs exactly the single-weight body,
-// so every output equals that of its own call bit for bit. The body ends on a cluster
-// barrier after the last remote read of this CTA's shared memory (each such load is
-// consumed before the arrive), so the next tile may overwrite it.
-constexpr int kGroupMax = 8;
-struct SmallGroupItem {
-  const uint8_t* codes; const int8_t* qabsmax; const float* gscale; const float* mean; const float* absmax;
-  const uint16_t* A; const uint16_t* B; uint16_t* Y;
-  int64_t N;
-  int r;
-  float s;
-  int b_pairs;
-};
-struct SmallGroup {
-  int count;
-  int cl_begin[kGroupMax + 1];
-  SmallGroupItem item[kGroupMax];
-};
-
-template <int NT, int FMT, int JT>
-__global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(256, 2)
-small_m_group_kernel(const SmallArgs a, const __grid_constant__ SmallGroup grp) {
-  __shared__ SmallArgs s_a;
-  const int total = grp.cl_begin[grp.count];
-  const int G = (int)(gridDim.x / kCS);
-  const uint32_t rank = cluster_rank();
-  const int64_t U = (a.K + 255) / 256;
-  const int64_t u0 = rank * U / kCS, u1 = (rank + 1) * U / kCS;
-  auto item_of = [&](int c) {
-    int g = 0;
-    while (g + 1 < grp.count && c >= grp.cl_begin[g + 1]) ++g;
-    return g;
-  };
-  for (int c = (int)(blockIdx.x / kCS); c < total; c += G) {
-    const int g = item_of(c);
-    if (threadIdx.x == 0) {
-      SmallArgs t = a;
-      const SmallGroupItem& it = grp.item[g];
-      t.codes = it.codes; t.qabsmax = it.qabsmax; t.gscale = it.gscale; t.mean = it.mean; t.absmax = it.absmax;
-      t.A = it.A; t.B = it.B; t.Y = it.Y; t.N = it.N; t.r = it.r; t.s = it.s; t.b_pairs = it.b_pairs;
-      s_a = t;
-    }
-    __syncthreads();
-    const int cn = c + G;
-    if (cn < total) {
-      const int gn = item_of(cn);
-      const SmallGroupItem& it = grp.item[gn];
-      l2_prefetch_tile<FMT>(it.codes, it.qabsmax, it.gscale, it.absmax, it.A, it.B, it.N, a.K, it.r,
-                            (int64_t)(cn - grp.cl_begin[gn]) * kRowsPerCta, u0, u1, threadIdx.x);
-    }
-    small_m_body<NT, FMT, JT, false>(s_a, c - grp.cl_begin[g]);
-  }
 }
 
 size_t small_m_smem(int NT, int units_max, int r) {
@@ -704,89 +624,6 @@ bool small_m_supported(int64_t K, int r) {
   const int64_t U = (K + 255) / 256;
   const int units_max = (int)((U + kCS - 1) / kCS);
   return small_m_smem(16, units_max, r) <= 200 * 1024;
-}
-
-template <int NT, int FMT, int JT>
-static ql_status launch_group(const SmallArgs& a, const SmallGroup& grp, cudaStream_t st) {
-  auto kern = small_m_group_kernel<NT, FMT, JT>;
-  const size_t smem = small_m_smem(NT, a.kr_max / 256, JT * 16);
-  if (smem > 227 * 1024) return QL_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return QL_ERR_CUDA;
-  cudaLaunchConfig_t cfg = {};
-  const int total = grp.cl_begin[grp.count];
-  cfg.gridDim = dim3(total * kCS);
-  cfg.blockDim = dim3(256);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  // as many clusters as can be resident at once; the occupancy query is made once per
-  // shared-memory size of this instantiation (cached as smem << 20 | clusters)
-  static std::atomic<int64_t> cache{-1};
-  int64_t c = cache.load(std::memory_order_relaxed);
-  if (c < 0 || (c >> 20) != (int64_t)smem) {
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
-      (void)cudaGetLastError();
-      n = 0;
-    }
-    c = ((int64_t)smem << 20) | (int64_t)(n & 0xFFFFF);
-    cache.store(c, std::memory_order_relaxed);
-  }
-  const int resident = (int)(c & 0xFFFFF);
-  if (resident > 0 && resident < total) cfg.gridDim = dim3(resident * kCS);
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, a, grp) != cudaSuccess) return QL_ERR_CUDA;
-  QL_CHECK_LAUNCH();
-  return QL_OK;
-}
-
-// Host entry for a group of weights sharing X (checked by the caller: 1 <= count <= 8,
-// M <= 16, one K and one format, 0 <= r <= 64 with small_m_supported(K, r)).
-ql_status small_m_forward_group(const ql_group_item* items, int count, const uint16_t* X, int64_t M,
-                                cudaStream_t st) {
-  if (count < 1 || count > kGroupMax) return QL_ERR_UNSUPPORTED;
-  const ql_weight* w0 = items[0].w;
-  SmallArgs a{};
-  a.flag = device_flag_ptr();
-  a.X = X; a.M = M; a.K = w0->K; a.fmt = w0->fmt; a.T_save = nullptr;
-  const int64_t U = (w0->K + 255) / 256;
-  a.kr_max = (int)(((U + kCS - 1) / kCS) * 256);
-  const Nf4Tables& t = nf4_tables();
-  for (int i = 0; i < 16; ++i) a.q[i] = t.q[i];
-  SmallGroup grp{};
-  grp.count = count;
-  int rmax = 0, cl = 0;
-  for (int g = 0; g < count; ++g) {
-    const ql_group_item& it = items[g];
-    SmallGroupItem& o = grp.item[g];
-    o.codes = static_cast<const uint8_t*>(it.w->codes);
-    o.qabsmax = it.w->qabsmax; o.gscale = it.w->group_scale; o.mean = it.w->mean; o.absmax = it.w->absmax;
-    o.A = it.A; o.B = it.B; o.Y = it.Y; o.N = it.w->N; o.r = it.r;
-    o.s = it.r > 0 ? it.alpha / (float)it.r : 0.0f;
-    o.b_pairs = (it.r % 2 == 0 && aligned(it.B, 4)) ? 1 : 0;
-    rmax = it.r > rmax ? it.r : rmax;
-    grp.cl_begin[g] = cl;
-    cl += (int)((it.w->N + kRowsPerCta - 1) / kRowsPerCta);
-  }
-  grp.cl_begin[count] = cl;
-  a.codes = grp.item[0].codes;                     // overwritten per cluster on the device
-  ProfScope prof(PK_FWD_SMALL, st, 1);
-  const int jt = (rmax + 15) / 16;
-  const bool nf4 = w0->fmt == QL_FMT_NF4_DQ;
-  if (M <= 8) {
-    if (nf4) return jt == 0 ? launch_group<8, QL_FMT_NF4_DQ, 0>(a, grp, st) : jt == 1 ? launch_group<8, QL_FMT_NF4_DQ, 1>(a, grp, st)
-                  : jt == 2 ? launch_group<8, QL_FMT_NF4_DQ, 2>(a, grp, st) : launch_group<8, QL_FMT_NF4_DQ, 4>(a, grp, st);
-    return jt == 0 ? launch_group<8, QL_FMT_INT8_B64, 0>(a, grp, st) : jt == 1 ? launch_group<8, QL_FMT_INT8_B64, 1>(a, grp, st)
-         : jt == 2 ? launch_group<8, QL_FMT_INT8_B64, 2>(a, grp, st) : launch_group<8, QL_FMT_INT8_B64, 4>(a, grp, st);
-  }
-  if (nf4) return jt == 0 ? launch_group<16, QL_FMT_NF4_DQ, 0>(a, grp, st) : jt == 1 ? launch_group<16, QL_FMT_NF4_DQ, 1>(a, grp, st)
-                : jt == 2 ? launch_group<16, QL_FMT_NF4_DQ, 2>(a, grp, st) : launch_group<16, QL_FMT_NF4_DQ, 4>(a, grp, st);
-  return jt == 0 ? launch_group<16, QL_FMT_INT8_B64, 0>(a, grp, st) : jt == 1 ? launch_group<16, QL_FMT_INT8_B64, 1>(a, grp, st)
-       : jt == 2 ? launch_group<16, QL_FMT_INT8_B64, 2>(a, grp, st) : launch_group<16, QL_FMT_INT8_B64, 4>(a, grp, st);
 }
 
 // Host entry used by qlora_linear_fwd when M <= 16.

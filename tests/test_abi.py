@@ -131,35 +131,6 @@ def test_argument_validation_without_a_device(lib):
     assert lib.ql_launch_count() == c0
     assert B.workspace_bytes(B.QL_OP_DQ_BATCH, 224, 0, 0, 0) == 128 * 16 * 8
     assert B.workspace_bytes(B.QL_OP_DQ_BATCH, 1, 0, 0, 0) == 256
-    # grouped decode-shaped forward: empty or oversize groups, too many tokens, a null or
-    # misaligned X, mixed K or format, a missing adapter, a rank past 64: all refused
-    # before anything is launched
-    wq = B.QLWeight(0, 0, 4096, 4096, 16, 0, 16, 16, 16)
-    wk = B.QLWeight(0, 0, 1024, 4096, 16, 0, 16, 16, 16)
-    wbadk = B.QLWeight(0, 0, 1024, 2048, 16, 0, 16, 16, 16)
-    wint8 = B.QLWeight(1, 0, 1024, 4096, 16, 16, 0, 0, 0)
-    G = B.QLGroupItem
-    def grp(*its):
-        arr = (G * len(its))(*its)
-        return arr, len(its)
-    good = [G(ctypes.addressof(wq), 16, 16, 16, 32.0, 16), G(ctypes.addressof(wk), None, None, 0, 0.0, 16)]
-    c0 = lib.ql_launch_count()
-    arr, n = grp(*good)
-    assert lib.qlora_linear_fwd_group(None, 1, 16, 1, None) == B.QL_ERR_INVALID_ARG
-    assert lib.qlora_linear_fwd_group(arr, 0, 16, 1, None) == B.QL_ERR_INVALID_ARG
-    assert lib.qlora_linear_fwd_group(arr, n, None, 1, None) == B.QL_ERR_INVALID_ARG
-    assert lib.qlora_linear_fwd_group(arr, n, 24, 1, None) == B.QL_ERR_INVALID_ARG
-    assert lib.qlora_linear_fwd_group(arr, n, 16, 17, None) == B.QL_ERR_UNSUPPORTED
-    nine, _ = grp(*([good[0]] * 9))
-    assert lib.qlora_linear_fwd_group(nine, 9, 16, 1, None) == B.QL_ERR_UNSUPPORTED
-    for bad in (G(ctypes.addressof(wbadk), None, None, 0, 0.0, 16), G(ctypes.addressof(wint8), None, None, 0, 0.0, 16),
-                G(ctypes.addressof(wk), None, 16, 8, 16.0, 16), G(ctypes.addressof(wk), 16, 16, 8, 16.0, None),
-                G(ctypes.addressof(wk), 24, 16, 8, 16.0, 16)):
-        arr2, n2 = grp(good[0], bad)
-        assert lib.qlora_linear_fwd_group(arr2, n2, 16, 1, None) == B.QL_ERR_INVALID_ARG
-    arr3, n3 = grp(good[0], G(ctypes.addressof(wk), 16, 16, 65, 16.0, 16))
-    assert lib.qlora_linear_fwd_group(arr3, n3, 16, 1, None) == B.QL_ERR_UNSUPPORTED
-    assert lib.ql_launch_count() == c0
     # misaligned or null pointers, bad shapes: all rejected synchronously
     assert lib.qlora_linear_fwd(ctypes.byref(w), None, 1, None, None, 8, 16.0, None, None,
                                 None, 0, None) == B.QL_ERR_INVALID_ARG
