@@ -185,6 +185,14 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// Store two floats at the same shared-memory offset in CTA `rank` of the cluster (8-byte
+// aligned). Visible to that CTA after a release/acquire cluster barrier.
+__device__ __forceinline__ void st_cluster_f32x2(float* local, uint32_t rank, float x, float y) {
+  uint32_t addr = static_cast<uint32_t>(__cvta_generic_to_shared(local)), remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(addr), "r"(rank));
+  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" :: "r"(remote), "f"(x), "f"(y) : "memory");
+}
+
 // Read a float from the same shared-memory offset in CTA `rank` of the cluster. The loads
 // stay in program order after the cluster barrier; callers issue several before using any,
 // so they are in flight together.
@@ -327,6 +335,9 @@ small_m_fwd_kernel(const SmallArgs a) {
   // The next launch on the stream may start now and warm L2 with its own weight while
   // this one finishes.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // First half of a cluster barrier whose wait, just before the partial sums are stored
+  // into other CTAs' shared memory, guarantees that every CTA of the cluster has started.
+  if constexpr (!QW) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 
   // Before the dependency wait this grid only warms L2 with what it is about to read: the
   // codes and constants of its blocks, the adapter rows of its K-range, its rows of B and
@@ -543,22 +554,25 @@ small_m_fwd_kernel(const SmallArgs a) {
     }
   }
 
-  // ---- partial sums -> smem, then the fixed-order cluster reduction ----
+  // ---- partial sums, then the fixed-order cluster reduction ----
+  // CTA c reduces the weight rows [16c, 16c + 16) of the cluster's 128, which warp c of
+  // every CTA holds. For each such row and token, Y is the sum of the eight CTAs' partials
+  // taken in cluster-rank order, so the result does not depend on timing.
+  constexpr int kRowsPerRank = kRowsPerCta / kCS;      // 16
+  if constexpr (QW) {
+    // pull form: partials in the CTA's own sD (rows in the cluster's order), the sparse
+    // sums added to the CTA's own rows, then every CTA reads its rows from all eight
 #pragma unroll
-  for (int t = 0; t < NTT; ++t) {
-    const int rg = warp * 16 + g;
-    sD[rg * NT + t * 8 + 2 * q] = d[t][0];
-    sD[rg * NT + t * 8 + 2 * q + 1] = d[t][1];
-    sD[(rg + 8) * NT + t * 8 + 2 * q] = d[t][2];
-    sD[(rg + 8) * NT + t * 8 + 2 * q + 1] = d[t][3];
-  }
-  if (QW) {
+    for (int t = 0; t < NTT; ++t) {
+      const int rg = warp * 16 + g;
+      sD[rg * NT + t * 8 + 2 * q] = d[t][0];
+      sD[rg * NT + t * 8 + 2 * q + 1] = d[t][1];
+      sD[(rg + 8) * NT + t * 8 + 2 * q] = d[t][2];
+      sD[(rg + 8) * NT + t * 8 + 2 * q + 1] = d[t][3];
+    }
     __syncthreads();
-    qwha_rows_add<NT>(a, n0 + rank * (kRowsPerCta / kCS), sD + (size_t)rank * (kRowsPerCta / kCS) * NT);
-  }
-  cluster_sync_all();
-  {
-    constexpr int kRowsPerRank = kRowsPerCta / kCS;    // 16
+    qwha_rows_add<NT>(a, n0 + rank * kRowsPerRank, sD + (size_t)rank * kRowsPerRank * NT);
+    cluster_sync_all();
     for (int i = threadIdx.x; i < kRowsPerRank * NT; i += blockDim.x) {
       const int rr = (int)rank * kRowsPerRank + i / NT, tok = i % NT;
       float part[kCS];
@@ -570,7 +584,32 @@ small_m_fwd_kernel(const SmallArgs a) {
       const int64_t row = n0 + rr;
       if (tok < a.M && row < a.N) a.Y[tok * a.N + row] = (uint16_t)float_to_bf16_bits(acc);
     }
-    if (a.T_save && blockIdx.x < (unsigned)kCS) {        // first cluster also reduces T
+  } else {
+    // push form: warp w stores its partials straight into CTA w's sD, in the slot of this
+    // source CTA (sD row 16 * rank + i holds this CTA's partial of the owner's row i); after
+    // one release/acquire barrier each CTA sums its eight slots from its own shared memory.
+    // Nothing reads another CTA's shared memory after that barrier (outside the T reduction
+    // below), so no second barrier is needed before the CTA exits.
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+    const int rs = (int)rank * kRowsPerRank + g;
+#pragma unroll
+    for (int t = 0; t < NTT; ++t) {
+      st_cluster_f32x2(sD + rs * NT + t * 8 + 2 * q, (uint32_t)warp, d[t][0], d[t][1]);
+      st_cluster_f32x2(sD + (rs + 8) * NT + t * 8 + 2 * q, (uint32_t)warp, d[t][2], d[t][3]);
+    }
+    cluster_sync_all();
+    for (int i = threadIdx.x; i < kRowsPerRank * NT; i += blockDim.x) {
+      const int rr = i / NT, tok = i % NT;
+      float acc = 0.0f;
+#pragma unroll
+      for (int c = 0; c < kCS; ++c) acc += sD[(c * kRowsPerRank + rr) * NT + tok];
+      const int64_t row = n0 + (int64_t)rank * kRowsPerRank + rr;
+      if (tok < a.M && row < a.N) a.Y[tok * a.N + row] = (uint16_t)float_to_bf16_bits(acc);
+    }
+  }
+  const bool reduce_T = a.T_save && blockIdx.x < (unsigned)kCS;   // uniform over the cluster
+  {
+    if (reduce_T) {                                       // first cluster also reduces T
       for (int i = threadIdx.x; i < RP * NT; i += blockDim.x) {
         const int j = i / NT, tok = i % NT;
         if ((int)(j % kCS) != (int)rank) continue;
@@ -584,7 +623,8 @@ small_m_fwd_kernel(const SmallArgs a) {
       }
     }
   }
-  cluster_sync_relaxed();                               // keep smem alive for the readers
+  // keep shared memory alive for the readers of the pull reductions
+  if (QW || reduce_T) cluster_sync_relaxed();
 }
 
 size_t small_m_smem(int NT, int units_max, int r) {
