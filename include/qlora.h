@@ -283,20 +283,25 @@ typedef struct {
 } ql_qwha;
 
 /* Forward of the quantised linear with a Walsh-Hadamard adapter, unmerged:
- *   Y [M, N] = bf16( bf16(X W'^T) + sum over row n's values of c_j * Z[m, col_j] ),
+ *   Y [M, N] = bf16( X W'^T + sum over row n's values of c_j * Z[m, col_j] ),
  *   Z = X H^{-T} = X H  (H^{-1} x per token), computed in fp32 by the add/subtract
- *   recursion and rounded once to bf16; the sparse sums accumulate in fp32.
+ *   recursion and rounded once to bf16; products and sums accumulate in fp32 and Y is
+ *   rounded once (the large-M form below rounds W' + dW to bf16 first).
  * Shapes and formats as qlora_linear_fwd (K a multiple of 64, K <= 65536, N a multiple
  * of 8); the Walsh-Hadamard block (the largest power of two dividing K) is at most
- * 16384, else QL_ERR_UNSUPPORTED. M <= 16: the base product of the decode-shaped kernel,
- * then the transform and a sparse product that gathers Z by column index; M > 16: F is
- * written out as a dense bf16 [N, K] and Z F^T runs on the tensor cores as K/64
- * extension chunks of the same fused GEMM as qlora_linear_fwd. Column indices >= K and row offsets outside [0, nnz] are skipped on the
- * device and reported as QL_ERR_INVALID_ARG by ql_get_device_status; the contents of
- * the index arrays are not read on the host.
+ * 16384, else QL_ERR_UNSUPPORTED. M <= 16: the transform of the tokens into one slab of
+ * Z, then the decode-shaped kernel, which adds each row's sparse sum (Z gathered by
+ * column index) to its partial sums before the cluster reduction. M > 16: since H is
+ * symmetric, Z F^T = X (F H)^T, so the update dW = bf16(F H) [N, K] is formed (straight
+ * from the compressed rows for blocks up to 4096 wide, else from F written out dense and
+ * transformed row by row) and the fused GEMM of qlora_linear_fwd adds it to the decoded
+ * weight before the product: Y = bf16(X bf16(W' + dW)^T). Column indices >= K and row
+ * offsets outside [0, nnz] are skipped on the device and reported as QL_ERR_INVALID_ARG
+ * by ql_get_device_status; the contents of the index arrays are not read on the host.
+ * Every argument check, the weight's included, is made before the first launch.
  * ws: ql_workspace_bytes(QL_OP_FWD_QWHA, M, N, K, 0) bytes, 256-byte aligned (M <= 16:
- * one slab of Z, [K][16] bf16; otherwise Z [M, K], the dense F [N, K] and the GEMM's
- * block scales). */
+ * one slab of Z, [K][16] bf16; otherwise dW [N, K], the dense F [N, K] as well for blocks
+ * wider than 4096, and the GEMM's block scales). */
 ql_status qlora_linear_fwd_qwha(const ql_weight* w, const ql_bf16* X, int64_t M,
                                 const ql_qwha* adapter, ql_bf16* Y, void* ws,
                                 size_t ws_bytes, void* stream);

@@ -14,6 +14,7 @@
 #include <cuda_fp16.h>
 
 #include "common.cuh"
+#include "weight_check.cuh"
 
 namespace qlb {
 
@@ -70,7 +71,11 @@ using namespace qlb;
 extern "C" ql_status qlora_linear_fwd_lordba(const ql_weight* w, const ql_bf16* X, int64_t M,
                                              const ql_lordba* ad, ql_bf16* Y, void* ws, size_t ws_bytes,
                                              void* stream) {
-  if (!w || !ad || !X || !Y || M < 1) return QL_ERR_INVALID_ARG;
+  // every refusal of the wrapped forward is made here, before the expansion is launched
+  const ql_status ws0 = weight_desc_status(w);
+  if (ws0 != QL_OK) return ws0;
+  if (!ad || !X || !Y || M < 1 || !aligned(X, 16) || !aligned(Y, 16)) return QL_ERR_INVALID_ARG;
+  if (M > (int64_t(1) << 31)) return QL_ERR_UNSUPPORTED;
   if (ad->R < 1 || ad->ell < 1 || !ad->B1 || !ad->B2 || !ad->alpha || !ad->beta || !ad->gamma)
     return QL_ERR_INVALID_ARG;
   const int64_t r64 = (int64_t)ad->R * ad->ell;
@@ -79,7 +84,6 @@ extern "C" ql_status qlora_linear_fwd_lordba(const ql_weight* w, const ql_bf16* 
   if (!aligned(ad->B1, 4) || !aligned(ad->B2, 4) || !aligned(ad->alpha, 2) || !aligned(ad->beta, 2) ||
       !aligned(ad->gamma, 2))
     return QL_ERR_INVALID_ARG;
-  if (w->N < 1 || w->K < 1 || w->K % 64 != 0) return QL_ERR_INVALID_ARG;
   const int64_t N = w->N, K = w->K;
   if (!ws || !aligned(ws, 256)) return QL_ERR_INVALID_ARG;
   if ((int64_t)ws_bytes < lordba_ws_bytes(M, N, K, r)) return QL_ERR_WORKSPACE;

@@ -23,6 +23,7 @@
 #include <cmath>
 
 #include "common.cuh"
+#include "weight_check.cuh"
 
 namespace qlb {
 
@@ -513,13 +514,17 @@ extern "C" {
 
 ql_status qlora_linear_fwd_qwha(const ql_weight* w, const ql_bf16* X, int64_t M, const ql_qwha* f, ql_bf16* Y,
                                 void* ws, size_t ws_bytes, void* stream) {
-  if (!w || !f || !X || !Y || M < 1 || !aligned(X, 16) || !aligned(Y, 16)) return QL_ERR_INVALID_ARG;
+  // every refusal of the wrapped forward is made here, before the transform or the update
+  // is launched
+  const ql_status ws0 = weight_desc_status(w);
+  if (ws0 != QL_OK) return ws0;
+  if (!f || !X || !Y || M < 1 || !aligned(X, 16) || !aligned(Y, 16)) return QL_ERR_INVALID_ARG;
+  if (M > (int64_t(1) << 31)) return QL_ERR_UNSUPPORTED;
   if (!f->row_ptr || f->nnz < 0 || (f->nnz > 0 && (!f->col || !f->c))) return QL_ERR_INVALID_ARG;
   if (!aligned(f->row_ptr, 4) || !aligned(f->col, 2) || !aligned(f->c, 2)) return QL_ERR_INVALID_ARG;
   if (f->nnz >= (int64_t(1) << 31) || w->K > 65536) return QL_ERR_UNSUPPORTED;
   if (!ws || !aligned(ws, 256)) return QL_ERR_INVALID_ARG;
   const int64_t N = w->N, K = w->K;
-  if (K < 64 || K % 64 != 0 || N % 8 != 0) return QL_ERR_UNSUPPORTED;
   if ((int64_t)ws_bytes < qwha_ws_bytes(M, N, K)) return QL_ERR_WORKSPACE;
   {
     const int64_t b = K & (-K);

@@ -136,6 +136,50 @@ def test_argument_validation_without_a_device(lib):
                                 None, 0, None) == B.QL_ERR_INVALID_ARG
 
 
+def test_adapter_entries_refuse_what_the_linear_refuses_before_any_launch(lib):
+    """The LoRDBA and Walsh-Hadamard forwards launch a preparation kernel before the fused
+    linear, so they must make every refusal of the linear first: a bad weight descriptor,
+    misaligned tokens or output, too many tokens. Each must return the linear's own status
+    and launch nothing (on a machine without a GPU a launch would fail with a CUDA error
+    instead)."""
+    P = 16                                                       # any 16-byte-aligned address
+    good = B.QLWeight(0, 0, 64, 64, P, 0, P, P, P)
+    bad_weights = {
+        "null descriptor": None,
+        "no codes": B.QLWeight(0, 0, 64, 64, 0, 0, P, P, P),
+        "misaligned codes": B.QLWeight(0, 0, 64, 64, 24, 0, P, P, P),
+        "N = 0": B.QLWeight(0, 0, 0, 64, P, 0, P, P, P),
+        "K below 64": B.QLWeight(0, 0, 64, 32, P, 0, P, P, P),
+        "K not a multiple of 64": B.QLWeight(0, 0, 64, 96, P, 0, P, P, P),
+        "N not a multiple of 8": B.QLWeight(0, 0, 60, 64, P, 0, P, P, P),
+        "NF4 without the DQ codes": B.QLWeight(0, 0, 64, 64, P, 0, 0, P, P),
+        "NF4 without the group scales": B.QLWeight(0, 0, 64, 64, P, 0, P, 0, P),
+        "NF4 without the mean": B.QLWeight(0, 0, 64, 64, P, 0, P, P, 0),
+        "int8 without absmax": B.QLWeight(1, 0, 64, 64, P, 0, 0, 0, 0),
+        "int8 with misaligned absmax": B.QLWeight(1, 0, 64, 64, P, 18, 0, 0, 0),
+        "unknown format": B.QLWeight(7, 0, 64, 64, P, P, P, P, P),
+    }
+    ad_l = B.QLLordba(4, 1, P, P, P, P, P)
+    ad_q = B.QLQwha(P, P, P, 4)
+    big = 1 << 40
+    c0 = lib.ql_launch_count()
+    for name, w in bad_weights.items():
+        wp = ctypes.byref(w) if w is not None else None
+        for M in (1, 40):
+            want = lib.qlora_linear_fwd(wp, P, M, P, P, 4, 4.0, P, None, 256, big, None)
+            assert want in (B.QL_ERR_INVALID_ARG, B.QL_ERR_UNSUPPORTED), name
+            assert lib.qlora_linear_fwd_lordba(wp, P, M, ctypes.addressof(ad_l), P, 256, big, None) == want, name
+            assert lib.qlora_linear_fwd_qwha(wp, P, M, ctypes.addressof(ad_q), P, 256, big, None) == want, name
+    for X, Y, M, want in ((24, P, 1, B.QL_ERR_INVALID_ARG), (P, 24, 40, B.QL_ERR_INVALID_ARG),
+                          (P, P, (1 << 31) + 1, B.QL_ERR_UNSUPPORTED)):
+        assert lib.qlora_linear_fwd(ctypes.byref(good), X, M, P, P, 4, 4.0, Y, None, 256, big, None) == want
+        assert lib.qlora_linear_fwd_lordba(ctypes.byref(good), X, M, ctypes.addressof(ad_l), Y, 256, big,
+                                           None) == want
+        assert lib.qlora_linear_fwd_qwha(ctypes.byref(good), X, M, ctypes.addressof(ad_q), Y, 256, big,
+                                         None) == want
+    assert lib.ql_launch_count() == c0
+
+
 def test_workspace_query(lib):
     assert B.workspace_bytes(B.QL_OP_DQ, 0, 0, 0, 0) >= 128
     # Walsh-Hadamard adapter: decode-shaped, one slab of Z (16 tokens); otherwise the update
