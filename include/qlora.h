@@ -181,7 +181,8 @@ ql_status int8_quantize(const ql_bf16* W, int64_t n, int8_t* codes, float* absma
 /* Dequantise a whole weight into bf16 W' [N, K] (device). NF4_DQ:
  * a' = fp32(fp32(qabsmax*group_scale) + mean), W'_j = bf16(fp32(q[code_j] * a'));
  * INT8_B64: W'_j = bf16(fp32(code_j * fp32(absmax/127))). Used for checks; the
- * linear kernels dequantise on the fly and never materialise W'. */
+ * linear kernels dequantise on the fly and never materialise W'. Wout needs 2-byte
+ * alignment; the constants (group_scale, mean, absmax) 4-byte. */
 ql_status ql_dequantize(const ql_weight* w, ql_bf16* Wout, void* stream);
 
 /* Forward of the quantised linear with an unmerged adapter (QLoRA page, "memory

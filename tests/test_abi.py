@@ -180,6 +180,57 @@ def test_adapter_entries_refuse_what_the_linear_refuses_before_any_launch(lib):
     assert lib.ql_launch_count() == c0
 
 
+def test_every_entry_refuses_documented_invalid_arguments(lib):
+    """One argument at a time made invalid by the header's own rules (a NULL pointer, an
+    address below the stated alignment, a size outside the stated range, a workspace too
+    small): every entry must return an argument status and launch nothing."""
+    P = 1 << 20                                               # a 16-byte-aligned address
+    big = 1 << 40
+    w = B.QLWeight(0, 0, 64, 64, P, 0, P, P, P)
+    hp_a = B.QLAdamw(1e-3, 0.9, 0.999, 1e-8, 0.0, 1.0, 1)
+    hp_l = B.QLLion(1e-4, 0.9, 0.99, 0.0)
+    items = (B.QLNf4DqItem * 1)(B.QLNf4DqItem(P, 128, P, P, P, P, P))
+    bad_items = (B.QLNf4DqItem * 1)(B.QLNf4DqItem(P + 1, 128, P, P, P, P, P))
+    table = [
+        ("nf4_quantize", [P, 128, P, P, None], {0: [None, P + 1], 1: [-1], 2: [None, P + 1, P + 2], 3: [None, P + 2]}),
+        ("int8_quantize", [P, 128, P, P, None], {0: [None, P + 1], 1: [-1], 2: [None], 3: [None, P + 2]}),
+        ("dq_quantize", [P, 4, P, P, P, P, big, None],
+         {0: [None, P + 2], 1: [0, (1 << 24) + 1], 2: [None], 3: [None, P + 2], 4: [None, P + 2], 5: [None], 6: [0]}),
+        ("nf4_dq_quantize", [P, 128, P, P, P, P, P, P, big, None],
+         {0: [None, P + 1], 1: [0, (1 << 30) + 64], 2: [None, P + 2], 3: [None, P + 2], 4: [None], 5: [None, P + 2],
+          6: [None, P + 2], 7: [None], 8: [0]}),
+        ("nf4_quantize_shard", [P, 16384, P, P, P, P, big, None],
+         {0: [None], 1: [-1], 2: [None], 3: [None], 4: [None, P + 4], 5: [None], 6: [0]}),
+        ("dq_quantize_shard", [P, 256, P, 512, P, P, P, None],
+         {0: [None], 1: [0], 2: [None, P + 4], 3: [255], 4: [None], 5: [None, P + 2], 6: [None, P + 2]}),
+        ("ql_wht", [P, 4, 64, P, None], {0: [None, P + 8], 1: [0], 2: [32, 100], 3: [None, P + 8]}),
+        ("ql_adamw_step", [P, P, P, P, P, 64, ctypes.addressof(hp_a), None],
+         {0: [None, P + 2], 1: [None, P + 1], 2: [None, P + 2], 3: [None, P + 2], 4: [None, P + 2], 5: [-1], 6: [None]}),
+        ("ql_lion_int8_step", [P, P, P, P, P, 64, ctypes.addressof(hp_l), None],
+         {0: [None, P + 2], 1: [None, P + 1], 2: [None, P + 2], 3: [None], 4: [None, P + 2], 5: [-1], 6: [None]}),
+        ("nf4_dq_quantize_batch", [ctypes.addressof(items), 1, P, big, None],
+         {0: [None, ctypes.addressof(bad_items)], 1: [-1], 2: [None, P + 8], 3: [0]}),
+        ("qlora_linear_fwd", [ctypes.byref(w), P, 40, P, P, 8, 8.0, P, P, P, big, None],
+         {0: [None], 1: [None, P + 8], 2: [0, (1 << 31) + 1], 3: [None, P + 8], 4: [None, P + 1], 5: [0, 257],
+          7: [None, P + 8], 8: [P + 1], 9: [None, P + 8], 10: [0]}),
+        ("qlora_linear_bwd", [ctypes.byref(w), P, P, 40, P, P, P, 8, 8.0, P, P, P, P, big, None],
+         {0: [None], 1: [None, P + 8], 2: [None, P + 8], 3: [0, (1 << 31) + 1], 4: [None, P + 1], 5: [None, P + 1],
+          6: [None, P + 1], 7: [0, 257], 9: [None, P + 8], 10: [None, P + 2], 11: [None, P + 2], 12: [None], 13: [0]}),
+        ("ql_dequantize", [ctypes.byref(w), P, None], {0: [None], 1: [None, P + 1]}),
+    ]
+    refusals = {B.QL_ERR_INVALID_ARG, B.QL_ERR_UNSUPPORTED, B.QL_ERR_WORKSPACE}
+    c0 = lib.ql_launch_count()
+    for name, args, bad in table:
+        f = getattr(lib, name)
+        for i, values in bad.items():
+            for v in values:
+                a = list(args)
+                a[i] = v
+                st = f(*a)
+                assert st in refusals, (name, i, v, B.status_string(st))
+    assert lib.ql_launch_count() == c0
+
+
 def test_workspace_query(lib):
     assert B.workspace_bytes(B.QL_OP_DQ, 0, 0, 0, 0) >= 128
     # Walsh-Hadamard adapter: decode-shaped, one slab of Z (16 tokens); otherwise the update
