@@ -71,8 +71,8 @@ def save(path: str, weights) -> None:
     is changed on the device."""
     items = list(weights.items()) if isinstance(weights, dict) else list(weights)
     names = [nm for nm, _ in items]
-    if len(set(names)) != len(names):
-        raise ValueError("weight names must be distinct")
+    if not all(isinstance(nm, str) for nm in names) or len(set(names)) != len(names):
+        raise ValueError("weight names must be distinct strings")
     for name, qw in items:                       # every check before the first byte
         if qw.fmt not in FORMATS:
             raise ValueError(f"{name}: unknown format {qw.fmt!r}")

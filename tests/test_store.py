@@ -86,6 +86,12 @@ def _rewrite_index(p, edit):
         f.write(data[:-16 - jlen] + new + struct.pack("<Q", len(new)) + data[-8:])
 
 
+def test_empty_file_round_trip(tmp_path):
+    p = str(tmp_path / "empty.qlb")
+    store.save(p, {})
+    assert store.load(p) == {}
+
+
 @pytest.mark.parametrize("damage", ["flip", "truncate", "magic", "count", "dtype", "offset", "format", "dup"])
 def test_damaged_files_are_refused(tmp_path, weights, damage):
     p = str(tmp_path / "w.qlb")
@@ -120,6 +126,8 @@ def test_save_refuses_inconsistent_weights(tmp_path, weights):
     p = str(tmp_path / "w.qlb")
     with pytest.raises(ValueError):
         store.save(p, [("a", q), ("a", q)])
+    with pytest.raises(ValueError):
+        store.save(p, [(3, q)])
     short = QuantWeight("nf4_dq", q.N, q.K, q.codes[:-1].clone(), None, q.qabsmax, q.group_scale, q.mean)
     with pytest.raises(ValueError):
         store.save(p, {"short": short})
